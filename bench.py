@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of compressed decode attention over a packed KV cache on B200.
+
+One step = one decode step of the whole hot path for a batch of sequences:
+quantize the newest token's K and V into the packed cache (rotation, Lloyd-Max
+codes, QJL sketch), pre-rotate the queries, split-K attention straight from
+the packed codes, log-sum-exp merge and the final inverse rotation.
+
+Headline `value`: KV tokens attended per second (B * T per step) with the
+packed cache and the step inputs resident in HBM.  `e2e`: the same metric with
+the step inputs (query, new K/V token) copied from pinned host memory and the
+output copied back inside the timed region.  Also reported: the roofline of
+the attention call against the measured HBM copy bandwidth, quantize
+throughput (Mvec/s) on the prefill-shaped sweep, SM clocks sampled during the
+run, and the CPU oracle timed on a bounded sample (`cpu_baseline`).
+
+`--impl reference` times the fp64 CPU oracle (the only reference
+implementation this method has here) on a bounded sample of the same workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+Under torchrun (N > 1) each rank runs an independent replica (the decode path
+needs no exchange between GPUs); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "compressed decode-attn KV tokens/s (% HBM roofline); quantize Mvec/s"
+UNIT = "KV tokens/s"
+
+WORKLOADS = {
+    # Llama-3-8B-shaped decode: GQA 4, k3v4 (keys 2 Lloyd-Max bits + 1 QJL bit, m=128; values 4 bits)
+    "llama3-8b-decode": dict(B=16, Hq=32, Hkv=8, d=128, T=32768, bits_k=3, bits_v=4, m=128),
+    # 70B-shaped long-context decode: GQA 8
+    "70b-decode-k3v4": dict(B=4, Hq=64, Hkv=8, d=128, T=131072, bits_k=3, bits_v=4, m=128),
+    "70b-decode-k4v4": dict(B=4, Hq=64, Hkv=8, d=128, T=131072, bits_k=4, bits_v=4, m=128),
+}
+QUANT_SWEEP = dict(tokens=131072, heads=8, d=128, bits=(2, 3, 4))
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        j = json.loads(p.read_text())
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "compressed_decode_attention_quantize_b200" / "csrc").glob("*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, or None if
+    the kernel sources changed since the counters were taken."""
+    p = ROOT / "profiles" / "attn_traffic.json"
+    if not p.exists():
+        return None
+    j = json.loads(p.read_text())
+    e = j.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def kv_bytes(w, ctx) -> int:
+    kb = ctx.key_layout["bytes_per_vector"]
+    vb = ctx.value_layout["bytes_per_vector"]
+    return w["B"] * w["Hkv"] * w["T"] * (kb + vb)
+
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.flush()
+        rows = []
+        for ln in Path(self.f.name).read_text().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except (ValueError, IndexError):
+                continue
+        os.unlink(self.f.name)
+        inside = [r for r in rows if any(a - 0.15 <= r[0] <= b + 0.15 for a, b in self.windows)]
+        use = inside or rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arms (the only places this script runs the oracle)
+# ---------------------------------------------------------------------------
+def oracle_decode_sample(w, kc_host, vc_host, q_host, tab):
+    """Oracle attention for the G query heads of one (sequence, kv head) slice."""
+    from oracle import tq_oracle as o
+    T = kc_host["norm"].shape[2]
+    return o.attention(tab, q_host, kc_host["codes"], kc_host.get("qjl"), kc_host["norm"],
+                       kc_host.get("rnorm"), vc_host["codes"], vc_host["norm"], [T], 1)
+
+
+def cpu_baseline_from_device(w, ctx, kc, vc, q, sample_T: int):
+    import numpy as np
+    import torch
+    from oracle import tq_oracle as o
+    G = w["Hq"] // w["Hkv"]
+
+    def host(t):
+        if t is None:
+            return None
+        a = t[0:1, 0:1, :sample_T].cpu()
+        return a.numpy().view(np.uint32) if a.dtype == torch.int32 else a.numpy()
+
+    kh = {k: host(v) for k, v in kc.items()}
+    vh = {k: host(v) for k, v in vc.items()}
+    qh = q[0:1, :G].float().cpu().numpy().astype(np.float64)
+    tab = o.make_tables(w["d"], w["bits_k"], w["bits_v"], w["m"], 0)
+    t0 = time.perf_counter()
+    oracle_decode_sample(w, kh, vh, qh, tab)
+    dt = time.perf_counter() - t0
+    tokens_equiv = sample_T / w["Hkv"]  # one of Hkv heads of sample_T tokens of one sequence
+    return {"value": tokens_equiv / dt, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"fp64 oracle attention of the {G} query heads of one (sequence, kv head) slice "
+                      f"over {sample_T} packed tokens ({dt:.2f} s); tokens/s counts the slice as "
+                      f"{sample_T}/{w['Hkv']} full-width KV tokens"}
+
+
+def run_reference(args, w):
+    """Reference arm: the fp64 CPU oracle on a bounded sample per step."""
+    import numpy as np
+    import tq_inputs
+    from oracle import tq_oracle as o
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    G = w["Hq"] // w["Hkv"]
+    sample_T = 2048
+    tab = o.make_tables(w["d"], w["bits_k"], w["bits_v"], w["m"], 0)
+    K = tq_inputs.outlier_kv(1, 1, sample_T, w["d"], seed=1)[0, 0].double().numpy()
+    V = tq_inputs.outlier_kv(1, 1, sample_T, w["d"], seed=2)[0, 0].double().numpy()
+    zk = o.quantize(K, tab, "k")
+    zv = o.quantize(V, tab, "v")
+    r = lambda a: None if a is None else a[None, None]
+    kh = {"codes": r(zk.codes), "qjl": r(zk.qjl), "norm": r(zk.norm), "rnorm": r(zk.rnorm)}
+    vh = {"codes": r(zv.codes), "norm": r(zv.norm)}
+    qs = [tq_inputs.iid((1, G, w["d"]), seed=100 + i).double().numpy() for i in range(4)]
+    knew = tq_inputs.outlier_kv(1, 1, 1, w["d"], seed=3)[0, 0].double().numpy()
+
+    def step(i):
+        # quantize the newest K/V token, then attend over the sample
+        o.quantize(knew, tab, "k")
+        o.quantize(knew, tab, "v")
+        oracle_decode_sample(w, kh, vh, qs[i % 4], tab)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    tokens_equiv = sample_T / w["Hkv"]
+    value = tokens_equiv / dt
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_of(args, w),
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: quantize one K and one V token, then fp64 oracle "
+                                   f"attention of {G} query heads over one (sequence, kv head) slice "
+                                   f"of {sample_T} tokens; counted as {sample_T}/{w['Hkv']} KV tokens"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(args, w):
+    return {"workload": args.workload, "batch": w["B"], "q_heads": w["Hq"], "kv_heads": w["Hkv"],
+            "head_dim": w["d"], "context": w["T"],
+            "kv_format": f"k{w['bits_k']}v{w['bits_v']} (keys {w['bits_k'] - 1} Lloyd-Max bits + 1 QJL bit, "
+                         f"m={w['m']}; values {w['bits_v']} bits)",
+            "inputs": "bf16 K/V with log-normal per-channel scales and 1% x20 outlier channels; bf16 N(0,1) queries",
+            "l2": "no flush: the packed cache read each step is larger than L2",
+            "parallelism": f"replicas x{args.gpus} (no exchange)"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak, steps=10, warmup=3):
+    s = QUANT_SWEEP
+    X = tq_inputs.outlier_kv(1, s["heads"], s["tokens"], s["d"], seed=31, device=dev)[0].reshape(-1, s["d"])
+    Y = tq_inputs.outlier_kv(1, s["heads"], s["tokens"], s["d"], seed=32, device=dev)[0].reshape(-1, s["d"])
+    n = X.shape[0]
+    points = []
+    for bits in s["bits"]:
+        for qjl in (True, False):
+            ctx = tq.Context(s["d"], bits, bits, s["d"] if qjl else 0, 0)
+            pk = ctx.empty_packed(tq.TQ_KEY, (n,), device=dev)
+            pv = ctx.empty_packed(tq.TQ_VALUE, (n,), device=dev)
+            for _ in range(warmup):
+                ctx.quantize_into(X, tq.TQ_KEY, pk)
+                ctx.quantize_into(Y, tq.TQ_VALUE, pv)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                ctx.quantize_into(X, tq.TQ_KEY, pk)
+                ctx.quantize_into(Y, tq.TQ_VALUE, pv)
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 1e3 / steps
+            byts = 2 * n * s["d"] * 2 + n * (ctx.key_layout["bytes_per_vector"] + ctx.value_layout["bytes_per_vector"])
+            points.append({"bits": bits, "qjl": qjl, "mvec_per_s": 2 * n / t / 1e6,
+                           "gbs": byts / t / 1e9, "frac_hbm": byts / t / 1e9 / hbm_peak})
+            ctx.close()
+            del pk, pv
+    del X, Y
+    torch.cuda.empty_cache()
+    head = next(p for p in points if p["bits"] == 3 and p["qjl"])
+    return {"config": f"{s['tokens']} tokens x {s['heads']} kv heads x d={s['d']} bf16 K and V "
+                      f"(outlier channels); K and V quantized each iteration; Mvec counts K+V vectors",
+            "value": head["mvec_per_s"], "unit": "Mvec/s", "point": "bits=3 with QJL",
+            "frac_hbm": head["frac_hbm"], "sweep": points}
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+    import compressed_decode_attention_quantize_b200 as tq
+    import tq_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    hbm_peak, peak_src = peaks()
+
+    B, Hq, Hkv, d, T = w["B"], w["Hq"], w["Hkv"], w["d"], w["T"]
+    ctx = tq.Context(d, w["bits_k"], w["bits_v"], w["m"], 0)
+    # Build the packed cache (setup, not timed): bf16 K/V with outlier channels.
+    kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
+    vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+    for b in range(B):
+        K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
+        V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+        ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
+        ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+        del K, V
+    torch.cuda.synchronize()
+    POOL = 8  # distinct step inputs, reused round-robin
+    qs = [tq_inputs.iid((B, Hq, d), seed=10 + i, device=dev, dtype=torch.bfloat16) for i in range(POOL)]
+    kn = [tq_inputs.outlier_kv(B, Hkv, 1, d, seed=20 + i, device=dev, scale_seed=1)[:, :, 0].contiguous()
+          for i in range(POOL)]
+    vn = [tq_inputs.outlier_kv(B, Hkv, 1, d, seed=40 + i, device=dev, scale_seed=2)[:, :, 0].contiguous()
+          for i in range(POOL)]
+    pos = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 + 3  # append K, append V, prerotate + split attention + merge
+
+    def step(i, ev=None):
+        j = i % POOL
+        ctx.quantize_append(kn[j], tq.TQ_KEY, kc, pos)
+        ctx.quantize_append(vn[j], tq.TQ_VALUE, vc, pos)
+        if ev is not None:
+            ev[0].record()
+        ctx.attn_decode(qs[j], kc, vc, lens, out=out, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record()
+    for i in range(args.steps):
+        step(i, evs[i])
+    e1.record()
+    barrier()
+    sampler.mark(w0, time.time())
+    t_ms = e0.elapsed_time(e1) / args.steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+
+    # End to end through the public API with host buffers: pinned host inputs
+    # copied in and the output copied out inside the timed region.
+    hq = [x.cpu().pin_memory() for x in qs]
+    hk = [x.cpu().pin_memory() for x in kn]
+    hv = [x.cpu().pin_memory() for x in vn]
+    hout = torch.empty(B, Hq, d, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(qs[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+
+    def e2e_step(i):
+        j = i % POOL
+        dq.copy_(hq[j], non_blocking=True)
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        ctx.quantize_append(dk, tq.TQ_KEY, kc, pos)
+        ctx.quantize_append(dv, tq.TQ_VALUE, vc, pos)
+        ctx.attn_decode(dq, kc, vc, lens, out=out, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    w0 = time.time()
+    e0.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record()
+    barrier()
+    sampler.mark(w0, time.time())
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    h2d = hq[0].numel() * hq[0].element_size() + 2 * hk[0].numel() * hk[0].element_size()
+    d2h = hout.numel() * hout.element_size()
+
+    quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
+    clocks = sampler.stop()
+
+    tm = torch.tensor([t_ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    t_ms, attn_ms, e2e_ms = tm.tolist()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline_from_device(w, ctx, kc, vc, qs[0], sample_T=8192)
+
+    if rank == 0:
+        tokens = world * B * T
+        kvb = kv_bytes(w, ctx)
+        alg = kvb + B * Hq * d * 2 + B * Hq * d * 4  # packed cache + bf16 queries + fp32 output
+        achieved = alg / (attn_ms / 1e3) / 1e9
+        traffic = recorded_traffic(args.workload)
+        line = {
+            "metric": METRIC, "value": tokens / (t_ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_of(args, w),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": traffic,
+                         "kernel": "tq_attn_decode (pre-rotate + split-K attention + merge)",
+                         "algorithmic_bytes_per_launch": alg, "launch_ms": attn_ms,
+                         "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                         "frac_of_nominal_8tbs": achieved / 8000.0},
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "quantize": quant,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=int(os.environ.get("WORLD_SIZE", "1")))
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama3-8b-decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

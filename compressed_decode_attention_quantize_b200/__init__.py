@@ -1,0 +1,273 @@
+"""Python binding of libtq: TurboQuant-style K/V quantization and decode
+attention from packed codes on an NVIDIA B200.
+
+Argument marshalling only: every step runs in libtq's CUDA kernels.  PyTorch
+supplies device memory (the tensors passed in, and the outputs this module
+allocates for convenience) and the current CUDA stream.  There is no CPU
+fallback: importing fails if libtq.so has not been built, and every call
+raises TQError when the library reports an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+_LIB_PATH = _PKG / "libtq.so"
+
+TQ_OK, TQ_ERR_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(5)
+TQ_KEY, TQ_VALUE = 0, 1
+TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
+
+_DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libtq status {status}: {msg}")
+        self.status = status
+
+
+class tq_layout_t(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("bits", ctypes.c_int32), ("words", ctypes.c_int32),
+                ("qjl_m", ctypes.c_int32), ("qjl_words", ctypes.c_int32),
+                ("has_rnorm", ctypes.c_int32), ("bytes_per_vector", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not _LIB_PATH.exists():
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m compressed_decode_attention_quantize_b200.build`")
+    lib = ctypes.CDLL(str(_LIB_PATH))
+    P, I, I64, U64, SZ, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                              ctypes.c_size_t, ctypes.c_float)
+    sig = {
+        "tq_last_error": (ctypes.c_char_p, []),
+        "tq_version": (ctypes.c_char_p, []),
+        "tq_init": (P, [I, I, I, I, U64]),
+        "tq_destroy": (None, [P]),
+        "tq_layout": (I, [P, I, ctypes.POINTER(tq_layout_t)]),
+        "tq_host_tables": (I, [I, I, I, I, U64, P, P, P, P, P, P]),
+        "tq_export_tables": (I, [P, P, P, P, P, P, P]),
+        "tq_quantize": (I, [P, I, P, I, I64, I64, P, P, P, P, P]),
+        "tq_quantize_append": (I, [P, I, P, I, I, I, I64, I64, P, P, P, P, P, P]),
+        "tq_dequantize": (I, [P, I, P, P, P, P, I64, P, P]),
+        "tq_logits": (I, [P, P, I, I64, P, P, P, P, I64, P, P]),
+        "tq_attn_workspace_bytes": (SZ, [P, I, I, I64]),
+        "tq_attn_decode": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P, SZ, P]),
+        "tq_topk_workspace_bytes": (SZ, [P, I64, I64, I]),
+        "tq_topk": (I, [P, P, I, I64, P, P, P, P, I64, I, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+EXPORTED = ("tq_last_error", "tq_version", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
+            "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
+            "tq_attn_workspace_bytes", "tq_attn_decode", "tq_topk_workspace_bytes", "tq_topk")
+
+
+def library_path() -> str:
+    return str(_LIB_PATH)
+
+
+def _check(status: int) -> None:
+    if status != TQ_OK:
+        raise TQError(status, _lib.tq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# Raw C-ABI wrappers (same names as the C entry points; pointers as ints or
+# ctypes values).  The Context class below builds on them.
+# ---------------------------------------------------------------------------
+def tq_init(d, bits_k, bits_v, qjl_m, seed):
+    p = _lib.tq_init(d, bits_k, bits_v, qjl_m, seed)
+    if not p:
+        raise TQError(-1, _lib.tq_last_error().decode())
+    return p
+
+
+def tq_destroy(ctx):
+    _lib.tq_destroy(ctx)
+
+
+def tq_version() -> str:
+    return _lib.tq_version().decode()
+
+
+def tq_layout(ctx, which) -> dict:
+    out = tq_layout_t()
+    _check(_lib.tq_layout(ctx, which, ctypes.byref(out)))
+    return {f: getattr(out, f) for f, _ in tq_layout_t._fields_}
+
+
+def tq_host_tables(d, bits_k, bits_v, qjl_m, seed):
+    """Tables computed by the library's host code (no GPU needed), fp64 numpy."""
+    import numpy as np
+    bk_lm = bits_k - 1 if qjl_m > 0 else bits_k
+    pi = np.zeros((d, d))
+    S = np.zeros((max(qjl_m, 1), d))
+    ck = np.zeros(1 << bk_lm)
+    bk = np.zeros((1 << bk_lm) - 1)
+    cv = np.zeros(1 << bits_v)
+    bv = np.zeros((1 << bits_v) - 1)
+    args = [a.ctypes.data_as(ctypes.c_void_p) for a in (pi, S, ck, bk, cv, bv)]
+    _check(_lib.tq_host_tables(d, bits_k, bits_v, qjl_m, seed, *args))
+    return {"Pi": pi, "S": S[:qjl_m], "ck": ck, "bk": bk, "cv": cv, "bv": bv}
+
+
+class Context:
+    """A libtq context: tables for one (d, bits_k, bits_v, qjl_m, seed) on the
+    current CUDA device."""
+
+    def __init__(self, d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int = 0):
+        self.d, self.bits_k, self.bits_v, self.qjl_m, self.seed = d, bits_k, bits_v, qjl_m, seed
+        self.ptr = tq_init(d, bits_k, bits_v, qjl_m, seed)
+        self.key_layout = tq_layout(self.ptr, TQ_KEY)
+        self.value_layout = tq_layout(self.ptr, TQ_VALUE)
+
+    def close(self):
+        if getattr(self, "ptr", None):
+            tq_destroy(self.ptr)
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def layout(self, which: int) -> dict:
+        return self.key_layout if which == TQ_KEY else self.value_layout
+
+    def tables(self):
+        import numpy as np
+        d, kl = self.d, self.key_layout
+        pi = np.zeros((d, d))
+        S = np.zeros((max(self.qjl_m, 1), d))
+        ck = np.zeros(1 << kl["bits"])
+        bk = np.zeros((1 << kl["bits"]) - 1)
+        cv = np.zeros(1 << self.bits_v)
+        bv = np.zeros((1 << self.bits_v) - 1)
+        args = [a.ctypes.data_as(ctypes.c_void_p) for a in (pi, S, ck, bk, cv, bv)]
+        _check(_lib.tq_export_tables(self.ptr, *args))
+        return {"Pi": pi, "S": S[:self.qjl_m], "ck": ck, "bk": bk, "cv": cv, "bv": bv}
+
+    # -- storage -------------------------------------------------------------
+    def empty_packed(self, which: int, lead_shape, device="cuda") -> dict:
+        """Caller-owned packed arrays for vectors of shape lead_shape."""
+        L = self.layout(which)
+        lead = tuple(lead_shape)
+        out = {
+            "codes": torch.empty(lead + (L["bits"], L["words"]), dtype=torch.int32, device=device),
+            "norm": torch.empty(lead, dtype=torch.float32, device=device),
+            "qjl": None, "rnorm": None,
+        }
+        if L["has_rnorm"]:
+            out["qjl"] = torch.empty(lead + (L["qjl_words"],), dtype=torch.int32, device=device)
+            out["rnorm"] = torch.empty(lead, dtype=torch.float32, device=device)
+        return out
+
+    # -- operations ----------------------------------------------------------
+    def quantize_into(self, x: torch.Tensor, which: int, packed: dict, stream=None) -> dict:
+        x2 = x.reshape(-1, x.shape[-1])
+        if x2.stride(-1) != 1:
+            raise TQError(TQ_ERR_ARG, "x must have a unit inner stride")
+        n = x2.shape[0]
+        _check(_lib.tq_quantize(self.ptr, which, _ptr(x2), _DTYPES[x.dtype], n, x2.stride(0),
+                                _ptr(packed["codes"]), _ptr(packed["qjl"]), _ptr(packed["norm"]),
+                                _ptr(packed["rnorm"]), _stream(stream)))
+        return packed
+
+    def quantize(self, x: torch.Tensor, which: int, stream=None) -> dict:
+        packed = self.empty_packed(which, x.shape[:-1], device=x.device)
+        return self.quantize_into(x, which, packed, stream)
+
+    def quantize_append(self, x: torch.Tensor, which: int, cache: dict, pos: torch.Tensor,
+                        stream=None) -> dict:
+        """x [B, H, d] (newest token per sequence and head) -> cache[b, g, pos[b]]."""
+        B, H, d = x.shape
+        if x.stride(2) != 1 or x.stride(0) != H * x.stride(1):
+            raise TQError(TQ_ERR_ARG, "x must be [B, H, d] with rows at a uniform stride")
+        max_T = cache["norm"].shape[2]
+        _check(_lib.tq_quantize_append(self.ptr, which, _ptr(x), _DTYPES[x.dtype], B, H,
+                                       x.stride(1), max_T, _ptr(pos), _ptr(cache["codes"]),
+                                       _ptr(cache["qjl"]), _ptr(cache["norm"]), _ptr(cache["rnorm"]),
+                                       _stream(stream)))
+        return cache
+
+    def dequantize(self, which: int, packed: dict, out: torch.Tensor | None = None, stream=None):
+        n = packed["norm"].numel()
+        if out is None:
+            out = torch.empty(packed["norm"].shape + (self.d,), dtype=torch.float32,
+                              device=packed["norm"].device)
+        _check(_lib.tq_dequantize(self.ptr, which, _ptr(packed["codes"]), _ptr(packed["qjl"]),
+                                  _ptr(packed["norm"]), _ptr(packed["rnorm"]), n, _ptr(out),
+                                  _stream(stream)))
+        return out
+
+    def logits(self, q: torch.Tensor, keys: dict, out: torch.Tensor | None = None, stream=None):
+        q2 = q.reshape(-1, self.d).contiguous()
+        nk = keys["norm"].numel()
+        if out is None:
+            out = torch.empty(q2.shape[0], nk, dtype=torch.float32, device=q.device)
+        _check(_lib.tq_logits(self.ptr, _ptr(q2), _DTYPES[q.dtype], q2.shape[0],
+                              _ptr(keys["codes"]), _ptr(keys["qjl"]), _ptr(keys["norm"]),
+                              _ptr(keys["rnorm"]), nk, _ptr(out), _stream(stream)))
+        return out
+
+    def attn_workspace_bytes(self, B: int, Hq: int, max_T: int) -> int:
+        return int(_lib.tq_attn_workspace_bytes(self.ptr, B, Hq, max_T))
+
+    def attn_decode(self, q: torch.Tensor, kcache: dict, vcache: dict, seq_lens: torch.Tensor,
+                    scale: float | None = None, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """q [B, Hq, d]; caches as dicts of [B, Hkv, max_T, ...] arrays."""
+        q = q.contiguous()
+        B, Hq, d = q.shape
+        Hkv, max_T = kcache["norm"].shape[1], kcache["norm"].shape[2]
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        need = self.attn_workspace_bytes(B, Hq, max_T)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _check(_lib.tq_attn_decode(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
+                                   _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(kcache["norm"]),
+                                   _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
+                                   max_T, _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+        return out
+
+    def topk_workspace_bytes(self, nq: int, n: int, k: int) -> int:
+        return int(_lib.tq_topk_workspace_bytes(self.ptr, nq, n, k))
+
+    def topk(self, q: torch.Tensor, db: dict, k: int, workspace: torch.Tensor | None = None,
+             stream=None):
+        q2 = q.reshape(-1, self.d).contiguous()
+        nq, n = q2.shape[0], db["norm"].numel()
+        idx = torch.empty(nq, k, dtype=torch.int32, device=q.device)
+        score = torch.empty(nq, k, dtype=torch.float32, device=q.device)
+        need = self.topk_workspace_bytes(nq, n, k)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _check(_lib.tq_topk(self.ptr, _ptr(q2), _DTYPES[q.dtype], nq, _ptr(db["codes"]),
+                            _ptr(db["qjl"]), _ptr(db["norm"]), _ptr(db["rnorm"]), n, k, _ptr(idx),
+                            _ptr(score), _ptr(workspace), workspace.numel(), _stream(stream)))
+        return idx, score

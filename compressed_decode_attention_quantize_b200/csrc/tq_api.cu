@@ -1,0 +1,414 @@
+// C ABI of libtq: argument checks, context set-up and kernel launches.
+// The operations and their sources are documented in include/tq.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "tq_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(TQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool valid_dims(int d, int bits_k, int bits_v, int qjl_m, int* code) {
+  if (d < 8 || d > 256 || d % 8 != 0) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "d=%d unsupported (need 8 <= d <= 256, d %% 8 == 0)", d);
+    return false;
+  }
+  const int J = (d + 31) / 32;
+  if (qjl_m < 0 || qjl_m % 8 != 0 || qjl_m > 32 * J) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "qjl_m=%d unsupported (need 0 <= m <= %d, m %% 8 == 0)", qjl_m, 32 * J);
+    return false;
+  }
+  const int bk_lm = qjl_m > 0 ? bits_k - 1 : bits_k;
+  if (bk_lm < 1 || bk_lm > 4) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "bits_k=%d with qjl_m=%d gives %d Lloyd-Max bits (need 1..4)",
+                 bits_k, qjl_m, bk_lm);
+    return false;
+  }
+  if (bits_v < 1 || bits_v > 4) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "bits_v=%d unsupported (need 1..4)", bits_v);
+    return false;
+  }
+  return true;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_ctx(const tq_ctx* c) {
+  if (!c) return fail(TQ_ERR_ARG, "null context");
+  return TQ_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* tq_last_error(void) { return g_err.c_str(); }
+
+const char* tq_version(void) { return "libtq 0.1 (sm_100a)"; }
+
+int tq_host_tables(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, double* pi,
+                   double* S, double* ck, double* bk, double* cv, double* bv) {
+  int code = TQ_OK;
+  if (!valid_dims(d, bits_k, bits_v, qjl_m, &code)) return code;
+  const int bk_lm = qjl_m > 0 ? bits_k - 1 : bits_k;
+  try {
+    if (pi) {
+      std::vector<double> P;
+      tqh::rotation(d, seed, P);
+      std::memcpy(pi, P.data(), P.size() * sizeof(double));
+    }
+    if (S && qjl_m > 0) {
+      std::vector<double> Sm;
+      tqh::qjl_matrix(qjl_m, d, seed, Sm);
+      std::memcpy(S, Sm.data(), Sm.size() * sizeof(double));
+    }
+    std::vector<double> c, b;
+    if (ck || bk) {
+      tqh::lloyd_max(d, bk_lm, c, b);
+      if (ck) std::memcpy(ck, c.data(), c.size() * sizeof(double));
+      if (bk) std::memcpy(bk, b.data(), b.size() * sizeof(double));
+    }
+    if (cv || bv) {
+      tqh::lloyd_max(d, bits_v, c, b);
+      if (cv) std::memcpy(cv, c.data(), c.size() * sizeof(double));
+      if (bv) std::memcpy(bv, b.data(), b.size() * sizeof(double));
+    }
+  } catch (const std::bad_alloc&) {
+    return fail(TQ_ERR_ARG, "host allocation failed");
+  }
+  return TQ_OK;
+}
+
+tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
+  int code = TQ_OK;
+  if (!valid_dims(d, bits_k, bits_v, qjl_m, &code)) return nullptr;
+  tq_ctx* c = new (std::nothrow) tq_ctx();
+  if (!c) {
+    fail(TQ_ERR_ARG, "host allocation failed");
+    return nullptr;
+  }
+  c->d = d;
+  c->J = (d + 31) / 32;
+  c->dpad = 32 * c->J;
+  c->bits_k = bits_k;
+  c->bk_lm = qjl_m > 0 ? bits_k - 1 : bits_k;
+  c->bits_v = bits_v;
+  c->qjl_m = qjl_m;
+  c->seed = seed;
+  tqh::rotation(d, seed, c->Pi);
+  tqh::qjl_matrix(qjl_m, d, seed, c->S);
+  tqh::lloyd_max(d, c->bk_lm, c->ck, c->bk);
+  tqh::lloyd_max(d, bits_v, c->cv, c->bv);
+
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "tq_init: cudaGetDevice");
+    delete c;
+    return nullptr;
+  }
+  const int dp = c->dpad;
+  const size_t nPiT = (size_t)d * dp, nPi = (size_t)d * d, nST = (size_t)d * dp, nS = (size_t)dp * d;
+  const size_t total = (nPiT + nPi + nST + nS + 4 * 16) * sizeof(float);
+  std::vector<float> h(total / sizeof(float), 0.f);
+  float* hPiT = h.data();
+  float* hPi = hPiT + nPiT;
+  float* hST = hPi + nPi;
+  float* hS = hST + nST;
+  float* hck = hS + nS;
+  float* hbk = hck + 16;
+  float* hcv = hbk + 16;
+  float* hbv = hcv + 16;
+  for (int j = 0; j < d; ++j)
+    for (int k = 0; k < d; ++k) {
+      hPiT[(size_t)k * dp + j] = (float)c->Pi[(size_t)j * d + k];
+      hPi[(size_t)j * d + k] = (float)c->Pi[(size_t)j * d + k];
+    }
+  for (int i = 0; i < qjl_m; ++i)
+    for (int k = 0; k < d; ++k) {
+      hST[(size_t)k * dp + i] = (float)c->S[(size_t)i * d + k];
+      hS[(size_t)i * d + k] = (float)c->S[(size_t)i * d + k];
+    }
+  for (int i = 0; i < 16; ++i) {
+    hbk[i] = INFINITY;
+    hbv[i] = INFINITY;
+  }
+  for (size_t i = 0; i < c->ck.size(); ++i) hck[i] = (float)c->ck[i];
+  for (size_t i = 0; i < c->bk.size(); ++i) hbk[i] = (float)c->bk[i];
+  for (size_t i = 0; i < c->cv.size(); ++i) hcv[i] = (float)c->cv[i];
+  for (size_t i = 0; i < c->bv.size(); ++i) hbv[i] = (float)c->bv[i];
+
+  e = cudaMalloc(&c->dev_block, total);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "tq_init: cudaMalloc");
+    delete c;
+    return nullptr;
+  }
+  e = cudaMemcpy(c->dev_block, h.data(), total, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "tq_init: cudaMemcpy");
+    cudaFree(c->dev_block);
+    delete c;
+    return nullptr;
+  }
+  const float* base = static_cast<const float*>(c->dev_block);
+  c->PiT = base;
+  c->Pi_f = base + (hPi - hPiT);
+  c->ST = base + (hST - hPiT);
+  c->S_f = base + (hS - hPiT);
+  c->ck_f = base + (hck - hPiT);
+  c->bk_f = base + (hbk - hPiT);
+  c->cv_f = base + (hcv - hPiT);
+  c->bv_f = base + (hbv - hPiT);
+  return c;
+}
+
+void tq_destroy(tq_ctx* c) {
+  if (!c) return;
+  if (c->dev_block) {
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != c->device) cudaSetDevice(c->device);
+    cudaFree(c->dev_block);
+    if (cur != c->device) cudaSetDevice(cur);
+  }
+  delete c;
+}
+
+int tq_layout(const tq_ctx* c, int which, tq_layout_t* out) {
+  if (int r = check_ctx(c)) return r;
+  if (!out) return fail(TQ_ERR_ARG, "tq_layout: null output");
+  if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "tq_layout: bad which=%d", which);
+  const bool key = which == TQ_KEY;
+  out->d = c->d;
+  out->bits = key ? c->bk_lm : c->bits_v;
+  out->words = c->J;
+  out->qjl_m = key ? c->qjl_m : 0;
+  out->qjl_words = (out->qjl_m + 31) / 32;
+  out->has_rnorm = (key && c->qjl_m > 0) ? 1 : 0;
+  out->bytes_per_vector = (int64_t)out->bits * c->J * 4 + (int64_t)out->qjl_words * 4 + 4 +
+                          (out->has_rnorm ? 4 : 0);
+  return TQ_OK;
+}
+
+int tq_export_tables(const tq_ctx* c, double* pi, double* S, double* ck, double* bk, double* cv,
+                     double* bv) {
+  if (int r = check_ctx(c)) return r;
+  if (pi) std::memcpy(pi, c->Pi.data(), c->Pi.size() * sizeof(double));
+  if (S && c->qjl_m > 0) std::memcpy(S, c->S.data(), c->S.size() * sizeof(double));
+  if (ck) std::memcpy(ck, c->ck.data(), c->ck.size() * sizeof(double));
+  if (bk) std::memcpy(bk, c->bk.data(), c->bk.size() * sizeof(double));
+  if (cv) std::memcpy(cv, c->cv.data(), c->cv.size() * sizeof(double));
+  if (bv) std::memcpy(bv, c->bv.data(), c->bv.size() * sizeof(double));
+  return TQ_OK;
+}
+
+static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64_t n, int64_t ld,
+                           uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm,
+                           const int32_t* pos, int H, int64_t max_T, void* stream,
+                           const char* name) {
+  if (int r = check_ctx(c)) return r;
+  if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "%s: bad which=%d", name, which);
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dtype);
+  if (n < 0 || ld < c->d)
+    return fail(TQ_ERR_ARG, "%s: n=%lld ld=%lld (need n >= 0, ld >= d)", name, (long long)n, (long long)ld);
+  if (n == 0) return TQ_OK;
+  const bool key = which == TQ_KEY;
+  const int m = key ? c->qjl_m : 0;
+  if (!x || !codes || !norm) return fail(TQ_ERR_ARG, "%s: null pointer", name);
+  if (m > 0 && (!qjl || !rnorm)) return fail(TQ_ERR_ARG, "%s: keys with QJL need qjl and rnorm", name);
+  if (!aligned(codes, 4) || !aligned(norm, 4)) return fail(TQ_ERR_ARG, "%s: misaligned output", name);
+  tqk::QuantArgs a{};
+  a.x = x;
+  a.dtype = dtype;
+  a.n = n;
+  a.ld = ld;
+  a.d = c->d;
+  a.bits = key ? c->bk_lm : c->bits_v;
+  a.nbnd = (1 << a.bits) - 1;
+  a.m = m;
+  a.PiT = c->PiT;
+  a.ST = c->ST;
+  a.cen = key ? c->ck_f : c->cv_f;
+  a.bnd = key ? c->bk_f : c->bv_f;
+  a.codes = codes;
+  a.qjl = qjl;
+  a.norm = norm;
+  a.rnorm = rnorm;
+  a.pos = pos;
+  a.H = H;
+  a.max_T = max_T;
+  cudaError_t e = tqk::launch_quantize(c, a, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  return TQ_OK;
+}
+
+int tq_quantize(tq_ctx* c, int which, const void* x, int dtype, int64_t n, int64_t ld,
+                uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm, void* stream) {
+  return quantize_common(c, which, x, dtype, n, ld, codes, qjl, norm, rnorm, nullptr, 0, 0, stream,
+                         "tq_quantize");
+}
+
+int tq_quantize_append(tq_ctx* c, int which, const void* x, int dtype, int B, int H, int64_t ld,
+                       int64_t max_T, const int32_t* pos, uint32_t* codes, uint32_t* qjl,
+                       float* norm, float* rnorm, void* stream) {
+  if (B < 0 || H <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "tq_quantize_append: bad sizes");
+  if (B > 0 && !pos) return fail(TQ_ERR_ARG, "tq_quantize_append: null pos");
+  return quantize_common(c, which, x, dtype, (int64_t)B * H, ld, codes, qjl, norm, rnorm, pos, H,
+                         max_T, stream, "tq_quantize_append");
+}
+
+int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* qjl,
+                  const float* norm, const float* rnorm, int64_t n, float* out, void* stream) {
+  if (int r = check_ctx(c)) return r;
+  if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "tq_dequantize: bad which=%d", which);
+  if (n < 0) return fail(TQ_ERR_ARG, "tq_dequantize: n < 0");
+  if (n == 0) return TQ_OK;
+  if (!codes || !norm || !out) return fail(TQ_ERR_ARG, "tq_dequantize: null pointer");
+  if (which == TQ_KEY && c->qjl_m > 0 && (!qjl || !rnorm))
+    return fail(TQ_ERR_ARG, "tq_dequantize: keys with QJL need qjl and rnorm");
+  cudaError_t e = tqk::launch_dequant(c, which, codes, qjl, norm, rnorm, n, out, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_dequantize");
+  return TQ_OK;
+}
+
+int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* kcodes,
+              const uint32_t* kqjl, const float* knorm, const float* krnorm, int64_t nk, float* out,
+              void* stream) {
+  if (int r = check_ctx(c)) return r;
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_ARG, "tq_logits: bad dtype=%d", dtype);
+  if (nq < 0 || nk < 0) return fail(TQ_ERR_ARG, "tq_logits: negative size");
+  if (nq == 0 || nk == 0) return TQ_OK;
+  if (!q || !kcodes || !knorm || !out) return fail(TQ_ERR_ARG, "tq_logits: null pointer");
+  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_logits: keys with QJL need kqjl and krnorm");
+  if (nq > 65535LL * 8) return fail(TQ_ERR_UNSUPPORTED, "tq_logits: nq too large");
+  cudaError_t e = tqk::launch_logits(c, q, dtype, nq, kcodes, kqjl, knorm, krnorm, nk, out,
+                                     as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_logits");
+  return TQ_OK;
+}
+
+size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
+  if (!c || B <= 0 || Hq <= 0 || max_T < 0) return 0;
+  int chunk = 0;
+  const int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
+  // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most splits).
+  const size_t rows = (size_t)B * Hq;
+  size_t b = 2 * rows * c->dpad * sizeof(float);
+  b = (b + 255) & ~(size_t)255;
+  b += rows * (size_t)splits * (c->dpad + 2) * sizeof(float);
+  return b + 256;
+}
+
+int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
+                   const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                   const float* krnorm, const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                   const int32_t* seq_lens, float scale, float* out, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  if (int r = check_ctx(c)) return r;
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_ARG, "tq_attn_decode: bad dtype=%d", dtype);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T < 0) return fail(TQ_ERR_ARG, "tq_attn_decode: bad sizes");
+  if (Hq % Hkv != 0 || Hq / Hkv > 16)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", Hq, Hkv);
+  if (B == 0) return TQ_OK;
+  if (!q || !kcodes || !knorm || !vcodes || !vnorm || !seq_lens || !out)
+    return fail(TQ_ERR_ARG, "tq_attn_decode: null pointer");
+  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_attn_decode: keys with QJL need kqjl and krnorm");
+  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: B or Hkv too large");
+  const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
+  if (!workspace || ws_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "tq_attn_decode: workspace %zu bytes < %zu", ws_bytes, need);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_attn_decode: workspace not 256-byte aligned");
+  cudaStream_t s = as_stream(stream);
+  const size_t rows = (size_t)B * Hq;
+  char* p = static_cast<char*>(workspace);
+  float* qr = reinterpret_cast<float*>(p);
+  float* qs = qr + rows * c->dpad;
+  size_t off = (2 * rows * c->dpad * sizeof(float) + 255) & ~(size_t)255;
+  float* part = reinterpret_cast<float*>(p + off);
+  cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, qr, qs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode: prerotate");
+  tqk::AttnArgs a{};
+  a.qr = qr;
+  a.qs = qs;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.d = c->d;
+  a.bk = c->bk_lm;
+  a.bv = c->bits_v;
+  a.m = c->qjl_m;
+  a.kcodes = kcodes;
+  a.kqjl = kqjl;
+  a.knorm = knorm;
+  a.krnorm = krnorm;
+  a.vcodes = vcodes;
+  a.vnorm = vnorm;
+  a.max_T = max_T;
+  a.seq_lens = seq_lens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
+  a.ck = c->ck_f;
+  a.cv = c->cv_f;
+  a.splits = tqk::attn_splits(c, B, Hkv, max_T > 0 ? max_T : 1, &a.chunk);
+  a.part = part;
+  e = tqk::launch_attn(c, a, out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
+  return TQ_OK;
+}
+
+size_t tq_topk_workspace_bytes(const tq_ctx* c, int64_t nq, int64_t n, int k) {
+  if (!c || nq < 0 || n < 0 || k < 1 || k > 32) return 0;
+  return tqk::topk_workspace(c, nq, n, k);
+}
+
+int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* codes,
+            const uint32_t* qjl, const float* norm, const float* rnorm, int64_t n, int k,
+            int32_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
+  if (int r = check_ctx(c)) return r;
+  if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
+    return fail(TQ_ERR_ARG, "tq_topk: bad dtype=%d", dtype);
+  if (nq < 0 || n < 0 || k < 1 || k > 32) return fail(TQ_ERR_ARG, "tq_topk: bad sizes (k must be 1..32)");
+  if (nq == 0) return TQ_OK;
+  if (n > 0x7ffffff0LL) return fail(TQ_ERR_UNSUPPORTED, "tq_topk: n too large");
+  if (nq > 65535LL * 16) return fail(TQ_ERR_UNSUPPORTED, "tq_topk: nq too large");
+  if (!q || !idx || !score || (n > 0 && (!codes || !norm)))
+    return fail(TQ_ERR_ARG, "tq_topk: null pointer");
+  if (n > 0 && c->qjl_m > 0 && (!qjl || !rnorm)) return fail(TQ_ERR_ARG, "tq_topk: keys with QJL need qjl and rnorm");
+  const size_t need = tq_topk_workspace_bytes(c, nq, n, k);
+  if (!workspace || ws_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "tq_topk: workspace %zu bytes < %zu", ws_bytes, need);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_topk: workspace not 256-byte aligned");
+  cudaError_t e = tqk::launch_topk(c, q, dtype, nq, codes, qjl, norm, rnorm, n, k, idx, score,
+                                   workspace, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_topk");
+  return TQ_OK;
+}
+
+}  // extern "C"

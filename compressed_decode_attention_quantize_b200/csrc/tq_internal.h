@@ -1,0 +1,104 @@
+// Internal declarations shared by the host table builder, the kernels and the
+// C ABI of libtq.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "tq.h"
+
+struct tq_ctx {
+  int d = 0;        // vector dimension
+  int J = 0;        // words per bit-plane, ceil(d/32)
+  int dpad = 0;     // 32*J
+  int bits_k = 0;   // key bits including the QJL bit
+  int bk_lm = 0;    // key Lloyd-Max bits
+  int bits_v = 0;   // value Lloyd-Max bits
+  int qjl_m = 0;    // QJL rows (0 = none)
+  int device = 0;
+  uint64_t seed = 0;
+  // fp64 host tables
+  std::vector<double> Pi, S, ck, bk, cv, bv;
+  // device tables (one allocation owned by the context)
+  void* dev_block = nullptr;
+  const float* PiT = nullptr;   // [d][dpad]  PiT[k*dpad+j] = Pi[j][k]; zero for j >= d
+  const float* Pi_f = nullptr;  // [d][d]     row-major Pi
+  const float* ST = nullptr;    // [d][dpad]  ST[k*dpad+i] = S[i][k]; zero for i >= m
+  const float* S_f = nullptr;   // [dpad][d]  row-major S; zero rows for i >= m
+  const float* ck_f = nullptr;  // [16] key centroids (padded)
+  const float* bk_f = nullptr;  // [16] key boundaries (padded with +inf)
+  const float* cv_f = nullptr;  // [16]
+  const float* bv_f = nullptr;  // [16]
+};
+
+namespace tqh {
+double round_to_half(double x);
+void rotation(int d, uint64_t seed, std::vector<double>& Pi);
+void qjl_matrix(int m, int d, uint64_t seed, std::vector<double>& S);
+void lloyd_max(int d, int bits, std::vector<double>& cen, std::vector<double>& bnd);
+}  // namespace tqh
+
+namespace tqk {
+
+struct QuantArgs {
+  const void* x;
+  int dtype;
+  int64_t n, ld;
+  int d, bits, nbnd, m;
+  const float* PiT;
+  const float* ST;
+  const float* cen;
+  const float* bnd;
+  uint32_t* codes;
+  uint32_t* qjl;
+  float* norm;
+  float* rnorm;
+  // Optional cache placement: when pos != nullptr, input row v = b*H + g is
+  // written to cache record (b*H + g)*max_T + pos[b]; otherwise to record v.
+  const int32_t* pos;
+  int H;
+  int64_t max_T;
+};
+
+struct AttnArgs {
+  const float* qr;   // [B*Hq][dpad] pre-rotated queries
+  const float* qs;   // [B*Hq][dpad] S q'
+  int B, Hq, Hkv, G, d, bk, bv, m;
+  const uint32_t* kcodes;
+  const uint32_t* kqjl;
+  const float* knorm;
+  const float* krnorm;
+  const uint32_t* vcodes;
+  const float* vnorm;
+  int64_t max_T;
+  const int32_t* seq_lens;
+  float scale_log2;  // softmax scale * log2(e)
+  float cq;          // sqrt(pi/2)/m
+  const float* ck;
+  const float* cv;
+  int splits;
+  int chunk;         // tokens per split
+  float* part;       // [B*Hq][splits][dpad+2]
+};
+
+cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
+cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
+                             float* qr, float* qs, cudaStream_t s);
+cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
+                          const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                          const float* krnorm, int64_t nk, float* out, cudaStream_t s);
+cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
+                           const uint32_t* qjl, const float* norm, const float* rnorm,
+                           int64_t n, float* out, cudaStream_t s);
+size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k);
+cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
+                        const uint32_t* codes, const uint32_t* qjl, const float* norm,
+                        const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
+                        void* ws, cudaStream_t s);
+int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk);
+
+}  // namespace tqk

@@ -1,0 +1,875 @@
+// CUDA kernels of libtq (sm_100a), plain fp32 versions.
+//
+// Each kernel states the operation it computes; the method follows "What is
+// TurboQuant?" (a2a-mcp.org), section "How TurboQuant works": stage 1 (rotate
+// the normalised vector with Pi, Lloyd-Max index per coordinate), stage 2 (1-bit
+// QJL sketch of the residual) and the closing paragraph (logits taken from the
+// compressed indices without dequantizing the keys).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <climits>
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tqk {
+
+namespace {
+
+constexpr float kNegInf = -INFINITY;
+
+__device__ __forceinline__ float load_elem(const void* p, int dtype, int64_t i) {
+  if (dtype == TQ_F32) return static_cast<const float*>(p)[i];
+  if (dtype == TQ_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  return __half2float(static_cast<const __half*>(p)[i]);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Index of a coordinate: number of boundaries at or below y (ties go up).
+__device__ __forceinline__ int lm_index(float y, const float* sb, int nb) {
+  int idx = 0;
+  for (int t = 0; t < nb; ++t) idx += (y >= sb[t]) ? 1 : 0;
+  return idx;
+}
+
+// Output record of input row v (cache placement when a.pos is set).
+__device__ __forceinline__ int64_t out_record(const QuantArgs& a, int64_t v) {
+  if (a.pos == nullptr) return v;
+  const int64_t b = v / a.H;
+  return v * a.max_T + a.pos[b];
+}
+
+// Lloyd-Max index of coordinate j from its bit-planes (plane stride J words).
+__device__ __forceinline__ int plane_index(const uint32_t* w, int bits, int J, int j) {
+  const int wi = j >> 5, e = j & 31;
+  int idx = 0;
+  for (int p = 0; p < bits; ++p) idx |= ((w[p * J + wi] >> e) & 1u) << p;
+  return idx;
+}
+
+// ----------------------------------------------------------------------------
+// Quantize: one warp quantizes QV vectors at a time.  Lane l owns the output
+// coordinates j = l + 32 i (i < J), so the Lloyd-Max bits of plane p, word i
+// of a vector are one __ballot_sync.  The rotation y = Pi x / |x| and the
+// sketch S r are fp32 FMA dot products (PiT and ST are k-major so lanes read
+// consecutive words).
+// ----------------------------------------------------------------------------
+constexpr int QV = 8;
+constexpr int QWARPS = 8;
+
+template <int J>
+__global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
+  constexpr int DP = J * 32;
+  extern __shared__ float smem[];
+  __shared__ float s_cen[16], s_bnd[16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* sx = smem + warp * (DP * QV);  // [DP][QV]
+  if (threadIdx.x < 16) {
+    s_cen[threadIdx.x] = (threadIdx.x < (1 << a.bits)) ? a.cen[threadIdx.x] : 0.f;
+    s_bnd[threadIdx.x] = (threadIdx.x < a.nbnd) ? a.bnd[threadIdx.x] : INFINITY;
+  }
+  __syncthreads();
+  const int64_t ngroups = (a.n + QV - 1) / QV;
+  const int words = a.bits * J;
+  const int mwords = (a.m + 31) >> 5;
+  for (int64_t g = (int64_t)blockIdx.x * QWARPS + warp; g < ngroups;
+       g += (int64_t)gridDim.x * QWARPS) {
+    const int64_t v0 = g * QV;
+    float ss[QV];
+#pragma unroll
+    for (int v = 0; v < QV; ++v) {
+      ss[v] = 0.f;
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const int k = lane + 32 * i;
+        float val = 0.f;
+        if (k < a.d && v0 + v < a.n) val = load_elem(a.x, a.dtype, (v0 + v) * a.ld + k);
+        sx[k * QV + v] = val;
+        ss[v] = fmaf(val, val, ss[v]);
+      }
+      ss[v] = warp_sum(ss[v]);
+    }
+    __syncwarp();
+    float acc[J][QV];
+#pragma unroll
+    for (int i = 0; i < J; ++i)
+#pragma unroll
+      for (int v = 0; v < QV; ++v) acc[i][v] = 0.f;
+    for (int k = 0; k < a.d; ++k) {
+      const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+      const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
+      const float xv[QV] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const float p = __ldg(a.PiT + (size_t)k * DP + lane + 32 * i);
+#pragma unroll
+        for (int v = 0; v < QV; ++v) acc[i][v] = fmaf(p, xv[v], acc[i][v]);
+      }
+    }
+    // y = Pi x / |x| (0 for a zero vector), then the Lloyd-Max index.
+    float nrm[QV];
+    unsigned char idx[J][QV];
+#pragma unroll
+    for (int v = 0; v < QV; ++v) {
+      nrm[v] = sqrtf(ss[v]);
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const float y = nrm[v] > 0.f ? acc[i][v] / nrm[v] : 0.f;
+        acc[i][v] = y;
+        idx[i][v] = (unsigned char)lm_index(y, s_bnd, a.nbnd);
+      }
+    }
+    // Bit-plane packing: word i of plane p is a ballot over the lanes.
+#pragma unroll
+    for (int v = 0; v < QV; ++v) {
+      uint32_t mine = 0;
+      for (int p = 0; p < a.bits; ++p) {
+#pragma unroll
+        for (int i = 0; i < J; ++i) {
+          const bool bit = ((idx[i][v] >> p) & 1) && (lane + 32 * i < a.d);
+          const uint32_t w = __ballot_sync(0xffffffffu, bit);
+          if (lane == p * J + i) mine = w;
+        }
+      }
+      if (v0 + v < a.n && lane < words) a.codes[out_record(a, v0 + v) * words + lane] = mine;
+    }
+    float my_norm = 0.f;
+#pragma unroll
+    for (int v = 0; v < QV; ++v)
+      if (lane == v) my_norm = nrm[v];
+    if (lane < QV && v0 + lane < a.n) a.norm[out_record(a, v0 + lane)] = my_norm;
+    if (a.m == 0) { __syncwarp(); continue; }
+
+    // Stage 2: residual r = y - c[idx], rho = |r|, QJL bits sign(S r).
+    __syncwarp();
+    float rr[QV];
+#pragma unroll
+    for (int v = 0; v < QV; ++v) {
+      rr[v] = 0.f;
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const int k = lane + 32 * i;
+        const float r = (k < a.d) ? acc[i][v] - s_cen[idx[i][v]] : 0.f;
+        sx[k * QV + v] = r;
+        rr[v] = fmaf(r, r, rr[v]);
+      }
+      rr[v] = warp_sum(rr[v]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < J; ++i)
+#pragma unroll
+      for (int v = 0; v < QV; ++v) acc[i][v] = 0.f;
+    for (int k = 0; k < a.d; ++k) {
+      const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+      const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
+      const float xv[QV] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const float p = __ldg(a.ST + (size_t)k * DP + lane + 32 * i);
+#pragma unroll
+        for (int v = 0; v < QV; ++v) acc[i][v] = fmaf(p, xv[v], acc[i][v]);
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < QV; ++v) {
+      uint32_t mine = 0;
+#pragma unroll
+      for (int i = 0; i < J; ++i) {
+        const bool bit = (acc[i][v] >= 0.f) && (lane + 32 * i < a.m);
+        const uint32_t w = __ballot_sync(0xffffffffu, bit);
+        if (lane == i) mine = w;
+      }
+      if (v0 + v < a.n && lane < mwords) a.qjl[out_record(a, v0 + v) * mwords + lane] = mine;
+    }
+    float my_rn = 0.f;
+#pragma unroll
+    for (int v = 0; v < QV; ++v)
+      if (lane == v) my_rn = nrm[v] * sqrtf(rr[v]);
+    if (lane < QV && v0 + lane < a.n) a.rnorm[out_record(a, v0 + lane)] = my_rn;
+    __syncwarp();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Query pre-rotation: q' = Pi q, s = S q' (one block per query row).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int d, int dpad,
+                                                   int m, const float* PiT, const float* ST,
+                                                   float* qr, float* qs) {
+  extern __shared__ float sh[];
+  float* sq = sh;          // [dpad]
+  float* sr = sh + dpad;   // [dpad]
+  const int64_t row = blockIdx.x;
+  for (int k = threadIdx.x; k < dpad; k += blockDim.x)
+    sq[k] = (k < d) ? load_elem(q, dtype, row * d + k) : 0.f;
+  __syncthreads();
+  for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc = fmaf(PiT[(size_t)k * dpad + j], sq[k], acc);
+    sr[j] = acc;
+    qr[row * dpad + j] = acc;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < dpad; i += blockDim.x) {
+    float acc = 0.f;
+    if (i < m)
+      for (int k = 0; k < d; ++k) acc = fmaf(ST[(size_t)k * dpad + i], sr[k], acc);
+    qs[row * dpad + i] = acc;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Split-K decode attention, one CTA per (split, kv head, sequence), 128
+// threads.  Per tile of 128 tokens: (1) thread t computes the logits of token
+// t for the G query heads of the group straight from the packed key codes,
+// (2) online-softmax update of the running max / sum per head, (3) thread j
+// accumulates o_rot[j] += p_t * |v_t| * cv[vidx_tj] (the rotated-domain value;
+// Pi^T is applied once after the merge).
+// ----------------------------------------------------------------------------
+constexpr int AT = 128;   // tokens per tile = threads per CTA
+constexpr int GMAX = 16;
+
+template <int J>
+__global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
+  constexpr int DP = J * 32;
+  constexpr int JJ = (DP + AT - 1) / AT;  // value dims per thread
+  extern __shared__ float sh[];
+  float* sq = sh;                       // [G][DP]
+  float* ssv = sq + a.G * DP;           // [G][DP]
+  float* sp = ssv + a.G * DP;           // [AT][G]   p * |v|
+  uint32_t* svc = reinterpret_cast<uint32_t*>(sp + AT * a.G);  // [AT][bv*J]
+  __shared__ float s_ck[16], s_cv[16];
+  __shared__ float s_wred[AT / 32][GMAX];
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = a.G;
+  if (tid < 16) {
+    s_ck[tid] = (tid < (1 << a.bk)) ? a.ck[tid] : 0.f;
+    s_cv[tid] = (tid < (1 << a.bv)) ? a.cv[tid] : 0.f;
+  }
+  for (int e = tid; e < G * DP; e += AT) {
+    const int h = e / DP, j = e % DP;
+    const int64_t row = (int64_t)b * a.Hq + (int64_t)g * G + h;
+    sq[e] = a.qr[row * DP + j];
+    ssv[e] = a.qs[row * DP + j];
+  }
+  const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
+  const int64_t t_begin = (int64_t)split * a.chunk;
+  const int64_t t_end = min(T, t_begin + a.chunk);
+  float m_run[GMAX], l_run[GMAX], o[GMAX][JJ];
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) {
+    m_run[h] = kNegInf;
+    l_run[h] = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < JJ; ++jj) o[h][jj] = 0.f;
+  }
+  __syncthreads();
+  const int64_t kv_row0 = ((int64_t)b * a.Hkv + g) * a.max_T;
+  const int kw = a.bk * J, vw = a.bv * J, mw = (a.m + 31) >> 5;
+
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += AT) {
+    const int64_t t = t0 + tid;
+    const bool valid = t < t_end;
+    const int ntile = (int)min((int64_t)AT, t_end - t0);
+    float sc[GMAX];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) sc[h] = kNegInf;
+    if (valid) {
+      const int64_t r = kv_row0 + t;
+      uint32_t w[4 * 8];
+      for (int e = 0; e < kw; ++e) w[e] = a.kcodes[r * kw + e];
+      float acc[GMAX], acc2[GMAX];
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h) acc[h] = acc2[h] = 0.f;
+      for (int j = 0; j < a.d; ++j) {
+        const float c = s_ck[plane_index(w, a.bk, J, j)];
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h)
+          if (h < G) acc[h] = fmaf(sq[h * DP + j], c, acc[h]);
+      }
+      for (int wi = 0; wi < mw; ++wi) {
+        const uint32_t bitsw = a.kqjl[r * mw + wi];
+        const int lim = min(32, a.m - 32 * wi);
+        for (int e = 0; e < lim; ++e) {
+          const bool pos = (bitsw >> e) & 1u;
+          const int i = 32 * wi + e;
+#pragma unroll
+          for (int h = 0; h < GMAX; ++h)
+            if (h < G) acc2[h] += pos ? ssv[h * DP + i] : -ssv[h * DP + i];
+        }
+      }
+      const float kn = a.knorm[r];
+      const float kg = a.m > 0 ? a.krnorm[r] * a.cq : 0.f;
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h)
+        if (h < G) sc[h] = (kn * acc[h] + kg * acc2[h]) * a.scale_log2;
+    }
+    // Tile max per head.
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        const float mx = warp_max(sc[h]);
+        if (lane == 0) s_wred[warp][h] = mx;
+      }
+    }
+    // Stage this tile's value codes (contiguous words) while the max settles.
+    for (int e = tid; e < ntile * vw; e += AT) svc[e] = a.vcodes[(kv_row0 + t0) * vw + e];
+    __syncthreads();
+    float alpha[GMAX], mnew[GMAX];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        float mx = s_wred[0][h];
+        for (int ww = 1; ww < AT / 32; ++ww) mx = fmaxf(mx, s_wred[ww][h]);
+        mnew[h] = fmaxf(m_run[h], mx);
+        alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
+      }
+    }
+    const float vn = valid ? a.vnorm[kv_row0 + t] : 0.f;
+    float psum[GMAX];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        const float p = valid ? exp2f(sc[h] - mnew[h]) : 0.f;
+        sp[tid * G + h] = p * vn;
+        psum[h] = p;
+      }
+    }
+    __syncthreads();  // s_wred reads done before reuse
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        const float sm = warp_sum(psum[h]);
+        if (lane == 0) s_wred[warp][h] = sm;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G) {
+        float sm = 0.f;
+        for (int ww = 0; ww < AT / 32; ++ww) sm += s_wred[ww][h];
+        l_run[h] = l_run[h] * alpha[h] + sm;
+        m_run[h] = mnew[h];
+#pragma unroll
+        for (int jj = 0; jj < JJ; ++jj) o[h][jj] *= alpha[h];
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < JJ; ++jj) {
+      const int j = tid + AT * jj;
+      if (j < a.d) {
+        for (int tt = 0; tt < ntile; ++tt) {
+          const float c = s_cv[plane_index(svc + tt * vw, a.bv, J, j)];
+#pragma unroll
+          for (int h = 0; h < GMAX; ++h)
+            if (h < G) o[h][jj] = fmaf(sp[tt * G + h], c, o[h][jj]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // Partial state (m, l, o_rot) per query head.
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) {
+    if (h >= G) break;
+    const int64_t row = (int64_t)b * a.Hq + (int64_t)g * G + h;
+    float* pp = a.part + (row * a.splits + split) * (DP + 2);
+    if (tid == 0) {
+      pp[0] = m_run[h];
+      pp[1] = l_run[h];
+    }
+#pragma unroll
+    for (int jj = 0; jj < JJ; ++jj) {
+      const int j = tid + AT * jj;
+      if (j < DP) pp[2 + j] = o[h][jj];
+    }
+  }
+}
+
+// Log-sum-exp merge of the split partials and the final o = Pi^T o_rot.
+__global__ void __launch_bounds__(128) k_attn_merge(const float* part, int splits, int d, int dpad,
+                                                    const float* Pi, float* out) {
+  extern __shared__ float sh[];
+  float* so = sh;  // [dpad]
+  const int64_t row = blockIdx.x;
+  const float* pr = part + row * splits * (dpad + 2);
+  float M = kNegInf;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, pr[s * (dpad + 2)]);
+  float L = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float ms = pr[s * (dpad + 2)];
+    if (ms != kNegInf) L += exp2f(ms - M) * pr[s * (dpad + 2) + 1];
+  }
+  for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float ms = pr[s * (dpad + 2)];
+      if (ms != kNegInf) acc = fmaf(exp2f(ms - M), pr[s * (dpad + 2) + 2 + j], acc);
+    }
+    so[j] = (L > 0.f) ? acc / L : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < d; ++j) acc = fmaf(Pi[(size_t)j * d + i], so[j], acc);
+    out[row * d + i] = acc;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Logits of nq queries against nk packed keys.  Each CTA pre-rotates its QB
+// queries into shared memory, then thread t scores key t of its slice.
+// ----------------------------------------------------------------------------
+constexpr int LQB = 8;
+
+template <int J>
+__global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_t nq, int d,
+                                                int bk, int m, const float* PiT, const float* ST,
+                                                const float* ck, float cq,
+                                                const uint32_t* kcodes, const uint32_t* kqjl,
+                                                const float* knorm, const float* krnorm,
+                                                int64_t nk, float* out) {
+  constexpr int DP = J * 32;
+  __shared__ float sx[LQB][DP], sq[LQB][DP], ss[LQB][DP];
+  __shared__ float s_ck[16];
+  const int tid = threadIdx.x;
+  const int64_t q0 = (int64_t)blockIdx.y * LQB;
+  if (tid < 16) s_ck[tid] = (tid < (1 << bk)) ? ck[tid] : 0.f;
+  for (int e = tid; e < LQB * DP; e += blockDim.x) {
+    const int qq = e / DP, k = e % DP;
+    sx[qq][k] = (k < d && q0 + qq < nq) ? load_elem(q, dtype, (q0 + qq) * d + k) : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < LQB * DP; e += blockDim.x) {
+    const int qq = e / DP, j = e % DP;
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc = fmaf(PiT[(size_t)k * DP + j], sx[qq][k], acc);
+    sq[qq][j] = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e < LQB * DP; e += blockDim.x) {
+    const int qq = e / DP, i = e % DP;
+    float acc = 0.f;
+    if (i < m)
+      for (int k = 0; k < d; ++k) acc = fmaf(ST[(size_t)k * DP + i], sq[qq][k], acc);
+    ss[qq][i] = acc;
+  }
+  __syncthreads();
+  const int64_t key = (int64_t)blockIdx.x * blockDim.x + tid;
+  if (key >= nk) return;
+  const int kw = bk * J, mw = (m + 31) >> 5;
+  uint32_t w[4 * 8];
+  for (int e = 0; e < kw; ++e) w[e] = kcodes[key * kw + e];
+  float acc[LQB], acc2[LQB];
+#pragma unroll
+  for (int qq = 0; qq < LQB; ++qq) acc[qq] = acc2[qq] = 0.f;
+  for (int j = 0; j < d; ++j) {
+    const float c = s_ck[plane_index(w, bk, J, j)];
+#pragma unroll
+    for (int qq = 0; qq < LQB; ++qq) acc[qq] = fmaf(sq[qq][j], c, acc[qq]);
+  }
+  for (int wi = 0; wi < mw; ++wi) {
+    const uint32_t bitsw = kqjl[key * mw + wi];
+    const int lim = min(32, m - 32 * wi);
+    for (int e = 0; e < lim; ++e) {
+      const bool pos = (bitsw >> e) & 1u;
+#pragma unroll
+      for (int qq = 0; qq < LQB; ++qq) acc2[qq] += pos ? ss[qq][32 * wi + e] : -ss[qq][32 * wi + e];
+    }
+  }
+  const float kn = knorm[key];
+  const float kg = m > 0 ? krnorm[key] * cq : 0.f;
+#pragma unroll
+  for (int qq = 0; qq < LQB; ++qq)
+    if (q0 + qq < nq) out[(q0 + qq) * nk + key] = kn * acc[qq] + kg * acc2[qq];
+}
+
+// ----------------------------------------------------------------------------
+// Dequantize one vector per CTA: rot_j = |x| c[idx_j] (+ C gamma (S^T sigma)_j),
+// then x_hat = Pi^T rot.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int m,
+                                                 const float* Pi, const float* S,
+                                                 const float* cen, float cq,
+                                                 const uint32_t* codes, const uint32_t* qjl,
+                                                 const float* norm, const float* rnorm,
+                                                 float* out) {
+  extern __shared__ float sh[];
+  float* srot = sh;  // [dpad]
+  const int64_t v = blockIdx.x;
+  const int J = dpad / 32;
+  const int words = bits * J, mw = (m + 31) >> 5;
+  const uint32_t* w = codes + v * words;
+  const float n = norm[v];
+  const float kg = m > 0 ? rnorm[v] * cq : 0.f;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float r = n * cen[plane_index(w, bits, J, j)];
+    if (m > 0) {
+      float acc = 0.f;
+      for (int i = 0; i < m; ++i) {
+        const bool pos = (qjl[v * mw + (i >> 5)] >> (i & 31)) & 1u;
+        acc += pos ? S[(size_t)i * d + j] : -S[(size_t)i * d + j];
+      }
+      r = fmaf(kg, acc, r);
+    }
+    srot[j] = r;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < d; k += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < d; ++j) acc = fmaf(Pi[(size_t)j * d + k], srot[j], acc);
+    out[v * d + k] = acc;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Top-k.  Phase 1: CTA (chunk, query tile) scores TQ queries against a chunk
+// of the database, 256 vectors per step (one per thread), and keeps each
+// query's running top-k in shared memory by warp-wide selection.  Phase 2:
+// one warp per query selects the final top-k from all chunk lists.
+// Order: score descending, then index ascending.
+// ----------------------------------------------------------------------------
+constexpr int TQ = 16;      // queries per CTA
+constexpr int TTH = 256;    // threads (= database vectors per step)
+constexpr int TSTEPS = 32;  // steps per chunk
+constexpr int TKMAX = 32;
+
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+template <int J>
+__global__ void __launch_bounds__(TTH) k_topk_chunk(const float* qr, const float* qs, int64_t nq,
+                                                    int d, int bk, int m, const float* ck, float cq,
+                                                    const uint32_t* codes, const uint32_t* qjl,
+                                                    const float* norm, const float* rnorm,
+                                                    int64_t n, int K, float* cand_v, int* cand_i,
+                                                    int nchunks) {
+  constexpr int DP = J * 32;
+  extern __shared__ float sh[];
+  float* sq = sh;                    // [DP][TQ]
+  float* ssv = sq + DP * TQ;         // [DP][TQ]
+  float* sscore = ssv + DP * TQ;     // [TQ][TTH]
+  float* stop_v = sscore + TQ * TTH; // [TQ][TKMAX]
+  int* stop_i = reinterpret_cast<int*>(stop_v + TQ * TKMAX);
+  __shared__ float s_ck[16];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t q0 = (int64_t)blockIdx.y * TQ;
+  const int chunk = blockIdx.x;
+  if (tid < 16) s_ck[tid] = (tid < (1 << bk)) ? ck[tid] : 0.f;
+  for (int e = tid; e < DP * TQ; e += TTH) {
+    const int j = e / TQ, qq = e % TQ;
+    const bool ok = q0 + qq < nq;
+    sq[e] = ok ? qr[(q0 + qq) * DP + j] : 0.f;
+    ssv[e] = ok ? qs[(q0 + qq) * DP + j] : 0.f;
+  }
+  for (int e = tid; e < TQ * TKMAX; e += TTH) {
+    stop_v[e] = kNegInf;
+    stop_i[e] = INT_MAX;
+  }
+  __syncthreads();
+  const int kw = bk * J, mw = (m + 31) >> 5;
+  const int64_t base = (int64_t)chunk * TSTEPS * TTH;
+  for (int step = 0; step < TSTEPS; ++step) {
+    const int64_t v = base + (int64_t)step * TTH + tid;
+    if (v < n) {
+      uint32_t w[4 * 8];
+      for (int e = 0; e < kw; ++e) w[e] = codes[v * kw + e];
+      float acc[TQ], acc2[TQ];
+#pragma unroll
+      for (int qq = 0; qq < TQ; ++qq) acc[qq] = acc2[qq] = 0.f;
+      for (int j = 0; j < d; ++j) {
+        const float c = s_ck[plane_index(w, bk, J, j)];
+        const float4* qp = reinterpret_cast<const float4*>(sq + j * TQ);
+#pragma unroll
+        for (int q4 = 0; q4 < TQ / 4; ++q4) {
+          const float4 qv = qp[q4];
+          acc[4 * q4 + 0] = fmaf(qv.x, c, acc[4 * q4 + 0]);
+          acc[4 * q4 + 1] = fmaf(qv.y, c, acc[4 * q4 + 1]);
+          acc[4 * q4 + 2] = fmaf(qv.z, c, acc[4 * q4 + 2]);
+          acc[4 * q4 + 3] = fmaf(qv.w, c, acc[4 * q4 + 3]);
+        }
+      }
+      for (int wi = 0; wi < mw; ++wi) {
+        const uint32_t bitsw = qjl[v * mw + wi];
+        const int lim = min(32, m - 32 * wi);
+        for (int e = 0; e < lim; ++e) {
+          const float sg = ((bitsw >> e) & 1u) ? 1.f : -1.f;
+          const float4* sp = reinterpret_cast<const float4*>(ssv + (32 * wi + e) * TQ);
+#pragma unroll
+          for (int q4 = 0; q4 < TQ / 4; ++q4) {
+            const float4 sv = sp[q4];
+            acc2[4 * q4 + 0] = fmaf(sg, sv.x, acc2[4 * q4 + 0]);
+            acc2[4 * q4 + 1] = fmaf(sg, sv.y, acc2[4 * q4 + 1]);
+            acc2[4 * q4 + 2] = fmaf(sg, sv.z, acc2[4 * q4 + 2]);
+            acc2[4 * q4 + 3] = fmaf(sg, sv.w, acc2[4 * q4 + 3]);
+          }
+        }
+      }
+      const float kn = norm[v];
+      const float kg = m > 0 ? rnorm[v] * cq : 0.f;
+#pragma unroll
+      for (int qq = 0; qq < TQ; ++qq) sscore[qq * TTH + tid] = kn * acc[qq] + kg * acc2[qq];
+    } else {
+#pragma unroll
+      for (int qq = 0; qq < TQ; ++qq) sscore[qq * TTH + tid] = kNegInf;
+    }
+    __syncthreads();
+    // Merge: warp w handles queries w, w+8, ...
+    for (int qq = warp; qq < TQ; qq += TTH / 32) {
+      const float kth_v = stop_v[qq * TKMAX + K - 1];
+      const int kth_i = stop_i[qq * TKMAX + K - 1];
+      float vals[TTH / 32 + 1];
+      int ids[TTH / 32 + 1];
+      bool any = false;
+#pragma unroll
+      for (int e = 0; e < TTH / 32; ++e) {
+        const int t = lane + 32 * e;
+        vals[e] = sscore[qq * TTH + t];
+        ids[e] = (int)(base + (int64_t)step * TTH + t);
+        if (vals[e] == kNegInf) ids[e] = INT_MAX;
+        any |= better(vals[e], ids[e], kth_v, kth_i);
+      }
+      if (!__any_sync(0xffffffffu, any)) continue;
+      vals[TTH / 32] = (lane < K) ? stop_v[qq * TKMAX + lane] : kNegInf;
+      ids[TTH / 32] = (lane < K) ? stop_i[qq * TKMAX + lane] : INT_MAX;
+      float nv = kNegInf;
+      int ni = INT_MAX;
+      for (int r = 0; r < K; ++r) {
+        float bv = vals[0];
+        int bi = ids[0];
+#pragma unroll
+        for (int e = 1; e <= TTH / 32; ++e)
+          if (better(vals[e], ids[e], bv, bi)) { bv = vals[e]; bi = ids[e]; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+        if (lane == r) { nv = bv; ni = bi; }
+#pragma unroll
+        for (int e = 0; e <= TTH / 32; ++e)
+          if (ids[e] == bi && vals[e] == bv) { vals[e] = kNegInf; ids[e] = INT_MAX; }
+      }
+      __syncwarp();
+      if (lane < K) {
+        stop_v[qq * TKMAX + lane] = nv;
+        stop_i[qq * TKMAX + lane] = ni;
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < TQ * K; e += TTH) {
+    const int qq = e / K, r = e % K;
+    if (q0 + qq < nq) {
+      const int64_t o = ((q0 + qq) * nchunks + chunk) * K + r;
+      cand_v[o] = stop_v[qq * TKMAX + r];
+      cand_i[o] = stop_i[qq * TKMAX + r];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(32) k_topk_final(const float* cand_v, const int* cand_i,
+                                                   int nchunks, int K, int32_t* idx, float* score) {
+  const int64_t q = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int total = nchunks * K;
+  const float* cv = cand_v + q * total;
+  const int* ci = cand_i + q * total;
+  float taken_v = INFINITY;
+  int taken_i = -1;
+  // K rounds; in each, the best candidate strictly after the previous pick.
+  for (int r = 0; r < K; ++r) {
+    float bv = kNegInf;
+    int bi = INT_MAX;
+    for (int e = lane; e < total; e += 32) {
+      const float v = cv[e];
+      const int i = ci[e];
+      const bool after = better(taken_v, taken_i, v, i);
+      if (after && better(v, i, bv, bi)) { bv = v; bi = i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) {
+      idx[q * K + r] = (bi == INT_MAX) ? -1 : bi;
+      score[q * K + r] = bv;
+    }
+    taken_v = bv;
+    taken_i = bi;
+  }
+}
+
+template <int J>
+cudaError_t quantize_J(const QuantArgs& a, cudaStream_t s) {
+  const size_t shm = (size_t)QWARPS * J * 32 * QV * sizeof(float);
+  if (shm > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_quantize<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t groups = (a.n + QV - 1) / QV;
+  int64_t blocks = (groups + QWARPS - 1) / QWARPS;
+  blocks = blocks < 148 * 16 ? blocks : 148 * 16;
+  k_quantize<J><<<(unsigned)blocks, QWARPS * 32, shm, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int J>
+cudaError_t attn_J(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
+  const size_t shm = (size_t)(2 * a.G * J * 32 + AT * a.G) * sizeof(float) +
+                     (size_t)AT * a.bv * J * sizeof(uint32_t);
+  if (shm > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(a.splits, a.Hkv, a.B);
+  k_attn_split<J><<<grid, AT, shm, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, c->dpad * sizeof(float), s>>>(
+      a.part, a.splits, c->d, c->dpad, c->Pi_f, out);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+#define TQ_DISPATCH_J(J, ...)                      \
+  switch (J) {                                     \
+    case 1: { constexpr int JV = 1; __VA_ARGS__; } \
+    case 2: { constexpr int JV = 2; __VA_ARGS__; } \
+    case 3: { constexpr int JV = 3; __VA_ARGS__; } \
+    case 4: { constexpr int JV = 4; __VA_ARGS__; } \
+    case 5: { constexpr int JV = 5; __VA_ARGS__; } \
+    case 6: { constexpr int JV = 6; __VA_ARGS__; } \
+    case 7: { constexpr int JV = 7; __VA_ARGS__; } \
+    case 8: { constexpr int JV = 8; __VA_ARGS__; } \
+    default: return cudaErrorInvalidValue;         \
+  }
+
+cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s) {
+  TQ_DISPATCH_J(c->J, return quantize_J<JV>(a, s));
+}
+
+cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
+                             float* qr, float* qs, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  k_prerotate<<<(unsigned)rows, 256, 2 * c->dpad * sizeof(float), s>>>(
+      q, dtype, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs);
+  return cudaGetLastError();
+}
+
+int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
+  (void)c;
+  // Aim for about 8 CTAs per SM over the 148 SMs, tiles of whole 128 tokens.
+  const int64_t pairs = (int64_t)B * Hkv;
+  const int64_t target = 148 * 8;
+  int64_t splits = (target + pairs - 1) / pairs;
+  int64_t ch = (max_T + splits - 1) / splits;
+  ch = ((ch + AT - 1) / AT) * AT;
+  if (ch < AT) ch = AT;
+  splits = (max_T + ch - 1) / ch;
+  if (splits < 1) splits = 1;
+  *chunk = (int)ch;
+  return (int)splits;
+}
+
+cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
+  TQ_DISPATCH_J(c->J, return attn_J<JV>(c, a, out, s));
+}
+
+cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
+                          const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                          const float* krnorm, int64_t nk, float* out, cudaStream_t s) {
+  if (nq == 0 || nk == 0) return cudaSuccess;
+  dim3 grid((unsigned)((nk + 127) / 128), (unsigned)((nq + LQB - 1) / LQB));
+  const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
+  TQ_DISPATCH_J(c->J, k_logits<JV><<<grid, 128, 0, s>>>(q, dtype, nq, c->d, c->bk_lm, c->qjl_m,
+                                                        c->PiT, c->ST, c->ck_f, cq, kcodes, kqjl,
+                                                        knorm, krnorm, nk, out);
+                return cudaGetLastError());
+}
+
+cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
+                           const uint32_t* qjl, const float* norm, const float* rnorm,
+                           int64_t n, float* out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const bool key = which == TQ_KEY;
+  const int m = key ? c->qjl_m : 0;
+  const float cq = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.f;
+  k_dequant<<<(unsigned)n, 128, c->dpad * sizeof(float), s>>>(
+      c->d, c->dpad, key ? c->bk_lm : c->bits_v, m, c->Pi_f, c->S_f, key ? c->ck_f : c->cv_f, cq,
+      codes, qjl, norm, rnorm, out);
+  return cudaGetLastError();
+}
+
+static int64_t topk_chunks(int64_t n) {
+  const int64_t per = (int64_t)TSTEPS * TTH;
+  return (n + per - 1) / per;
+}
+
+size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k) {
+  const int64_t nch = topk_chunks(n > 0 ? n : 1);
+  size_t b = 2 * (size_t)nq * c->dpad * sizeof(float);        // q', s
+  b += (size_t)nq * nch * k * (sizeof(float) + sizeof(int));  // candidates
+  return b + 1024;
+}
+
+cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
+                        const uint32_t* codes, const uint32_t* qjl, const float* norm,
+                        const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
+                        void* ws, cudaStream_t s) {
+  if (nq == 0) return cudaSuccess;
+  const int64_t nch = topk_chunks(n > 0 ? n : 1);
+  char* p = static_cast<char*>(ws);
+  auto take = [&](size_t bytes) {
+    char* r = p;
+    p += (bytes + 255) & ~(size_t)255;
+    return r;
+  };
+  float* qr = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
+  float* qs = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
+  float* cv = reinterpret_cast<float*>(take((size_t)nq * nch * k * sizeof(float)));
+  int* ci = reinterpret_cast<int*>(take((size_t)nq * nch * k * sizeof(int)));
+  cudaError_t e = launch_prerotate(c, q, dtype, nq, qr, qs, s);
+  if (e != cudaSuccess) return e;
+  const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
+  const size_t shm = (size_t)(2 * c->dpad * TQ + TQ * TTH + TQ * TKMAX) * sizeof(float) +
+                     (size_t)TQ * TKMAX * sizeof(int);
+  dim3 grid((unsigned)nch, (unsigned)((nq + TQ - 1) / TQ));
+  TQ_DISPATCH_J(c->J, {
+    e = cudaFuncSetAttribute(k_topk_chunk<JV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+    k_topk_chunk<JV><<<grid, TTH, shm, s>>>(qr, qs, nq, c->d, c->bk_lm, c->qjl_m, c->ck_f, cq,
+                                             codes, qjl, norm, rnorm, n, k, cv, ci, (int)nch);
+    break;
+  });
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, (int)nch, k, idx, score);
+  return cudaGetLastError();
+}
+
+}  // namespace tqk

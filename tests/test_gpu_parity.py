@@ -1,0 +1,336 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (libtq via its binding).
+
+Small cases run the oracle on every output; the full-size workloads (decode
+attention shaped like Llama-3-8B and a 70B model, the vector-search top-k)
+check sampled outputs.  Rules are in tests/_parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_decode_attention_quantize_b200 as tq
+import tq_inputs
+from oracle import tq_oracle as o
+import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _ctx(d, bk, bv, m, seed=0):
+    return tq.Context(d, bk, bv, m, seed)
+
+
+def _flat(p, n):
+    return {k: (None if v is None else v.reshape(n, -1) if v.ndim > 1 else v) for k, v in P.packed_np(p).items()}
+
+
+# --- layout and tables ------------------------------------------------------
+def test_layout_bytes(cuda):
+    c = _ctx(128, 3, 4, 128)
+    assert c.key_layout["bytes_per_vector"] == 56      # 2 planes x 16 B + 16 B QJL + |k| + gamma
+    assert c.value_layout["bytes_per_vector"] == 68    # 4 planes x 16 B + |v|
+    c2 = _ctx(200, 4, 3, 200)
+    assert c2.key_layout["words"] == 7 and c2.key_layout["qjl_words"] == 7
+
+
+def test_device_context_tables_match_oracle(cuda):
+    c = _ctx(128, 3, 4, 128, seed=42)
+    t = c.tables()
+    ot = o.make_tables(128, 3, 4, 128, 42)
+    assert np.abs(t["Pi"] - ot.Pi).max() < 1e-12
+    assert np.array_equal(t["S"], ot.S)
+    assert np.abs(t["ck"] - ot.cb_k.centroids).max() < 1e-12
+    assert np.abs(t["cv"] - ot.cb_v.centroids).max() < 1e-12
+
+
+# --- quantize ------------------------------------------------------------------
+def test_quantize_single_head_fp32(cuda):
+    """1024 keys + 1024 values, d=128, fp32 N(0,1), seed 0; k3 (2+1, m=128), v4."""
+    c = _ctx(128, 3, 4, 128, seed=0)
+    tab = P.oracle_tables(c)
+    K = tq_inputs.iid((1024, 128), seed=0)
+    V = tq_inputs.iid((1024, 128), seed=1)
+    pk = c.quantize(K.to(cuda), tq.TQ_KEY)
+    pv = c.quantize(V.to(cuda), tq.TQ_VALUE)
+    torch.cuda.synchronize()
+    P.check_quantized(tab, "k", K.double().numpy(), _flat(pk, 1024))
+    P.check_quantized(tab, "v", V.double().numpy(), _flat(pv, 1024))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("qjl", [True, False])
+def test_quantize_bit_sweep_outlier_bf16(cuda, bits, qjl):
+    """Prefill-style quantization sweep on bf16 K/V with outlier channels
+    (8 heads x 1031 tokens, a ragged count)."""
+    m = 128 if qjl else 0
+    c = _ctx(128, bits, bits, m, seed=3)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.outlier_kv(1, 8, 1031, 128, seed=bits * 10 + qjl)[0].reshape(-1, 128)
+    n = X.shape[0]
+    pk = c.quantize(X.to(cuda), tq.TQ_KEY)
+    pv = c.quantize(X.to(cuda), tq.TQ_VALUE)
+    torch.cuda.synchronize()
+    x = X.double().numpy()
+    P.check_quantized(tab, "k", x, _flat(pk, n))
+    P.check_quantized(tab, "v", x, _flat(pv, n))
+
+
+def test_quantize_d200_mixture(cuda):
+    """d=200 (7 words per plane), 3-bit Lloyd-Max + QJL with m=200, unit-norm mixture."""
+    c = _ctx(200, 4, 3, 200, seed=5)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(3000, 200, seed=1)
+    pk = c.quantize(X.to(cuda), tq.TQ_KEY)
+    torch.cuda.synchronize()
+    P.check_quantized(tab, "k", X.double().numpy(), _flat(pk, 3000))
+
+
+def test_quantize_edge_cases(cuda):
+    c = _ctx(64, 3, 2, 64, seed=8)
+    tab = P.oracle_tables(c)
+    # n = 0 is a no-op
+    empty = torch.empty(0, 64, device=cuda)
+    c.quantize(empty, tq.TQ_KEY)
+    # zero vectors, a single vector, fp16 input, and a strided (ld > d) view
+    X = tq_inputs.iid((37, 64), seed=4)
+    X[0] = 0
+    X[5] = 0
+    big = torch.zeros(37, 80)
+    big[:, :64] = X
+    for src in (X.to(cuda), X.half().to(cuda), big.to(cuda)[:, :64]):
+        pk = c.quantize(src, tq.TQ_KEY) if src.stride(0) == 64 else None
+        if pk is None:
+            pk = c.empty_packed(tq.TQ_KEY, (37,))
+            c.quantize_into(src, tq.TQ_KEY, pk)
+        torch.cuda.synchronize()
+        x = src.double().cpu().numpy()
+        P.check_quantized(tab, "k", x, _flat(pk, 37))
+        g = P.packed_np(pk)
+        assert g["norm"][0] == 0 and g["rnorm"][0] == 0
+        assert np.all(o.unpack_planes(g["codes"][0], 2, 64) == 2)
+
+
+# --- dequantize / logits ---------------------------------------------------------
+def test_dequantize_matches_oracle(cuda):
+    c = _ctx(128, 3, 4, 128, seed=0)
+    tab = P.oracle_tables(c)
+    K = tq_inputs.iid((500, 128), seed=2) * 3
+    for which, wch in ((tq.TQ_KEY, "k"), (tq.TQ_VALUE, "v")):
+        p = c.quantize(K.to(cuda), which)
+        xh = c.dequantize(which, p)
+        torch.cuda.synchronize()
+        g = _flat(p, 500)
+        ref = o.dequantize(tab, wch, g["codes"].reshape(500, -1, 4), g["norm"], g["qjl"], g["rnorm"])
+        err = np.linalg.norm(xh.cpu().double().numpy() - ref, axis=1) / np.linalg.norm(ref, axis=1)
+        assert err.max() < 1e-5
+
+
+def test_logits_single_head(cuda):
+    """Logits of 8 N(0,1) queries against the 1024 packed keys, from codes."""
+    c = _ctx(128, 3, 4, 128, seed=0)
+    tab = P.oracle_tables(c)
+    K = tq_inputs.iid((1024, 128), seed=0)
+    Q = tq_inputs.iid((8, 128), seed=2)
+    pk = c.quantize(K.to(cuda), tq.TQ_KEY)
+    lg = c.logits(Q.to(cuda), pk)
+    torch.cuda.synchronize()
+    P.check_logits(tab, Q.double().numpy(), _flat(pk, 1024), lg.cpu().double().numpy())
+
+
+# --- decode attention ---------------------------------------------------------
+def _cache(c, K, V, cuda):
+    return c.quantize(K.to(cuda), tq.TQ_KEY), c.quantize(V.to(cuda), tq.TQ_VALUE)
+
+
+def test_attention_single_head(cuda):
+    """8 queries over 1024 keys/values of one KV head (softmax . V)."""
+    c = _ctx(128, 3, 4, 128, seed=0)
+    tab = P.oracle_tables(c)
+    K = tq_inputs.iid((1, 1, 1024, 128), seed=0)
+    V = tq_inputs.iid((1, 1, 1024, 128), seed=1)
+    Q = tq_inputs.iid((1, 8, 128), seed=2)
+    kc, vc = _cache(c, K, V, cuda)
+    lens = torch.tensor([1024], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), 1,
+                      out.cpu().numpy())
+
+
+@pytest.mark.parametrize("d,Hq,Hkv,bk,bv,m", [(128, 8, 2, 3, 4, 128), (128, 16, 2, 4, 4, 128),
+                                             (200, 6, 3, 4, 3, 200), (64, 4, 4, 2, 2, 0)])
+def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m):
+    """Ragged lengths (0, 1, odd, full), GQA groups 1/2/4/8, d=64/128/200."""
+    c = _ctx(d, bk, bv, m, seed=7)
+    tab = P.oracle_tables(c)
+    B, T = 5, 1000
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=1)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=2)
+    Q = tq_inputs.iid((B, Hq, d), seed=3, dtype=torch.bfloat16)
+    kc, vc = _cache(c, K, V, cuda)
+    lens = torch.tensor([0, 1, 129, 777, 1000], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+
+
+def _slice_pairs(kc, vc, pairs, Hq, Hkv):
+    """Host copies of the (b, kv-head) slices the sampled (b, h) pairs read."""
+    G = Hq // Hkv
+    out = []
+    for b, h in pairs:
+        g = h // G
+        sl = lambda t: None if t is None else P.to_np(t[b:b + 1, g:g + 1])
+        out.append(({k: sl(v) for k, v in kc.items()}, {k: sl(v) for k, v in vc.items()}))
+    return out
+
+
+def _full_size(cuda, B, Hq, Hkv, T, bk, bv, pairs, seed):
+    c = _ctx(128, bk, bv, 128, seed=0)
+    tab = P.oracle_tables(c)
+    K = tq_inputs.outlier_kv(B, Hkv, T, 128, seed=seed, device=cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, T, 128, seed=seed + 1, device=cuda)
+    Q = tq_inputs.iid((B, Hq, 128), seed=seed + 2, device=cuda, dtype=torch.bfloat16)
+    kc, vc = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    # quantize parity on one sampled slice of each
+    n = 4096
+    P.check_quantized(tab, "k", P.to_np(K[0, 0, :n]), _flat({k: (None if v is None else v[0, 0, :n]) for k, v in kc.items()}, n))
+    P.check_quantized(tab, "v", P.to_np(V[B - 1, Hkv - 1, -n:]), _flat({k: (None if v is None else v[B - 1, Hkv - 1, -n:]) for k, v in vc.items()}, n))
+    del K, V
+    lens = torch.full((B,), T, dtype=torch.int32, device=cuda)
+    out = c.attn_decode(Q, kc, vc, lens)
+    torch.cuda.synchronize()
+    qn = P.to_np(Q)
+    G = Hq // Hkv
+    for (b, h), (ks, vs) in zip(pairs, _slice_pairs(kc, vc, pairs, Hq, Hkv)):
+        P.check_attention(tab, qn[b:b + 1, h:h + 1], ks, vs, np.array([T]), 1,
+                          P.to_np(out[b:b + 1, h:h + 1]))
+    del kc, vc
+    torch.cuda.empty_cache()
+
+
+def test_attention_llama8b_shape_sampled(cuda):
+    """B=16, Hq=32, Hkv=8 (GQA 4), d=128, T=32768, bf16 outlier K/V, k3v4."""
+    _full_size(cuda, 16, 32, 8, 32768, 3, 4, [(0, 0), (7, 13), (15, 31)], seed=100)
+
+
+@pytest.mark.parametrize("bk", [3, 4])
+def test_attention_70b_shape_sampled(cuda, bk):
+    """B=4, Hq=64, Hkv=8 (GQA 8), d=128, T=131072, bf16 outlier K/V, k3v4 / k4v4."""
+    _full_size(cuda, 4, 64, 8, 131072, bk, 4, [(0, 5), (3, 63)], seed=200 + bk)
+
+
+# --- top-k --------------------------------------------------------------------
+def _oracle_topk_chunked(tab, q, g, k, chunk=25_000):
+    n = g["norm"].size
+    best_v = np.full((q.shape[0], 0), -np.inf)
+    best_i = np.zeros((q.shape[0], 0), dtype=np.int64)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        sc = o.logits(tab, q, g["codes"][s:e].reshape(e - s, tab.bits_k_lm, -1), g["norm"][s:e],
+                      g["qjl"][s:e].reshape(e - s, -1), g["rnorm"][s:e])
+        best_v = np.concatenate([best_v, sc], axis=1)
+        best_i = np.concatenate([best_i, np.broadcast_to(np.arange(s, e), sc.shape)], axis=1)
+        order = np.lexsort((best_i, -best_v), axis=1)[:, :k]
+        best_v = np.take_along_axis(best_v, order, 1)
+        best_i = np.take_along_axis(best_i, order, 1)
+    return best_i, best_v
+
+
+def _check_topk(tab, q, g, idx, score, k):
+    ref_i, ref_v = _oracle_topk_chunked(tab, q, g, k)
+    qn = np.linalg.norm(q, axis=1)
+    for r in range(q.shape[0]):
+        tol = P.LOGIT_TOL * qn[r] * max(1.0, float(np.max(g["norm"])))
+        assert np.all(np.abs(score[r] - ref_v[r]) <= tol)
+        if list(idx[r]) != list(ref_i[r]):
+            # near-ties may swap: any differing member must score within tol of the k-th
+            diff = set(idx[r]) ^ set(ref_i[r])
+            kth = ref_v[r, -1]
+            for j in diff:
+                sc = o.logits(tab, q[r:r + 1], g["codes"][j:j + 1].reshape(1, tab.bits_k_lm, -1),
+                              g["norm"][j:j + 1], g["qjl"][j:j + 1].reshape(1, -1), g["rnorm"][j:j + 1])[0, 0]
+                assert abs(sc - kth) <= 2 * tol, (r, j, sc, kth)
+
+
+def test_topk_small_with_ties_and_short_db(cuda):
+    c = _ctx(200, 4, 3, 200, seed=5)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(5000, 200, seed=3)
+    X[17] = X[4]
+    Q = tq_inputs.mixture(40, 200, seed=4, means_seed=3)
+    db = c.quantize(X.to(cuda), tq.TQ_KEY)
+    idx, score = c.topk(Q.to(cuda), db, 10)
+    torch.cuda.synchronize()
+    g = _flat(db, 5000)
+    _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), 10)
+    # fewer database vectors than k: the rest is (-1, -inf)
+    small = {k: (None if v is None else v[:5]) for k, v in db.items()}
+    idx2, score2 = c.topk(Q[:3].to(cuda), small, 10)
+    torch.cuda.synchronize()
+    assert np.all(idx2.cpu().numpy()[:, 5:] == -1) and np.all(np.isneginf(score2.cpu().numpy()[:, 5:]))
+    assert sorted(idx2.cpu().numpy()[0, :5].tolist()) == [0, 1, 2, 3, 4]
+
+
+def test_topk_vector_search_full(cuda):
+    """1e6 unit-norm d=200 mixture vectors, 1e4 queries, 3-bit + QJL, top-10;
+    the oracle checks the first 32 queries on the same codes."""
+    c = _ctx(200, 4, 3, 200, seed=11)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(1_000_000, 200, seed=21, device=cuda)
+    Q = tq_inputs.mixture(10_000, 200, seed=22, means_seed=21, device=cuda)
+    db = c.quantize(X, tq.TQ_KEY)
+    n = 8192
+    P.check_quantized(tab, "k", P.to_np(X[:n]), _flat({k: v[:n] for k, v in db.items()}, n))
+    idx, score = c.topk(Q, db, 10)
+    torch.cuda.synchronize()
+    g = _flat(db, 1_000_000)
+    _check_topk(tab, P.to_np(Q[:32]), g, idx[:32].cpu().numpy(), score[:32].cpu().numpy(), 10)
+    assert np.all(np.diff(score.cpu().numpy(), axis=1) <= 0)
+
+
+# --- error reporting through the C ABI ----------------------------------------------
+def test_errors_are_reported(cuda):
+    c = _ctx(128, 3, 4, 128)
+    K = torch.randn(4, 1, 16, 128, device=cuda)
+    kc, vc = _cache(c, K, K, cuda)
+    q = torch.randn(4, 8, 128, device=cuda)
+    lens = torch.full((4,), 16, dtype=torch.int32, device=cuda)
+    small = torch.empty(16, dtype=torch.uint8, device=cuda)
+    with pytest.raises(tq.TQError) as e:
+        c.attn_decode(q, kc, vc, lens, workspace=small)
+    assert e.value.status == tq.TQ_ERR_WORKSPACE
+    with pytest.raises(tq.TQError) as e:
+        c.attn_decode(torch.randn(4, 34, 128, device=cuda), kc, vc, lens)
+    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+    with pytest.raises(tq.TQError) as e:
+        tq._check(tq._lib.tq_quantize(c.ptr, 7, None, 0, 1, 128, None, None, None, None, None))
+    assert e.value.status == tq.TQ_ERR_ARG
+
+
+def test_quantize_append_writes_addressed_slots(cuda):
+    c = _ctx(128, 3, 4, 128, seed=0)
+    B, H, T = 3, 2, 50
+    x = tq_inputs.outlier_kv(B, H, 1, 128, seed=9)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([0, 49, 17], dtype=torch.int32, device=cuda)
+    for which in (tq.TQ_KEY, tq.TQ_VALUE):
+        cache = c.empty_packed(which, (B, H, T), device=cuda)
+        for v in cache.values():
+            if v is not None:
+                v.fill_(-7)
+        c.quantize_append(x, which, cache, pos)
+        ref = c.quantize(x.reshape(B * H, 128), which)
+        torch.cuda.synchronize()
+        for k, v in cache.items():
+            if v is None:
+                continue
+            got = v.cpu()
+            want = ref[k].cpu().reshape((B, H) + tuple(v.shape[3:]))
+            for b in range(B):
+                p = int(pos[b])
+                assert torch.equal(got[b, :, p], want[b]), (k, b)
+                mask = torch.ones(T, dtype=torch.bool)
+                mask[p] = False
+                assert torch.all(got[b][:, mask] == -7), (k, b)

@@ -35,10 +35,14 @@ def iid(shape, seed: int, device="cpu", dtype=torch.float32) -> torch.Tensor:
 
 
 def outlier_kv(B: int, H: int, T: int, d: int, seed: int, device="cpu",
-               outlier_p: float = 0.01, outlier_scale: float = 20.0) -> torch.Tensor:
+               outlier_p: float = 0.01, outlier_scale: float = 20.0,
+               scale_seed: int | None = None) -> torch.Tensor:
+    """`scale_seed` fixes the per-(head, channel) scales independently of
+    `seed`, so that several calls (e.g. one per sequence) share them."""
     g = _gen(seed, device)
-    scale = torch.exp(torch.randn(H, d, generator=g, device=device))
-    heavy = torch.rand(H, d, generator=g, device=device) < outlier_p
+    gs = g if scale_seed is None else _gen(scale_seed, device)
+    scale = torch.exp(torch.randn(H, d, generator=gs, device=device))
+    heavy = torch.rand(H, d, generator=gs, device=device) < outlier_p
     scale = torch.where(heavy, scale * outlier_scale, scale)
     out = torch.empty(B, H, T, d, device=device, dtype=torch.bfloat16)
     # Draw per (b, h) slice to bound the fp32 temporary.
