@@ -175,7 +175,7 @@ class Context:
         L = self.layout(which)
         lead = tuple(lead_shape)
         out = {
-            "codes": torch.empty(lead + (L["bits"], L["words"]), dtype=torch.int32, device=device),
+            "codes": torch.empty(lead + (L["words"],), dtype=torch.int32, device=device),
             "norm": torch.empty(lead, dtype=torch.float32, device=device),
             "qjl": None, "rnorm": None,
         }

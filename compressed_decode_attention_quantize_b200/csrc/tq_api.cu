@@ -118,6 +118,8 @@ tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
   c->bits_v = bits_v;
   c->qjl_m = qjl_m;
   c->seed = seed;
+  c->wk = tq_code_words(d, c->bk_lm);
+  c->wv = tq_code_words(d, bits_v);
   tqh::rotation(d, seed, c->Pi);
   tqh::qjl_matrix(qjl_m, d, seed, c->S);
   tqh::lloyd_max(d, c->bk_lm, c->ck, c->bk);
@@ -204,11 +206,11 @@ int tq_layout(const tq_ctx* c, int which, tq_layout_t* out) {
   const bool key = which == TQ_KEY;
   out->d = c->d;
   out->bits = key ? c->bk_lm : c->bits_v;
-  out->words = c->J;
+  out->words = key ? c->wk : c->wv;
   out->qjl_m = key ? c->qjl_m : 0;
   out->qjl_words = (out->qjl_m + 31) / 32;
   out->has_rnorm = (key && c->qjl_m > 0) ? 1 : 0;
-  out->bytes_per_vector = (int64_t)out->bits * c->J * 4 + (int64_t)out->qjl_words * 4 + 4 +
+  out->bytes_per_vector = (int64_t)out->words * 4 + (int64_t)out->qjl_words * 4 + 4 +
                           (out->has_rnorm ? 4 : 0);
   return TQ_OK;
 }
@@ -250,6 +252,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.bits = key ? c->bk_lm : c->bits_v;
   a.nbnd = (1 << a.bits) - 1;
   a.m = m;
+  a.words = key ? c->wk : c->wv;
   a.PiT = c->PiT;
   a.ST = c->ST;
   a.cen = key ? c->ck_f : c->cv_f;
@@ -364,6 +367,8 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.bk = c->bk_lm;
   a.bv = c->bits_v;
   a.m = c->qjl_m;
+  a.wk = c->wk;
+  a.wv = c->wv;
   a.kcodes = kcodes;
   a.kqjl = kqjl;
   a.knorm = knorm;

@@ -18,6 +18,8 @@ struct tq_ctx {
   int bk_lm = 0;    // key Lloyd-Max bits
   int bits_v = 0;   // value Lloyd-Max bits
   int qjl_m = 0;    // QJL rows (0 = none)
+  int wk = 0;       // code words per key vector
+  int wv = 0;       // code words per value vector
   int device = 0;
   uint64_t seed = 0;
   // fp64 host tables
@@ -41,13 +43,20 @@ void qjl_matrix(int m, int d, uint64_t seed, std::vector<double>& S);
 void lloyd_max(int d, int bits, std::vector<double>& cen, std::vector<double>& bnd);
 }  // namespace tqh
 
+// Code words per vector for d coordinates of b-bit indices (field layout).
+inline int tq_code_words(int d, int b) {
+  if (b == 3) return (d + 15) / 16 + (d + 31) / 32;
+  const int per = 32 / b;
+  return (d + per - 1) / per;
+}
+
 namespace tqk {
 
 struct QuantArgs {
   const void* x;
   int dtype;
   int64_t n, ld;
-  int d, bits, nbnd, m;
+  int d, bits, nbnd, m, words;
   const float* PiT;
   const float* ST;
   const float* cen;
@@ -66,7 +75,7 @@ struct QuantArgs {
 struct AttnArgs {
   const float* qr;   // [B*Hq][dpad] pre-rotated queries
   const float* qs;   // [B*Hq][dpad] S q'
-  int B, Hq, Hkv, G, d, bk, bv, m;
+  int B, Hq, Hkv, G, d, bk, bv, m, wk, wv;
   const uint32_t* kcodes;
   const uint32_t* kqjl;
   const float* knorm;

@@ -53,12 +53,25 @@ __device__ __forceinline__ int64_t out_record(const QuantArgs& a, int64_t v) {
   return v * a.max_T + a.pos[b];
 }
 
-// Lloyd-Max index of coordinate j from its bit-planes (plane stride J words).
-__device__ __forceinline__ int plane_index(const uint32_t* w, int bits, int J, int j) {
-  const int wi = j >> 5, e = j & 31;
-  int idx = 0;
-  for (int p = 0; p < bits; ++p) idx |= ((w[p * J + wi] >> e) & 1u) << p;
-  return idx;
+// Lloyd-Max index of coordinate j of a packed vector (b-bit fields; for b = 3
+// a 2-bit stream of the low bits followed by a 1-bit stream of the top bits).
+__device__ __forceinline__ int code_index(const uint32_t* w, int bits, int d, int j) {
+  if (bits == 3) {
+    const int lo = (w[j >> 4] >> ((j & 15) * 2)) & 3;
+    const int hi = (w[((d + 15) >> 4) + (j >> 5)] >> (j & 31)) & 1;
+    return lo | (hi << 2);
+  }
+  const int per = 32 / bits;
+  return (w[j / per] >> (bits * (j % per))) & ((1 << bits) - 1);
+}
+
+// OR of the b-bit field of each lane placed at its slot, over groups of 32/b
+// consecutive lanes (every lane of the group ends with the group's word).
+__device__ __forceinline__ uint32_t field_word(uint32_t val, int b, int lane) {
+  const int per = 32 / b;
+  uint32_t x = val << (b * (lane % per));
+  for (int o = 1; o < per; o <<= 1) x |= __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
 }
 
 // ----------------------------------------------------------------------------
@@ -84,7 +97,6 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
   }
   __syncthreads();
   const int64_t ngroups = (a.n + QV - 1) / QV;
-  const int words = a.bits * J;
   const int mwords = (a.m + 31) >> 5;
   for (int64_t g = (int64_t)blockIdx.x * QWARPS + warp; g < ngroups;
        g += (int64_t)gridDim.x * QWARPS) {
@@ -133,19 +145,29 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
         idx[i][v] = (unsigned char)lm_index(y, s_bnd, a.nbnd);
       }
     }
-    // Bit-plane packing: word i of plane p is a ballot over the lanes.
+    // Field packing: lane owns coordinates lane + 32 i; a group of 32/b lanes
+    // fills one word (b = 3: 2-bit stream of low bits, then 1-bit stream).
 #pragma unroll
     for (int v = 0; v < QV; ++v) {
-      uint32_t mine = 0;
-      for (int p = 0; p < a.bits; ++p) {
+      const bool live = v0 + v < a.n;
+      const int64_t base = live ? out_record(a, v0 + v) * a.words : 0;
 #pragma unroll
-        for (int i = 0; i < J; ++i) {
-          const bool bit = ((idx[i][v] >> p) & 1) && (lane + 32 * i < a.d);
-          const uint32_t w = __ballot_sync(0xffffffffu, bit);
-          if (lane == p * J + i) mine = w;
+      for (int i = 0; i < J; ++i) {
+        const uint32_t iv = (lane + 32 * i < a.d) ? idx[i][v] : 0u;
+        if (a.bits == 3) {
+          const int w2 = (a.d + 15) >> 4;
+          const uint32_t lo = field_word(iv & 3u, 2, lane);
+          const uint32_t hi = field_word(iv >> 2, 1, lane);
+          const int wlo = 2 * i + (lane >> 4);
+          if (live && (lane & 15) == 0 && wlo < w2) a.codes[base + wlo] = lo;
+          if (live && lane == 0) a.codes[base + w2 + i] = hi;
+        } else {
+          const int per = 32 / a.bits;
+          const uint32_t wv = field_word(iv, a.bits, lane);
+          const int wi = a.bits * i + lane / per;
+          if (live && lane % per == 0 && wi < a.words) a.codes[base + wi] = wv;
         }
       }
-      if (v0 + v < a.n && lane < words) a.codes[out_record(a, v0 + v) * words + lane] = mine;
     }
     float my_norm = 0.f;
 #pragma unroll
@@ -252,7 +274,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
   float* sq = sh;                       // [G][DP]
   float* ssv = sq + a.G * DP;           // [G][DP]
   float* sp = ssv + a.G * DP;           // [AT][G]   p * |v|
-  uint32_t* svc = reinterpret_cast<uint32_t*>(sp + AT * a.G);  // [AT][bv*J]
+  uint32_t* svc = reinterpret_cast<uint32_t*>(sp + AT * a.G);  // [AT][wv]
   __shared__ float s_ck[16], s_cv[16];
   __shared__ float s_wred[AT / 32][GMAX];
 
@@ -282,7 +304,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
   }
   __syncthreads();
   const int64_t kv_row0 = ((int64_t)b * a.Hkv + g) * a.max_T;
-  const int kw = a.bk * J, vw = a.bv * J, mw = (a.m + 31) >> 5;
+  const int kw = a.wk, vw = a.wv, mw = (a.m + 31) >> 5;
 
   for (int64_t t0 = t_begin; t0 < t_end; t0 += AT) {
     const int64_t t = t0 + tid;
@@ -299,7 +321,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
 #pragma unroll
       for (int h = 0; h < GMAX; ++h) acc[h] = acc2[h] = 0.f;
       for (int j = 0; j < a.d; ++j) {
-        const float c = s_ck[plane_index(w, a.bk, J, j)];
+        const float c = s_ck[code_index(w, a.bk, a.d, j)];
 #pragma unroll
         for (int h = 0; h < GMAX; ++h)
           if (h < G) acc[h] = fmaf(sq[h * DP + j], c, acc[h]);
@@ -377,7 +399,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
       const int j = tid + AT * jj;
       if (j < a.d) {
         for (int tt = 0; tt < ntile; ++tt) {
-          const float c = s_cv[plane_index(svc + tt * vw, a.bv, J, j)];
+          const float c = s_cv[code_index(svc + tt * vw, a.bv, a.d, j)];
 #pragma unroll
           for (int h = 0; h < GMAX; ++h)
             if (h < G) o[h][jj] = fmaf(sp[tt * G + h], c, o[h][jj]);
@@ -442,8 +464,8 @@ constexpr int LQB = 8;
 
 template <int J>
 __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_t nq, int d,
-                                                int bk, int m, const float* PiT, const float* ST,
-                                                const float* ck, float cq,
+                                                int bk, int kw, int m, const float* PiT,
+                                                const float* ST, const float* ck, float cq,
                                                 const uint32_t* kcodes, const uint32_t* kqjl,
                                                 const float* knorm, const float* krnorm,
                                                 int64_t nk, float* out) {
@@ -475,14 +497,14 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
   __syncthreads();
   const int64_t key = (int64_t)blockIdx.x * blockDim.x + tid;
   if (key >= nk) return;
-  const int kw = bk * J, mw = (m + 31) >> 5;
+  const int mw = (m + 31) >> 5;
   uint32_t w[4 * 8];
   for (int e = 0; e < kw; ++e) w[e] = kcodes[key * kw + e];
   float acc[LQB], acc2[LQB];
 #pragma unroll
   for (int qq = 0; qq < LQB; ++qq) acc[qq] = acc2[qq] = 0.f;
   for (int j = 0; j < d; ++j) {
-    const float c = s_ck[plane_index(w, bk, J, j)];
+    const float c = s_ck[code_index(w, bk, d, j)];
 #pragma unroll
     for (int qq = 0; qq < LQB; ++qq) acc[qq] = fmaf(sq[qq][j], c, acc[qq]);
   }
@@ -506,7 +528,7 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
 // Dequantize one vector per CTA: rot_j = |x| c[idx_j] (+ C gamma (S^T sigma)_j),
 // then x_hat = Pi^T rot.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int m,
+__global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int words, int m,
                                                  const float* Pi, const float* S,
                                                  const float* cen, float cq,
                                                  const uint32_t* codes, const uint32_t* qjl,
@@ -515,13 +537,12 @@ __global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int 
   extern __shared__ float sh[];
   float* srot = sh;  // [dpad]
   const int64_t v = blockIdx.x;
-  const int J = dpad / 32;
-  const int words = bits * J, mw = (m + 31) >> 5;
+  const int mw = (m + 31) >> 5;
   const uint32_t* w = codes + v * words;
   const float n = norm[v];
   const float kg = m > 0 ? rnorm[v] * cq : 0.f;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float r = n * cen[plane_index(w, bits, J, j)];
+    float r = n * cen[code_index(w, bits, d, j)];
     if (m > 0) {
       float acc = 0.f;
       for (int i = 0; i < m; ++i) {
@@ -558,7 +579,8 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
 
 template <int J>
 __global__ void __launch_bounds__(TTH) k_topk_chunk(const float* qr, const float* qs, int64_t nq,
-                                                    int d, int bk, int m, const float* ck, float cq,
+                                                    int d, int bk, int kw, int m, const float* ck,
+                                                    float cq,
                                                     const uint32_t* codes, const uint32_t* qjl,
                                                     const float* norm, const float* rnorm,
                                                     int64_t n, int K, float* cand_v, int* cand_i,
@@ -586,7 +608,7 @@ __global__ void __launch_bounds__(TTH) k_topk_chunk(const float* qr, const float
     stop_i[e] = INT_MAX;
   }
   __syncthreads();
-  const int kw = bk * J, mw = (m + 31) >> 5;
+  const int mw = (m + 31) >> 5;
   const int64_t base = (int64_t)chunk * TSTEPS * TTH;
   for (int step = 0; step < TSTEPS; ++step) {
     const int64_t v = base + (int64_t)step * TTH + tid;
@@ -597,7 +619,7 @@ __global__ void __launch_bounds__(TTH) k_topk_chunk(const float* qr, const float
 #pragma unroll
       for (int qq = 0; qq < TQ; ++qq) acc[qq] = acc2[qq] = 0.f;
       for (int j = 0; j < d; ++j) {
-        const float c = s_ck[plane_index(w, bk, J, j)];
+        const float c = s_ck[code_index(w, bk, d, j)];
         const float4* qp = reinterpret_cast<const float4*>(sq + j * TQ);
 #pragma unroll
         for (int q4 = 0; q4 < TQ / 4; ++q4) {
@@ -740,7 +762,7 @@ cudaError_t quantize_J(const QuantArgs& a, cudaStream_t s) {
 template <int J>
 cudaError_t attn_J(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
   const size_t shm = (size_t)(2 * a.G * J * 32 + AT * a.G) * sizeof(float) +
-                     (size_t)AT * a.bv * J * sizeof(uint32_t);
+                     (size_t)AT * a.wv * sizeof(uint32_t);
   if (shm > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
@@ -806,7 +828,7 @@ cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   if (nq == 0 || nk == 0) return cudaSuccess;
   dim3 grid((unsigned)((nk + 127) / 128), (unsigned)((nq + LQB - 1) / LQB));
   const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
-  TQ_DISPATCH_J(c->J, k_logits<JV><<<grid, 128, 0, s>>>(q, dtype, nq, c->d, c->bk_lm, c->qjl_m,
+  TQ_DISPATCH_J(c->J, k_logits<JV><<<grid, 128, 0, s>>>(q, dtype, nq, c->d, c->bk_lm, c->wk, c->qjl_m,
                                                         c->PiT, c->ST, c->ck_f, cq, kcodes, kqjl,
                                                         knorm, krnorm, nk, out);
                 return cudaGetLastError());
@@ -820,7 +842,8 @@ cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
   const int m = key ? c->qjl_m : 0;
   const float cq = m > 0 ? (float)(std::sqrt(M_PI / 2.0) / m) : 0.f;
   k_dequant<<<(unsigned)n, 128, c->dpad * sizeof(float), s>>>(
-      c->d, c->dpad, key ? c->bk_lm : c->bits_v, m, c->Pi_f, c->S_f, key ? c->ck_f : c->cv_f, cq,
+      c->d, c->dpad, key ? c->bk_lm : c->bits_v, key ? c->wk : c->wv, m, c->Pi_f, c->S_f,
+      key ? c->ck_f : c->cv_f, cq,
       codes, qjl, norm, rnorm, out);
   return cudaGetLastError();
 }
@@ -862,7 +885,7 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   TQ_DISPATCH_J(c->J, {
     e = cudaFuncSetAttribute(k_topk_chunk<JV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
-    k_topk_chunk<JV><<<grid, TTH, shm, s>>>(qr, qs, nq, c->d, c->bk_lm, c->qjl_m, c->ck_f, cq,
+    k_topk_chunk<JV><<<grid, TTH, shm, s>>>(qr, qs, nq, c->d, c->bk_lm, c->wk, c->qjl_m, c->ck_f, cq,
                                              codes, qjl, norm, rnorm, n, k, cv, ci, (int)nch);
     break;
   });

@@ -36,18 +36,23 @@
  * - Sizes: 8 <= d <= 256 with d % 8 == 0; Lloyd-Max bits 1..4;
  *   0 <= qjl_m <= 32*ceil(d/32), qjl_m % 8 == 0.
  *
- * Packed layout of one vector (W = ceil(d/32) words per bit-plane)
- * -----------------------------------------------------------------
- *   codes  uint32[b][W]  plane p holds bit p of every Lloyd-Max index;
- *                        coordinate j sits at bit j%32 of word j/32 (LSB
- *                        first); padding bits are 0.
- *   qjl    uint32[ceil(m/32)]  keys only: bit i = 1 when (S r)_i >= 0.
- *   norm   float         |x| (fp32).
- *   rnorm  float         keys with QJL only: gamma = |x| * |r|, r the residual
- *                        of the rotated unit vector.
+ * Packed layout of one vector
+ * ---------------------------
+ *   codes  uint32[W]   Lloyd-Max indices as b-bit fields, LSB first, 32/b
+ *                      fields per word, for b in {1, 2, 4}: coordinate j sits
+ *                      in word j/(32/b) at bit b*(j%(32/b)); W = ceil(d*b/32).
+ *                      For b = 3 the low two bits of every index form a 2-bit
+ *                      field stream (ceil(d/16) words) followed by a 1-bit
+ *                      stream of the top bits (ceil(d/32) words).  Padding
+ *                      bits are 0.
+ *   qjl    uint32[ceil(m/32)]  keys only: bit i%32 of word i/32 is 1 when
+ *                      (S r)_i >= 0.
+ *   norm   float       |x| (fp32).
+ *   rnorm  float       keys with QJL only: gamma = |x| * |r|, r the residual
+ *                      of the rotated unit vector.
  * Arrays of vectors are these records laid out as separate dense arrays
- * (codes [N][b][W], qjl [N][ceil(m/32)], norm [N], rnorm [N]).  A KV cache is
- * [B][Hkv][max_T] records in each array.
+ * (codes [N][W], qjl [N][ceil(m/32)], norm [N], rnorm [N]).  A KV cache is
+ * [B][Hkv][max_T] records in each array.  tq_layout reports W.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -74,8 +79,8 @@ typedef struct tq_ctx tq_ctx;
 
 typedef struct tq_layout_t {
   int32_t d;              /* head / vector dimension                        */
-  int32_t bits;           /* Lloyd-Max bits per coordinate (planes)          */
-  int32_t words;          /* W = ceil(d/32) words per plane                  */
+  int32_t bits;           /* Lloyd-Max bits per coordinate                    */
+  int32_t words;          /* W, code words per vector                         */
   int32_t qjl_m;          /* QJL rows (0 for values or when disabled)        */
   int32_t qjl_words;      /* ceil(qjl_m/32)                                  */
   int32_t has_rnorm;      /* 1 when an rnorm (gamma) array is produced       */
@@ -135,7 +140,7 @@ int tq_export_tables(const tq_ctx* ctx, double* pi, double* S, double* ck,
  *   which   TQ_KEY or TQ_VALUE.
  *   x       device, [n][ld] elements of `dtype` (TQ_F32/TQ_BF16/TQ_F16),
  *           ld >= d; rows 16-byte aligned when dtype is 16-bit and ld%8==0.
- *   codes   device, uint32 [n][bits][W].
+ *   codes   device, uint32 [n][W].
  *   qjl     device, uint32 [n][ceil(m/32)] (keys with QJL; else ignored, may be NULL).
  *   norm    device, float [n].
  *   rnorm   device, float [n] (keys with QJL; else ignored, may be NULL).
@@ -200,9 +205,9 @@ size_t tq_attn_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int64_t max_T);
  * The context is split over CTAs; partial softmax states are merged by
  * log-sum-exp and the Pi^T is applied once per head after the merge.
  *   q        device, [B][Hq][d] of `dtype`.
- *   kcodes   device, uint32 [B][Hkv][max_T][bits_k_lm][W]; kqjl [B][Hkv][max_T][ceil(m/32)];
+ *   kcodes   device, uint32 [B][Hkv][max_T][Wk]; kqjl [B][Hkv][max_T][ceil(m/32)];
  *   knorm, krnorm  device, float [B][Hkv][max_T].
- *   vcodes   device, uint32 [B][Hkv][max_T][bits_v][W]; vnorm float [B][Hkv][max_T].
+ *   vcodes   device, uint32 [B][Hkv][max_T][Wv]; vnorm float [B][Hkv][max_T].
  *   seq_lens device, int32 [B], each in [0, max_T]; a length of 0 gives out = 0.
  *   scale    softmax scale (callers usually pass 1/sqrt(d)).
  *   out      device, float [B][Hq][d].

@@ -224,40 +224,67 @@ def make_tables(d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int) -> Tabl
 
 
 # ----------------------------------------------------------------------------
-# Bit packing.  codes: uint32 [N, b, W]; plane p holds bit p of every index,
-# coordinate j at bit j%32 of word j/32 (LSB first), W = ceil(d/32), padding
-# bits zero.  QJL: uint32 [N, ceil(m/32)], bit i set when sigma_i = +1.
+# Bit packing (the library's own layout; the pages only say the fused kernel
+# reads the indices directly).  A vector's Lloyd-Max indices are packed as
+# b-bit fields, LSB first, 32/b fields per uint32 word, for b in {1, 2, 4}:
+# coordinate j sits in word j // (32/b) at bit b * (j % (32/b)).  For b = 3
+# the low two bits of every index form a 2-bit field stream and the top bit a
+# 1-bit stream that follows it.  Padding bits are zero.  QJL bits form a 1-bit
+# stream (bit i set when sigma_i = +1).
 # ----------------------------------------------------------------------------
+def field_words(n: int, b: int) -> int:
+    per = 32 // b
+    return (n + per - 1) // per
+
+
+def code_words(d: int, bits: int) -> int:
+    if bits == 3:
+        return field_words(d, 2) + field_words(d, 1)
+    return field_words(d, bits)
+
+
+def pack_fields(vals: np.ndarray, b: int) -> np.ndarray:
+    """vals: [..., n] integers in [0, 2^b) -> uint32 [..., ceil(n*b/32)]."""
+    vals = np.asarray(vals, dtype=np.uint64)
+    n = vals.shape[-1]
+    per = 32 // b
+    W = field_words(n, b)
+    pad = np.zeros(vals.shape[:-1] + (W * per - n,), dtype=np.uint64)
+    v = np.concatenate([vals, pad], axis=-1).reshape(vals.shape[:-1] + (W, per))
+    shifts = (np.uint64(b) * np.arange(per, dtype=np.uint64))
+    return (v << shifts).sum(axis=-1).astype(np.uint32)
+
+
+def unpack_fields(words: np.ndarray, n: int, b: int) -> np.ndarray:
+    words = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    per = 32 // b
+    shifts = np.uint64(b) * np.arange(per, dtype=np.uint64)
+    v = (words[..., :, None] >> shifts) & np.uint64((1 << b) - 1)
+    return v.reshape(words.shape[:-1] + (-1,))[..., :n].astype(np.int64)
+
+
 def pack_bits(bits: np.ndarray) -> np.ndarray:
     """bits: [..., n] of 0/1 -> uint32 [..., ceil(n/32)], LSB first."""
-    bits = np.asarray(bits, dtype=np.uint64)
-    n = bits.shape[-1]
-    W = (n + 31) // 32
-    pad = np.zeros(bits.shape[:-1] + (W * 32 - n,), dtype=np.uint64)
-    b = np.concatenate([bits, pad], axis=-1).reshape(bits.shape[:-1] + (W, 32))
-    weights = np.uint64(1) << np.arange(32, dtype=np.uint64)
-    return (b * weights).sum(axis=-1).astype(np.uint32)
+    return pack_fields(bits, 1)
 
 
 def unpack_bits(words: np.ndarray, n: int) -> np.ndarray:
-    words = np.asarray(words, dtype=np.uint32)
-    shifts = np.arange(32, dtype=np.uint32)
-    b = (words[..., :, None] >> shifts) & np.uint32(1)
-    return b.reshape(words.shape[:-1] + (-1,))[..., :n].astype(np.int64)
+    return unpack_fields(words, n, 1)
 
 
-def pack_planes(idx: np.ndarray, bits: int) -> np.ndarray:
+def pack_codes(idx: np.ndarray, bits: int) -> np.ndarray:
     idx = np.asarray(idx, dtype=np.int64)
-    planes = [pack_bits((idx >> p) & 1) for p in range(bits)]
-    return np.stack(planes, axis=-2)
+    if bits == 3:
+        return np.concatenate([pack_fields(idx & 3, 2), pack_fields(idx >> 2, 1)], axis=-1)
+    return pack_fields(idx, bits)
 
 
-def unpack_planes(codes: np.ndarray, bits: int, d: int) -> np.ndarray:
+def unpack_codes(codes: np.ndarray, bits: int, d: int) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.uint32)
-    idx = np.zeros(codes.shape[:-2] + (d,), dtype=np.int64)
-    for p in range(bits):
-        idx |= unpack_bits(codes[..., p, :], d) << p
-    return idx
+    if bits == 3:
+        w2 = field_words(d, 2)
+        return unpack_fields(codes[..., :w2], d, 2) | (unpack_fields(codes[..., w2:], d, 1) << 2)
+    return unpack_fields(codes, d, bits)
 
 
 # ----------------------------------------------------------------------------
@@ -277,7 +304,7 @@ def qjl_signs(S: np.ndarray, r: np.ndarray) -> np.ndarray:
 @dataclass
 class Quantized:
     idx: np.ndarray        # [N, d] int64 Lloyd-Max indices
-    codes: np.ndarray      # [N, b, W] uint32
+    codes: np.ndarray      # [N, code_words(d, b)] uint32
     norm: np.ndarray       # [N] fp32 (R4)
     y: np.ndarray          # [N, d] rotated unit vectors (fp64), for band checks
     qjl_bits: np.ndarray | None = None   # [N, m] 0/1
@@ -300,7 +327,7 @@ def quantize(x: np.ndarray, tab: Tables, which: str) -> Quantized:
     u = np.where((n > 0.0)[:, None], x / safe[:, None], 0.0)
     y = u @ tab.Pi.T
     idx = lloyd_max_index(y, cb)
-    q = Quantized(idx=idx, codes=pack_planes(idx, cb.bits),
+    q = Quantized(idx=idx, codes=pack_codes(idx, cb.bits),
                   norm=n.astype(np.float32), y=y)
     if which == "k" and tab.qjl_m > 0:
         sketch_from_indices(q, tab)
@@ -338,7 +365,7 @@ def qjl_constant(m: int) -> float:
 def dequantize(tab: Tables, which: str, codes, norm, qjl=None, rnorm=None) -> np.ndarray:
     """x_hat = n Pi^T c[idx]  (+ C gamma Pi^T S^T sigma for keys with QJL, R12)."""
     cb = tab.cb_k if which == "k" else tab.cb_v
-    idx = unpack_planes(codes, cb.bits, tab.d)
+    idx = unpack_codes(codes, cb.bits, tab.d)
     rot = cb.centroids[idx] * np.asarray(norm, dtype=np.float64)[:, None]
     if which == "k" and tab.qjl_m > 0:
         sigma = 2.0 * unpack_bits(qjl, tab.qjl_m) - 1.0
@@ -351,7 +378,7 @@ def logits(tab: Tables, q: np.ndarray, codes, norm, qjl=None, rnorm=None) -> np.
     q: [nq, d]; codes etc. for nk keys; returns [nq, nk]."""
     q = np.asarray(q, dtype=np.float64)
     qr = q @ tab.Pi.T                       # pre-rotated query
-    idx = unpack_planes(codes, tab.cb_k.bits, tab.d)
+    idx = unpack_codes(codes, tab.cb_k.bits, tab.d)
     chat = tab.cb_k.centroids[idx]          # [nk, d]
     out = (qr @ chat.T) * np.asarray(norm, dtype=np.float64)[None, :]
     if tab.qjl_m > 0:

@@ -50,9 +50,10 @@ def check_quantized(tab, which, x, gpu, report=None):
     cb = tab.cb_k if which == "k" else tab.cb_v
     n = x.shape[0]
     q = o.quantize(x, tab, which)
-    codes = gpu["codes"].reshape(n, cb.bits, -1)
-    gidx = o.unpack_planes(codes, cb.bits, d)
-    assert np.array_equal(codes, o.pack_planes(gidx, cb.bits)), "non-canonical packing"
+    codes = gpu["codes"].reshape(n, -1)
+    assert codes.shape[1] == o.code_words(d, cb.bits)
+    gidx = o.unpack_codes(codes, cb.bits, d)
+    assert np.array_equal(codes, o.pack_codes(gidx, cb.bits)), "non-canonical packing"
     mism = gidx != q.idx
     band = o.boundary_distance(q.y, cb) < BAND
     assert not np.any(mism & ~band), f"{int(np.sum(mism & ~band))} index mismatches outside the band"
@@ -82,7 +83,7 @@ def check_quantized(tab, which, x, gpu, report=None):
 def check_logits(tab, q, gpu_keys, gpu_logits):
     """q: fp64 [nq, d]; gpu_keys: numpy dict [nk, ...]; gpu_logits [nq, nk]."""
     nk = gpu_keys["norm"].size
-    ref = o.logits(tab, q, gpu_keys["codes"].reshape(nk, tab.bits_k_lm, -1),
+    ref = o.logits(tab, q, gpu_keys["codes"].reshape(nk, -1),
                    gpu_keys["norm"].reshape(nk),
                    None if gpu_keys.get("qjl") is None else gpu_keys["qjl"].reshape(nk, -1),
                    None if gpu_keys.get("rnorm") is None else gpu_keys["rnorm"].reshape(nk))

@@ -28,10 +28,10 @@ def _flat(p, n):
 # --- layout and tables ------------------------------------------------------
 def test_layout_bytes(cuda):
     c = _ctx(128, 3, 4, 128)
-    assert c.key_layout["bytes_per_vector"] == 56      # 2 planes x 16 B + 16 B QJL + |k| + gamma
-    assert c.value_layout["bytes_per_vector"] == 68    # 4 planes x 16 B + |v|
+    assert c.key_layout["bytes_per_vector"] == 56      # 2-bit fields 32 B + 16 B QJL + |k| + gamma
+    assert c.value_layout["bytes_per_vector"] == 68    # 4-bit fields 64 B + |v|
     c2 = _ctx(200, 4, 3, 200)
-    assert c2.key_layout["words"] == 7 and c2.key_layout["qjl_words"] == 7
+    assert c2.key_layout["words"] == 13 + 7 and c2.key_layout["qjl_words"] == 7  # 3-bit: 2-bit + 1-bit streams
 
 
 def test_device_context_tables_match_oracle(cuda):
@@ -108,7 +108,7 @@ def test_quantize_edge_cases(cuda):
         P.check_quantized(tab, "k", x, _flat(pk, 37))
         g = P.packed_np(pk)
         assert g["norm"][0] == 0 and g["rnorm"][0] == 0
-        assert np.all(o.unpack_planes(g["codes"][0], 2, 64) == 2)
+        assert np.all(o.unpack_codes(g["codes"][0], 2, 64) == 2)
 
 
 # --- dequantize / logits ---------------------------------------------------------
@@ -121,7 +121,7 @@ def test_dequantize_matches_oracle(cuda):
         xh = c.dequantize(which, p)
         torch.cuda.synchronize()
         g = _flat(p, 500)
-        ref = o.dequantize(tab, wch, g["codes"].reshape(500, -1, 4), g["norm"], g["qjl"], g["rnorm"])
+        ref = o.dequantize(tab, wch, g["codes"], g["norm"], g["qjl"], g["rnorm"])
         err = np.linalg.norm(xh.cpu().double().numpy() - ref, axis=1) / np.linalg.norm(ref, axis=1)
         assert err.max() < 1e-5
 
@@ -229,7 +229,7 @@ def _oracle_topk_chunked(tab, q, g, k, chunk=25_000):
     best_i = np.zeros((q.shape[0], 0), dtype=np.int64)
     for s in range(0, n, chunk):
         e = min(n, s + chunk)
-        sc = o.logits(tab, q, g["codes"][s:e].reshape(e - s, tab.bits_k_lm, -1), g["norm"][s:e],
+        sc = o.logits(tab, q, g["codes"][s:e], g["norm"][s:e],
                       g["qjl"][s:e].reshape(e - s, -1), g["rnorm"][s:e])
         best_v = np.concatenate([best_v, sc], axis=1)
         best_i = np.concatenate([best_i, np.broadcast_to(np.arange(s, e), sc.shape)], axis=1)
@@ -250,7 +250,7 @@ def _check_topk(tab, q, g, idx, score, k):
             diff = set(idx[r]) ^ set(ref_i[r])
             kth = ref_v[r, -1]
             for j in diff:
-                sc = o.logits(tab, q[r:r + 1], g["codes"][j:j + 1].reshape(1, tab.bits_k_lm, -1),
+                sc = o.logits(tab, q[r:r + 1], g["codes"][j:j + 1],
                               g["norm"][j:j + 1], g["qjl"][j:j + 1].reshape(1, -1), g["rnorm"][j:j + 1])[0, 0]
                 assert abs(sc - kth) <= 2 * tol, (r, j, sc, kth)
 

@@ -148,19 +148,21 @@ def test_printed_three_bit_cosine():
 
 # --- packing ---------------------------------------------------------------
 def test_packing_worked_example():
-    rows = {r[0]: [int(t, 16) for t in r[1:]] for r in _golden_lines("packing_d40_b2.txt")}
-    idx = (np.arange(40) % 4)[None, :]
-    codes = o.pack_planes(idx, 2)
-    assert codes.dtype == np.uint32 and codes.shape == (1, 2, 2)
-    assert list(codes[0, 0]) == rows["plane0"]
-    assert list(codes[0, 1]) == rows["plane1"]
-    assert np.array_equal(o.unpack_planes(codes, 2, 40), idx)
+    rows = {r[0]: [int(t, 16) for t in r[1:]] for r in _golden_lines("packing_fields.txt")}
+    for bits in (1, 2, 3, 4):
+        idx = (np.arange(40) % (1 << bits))[None, :]
+        codes = o.pack_codes(idx, bits)
+        assert codes.dtype == np.uint32 and codes.shape == (1, o.code_words(40, bits))
+        assert list(codes[0]) == rows[f"b{bits}"], bits
+        assert np.array_equal(o.unpack_codes(codes, bits, 40), idx)
 
 
 def test_pack_roundtrip_random():
     rng = np.random.default_rng(1)
-    idx = rng.integers(0, 16, size=(50, 200))
-    assert np.array_equal(o.unpack_planes(o.pack_planes(idx, 4), 4, 200), idx)
+    for bits in (1, 2, 3, 4):
+        for d in (200, 128, 8):
+            idx = rng.integers(0, 1 << bits, size=(50, d))
+            assert np.array_equal(o.unpack_codes(o.pack_codes(idx, bits), bits, d), idx)
     bits = rng.integers(0, 2, size=(50, 72))
     w = o.pack_bits(bits)
     assert w.shape == (50, 3) and np.all(w[:, 2] >> np.uint32(8) == 0)
@@ -220,9 +222,9 @@ def _cache(tab, B, Hkv, T, rng):
     zk = o.quantize(k.reshape(-1, tab.d), tab, "k")
     zv = o.quantize(v.reshape(-1, tab.d), tab, "v")
     r = lambda a, *tail: None if a is None else a.reshape((B, Hkv, T) + tail)
-    W, mw = (tab.d + 31) // 32, (tab.qjl_m + 31) // 32
-    return (r(zk.codes, tab.bits_k_lm, W), r(zk.qjl, mw), r(zk.norm), r(zk.rnorm),
-            r(zv.codes, tab.bits_v, W), r(zv.norm))
+    mw = (tab.qjl_m + 31) // 32
+    return (r(zk.codes, o.code_words(tab.d, tab.bits_k_lm)), r(zk.qjl, mw), r(zk.norm), r(zk.rnorm),
+            r(zv.codes, o.code_words(tab.d, tab.bits_v)), r(zv.norm))
 
 
 def test_attention_brute_force_tiny():
