@@ -318,8 +318,11 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
 size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   if (!c || B <= 0 || Hq <= 0 || max_T < 0) return 0;
   int chunk = 0;
-  const int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
-  // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most splits).
+  int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
+  // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most
+  // splits), and for the tensor-core path's fixed chunk.
+  const int64_t mma_splits = (max_T + tqk::attn_mma_chunk() - 1) / tqk::attn_mma_chunk();
+  if (mma_splits > splits) splits = (int)mma_splits;
   const size_t rows = (size_t)B * Hq;
   size_t b = 2 * rows * c->dpad * sizeof(float);
   b = (b + 255) & ~(size_t)255;
@@ -383,7 +386,14 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.cv = c->cv_f;
   a.splits = tqk::attn_splits(c, B, Hkv, max_T > 0 ? max_T : 1, &a.chunk);
   a.part = part;
-  e = tqk::launch_attn(c, a, out, s);
+  if (tqk::attn_mma_supported(c, a) && max_T > 0) {
+    a.chunk = tqk::attn_mma_chunk();
+    a.splits = (int)((max_T + a.chunk - 1) / a.chunk);
+    if (a.splits > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: context too long");
+    e = tqk::launch_attn_mma(c, a, out, s);
+  } else {
+    e = tqk::launch_attn(c, a, out, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
   return TQ_OK;
 }

@@ -1,0 +1,469 @@
+// Split-K decode attention from packed codes on the tensor cores (sm_100a).
+//
+// Computes, for every query head h of a KV group g of sequence b, the
+// partial softmax state over one chunk of the context ("What is TurboQuant?",
+// "How TurboQuant works", closing paragraph: the logits come straight from
+// the compressed indices; "How to implement" part 1: the query is rotated
+// once and dotted with centroid values):
+//   l_i  = |k_i| <q', c_k[idx_i]> + sqrt(pi/2)/m * gamma_i <S q', sigma_i>
+//   s_i  = scale * l_i,   m = max s,   l = sum exp(s - m),
+//   o    = sum exp(s_i - m) |v_i| c_v[vidx_i]          (rotated domain)
+// The merge kernel combines chunks by log-sum-exp and applies Pi^T once.
+//
+// Fast path: d = 128, keys 2 Lloyd-Max bits + 128 QJL rows, values 4 bits,
+// GQA group size G <= 8.  One CTA = 4 warps over one chunk of tokens of one
+// (sequence, kv head); each warp walks 16-token tiles with its own online
+// softmax and its own cp.async pipeline (4 stages), and the 4 warps merge at
+// the end.  Per tile:
+//  * logits: mma.sync m16n8k16, A = dequantized keys (16 tokens x 16 dims,
+//    fp16), B = pre-rotated query (16 dims x 8 heads, fp16), fp32 accumulate.
+//    2-bit codes become fp16 centroids with one byte-permute per two values
+//    (a 4-entry table in two registers).  QJL bits become +-1 fp16 with one
+//    shift and one logic op per two values; a second accumulator collects
+//    <S q', sigma>.  fp16 alone would round q', S q' and the centroids to 11
+//    bits, which moves the softmax exponent by ~1e-3 for keys with large
+//    norms; each of them is therefore split into an fp16 head and an fp16
+//    tail scaled by 2^12 (c = c_hi + 2^-12 c_lo, likewise q' and S q'), and
+//    the tail products (hi*lo and lo*hi) go to a correction accumulator that
+//    is added in fp32 with weight 2^-12 (error ~2^-22 relative).
+//  * the 16x8 probability tile is transposed into the B operand of the value
+//    product with movmatrix.
+//  * values: mma.sync m16n8k16, A = dequantized values (16 dims x 16 tokens),
+//    B = p * |v| (16 tokens x 8 heads).  A 4-bit code pair (two tokens, one
+//    dim) indexes a 256-entry half2 table in shared memory, one copy per
+//    lane so that every lookup of a warp hits 32 different banks.
+// The head dimension is permuted inside the tiles (a thread owns contiguous
+// code words); the permutation is undone when the partials are written.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tqk {
+namespace {
+
+constexpr int MW = 4;           // warps per CTA
+constexpr int MT = 16;          // tokens per tile
+constexpr int NST = 4;          // pipeline stages per warp
+constexpr int D = 128;
+constexpr int KW = 8;           // key code words per token (2-bit fields)
+constexpr int QW = 4;           // QJL words per token (m = 128)
+constexpr int VW = 16;          // value code words per token (4-bit fields)
+constexpr int VROW = 20;        // padded value row (words): conflict-free LDS.64
+
+struct Stage {
+  uint32_t k[MT][KW];           // 512 B
+  uint32_t q[MT][QW];           // 256 B
+  float kn[MT];                 // 64 B
+  float kr[MT];                 // 64 B
+  float vn[MT];                 // 64 B
+  uint32_t pad_[4];             // keep v 16-byte aligned
+  uint32_t v[MT][VROW];         // 1280 B
+};
+static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
+
+constexpr int LUT_WORDS = 256 * 32;
+constexpr size_t SMEM_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST * sizeof(Stage);
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// QJL bit pair (e, e+16) of w as a half2 of +-1 (bit 1 -> +1).
+__device__ __forceinline__ uint32_t sign_pair(uint32_t w, int e) {
+  return ((w << (15 - e)) & 0x80008000u) ^ 0xBC00BC00u;
+}
+
+struct TileSrc {
+  const uint32_t* k;   // key codes of token 0 of the (b, g) row
+  const uint32_t* q;
+  const float* kn;
+  const float* kr;
+  const uint32_t* v;
+  const float* vn;
+};
+
+// Issue the cp.async copies of tile tokens [t0, t0+16) into stage st.
+__device__ __forceinline__ void load_tile(const TileSrc& src, Stage* st, int64_t t0, int64_t t_end,
+                                          int lane) {
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(st);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = lane + 32 * i;
+    if (c < 32) {                              // key codes: 16 tokens x 2 chunks
+      const int tok = c >> 1, part = c & 1;
+      const int64_t t = t0 + tok;
+      cp16(sbase + offsetof(Stage, k) + tok * 32 + part * 16, src.k + t * KW + part * 4, t < t_end);
+    } else if (c < 48) {                       // QJL: 16 tokens x 1 chunk
+      const int tok = c - 32;
+      const int64_t t = t0 + tok;
+      cp16(sbase + offsetof(Stage, q) + tok * 16, src.q + t * QW, t < t_end);
+    } else if (c < 60) {                       // norms: 3 arrays x 4 chunks of 4 tokens
+      const int which = (c - 48) >> 2, part = (c - 48) & 3;
+      const int64_t t = t0 + 4 * part;
+      const float* base = which == 0 ? src.kn : which == 1 ? src.kr : src.vn;
+      const uint32_t off = which == 0 ? offsetof(Stage, kn) : which == 1 ? offsetof(Stage, kr)
+                                                                           : offsetof(Stage, vn);
+      cp16(sbase + off + part * 16, base + t, t < t_end);
+    } else if (c < 124) {                      // value codes: 16 tokens x 4 chunks
+      const int cc = c - 60;
+      const int tok = cc >> 2, part = cc & 3;
+      const int64_t t = t0 + tok;
+      cp16(sbase + offsetof(Stage, v) + tok * (VROW * 4) + part * 16, src.v + t * VW + part * 4,
+           t < t_end);
+    }
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(MW * 32, 2) k_attn_mma(AttnArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+  Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  // Value table: entry (byte, lane) = half2(cv[byte & 15], cv[byte >> 4]).
+  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
+    const int byte = e >> 5;
+    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
+  }
+  // Key centroid tables (4 fp16 heads, 4 scaled fp16 tails) for the
+  // byte-permute dequantizer.
+  float ch[4], cl[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ch[i] = __half2float(__float2half_rn(a.ck[i]));
+    cl[i] = (a.ck[i] - ch[i]) * 4096.f;
+  }
+  const uint32_t T0 = pack_half2(ch[0], ch[1]), T1 = pack_half2(ch[2], ch[3]);
+  const uint32_t L0 = pack_half2(cl[0], cl[1]), L1 = pack_half2(cl[2], cl[3]);
+
+  // B fragments of the pre-rotated query q' and of s = S q' for head g.
+  const int hq = kvh * G + g;
+  const bool head_ok = g < G;
+  const float* qrow = a.qr + ((int64_t)b * a.Hq + (head_ok ? hq : kvh * G)) * 128;
+  const float* srow = a.qs + ((int64_t)b * a.Hq + (head_ok ? hq : kvh * G)) * 128;
+  float qv[32], sv[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 x = reinterpret_cast<const float4*>(qrow + 32 * t)[i];
+    const float4 y = reinterpret_cast<const float4*>(srow + 32 * t)[i];
+    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
+    sv[4 * i] = y.x; sv[4 * i + 1] = y.y; sv[4 * i + 2] = y.z; sv[4 * i + 3] = y.w;
+  }
+  float mq = 0.f, ms = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    mq = fmaxf(mq, fabsf(qv[i]));
+    ms = fmaxf(ms, fabsf(sv[i]));
+  }
+  mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
+  mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 2));
+  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 1));
+  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 2));
+  // Power-of-two scales keep the fp16 operands in range without extra rounding.
+  const int eq = mq > 0.f ? ilogbf(mq) : 0;
+  const int es = ms > 0.f ? ilogbf(ms) : 0;
+  const float sq_ = head_ok ? ldexpf(1.f, -eq) : 0.f;
+  const float ss_ = head_ok ? ldexpf(1.f, -es) : 0.f;
+  uint32_t bq[8][2], bql[8][2], bs[8][2], bsl[8][2];
+  auto split2 = [](float x, float y, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 f = __half22float2(h);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = pack_half2((x - f.x) * 4096.f, (y - f.y) * 4096.f);
+  };
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int base = 16 * (s >> 2) + (s & 3);   // local dims of k-step s
+    split2(qv[base] * sq_, qv[base + 4] * sq_, bq[s][0], bql[s][0]);
+    split2(qv[base + 8] * sq_, qv[base + 12] * sq_, bq[s][1], bql[s][1]);
+    split2(sv[2 * s] * ss_, sv[2 * s + 16] * ss_, bs[s][0], bsl[s][0]);
+    split2(sv[2 * s + 1] * ss_, sv[2 * s + 17] * ss_, bs[s][1], bsl[s][1]);
+  }
+  // Logit scales for the C-fragment columns (heads 2t, 2t+1).
+  float cqs[2], css[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int eqj = __shfl_sync(0xffffffffu, eq, (2 * t + j) * 4);
+    const int esj = __shfl_sync(0xffffffffu, es, (2 * t + j) * 4);
+    cqs[j] = ldexpf(a.scale_log2, eqj);
+    css[j] = ldexpf(a.scale_log2 * a.cq, esj);
+  }
+
+  const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
+  const int64_t c_begin = (int64_t)split * a.chunk;
+  const int64_t c_end = min(T, c_begin + a.chunk);
+  const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
+  TileSrc src{a.kcodes + row0 * KW, a.kqjl + row0 * QW, a.knorm + row0, a.krnorm + row0,
+              a.vcodes + row0 * VW, a.vnorm + row0};
+
+  Stage* my = stages + warp * NST;
+  // Tiles of this warp: c_begin + 16 * (warp + MW * i).
+  const int64_t ntiles_cta = c_end > c_begin ? (c_end - c_begin + MT - 1) / MT : 0;
+  const int nt = ntiles_cta > warp ? (int)((ntiles_cta - warp + MW - 1) / MW) : 0;
+
+#pragma unroll
+  for (int i = 0; i < NST - 1; ++i) {
+    if (i < nt) load_tile(src, my + i, c_begin + (int64_t)MT * (warp + MW * i), c_end, lane);
+    cp_commit();
+  }
+  __syncthreads();  // value table ready
+
+  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_part[2] = {0.f, 0.f};
+  int kv_run = -1000;
+  float o[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+  for (int i = 0; i < nt; ++i) {
+    {
+      const int ip = i + NST - 1;
+      if (ip < nt) load_tile(src, my + (ip % NST), c_begin + (int64_t)MT * (warp + MW * ip), c_end, lane);
+      cp_commit();
+    }
+    cp_wait<NST - 1>();
+    __syncwarp();
+    const Stage& st = my[i % NST];
+    const int64_t t0 = c_begin + (int64_t)MT * (warp + MW * i);
+
+    // ---- logits ----------------------------------------------------------
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc_t[4] = {0.f, 0.f, 0.f, 0.f}, acs_t[4] = {0.f, 0.f, 0.f, 0.f};  // tails
+    const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
+    const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int sh = 2 * (s & 3);
+      const uint32_t x0 = (s < 4) ? kg0.x : kg0.y;
+      const uint32_t x8 = (s < 4) ? kg8.x : kg8.y;
+      const uint32_t y0 = ((x0 >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
+      const uint32_t y8 = ((x8 >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
+      const uint32_t a0 = __byte_perm(T0, T1, y0);
+      const uint32_t a2 = __byte_perm(T0, T1, y0 >> 16);
+      const uint32_t a1 = __byte_perm(T0, T1, y8);
+      const uint32_t a3 = __byte_perm(T0, T1, y8 >> 16);
+      mma16816(acc, a0, a1, a2, a3, bq[s][0], bq[s][1]);
+      mma16816(acc_t, a0, a1, a2, a3, bql[s][0], bql[s][1]);
+      mma16816(acc_t, __byte_perm(L0, L1, y0), __byte_perm(L0, L1, y8), __byte_perm(L0, L1, y0 >> 16),
+               __byte_perm(L0, L1, y8 >> 16), bq[s][0], bq[s][1]);
+    }
+    const uint32_t qg0 = st.q[g][t], qg8 = st.q[g + 8][t];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t a0 = sign_pair(qg0, 2 * s), a1 = sign_pair(qg8, 2 * s);
+      const uint32_t a2 = sign_pair(qg0, 2 * s + 1), a3 = sign_pair(qg8, 2 * s + 1);
+      mma16816(acs, a0, a1, a2, a3, bs[s][0], bs[s][1]);
+      mma16816(acs_t, a0, a1, a2, a3, bsl[s][0], bsl[s][1]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      acc[r] = fmaf(acc_t[r], 1.f / 4096.f, acc[r]);
+      acs[r] = fmaf(acs_t[r], 1.f / 4096.f, acs[r]);
+    }
+    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
+    const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
+    float sc[4];
+    sc[0] = v0 ? fmaf(kr0 * css[0], acs[0], kn0 * cqs[0] * acc[0]) : -INFINITY;
+    sc[1] = v0 ? fmaf(kr0 * css[1], acs[1], kn0 * cqs[1] * acc[1]) : -INFINITY;
+    sc[2] = v8 ? fmaf(kr8 * css[0], acs[2], kn8 * cqs[0] * acc[2]) : -INFINITY;
+    sc[3] = v8 ? fmaf(kr8 * css[1], acs[3], kn8 * cqs[1] * acc[3]) : -INFINITY;
+
+    // ---- online softmax (heads 2t, 2t+1) ------------------------------------
+    float tmax[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 4));
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 8));
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 16));
+    }
+    // Value-norm scale: p * |v| * 2^-kv stays below 2^15 in fp16.
+    const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
+    float vmax = fmaxf(vn0, vn8);
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
+    const int kv_tile = vmax > 0.f ? ilogbf(vmax) - 14 : -1000;
+    const int kv_new = max(kv_run, kv_tile);
+    const float vscale_change = exp2f((float)(kv_run - kv_new));
+    kv_run = kv_new;
+    const float vmul = ldexpf(1.f, -kv_new);
+    float alpha[2], mnew[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      mnew[j] = fmaxf(m_run[j], tmax[j]);
+      alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(m_run[j] - mnew[j]);
+      m_run[j] = mnew[j];
+    }
+    float p[4];
+    p[0] = (mnew[0] == -INFINITY) ? 0.f : exp2f(sc[0] - mnew[0]);
+    p[1] = (mnew[1] == -INFINITY) ? 0.f : exp2f(sc[1] - mnew[1]);
+    p[2] = (mnew[0] == -INFINITY) ? 0.f : exp2f(sc[2] - mnew[0]);
+    p[3] = (mnew[1] == -INFINITY) ? 0.f : exp2f(sc[3] - mnew[1]);
+    l_part[0] = fmaf(l_part[0], alpha[0], p[0] + p[2]);
+    l_part[1] = fmaf(l_part[1], alpha[1], p[1] + p[3]);
+    const float oa0 = alpha[0] * vscale_change, oa1 = alpha[1] * vscale_change;
+    if (__any_sync(0xffffffffu, oa0 != 1.f || oa1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= oa0; o[mt][1] *= oa1; o[mt][2] *= oa0; o[mt][3] *= oa1;
+      }
+    }
+    const float w0 = vn0 * vmul, w8 = vn8 * vmul;
+    const uint32_t pb0 = movtrans(pack_half2(p[0] * w0, p[1] * w0));
+    const uint32_t pb1 = movtrans(pack_half2(p[2] * w8, p[3] * w8));
+
+    // ---- values ---------------------------------------------------------------
+    const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
+    const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
+    const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
+    const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
+    // byte k of ye = (nibble 2k of the first token) | (nibble 2k of the second) << 4
+    const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
+                            (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
+                            (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
+                            (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
+    const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
+                            ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
+                            ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
+                            ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int k = mt >> 1;
+      const uint32_t* y = (mt & 1) ? yo : ye;
+      uint32_t av[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t off = (k == 0) ? ((y[r] << 7) & 0x7F80u) : ((y[r] >> (8 * k - 7)) & 0x7F80u);
+        av[r] = lds32(lut_lane + off);
+      }
+      // rows: word 2g -> dim row g (a0/a2), word 2g+1 -> row g+8 (a1/a3)
+      mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+    }
+    __syncwarp();
+  }
+  cp_wait<0>();
+
+  // ---- merge the four warps of the CTA ---------------------------------------
+  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 4);
+  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 8);
+  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 16);
+  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 4);
+  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 8);
+  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 16);
+  __syncthreads();  // stages are reused as merge scratch below
+  float* sm = reinterpret_cast<float*>(stages);   // [MW][8][130]
+  const float vback = ldexpf(1.f, kv_run);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int h = 2 * t + j;
+    float* row = sm + (warp * 8 + h) * 130;
+    if (g == 0) {
+      row[0] = m_run[j];
+      row[1] = l_part[j];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      row[2 + 16 * g + mt] = o[mt][j] * vback;
+      row[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * 130; e += MW * 32) {
+    const int h = e / 130, c = e % 130;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) M = fmaxf(M, sm[(w * 8 + h) * 130]);
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) {
+      const float mw_ = sm[(w * 8 + h) * 130];
+      if (mw_ != -INFINITY) acc = fmaf(exp2f(mw_ - M), sm[(w * 8 + h) * 130 + (c == 0 ? 1 : c)], acc);
+    }
+    const int64_t prow = (int64_t)b * a.Hq + (int64_t)kvh * G + h;
+    float* pp = a.part + (prow * a.splits + split) * (128 + 2);
+    if (c == 0) {
+      pp[0] = M;
+    } else {
+      pp[c] = acc;   // c == 1: l, c >= 2: o_rot[c - 2]
+    }
+  }
+}
+
+}  // namespace
+
+bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
+  if (c->d != D || c->bk_lm != 2 || c->bits_v != 4 || c->qjl_m != 128) return false;
+  if (!(a.G == 1 || a.G == 2 || a.G == 4 || a.G == 8)) return false;
+  if (a.max_T % 4 != 0) return false;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.kqjl) |
+                       reinterpret_cast<uintptr_t>(a.knorm) | reinterpret_cast<uintptr_t>(a.krnorm) |
+                       reinterpret_cast<uintptr_t>(a.vcodes) | reinterpret_cast<uintptr_t>(a.vnorm);
+  return (al & 15) == 0;
+}
+
+int attn_mma_chunk() { return 512; }
+
+cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
+  dim3 grid(a.splits, a.Hkv, a.B);
+  cudaError_t e = cudaSuccess;
+  switch (a.G) {
+#define TQ_G(GG)                                                                               \
+  case GG:                                                                                     \
+    e = cudaFuncSetAttribute(k_attn_mma<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+                             (int)SMEM_BYTES);                                                 \
+    if (e != cudaSuccess) return e;                                                            \
+    k_attn_mma<GG><<<grid, MW * 32, SMEM_BYTES, s>>>(a);                                       \
+    break;
+    TQ_G(1)
+    TQ_G(2)
+    TQ_G(4)
+    TQ_G(8)
+#undef TQ_G
+    default:
+      return cudaErrorInvalidValue;
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attn_merge(c, a, out, s);
+}
+
+}  // namespace tqk

@@ -97,6 +97,11 @@ cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s)
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
                              float* qr, float* qs, cudaStream_t s);
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+// Tensor-core decode path (d = 128, k3 with m = 128, v4, group <= 8).
+bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
+int attn_mma_chunk();
+cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
                           const float* krnorm, int64_t nk, float* out, cudaStream_t s);

@@ -771,9 +771,7 @@ cudaError_t attn_J(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t 
   k_attn_split<J><<<grid, AT, shm, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, c->dpad * sizeof(float), s>>>(
-      a.part, a.splits, c->d, c->dpad, c->Pi_f, out);
-  return cudaGetLastError();
+  return launch_attn_merge(c, a, out, s);
 }
 
 }  // namespace
@@ -816,6 +814,12 @@ int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
   if (splits < 1) splits = 1;
   *chunk = (int)ch;
   return (int)splits;
+}
+
+cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
+  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, c->dpad * sizeof(float), s>>>(
+      a.part, a.splits, c->d, c->dpad, c->Pi_f, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {

@@ -158,18 +158,24 @@ def test_attention_single_head(cuda):
                       out.cpu().numpy())
 
 
-@pytest.mark.parametrize("d,Hq,Hkv,bk,bv,m", [(128, 8, 2, 3, 4, 128), (128, 16, 2, 4, 4, 128),
-                                             (200, 6, 3, 4, 3, 200), (64, 4, 4, 2, 2, 0)])
-def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m):
-    """Ragged lengths (0, 1, odd, full), GQA groups 1/2/4/8, d=64/128/200."""
+@pytest.mark.parametrize("d,Hq,Hkv,bk,bv,m,T", [
+    (128, 8, 2, 3, 4, 128, 1100),   # tensor-core path, group 4, 3 chunks
+    (128, 4, 4, 3, 4, 128, 1100),   # tensor-core path, group 1
+    (128, 4, 2, 3, 4, 128, 1100),   # tensor-core path, group 2
+    (128, 16, 2, 3, 4, 128, 1100),  # tensor-core path, group 8
+    (128, 8, 2, 3, 4, 128, 1002),   # max_T % 4 != 0: generic path
+    (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: generic path
+    (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000)])
+def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
+    """Ragged lengths (0, 1, odd, chunk edges, full), GQA groups 1-8, d=64/128/200."""
     c = _ctx(d, bk, bv, m, seed=7)
     tab = P.oracle_tables(c)
-    B, T = 5, 1000
+    B = 6
     K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=1)
     V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=2)
     Q = tq_inputs.iid((B, Hq, d), seed=3, dtype=torch.bfloat16)
     kc, vc = _cache(c, K, V, cuda)
-    lens = torch.tensor([0, 1, 129, 777, 1000], dtype=torch.int32)
+    lens = torch.tensor([0, 1, 129, 513, 777, T], dtype=torch.int32)
     out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
     torch.cuda.synchronize()
     P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
