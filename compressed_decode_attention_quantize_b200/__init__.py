@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "tq_logits": (I, [P, P, I, I64, P, P, P, P, I64, P, P]),
         "tq_attn_workspace_bytes": (SZ, [P, I, I, I64]),
         "tq_attn_decode": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P, SZ, P]),
+        "tq_attn_decode_static": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P]),
+        "tq_attn_static_scratch_bytes": (SZ, []),
         "tq_topk_workspace_bytes": (SZ, [P, I64, I64, I]),
         "tq_topk": (I, [P, P, I, I64, P, P, P, P, I64, I, P, P, P, SZ, P]),
     }
@@ -71,7 +73,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("tq_last_error", "tq_version", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
-            "tq_attn_workspace_bytes", "tq_attn_decode", "tq_topk_workspace_bytes", "tq_topk")
+            "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
+            "tq_attn_static_scratch_bytes", "tq_topk_workspace_bytes", "tq_topk")
 
 
 def library_path() -> str:
@@ -253,6 +256,24 @@ class Context:
                                    _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
                                    max_T, _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+        return out
+
+    def attn_decode_static(self, q: torch.Tensor, kcache: dict, vcache: dict,
+                           seq_lens: torch.Tensor, scale: float | None = None,
+                           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """attn_decode using the library's static device scratch instead of a
+        workspace (for callers that cannot allocate); calls must not overlap."""
+        q = q.contiguous()
+        B, Hq, d = q.shape
+        Hkv, max_T = kcache["norm"].shape[1], kcache["norm"].shape[2]
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        _check(_lib.tq_attn_decode_static(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
+                                          _ptr(kcache["codes"]), _ptr(kcache["qjl"]),
+                                          _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
+                                          _ptr(vcache["codes"]), _ptr(vcache["norm"]), max_T,
+                                          _ptr(seq_lens), float(scale), _ptr(out), _stream(stream)))
         return out
 
     def topk_workspace_bytes(self, nq: int, n: int, k: int) -> int:

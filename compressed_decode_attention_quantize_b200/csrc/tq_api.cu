@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -427,3 +428,64 @@ int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* cod
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without caller-provided scratch.
+//
+// Some callers cannot allocate device memory on the call path: a plugin whose
+// host framework owns every device allocation, or a serving loop that has
+// banned allocation after start-up to keep latency flat.  They also may not be
+// able to carry a workspace buffer through their interface.  For them the
+// scratch of tq_attn_decode lives in this file-scope device array; every GPU
+// that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)32 << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The array's
+// name in host code is only a stand-in for the symbol, so the address is
+// looked up (once per device, with that device current) and cached.
+int static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode_static: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode_static: device %d", dev);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode_static: cudaGetSymbolAddress");
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" size_t tq_attn_static_scratch_bytes(void) { return kStaticScratchBytes; }
+
+extern "C" int tq_attn_decode_static(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
+                                     const uint32_t* kcodes, const uint32_t* kqjl,
+                                     const float* knorm, const float* krnorm,
+                                     const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                                     const int32_t* seq_lens, float scale, float* out,
+                                     void* stream) {
+  if (int r = check_ctx(c)) return r;
+  const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
+  if (need > kStaticScratchBytes)
+    return fail(TQ_ERR_WORKSPACE,
+                "tq_attn_decode_static: these sizes need %zu bytes of scratch, above the %zu-byte "
+                "static limit; use tq_attn_decode with a workspace",
+                need, kStaticScratchBytes);
+  void* ws = nullptr;
+  if (int r = static_scratch(&ws)) return r;
+  return tq_attn_decode(c, q, dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm, vcodes, vnorm, max_T,
+                        seq_lens, scale, out, ws, kStaticScratchBytes, stream);
+}

@@ -221,6 +221,33 @@ int tq_attn_decode(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
                    const int32_t* seq_lens, float scale, float* out,
                    void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * tq_attn_decode_static - tq_attn_decode for callers that cannot allocate
+ * device memory on the call path (for example a plugin whose host framework
+ * owns every device allocation, or a serving loop that forbids allocation
+ * after start-up) and cannot pass a workspace.  The method's sources have no
+ * counterpart: this is an interface convenience.
+ * The scratch is a file-scope device array of tq_attn_static_scratch_bytes()
+ * bytes (32 MiB) that every GPU loading the library holds until exit; sizes
+ * whose tq_attn_workspace_bytes() exceed it are rejected with
+ * TQ_ERR_WORKSPACE.  The first call on a device looks up the array's device
+ * address (once per device, with that device current); make that first call
+ * before any stream capture.  The call allocates nothing.  All calls share
+ * the one array and it keeps the last call's contents (nothing in it needs to
+ * start at zero), so calls that overlap on the GPU - on different streams,
+ * or from different threads - race and must be serialised by the caller.
+ * Arguments and results are those of tq_attn_decode.
+ */
+int tq_attn_decode_static(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
+                          int Hkv, const uint32_t* kcodes, const uint32_t* kqjl,
+                          const float* knorm, const float* krnorm,
+                          const uint32_t* vcodes, const float* vnorm,
+                          int64_t max_T, const int32_t* seq_lens, float scale,
+                          float* out, void* stream);
+
+/* Size in bytes of the static scratch used by tq_attn_decode_static. */
+size_t tq_attn_static_scratch_bytes(void);
+
 /* Bytes of workspace tq_topk needs. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 
