@@ -47,6 +47,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_version": (ctypes.c_char_p, []),
+        "tq_device_fault": (I, [ctypes.POINTER(ctypes.c_int)]),
         "tq_init": (P, [I, I, I, I, U64]),
         "tq_destroy": (None, [P]),
         "tq_layout": (I, [P, I, ctypes.POINTER(tq_layout_t)]),
@@ -71,7 +72,7 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("tq_last_error", "tq_version", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
+EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
             "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
             "tq_attn_static_scratch_bytes", "tq_topk_workspace_bytes", "tq_topk")
@@ -108,6 +109,13 @@ def tq_init(d, bits_k, bits_v, qjl_m, seed):
 
 def tq_destroy(ctx):
     _lib.tq_destroy(ctx)
+
+
+def tq_device_fault() -> int:
+    """Read and clear the device fault code (0 = none); synchronises."""
+    v = ctypes.c_int(0)
+    _check(_lib.tq_device_fault(ctypes.byref(v)))
+    return v.value
 
 
 def tq_version() -> str:

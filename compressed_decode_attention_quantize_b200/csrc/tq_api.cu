@@ -1,5 +1,6 @@
 // C ABI of libtq: argument checks, context set-up and kernel launches.
 // The operations and their sources are documented in include/tq.h.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -69,6 +70,13 @@ extern "C" {
 const char* tq_last_error(void) { return g_err.c_str(); }
 
 const char* tq_version(void) { return "libtq 0.1 (sm_100a)"; }
+
+int tq_device_fault(int* code) {
+  if (!code) return fail(TQ_ERR_ARG, "tq_device_fault: null output");
+  cudaError_t e = tqk::read_and_clear_fault(code);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_device_fault");
+  return TQ_OK;
+}
 
 int tq_host_tables(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, double* pi,
                    double* S, double* ck, double* bk, double* cv, double* bv) {
@@ -163,6 +171,12 @@ tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
   for (size_t i = 0; i < c->cv.size(); ++i) hcv[i] = (float)c->cv[i];
   for (size_t i = 0; i < c->bv.size(); ++i) hbv[i] = (float)c->bv[i];
 
+  e = tqk::configure_kernels();
+  if (e != cudaSuccess) {
+    cuda_fail(e, "tq_init: kernel attributes");
+    delete c;
+    return nullptr;
+  }
   e = cudaMalloc(&c->dev_block, total);
   if (e != cudaSuccess) {
     cuda_fail(e, "tq_init: cudaMalloc");
@@ -175,6 +189,57 @@ tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
     cudaFree(c->dev_block);
     delete c;
     return nullptr;
+  }
+  // Operand images of the tensor-core quantizer (d = 128): 128 x 128 fp16,
+  // K-major, two 64-wide K blocks, 16-byte chunks swizzled with the row.
+  if (d == 128) {
+    e = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device);
+    if (e != cudaSuccess) c->sms = 148;
+    std::vector<uint16_t> img(3 * 128 * 128, 0);
+    std::vector<float> snorm(128, 0.f);
+    auto put = [&](int which, int r, int k, double v) {
+      const int kb = k >> 6, kk = k & 63, ch = kk >> 3, w = kk & 7;
+      const size_t off = (size_t)kb * 16384 + (size_t)(r >> 3) * 1024 + (size_t)(r & 7) * 128 +
+                         (size_t)((ch ^ (r & 7)) << 4) + (size_t)w * 2;
+      const __half h = __float2half_rn((float)v);
+      img[(size_t)which * 16384 + off / 2] = *reinterpret_cast<const uint16_t*>(&h);
+    };
+    for (int j = 0; j < 128; ++j)
+      for (int k = 0; k < 128; ++k) {
+        const double v = 256.0 * c->Pi[(size_t)j * d + k];
+        const double hi = tqh::round_to_half(v);
+        put(0, j, k, hi);
+        put(1, j, k, tqh::round_to_half(v - hi));
+      }
+    for (int i = 0; i < qjl_m; ++i) {
+      double nn = 0.0;
+      for (int k = 0; k < 128; ++k) {
+        put(2, i, k, c->S[(size_t)i * d + k]);
+        nn += c->S[(size_t)i * d + k] * c->S[(size_t)i * d + k];
+      }
+      snorm[i] = (float)std::sqrt(nn);
+    }
+    void* tc = nullptr;
+    e = cudaMalloc(&tc, img.size() * 2 + snorm.size() * 4);
+    if (e == cudaSuccess) {
+      e = cudaMemcpy(tc, img.data(), img.size() * 2, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(static_cast<char*>(tc) + img.size() * 2, snorm.data(), snorm.size() * 4,
+                       cudaMemcpyHostToDevice);
+    }
+    if (e != cudaSuccess) {
+      cuda_fail(e, "tq_init: tensor-core tables");
+      if (tc) cudaFree(tc);
+      cudaFree(c->dev_block);
+      delete c;
+      return nullptr;
+    }
+    c->tc_block = tc;
+    c->tc_pih = tc;
+    c->tc_pil = static_cast<char*>(tc) + 32768;
+    c->tc_s = static_cast<char*>(tc) + 65536;
+    c->tc_snorm = reinterpret_cast<const float*>(static_cast<char*>(tc) + 98304);
+    c->tc_ok = true;
   }
   const float* base = static_cast<const float*>(c->dev_block);
   c->PiT = base;
@@ -195,6 +260,7 @@ void tq_destroy(tq_ctx* c) {
     cudaGetDevice(&cur);
     if (cur != c->device) cudaSetDevice(c->device);
     cudaFree(c->dev_block);
+    if (c->tc_block) cudaFree(c->tc_block);
     if (cur != c->device) cudaSetDevice(cur);
   }
   delete c;
@@ -265,6 +331,38 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.pos = pos;
   a.H = H;
   a.max_T = max_T;
+  const bool tc = c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+                  aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
+  if (tc) {
+    tqk::QuantTcArgs t{};
+    t.x = x;
+    t.dtype = dtype;
+    t.n = n;
+    t.ld = ld;
+    t.bits = a.bits;
+    t.m = m;
+    t.pi_hi = c->tc_pih;
+    t.pi_lo = c->tc_pil;
+    t.s_img = c->tc_s;
+    t.snorm = c->tc_snorm;
+    t.s_f32 = c->S_f;
+    t.codes = codes;
+    t.qjl = qjl;
+    t.norm = norm;
+    t.rnorm = rnorm;
+    t.pos = pos;
+    t.H = H;
+    t.max_T = max_T;
+    const std::vector<double>& cen = key ? c->ck : c->cv;
+    const std::vector<double>& bnd = key ? c->bk : c->bv;
+    for (int i = 0; i < 16; ++i) {
+      t.cen[i] = i < (int)cen.size() ? (float)cen[i] : 0.f;
+      t.bnd[i] = i < (int)bnd.size() ? (float)bnd[i] : INFINITY;
+    }
+    cudaError_t e = tqk::launch_quant_tc(t, c->sms, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return TQ_OK;
+  }
   cudaError_t e = tqk::launch_quantize(c, a, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;

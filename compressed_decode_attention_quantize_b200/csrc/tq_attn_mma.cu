@@ -428,6 +428,374 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_mma(AttnArgs a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Group size <= 4.  Half of the MMA's eight columns would be idle, so columns
+// 4..7 carry the fp16 tails (x 2^12) of the query-side operands of columns
+// 0..3: one MMA yields head and tail products of every k-step.
+//
+// Keys use exact binary A operands.  A symmetric 2-bit codebook is affine in
+// the index bits, c[i0 + 2 i1] = c0 + (c1 - c0) i0 + (c2 - c0) i1, so
+//   <q', c[idx]> = c0 sum_j q'_j + (c1 - c0) <q', i0> + (c2 - c0) <q', i1>,
+// and the QJL term is <s, sigma> = 2 <s, bit> - sum_i s_i.  A bit becomes an
+// fp16 operand by masking it into the exponent field: a lone bit at position
+// p in 10..14 of a half reads as 2^E(p), E = -14, -13, -11, -7, 1, and the
+// B operand carries the inverse power of two.  Four rotations of a 32-bit
+// code word and sixteen masks give sixteen half2 registers: register u holds
+// bit 10+u in its low half and bit (26+u) mod 32 in its high half.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int bit_pos(int u) {
+  return u < 5 ? 10 + u : (u < 10 ? 5 + u : (u < 15 ? u : 10));
+}
+__host__ __device__ constexpr int bit_rot(int u) { return u < 5 ? 0 : (u < 10 ? 5 : (u < 15 ? 10 : 15)); }
+__device__ __forceinline__ float bit_inv(int p) {
+  return p == 10 ? 16384.f : (p == 11 ? 8192.f : (p == 12 ? 2048.f : (p == 13 ? 128.f : 0.5f)));
+}
+
+struct Rot4 {
+  uint32_t r[4];
+};
+__device__ __forceinline__ Rot4 rotations(uint32_t w) {
+  return Rot4{{w, __funnelshift_r(w, w, 5), __funnelshift_r(w, w, 10), __funnelshift_r(w, w, 15)}};
+}
+template <int U>
+__device__ __forceinline__ uint32_t bit_half2(const Rot4& R) {
+  constexpr int p = bit_pos(U);
+  return R.r[bit_rot(U) / 5] & ((1u << p) | (1u << (p + 16)));
+}
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^e for an integer e in the normal fp32 range.
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+// floor(log2(x)) for a positive normal float.
+__device__ __forceinline__ int ilog2f(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
+
+template <int G>
+__global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
+  static_assert(G <= 4, "packed path");
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+  Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
+    const int byte = e >> 5;
+    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
+  }
+
+  // ---- query-side operands: column g carries head (g & 3); g >= 4 the tails
+  const int hh = g & 3;
+  const bool tail_col = g >= 4;
+  const bool head_ok = hh < G;
+  const int64_t qrow_i = (int64_t)b * a.Hq + (int64_t)kvh * G + (head_ok ? hh : 0);
+  const float* qrow = a.qr + qrow_i * 128 + 32 * t;
+  const float* srow = a.qs + qrow_i * 128 + 32 * t;
+  float qv[32], sv[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 x = reinterpret_cast<const float4*>(qrow)[i];
+    const float4 y = reinterpret_cast<const float4*>(srow)[i];
+    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
+    sv[4 * i] = y.x; sv[4 * i + 1] = y.y; sv[4 * i + 2] = y.z; sv[4 * i + 3] = y.w;
+  }
+  float mq = 0.f, ms = 0.f, sumq = 0.f, sums = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    mq = fmaxf(mq, fabsf(qv[i]));
+    ms = fmaxf(ms, fabsf(sv[i]));
+    sumq += qv[i];
+    sums += sv[i];
+  }
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+    ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+    sumq += __shfl_xor_sync(0xffffffffu, sumq, o);
+    sums += __shfl_xor_sync(0xffffffffu, sums, o);
+  }
+  const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
+  const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
+  const int eq = mq > 0.f ? ilog2f(mq) : 0;
+  const int es = ms > 0.f ? ilog2f(ms) : 0;
+  // q' * w * 2^-(eq+ew+1) < 2, times at most 2^14: fits fp16.
+  const float kq = head_ok ? pow2i(-(eq + ew + 1)) : 0.f;
+  const float ks = head_ok ? pow2i(-es) : 0.f;
+  const float wq0 = w0 * kq, wq1 = w1 * kq;
+  auto operand = [&](float lo, float hi) -> uint32_t {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    if (!tail_col) return *reinterpret_cast<const uint32_t*>(&h);
+    const float2 f = __half22float2(h);
+    return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
+  };
+  // Keys: k-step s (0..15) reads word s>>3 of the thread's two code words;
+  // slot 0/1 use registers u = 2(s&7) and 2(s&7)+1.
+  uint32_t bk[16][2];
+#pragma unroll
+  for (int s = 0; s < 16; ++s) {
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) {
+      const int u = 2 * (s & 7) + slot;
+      const int elo = 10 + u, ehi = (26 + u) & 31;
+      const float inv = bit_inv(bit_pos(u));
+      const int dlo = 16 * (s >> 3) + (elo >> 1), dhi = 16 * (s >> 3) + (ehi >> 1);
+      const float vlo = qv[dlo] * ((elo & 1) ? wq1 : wq0) * inv;
+      const float vhi = qv[dhi] * ((ehi & 1) ? wq1 : wq0) * inv;
+      bk[s][slot] = operand(vlo, vhi);
+    }
+  }
+  // QJL: k-step s (0..7), slot 0/1 use registers 2s, 2s+1 of the thread's word.
+  uint32_t bj[8][2];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) {
+      const int u = 2 * s + slot;
+      const int elo = 10 + u, ehi = (26 + u) & 31;
+      const float inv = bit_inv(bit_pos(u)) * ks;
+      bj[s][slot] = operand(sv[elo] * inv, sv[ehi] * inv);
+    }
+  }
+  // Logit constants for heads 2t, 2t+1 (threads t < 2):
+  //   s2 = kn * (acc * KA + KB) + kr * (acs * QA + QB)
+  float KA[2], KB[2], QA[2], QB[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int src = ((2 * t + j) & 3) * 4;
+    const int eqj = __shfl_sync(0xffffffffu, eq, src);
+    const int esj = __shfl_sync(0xffffffffu, es, src);
+    const float sqj = __shfl_sync(0xffffffffu, sumq, src);
+    const float ssj = __shfl_sync(0xffffffffu, sums, src);
+    KA[j] = pow2i(eqj + ew + 1) * a.scale_log2;
+    KB[j] = c0 * sqj * a.scale_log2;
+    QA[j] = 2.f * pow2i(esj) * a.cq * a.scale_log2;
+    QB[j] = -ssj * a.cq * a.scale_log2;
+  }
+
+  const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
+  const int c_begin = split * a.chunk;
+  const int c_end = (int)min(T, (int64_t)c_begin + a.chunk);
+  const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
+
+  // Per-lane cp.async assignment (fixed for all tiles): slot 0 = key codes,
+  // slots 1-2 = value codes, slot 3 = QJL words or norms.
+  Stage* my = stages + warp * NST;
+  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
+  const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;   // tok lane>>1
+  const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;   // tok lane>>2
+  const char* p2 = p1 + 8 * 64;                                                         // tok 8+lane>>2
+  const char* p3;
+  int stride3, tok3;
+  uint32_t d3;
+  if (lane < 16) {
+    p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
+    stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
+  } else if (lane < 28) {
+    const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
+    const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
+    p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
+    stride3 = 4; tok3 = 4 * part;
+    d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
+  } else {
+    p3 = nullptr; stride3 = 0; tok3 = 1 << 30; d3 = 0;
+  }
+  const uint32_t d0 = offsetof(Stage, k) + lane * 16;
+  const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
+  const uint32_t d2 = d1 + 8 * (VROW * 4);
+  auto issue = [&](int tile, int stage) {
+    const int t0 = c_begin + MT * (warp + MW * tile);
+    const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
+    cp16(sb + d0, p0 + (int64_t)t0 * 32, t0 + (lane >> 1) < c_end);
+    cp16(sb + d1, p1 + (int64_t)t0 * 64, t0 + (lane >> 2) < c_end);
+    cp16(sb + d2, p2 + (int64_t)t0 * 64, t0 + 8 + (lane >> 2) < c_end);
+    if (lane < 28) cp16(sb + d3, p3 + (int64_t)t0 * stride3, t0 + tok3 < c_end);
+  };
+
+  const int ntiles_cta = c_end > c_begin ? (c_end - c_begin + MT - 1) / MT : 0;
+  const int nt = ntiles_cta > warp ? (ntiles_cta - warp + MW - 1) / MW : 0;
+#pragma unroll
+  for (int i = 0; i < NST - 1; ++i) {
+    if (i < nt) issue(i, i);
+    cp_commit();
+  }
+  __syncthreads();
+
+  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_part[2] = {0.f, 0.f};
+  int kv_run = -126;
+  float o[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  const bool own_heads = t < 2;
+
+  for (int i = 0; i < nt; ++i) {
+    if (i + NST - 1 < nt) issue(i + NST - 1, (i + NST - 1) % NST);
+    cp_commit();
+    cp_wait<NST - 1>();
+    __syncwarp();
+    const Stage& st = my[i % NST];
+    const int t0 = c_begin + MT * (warp + MW * i);
+
+    // ---- logits -------------------------------------------------------------
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
+      const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
+      const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
+      const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
+#define TQ_KSTEP(S)                                                                               \
+  mma16816(acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                                    \
+           bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81),                                         \
+           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01),                                     \
+           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S][0], bk[S][1]);
+      TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6)
+      TQ_KSTEP(7) TQ_KSTEP(8) TQ_KSTEP(9) TQ_KSTEP(10) TQ_KSTEP(11) TQ_KSTEP(12) TQ_KSTEP(13)
+      TQ_KSTEP(14) TQ_KSTEP(15)
+#undef TQ_KSTEP
+      const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
+#define TQ_QSTEP(S)                                                                               \
+  mma16816(acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8), bit_half2<2 * (S) + 1>(Q0),      \
+           bit_half2<2 * (S) + 1>(Q8), bj[S][0], bj[S][1]);
+      TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
+      TQ_QSTEP(7)
+#undef TQ_QSTEP
+    }
+    // Tails sit in columns 2t+4, 2t+5 (lane ^ 2).
+    float sc[4];
+    {
+      const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
+      const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float lm = fmaf(__shfl_xor_sync(0xffffffffu, acc[r], 2), 1.f / 4096.f, acc[r]);
+        const float qj = fmaf(__shfl_xor_sync(0xffffffffu, acs[r], 2), 1.f / 4096.f, acs[r]);
+        const int j = r & 1;
+        const float kn = r < 2 ? kn0 : kn8, kr = r < 2 ? kr0 : kr8;
+        const bool ok = own_heads && (r < 2 ? v0 : v8);
+        sc[r] = ok ? fmaf(kn, fmaf(lm, KA[j], KB[j]), kr * fmaf(qj, QA[j], QB[j])) : -INFINITY;
+      }
+    }
+
+    // ---- online softmax (heads 2t, 2t+1 for t < 2) ------------------------------
+    float tmax[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 4));
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 8));
+      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 16));
+    }
+    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
+    const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
+    float vmax = fmaxf(vn0, vn8);
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
+    // p * |v| * 2^-kv stays below 2^15 in fp16.
+    const int kv_tile = vmax > 1e-30f ? ilog2f(vmax) - 14 : -126;
+    const int kv_new = max(kv_run, kv_tile);
+    const float vchange = pow2i(max(kv_run - kv_new, -126));
+    kv_run = kv_new;
+    const float vmul = pow2i(-kv_new);
+    float alpha[2], mnew[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      mnew[j] = fmaxf(m_run[j], tmax[j]);
+      alpha[j] = (mnew[j] == -INFINITY) ? 1.f : ex2f(m_run[j] - mnew[j]);
+      m_run[j] = mnew[j];
+    }
+    float p[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) p[r] = (sc[r] == -INFINITY) ? 0.f : ex2f(sc[r] - mnew[r & 1]);
+    l_part[0] = fmaf(l_part[0], alpha[0], p[0] + p[2]);
+    l_part[1] = fmaf(l_part[1], alpha[1], p[1] + p[3]);
+    const float oa0 = alpha[0] * vchange, oa1 = alpha[1] * vchange;
+    if (__any_sync(0xffffffffu, oa0 != 1.f || oa1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= oa0; o[mt][1] *= oa1; o[mt][2] *= oa0; o[mt][3] *= oa1;
+      }
+    }
+    const float w0v = vn0 * vmul, w8v = vn8 * vmul;
+    const uint32_t pb0 = movtrans(pack_half2(p[0] * w0v, p[1] * w0v));
+    const uint32_t pb1 = movtrans(pack_half2(p[2] * w8v, p[3] * w8v));
+
+    // ---- values ---------------------------------------------------------------
+    const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
+    const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
+    const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
+    const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
+    const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
+                            (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
+                            (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
+                            (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
+    const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
+                            ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
+                            ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
+                            ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int k = mt >> 1;
+      const uint32_t* y = (mt & 1) ? yo : ye;
+      uint32_t av[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
+      mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+    }
+    __syncwarp();
+  }
+  cp_wait<0>();
+
+  // ---- merge the four warps of the CTA -------------------------------------------
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 4);
+    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 8);
+    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 16);
+  }
+  __syncthreads();
+  float* sm = reinterpret_cast<float*>(stages);   // [MW][4][130]
+  const float vback = pow2i(kv_run);
+  if (own_heads) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int h = 2 * t + j;
+      float* row = sm + (warp * 4 + h) * 130;
+      if (g == 0) {
+        row[0] = m_run[j];
+        row[1] = l_part[j];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        row[2 + 16 * g + mt] = o[mt][j] * vback;
+        row[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * 130; e += MW * 32) {
+    const int h = e / 130, c = e % 130;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) M = fmaxf(M, sm[(w * 4 + h) * 130]);
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) {
+      const float mw_ = sm[(w * 4 + h) * 130];
+      if (mw_ != -INFINITY) acc = fmaf(exp2f(mw_ - M), sm[(w * 4 + h) * 130 + (c == 0 ? 1 : c)], acc);
+    }
+    const int64_t prow = (int64_t)b * a.Hq + (int64_t)kvh * G + h;
+    float* pp = a.part + (prow * a.splits + split) * (128 + 2);
+    pp[c] = (c == 0) ? M : acc;
+  }
+}
+
 }  // namespace
 
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
@@ -446,16 +814,18 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cuda
   dim3 grid(a.splits, a.Hkv, a.B);
   cudaError_t e = cudaSuccess;
   switch (a.G) {
+#define TQ_G4(GG)                                                                              \
+  case GG:                                                                                     \
+    k_attn_g4<GG><<<grid, MW * 32, SMEM_BYTES, s>>>(a);                                        \
+    break;
+    TQ_G4(1)
+    TQ_G4(2)
+    TQ_G4(4)
+#undef TQ_G4
 #define TQ_G(GG)                                                                               \
   case GG:                                                                                     \
-    e = cudaFuncSetAttribute(k_attn_mma<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
-                             (int)SMEM_BYTES);                                                 \
-    if (e != cudaSuccess) return e;                                                            \
     k_attn_mma<GG><<<grid, MW * 32, SMEM_BYTES, s>>>(a);                                       \
     break;
-    TQ_G(1)
-    TQ_G(2)
-    TQ_G(4)
     TQ_G(8)
 #undef TQ_G
     default:
@@ -464,6 +834,15 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cuda
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_merge(c, a, out, s);
+}
+
+cudaError_t configure_attn_mma() {
+  const int b = (int)SMEM_BYTES;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(k_attn_g4<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_g4<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_g4<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  return cudaFuncSetAttribute(k_attn_mma<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
 }
 
 }  // namespace tqk

@@ -34,6 +34,14 @@ struct tq_ctx {
   const float* bk_f = nullptr;  // [16] key boundaries (padded with +inf)
   const float* cv_f = nullptr;  // [16]
   const float* bv_f = nullptr;  // [16]
+  // Tensor-core quantize (d = 128): swizzled fp16 operand images and QJL row norms.
+  bool tc_ok = false;
+  void* tc_block = nullptr;
+  int sms = 148;
+  const void* tc_pih = nullptr;   // 2^8 Pi, fp16 head
+  const void* tc_pil = nullptr;   // 2^8 Pi - head, fp16
+  const void* tc_s = nullptr;     // S, fp16 (exact)
+  const float* tc_snorm = nullptr;  // |S_i|
 };
 
 namespace tqh {
@@ -93,7 +101,32 @@ struct AttnArgs {
   float* part;       // [B*Hq][splits][dpad+2]
 };
 
+struct QuantTcArgs {
+  const void* x;
+  int dtype;
+  int64_t n, ld;
+  int bits, m;
+  const void* pi_hi;
+  const void* pi_lo;
+  const void* s_img;
+  const float* snorm;
+  const float* s_f32;
+  uint32_t* codes;
+  uint32_t* qjl;
+  float* norm;
+  float* rnorm;
+  const int32_t* pos;
+  int H;
+  int64_t max_T;
+  float cen[16];
+  float bnd[16];
+};
+
 cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
+// Tensor-core quantize for d = 128 (16-bit inputs).
+cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s);
+cudaError_t configure_quant_tc();
+cudaError_t read_and_clear_fault(int* value);
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
                              float* qr, float* qs, cudaStream_t s);
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
@@ -114,5 +147,8 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                         const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
                         void* ws, cudaStream_t s);
 int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk);
+// Shared-memory limits of all kernels on the current device (tq_init).
+cudaError_t configure_kernels();
+cudaError_t configure_attn_mma();
 
 }  // namespace tqk

@@ -748,10 +748,6 @@ __global__ void __launch_bounds__(32) k_topk_final(const float* cand_v, const in
 template <int J>
 cudaError_t quantize_J(const QuantArgs& a, cudaStream_t s) {
   const size_t shm = (size_t)QWARPS * J * 32 * QV * sizeof(float);
-  if (shm > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_quantize<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
-    if (e != cudaSuccess) return e;
-  }
   const int64_t groups = (a.n + QV - 1) / QV;
   int64_t blocks = (groups + QWARPS - 1) / QWARPS;
   blocks = blocks < 148 * 16 ? blocks : 148 * 16;
@@ -763,10 +759,6 @@ template <int J>
 cudaError_t attn_J(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
   const size_t shm = (size_t)(2 * a.G * J * 32 + AT * a.G) * sizeof(float) +
                      (size_t)AT * a.wv * sizeof(uint32_t);
-  if (shm > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
-    if (e != cudaSuccess) return e;
-  }
   dim3 grid(a.splits, a.Hkv, a.B);
   k_attn_split<J><<<grid, AT, shm, s>>>(a);
   cudaError_t e = cudaGetLastError();
@@ -887,8 +879,6 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                      (size_t)TQ * TKMAX * sizeof(int);
   dim3 grid((unsigned)nch, (unsigned)((nq + TQ - 1) / TQ));
   TQ_DISPATCH_J(c->J, {
-    e = cudaFuncSetAttribute(k_topk_chunk<JV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
-    if (e != cudaSuccess) return e;
     k_topk_chunk<JV><<<grid, TTH, shm, s>>>(qr, qs, nq, c->d, c->bk_lm, c->wk, c->qjl_m, c->ck_f, cq,
                                              codes, qjl, norm, rnorm, n, k, cv, ci, (int)nch);
     break;
@@ -897,6 +887,34 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   if (e != cudaSuccess) return e;
   k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, (int)nch, k, idx, score);
   return cudaGetLastError();
+}
+
+// Raise the dynamic shared-memory limit of every kernel that needs more
+// than the default 48 KB, on the current device (called by tq_init).
+template <int J>
+static cudaError_t configure_J() {
+  cudaError_t e = cudaFuncSetAttribute(k_quantize<J>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(QWARPS * J * 32 * QV * sizeof(float)));
+  if (e != cudaSuccess) return e;
+  const int attn_max = (2 * GMAX * J * 32 + AT * GMAX) * (int)sizeof(float) + AT * 32 * (int)sizeof(uint32_t);
+  e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_max);
+  if (e != cudaSuccess) return e;
+  const int topk = (2 * J * 32 * TQ + TQ * TTH + TQ * TKMAX) * (int)sizeof(float) + TQ * TKMAX * (int)sizeof(int);
+  return cudaFuncSetAttribute(k_topk_chunk<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, topk);
+}
+
+cudaError_t configure_kernels() {
+  cudaError_t e;
+  if ((e = configure_J<1>()) != cudaSuccess) return e;
+  if ((e = configure_J<2>()) != cudaSuccess) return e;
+  if ((e = configure_J<3>()) != cudaSuccess) return e;
+  if ((e = configure_J<4>()) != cudaSuccess) return e;
+  if ((e = configure_J<5>()) != cudaSuccess) return e;
+  if ((e = configure_J<6>()) != cudaSuccess) return e;
+  if ((e = configure_J<7>()) != cudaSuccess) return e;
+  if ((e = configure_J<8>()) != cudaSuccess) return e;
+  if ((e = configure_quant_tc()) != cudaSuccess) return e;
+  return configure_attn_mma();
 }
 
 }  // namespace tqk

@@ -1,0 +1,473 @@
+// Online quantization on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// "What is TurboQuant?", section "How TurboQuant works": stage 1 rotates the
+// normalised vector with the random orthogonal Pi and maps every coordinate
+// to its Lloyd-Max index; stage 2 keeps sign(S r) of the residual r.  Here
+// both products are GEMMs over a tile of 128 vectors:
+//   D_rot[v][j] = sum_k x[v][k] Pi'[j][k]      (M = 128 vectors, N = K = 128)
+//   D_qjl[v][i] = sum_k r[v][k] S[i][k]
+// issued by one thread per warpgroup with operands in shared memory (128-byte
+// swizzled, K-major) and fp32 accumulators in tensor memory.  Thread v of the
+// warpgroup owns TMEM lane v, i.e. one whole vector, so index computation and
+// bit packing need no cross-thread exchange.
+//
+// Exactness.  x (bf16 or fp16) is exact in fp16 after a per-vector power of
+// two scale.  Pi' = 2^8 Pi is split into an fp16 head and tail; both products
+// accumulate into the same TMEM columns, so y carries ~2^-22 relative error,
+// far inside the 1e-5 decision band.  r (scaled by 2^14) is likewise fed as an
+// fp16 head and tail tile against the exact fp16 S.  A QJL sign is recomputed
+// in fp32 whenever |(S r)_i| is within 2^-17 |S_i| |r| of zero, a bound on the
+// operand and accumulation rounding of the tensor-core product (a few bits
+// per thousand vectors).
+//
+// Two warpgroups per CTA work on different tiles, so one group's MMAs overlap
+// the other's epilogue.  Waits on MMA completion are bounded; on timeout the
+// kernel records a fault code, releases its tensor memory and returns.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace tqk {
+
+__device__ int g_tq_fault = 0;
+
+namespace {
+
+constexpr int TILE = 128;
+constexpr uint32_t SMEM_TILE = 32768;            // one 128 x 128 fp16 operand
+constexpr uint32_t OFF_PIH = 0, OFF_PIL = SMEM_TILE, OFF_S = 2 * SMEM_TILE;
+constexpr uint32_t OFF_A = 3 * SMEM_TILE;        // + wg * 2 * SMEM_TILE: head, tail
+constexpr uint32_t OFF_MISC = 7 * SMEM_TILE;
+constexpr uint32_t TC_SMEM = OFF_MISC + 1024 + 1024;  // misc + alignment slack
+// Instruction descriptor: D f32, A/B f16, both K-major, N = 128, M = 128.
+constexpr uint32_t IDESC = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr int WAIT_LIMIT = 1 << 22;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  // start address >> 4, leading byte offset 1 (unused for swizzled K-major),
+  // stride byte offset 1024 B between 8-row groups, version 1, 128-byte swizzle.
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(IDESC), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (int it = 0; it < WAIT_LIMIT; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// True on every thread of the warpgroup if any of its threads passes true.
+__device__ __forceinline__ bool wg_any(int wg, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(1 + wg)
+      : "memory");
+  return r != 0u;
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void wg_sync(int wg) {
+  asm volatile("bar.sync %0, 128;\n" ::"r"(1 + wg) : "memory");
+}
+
+// 32 fp32 columns [col, col+32) of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Byte offset of the 16-byte chunk c (8 fp16 values k = 8c..8c+7) of row r in
+// a 128 x 128 K-major operand with 128-byte swizzle (two 64-wide K blocks).
+__device__ __forceinline__ uint32_t chunk_off(int r, int c) {
+  return (uint32_t)((c >> 3) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t h2bits(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+__device__ __forceinline__ int flog2(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
+
+__device__ __forceinline__ int64_t out_rec(const QuantTcArgs& a, int64_t v) {
+  if (a.pos == nullptr) return v;
+  return v * a.max_T + a.pos[v / a.H];
+}
+
+// Lloyd-Max index of y for 2^BITS symmetric levels: binary search over the
+// positive boundaries (pb, L/2 - 1 of them, ascending) on |y|, then mirrored.
+// The first level compares with a register (pmid = pb[L/4 - 1]); deeper
+// levels read the thresholds from shared memory (distinct banks).
+template <int BITS>
+__device__ __forceinline__ int lm_idx(float y, float pmid, const float* pb) {
+  constexpr int H = 1 << (BITS - 1);
+  const float a = fabsf(y);
+  int j = 0;
+  if (BITS >= 2) j = (a >= pmid) ? (H >> 1) : 0;
+  if (BITS >= 4) j += (a >= pb[j + 1]) ? 2 : 0;
+  if (BITS >= 3) j += (a >= pb[j]) ? 1 : 0;
+  return (y >= 0.f) ? H + j : H - 1 - j;
+}
+
+template <int BITS, bool QJL>
+__global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  unsigned char* base = smem_raw + (base_s - raw_s);
+  float* s_snorm = reinterpret_cast<float*>(base + OFF_MISC + 64);   // [128]
+  float* s_cen = s_snorm + 128;                                        // [16]
+  float* s_pb = s_cen + 16;                                            // [8]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC + 32);
+  const uint32_t bar0 = base_s + OFF_MISC;   // 4 barriers: rot wg0, rot wg1, qjl wg0, qjl wg1
+
+  const int tid = threadIdx.x, wg = tid >> 7, row = tid & 127, warp = tid >> 5;
+  constexpr int L = 1 << BITS;
+  constexpr int PER = (BITS == 3) ? 16 : 32 / BITS;   // fields per word of the main stream
+  constexpr int W_MAIN = 128 / PER;                     // words of the main stream
+  constexpr int WORDS = (BITS == 3) ? W_MAIN + 4 : W_MAIN;
+
+  // ---- shared tables: operand images, QJL row norms, codebook --------------------
+  {
+    const int4* src_pih = reinterpret_cast<const int4*>(a.pi_hi);
+    const int4* src_pil = reinterpret_cast<const int4*>(a.pi_lo);
+    const int4* src_s = reinterpret_cast<const int4*>(a.s_img);
+    int4* dst = reinterpret_cast<int4*>(base);
+    for (int e = tid; e < (int)(SMEM_TILE / 16); e += 256) {
+      dst[OFF_PIH / 16 + e] = src_pih[e];
+      dst[OFF_PIL / 16 + e] = src_pil[e];
+      if (QJL) dst[OFF_S / 16 + e] = src_s[e];
+    }
+    if (tid < 128) s_snorm[tid] = QJL ? a.snorm[tid] : 0.f;
+    if (tid < 16) s_cen[tid] = tid < L ? a.cen[tid] : 0.f;
+    if (tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar0 + 8 * i) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(
+                     base_s + OFF_MISC + 32)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  fence_async_smem();
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  const uint32_t d_rot = tmem + (uint32_t)(wg * 256);
+  const uint32_t d_qjl = d_rot + 128;
+  const uint32_t sA = base_s + OFF_A + wg * 2 * SMEM_TILE;
+  unsigned char* A = base + OFF_A + wg * 2 * SMEM_TILE;
+  unsigned char* A2 = A + SMEM_TILE;
+  const uint32_t bar_rot = bar0 + 8 * wg, bar_q = bar0 + 16 + 8 * wg;
+  const bool leader = row == 0;
+  const float* pb = s_pb;
+  const float pmid = BITS >= 2 ? s_pb[(L >> 2) - 1] : 0.f;
+
+  const int64_t ntiles = (a.n + TILE - 1) / TILE;
+  uint32_t iter = 0;
+  bool fault = false;
+  for (int64_t tile = (int64_t)blockIdx.x * 2 + wg; tile < ntiles; tile += (int64_t)gridDim.x * 2, ++iter) {
+    const int64_t v = tile * TILE + row;
+    const bool live = v < a.n;
+    // ---- load x, norm, scaled fp16 operand ----------------------------------------
+    uint4 xr[16];
+    if (live) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.x) + v * a.ld);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) xr[c] = src[c];
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) xr[c] = make_uint4(0, 0, 0, 0);
+    }
+    const bool is_bf = a.dtype == TQ_BF16;
+    auto lo_f = [&](uint32_t w) {
+      return is_bf ? __uint_as_float(w << 16) : __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
+    };
+    auto hi_f = [&](uint32_t w) {
+      return is_bf ? __uint_as_float(w & 0xFFFF0000u) : __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    };
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint32_t w4[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float f0 = lo_f(w4[q]), f1 = hi_f(w4[q]);
+        ss = fmaf(f0, f0, ss);
+        ss = fmaf(f1, f1, ss);
+      }
+    }
+    const float nrm = sqrtf(ss);
+    const int e = nrm > 0.f ? 14 - flog2(nrm) : 0;
+    const float sc = pow2f(e);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const uint32_t w4[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
+      uint4 o;
+      o.x = h2bits(lo_f(w4[0]) * sc, hi_f(w4[0]) * sc);
+      o.y = h2bits(lo_f(w4[1]) * sc, hi_f(w4[1]) * sc);
+      o.z = h2bits(lo_f(w4[2]) * sc, hi_f(w4[2]) * sc);
+      o.w = h2bits(lo_f(w4[3]) * sc, hi_f(w4[3]) * sc);
+      *reinterpret_cast<uint4*>(A + chunk_off(row, c)) = o;
+    }
+    fence_async_smem();
+    tc_before_sync();
+    wg_sync(wg);
+    // ---- rotation: D_rot = A (Pi'_hi + Pi'_lo)^T -----------------------------------
+    if (leader) {
+      tc_after_sync();
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t koff = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+        mma_f16(d_rot, smem_desc(sA + koff), smem_desc(base_s + OFF_PIH + koff), s > 0 ? 1u : 0u);
+        mma_f16(d_rot, smem_desc(sA + koff), smem_desc(base_s + OFF_PIL + koff), 1u);
+      }
+      mma_commit(bar_rot);
+    }
+    if (wg_any(wg, !mbar_wait(bar_rot, iter & 1))) { fault = true; break; }
+    tc_after_sync();
+
+    // ---- epilogue 1: indices, packing, residual --------------------------------------
+    // y = D_rot / (sc * nrm * 2^8)
+    const float inv = nrm > 0.f ? 1.f / (sc * nrm * 256.f) : 0.f;
+    uint32_t words[WORDS];
+#pragma unroll
+    for (int w = 0; w < WORDS; ++w) words[w] = 0u;
+    float rho2 = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      float d[32];
+      tmem_ld32(d_rot + lane_base + ch * 32, d);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int j = ch * 32 + i;
+        const float y = d[i] * inv;
+        const int idx = lm_idx<BITS>(y, pmid, pb);
+        if (BITS == 3) {
+          words[j / 16] |= (uint32_t)(idx & 3) << (2 * (j % 16));
+          words[W_MAIN + j / 32] |= (uint32_t)(idx >> 2) << (j % 32);
+        } else {
+          words[j / PER] |= (uint32_t)idx << (BITS * (j % PER));
+        }
+        if (QJL) {
+          const float r = y - s_cen[idx];
+          rho2 = fmaf(r, r, rho2);
+          d[i] = r * 16384.f;
+        }
+      }
+      if (QJL) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float r0 = d[8 * q + 2 * u], r1 = d[8 * q + 2 * u + 1];
+            const __half2 h = __floats2half2_rn(r0, r1);
+            const float2 f = __half22float2(h);
+            hv[u] = *reinterpret_cast<const uint32_t*>(&h);
+            lv[u] = h2bits(r0 - f.x, r1 - f.y);
+          }
+          *reinterpret_cast<uint4*>(A + chunk_off(row, ch * 4 + q)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(A2 + chunk_off(row, ch * 4 + q)) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
+      }
+    }
+    const int64_t rec = live ? out_rec(a, v) : 0;
+    if (live) {
+      uint4* dst = reinterpret_cast<uint4*>(a.codes + rec * WORDS);
+#pragma unroll
+      for (int q = 0; q < WORDS / 4; ++q)
+        dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+      a.norm[rec] = nrm;
+    }
+    if (!QJL) {
+      tc_before_sync();
+      wg_sync(wg);   // A and D_rot are free for the next tile
+      continue;
+    }
+    fence_async_smem();
+    tc_before_sync();
+    wg_sync(wg);
+    // ---- QJL product: D_qjl = (2^14 r) S^T ----------------------------------------------
+    if (leader) {
+      tc_after_sync();
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const uint32_t koff = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+        mma_f16(d_qjl, smem_desc(sA + koff), smem_desc(base_s + OFF_S + koff), s > 0 ? 1u : 0u);
+        mma_f16(d_qjl, smem_desc(sA + SMEM_TILE + koff), smem_desc(base_s + OFF_S + koff), 1u);
+      }
+      mma_commit(bar_q);
+    }
+    if (wg_any(wg, !mbar_wait(bar_q, iter & 1))) { fault = true; break; }
+    tc_after_sync();
+    const float rho = sqrtf(rho2);
+    // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 |S_i| rho.
+    const float thr_scale = 0.125f * rho;
+    uint32_t qw[4] = {0u, 0u, 0u, 0u};
+    uint32_t flag[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      float d[32];
+      tmem_ld32(d_qjl + lane_base + ch * 32, d);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        qw[ch] |= (d[i] >= 0.f ? 1u : 0u) << i;
+        flag[ch] |= (fabsf(d[i]) <= thr_scale * s_snorm[ch * 32 + i] ? 1u : 0u) << i;
+      }
+    }
+    if (!live) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
+    // Exact fp32 signs for flagged rows, two rows per lane per pass; r is rebuilt
+    // from y exactly as above (tcgen05.ld is warp-collective, so whole warps loop).
+    while (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
+      int rows[2] = {-1, -1};
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int fw = 0; fw < 4; ++fw) {
+          if (rows[q] < 0 && flag[fw] != 0u) {
+            const int bit = __ffs(flag[fw]) - 1;
+            flag[fw] &= flag[fw] - 1;
+            rows[q] = fw * 32 + bit;
+          }
+        }
+      }
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float d[32];
+        tmem_ld32(d_rot + lane_base + ch * 32, d);
+        if (rows[0] >= 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float y = d[i] * inv;
+            const float r = y - s_cen[lm_idx<BITS>(y, pmid, pb)];
+            acc0 = fmaf(__ldg(a.s_f32 + (size_t)rows[0] * 128 + ch * 32 + i), r, acc0);
+            if (rows[1] >= 0) acc1 = fmaf(__ldg(a.s_f32 + (size_t)rows[1] * 128 + ch * 32 + i), r, acc1);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (rows[q] >= 0) {
+          const int fw = rows[q] >> 5, bit = rows[q] & 31;
+          const bool pos = (q == 0 ? acc0 : acc1) >= 0.f;
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (w == fw) qw[w] = (qw[w] & ~(1u << bit)) | ((pos ? 1u : 0u) << bit);
+        }
+      }
+    }
+    if (live) {
+      *reinterpret_cast<uint4*>(a.qjl + rec * 4) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+      a.rnorm[rec] = nrm * rho;
+    }
+    tc_before_sync();
+    wg_sync(wg);
+  }
+  if (fault) atomicExch(&g_tq_fault, 1);
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem) : "memory");
+  }
+}
+
+template <int BITS>
+cudaError_t launch_bits(const QuantTcArgs& a, bool qjl, int grid, cudaStream_t s) {
+  if (qjl) {
+    k_quant_tc<BITS, true><<<grid, 256, TC_SMEM, s>>>(a);
+  } else {
+    k_quant_tc<BITS, false><<<grid, 256, TC_SMEM, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t configure_bits() {
+  cudaError_t e = cudaFuncSetAttribute(k_quant_tc<BITS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_quant_tc<BITS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_fault(int* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_tq_fault, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_tq_fault, &zero, sizeof(int));
+}
+
+cudaError_t configure_quant_tc() {
+  cudaError_t e;
+  if ((e = configure_bits<1>()) != cudaSuccess) return e;
+  if ((e = configure_bits<2>()) != cudaSuccess) return e;
+  if ((e = configure_bits<3>()) != cudaSuccess) return e;
+  return configure_bits<4>();
+}
+
+cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s) {
+  const int64_t tiles = (a.n + TILE - 1) / TILE;
+  int64_t grid = (tiles + 1) / 2;
+  if (grid > sms) grid = sms;
+  if (grid < 1) grid = 1;
+  const bool qjl = a.m > 0;
+  switch (a.bits) {
+    case 1: return launch_bits<1>(a, qjl, (int)grid, s);
+    case 2: return launch_bits<2>(a, qjl, (int)grid, s);
+    case 3: return launch_bits<3>(a, qjl, (int)grid, s);
+    case 4: return launch_bits<4>(a, qjl, (int)grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tqk

@@ -94,6 +94,14 @@ const char* tq_last_error(void);
 const char* tq_version(void);
 
 /*
+ * tq_device_fault - synchronising diagnostic: reads and clears the device
+ * fault code that kernels set when a bounded wait on the tensor cores gives
+ * up (0 = none).  The kernel that set it has released its resources and
+ * returned; its outputs for the affected tiles are undefined.
+ */
+int tq_device_fault(int* code);
+
+/*
  * tq_init - build the per-context tables on the host in fp64 and upload them
  * to the current CUDA device ([WHAT] stage 1 steps 1-2, stage 2).
  *   d       vector dimension.
