@@ -192,9 +192,8 @@ tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
   }
   // Operand images of the tensor-core quantizer (d = 128): 128 x 128 fp16,
   // K-major, two 64-wide K blocks, 16-byte chunks swizzled with the row.
+  if (cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) c->sms = 148;
   if (d == 128) {
-    e = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device);
-    if (e != cudaSuccess) c->sms = 148;
     std::vector<uint16_t> img(3 * 128 * 128, 0);
     std::vector<float> snorm(128, 0.f);
     auto put = [&](int which, int r, int k, double v) {

@@ -481,7 +481,6 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
   Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
@@ -490,6 +489,14 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
     lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
   }
 
+  __syncthreads();
+  // Persistent CTAs: the value table is built once; items are (sequence, kv
+  // head, context chunk), taken round-robin.
+  const int64_t n_items = (int64_t)a.splits * a.Hkv * a.B;
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  const int split = (int)(item % a.splits);
+  const int kvh = (int)((item / a.splits) % a.Hkv);
+  const int b = (int)(item / ((int64_t)a.splits * a.Hkv));
   // ---- query-side operands: column g carries head (g & 3); g >= 4 the tails
   const int hh = g & 3;
   const bool tail_col = g >= 4;
@@ -794,6 +801,8 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
     float* pp = a.part + (prow * a.splits + split) * (128 + 2);
     pp[c] = (c == 0) ? M : acc;
   }
+  __syncthreads();  // merge scratch aliases the next item's pipeline stages
+  }
 }
 
 }  // namespace
@@ -812,11 +821,13 @@ int attn_mma_chunk() { return 512; }
 
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
   dim3 grid(a.splits, a.Hkv, a.B);
+  const int64_t items = (int64_t)a.splits * a.Hkv * a.B;
+  const unsigned pgrid = (unsigned)(items < (int64_t)c->sms * 3 ? items : (int64_t)c->sms * 3);
   cudaError_t e = cudaSuccess;
   switch (a.G) {
 #define TQ_G4(GG)                                                                              \
   case GG:                                                                                     \
-    k_attn_g4<GG><<<grid, MW * 32, SMEM_BYTES, s>>>(a);                                        \
+    k_attn_g4<GG><<<pgrid, MW * 32, SMEM_BYTES, s>>>(a);                                       \
     break;
     TQ_G4(1)
     TQ_G4(2)

@@ -150,6 +150,58 @@ __device__ __forceinline__ int lm_idx(float y, float pmid, const float* pb) {
   return (y >= 0.f) ? H + j : H - 1 - j;
 }
 
+struct Q4 {
+  uint32_t w[4];
+};
+
+// Exact fp32 signs of the flagged QJL rows (rare), two rows per lane per
+// pass; r is rebuilt from the rotation accumulator exactly as in the main
+// epilogue.  tcgen05.ld is warp-collective, so whole warps call and loop.
+template <int BITS>
+__device__ __noinline__ Q4 qjl_fixup(uint32_t taddr, float inv, float pmid, const float* pb,
+                                     const float* s_cen, const float* s_f32, Q4 flag, Q4 qw) {
+  while (__any_sync(0xffffffffu, (flag.w[0] | flag.w[1] | flag.w[2] | flag.w[3]) != 0u)) {
+    int rows[2] = {-1, -1};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+      for (int fw = 0; fw < 4; ++fw) {
+        if (rows[q] < 0 && flag.w[fw] != 0u) {
+          const int bit = __ffs(flag.w[fw]) - 1;
+          flag.w[fw] &= flag.w[fw] - 1;
+          rows[q] = fw * 32 + bit;
+        }
+      }
+    }
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      float d[32];
+      tmem_ld32(taddr + ch * 32, d);
+      if (rows[0] >= 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float y = d[i] * inv;
+          const float r = fmaf(y, 16384.f, -s_cen[lm_idx<BITS>(y, pmid, pb)]);
+          acc0 = fmaf(__ldg(s_f32 + (size_t)rows[0] * 128 + ch * 32 + i), r, acc0);
+          if (rows[1] >= 0) acc1 = fmaf(__ldg(s_f32 + (size_t)rows[1] * 128 + ch * 32 + i), r, acc1);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (rows[q] >= 0) {
+        const int fw = rows[q] >> 5, bit = rows[q] & 31;
+        const bool pos = (q == 0 ? acc0 : acc1) >= 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (w == fw) qw.w[w] = (qw.w[w] & ~(1u << bit)) | ((pos ? 1u : 0u) << bit);
+      }
+    }
+  }
+  return qw;
+}
+
 template <int BITS, bool QJL>
 __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
   extern __shared__ unsigned char smem_raw[];
@@ -180,7 +232,7 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
       if (QJL) dst[OFF_S / 16 + e] = src_s[e];
     }
     if (tid < 128) s_snorm[tid] = QJL ? a.snorm[tid] : 0.f;
-    if (tid < 16) s_cen[tid] = tid < L ? a.cen[tid] : 0.f;
+    if (tid < 16) s_cen[tid] = tid < L ? a.cen[tid] * (QJL ? 16384.f : 1.f) : 0.f;
     if (tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
   }
   if (tid == 0) {
@@ -208,43 +260,60 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
   const uint32_t bar_rot = bar0 + 8 * wg, bar_q = bar0 + 16 + 8 * wg;
   const bool leader = row == 0;
   const float* pb = s_pb;
+  float snorm_max = 0.f;
+  if (QJL)
+    for (int i = 0; i < 128; ++i) snorm_max = fmaxf(snorm_max, s_snorm[i]);
   const float pmid = BITS >= 2 ? s_pb[(L >> 2) - 1] : 0.f;
 
   const int64_t ntiles = (a.n + TILE - 1) / TILE;
-  uint32_t iter = 0;
-  bool fault = false;
-  for (int64_t tile = (int64_t)blockIdx.x * 2 + wg; tile < ntiles; tile += (int64_t)gridDim.x * 2, ++iter) {
-    const int64_t v = tile * TILE + row;
-    const bool live = v < a.n;
-    // ---- load x, norm, scaled fp16 operand ----------------------------------------
-    uint4 xr[16];
-    if (live) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.x) + v * a.ld);
+  const int64_t tstride = (int64_t)gridDim.x * 2;
+  const bool is_bf = a.dtype == TQ_BF16;
+  auto lo_f = [&](uint32_t w) {
+    return is_bf ? __uint_as_float(w << 16) : __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
+  };
+  auto hi_f = [&](uint32_t w) {
+    return is_bf ? __uint_as_float(w & 0xFFFF0000u) : __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+  };
+  uint4 xr[16];
+  auto load_x = [&](int64_t t) {
+    const int64_t vv = t * TILE + row;
+    if (vv < a.n) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.x) + vv * a.ld);
 #pragma unroll
       for (int c = 0; c < 16; ++c) xr[c] = src[c];
     } else {
 #pragma unroll
       for (int c = 0; c < 16; ++c) xr[c] = make_uint4(0, 0, 0, 0);
     }
-    const bool is_bf = a.dtype == TQ_BF16;
-    auto lo_f = [&](uint32_t w) {
-      return is_bf ? __uint_as_float(w << 16) : __half2float(__ushort_as_half((unsigned short)(w & 0xFFFF)));
-    };
-    auto hi_f = [&](uint32_t w) {
-      return is_bf ? __uint_as_float(w & 0xFFFF0000u) : __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-    };
-    float ss = 0.f;
+  };
+  uint32_t iter = 0;
+  bool fault = false;
+  for (int64_t tile = (int64_t)blockIdx.x * 2 + wg; tile < ntiles; tile += tstride, ++iter) {
+    const int64_t v = tile * TILE + row;
+    const bool live = v < a.n;
+    {
+      const int64_t nxt = tile + tstride;
+      if (leader && a.ld == 128 && nxt < ntiles) {
+        const int64_t rows_left = a.n - nxt * TILE;
+        const uint32_t bytes = (uint32_t)((rows_left < TILE ? rows_left : TILE) * 256);
+        const void* p = static_cast<const unsigned short*>(a.x) + nxt * TILE * 128;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+      }
+    }
+    load_x(tile);
+    // ---- norm and the scaled fp16 operand ------------------------------------------
+    float ssp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t w4[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float f0 = lo_f(w4[q]), f1 = hi_f(w4[q]);
-        ss = fmaf(f0, f0, ss);
-        ss = fmaf(f1, f1, ss);
+        ssp[q] = fmaf(f0, f0, ssp[q]);
+        ssp[q] = fmaf(f1, f1, ssp[q]);
       }
     }
-    const float nrm = sqrtf(ss);
+    const float nrm = sqrtf((ssp[0] + ssp[1]) + (ssp[2] + ssp[3]));
     const int e = nrm > 0.f ? 14 - flog2(nrm) : 0;
     const float sc = pow2f(e);
 #pragma unroll
@@ -274,32 +343,41 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
     if (wg_any(wg, !mbar_wait(bar_rot, iter & 1))) { fault = true; break; }
     tc_after_sync();
 
-    // ---- epilogue 1: indices, packing, residual --------------------------------------
-    // y = D_rot / (sc * nrm * 2^8)
+    // ---- epilogue 1: indices, packing, residual (32 coordinates per pass) -------------
+    // y = D_rot / (sc * nrm * 2^8); the residual goes out scaled by 2^14.
     const float inv = nrm > 0.f ? 1.f / (sc * nrm * 256.f) : 0.f;
-    uint32_t words[WORDS];
-#pragma unroll
-    for (int w = 0; w < WORDS; ++w) words[w] = 0u;
-    float rho2 = 0.f;
-#pragma unroll
+    const int64_t rec = live ? out_rec(a, v) : 0;
+    uint32_t* crow = a.codes + rec * WORDS;
+    float rho2v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
     for (int ch = 0; ch < 4; ++ch) {
       float d[32];
       tmem_ld32(d_rot + lane_base + ch * 32, d);
+      // words of this chunk: b words of b-bit fields (b = 3: two 2-bit words + one bit word)
+      uint32_t cw[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int j = ch * 32 + i;
         const float y = d[i] * inv;
         const int idx = lm_idx<BITS>(y, pmid, pb);
         if (BITS == 3) {
-          words[j / 16] |= (uint32_t)(idx & 3) << (2 * (j % 16));
-          words[W_MAIN + j / 32] |= (uint32_t)(idx >> 2) << (j % 32);
+          cw[i >> 4] |= (uint32_t)(idx & 3) << (2 * (i & 15));
+          cw[2] |= (uint32_t)(idx >> 2) << i;
         } else {
-          words[j / PER] |= (uint32_t)idx << (BITS * (j % PER));
+          cw[i / PER] |= (uint32_t)idx << (BITS * (i % PER));
         }
         if (QJL) {
-          const float r = y - s_cen[idx];
-          rho2 = fmaf(r, r, rho2);
-          d[i] = r * 16384.f;
+          const float r = fmaf(y, 16384.f, -s_cen[idx]);   // s_cen holds 2^14 c
+          rho2v[i & 3] = fmaf(r, r, rho2v[i & 3]);
+          d[i] = r;
+        }
+      }
+      if (live) {
+        if (BITS == 4) *reinterpret_cast<uint4*>(crow + 4 * ch) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        if (BITS == 2) *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
+        if (BITS == 1) crow[ch] = cw[0];
+        if (BITS == 3) {
+          *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
+          crow[W_MAIN + ch] = cw[2];
         }
       }
       if (QJL) {
@@ -319,14 +397,7 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
         }
       }
     }
-    const int64_t rec = live ? out_rec(a, v) : 0;
-    if (live) {
-      uint4* dst = reinterpret_cast<uint4*>(a.codes + rec * WORDS);
-#pragma unroll
-      for (int q = 0; q < WORDS / 4; ++q)
-        dst[q] = make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-      a.norm[rec] = nrm;
-    }
+    if (live) a.norm[rec] = nrm;
     if (!QJL) {
       tc_before_sync();
       wg_sync(wg);   // A and D_rot are free for the next tile
@@ -348,9 +419,9 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
     }
     if (wg_any(wg, !mbar_wait(bar_q, iter & 1))) { fault = true; break; }
     tc_after_sync();
-    const float rho = sqrtf(rho2);
-    // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 |S_i| rho.
-    const float thr_scale = 0.125f * rho;
+    const float rho = sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) * (1.f / 16384.f);
+    // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho.
+    const float thr = 0.125f * rho * snorm_max;
     uint32_t qw[4] = {0u, 0u, 0u, 0u};
     uint32_t flag[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -360,50 +431,16 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         qw[ch] |= (d[i] >= 0.f ? 1u : 0u) << i;
-        flag[ch] |= (fabsf(d[i]) <= thr_scale * s_snorm[ch * 32 + i] ? 1u : 0u) << i;
+        flag[ch] |= (fabsf(d[i]) <= thr ? 1u : 0u) << i;
       }
     }
     if (!live) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
-    // Exact fp32 signs for flagged rows, two rows per lane per pass; r is rebuilt
-    // from y exactly as above (tcgen05.ld is warp-collective, so whole warps loop).
-    while (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
-      int rows[2] = {-1, -1};
+    if (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
+      const Q4 fixed = qjl_fixup<BITS>(d_rot + lane_base, inv, pmid, pb, s_cen, a.s_f32,
+                                       Q4{{flag[0], flag[1], flag[2], flag[3]}},
+                                       Q4{{qw[0], qw[1], qw[2], qw[3]}});
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int fw = 0; fw < 4; ++fw) {
-          if (rows[q] < 0 && flag[fw] != 0u) {
-            const int bit = __ffs(flag[fw]) - 1;
-            flag[fw] &= flag[fw] - 1;
-            rows[q] = fw * 32 + bit;
-          }
-        }
-      }
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        float d[32];
-        tmem_ld32(d_rot + lane_base + ch * 32, d);
-        if (rows[0] >= 0) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float y = d[i] * inv;
-            const float r = y - s_cen[lm_idx<BITS>(y, pmid, pb)];
-            acc0 = fmaf(__ldg(a.s_f32 + (size_t)rows[0] * 128 + ch * 32 + i), r, acc0);
-            if (rows[1] >= 0) acc1 = fmaf(__ldg(a.s_f32 + (size_t)rows[1] * 128 + ch * 32 + i), r, acc1);
-          }
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (rows[q] >= 0) {
-          const int fw = rows[q] >> 5, bit = rows[q] & 31;
-          const bool pos = (q == 0 ? acc0 : acc1) >= 0.f;
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            if (w == fw) qw[w] = (qw[w] & ~(1u << bit)) | ((pos ? 1u : 0u) << bit);
-        }
-      }
+      for (int w = 0; w < 4; ++w) qw[w] = fixed.w[w];
     }
     if (live) {
       *reinterpret_cast<uint4*>(a.qjl + rec * 4) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
