@@ -364,10 +364,12 @@ def run_gpu(args, w):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.time()
+    torch.cuda.nvtx.range_push("tq:decode_steps")
     e0.record()
     for i in range(args.steps):
         step(i, evs[i])
     e1.record()
+    torch.cuda.nvtx.range_pop()
     barrier()
     sampler.mark(w0, time.time())
     t_ms = e0.elapsed_time(e1) / args.steps
@@ -414,7 +416,9 @@ def run_gpu(args, w):
     d2h = hout.numel() * hout.element_size()
     del g_app, g_att, g_e2e
 
+    torch.cuda.nvtx.range_push("tq:quantize_sweep")
     quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
+    torch.cuda.nvtx.range_pop()
     clocks = sampler.stop()
 
     tm = torch.tensor([t_ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)

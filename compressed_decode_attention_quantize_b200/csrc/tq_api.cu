@@ -330,6 +330,11 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.pos = pos;
   a.H = H;
   a.max_T = max_T;
+  if (n <= tqk::kSmallQuantize) {
+    cudaError_t e = tqk::launch_quantize_small(c, a, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return TQ_OK;
+  }
   const bool tc = c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
@@ -487,9 +492,10 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   if (tqk::attn_mma_supported(c, a) && max_T > 0) {
     a.chunk = tqk::attn_mma_chunk();
     a.splits = (int)((max_T + a.chunk - 1) / a.chunk);
-    if (a.splits > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: context too long");
+    if (a.splits > 4096) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: context too long (max 2M tokens)");
     e = tqk::launch_attn_mma(c, a, out, s);
   } else {
+    if (a.splits > 4096) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
     e = tqk::launch_attn(c, a, out, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");

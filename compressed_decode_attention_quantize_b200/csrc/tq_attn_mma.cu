@@ -543,9 +543,10 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   };
   // Keys: k-step s (0..15) reads word s>>3 of the thread's two code words;
   // slot 0/1 use registers u = 2(s&7) and 2(s&7)+1.
-  uint32_t bk[16][2];
+  uint2 bk[16];  // 64-bit pairs: each B fragment sits in an aligned register pair
 #pragma unroll
   for (int s = 0; s < 16; ++s) {
+    uint32_t pr[2];
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
       const int u = 2 * (s & 7) + slot;
@@ -554,20 +555,23 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
       const int dlo = 16 * (s >> 3) + (elo >> 1), dhi = 16 * (s >> 3) + (ehi >> 1);
       const float vlo = qv[dlo] * ((elo & 1) ? wq1 : wq0) * inv;
       const float vhi = qv[dhi] * ((ehi & 1) ? wq1 : wq0) * inv;
-      bk[s][slot] = operand(vlo, vhi);
+      pr[slot] = operand(vlo, vhi);
     }
+    bk[s] = make_uint2(pr[0], pr[1]);
   }
   // QJL: k-step s (0..7), slot 0/1 use registers 2s, 2s+1 of the thread's word.
-  uint32_t bj[8][2];
+  uint2 bj[8];
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
+    uint32_t pr[2];
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) {
       const int u = 2 * s + slot;
       const int elo = 10 + u, ehi = (26 + u) & 31;
       const float inv = bit_inv(bit_pos(u)) * ks;
-      bj[s][slot] = operand(sv[elo] * inv, sv[ehi] * inv);
+      pr[slot] = operand(sv[elo] * inv, sv[ehi] * inv);
     }
+    bj[s] = make_uint2(pr[0], pr[1]);
   }
   // Logit constants for heads 2t, 2t+1 (threads t < 2):
   //   s2 = kn * (acc * KA + KB) + kr * (acs * QA + QB)
@@ -661,7 +665,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   mma16816(acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                                    \
            bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81),                                         \
            bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01),                                     \
-           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S][0], bk[S][1]);
+           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S].x, bk[S].y);
       TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6)
       TQ_KSTEP(7) TQ_KSTEP(8) TQ_KSTEP(9) TQ_KSTEP(10) TQ_KSTEP(11) TQ_KSTEP(12) TQ_KSTEP(13)
       TQ_KSTEP(14) TQ_KSTEP(15)
@@ -669,7 +673,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
       const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
 #define TQ_QSTEP(S)                                                                               \
   mma16816(acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8), bit_half2<2 * (S) + 1>(Q0),      \
-           bit_half2<2 * (S) + 1>(Q8), bj[S][0], bj[S][1]);
+           bit_half2<2 * (S) + 1>(Q8), bj[S].x, bj[S].y);
       TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
       TQ_QSTEP(7)
 #undef TQ_QSTEP

@@ -123,6 +123,9 @@ struct QuantTcArgs {
 };
 
 cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
+// One block per vector, for small batches (n <= kSmallQuantize).
+constexpr int64_t kSmallQuantize = 4096;
+cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
 // Tensor-core quantize for d = 128 (16-bit inputs).
 cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s);
 cudaError_t configure_quant_tc();

@@ -228,9 +228,85 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 }
 
 // ----------------------------------------------------------------------------
+// Quantize, small batches (the per-step cache append): one block per vector,
+// thread j owns coordinate j (and QJL row j), so a few hundred vectors spread
+// over all SMs instead of filling one tile.  Same fp32 arithmetic as above.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int w = 0; w < nw; ++w) t += red[w];
+  return t;
+}
+
+__global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
+  extern __shared__ float sh[];
+  float* sx = sh;            // [dpad] x, later r
+  __shared__ float red[8];
+  __shared__ float s_cen[16], s_bnd[16];
+  const int j = threadIdx.x, lane = j & 31;
+  const int64_t v = blockIdx.x;
+  if (j < 16) {
+    s_cen[j] = (j < (1 << a.bits)) ? a.cen[j] : 0.f;
+    s_bnd[j] = (j < a.nbnd) ? a.bnd[j] : INFINITY;
+  }
+  const float xj = (j < a.d) ? load_elem(a.x, a.dtype, v * a.ld + j) : 0.f;
+  sx[j] = xj;
+  const float nrm = sqrtf(block_sum(xj * xj, red));   // includes the barrier for sx / tables
+  float a4[4] = {0.f, 0.f, 0.f, 0.f};
+  int k = 0;
+  for (; k + 4 <= a.d; k += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a4[u] = fmaf(a.PiT[(size_t)(k + u) * dpad + j], sx[k + u], a4[u]);
+  }
+  for (; k < a.d; ++k) a4[0] = fmaf(a.PiT[(size_t)k * dpad + j], sx[k], a4[0]);
+  const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+  const float y = (nrm > 0.f && j < a.d) ? acc / nrm : 0.f;
+  const int idx = lm_index(y, s_bnd, a.nbnd);
+  const int64_t rec = out_record(a, v);
+  // b-bit field packing within each warp (b = 3: 2-bit stream, then 1-bit stream)
+  const uint32_t iv = (j < a.d) ? (uint32_t)idx : 0u;
+  const int i32 = j >> 5;
+  if (a.bits == 3) {
+    const int w2 = (a.d + 15) >> 4;
+    const uint32_t lo = field_word(iv & 3u, 2, lane);
+    const uint32_t hi = field_word(iv >> 2, 1, lane);
+    const int wlo = 2 * i32 + (lane >> 4);
+    if ((lane & 15) == 0 && wlo < w2) a.codes[rec * a.words + wlo] = lo;
+    if (lane == 0) a.codes[rec * a.words + w2 + i32] = hi;
+  } else {
+    const int per = 32 / a.bits;
+    const uint32_t wv = field_word(iv, a.bits, lane);
+    const int wi = a.bits * i32 + lane / per;
+    if (lane % per == 0 && wi < a.words) a.codes[rec * a.words + wi] = wv;
+  }
+  if (j == 0) a.norm[rec] = nrm;
+  if (a.m == 0) return;
+  const float r = (j < a.d) ? y - s_cen[idx] : 0.f;
+  __syncthreads();   // everyone has read x
+  sx[j] = r;
+  const float rho = sqrtf(block_sum(r * r, red));
+  float b4[4] = {0.f, 0.f, 0.f, 0.f};
+  k = 0;
+  for (; k + 4 <= a.d; k += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) b4[u] = fmaf(a.ST[(size_t)(k + u) * dpad + j], sx[k + u], b4[u]);
+  }
+  for (; k < a.d; ++k) b4[0] = fmaf(a.ST[(size_t)k * dpad + j], sx[k], b4[0]);
+  const float sr = (b4[0] + b4[1]) + (b4[2] + b4[3]);
+  const uint32_t bits = __ballot_sync(0xffffffffu, sr >= 0.f && j < a.m);
+  if (lane == 0 && j < a.m) a.qjl[rec * ((a.m + 31) >> 5) + i32] = bits;
+  if (j == 0) a.rnorm[rec] = nrm * rho;
+}
+
+// ----------------------------------------------------------------------------
 // Query pre-rotation: q' = Pi q, s = S q' (one block per query row).
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int d, int dpad,
+__global__ void __launch_bounds__(128) k_prerotate(const void* q, int dtype, int d, int dpad,
                                                    int m, const float* PiT, const float* ST,
                                                    float* qr, float* qs) {
   extern __shared__ float sh[];
@@ -241,17 +317,29 @@ __global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int
     sq[k] = (k < d) ? load_elem(q, dtype, row * d + k) : 0.f;
   __syncthreads();
   for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
-    float acc = 0.f;
-    for (int k = 0; k < d; ++k) acc = fmaf(PiT[(size_t)k * dpad + j], sq[k], acc);
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    int k = 0;
+    for (; k + 4 <= d; k += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a4[u] = fmaf(PiT[(size_t)(k + u) * dpad + j], sq[k + u], a4[u]);
+    }
+    for (; k < d; ++k) a4[0] = fmaf(PiT[(size_t)k * dpad + j], sq[k], a4[0]);
+    const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
     sr[j] = acc;
     qr[row * dpad + j] = acc;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < dpad; i += blockDim.x) {
-    float acc = 0.f;
-    if (i < m)
-      for (int k = 0; k < d; ++k) acc = fmaf(ST[(size_t)k * dpad + i], sr[k], acc);
-    qs[row * dpad + i] = acc;
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (i < m) {
+      int k = 0;
+      for (; k + 4 <= d; k += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a4[u] = fmaf(ST[(size_t)(k + u) * dpad + i], sr[k + u], a4[u]);
+      }
+      for (; k < d; ++k) a4[0] = fmaf(ST[(size_t)k * dpad + i], sr[k], a4[0]);
+    }
+    qs[row * dpad + i] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
   }
 }
 
@@ -427,32 +515,67 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
 }
 
 // Log-sum-exp merge of the split partials and the final o = Pi^T o_rot.
+// The split maxima and sums are staged in shared memory with one load per
+// thread; each thread then folds its coordinate over the splits with
+// independent loads (eight in flight).
 __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int splits, int d, int dpad,
                                                     const float* Pi, float* out) {
   extern __shared__ float sh[];
-  float* so = sh;  // [dpad]
+  float* so = sh;                 // [dpad]
+  float* sw = sh + dpad;          // [splits] weights exp2(m_s - M)
+  __shared__ float s_red[4];
+  __shared__ float s_M, s_L;
   const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* pr = part + row * splits * (dpad + 2);
-  float M = kNegInf;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, pr[s * (dpad + 2)]);
-  float L = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = pr[s * (dpad + 2)];
-    if (ms != kNegInf) L += exp2f(ms - M) * pr[s * (dpad + 2) + 1];
+  float mloc = -INFINITY;
+  for (int sidx = tid; sidx < splits; sidx += blockDim.x) {
+    const float ms = pr[(int64_t)sidx * (dpad + 2)];
+    sw[sidx] = ms;
+    mloc = fmaxf(mloc, ms);
   }
-  for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float ms = pr[s * (dpad + 2)];
-      if (ms != kNegInf) acc = fmaf(exp2f(ms - M), pr[s * (dpad + 2) + 2 + j], acc);
+  mloc = warp_max(mloc);
+  if (lane == 0) s_red[warp] = mloc;
+  __syncthreads();
+  if (tid == 0) s_M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  __syncthreads();
+  const float M = s_M;
+  float lloc = 0.f;
+  for (int sidx = tid; sidx < splits; sidx += blockDim.x) {
+    const float ms = sw[sidx];
+    const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    sw[sidx] = w;
+    lloc = fmaf(w, pr[(int64_t)sidx * (dpad + 2) + 1], lloc);
+  }
+  lloc = warp_sum(lloc);
+  __syncthreads();
+  if (lane == 0) s_red[warp] = lloc;
+  __syncthreads();
+  if (tid == 0) s_L = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
+  __syncthreads();
+  const float L = s_L;
+  for (int j = tid; j < dpad; j += blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int sidx = 0;
+    for (; sidx + 8 <= splits; sidx += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        acc[u] = fmaf(sw[sidx + u], pr[(int64_t)(sidx + u) * (dpad + 2) + 2 + j], acc[u]);
     }
-    so[j] = (L > 0.f) ? acc / L : 0.f;
+    for (; sidx < splits; ++sidx) acc[0] = fmaf(sw[sidx], pr[(int64_t)sidx * (dpad + 2) + 2 + j], acc[0]);
+    const float tot = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    so[j] = (L > 0.f) ? tot / L : 0.f;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc = 0.f;
-    for (int j = 0; j < d; ++j) acc = fmaf(Pi[(size_t)j * d + i], so[j], acc);
-    out[row * d + i] = acc;
+  for (int i = tid; i < d; i += blockDim.x) {
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    int j = 0;
+    for (; j + 4 <= d; j += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a4[u] = fmaf(Pi[(size_t)(j + u) * d + i], so[j + u], a4[u]);
+    }
+    for (; j < d; ++j) a4[0] = fmaf(Pi[(size_t)j * d + i], so[j], a4[0]);
+    out[row * d + i] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
   }
 }
 
@@ -785,10 +908,16 @@ cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s)
   TQ_DISPATCH_J(c->J, return quantize_J<JV>(a, s));
 }
 
+cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStream_t s) {
+  if (a.n == 0) return cudaSuccess;
+  k_quantize_small<<<(unsigned)a.n, c->dpad, c->dpad * sizeof(float), s>>>(a, c->dpad);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
                              float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
-  k_prerotate<<<(unsigned)rows, 256, 2 * c->dpad * sizeof(float), s>>>(
+  k_prerotate<<<(unsigned)rows, 128, 2 * c->dpad * sizeof(float), s>>>(
       q, dtype, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs);
   return cudaGetLastError();
 }
@@ -809,7 +938,7 @@ int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
 }
 
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
-  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, c->dpad * sizeof(float), s>>>(
+  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, (c->dpad + a.splits) * sizeof(float), s>>>(
       a.part, a.splits, c->d, c->dpad, c->Pi_f, out);
   return cudaGetLastError();
 }

@@ -340,3 +340,42 @@ def test_quantize_append_writes_addressed_slots(cuda):
                 mask = torch.ones(T, dtype=torch.bool)
                 mask[p] = False
                 assert torch.all(got[b][:, mask] == -7), (k, b)
+
+
+def test_quantize_tensor_core_fp16_strided(cuda):
+    """More than 4096 vectors of fp16 input with a row pitch of 136 elements
+    (the tensor-core path), including zero rows and a ragged last tile."""
+    c = _ctx(128, 3, 4, 128, seed=2)
+    tab = P.oracle_tables(c)
+    n = 5000
+    X = tq_inputs.outlier_kv(1, 1, n, 128, seed=12)[0, 0].half()
+    X[7] = 0
+    big = torch.zeros(n, 136, dtype=torch.float16)
+    big[:, :128] = X
+    src = big.to(cuda)[:, :128]
+    for which, wch in ((tq.TQ_KEY, "k"), (tq.TQ_VALUE, "v")):
+        pk = c.empty_packed(which, (n,))
+        c.quantize_into(src, which, pk)
+        torch.cuda.synchronize()
+        assert tq.tq_device_fault() == 0
+        P.check_quantized(tab, wch, X.double().numpy(), _flat(pk, n))
+
+
+def test_quantize_append_large_batch(cuda):
+    """Appending 8192 (sequence, head) rows at per-sequence slots (tensor-core
+    path with cache placement)."""
+    c = _ctx(128, 3, 4, 128, seed=0)
+    B, H, T = 64, 128, 6
+    x = tq_inputs.outlier_kv(B, H, 1, 128, seed=19)[:, :, 0].contiguous().to(cuda)
+    pos = torch.randint(0, T, (B,), generator=torch.Generator().manual_seed(3), dtype=torch.int32).to(cuda)
+    for which in (tq.TQ_KEY, tq.TQ_VALUE):
+        cache = c.empty_packed(which, (B, H, T), device=cuda)
+        c.quantize_append(x, which, cache, pos)
+        ref = c.quantize(x.reshape(B * H, 128), which)
+        torch.cuda.synchronize()
+        for k, v in cache.items():
+            if v is None:
+                continue
+            want = ref[k].reshape((B, H) + tuple(v.shape[3:]))
+            got = v[torch.arange(B, device=cuda), :, pos.long()]
+            assert torch.equal(got, want), k
