@@ -60,9 +60,12 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources of the decode-attention kernel (its counters go stale
+    when these change)."""
     h = hashlib.sha256()
-    for f in sorted((ROOT / "compressed_decode_attention_quantize_b200" / "csrc").glob("*")):
-        h.update(f.read_bytes())
+    csrc = ROOT / "compressed_decode_attention_quantize_b200" / "csrc"
+    for name in ("tq_attn_mma.cu", "tq_internal.h"):
+        h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
 
