@@ -497,9 +497,10 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   const int split = (int)(item % a.splits);
   const int kvh = (int)((item / a.splits) % a.Hkv);
   const int b = (int)(item / ((int64_t)a.splits * a.Hkv));
-  // ---- query-side operands: column g carries head (g & 3); g >= 4 the tails
-  const int hh = g & 3;
-  const bool tail_col = g >= 4;
+  // ---- query-side operands: column g carries head g/2, even columns the fp16
+  // head and odd columns the tail of the same operand.
+  const int hh = g >> 1;
+  const bool tail_col = (g & 1) != 0;
   const bool head_ok = hh < G;
   const int64_t qrow_i = (int64_t)b * a.Hq + (int64_t)kvh * G + (head_ok ? hh : 0);
   const float* qrow = a.qr + qrow_i * 128 + 32 * t;
@@ -573,20 +574,19 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
     }
     bj[s] = make_uint2(pr[0], pr[1]);
   }
-  // Logit constants for heads 2t, 2t+1 (threads t < 2):
+  // Logit constants for head t (the head of this thread's accumulator columns):
   //   s2 = kn * (acc * KA + KB) + kr * (acs * QA + QB)
-  float KA[2], KB[2], QA[2], QB[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int src = ((2 * t + j) & 3) * 4;
+  float KA, KB, QA, QB;
+  {
+    const int src = 8 * t;   // lane (g = 2t, any t') holds head t's operand exponents
     const int eqj = __shfl_sync(0xffffffffu, eq, src);
     const int esj = __shfl_sync(0xffffffffu, es, src);
     const float sqj = __shfl_sync(0xffffffffu, sumq, src);
     const float ssj = __shfl_sync(0xffffffffu, sums, src);
-    KA[j] = pow2i(eqj + ew + 1) * a.scale_log2;
-    KB[j] = c0 * sqj * a.scale_log2;
-    QA[j] = 2.f * pow2i(esj) * a.cq * a.scale_log2;
-    QB[j] = -ssj * a.cq * a.scale_log2;
+    KA = pow2i(eqj + ew + 1) * a.scale_log2;
+    KB = c0 * sqj * a.scale_log2;
+    QA = 2.f * pow2i(esj) * a.cq * a.scale_log2;
+    QB = -ssj * a.cq * a.scale_log2;
   }
 
   const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
@@ -638,13 +638,12 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   __syncthreads();
 
   const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_part[2] = {0.f, 0.f};
+  float m_run = -INFINITY, l_part = 0.f;
   int kv_run = -126;
   float o[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  const bool own_heads = t < 2;
+  const bool own_head = t < G;
 
   for (int i = 0; i < nt; ++i) {
     if (i + NST - 1 < nt) issue(i + NST - 1, (i + NST - 1) % NST);
@@ -678,31 +677,22 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
       TQ_QSTEP(7)
 #undef TQ_QSTEP
     }
-    // Tails sit in columns 2t+4, 2t+5 (lane ^ 2).
-    float sc[4];
+    // Columns 2t (head) and 2t+1 (tail) of head t.
+    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
+    float sc0, sc1;
     {
-      const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
-      const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float lm = fmaf(__shfl_xor_sync(0xffffffffu, acc[r], 2), 1.f / 4096.f, acc[r]);
-        const float qj = fmaf(__shfl_xor_sync(0xffffffffu, acs[r], 2), 1.f / 4096.f, acs[r]);
-        const int j = r & 1;
-        const float kn = r < 2 ? kn0 : kn8, kr = r < 2 ? kr0 : kr8;
-        const bool ok = own_heads && (r < 2 ? v0 : v8);
-        sc[r] = ok ? fmaf(kn, fmaf(lm, KA[j], KB[j]), kr * fmaf(qj, QA[j], QB[j])) : -INFINITY;
-      }
+      const float lm0 = fmaf(acc[1], 1.f / 4096.f, acc[0]), lm8 = fmaf(acc[3], 1.f / 4096.f, acc[2]);
+      const float qj0 = fmaf(acs[1], 1.f / 4096.f, acs[0]), qj8 = fmaf(acs[3], 1.f / 4096.f, acs[2]);
+      sc0 = (own_head && v0) ? fmaf(st.kn[g], fmaf(lm0, KA, KB), st.kr[g] * fmaf(qj0, QA, QB)) : -INFINITY;
+      sc1 = (own_head && v8) ? fmaf(st.kn[g + 8], fmaf(lm8, KA, KB), st.kr[g + 8] * fmaf(qj8, QA, QB))
+                             : -INFINITY;
     }
 
-    // ---- online softmax (heads 2t, 2t+1 for t < 2) ------------------------------
-    float tmax[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 4));
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 8));
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 16));
-    }
-    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
+    // ---- online softmax (head t) --------------------------------------------------
+    float tmax = fmaxf(sc0, sc1);
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
     const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
     float vmax = fmaxf(vn0, vn8);
     vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
@@ -714,28 +704,23 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
     const float vchange = pow2i(max(kv_run - kv_new, -126));
     kv_run = kv_new;
     const float vmul = pow2i(-kv_new);
-    float alpha[2], mnew[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      mnew[j] = fmaxf(m_run[j], tmax[j]);
-      alpha[j] = (mnew[j] == -INFINITY) ? 1.f : ex2f(m_run[j] - mnew[j]);
-      m_run[j] = mnew[j];
-    }
-    float p[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) p[r] = (sc[r] == -INFINITY) ? 0.f : ex2f(sc[r] - mnew[r & 1]);
-    l_part[0] = fmaf(l_part[0], alpha[0], p[0] + p[2]);
-    l_part[1] = fmaf(l_part[1], alpha[1], p[1] + p[3]);
-    const float oa0 = alpha[0] * vchange, oa1 = alpha[1] * vchange;
-    if (__any_sync(0xffffffffu, oa0 != 1.f || oa1 != 1.f)) {
+    const float mnew = fmaxf(m_run, tmax);
+    const float alpha = (mnew == -INFINITY) ? 1.f : ex2f(m_run - mnew);
+    m_run = mnew;
+    const float p0 = (sc0 == -INFINITY) ? 0.f : ex2f(sc0 - mnew);
+    const float p1 = (sc1 == -INFINITY) ? 0.f : ex2f(sc1 - mnew);
+    l_part = fmaf(l_part, alpha, p0 + p1);
+    const float oa = alpha * vchange;
+    if (__any_sync(0xffffffffu, oa != 1.f)) {
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        o[mt][0] *= oa0; o[mt][1] *= oa1; o[mt][2] *= oa0; o[mt][3] *= oa1;
+        o[mt][0] *= oa;
+        o[mt][2] *= oa;
       }
     }
-    const float w0v = vn0 * vmul, w8v = vn8 * vmul;
-    const uint32_t pb0 = movtrans(pack_half2(p[0] * w0v, p[1] * w0v));
-    const uint32_t pb1 = movtrans(pack_half2(p[2] * w8v, p[3] * w8v));
+    // P tile (16 tokens x 8 columns): column 2t = head t, odd columns zero.
+    const uint32_t pb0 = movtrans(pack_half2(p0 * vn0 * vmul, 0.f));
+    const uint32_t pb1 = movtrans(pack_half2(p1 * vn8 * vmul, 0.f));
 
     // ---- values ---------------------------------------------------------------
     const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
@@ -764,29 +749,22 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
   cp_wait<0>();
 
   // ---- merge the four warps of the CTA -------------------------------------------
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 4);
-    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 8);
-    l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 16);
-  }
+  l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
+  l_part += __shfl_xor_sync(0xffffffffu, l_part, 8);
+  l_part += __shfl_xor_sync(0xffffffffu, l_part, 16);
   __syncthreads();
   float* sm = reinterpret_cast<float*>(stages);   // [MW][4][130]
   const float vback = pow2i(kv_run);
-  if (own_heads) {
+  if (own_head) {
+    float* rowp = sm + (warp * 4 + t) * 130;
+    if (g == 0) {
+      rowp[0] = m_run;
+      rowp[1] = l_part;
+    }
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int h = 2 * t + j;
-      float* row = sm + (warp * 4 + h) * 130;
-      if (g == 0) {
-        row[0] = m_run[j];
-        row[1] = l_part[j];
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        row[2 + 16 * g + mt] = o[mt][j] * vback;
-        row[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
-      }
+    for (int mt = 0; mt < 8; ++mt) {
+      rowp[2 + 16 * g + mt] = o[mt][0] * vback;
+      rowp[2 + 16 * g + 8 + mt] = o[mt][2] * vback;
     }
   }
   __syncthreads();
