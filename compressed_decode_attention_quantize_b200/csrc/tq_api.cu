@@ -418,8 +418,14 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
   return TQ_OK;
 }
 
-size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
-  if (!c || B <= 0 || Hq <= 0 || max_T < 0) return 0;
+// Workspace: [q' and S q' rows][tile prefix][partials].  The partials are
+// sized for the larger of the split layout ([B Hq][splits][dpad + 2]) and
+// the segment layout ([warps + B Hkv][G][dpad + 2] <= [4 warps + B Hq][...]).
+namespace {
+struct AttnWs {
+  size_t q_bytes, tiles_off, part_off, total;
+};
+AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   int chunk = 0;
   int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
   // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most
@@ -427,10 +433,21 @@ size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   const int64_t mma_splits = (max_T + tqk::attn_mma_chunk() - 1) / tqk::attn_mma_chunk();
   if (mma_splits > splits) splits = (int)mma_splits;
   const size_t rows = (size_t)B * Hq;
-  size_t b = 2 * rows * c->dpad * sizeof(float);
-  b = (b + 255) & ~(size_t)255;
-  b += rows * (size_t)splits * (c->dpad + 2) * sizeof(float);
-  return b + 256;
+  const size_t row_bytes = (size_t)(c->dpad + 2) * sizeof(float);
+  const size_t split_part = rows * (size_t)splits * row_bytes;
+  const size_t seg_part = ((size_t)tqk::attn_seg_max_warps(c) * 4 + rows) * row_bytes;
+  AttnWs w;
+  w.q_bytes = 2 * rows * c->dpad * sizeof(float);
+  w.tiles_off = (w.q_bytes + 255) & ~(size_t)255;
+  w.part_off = (w.tiles_off + ((size_t)B + 1) * sizeof(int64_t) + 255) & ~(size_t)255;
+  w.total = w.part_off + (split_part > seg_part ? split_part : seg_part) + 256;
+  return w;
+}
+}  // namespace
+
+size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
+  if (!c || B <= 0 || Hq <= 0 || max_T < 0) return 0;
+  return attn_ws_layout(c, B, Hq, max_T).total;
 }
 
 int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
@@ -455,13 +472,11 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_attn_decode: workspace not 256-byte aligned");
   cudaStream_t s = as_stream(stream);
   const size_t rows = (size_t)B * Hq;
+  const AttnWs lay = attn_ws_layout(c, B, Hq, max_T);
   char* p = static_cast<char*>(workspace);
   float* qr = reinterpret_cast<float*>(p);
   float* qs = qr + rows * c->dpad;
-  size_t off = (2 * rows * c->dpad * sizeof(float) + 255) & ~(size_t)255;
-  float* part = reinterpret_cast<float*>(p + off);
-  cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, qr, qs, s);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode: prerotate");
+  float* part = reinterpret_cast<float*>(p + lay.part_off);
   tqk::AttnArgs a{};
   a.qr = qr;
   a.qs = qs;
@@ -489,15 +504,20 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.cv = c->cv_f;
   a.splits = tqk::attn_splits(c, B, Hkv, max_T > 0 ? max_T : 1, &a.chunk);
   a.part = part;
-  if (tqk::attn_mma_supported(c, a) && max_T > 0) {
+  a.tiles = nullptr;
+  const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
+  if (mma && tqk::attn_seg_path(a)) {
+    a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
+  } else if (mma) {
     a.chunk = tqk::attn_mma_chunk();
     a.splits = (int)((max_T + a.chunk - 1) / a.chunk);
     if (a.splits > 4096) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: context too long (max 2M tokens)");
-    e = tqk::launch_attn_mma(c, a, out, s);
-  } else {
-    if (a.splits > 4096) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
-    e = tqk::launch_attn(c, a, out, s);
+  } else if (a.splits > 4096) {
+    return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
   }
+  cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode: prerotate");
+  e = mma ? tqk::launch_attn_mma(c, a, out, s) : tqk::launch_attn(c, a, out, s);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
   return TQ_OK;
 }

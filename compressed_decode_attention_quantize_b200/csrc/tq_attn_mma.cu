@@ -474,8 +474,28 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) 
 // floor(log2(x)) for a positive normal float.
 __device__ __forceinline__ int ilog2f(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
 
+// ---------------------------------------------------------------------------
+// Group size <= 4, balanced segments.  The 16-token tiles of all (sequence,
+// kv head) rows form one sequence of W tiles (row-major over b, kv head,
+// tile; the prefix a.tiles[b] counts the tiles of rows before sequence b).
+// Warp w of the launch takes tiles [w W / N, (w + 1) W / N), N = min(warps,
+// W), so every warp gets a non-empty, equal share whatever the length mix.
+// A warp's range crosses row boundaries at most a few times; for each row
+// piece it builds the query operands once, streams the tiles through its own
+// cp.async ring and writes one partial (m, l, o) per head to slot
+// w + b Hkv + kv head, which is unique because consecutive rows' pieces come
+// from non-decreasing warps.  The merge finds a row's slots from the same
+// arithmetic.
+//
+// Softmax: the running maximum only moves when a tile's maximum exceeds it
+// by more than 2^8 (in exp2 units); probabilities then stay below 2^8, and
+// the value norms of a piece are scaled once, from the piece's largest norm,
+// so that p |v| stays below 2^15 in fp16.
+// ---------------------------------------------------------------------------
+constexpr float LAZY_TAU = 8.f;
+
 template <int G>
-__global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
+__global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   static_assert(G <= 4, "packed path");
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
@@ -488,302 +508,310 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_g4(AttnArgs a) {
     const int byte = e >> 5;
     lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
   }
+  __syncthreads();   // the only block-wide barrier: warps run independently below
 
-  __syncthreads();
-  // Persistent CTAs: the value table is built once; items are (sequence, kv
-  // head, context chunk), taken round-robin.
-  const int64_t n_items = (int64_t)a.splits * a.Hkv * a.B;
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-  const int split = (int)(item % a.splits);
-  const int kvh = (int)((item / a.splits) % a.Hkv);
-  const int b = (int)(item / ((int64_t)a.splits * a.Hkv));
-  // ---- query-side operands: column g carries head g/2, even columns the fp16
-  // head and odd columns the tail of the same operand.
+  const int64_t* P = a.tiles;
+  const int64_t W = P[a.B];
+  const int64_t NW = min((int64_t)gridDim.x * MW, W);
+  const int64_t wid = (int64_t)blockIdx.x * MW + warp;
+  if (wid >= NW) return;
+  int64_t x = wid * W / NW;
+  const int64_t x1 = (wid + 1) * W / NW;
+
+  // Sequence holding tile x: P[b] <= x < P[b + 1].
+  int b = 0;
+  {
+    int hi = a.B;
+    while (hi - b > 1) {
+      const int mid = (b + hi) >> 1;
+      if (P[mid] <= x) b = mid; else hi = mid;
+    }
+  }
+
+  const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
+  const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
+  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  Stage* my = stages + warp * NST;
+  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
+  // Column g of the query-side B operands carries head g/2: even columns the
+  // fp16 head of the operand, odd columns its tail (x 2^12).
   const int hh = g >> 1;
   const bool tail_col = (g & 1) != 0;
   const bool head_ok = hh < G;
-  const int64_t qrow_i = (int64_t)b * a.Hq + (int64_t)kvh * G + (head_ok ? hh : 0);
-  const float* qrow = a.qr + qrow_i * 128 + 32 * t;
-  const float* srow = a.qs + qrow_i * 128 + 32 * t;
-  float qv[32], sv[32];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 x = reinterpret_cast<const float4*>(qrow)[i];
-    const float4 y = reinterpret_cast<const float4*>(srow)[i];
-    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
-    sv[4 * i] = y.x; sv[4 * i + 1] = y.y; sv[4 * i + 2] = y.z; sv[4 * i + 3] = y.w;
-  }
-  float mq = 0.f, ms = 0.f, sumq = 0.f, sums = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    mq = fmaxf(mq, fabsf(qv[i]));
-    ms = fmaxf(ms, fabsf(sv[i]));
-    sumq += qv[i];
-    sums += sv[i];
-  }
-#pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
-    ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
-    sumq += __shfl_xor_sync(0xffffffffu, sumq, o);
-    sums += __shfl_xor_sync(0xffffffffu, sums, o);
-  }
-  const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
-  const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
-  const int eq = mq > 0.f ? ilog2f(mq) : 0;
-  const int es = ms > 0.f ? ilog2f(ms) : 0;
-  // q' * w * 2^-(eq+ew+1) < 2, times at most 2^14: fits fp16.
-  const float kq = head_ok ? pow2i(-(eq + ew + 1)) : 0.f;
-  const float ks = head_ok ? pow2i(-es) : 0.f;
-  const float wq0 = w0 * kq, wq1 = w1 * kq;
-  auto operand = [&](float lo, float hi) -> uint32_t {
-    const __half2 h = __floats2half2_rn(lo, hi);
-    if (!tail_col) return *reinterpret_cast<const uint32_t*>(&h);
-    const float2 f = __half22float2(h);
-    return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
-  };
-  // Keys: k-step s (0..15) reads word s>>3 of the thread's two code words;
-  // slot 0/1 use registers u = 2(s&7) and 2(s&7)+1.
-  uint2 bk[16];  // 64-bit pairs: each B fragment sits in an aligned register pair
-#pragma unroll
-  for (int s = 0; s < 16; ++s) {
-    uint32_t pr[2];
-#pragma unroll
-    for (int slot = 0; slot < 2; ++slot) {
-      const int u = 2 * (s & 7) + slot;
-      const int elo = 10 + u, ehi = (26 + u) & 31;
-      const float inv = bit_inv(bit_pos(u));
-      const int dlo = 16 * (s >> 3) + (elo >> 1), dhi = 16 * (s >> 3) + (ehi >> 1);
-      const float vlo = qv[dlo] * ((elo & 1) ? wq1 : wq0) * inv;
-      const float vhi = qv[dhi] * ((ehi & 1) ? wq1 : wq0) * inv;
-      pr[slot] = operand(vlo, vhi);
+  const bool own_head = t < G;   // accumulator columns 2t, 2t+1 belong to head t
+
+  while (x < x1) {
+    while (P[b + 1] <= x) ++b;
+    const int64_t tb = (P[b + 1] - P[b]) / a.Hkv;
+    const int64_t rel = x - P[b];
+    const int kvh = (int)(rel / tb);
+    const int64_t tt = rel - (int64_t)kvh * tb;
+    const int64_t te = min(tb, tt + (x1 - x));
+    const int nt = (int)(te - tt);
+    const int64_t slot = wid + (int64_t)b * a.Hkv + kvh;
+    x += nt;
+
+    const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
+    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
+    const int64_t tok0 = tt * MT;
+    const int64_t tok1 = min(te * MT, len);
+
+    // ---- cp.async ring: lane assignment fixed for the piece -------------------
+    // slot 0 = key codes, slots 1-2 = value codes, slot 3 = QJL words or norms.
+    const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;
+    const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;
+    const char* p2 = p1 + 8 * 64;
+    const char* p3;
+    int stride3, tok3;
+    uint32_t d3;
+    if (lane < 16) {
+      p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
+      stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
+    } else if (lane < 28) {
+      const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
+      const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
+      p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
+      stride3 = 4; tok3 = 4 * part;
+      d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
+    } else {
+      p3 = nullptr; stride3 = 0; tok3 = 1 << 30; d3 = 0;
     }
-    bk[s] = make_uint2(pr[0], pr[1]);
-  }
-  // QJL: k-step s (0..7), slot 0/1 use registers 2s, 2s+1 of the thread's word.
-  uint2 bj[8];
+    const uint32_t d0 = offsetof(Stage, k) + lane * 16;
+    const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
+    const uint32_t d2 = d1 + 8 * (VROW * 4);
+    auto issue = [&](int i, int stage) {
+      const int64_t t0 = tok0 + (int64_t)MT * i;
+      const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
+      cp16(sb + d0, p0 + t0 * 32, t0 + (lane >> 1) < tok1);
+      cp16(sb + d1, p1 + t0 * 64, t0 + (lane >> 2) < tok1);
+      cp16(sb + d2, p2 + t0 * 64, t0 + 8 + (lane >> 2) < tok1);
+      if (lane < 28) cp16(sb + d3, p3 + t0 * stride3, t0 + tok3 < tok1);
+    };
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    uint32_t pr[2];
-#pragma unroll
-    for (int slot = 0; slot < 2; ++slot) {
-      const int u = 2 * s + slot;
-      const int elo = 10 + u, ehi = (26 + u) & 31;
-      const float inv = bit_inv(bit_pos(u)) * ks;
-      pr[slot] = operand(sv[elo] * inv, sv[ehi] * inv);
+    for (int i = 0; i < NST - 1; ++i) {
+      if (i < nt) issue(i, i);
+      cp_commit();
     }
-    bj[s] = make_uint2(pr[0], pr[1]);
-  }
-  // Logit constants for head t (the head of this thread's accumulator columns):
-  //   s2 = kn * (acc * KA + KB) + kr * (acs * QA + QB)
-  float KA, KB, QA, QB;
-  {
-    const int src = 8 * t;   // lane (g = 2t, any t') holds head t's operand exponents
-    const int eqj = __shfl_sync(0xffffffffu, eq, src);
-    const int esj = __shfl_sync(0xffffffffu, es, src);
-    const float sqj = __shfl_sync(0xffffffffu, sumq, src);
-    const float ssj = __shfl_sync(0xffffffffu, sums, src);
-    KA = pow2i(eqj + ew + 1) * a.scale_log2;
-    KB = c0 * sqj * a.scale_log2;
-    QA = 2.f * pow2i(esj) * a.cq * a.scale_log2;
-    QB = -ssj * a.cq * a.scale_log2;
-  }
 
-  const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
-  const int c_begin = split * a.chunk;
-  const int c_end = (int)min(T, (int64_t)c_begin + a.chunk);
-  const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
-
-  // Per-lane cp.async assignment (fixed for all tiles): slot 0 = key codes,
-  // slots 1-2 = value codes, slot 3 = QJL words or norms.
-  Stage* my = stages + warp * NST;
-  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
-  const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;   // tok lane>>1
-  const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;   // tok lane>>2
-  const char* p2 = p1 + 8 * 64;                                                         // tok 8+lane>>2
-  const char* p3;
-  int stride3, tok3;
-  uint32_t d3;
-  if (lane < 16) {
-    p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
-    stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
-  } else if (lane < 28) {
-    const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
-    const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
-    p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
-    stride3 = 4; tok3 = 4 * part;
-    d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
-  } else {
-    p3 = nullptr; stride3 = 0; tok3 = 1 << 30; d3 = 0;
-  }
-  const uint32_t d0 = offsetof(Stage, k) + lane * 16;
-  const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
-  const uint32_t d2 = d1 + 8 * (VROW * 4);
-  auto issue = [&](int tile, int stage) {
-    const int t0 = c_begin + MT * (warp + MW * tile);
-    const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
-    cp16(sb + d0, p0 + (int64_t)t0 * 32, t0 + (lane >> 1) < c_end);
-    cp16(sb + d1, p1 + (int64_t)t0 * 64, t0 + (lane >> 2) < c_end);
-    cp16(sb + d2, p2 + (int64_t)t0 * 64, t0 + 8 + (lane >> 2) < c_end);
-    if (lane < 28) cp16(sb + d3, p3 + (int64_t)t0 * stride3, t0 + tok3 < c_end);
-  };
-
-  const int ntiles_cta = c_end > c_begin ? (c_end - c_begin + MT - 1) / MT : 0;
-  const int nt = ntiles_cta > warp ? (ntiles_cta - warp + MW - 1) / MW : 0;
+    // ---- query-side operands (while the first tiles are in flight) ------------
+    const int64_t qrow_i = (int64_t)b * a.Hq + (int64_t)kvh * G + (head_ok ? hh : 0);
+    const float* qrow = a.qr + qrow_i * 128 + 32 * t;
+    const float* srow = a.qs + qrow_i * 128 + 32 * t;
+    float qv[32], sv[32];
 #pragma unroll
-  for (int i = 0; i < NST - 1; ++i) {
-    if (i < nt) issue(i, i);
-    cp_commit();
-  }
-  __syncthreads();
-
-  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
-  float m_run = -INFINITY, l_part = 0.f;
-  int kv_run = -126;
-  float o[8][4];
+    for (int i = 0; i < 8; ++i) {
+      const float4 xq = reinterpret_cast<const float4*>(qrow)[i];
+      const float4 yq = reinterpret_cast<const float4*>(srow)[i];
+      qv[4 * i] = xq.x; qv[4 * i + 1] = xq.y; qv[4 * i + 2] = xq.z; qv[4 * i + 3] = xq.w;
+      sv[4 * i] = yq.x; sv[4 * i + 1] = yq.y; sv[4 * i + 2] = yq.z; sv[4 * i + 3] = yq.w;
+    }
+    float mq = 0.f, ms = 0.f, sumq = 0.f, sums = 0.f;
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  const bool own_head = t < G;
-
-  for (int i = 0; i < nt; ++i) {
-    if (i + NST - 1 < nt) issue(i + NST - 1, (i + NST - 1) % NST);
-    cp_commit();
-    cp_wait<NST - 1>();
-    __syncwarp();
-    const Stage& st = my[i % NST];
-    const int t0 = c_begin + MT * (warp + MW * i);
-
-    // ---- logits -------------------------------------------------------------
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < 32; ++i) {
+      mq = fmaxf(mq, fabsf(qv[i]));
+      ms = fmaxf(ms, fabsf(sv[i]));
+      sumq += qv[i];
+      sums += sv[i];
+    }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+      sumq += __shfl_xor_sync(0xffffffffu, sumq, o);
+      sums += __shfl_xor_sync(0xffffffffu, sums, o);
+    }
+    const int eq = mq > 0.f ? ilog2f(mq) : 0;
+    const int es = ms > 0.f ? ilog2f(ms) : 0;
+    // q' * w * 2^-(eq+ew+1) < 2, times at most 2^14: fits fp16.
+    const float kq = head_ok ? pow2i(-(eq + ew + 1)) : 0.f;
+    const float ks = head_ok ? pow2i(-es) : 0.f;
+    const float wq0 = w0 * kq, wq1 = w1 * kq;
+    auto operand = [&](float lo, float hi) -> uint32_t {
+      const __half2 h = __floats2half2_rn(lo, hi);
+      if (!tail_col) return *reinterpret_cast<const uint32_t*>(&h);
+      const float2 f = __half22float2(h);
+      return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
+    };
+    // Keys: k-step s (0..15) reads word s>>3 of the thread's two code words;
+    // slots 0/1 use registers u = 2(s&7) and 2(s&7)+1.
+    uint2 bk[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+      uint32_t pr[2];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        const int u = 2 * (s & 7) + sl;
+        const int elo = 10 + u, ehi = (26 + u) & 31;
+        const float inv = bit_inv(bit_pos(u));
+        const int dlo = 16 * (s >> 3) + (elo >> 1), dhi = 16 * (s >> 3) + (ehi >> 1);
+        const float vlo = qv[dlo] * ((elo & 1) ? wq1 : wq0) * inv;
+        const float vhi = qv[dhi] * ((ehi & 1) ? wq1 : wq0) * inv;
+        pr[sl] = operand(vlo, vhi);
+      }
+      bk[s] = make_uint2(pr[0], pr[1]);
+    }
+    // QJL: k-step s (0..7), slots 0/1 use registers 2s, 2s+1 of the thread's word.
+    uint2 bj[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      uint32_t pr[2];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        const int u = 2 * s + sl;
+        const int elo = 10 + u, ehi = (26 + u) & 31;
+        const float inv = bit_inv(bit_pos(u)) * ks;
+        pr[sl] = operand(sv[elo] * inv, sv[ehi] * inv);
+      }
+      bj[s] = make_uint2(pr[0], pr[1]);
+    }
+    // Logit constants of head t:  s2 = kn (acc KA + KB) + kr (acs QA + QB).
+    float KA, KB, QA, QB;
     {
-      const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
-      const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
-      const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
-      const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
+      const int src = 8 * t;   // lanes with g = 2t hold head t's operand scales
+      const int eqj = __shfl_sync(0xffffffffu, eq, src);
+      const int esj = __shfl_sync(0xffffffffu, es, src);
+      const float sqj = __shfl_sync(0xffffffffu, sumq, src);
+      const float ssj = __shfl_sync(0xffffffffu, sums, src);
+      KA = pow2i(eqj + ew + 1) * a.scale_log2;
+      KB = c0 * sqj * a.scale_log2;
+      QA = 2.f * pow2i(esj) * a.cq * a.scale_log2;
+      QB = -ssj * a.cq * a.scale_log2;
+    }
+
+    // ---- value-norm scale of the piece ---------------------------------------
+    float vmax = 0.f;
+    {
+      const float* vr = a.vnorm + row0;
+      for (int64_t j = tok0 + 4 * lane; j < tok1; j += 128) {
+        if (j + 4 <= tok1) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
+        } else {
+          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    // p <= 2^8 and |v| 2^-kv < 2^7 keep p |v| 2^-kv below 2^15.
+    const int kv = vmax >= FLT_MIN ? max(ilog2f(vmax) - 6, -120) : -120;
+    const float vmul = pow2i(-kv);
+
+    float m_run = own_head ? -INFINITY : 0.f;
+    float l_part = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    for (int i = 0; i < nt; ++i) {
+      if (i + NST - 1 < nt) issue(i + NST - 1, (i + NST - 1) % NST);
+      cp_commit();
+      cp_wait<NST - 1>();
+      __syncwarp();
+      const Stage& st = my[i % NST];
+      const int64_t t0 = tok0 + (int64_t)MT * i;
+
+      // ---- logits -----------------------------------------------------------
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
+        const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
+        const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
+        const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
 #define TQ_KSTEP(S)                                                                               \
   mma16816(acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                                    \
            bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81),                                         \
            bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01),                                     \
            bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S].x, bk[S].y);
-      TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6)
-      TQ_KSTEP(7) TQ_KSTEP(8) TQ_KSTEP(9) TQ_KSTEP(10) TQ_KSTEP(11) TQ_KSTEP(12) TQ_KSTEP(13)
-      TQ_KSTEP(14) TQ_KSTEP(15)
+        TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6)
+        TQ_KSTEP(7) TQ_KSTEP(8) TQ_KSTEP(9) TQ_KSTEP(10) TQ_KSTEP(11) TQ_KSTEP(12) TQ_KSTEP(13)
+        TQ_KSTEP(14) TQ_KSTEP(15)
 #undef TQ_KSTEP
-      const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
+        const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
 #define TQ_QSTEP(S)                                                                               \
   mma16816(acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8), bit_half2<2 * (S) + 1>(Q0),      \
            bit_half2<2 * (S) + 1>(Q8), bj[S].x, bj[S].y);
-      TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
-      TQ_QSTEP(7)
+        TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
+        TQ_QSTEP(7)
 #undef TQ_QSTEP
-    }
-    // Columns 2t (head) and 2t+1 (tail) of head t.
-    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
-    float sc0, sc1;
-    {
+      }
+      // Columns 2t (head) and 2t+1 (tail) of head t; rows g and g+8 are tokens.
+      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
       const float lm0 = fmaf(acc[1], 1.f / 4096.f, acc[0]), lm8 = fmaf(acc[3], 1.f / 4096.f, acc[2]);
       const float qj0 = fmaf(acs[1], 1.f / 4096.f, acs[0]), qj8 = fmaf(acs[3], 1.f / 4096.f, acs[2]);
-      sc0 = (own_head && v0) ? fmaf(st.kn[g], fmaf(lm0, KA, KB), st.kr[g] * fmaf(qj0, QA, QB)) : -INFINITY;
-      sc1 = (own_head && v8) ? fmaf(st.kn[g + 8], fmaf(lm8, KA, KB), st.kr[g + 8] * fmaf(qj8, QA, QB))
-                             : -INFINITY;
-    }
+      const float sc0 = (own_head && v0) ? fmaf(st.kn[g], fmaf(lm0, KA, KB), st.kr[g] * fmaf(qj0, QA, QB))
+                                         : -INFINITY;
+      const float sc1 = (own_head && v8)
+                            ? fmaf(st.kn[g + 8], fmaf(lm8, KA, KB), st.kr[g + 8] * fmaf(qj8, QA, QB))
+                            : -INFINITY;
 
-    // ---- online softmax (head t) --------------------------------------------------
-    float tmax = fmaxf(sc0, sc1);
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-    const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
-    float vmax = fmaxf(vn0, vn8);
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
-    // p * |v| * 2^-kv stays below 2^15 in fp16.
-    const int kv_tile = vmax > 1e-30f ? ilog2f(vmax) - 14 : -126;
-    const int kv_new = max(kv_run, kv_tile);
-    const float vchange = pow2i(max(kv_run - kv_new, -126));
-    kv_run = kv_new;
-    const float vmul = pow2i(-kv_new);
-    const float mnew = fmaxf(m_run, tmax);
-    const float alpha = (mnew == -INFINITY) ? 1.f : ex2f(m_run - mnew);
-    m_run = mnew;
-    const float p0 = (sc0 == -INFINITY) ? 0.f : ex2f(sc0 - mnew);
-    const float p1 = (sc1 == -INFINITY) ? 0.f : ex2f(sc1 - mnew);
-    l_part = fmaf(l_part, alpha, p0 + p1);
-    const float oa = alpha * vchange;
-    if (__any_sync(0xffffffffu, oa != 1.f)) {
+      // ---- online softmax, head t ---------------------------------------------
+      const float loc = fmaxf(sc0, sc1);
+      if (__any_sync(0xffffffffu, loc > m_run + LAZY_TAU)) {
+        float tmax = loc;
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        const float mnew = fmaxf(m_run, tmax);
+        const float alpha = ex2f(m_run - mnew);   // 0 on the first update, 1 if unchanged
+        m_run = mnew;
+        l_part *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= alpha;
+          o[mt][2] *= alpha;
+        }
+      }
+      const float p0 = ex2f(sc0 - m_run), p1 = ex2f(sc1 - m_run);
+      l_part += p0 + p1;
+      // P tile (16 tokens x 8 columns): column 2t = head t, odd columns zero.
+      const uint32_t pb0 = movtrans(pack_half2(p0 * (st.vn[g] * vmul), 0.f));
+      const uint32_t pb1 = movtrans(pack_half2(p1 * (st.vn[g + 8] * vmul), 0.f));
+
+      // ---- values ---------------------------------------------------------------
+      const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
+      const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
+      const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
+      const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
+      const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
+                              (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
+                              (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
+                              (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
+      const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
+                              ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
+                              ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
+                              ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        o[mt][0] *= oa;
-        o[mt][2] *= oa;
+        const int k = mt >> 1;
+        const uint32_t* y = (mt & 1) ? yo : ye;
+        uint32_t av[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
+        mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+      }
+      __syncwarp();
+    }
+    cp_wait<0>();
+    __syncwarp();   // the next piece's ring refills stages this one read
+
+    // ---- partial of the piece ------------------------------------------------
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 8);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 16);
+    if (own_head) {
+      float* pp = a.part + (slot * G + t) * (128 + 2);
+      const float vback = pow2i(kv);
+      if (g == 0) {
+        pp[0] = m_run;
+        pp[1] = l_part;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        pp[2 + 16 * g + mt] = o[mt][0] * vback;
+        pp[2 + 16 * g + 8 + mt] = o[mt][2] * vback;
       }
     }
-    // P tile (16 tokens x 8 columns): column 2t = head t, odd columns zero.
-    const uint32_t pb0 = movtrans(pack_half2(p0 * vn0 * vmul, 0.f));
-    const uint32_t pb1 = movtrans(pack_half2(p1 * vn8 * vmul, 0.f));
-
-    // ---- values ---------------------------------------------------------------
-    const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
-    const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
-    const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
-    const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
-    const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
-                            (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
-                            (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
-                            (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
-    const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
-                            ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
-                            ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
-                            ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const int k = mt >> 1;
-      const uint32_t* y = (mt & 1) ? yo : ye;
-      uint32_t av[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
-      mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
-    }
-    __syncwarp();
-  }
-  cp_wait<0>();
-
-  // ---- merge the four warps of the CTA -------------------------------------------
-  l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
-  l_part += __shfl_xor_sync(0xffffffffu, l_part, 8);
-  l_part += __shfl_xor_sync(0xffffffffu, l_part, 16);
-  __syncthreads();
-  float* sm = reinterpret_cast<float*>(stages);   // [MW][4][130]
-  const float vback = pow2i(kv_run);
-  if (own_head) {
-    float* rowp = sm + (warp * 4 + t) * 130;
-    if (g == 0) {
-      rowp[0] = m_run;
-      rowp[1] = l_part;
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      rowp[2 + 16 * g + mt] = o[mt][0] * vback;
-      rowp[2 + 16 * g + 8 + mt] = o[mt][2] * vback;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * 130; e += MW * 32) {
-    const int h = e / 130, c = e % 130;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < MW; ++w) M = fmaxf(M, sm[(w * 4 + h) * 130]);
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < MW; ++w) {
-      const float mw_ = sm[(w * 4 + h) * 130];
-      if (mw_ != -INFINITY) acc = fmaf(exp2f(mw_ - M), sm[(w * 4 + h) * 130 + (c == 0 ? 1 : c)], acc);
-    }
-    const int64_t prow = (int64_t)b * a.Hq + (int64_t)kvh * G + h;
-    float* pp = a.part + (prow * a.splits + split) * (128 + 2);
-    pp[c] = (c == 0) ? M : acc;
-  }
-  __syncthreads();  // merge scratch aliases the next item's pipeline stages
   }
 }
 
@@ -801,30 +829,34 @@ bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
 
 int attn_mma_chunk() { return 512; }
 
-cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
-  dim3 grid(a.splits, a.Hkv, a.B);
-  const int64_t items = (int64_t)a.splits * a.Hkv * a.B;
-  const unsigned pgrid = (unsigned)(items < (int64_t)c->sms * 3 ? items : (int64_t)c->sms * 3);
-  cudaError_t e = cudaSuccess;
-  switch (a.G) {
-#define TQ_G4(GG)                                                                              \
-  case GG:                                                                                     \
-    k_attn_g4<GG><<<pgrid, MW * 32, SMEM_BYTES, s>>>(a);                                       \
-    break;
-    TQ_G4(1)
-    TQ_G4(2)
-    TQ_G4(4)
-#undef TQ_G4
-#define TQ_G(GG)                                                                               \
-  case GG:                                                                                     \
-    k_attn_mma<GG><<<grid, MW * 32, SMEM_BYTES, s>>>(a);                                       \
-    break;
-    TQ_G(8)
-#undef TQ_G
-    default:
-      return cudaErrorInvalidValue;
+bool attn_seg_path(const AttnArgs& a) { return a.G == 1 || a.G == 2 || a.G == 4; }
+
+// Three 4-warp CTAs per SM (the register limit of the segment kernel).
+int64_t attn_seg_max_warps(const tq_ctx* c) { return (int64_t)c->sms * 3 * MW; }
+
+cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
+  AttnArgs a = a_in;
+  if (attn_seg_path(a)) {
+    if (!a.tiles) return cudaErrorInvalidValue;
+    // At least four tiles per warp, at most attn_seg_max_warps warps; the
+    // kernel trims the warp count to the real tile count.
+    const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
+    int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
+    blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
+    a.nw = (int)(blocks * MW);
+    switch (a.G) {
+      case 1: k_attn_seg<1><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      case 2: k_attn_seg<2><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      default: k_attn_seg<4><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+    }
+  } else if (a.G == 8) {
+    a.tiles = nullptr;
+    dim3 grid(a.splits, a.Hkv, a.B);
+    k_attn_mma<8><<<grid, MW * 32, SMEM_BYTES, s>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
   }
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_merge(c, a, out, s);
 }
@@ -832,9 +864,9 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cuda
 cudaError_t configure_attn_mma() {
   const int b = (int)SMEM_BYTES;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_attn_g4<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_g4<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_g4<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
   return cudaFuncSetAttribute(k_attn_mma<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
 }
 

@@ -98,7 +98,12 @@ struct AttnArgs {
   const float* cv;
   int splits;
   int chunk;         // tokens per split
-  float* part;       // [B*Hq][splits][dpad+2]
+  float* part;       // [B*Hq][splits][dpad+2], or [slots][G][dpad+2] on the segment path
+  // Segment path (tensor-core decode, group <= 4): 16-token tile prefix over
+  // sequences, tiles[b] = Hkv * sum_{b' < b} ceil(len_b' / 16), written by the
+  // pre-rotation kernel; null on the split path.  nw = warps of the launch.
+  int64_t* tiles;
+  int nw;
 };
 
 struct QuantTcArgs {
@@ -130,13 +135,19 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
 cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s);
 cudaError_t configure_quant_tc();
 cudaError_t read_and_clear_fault(int* value);
-cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
+// With plan != null the kernel also writes plan->tiles (the segment path's
+// tile prefix) from plan->seq_lens, B, Hkv and max_T.
+cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
                              float* qr, float* qs, cudaStream_t s);
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 // Tensor-core decode path (d = 128, k3 with m = 128, v4, group <= 8).
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
 int attn_mma_chunk();
+// Segment path: taken for group sizes 1, 2 and 4 of the tensor-core decode.
+bool attn_seg_path(const AttnArgs& a);
+// Upper bound on the warps of a segment-path launch (sizes the partials).
+int64_t attn_seg_max_warps(const tq_ctx* c);
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,

@@ -306,9 +306,44 @@ __global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
 // ----------------------------------------------------------------------------
 // Query pre-rotation: q' = Pi q, s = S q' (one block per query row).
 // ----------------------------------------------------------------------------
+// Tile prefix of the segment-partitioned decode: tiles[b] = Hkv * sum over
+// b' < b of ceil(len_b' / 16), len = min(max(seq_lens, 0), max_T); one block.
+__device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T, int64_t* tiles) {
+  __shared__ int64_t s_w[4];
+  __shared__ int64_t s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    s_carry = 0;
+    tiles[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < B; base += 128) {
+    const int b = base + tid;
+    int64_t v = 0;
+    if (b < B) {
+      const int64_t len = min((int64_t)max(seq_lens[b], 0), max_T);
+      v = (len + 15) / 16 * Hkv;
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += n;
+    }
+    if (lane == 31) s_w[warp] = v;
+    __syncthreads();
+    int64_t off = s_carry;
+    for (int w = 0; w < warp; ++w) off += s_w[w];
+    if (b < B) tiles[b + 1] = off + v;
+    __syncthreads();
+    if (tid == 127) s_carry = off + v;
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(128) k_prerotate(const void* q, int dtype, int d, int dpad,
                                                    int m, const float* PiT, const float* ST,
-                                                   float* qr, float* qs) {
+                                                   float* qr, float* qs, const int32_t* seq_lens,
+                                                   int B, int Hkv, int64_t max_T, int64_t* tiles) {
   extern __shared__ float sh[];
   float* sq = sh;          // [dpad]
   float* sr = sh + dpad;   // [dpad]
@@ -341,6 +376,7 @@ __global__ void __launch_bounds__(128) k_prerotate(const void* q, int dtype, int
     }
     qs[row * dpad + i] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
   }
+  if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
 }
 
 // ----------------------------------------------------------------------------
@@ -518,8 +554,15 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
 // The split maxima and sums are staged in shared memory with one load per
 // thread; each thread then folds its coordinate over the splits with
 // independent loads (eight in flight).
+//
+// Split path: row r's partials are part[r][0..splits).  Segment path (tiles
+// != null): the partials of row (b, h) sit in slots f + b Hkv + kv head ..
+// l + b Hkv + kv head, [slot][G][dpad + 2], where f and l are the first and
+// last warps whose tile ranges [w W / N, (w + 1) W / N) meet the row's tiles.
 __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int splits, int d, int dpad,
-                                                    const float* Pi, float* out) {
+                                                    const float* Pi, float* out,
+                                                    const int64_t* tiles, int B, int Hq, int Hkv,
+                                                    int nw) {
   extern __shared__ float sh[];
   float* so = sh;                 // [dpad]
   float* sw = sh + dpad;          // [splits] weights exp2(m_s - M)
@@ -528,9 +571,25 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int split
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* pr = part + row * splits * (dpad + 2);
+  int64_t sstride = dpad + 2;
+  if (tiles) {
+    const int b = (int)(row / Hq), h = (int)(row % Hq), G = Hq / Hkv;
+    const int kvh = h / G, hg = h % G;
+    const int64_t W = tiles[B];
+    const int64_t tb = (tiles[b + 1] - tiles[b]) / Hkv;
+    splits = 0;
+    if (tb > 0) {
+      const int64_t N = min((int64_t)nw, W);
+      const int64_t S = tiles[b] + kvh * tb, E = S + tb;
+      const int64_t f = ((S + 1) * N + W - 1) / W - 1, l = (E * N + W - 1) / W - 1;
+      pr = part + ((f + (int64_t)b * Hkv + kvh) * G + hg) * (dpad + 2);
+      sstride = (int64_t)G * (dpad + 2);
+      splits = (int)(l - f + 1);
+    }
+  }
   float mloc = -INFINITY;
   for (int sidx = tid; sidx < splits; sidx += blockDim.x) {
-    const float ms = pr[(int64_t)sidx * (dpad + 2)];
+    const float ms = pr[(int64_t)sidx * sstride];
     sw[sidx] = ms;
     mloc = fmaxf(mloc, ms);
   }
@@ -545,7 +604,7 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int split
     const float ms = sw[sidx];
     const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
     sw[sidx] = w;
-    lloc = fmaf(w, pr[(int64_t)sidx * (dpad + 2) + 1], lloc);
+    lloc = fmaf(w, pr[(int64_t)sidx * sstride + 1], lloc);
   }
   lloc = warp_sum(lloc);
   __syncthreads();
@@ -560,9 +619,9 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int split
     for (; sidx + 8 <= splits; sidx += 8) {
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        acc[u] = fmaf(sw[sidx + u], pr[(int64_t)(sidx + u) * (dpad + 2) + 2 + j], acc[u]);
+        acc[u] = fmaf(sw[sidx + u], pr[(int64_t)(sidx + u) * sstride + 2 + j], acc[u]);
     }
-    for (; sidx < splits; ++sidx) acc[0] = fmaf(sw[sidx], pr[(int64_t)sidx * (dpad + 2) + 2 + j], acc[0]);
+    for (; sidx < splits; ++sidx) acc[0] = fmaf(sw[sidx], pr[(int64_t)sidx * sstride + 2 + j], acc[0]);
     const float tot = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     so[j] = (L > 0.f) ? tot / L : 0.f;
   }
@@ -914,11 +973,12 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
   return cudaGetLastError();
 }
 
-cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows,
+cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
                              float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
   k_prerotate<<<(unsigned)rows, 128, 2 * c->dpad * sizeof(float), s>>>(
-      q, dtype, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs);
+      q, dtype, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, plan ? plan->seq_lens : nullptr,
+      plan ? plan->B : 0, plan ? plan->Hkv : 1, plan ? plan->max_T : 0, plan ? plan->tiles : nullptr);
   return cudaGetLastError();
 }
 
@@ -938,8 +998,9 @@ int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
 }
 
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
-  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, (c->dpad + a.splits) * sizeof(float), s>>>(
-      a.part, a.splits, c->d, c->dpad, c->Pi_f, out);
+  const int slots = a.tiles ? a.nw : a.splits;
+  k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, (c->dpad + slots) * sizeof(float), s>>>(
+      a.part, a.splits, c->d, c->dpad, c->Pi_f, out, a.tiles, a.B, a.Hq, a.Hkv, a.nw);
   return cudaGetLastError();
 }
 
@@ -1001,7 +1062,7 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   float* qs = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
   float* cv = reinterpret_cast<float*>(take((size_t)nq * nch * k * sizeof(float)));
   int* ci = reinterpret_cast<int*>(take((size_t)nq * nch * k * sizeof(int)));
-  cudaError_t e = launch_prerotate(c, q, dtype, nq, qr, qs, s);
+  cudaError_t e = launch_prerotate(c, q, dtype, nq, nullptr, qr, qs, s);
   if (e != cudaSuccess) return e;
   const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
   const size_t shm = (size_t)(2 * c->dpad * TQ + TQ * TTH + TQ * TKMAX) * sizeof(float) +
