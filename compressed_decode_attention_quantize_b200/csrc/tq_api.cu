@@ -420,22 +420,21 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
 
 // Workspace: [q' and S q' rows][tile prefix][partials].  The partials are
 // sized for the larger of the split layout ([B Hq][splits][dpad + 2]) and
-// the segment layout ([warps + B Hkv][G][dpad + 2] <= [4 warps + B Hq][...]).
+// the segment layouts: [warps + B Hkv][G][dpad + 2] for groups up to 4, and
+// [4 (CTAs + B Hkv)][8][dpad + 2] for group 8; both are at most
+// [8 warps + 4 B Hq][dpad + 2].
 namespace {
 struct AttnWs {
   size_t q_bytes, tiles_off, part_off, total;
 };
 AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   int chunk = 0;
-  int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
-  // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most
-  // splits), and for the tensor-core path's fixed chunk.
-  const int64_t mma_splits = (max_T + tqk::attn_mma_chunk() - 1) / tqk::attn_mma_chunk();
-  if (mma_splits > splits) splits = (int)mma_splits;
+  // Split count depends on Hkv; size for the largest (Hkv = 1 gives the most).
+  const int splits = tqk::attn_splits(c, B, 1, max_T > 0 ? max_T : 1, &chunk);
   const size_t rows = (size_t)B * Hq;
   const size_t row_bytes = (size_t)(c->dpad + 2) * sizeof(float);
   const size_t split_part = rows * (size_t)splits * row_bytes;
-  const size_t seg_part = ((size_t)tqk::attn_seg_max_warps(c) * 4 + rows) * row_bytes;
+  const size_t seg_part = ((size_t)tqk::attn_seg_max_warps(c) * 8 + 4 * rows) * row_bytes;
   AttnWs w;
   w.q_bytes = 2 * rows * c->dpad * sizeof(float);
   w.tiles_off = (w.q_bytes + 255) & ~(size_t)255;
@@ -506,12 +505,8 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.part = part;
   a.tiles = nullptr;
   const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
-  if (mma && tqk::attn_seg_path(a)) {
+  if (mma) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
-  } else if (mma) {
-    a.chunk = tqk::attn_mma_chunk();
-    a.splits = (int)((max_T + a.chunk - 1) / a.chunk);
-    if (a.splits > 4096) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: context too long (max 2M tokens)");
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
   }

@@ -1,35 +1,27 @@
-// Split-K decode attention from packed codes on the tensor cores (sm_100a).
+// Decode attention from packed codes on the tensor cores (sm_100a).
 //
-// Computes, for every query head h of a KV group g of sequence b, the
-// partial softmax state over one chunk of the context ("What is TurboQuant?",
-// "How TurboQuant works", closing paragraph: the logits come straight from
-// the compressed indices; "How to implement" part 1: the query is rotated
-// once and dotted with centroid values):
+// Computes, for every query head h of a KV group of sequence b, the softmax
+// state over a piece of the context ("What is TurboQuant?", "How TurboQuant
+// works", closing paragraph: the logits come straight from the compressed
+// indices; "How to implement" part 1: the query is rotated once and dotted
+// with centroid values):
 //   l_i  = |k_i| <q', c_k[idx_i]> + sqrt(pi/2)/m * gamma_i <S q', sigma_i>
 //   s_i  = scale * l_i,   m = max s,   l = sum exp(s - m),
 //   o    = sum exp(s_i - m) |v_i| c_v[vidx_i]          (rotated domain)
-// The merge kernel combines chunks by log-sum-exp and applies Pi^T once.
+// The merge kernel combines the pieces by log-sum-exp and applies Pi^T once.
 //
 // Fast path: d = 128, keys 2 Lloyd-Max bits + 128 QJL rows, values 4 bits,
-// GQA group size G <= 8.  One CTA = 4 warps over one chunk of tokens of one
-// (sequence, kv head); each warp walks 16-token tiles with its own online
-// softmax and its own cp.async pipeline (4 stages), and the 4 warps merge at
-// the end.  Per tile:
-//  * logits: mma.sync m16n8k16, A = dequantized keys (16 tokens x 16 dims,
-//    fp16), B = pre-rotated query (16 dims x 8 heads, fp16), fp32 accumulate.
-//    2-bit codes become fp16 centroids with one byte-permute per two values
-//    (a 4-entry table in two registers).  QJL bits become +-1 fp16 with one
-//    shift and one logic op per two values; a second accumulator collects
-//    <S q', sigma>.  fp16 alone would round q', S q' and the centroids to 11
-//    bits, which moves the softmax exponent by ~1e-3 for keys with large
-//    norms; each of them is therefore split into an fp16 head and an fp16
-//    tail scaled by 2^12 (c = c_hi + 2^-12 c_lo, likewise q' and S q'), and
-//    the tail products (hi*lo and lo*hi) go to a correction accumulator that
-//    is added in fp32 with weight 2^-12 (error ~2^-22 relative).
+// GQA group size 1, 2, 4 or 8.  Work is split into balanced contiguous ranges
+// of 16-token tiles over all (sequence, kv head) rows; a warp walks its tiles
+// with its own cp.async ring and online softmax.  Per tile:
+//  * logits: mma.sync m16n8k16, A = key code bits as exact fp16 powers of two
+//    (16 tokens x 16 bit-planes), B = pre-rotated query (fp16 head and tail
+//    per head), fp32 accumulate; the centroid values enter through an affine
+//    identity in fp32.  A second product takes the QJL sign bits against S q'.
 //  * the 16x8 probability tile is transposed into the B operand of the value
 //    product with movmatrix.
 //  * values: mma.sync m16n8k16, A = dequantized values (16 dims x 16 tokens),
-//    B = p * |v| (16 tokens x 8 heads).  A 4-bit code pair (two tokens, one
+//    B = p * |v| (16 tokens x 8 columns).  A 4-bit code pair (two tokens, one
 //    dim) indexes a 256-entry half2 table in shared memory, one copy per
 //    lane so that every lookup of a warp hits 32 different banks.
 // The head dimension is permuted inside the tiles (a thread owns contiguous
@@ -70,7 +62,7 @@ constexpr size_t SMEM_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST * sizeof(
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -79,7 +71,7 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ uint32_t movtrans(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
   return y;
 }
 
@@ -102,337 +94,10 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-// QJL bit pair (e, e+16) of w as a half2 of +-1 (bit 1 -> +1).
-__device__ __forceinline__ uint32_t sign_pair(uint32_t w, int e) {
-  return ((w << (15 - e)) & 0x80008000u) ^ 0xBC00BC00u;
-}
-
-struct TileSrc {
-  const uint32_t* k;   // key codes of token 0 of the (b, g) row
-  const uint32_t* q;
-  const float* kn;
-  const float* kr;
-  const uint32_t* v;
-  const float* vn;
-};
-
-// Issue the cp.async copies of tile tokens [t0, t0+16) into stage st.
-__device__ __forceinline__ void load_tile(const TileSrc& src, Stage* st, int64_t t0, int64_t t_end,
-                                          int lane) {
-  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(st);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = lane + 32 * i;
-    if (c < 32) {                              // key codes: 16 tokens x 2 chunks
-      const int tok = c >> 1, part = c & 1;
-      const int64_t t = t0 + tok;
-      cp16(sbase + offsetof(Stage, k) + tok * 32 + part * 16, src.k + t * KW + part * 4, t < t_end);
-    } else if (c < 48) {                       // QJL: 16 tokens x 1 chunk
-      const int tok = c - 32;
-      const int64_t t = t0 + tok;
-      cp16(sbase + offsetof(Stage, q) + tok * 16, src.q + t * QW, t < t_end);
-    } else if (c < 60) {                       // norms: 3 arrays x 4 chunks of 4 tokens
-      const int which = (c - 48) >> 2, part = (c - 48) & 3;
-      const int64_t t = t0 + 4 * part;
-      const float* base = which == 0 ? src.kn : which == 1 ? src.kr : src.vn;
-      const uint32_t off = which == 0 ? offsetof(Stage, kn) : which == 1 ? offsetof(Stage, kr)
-                                                                           : offsetof(Stage, vn);
-      cp16(sbase + off + part * 16, base + t, t < t_end);
-    } else if (c < 124) {                      // value codes: 16 tokens x 4 chunks
-      const int cc = c - 60;
-      const int tok = cc >> 2, part = cc & 3;
-      const int64_t t = t0 + tok;
-      cp16(sbase + offsetof(Stage, v) + tok * (VROW * 4) + part * 16, src.v + t * VW + part * 4,
-           t < t_end);
-    }
-  }
-}
-
-template <int G>
-__global__ void __launch_bounds__(MW * 32, 2) k_attn_mma(AttnArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
-
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-
-  // Value table: entry (byte, lane) = half2(cv[byte & 15], cv[byte >> 4]).
-  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
-    const int byte = e >> 5;
-    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
-  }
-  // Key centroid tables (4 fp16 heads, 4 scaled fp16 tails) for the
-  // byte-permute dequantizer.
-  float ch[4], cl[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    ch[i] = __half2float(__float2half_rn(a.ck[i]));
-    cl[i] = (a.ck[i] - ch[i]) * 4096.f;
-  }
-  const uint32_t T0 = pack_half2(ch[0], ch[1]), T1 = pack_half2(ch[2], ch[3]);
-  const uint32_t L0 = pack_half2(cl[0], cl[1]), L1 = pack_half2(cl[2], cl[3]);
-
-  // B fragments of the pre-rotated query q' and of s = S q' for head g.
-  const int hq = kvh * G + g;
-  const bool head_ok = g < G;
-  const float* qrow = a.qr + ((int64_t)b * a.Hq + (head_ok ? hq : kvh * G)) * 128;
-  const float* srow = a.qs + ((int64_t)b * a.Hq + (head_ok ? hq : kvh * G)) * 128;
-  float qv[32], sv[32];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 x = reinterpret_cast<const float4*>(qrow + 32 * t)[i];
-    const float4 y = reinterpret_cast<const float4*>(srow + 32 * t)[i];
-    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
-    sv[4 * i] = y.x; sv[4 * i + 1] = y.y; sv[4 * i + 2] = y.z; sv[4 * i + 3] = y.w;
-  }
-  float mq = 0.f, ms = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    mq = fmaxf(mq, fabsf(qv[i]));
-    ms = fmaxf(ms, fabsf(sv[i]));
-  }
-  mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
-  mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 2));
-  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 1));
-  ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, 2));
-  // Power-of-two scales keep the fp16 operands in range without extra rounding.
-  const int eq = mq > 0.f ? ilogbf(mq) : 0;
-  const int es = ms > 0.f ? ilogbf(ms) : 0;
-  const float sq_ = head_ok ? ldexpf(1.f, -eq) : 0.f;
-  const float ss_ = head_ok ? ldexpf(1.f, -es) : 0.f;
-  uint32_t bq[8][2], bql[8][2], bs[8][2], bsl[8][2];
-  auto split2 = [](float x, float y, uint32_t& hi, uint32_t& lo) {
-    const __half2 h = __floats2half2_rn(x, y);
-    const float2 f = __half22float2(h);
-    hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = pack_half2((x - f.x) * 4096.f, (y - f.y) * 4096.f);
-  };
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    const int base = 16 * (s >> 2) + (s & 3);   // local dims of k-step s
-    split2(qv[base] * sq_, qv[base + 4] * sq_, bq[s][0], bql[s][0]);
-    split2(qv[base + 8] * sq_, qv[base + 12] * sq_, bq[s][1], bql[s][1]);
-    split2(sv[2 * s] * ss_, sv[2 * s + 16] * ss_, bs[s][0], bsl[s][0]);
-    split2(sv[2 * s + 1] * ss_, sv[2 * s + 17] * ss_, bs[s][1], bsl[s][1]);
-  }
-  // Logit scales for the C-fragment columns (heads 2t, 2t+1).
-  float cqs[2], css[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int eqj = __shfl_sync(0xffffffffu, eq, (2 * t + j) * 4);
-    const int esj = __shfl_sync(0xffffffffu, es, (2 * t + j) * 4);
-    cqs[j] = ldexpf(a.scale_log2, eqj);
-    css[j] = ldexpf(a.scale_log2 * a.cq, esj);
-  }
-
-  const int64_t T = min((int64_t)a.seq_lens[b], a.max_T);
-  const int64_t c_begin = (int64_t)split * a.chunk;
-  const int64_t c_end = min(T, c_begin + a.chunk);
-  const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
-  TileSrc src{a.kcodes + row0 * KW, a.kqjl + row0 * QW, a.knorm + row0, a.krnorm + row0,
-              a.vcodes + row0 * VW, a.vnorm + row0};
-
-  Stage* my = stages + warp * NST;
-  // Tiles of this warp: c_begin + 16 * (warp + MW * i).
-  const int64_t ntiles_cta = c_end > c_begin ? (c_end - c_begin + MT - 1) / MT : 0;
-  const int nt = ntiles_cta > warp ? (int)((ntiles_cta - warp + MW - 1) / MW) : 0;
-
-#pragma unroll
-  for (int i = 0; i < NST - 1; ++i) {
-    if (i < nt) load_tile(src, my + i, c_begin + (int64_t)MT * (warp + MW * i), c_end, lane);
-    cp_commit();
-  }
-  __syncthreads();  // value table ready
-
-  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_part[2] = {0.f, 0.f};
-  int kv_run = -1000;
-  float o[8][4];
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-  for (int i = 0; i < nt; ++i) {
-    {
-      const int ip = i + NST - 1;
-      if (ip < nt) load_tile(src, my + (ip % NST), c_begin + (int64_t)MT * (warp + MW * ip), c_end, lane);
-      cp_commit();
-    }
-    cp_wait<NST - 1>();
-    __syncwarp();
-    const Stage& st = my[i % NST];
-    const int64_t t0 = c_begin + (int64_t)MT * (warp + MW * i);
-
-    // ---- logits ----------------------------------------------------------
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
-    float acc_t[4] = {0.f, 0.f, 0.f, 0.f}, acs_t[4] = {0.f, 0.f, 0.f, 0.f};  // tails
-    const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
-    const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int sh = 2 * (s & 3);
-      const uint32_t x0 = (s < 4) ? kg0.x : kg0.y;
-      const uint32_t x8 = (s < 4) ? kg8.x : kg8.y;
-      const uint32_t y0 = ((x0 >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
-      const uint32_t y8 = ((x8 >> sh) & 0x03030303u) * 0x22u + 0x10101010u;
-      const uint32_t a0 = __byte_perm(T0, T1, y0);
-      const uint32_t a2 = __byte_perm(T0, T1, y0 >> 16);
-      const uint32_t a1 = __byte_perm(T0, T1, y8);
-      const uint32_t a3 = __byte_perm(T0, T1, y8 >> 16);
-      mma16816(acc, a0, a1, a2, a3, bq[s][0], bq[s][1]);
-      mma16816(acc_t, a0, a1, a2, a3, bql[s][0], bql[s][1]);
-      mma16816(acc_t, __byte_perm(L0, L1, y0), __byte_perm(L0, L1, y8), __byte_perm(L0, L1, y0 >> 16),
-               __byte_perm(L0, L1, y8 >> 16), bq[s][0], bq[s][1]);
-    }
-    const uint32_t qg0 = st.q[g][t], qg8 = st.q[g + 8][t];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t a0 = sign_pair(qg0, 2 * s), a1 = sign_pair(qg8, 2 * s);
-      const uint32_t a2 = sign_pair(qg0, 2 * s + 1), a3 = sign_pair(qg8, 2 * s + 1);
-      mma16816(acs, a0, a1, a2, a3, bs[s][0], bs[s][1]);
-      mma16816(acs_t, a0, a1, a2, a3, bsl[s][0], bsl[s][1]);
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      acc[r] = fmaf(acc_t[r], 1.f / 4096.f, acc[r]);
-      acs[r] = fmaf(acs_t[r], 1.f / 4096.f, acs[r]);
-    }
-    const bool v0 = t0 + g < c_end, v8 = t0 + g + 8 < c_end;
-    const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
-    float sc[4];
-    sc[0] = v0 ? fmaf(kr0 * css[0], acs[0], kn0 * cqs[0] * acc[0]) : -INFINITY;
-    sc[1] = v0 ? fmaf(kr0 * css[1], acs[1], kn0 * cqs[1] * acc[1]) : -INFINITY;
-    sc[2] = v8 ? fmaf(kr8 * css[0], acs[2], kn8 * cqs[0] * acc[2]) : -INFINITY;
-    sc[3] = v8 ? fmaf(kr8 * css[1], acs[3], kn8 * cqs[1] * acc[3]) : -INFINITY;
-
-    // ---- online softmax (heads 2t, 2t+1) ------------------------------------
-    float tmax[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 4));
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 8));
-      tmax[j] = fmaxf(tmax[j], __shfl_xor_sync(0xffffffffu, tmax[j], 16));
-    }
-    // Value-norm scale: p * |v| * 2^-kv stays below 2^15 in fp16.
-    const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
-    float vmax = fmaxf(vn0, vn8);
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
-    const int kv_tile = vmax > 0.f ? ilogbf(vmax) - 14 : -1000;
-    const int kv_new = max(kv_run, kv_tile);
-    const float vscale_change = exp2f((float)(kv_run - kv_new));
-    kv_run = kv_new;
-    const float vmul = ldexpf(1.f, -kv_new);
-    float alpha[2], mnew[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      mnew[j] = fmaxf(m_run[j], tmax[j]);
-      alpha[j] = (mnew[j] == -INFINITY) ? 1.f : exp2f(m_run[j] - mnew[j]);
-      m_run[j] = mnew[j];
-    }
-    float p[4];
-    p[0] = (mnew[0] == -INFINITY) ? 0.f : exp2f(sc[0] - mnew[0]);
-    p[1] = (mnew[1] == -INFINITY) ? 0.f : exp2f(sc[1] - mnew[1]);
-    p[2] = (mnew[0] == -INFINITY) ? 0.f : exp2f(sc[2] - mnew[0]);
-    p[3] = (mnew[1] == -INFINITY) ? 0.f : exp2f(sc[3] - mnew[1]);
-    l_part[0] = fmaf(l_part[0], alpha[0], p[0] + p[2]);
-    l_part[1] = fmaf(l_part[1], alpha[1], p[1] + p[3]);
-    const float oa0 = alpha[0] * vscale_change, oa1 = alpha[1] * vscale_change;
-    if (__any_sync(0xffffffffu, oa0 != 1.f || oa1 != 1.f)) {
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        o[mt][0] *= oa0; o[mt][1] *= oa1; o[mt][2] *= oa0; o[mt][3] *= oa1;
-      }
-    }
-    const float w0 = vn0 * vmul, w8 = vn8 * vmul;
-    const uint32_t pb0 = movtrans(pack_half2(p[0] * w0, p[1] * w0));
-    const uint32_t pb1 = movtrans(pack_half2(p[2] * w8, p[3] * w8));
-
-    // ---- values ---------------------------------------------------------------
-    const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
-    const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
-    const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
-    const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
-    // byte k of ye = (nibble 2k of the first token) | (nibble 2k of the second) << 4
-    const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
-                            (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
-                            (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
-                            (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
-    const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
-                            ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
-                            ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
-                            ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const int k = mt >> 1;
-      const uint32_t* y = (mt & 1) ? yo : ye;
-      uint32_t av[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint32_t off = (k == 0) ? ((y[r] << 7) & 0x7F80u) : ((y[r] >> (8 * k - 7)) & 0x7F80u);
-        av[r] = lds32(lut_lane + off);
-      }
-      // rows: word 2g -> dim row g (a0/a2), word 2g+1 -> row g+8 (a1/a3)
-      mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
-    }
-    __syncwarp();
-  }
-  cp_wait<0>();
-
-  // ---- merge the four warps of the CTA ---------------------------------------
-  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 4);
-  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 8);
-  l_part[0] += __shfl_xor_sync(0xffffffffu, l_part[0], 16);
-  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 4);
-  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 8);
-  l_part[1] += __shfl_xor_sync(0xffffffffu, l_part[1], 16);
-  __syncthreads();  // stages are reused as merge scratch below
-  float* sm = reinterpret_cast<float*>(stages);   // [MW][8][130]
-  const float vback = ldexpf(1.f, kv_run);
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int h = 2 * t + j;
-    float* row = sm + (warp * 8 + h) * 130;
-    if (g == 0) {
-      row[0] = m_run[j];
-      row[1] = l_part[j];
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      row[2 + 16 * g + mt] = o[mt][j] * vback;
-      row[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * 130; e += MW * 32) {
-    const int h = e / 130, c = e % 130;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < MW; ++w) M = fmaxf(M, sm[(w * 8 + h) * 130]);
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < MW; ++w) {
-      const float mw_ = sm[(w * 8 + h) * 130];
-      if (mw_ != -INFINITY) acc = fmaf(exp2f(mw_ - M), sm[(w * 8 + h) * 130 + (c == 0 ? 1 : c)], acc);
-    }
-    const int64_t prow = (int64_t)b * a.Hq + (int64_t)kvh * G + h;
-    float* pp = a.part + (prow * a.splits + split) * (128 + 2);
-    if (c == 0) {
-      pp[0] = M;
-    } else {
-      pp[c] = acc;   // c == 1: l, c >= 2: o_rot[c - 2]
-    }
-  }
-}
-
-
 // ---------------------------------------------------------------------------
-// Group size <= 4.  Half of the MMA's eight columns would be idle, so columns
-// 4..7 carry the fp16 tails (x 2^12) of the query-side operands of columns
-// 0..3: one MMA yields head and tail products of every k-step.
+// Key operands.  A query head takes two B columns of the key MMA: the fp16
+// head of its operand and the fp16 tail (x 2^12), so one MMA yields both
+// products of every k-step and the fp32 sum restores ~22 bits.
 //
 // Keys use exact binary A operands.  A symmetric 2-bit codebook is affine in
 // the index bits, c[i0 + 2 i1] = c0 + (c1 - c0) i0 + (c2 - c0) i1, so
@@ -712,14 +377,16 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
       const int64_t t0 = tok0 + (int64_t)MT * i;
 
       // ---- logits -----------------------------------------------------------
+      // Two accumulators per product halve the dependent MMA chains.
       float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc2[4] = {0.f, 0.f, 0.f, 0.f}, acs2[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
         const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
         const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
         const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
 #define TQ_KSTEP(S)                                                                               \
-  mma16816(acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                                    \
+  mma16816(((S) & 1) ? acc2 : acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                 \
            bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81),                                         \
            bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01),                                     \
            bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S].x, bk[S].y);
@@ -729,11 +396,17 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
 #undef TQ_KSTEP
         const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
 #define TQ_QSTEP(S)                                                                               \
-  mma16816(acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8), bit_half2<2 * (S) + 1>(Q0),      \
+  mma16816(((S) & 1) ? acs2 : acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8),                \
+           bit_half2<2 * (S) + 1>(Q0),                                                             \
            bit_half2<2 * (S) + 1>(Q8), bj[S].x, bj[S].y);
         TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
         TQ_QSTEP(7)
 #undef TQ_QSTEP
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          acc[r] += acc2[r];
+          acs[r] += acs2[r];
+        }
       }
       // Columns 2t (head) and 2t+1 (tail) of head t; rows g and g+8 are tokens.
       const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
@@ -815,6 +488,361 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Group size 8.  Eight heads with fp16 head and tail columns need sixteen B
+// columns (two MMAs per k-step), and the query operands of all k-steps would
+// take 96 registers per thread; they live in shared memory instead, built once
+// per row piece by the whole CTA.  So the CTA, not the warp, owns a tile range
+// ([c W / N, (c + 1) W / N), N = min(CTAs, W)); tile i of a row piece goes to
+// warp i mod 4, and every warp writes its own partial per piece (an empty one,
+// m = -inf, if it had no tile), to slot 4 (c + b Hkv + kv head) + warp.
+//
+// Thread (g, t) owns heads t and 4 + t: the first MMA of a k-step carries
+// heads 0..3 (columns 2h, 2h+1 = fp16 head, tail), the second heads 4..7.
+// In the value product, column 2t of P carries head t and column 2t+1 head
+// 4 + t.
+// ---------------------------------------------------------------------------
+constexpr int NST8 = 3;                       // pipeline stages per warp
+constexpr int QOP_STEPS = 24;                 // 16 key k-steps + 8 QJL k-steps
+constexpr size_t SMEM8_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST8 * sizeof(Stage) +
+                               (size_t)QOP_STEPS * 32 * 16 + 8 * 16 + MW * 4 + 16 * 4;
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
+  constexpr int G = 8;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
+  Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
+  uint32_t* qop = reinterpret_cast<uint32_t*>(smem + (size_t)LUT_WORDS * 4 +
+                                              (size_t)MW * NST8 * sizeof(Stage));   // [24][32][4]
+  float4* s_head = reinterpret_cast<float4*>(qop + QOP_STEPS * 32 * 4);           // [8] KA, KB, QA, QB
+  float* s_vmax = reinterpret_cast<float*>(s_head + 8);                             // [MW]
+  int* s_scale = reinterpret_cast<int*>(s_vmax + MW);                               // [16] q', S q' exponents
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
+    const int byte = e >> 5;
+    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
+  }
+  __syncthreads();
+
+  const int64_t* P = a.tiles;
+  const int64_t W = P[a.B];
+  const int64_t NC = min((int64_t)gridDim.x, W);
+  const int64_t cta = blockIdx.x;
+  if (cta >= NC) return;   // uniform over the CTA
+  int64_t x = cta * W / NC;
+  const int64_t x1 = (cta + 1) * W / NC;
+  int b = 0;
+  {
+    int hi = a.B;
+    while (hi - b > 1) {
+      const int mid = (b + hi) >> 1;
+      if (P[mid] <= x) b = mid; else hi = mid;
+    }
+  }
+
+  const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
+  const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
+  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  const uint32_t qop_lane = (uint32_t)__cvta_generic_to_shared(qop) + lane * 16;
+  Stage* my = stages + warp * NST8;
+  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
+
+  while (x < x1) {
+    while (P[b + 1] <= x) ++b;
+    const int64_t tb = (P[b + 1] - P[b]) / a.Hkv;
+    const int64_t rel = x - P[b];
+    const int kvh = (int)(rel / tb);
+    const int64_t tt = rel - (int64_t)kvh * tb;
+    const int64_t te = min(tb, tt + (x1 - x));
+    const int nt = (int)(te - tt);
+    const int64_t slot = 4 * (cta + (int64_t)b * a.Hkv + kvh) + warp;
+    x += nt;
+
+    const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
+    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
+    const int64_t tok0 = tt * MT;
+    const int64_t tok1 = min(te * MT, len);
+    const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * G;
+
+    __syncthreads();   // the previous piece's readers of qop / s_head are done
+    // ---- per-head operand scales (warp w: heads 2w, 2w+1) and value-norm max ----
+#pragma unroll
+    for (int hsel = 0; hsel < 2; ++hsel) {
+      const int h = 2 * warp + hsel;
+      const float4 q4 = reinterpret_cast<const float4*>(a.qr + (qbase + h) * 128)[lane];
+      const float4 s4 = reinterpret_cast<const float4*>(a.qs + (qbase + h) * 128)[lane];
+      float mq = fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w)));
+      float ms = fmaxf(fmaxf(fabsf(s4.x), fabsf(s4.y)), fmaxf(fabsf(s4.z), fabsf(s4.w)));
+      float sq = (q4.x + q4.y) + (q4.z + q4.w), ss = (s4.x + s4.y) + (s4.z + s4.w);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+        ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      }
+      if (lane == 0) {
+        const int eq = mq > 0.f ? ilog2f(mq) : 0;
+        const int es = ms > 0.f ? ilog2f(ms) : 0;
+        s_scale[h] = eq;
+        s_scale[8 + h] = es;
+        s_head[h] = make_float4(pow2i(eq + ew + 1) * a.scale_log2, c0 * sq * a.scale_log2,
+                                2.f * pow2i(es) * a.cq * a.scale_log2, -ss * a.cq * a.scale_log2);
+      }
+    }
+    {
+      float vmax = 0.f;
+      const float* vr = a.vnorm + row0;
+      for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
+        if (j + 4 <= tok1) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
+        } else {
+          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      if (lane == 0) s_vmax[warp] = vmax;
+    }
+    __syncthreads();
+    // ---- query operands: warp w builds key k-steps 4w..4w+3, QJL k-steps 2w, 2w+1 ----
+    {
+      const int hcol = g >> 1;           // head within the MMA's group of four
+      const bool tail_col = (g & 1) != 0;
+      auto operand = [&](float lo, float hi) -> uint32_t {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        if (!tail_col) return *reinterpret_cast<const uint32_t*>(&h);
+        const float2 f = __half22float2(h);
+        return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
+      };
+#pragma unroll
+      for (int k = 0; k < 6; ++k) {
+        const bool key = k < 4;
+        const int s = key ? 4 * warp + k : 2 * warp + (k - 4);
+        uint32_t fr[4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int h = 4 * j + hcol;
+          const float* row = (key ? a.qr : a.qs) + (qbase + h) * 128 + 32 * t;
+          const float kq = key ? pow2i(-(s_scale[h] + ew + 1)) : pow2i(-s_scale[8 + h]);
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            const int u = key ? 2 * (s & 7) + sl : 2 * s + sl;
+            const int elo = 10 + u, ehi = (26 + u) & 31;
+            const float inv = bit_inv(bit_pos(u)) * kq;
+            float vlo, vhi;
+            if (key) {
+              vlo = row[16 * (s >> 3) + (elo >> 1)] * ((elo & 1) ? w1 : w0) * inv;
+              vhi = row[16 * (s >> 3) + (ehi >> 1)] * ((ehi & 1) ? w1 : w0) * inv;
+            } else {
+              vlo = row[elo] * inv;
+              vhi = row[ehi] * inv;
+            }
+            fr[2 * j + sl] = operand(vlo, vhi);
+          }
+        }
+        const int step = key ? s : 16 + s;
+        *reinterpret_cast<uint4*>(qop + (step * 32 + lane) * 4) = make_uint4(fr[0], fr[1], fr[2], fr[3]);
+      }
+    }
+    __syncthreads();
+    const float4 H0 = s_head[t], H1 = s_head[4 + t];
+    const float vmax = fmaxf(fmaxf(s_vmax[0], s_vmax[1]), fmaxf(s_vmax[2], s_vmax[3]));
+    const int kv = vmax >= FLT_MIN ? max(ilog2f(vmax) - 6, -120) : -120;
+    const float vmul = pow2i(-kv);
+
+    // ---- this warp's tiles: i = warp, warp + 4, ... of the piece ------------------
+    const int ntw = nt > warp ? (nt - warp + MW - 1) / MW : 0;
+    const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;
+    const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;
+    const char* p2 = p1 + 8 * 64;
+    const char* p3;
+    int stride3, tok3;
+    uint32_t d3;
+    if (lane < 16) {
+      p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
+      stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
+    } else if (lane < 28) {
+      const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
+      const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
+      p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
+      stride3 = 4; tok3 = 4 * part;
+      d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
+    } else {
+      p3 = nullptr; stride3 = 0; tok3 = 1 << 30; d3 = 0;
+    }
+    const uint32_t d0 = offsetof(Stage, k) + lane * 16;
+    const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
+    const uint32_t d2 = d1 + 8 * (VROW * 4);
+    auto issue = [&](int k, int stage) {
+      const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
+      const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
+      cp16(sb + d0, p0 + t0 * 32, t0 + (lane >> 1) < tok1);
+      cp16(sb + d1, p1 + t0 * 64, t0 + (lane >> 2) < tok1);
+      cp16(sb + d2, p2 + t0 * 64, t0 + 8 + (lane >> 2) < tok1);
+      if (lane < 28) cp16(sb + d3, p3 + t0 * stride3, t0 + tok3 < tok1);
+    };
+#pragma unroll
+    for (int k = 0; k < NST8 - 1; ++k) {
+      if (k < ntw) issue(k, k);
+      cp_commit();
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_part[2] = {0.f, 0.f};
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    for (int k = 0; k < ntw; ++k) {
+      if (k + NST8 - 1 < ntw) issue(k + NST8 - 1, (k + NST8 - 1) % NST8);
+      cp_commit();
+      cp_wait<NST8 - 1>();
+      __syncwarp();
+      const Stage& st = my[k % NST8];
+      const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
+
+      // ---- logits: acc[j] for heads 4j + t ----------------------------------------
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float acs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
+        const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
+        const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
+        const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
+#define TQ_KSTEP8(S)                                                                              \
+  {                                                                                               \
+    const uint4 bq = lds128(qop_lane + (S) * 512);                                                \
+    const uint32_t x0 = bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01);                            \
+    const uint32_t x1 = bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81);                            \
+    const uint32_t x2 = bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01);                        \
+    const uint32_t x3 = bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81);                        \
+    mma16816(acc[0], x0, x1, x2, x3, bq.x, bq.y);                                                 \
+    mma16816(acc[1], x0, x1, x2, x3, bq.z, bq.w);                                                 \
+  }
+        TQ_KSTEP8(0) TQ_KSTEP8(1) TQ_KSTEP8(2) TQ_KSTEP8(3) TQ_KSTEP8(4) TQ_KSTEP8(5)
+        TQ_KSTEP8(6) TQ_KSTEP8(7) TQ_KSTEP8(8) TQ_KSTEP8(9) TQ_KSTEP8(10) TQ_KSTEP8(11)
+        TQ_KSTEP8(12) TQ_KSTEP8(13) TQ_KSTEP8(14) TQ_KSTEP8(15)
+#undef TQ_KSTEP8
+        const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
+#define TQ_QSTEP8(S)                                                                              \
+  {                                                                                               \
+    const uint4 bq = lds128(qop_lane + (16 + (S)) * 512);                                         \
+    const uint32_t x0 = bit_half2<2 * (S)>(Q0), x1 = bit_half2<2 * (S)>(Q8);                      \
+    const uint32_t x2 = bit_half2<2 * (S) + 1>(Q0), x3 = bit_half2<2 * (S) + 1>(Q8);              \
+    mma16816(acs[0], x0, x1, x2, x3, bq.x, bq.y);                                                 \
+    mma16816(acs[1], x0, x1, x2, x3, bq.z, bq.w);                                                 \
+  }
+        TQ_QSTEP8(0) TQ_QSTEP8(1) TQ_QSTEP8(2) TQ_QSTEP8(3) TQ_QSTEP8(4) TQ_QSTEP8(5)
+        TQ_QSTEP8(6) TQ_QSTEP8(7)
+#undef TQ_QSTEP8
+      }
+      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
+      const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
+      float sc[2][2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float4 Hj = j ? H1 : H0;
+        const float lm0 = fmaf(acc[j][1], 1.f / 4096.f, acc[j][0]);
+        const float lm8 = fmaf(acc[j][3], 1.f / 4096.f, acc[j][2]);
+        const float qj0 = fmaf(acs[j][1], 1.f / 4096.f, acs[j][0]);
+        const float qj8 = fmaf(acs[j][3], 1.f / 4096.f, acs[j][2]);
+        sc[j][0] = v0 ? fmaf(kn0, fmaf(lm0, Hj.x, Hj.y), kr0 * fmaf(qj0, Hj.z, Hj.w)) : -INFINITY;
+        sc[j][1] = v8 ? fmaf(kn8, fmaf(lm8, Hj.x, Hj.y), kr8 * fmaf(qj8, Hj.z, Hj.w)) : -INFINITY;
+      }
+
+      // ---- online softmax, heads t and 4 + t ----------------------------------------
+      const float loc0 = fmaxf(sc[0][0], sc[0][1]), loc1 = fmaxf(sc[1][0], sc[1][1]);
+      if (__any_sync(0xffffffffu, loc0 > m_run[0] + LAZY_TAU || loc1 > m_run[1] + LAZY_TAU)) {
+        float tm0 = loc0, tm1 = loc1;
+#pragma unroll
+        for (int o_ = 4; o_ <= 16; o_ <<= 1) {
+          tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o_));
+          tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o_));
+        }
+        const float mn0 = fmaxf(m_run[0], tm0), mn1 = fmaxf(m_run[1], tm1);
+        const float al0 = ex2f(m_run[0] - mn0), al1 = ex2f(m_run[1] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        l_part[0] *= al0;
+        l_part[1] *= al1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= al0; o[mt][2] *= al0;
+          o[mt][1] *= al1; o[mt][3] *= al1;
+        }
+      }
+      const float p00 = ex2f(sc[0][0] - m_run[0]), p01 = ex2f(sc[0][1] - m_run[0]);
+      const float p10 = ex2f(sc[1][0] - m_run[1]), p11 = ex2f(sc[1][1] - m_run[1]);
+      l_part[0] += p00 + p01;
+      l_part[1] += p10 + p11;
+      const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
+      const uint32_t pb0 = movtrans(pack_half2(p00 * w0s, p10 * w0s));
+      const uint32_t pb1 = movtrans(pack_half2(p01 * w8s, p11 * w8s));
+
+      // ---- values ---------------------------------------------------------------
+      const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
+      const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
+      const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
+      const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
+      const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
+                              (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
+                              (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
+                              (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
+      const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
+                              ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
+                              ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
+                              ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const int kk = mt >> 1;
+        const uint32_t* y = (mt & 1) ? yo : ye;
+        uint32_t av[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + kk) * 128u + lut_lane);
+        mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+      }
+      __syncwarp();
+    }
+    cp_wait<0>();
+    __syncwarp();
+
+    // ---- this warp's partial of the piece (heads t and 4 + t) --------------------------
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 4);
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 8);
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 16);
+    }
+    const float vback = pow2i(kv);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float* pp = a.part + (slot * G + 4 * j + t) * (128 + 2);
+      if (g == 0) {
+        pp[0] = m_run[j];
+        pp[1] = l_part[j];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        pp[2 + 16 * g + mt] = o[mt][j] * vback;
+        pp[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
@@ -827,16 +855,12 @@ bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
   return (al & 15) == 0;
 }
 
-int attn_mma_chunk() { return 512; }
-
-bool attn_seg_path(const AttnArgs& a) { return a.G == 1 || a.G == 2 || a.G == 4; }
-
 // Three 4-warp CTAs per SM (the register limit of the segment kernel).
 int64_t attn_seg_max_warps(const tq_ctx* c) { return (int64_t)c->sms * 3 * MW; }
 
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
   AttnArgs a = a_in;
-  if (attn_seg_path(a)) {
+  if (a.G == 1 || a.G == 2 || a.G == 4) {
     if (!a.tiles) return cudaErrorInvalidValue;
     // At least four tiles per warp, at most attn_seg_max_warps warps; the
     // kernel trims the warp count to the real tile count.
@@ -844,15 +868,21 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, c
     int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
     blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
     a.nw = (int)(blocks * MW);
+    a.wpu = 1;
     switch (a.G) {
       case 1: k_attn_seg<1><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
       case 2: k_attn_seg<2><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
       default: k_attn_seg<4><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
     }
   } else if (a.G == 8) {
-    a.tiles = nullptr;
-    dim3 grid(a.splits, a.Hkv, a.B);
-    k_attn_mma<8><<<grid, MW * 32, SMEM_BYTES, s>>>(a);
+    if (!a.tiles) return cudaErrorInvalidValue;
+    // CTA-owned ranges of at least four tiles per warp.
+    const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
+    int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
+    blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
+    a.nw = (int)blocks;
+    a.wpu = MW;
+    k_attn_seg8<<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
   } else {
     return cudaErrorInvalidValue;
   }
@@ -867,7 +897,7 @@ cudaError_t configure_attn_mma() {
   if ((e = cudaFuncSetAttribute(k_attn_seg<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
   if ((e = cudaFuncSetAttribute(k_attn_seg<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
   if ((e = cudaFuncSetAttribute(k_attn_seg<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  return cudaFuncSetAttribute(k_attn_mma<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+  return cudaFuncSetAttribute(k_attn_seg8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8_BYTES);
 }
 
 }  // namespace tqk

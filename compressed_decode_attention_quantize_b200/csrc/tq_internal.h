@@ -101,9 +101,11 @@ struct AttnArgs {
   float* part;       // [B*Hq][splits][dpad+2], or [slots][G][dpad+2] on the segment path
   // Segment path (tensor-core decode, group <= 4): 16-token tile prefix over
   // sequences, tiles[b] = Hkv * sum_{b' < b} ceil(len_b' / 16), written by the
-  // pre-rotation kernel; null on the split path.  nw = warps of the launch.
+  // pre-rotation kernel; null on the split path.  nw = owners of tile ranges
+  // (warps, or CTAs for group 8), wpu = partial writers per owner.
   int64_t* tiles;
   int nw;
+  int wpu;
 };
 
 struct QuantTcArgs {
@@ -141,11 +143,9 @@ cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t 
                              float* qr, float* qs, cudaStream_t s);
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
-// Tensor-core decode path (d = 128, k3 with m = 128, v4, group <= 8).
+// Tensor-core decode path (d = 128, k3 with m = 128, v4, group 1, 2, 4 or 8);
+// it needs AttnArgs::tiles (the tile prefix) set.
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
-int attn_mma_chunk();
-// Segment path: taken for group sizes 1, 2 and 4 of the tensor-core decode.
-bool attn_seg_path(const AttnArgs& a);
 // Upper bound on the warps of a segment-path launch (sizes the partials).
 int64_t attn_seg_max_warps(const tq_ctx* c);
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);

@@ -556,13 +556,15 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
 // independent loads (eight in flight).
 //
 // Split path: row r's partials are part[r][0..splits).  Segment path (tiles
-// != null): the partials of row (b, h) sit in slots f + b Hkv + kv head ..
-// l + b Hkv + kv head, [slot][G][dpad + 2], where f and l are the first and
-// last warps whose tile ranges [w W / N, (w + 1) W / N) meet the row's tiles.
+// != null): the tiles are split into ranges [w W / N, (w + 1) W / N) over
+// N = min(nw, W) owners, each with wpu partial writers; the partials of row
+// (b, h) sit in slots wpu (f + i) .. wpu (l + i) + wpu - 1, i = b Hkv + kv
+// head, laid out [slot][G][dpad + 2], where f and l are the first and last
+// owners whose ranges meet the row's tiles.
 __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int splits, int d, int dpad,
                                                     const float* Pi, float* out,
                                                     const int64_t* tiles, int B, int Hq, int Hkv,
-                                                    int nw) {
+                                                    int nw, int wpu) {
   extern __shared__ float sh[];
   float* so = sh;                 // [dpad]
   float* sw = sh + dpad;          // [splits] weights exp2(m_s - M)
@@ -582,9 +584,9 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int split
       const int64_t N = min((int64_t)nw, W);
       const int64_t S = tiles[b] + kvh * tb, E = S + tb;
       const int64_t f = ((S + 1) * N + W - 1) / W - 1, l = (E * N + W - 1) / W - 1;
-      pr = part + ((f + (int64_t)b * Hkv + kvh) * G + hg) * (dpad + 2);
+      pr = part + (wpu * (f + (int64_t)b * Hkv + kvh) * G + hg) * (dpad + 2);
       sstride = (int64_t)G * (dpad + 2);
-      splits = (int)(l - f + 1);
+      splits = (int)(wpu * (l - f + 1));
     }
   }
   float mloc = -INFINITY;
@@ -998,9 +1000,9 @@ int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
 }
 
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
-  const int slots = a.tiles ? a.nw : a.splits;
+  const int slots = a.tiles ? a.nw * a.wpu : a.splits;
   k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, (c->dpad + slots) * sizeof(float), s>>>(
-      a.part, a.splits, c->d, c->dpad, c->Pi_f, out, a.tiles, a.B, a.Hq, a.Hkv, a.nw);
+      a.part, a.splits, c->d, c->dpad, c->Pi_f, out, a.tiles, a.B, a.Hq, a.Hkv, a.nw, a.wpu);
   return cudaGetLastError();
 }
 

@@ -159,7 +159,7 @@ def test_attention_single_head(cuda):
 
 
 @pytest.mark.parametrize("d,Hq,Hkv,bk,bv,m,T", [
-    (128, 8, 2, 3, 4, 128, 1100),   # tensor-core path, group 4, 3 chunks
+    (128, 8, 2, 3, 4, 128, 1100),   # tensor-core path, group 4
     (128, 4, 4, 3, 4, 128, 1100),   # tensor-core path, group 1
     (128, 4, 2, 3, 4, 128, 1100),   # tensor-core path, group 2
     (128, 16, 2, 3, 4, 128, 1100),  # tensor-core path, group 8
@@ -176,6 +176,32 @@ def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
     Q = tq_inputs.iid((B, Hq, d), seed=3, dtype=torch.bfloat16)
     kc, vc = _cache(c, K, V, cuda)
     lens = torch.tensor([0, 1, 129, 513, 777, T], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+
+
+@pytest.mark.parametrize("Hq,Hkv,lens_kind", [
+    (8, 2, "mixed"), (16, 2, "mixed"), (4, 4, "mixed"), (2, 1, "mixed"),
+    (8, 2, "tiny"), (16, 2, "tiny")])
+def test_attention_many_short_rows(cuda, Hq, Hkv, lens_kind):
+    """Tensor-core path with many short sequences: the balanced tile ranges
+    cross many (sequence, kv head) rows, and with tiny lengths there are
+    fewer tiles than warps."""
+    c = _ctx(128, 3, 4, 128, seed=5)
+    tab = P.oracle_tables(c)
+    B, T = 37, 256
+    g = torch.Generator().manual_seed(11)
+    if lens_kind == "mixed":
+        lens = torch.randint(0, T + 1, (B,), generator=g, dtype=torch.int32)
+        lens[:4] = torch.tensor([0, T, 16, 17], dtype=torch.int32)
+    else:
+        lens = torch.randint(0, 3, (B,), generator=g, dtype=torch.int32)
+    K = tq_inputs.outlier_kv(B, Hkv, T, 128, seed=21)
+    V = tq_inputs.outlier_kv(B, Hkv, T, 128, seed=22)
+    Q = tq_inputs.iid((B, Hq, 128), seed=23, dtype=torch.bfloat16)
+    kc, vc = _cache(c, K, V, cuda)
     out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
     torch.cuda.synchronize()
     P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
