@@ -81,6 +81,69 @@ __device__ __forceinline__ uint32_t field_word(uint32_t val, int b, int lane) {
 // sketch S r are fp32 FMA dot products (PiT and ST are k-major so lanes read
 // consecutive words).
 // ----------------------------------------------------------------------------
+// ----------------------------------------------------------------------------
+// Row-batched matrix-vector products for the latency-bound small kernels:
+// thread j (blockDim = dpad) computes acc[r] = sum_k M[k][j] x_r[k] for R
+// vectors x_r held in shared memory.  M ([d][dpad] fp32) streams through
+// shared memory in chunks of MV_KC rows, two chunks in flight (cp.async), so
+// the block pays the L2 latency about once per chunk, not once per row.
+// ----------------------------------------------------------------------------
+constexpr int MV_KC = 32;
+
+__device__ __forceinline__ void mv_cp16(float* dst, const float* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src));
+}
+
+__device__ __forceinline__ void mv_issue(const float* M, int d, int dpad, int chunk, float* buf) {
+  const int k0 = chunk * MV_KC;
+  const int rows = min(MV_KC, d - k0);
+  const int pieces = rows * dpad / 4;
+  for (int e = threadIdx.x; e < pieces; e += blockDim.x) mv_cp16(buf + 4 * e, M + (size_t)k0 * dpad + 4 * e);
+  asm volatile("cp.async.commit_group;\n" ::);
+}
+
+// Ms: shared [2][MV_KC][dpad].  Ends with a barrier (Ms and xs reusable).
+template <int R>
+__device__ __forceinline__ void mv_rows(const float* M, int d, int dpad, const float* xs, float* Ms,
+                                        float (&acc)[R]) {
+  const int j = threadIdx.x;
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+  const int nchunk = (d + MV_KC - 1) / MV_KC;
+  mv_issue(M, d, dpad, 0, Ms);
+  for (int c = 0; c < nchunk; ++c) {
+    if (c + 1 < nchunk) {
+      mv_issue(M, d, dpad, c + 1, Ms + ((c + 1) & 1) * MV_KC * dpad);
+      asm volatile("cp.async.wait_group 1;\n" ::);
+    } else {
+      asm volatile("cp.async.wait_group 0;\n" ::);
+    }
+    __syncthreads();
+    const float* mb = Ms + (c & 1) * MV_KC * dpad;
+    const int k0 = c * MV_KC, rows = min(MV_KC, d - k0);
+    int kk = 0;
+    for (; kk + 4 <= rows; kk += 4) {   // x rows read as float4 (k0 + kk is a multiple of 4)
+      const float m0 = mb[kk * dpad + j], m1 = mb[(kk + 1) * dpad + j];
+      const float m2 = mb[(kk + 2) * dpad + j], m3 = mb[(kk + 3) * dpad + j];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float4 x4 = *reinterpret_cast<const float4*>(xs + r * dpad + k0 + kk);
+        acc[r] = fmaf(m0, x4.x, acc[r]);
+        acc[r] = fmaf(m1, x4.y, acc[r]);
+        acc[r] = fmaf(m2, x4.z, acc[r]);
+        acc[r] = fmaf(m3, x4.w, acc[r]);
+      }
+    }
+    for (; kk < rows; ++kk) {
+      const float m = mb[kk * dpad + j];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = fmaf(m, xs[r * dpad + k0 + kk], acc[r]);
+    }
+    __syncthreads();   // the chunk buffer is refilled two chunks later
+  }
+}
+
 constexpr int QV = 8;
 constexpr int QWARPS = 8;
 
@@ -228,96 +291,114 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 }
 
 // ----------------------------------------------------------------------------
-// Quantize, small batches (the per-step cache append): one block per vector,
-// thread j owns coordinate j (and QJL row j), so a few hundred vectors spread
-// over all SMs instead of filling one tile.  Same fp32 arithmetic as above.
+// Quantize, small batches (the per-step cache append): QS vectors per block,
+// thread j owns coordinate j (and QJL row j) of each, so the block reads Pi
+// and S once for all QS vectors, and a few hundred vectors spread over many
+// SMs instead of filling one tile.  Same fp32 arithmetic as above.
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ float block_sum(float v, float* red) {
-  v = warp_sum(v);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float t = 0.f;
-  for (int w = 0; w < nw; ++w) t += red[w];
-  return t;
-}
-
+template <int QS>
 __global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
-  extern __shared__ float sh[];
-  float* sx = sh;            // [dpad] x, later r
-  __shared__ float red[8];
+  extern __shared__ float sh[];   // [QS][dpad]: x, later r; then [2][MV_KC][dpad] matrix chunks
+  float* Ms = sh + QS * dpad;
+  __shared__ float red[QS][8];
   __shared__ float s_cen[16], s_bnd[16];
-  const int j = threadIdx.x, lane = j & 31;
-  const int64_t v = blockIdx.x;
+  const int j = threadIdx.x, lane = j & 31, warp = j >> 5, nwarp = blockDim.x >> 5;
+  const int64_t v0 = (int64_t)blockIdx.x * QS;
+  const int nv = (int)min((int64_t)QS, a.n - v0);
   if (j < 16) {
     s_cen[j] = (j < (1 << a.bits)) ? a.cen[j] : 0.f;
     s_bnd[j] = (j < a.nbnd) ? a.bnd[j] : INFINITY;
   }
-  const float xj = (j < a.d) ? load_elem(a.x, a.dtype, v * a.ld + j) : 0.f;
-  sx[j] = xj;
-  const float nrm = sqrtf(block_sum(xj * xj, red));   // includes the barrier for sx / tables
-  float a4[4] = {0.f, 0.f, 0.f, 0.f};
-  int k = 0;
-  for (; k + 4 <= a.d; k += 4) {
+  float nrm[QS];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) a4[u] = fmaf(a.PiT[(size_t)(k + u) * dpad + j], sx[k + u], a4[u]);
+  for (int u = 0; u < QS; ++u) {
+    const float xj = (u < nv && j < a.d) ? load_elem(a.x, a.dtype, (v0 + u) * a.ld + j) : 0.f;
+    sh[u * dpad + j] = xj;
+    nrm[u] = warp_sum(xj * xj);
   }
-  for (; k < a.d; ++k) a4[0] = fmaf(a.PiT[(size_t)k * dpad + j], sx[k], a4[0]);
-  const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-  const float y = (nrm > 0.f && j < a.d) ? acc / nrm : 0.f;
-  const int idx = lm_index(y, s_bnd, a.nbnd);
-  const int64_t rec = out_record(a, v);
-  // b-bit field packing within each warp (b = 3: 2-bit stream, then 1-bit stream)
-  const uint32_t iv = (j < a.d) ? (uint32_t)idx : 0u;
+  if (lane == 0) {
+#pragma unroll
+    for (int u = 0; u < QS; ++u) red[u][warp] = nrm[u];
+  }
+  __syncthreads();   // x, tables and the per-warp sums are in shared memory
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    float t = 0.f;
+    for (int w = 0; w < nwarp; ++w) t += red[u][w];
+    nrm[u] = sqrtf(t);
+  }
+  float acc[QS];
+  mv_rows<QS>(a.PiT, a.d, dpad, sh, Ms, acc);
+  float r[QS];
   const int i32 = j >> 5;
-  if (a.bits == 3) {
-    const int w2 = (a.d + 15) >> 4;
-    const uint32_t lo = field_word(iv & 3u, 2, lane);
-    const uint32_t hi = field_word(iv >> 2, 1, lane);
-    const int wlo = 2 * i32 + (lane >> 4);
-    if ((lane & 15) == 0 && wlo < w2) a.codes[rec * a.words + wlo] = lo;
-    if (lane == 0) a.codes[rec * a.words + w2 + i32] = hi;
-  } else {
-    const int per = 32 / a.bits;
-    const uint32_t wv = field_word(iv, a.bits, lane);
-    const int wi = a.bits * i32 + lane / per;
-    if (lane % per == 0 && wi < a.words) a.codes[rec * a.words + wi] = wv;
-  }
-  if (j == 0) a.norm[rec] = nrm;
-  if (a.m == 0) return;
-  const float r = (j < a.d) ? y - s_cen[idx] : 0.f;
-  __syncthreads();   // everyone has read x
-  sx[j] = r;
-  const float rho = sqrtf(block_sum(r * r, red));
-  float b4[4] = {0.f, 0.f, 0.f, 0.f};
-  k = 0;
-  for (; k + 4 <= a.d; k += 4) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) b4[u] = fmaf(a.ST[(size_t)(k + u) * dpad + j], sx[k + u], b4[u]);
+  for (int u = 0; u < QS; ++u) {
+    const float y = (nrm[u] > 0.f && j < a.d) ? acc[u] / nrm[u] : 0.f;
+    const int idx = lm_index(y, s_bnd, a.nbnd);
+    r[u] = (j < a.d) ? y - s_cen[idx] : 0.f;
+    if (u >= nv) continue;   // uniform over the block
+    const int64_t rec = out_record(a, v0 + u);
+    // b-bit field packing within each warp (b = 3: 2-bit stream, then 1-bit stream)
+    const uint32_t iv = (j < a.d) ? (uint32_t)idx : 0u;
+    if (a.bits == 3) {
+      const int w2 = (a.d + 15) >> 4;
+      const uint32_t lo = field_word(iv & 3u, 2, lane);
+      const uint32_t hi = field_word(iv >> 2, 1, lane);
+      const int wlo = 2 * i32 + (lane >> 4);
+      if ((lane & 15) == 0 && wlo < w2) a.codes[rec * a.words + wlo] = lo;
+      if (lane == 0) a.codes[rec * a.words + w2 + i32] = hi;
+    } else {
+      const int per = 32 / a.bits;
+      const uint32_t wv = field_word(iv, a.bits, lane);
+      const int wi = a.bits * i32 + lane / per;
+      if (lane % per == 0 && wi < a.words) a.codes[rec * a.words + wi] = wv;
+    }
+    if (j == 0) a.norm[rec] = nrm[u];
   }
-  for (; k < a.d; ++k) b4[0] = fmaf(a.ST[(size_t)k * dpad + j], sx[k], b4[0]);
-  const float sr = (b4[0] + b4[1]) + (b4[2] + b4[3]);
-  const uint32_t bits = __ballot_sync(0xffffffffu, sr >= 0.f && j < a.m);
-  if (lane == 0 && j < a.m) a.qjl[rec * ((a.m + 31) >> 5) + i32] = bits;
-  if (j == 0) a.rnorm[rec] = nrm * rho;
+  if (a.m == 0) return;
+  float rho[QS];
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    sh[u * dpad + j] = r[u];
+    rho[u] = warp_sum(r[u] * r[u]);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int u = 0; u < QS; ++u) red[u][warp] = rho[u];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    float t = 0.f;
+    for (int w = 0; w < nwarp; ++w) t += red[u][w];
+    rho[u] = sqrtf(t);
+  }
+  mv_rows<QS>(a.ST, a.d, dpad, sh, Ms, acc);
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    const uint32_t bits = __ballot_sync(0xffffffffu, acc[u] >= 0.f && j < a.m);
+    if (u >= nv) continue;
+    const int64_t rec = out_record(a, v0 + u);
+    if (lane == 0 && j < a.m) a.qjl[rec * ((a.m + 31) >> 5) + i32] = bits;
+    if (j == 0) a.rnorm[rec] = nrm[u] * rho[u];
+  }
 }
 
 // ----------------------------------------------------------------------------
-// Query pre-rotation: q' = Pi q, s = S q' (one block per query row).
+// Query pre-rotation: q' = Pi q, s = S q' (PR rows per block).
 // ----------------------------------------------------------------------------
 // Tile prefix of the segment-partitioned decode: tiles[b] = Hkv * sum over
 // b' < b of ceil(len_b' / 16), len = min(max(seq_lens, 0), max_T); one block.
 __device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T, int64_t* tiles) {
-  __shared__ int64_t s_w[4];
+  __shared__ int64_t s_w[8];
   __shared__ int64_t s_carry;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
   if (tid == 0) {
     s_carry = 0;
     tiles[0] = 0;
   }
   __syncthreads();
-  for (int base = 0; base < B; base += 128) {
+  for (int base = 0; base < B; base += nt) {
     const int b = base + tid;
     int64_t v = 0;
     if (b < B) {
@@ -335,47 +416,39 @@ __device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T
     for (int w = 0; w < warp; ++w) off += s_w[w];
     if (b < B) tiles[b + 1] = off + v;
     __syncthreads();
-    if (tid == 127) s_carry = off + v;
+    if (tid == nt - 1) s_carry = off + v;
     __syncthreads();
   }
 }
 
-__global__ void __launch_bounds__(128) k_prerotate(const void* q, int dtype, int d, int dpad,
-                                                   int m, const float* PiT, const float* ST,
+// PR query rows per block: thread j owns coordinate j of each row, so Pi and
+// S are read once per block.
+template <int PR>
+__global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int64_t rows, int d,
+                                                   int dpad, int m, const float* PiT, const float* ST,
                                                    float* qr, float* qs, const int32_t* seq_lens,
                                                    int B, int Hkv, int64_t max_T, int64_t* tiles) {
   extern __shared__ float sh[];
-  float* sq = sh;          // [dpad]
-  float* sr = sh + dpad;   // [dpad]
-  const int64_t row = blockIdx.x;
-  for (int k = threadIdx.x; k < dpad; k += blockDim.x)
-    sq[k] = (k < d) ? load_elem(q, dtype, row * d + k) : 0.f;
-  __syncthreads();
-  for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
-    float a4[4] = {0.f, 0.f, 0.f, 0.f};
-    int k = 0;
-    for (; k + 4 <= d; k += 4) {
+  float* sq = sh;                  // [PR][dpad]: q, later q'
+  float* Ms = sh + PR * dpad;      // [2][MV_KC][dpad]
+  const int j = threadIdx.x;       // blockDim = dpad
+  const int64_t row0 = (int64_t)blockIdx.x * PR;
+  const int nr = (int)min((int64_t)PR, rows - row0);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) a4[u] = fmaf(PiT[(size_t)(k + u) * dpad + j], sq[k + u], a4[u]);
-    }
-    for (; k < d; ++k) a4[0] = fmaf(PiT[(size_t)k * dpad + j], sq[k], a4[0]);
-    const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-    sr[j] = acc;
-    qr[row * dpad + j] = acc;
+  for (int r = 0; r < PR; ++r) sq[r * dpad + j] = (r < nr && j < d) ? load_elem(q, dtype, (row0 + r) * d + j) : 0.f;
+  __syncthreads();
+  float acc[PR];
+  mv_rows<PR>(PiT, d, dpad, sq, Ms, acc);
+#pragma unroll
+  for (int r = 0; r < PR; ++r) {
+    sq[r * dpad + j] = acc[r];
+    if (r < nr) qr[(row0 + r) * dpad + j] = acc[r];
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < dpad; i += blockDim.x) {
-    float a4[4] = {0.f, 0.f, 0.f, 0.f};
-    if (i < m) {
-      int k = 0;
-      for (; k + 4 <= d; k += 4) {
+  mv_rows<PR>(ST, d, dpad, sq, Ms, acc);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) a4[u] = fmaf(ST[(size_t)(k + u) * dpad + i], sr[k + u], a4[u]);
-      }
-      for (; k < d; ++k) a4[0] = fmaf(ST[(size_t)k * dpad + i], sr[k], a4[0]);
-    }
-    qs[row * dpad + i] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-  }
+  for (int r = 0; r < PR; ++r)
+    if (r < nr) qs[(row0 + r) * dpad + j] = (j < m) ? acc[r] : 0.f;
   if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
 }
 
@@ -971,16 +1044,31 @@ cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s)
 
 cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;
-  k_quantize_small<<<(unsigned)a.n, c->dpad, c->dpad * sizeof(float), s>>>(a, c->dpad);
+  // One vector per block while that still fills the GPU; eight per block
+  // (one read of Pi and S for all eight) beyond.
+  if (a.n <= 1024) {
+    k_quantize_small<1><<<(unsigned)a.n, c->dpad, (1 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(a, c->dpad);
+  } else {
+    k_quantize_small<8><<<(unsigned)((a.n + 7) / 8), c->dpad, (8 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
+        a, c->dpad);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
                              float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
-  k_prerotate<<<(unsigned)rows, 128, 2 * c->dpad * sizeof(float), s>>>(
-      q, dtype, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, plan ? plan->seq_lens : nullptr,
-      plan ? plan->B : 0, plan ? plan->Hkv : 1, plan ? plan->max_T : 0, plan ? plan->tiles : nullptr);
+  const int32_t* sl = plan ? plan->seq_lens : nullptr;
+  const int pB = plan ? plan->B : 0, pH = plan ? plan->Hkv : 1;
+  const int64_t pT = plan ? plan->max_T : 0;
+  int64_t* tl = plan ? plan->tiles : nullptr;
+  if (rows <= 1024) {
+    k_prerotate<2><<<(unsigned)((rows + 1) / 2), c->dpad, (2 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
+        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl);
+  } else {
+    k_prerotate<8><<<(unsigned)((rows + 7) / 8), c->dpad, (8 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
+        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl);
+  }
   return cudaGetLastError();
 }
 
@@ -1105,6 +1193,13 @@ cudaError_t configure_kernels() {
   if ((e = configure_J<6>()) != cudaSuccess) return e;
   if ((e = configure_J<7>()) != cudaSuccess) return e;
   if ((e = configure_J<8>()) != cudaSuccess) return e;
+  // Row-batched small kernels: up to (8 + 2 * MV_KC) rows of dpad = 256 floats.
+  const int small_smem = (8 + 2 * MV_KC) * 256 * (int)sizeof(float);
+  const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if ((e = cudaFuncSetAttribute(k_quantize_small<1>, ms, small_smem))) return e;
+  if ((e = cudaFuncSetAttribute(k_quantize_small<8>, ms, small_smem))) return e;
+  if ((e = cudaFuncSetAttribute(k_prerotate<2>, ms, small_smem))) return e;
+  if ((e = cudaFuncSetAttribute(k_prerotate<8>, ms, small_smem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   return configure_attn_mma();
 }
