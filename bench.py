@@ -279,6 +279,87 @@ def quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak, steps=10, warmup=3):
             "frac_hbm": head["frac_hbm"], "sweep": points}
 
 
+VSEARCH = dict(n=1_000_000, nq=10_000, k=10, d=200, bits_k=4, m=200)
+
+
+def vector_search(tq, tq_inputs, torch, dev, sm_mhz_max, steps=3, warmup=1):
+    """Inner-product top-k over a compressed database (3 Lloyd-Max bits + QJL,
+    m = d = 200): 1e6 mixture vectors, 1e4 queries, top-10 per query."""
+    s = VSEARCH
+    ctx = tq.Context(s["d"], s["bits_k"], 3, s["m"], 0)
+    X = tq_inputs.mixture(s["n"], s["d"], seed=21, device=dev)
+    Q = tq_inputs.mixture(s["nq"], s["d"], seed=22, means_seed=21, device=dev)
+    db = ctx.quantize(X, tq.TQ_KEY)
+    del X
+    ws = torch.empty(ctx.topk_workspace_bytes(s["nq"], s["n"], s["k"]), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        ctx.topk(Q, db, s["k"], workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        ctx.topk(Q, db, s["k"], workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / steps
+    flop = 2.0 * s["nq"] * s["n"] * (s["d"] + s["m"])   # <q', c[idx]> over d, <s, sigma> over m
+    # FP32 FMA peak from unit counts: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock.
+    peak = 148 * 128 * 2 * sm_mhz_max * 1e6 / 1e12
+    ctx.close()
+    del db, Q, ws
+    torch.cuda.empty_cache()
+    return {"config": f"{s['n']} db vectors x d={s['d']} (Gaussian mixture), {s['nq']} queries, "
+                      f"top-{s['k']}; keys 3 Lloyd-Max bits + QJL (m={s['m']})",
+            "value": s["nq"] / t, "unit": "queries/s", "ms_per_call": t * 1e3,
+            "roofline": {"bound": "alu", "achieved": flop / t / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flop / t / 1e12 / peak,
+                         "peak_source": "FP32 FMA lanes x 2 x max SM clock (148 x 128 x 2 x clock)"}}
+
+
+def small_case(tq, tq_inputs, torch, dev, reps=50):
+    """Latency of the smallest workload: quantize 1024 K and 1024 V (fp32,
+    d = 128, k3v4), then attention of 8 query heads over them (one kv head)."""
+    ctx = tq.Context(128, 3, 4, 128, 0)
+    K = tq_inputs.iid((1, 1, 1024, 128), seed=0, device=dev)
+    V = tq_inputs.iid((1, 1, 1024, 128), seed=1, device=dev)
+    q = tq_inputs.iid((1, 8, 128), seed=2, device=dev)
+    kc = ctx.empty_packed(tq.TQ_KEY, (1, 1, 1024), device=dev)
+    vc = ctx.empty_packed(tq.TQ_VALUE, (1, 1, 1024), device=dev)
+    lens = torch.full((1,), 1024, dtype=torch.int32, device=dev)
+    out = torch.empty(1, 8, 128, device=dev)
+    ws = torch.empty(ctx.attn_workspace_bytes(1, 8, 1024), dtype=torch.uint8, device=dev)
+
+    def quant():
+        ctx.quantize_into(K, tq.TQ_KEY, kc)
+        ctx.quantize_into(V, tq.TQ_VALUE, vc)
+
+    def attend():
+        ctx.attn_decode(q, kc, vc, lens, out=out, workspace=ws)
+
+    res = {}
+    for name, fn in (("quantize_kv_us", quant), ("attn_decode_us", attend)):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(10):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / (reps * 10)
+        del g
+    ctx.close()
+    res["config"] = "1024 K + 1024 V fp32 N(0,1), d=128, k3v4; 8 query heads over one kv head"
+    res["timing"] = "CUDA-graph replays of 10 calls, device time per call"
+    return res
+
+
 def run_gpu(args, w):
     import torch
     import torch.distributed as dist
@@ -423,6 +504,12 @@ def run_gpu(args, w):
     quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
     torch.cuda.nvtx.range_pop()
     clocks = sampler.stop()
+    vsearch = small = None
+    if not args.skip_extra:
+        torch.cuda.nvtx.range_push("tq:vector_search")
+        vsearch = vector_search(tq, tq_inputs, torch, dev, clocks.get("sm_max_mhz") or 1965.0)
+        torch.cuda.nvtx.range_pop()
+        small = small_case(tq, tq_inputs, torch, dev)
 
     tm = torch.tensor([t_ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -456,6 +543,9 @@ def run_gpu(args, w):
             "clocks": clocks,
             "quantize": quant,
         }
+        if vsearch is not None:
+            line["vector_search"] = vsearch
+            line["small_case"] = small
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
@@ -472,6 +562,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama3-8b-decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--skip-extra", dest="skip_extra", action="store_true",
+                    help="omit the vector-search and small-case measurements")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]

@@ -505,14 +505,16 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.part = part;
   a.tiles = nullptr;
   const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
-  if (mma) {
+  const bool k4 = !mma && tqk::attn_k4_supported(c, a) && max_T > 0;
+  if (mma || k4) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
   }
   cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s);
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode: prerotate");
-  e = mma ? tqk::launch_attn_mma(c, a, out, s) : tqk::launch_attn(c, a, out, s);
+  e = mma ? tqk::launch_attn_mma(c, a, out, s)
+          : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
   return TQ_OK;
 }

@@ -1,0 +1,431 @@
+// Decode attention from packed codes with 3-bit Lloyd-Max keys (k4v4: keys
+// 3 Lloyd-Max bits + 1 QJL bit with m = 128 rows, values 4 bits), d = 128,
+// GQA group 8, on the tensor cores (sm_100a).
+//
+// Same quantities as the 2-bit-key kernels ("What is TurboQuant?", "How
+// TurboQuant works", closing paragraph; "How to implement" part 1):
+//   l_i = |k_i| <q', c_k[idx_i]> + sqrt(pi/2)/m * gamma_i <S q', sigma_i>,
+// online softmax, o = sum p_i |v_i| c_v[vidx_i] in the rotated domain; the
+// merge kernel combines the partials by log-sum-exp and applies Pi^T.
+//
+// An 8-level codebook is not affine in its index bits, so the key product
+// dequantizes instead: two neighbouring coordinates of a token (their two
+// 2-bit fields and two top bits, a 6-bit index) select a half2 of centroids
+// from a 64-entry table in shared memory, one copy per lane.  Each entry holds
+// the fp16 head of the centroid pair and its tail x 2^12; the query operand
+// likewise carries an fp16 head and tail, and three MMAs per k-step form
+// head*head + head*tail + tail*head (~22 bits).  The QJL product, the
+// softmax, the value product and the work split are those of the group-8
+// kernel for 2-bit keys: balanced CTA ranges of 16-token tiles, query
+// operands built once per row piece into shared memory.
+//
+// Key layout (3-bit fields of d = 128): words 0..7 hold the low two bits of
+// the indices (16 coordinates per word), words 8..11 the top bits (32 per
+// word).  Thread t of a quad owns coordinates 32t .. 32t+31: 2-bit words 2t,
+// 2t+1 and top-bit word t.  k-step s (0..7) pairs coordinates 32t + 2s, +1
+// (MMA k 2t, 2t+1) and 32t + 16 + 2s, +1 (k 2t+8, 2t+9).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cmath>
+
+#include "tq_attn_common.cuh"
+#include "tq_internal.h"
+
+namespace tqk {
+namespace {
+
+constexpr int NSTK = 3;      // pipeline stages per warp
+constexpr int K2W = 8;       // 2-bit stream words per key (d = 128)
+constexpr int K1W = 4;       // top-bit stream words per key
+constexpr int KLUT = 64;     // key table entries (two coordinates' 3-bit indices)
+constexpr int QOPK = 8;      // words per lane and key k-step (6 used: 3 MMAs x 2)
+constexpr int QOPQ = 4;      // words per lane and QJL k-step (2 MMAs x 2)
+
+struct StageK4 {
+  uint32_t k2[MT][K2W];      // 512 B
+  uint32_t k1[MT][K1W];      // 256 B
+  uint32_t q[MT][QW];        // 256 B
+  float kn[MT];              // 64 B
+  float kr[MT];              // 64 B
+  float vn[MT];              // 64 B
+  uint32_t pad_[4];          // keep v 16-byte aligned
+  uint32_t v[MT][VROW];      // 1280 B
+};
+static_assert(sizeof(StageK4) % 16 == 0, "stage alignment");
+static_assert(offsetof(StageK4, v) % 16 == 0, "value rows alignment");
+
+constexpr size_t KLUT_BYTES = (size_t)KLUT * 32 * 8;
+constexpr size_t SMEMK4_BYTES = KLUT_BYTES + (size_t)LUT_WORDS * 4 + (size_t)MW * NSTK * sizeof(StageK4) +
+                                (size_t)8 * 32 * QOPK * 4 + (size_t)8 * 32 * QOPQ * 4 + 8 * 16 + MW * 4 +
+                                16 * 4;
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+// Byte offset of key-table entry (index of coordinates 2s, 2s+1 of word pair
+// (w2, w1 >> sh)), without the lane offset: idx * 32 lanes * 8 bytes.
+template <int S, int SH>
+__device__ __forceinline__ uint32_t klut_off(uint32_t w2, uint32_t w1) {
+  const uint32_t nib = (w2 >> (4 * S)) & 0xFu;
+  const uint32_t top = (w1 >> (SH + 2 * S)) & 3u;
+  return (nib | (top << 4)) << 8;
+}
+
+__global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
+  constexpr int G = 8;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint2* klut = reinterpret_cast<uint2*>(smem);                                          // [64][32]
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + KLUT_BYTES);                       // values
+  StageK4* stages = reinterpret_cast<StageK4*>(smem + KLUT_BYTES + (size_t)LUT_WORDS * 4);
+  uint32_t* qopk = reinterpret_cast<uint32_t*>(stages + MW * NSTK);                      // [8][32][8]
+  uint32_t* qopq = qopk + 8 * 32 * QOPK;                                                  // [8][32][4]
+  float4* s_head = reinterpret_cast<float4*>(qopq + 8 * 32 * QOPQ);                      // [8]
+  float* s_vmax = reinterpret_cast<float*>(s_head + 8);                                  // [MW]
+  int* s_scale = reinterpret_cast<int*>(s_vmax + MW);                                    // [16]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  build_value_lut(lut, a.cv, tid, MW * 32);
+  // Key table: entry (idx, lane) = (fp16 heads, fp16 tails x 2^12) of the
+  // centroids of two coordinates, idx = f0 | f1 << 2 | top0 << 4 | top1 << 5
+  // (f = 2-bit field, top = third index bit).
+  for (int e = tid; e < KLUT * 32; e += MW * 32) {
+    const int idx = e >> 5;
+    const int i0 = (idx & 3) | (((idx >> 4) & 1) << 2);
+    const int i1 = ((idx >> 2) & 3) | (((idx >> 5) & 1) << 2);
+    const float c0 = a.ck[i0], c1 = a.ck[i1];
+    const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
+    klut[e] = make_uint2(pack_half2(h0, h1), pack_half2((c0 - h0) * 4096.f, (c1 - h1) * 4096.f));
+  }
+  __syncthreads();
+
+  const int64_t* P = a.tiles;
+  const int64_t W = P[a.B];
+  const int64_t NC = min((int64_t)gridDim.x, W);
+  const int64_t cta = blockIdx.x;
+  if (cta >= NC) return;   // uniform over the CTA
+  int64_t x = cta * W / NC;
+  const int64_t x1 = (cta + 1) * W / NC;
+  int b = locate_sequence(P, a.B, x);
+
+  const uint32_t klut_lane = (uint32_t)__cvta_generic_to_shared(klut) + lane * 8;
+  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  const uint32_t qopk_lane = (uint32_t)__cvta_generic_to_shared(qopk) + lane * QOPK * 4;
+  const uint32_t qopq_lane = (uint32_t)__cvta_generic_to_shared(qopq) + lane * QOPQ * 4;
+  StageK4* my = stages + warp * NSTK;
+  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
+
+  while (x < x1) {
+    while (P[b + 1] <= x) ++b;
+    const int64_t tb = (P[b + 1] - P[b]) / a.Hkv;
+    const int64_t rel = x - P[b];
+    const int kvh = (int)(rel / tb);
+    const int64_t tt = rel - (int64_t)kvh * tb;
+    const int64_t te = min(tb, tt + (x1 - x));
+    const int nt = (int)(te - tt);
+    const int64_t slot = 4 * (cta + (int64_t)b * a.Hkv + kvh) + warp;
+    x += nt;
+
+    const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
+    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
+    const int64_t tok0 = tt * MT;
+    const int64_t tok1 = min(te * MT, len);
+    const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * G;
+
+    __syncthreads();   // the previous piece's readers of the operands are done
+    // ---- per-head scales (warp w: heads 2w, 2w+1) and the value-norm maximum ----
+#pragma unroll
+    for (int hsel = 0; hsel < 2; ++hsel) {
+      const int h = 2 * warp + hsel;
+      const float4 q4 = reinterpret_cast<const float4*>(a.qr + (qbase + h) * 128)[lane];
+      const float4 s4 = reinterpret_cast<const float4*>(a.qs + (qbase + h) * 128)[lane];
+      float mq = fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w)));
+      float ms = fmaxf(fmaxf(fabsf(s4.x), fabsf(s4.y)), fmaxf(fabsf(s4.z), fabsf(s4.w)));
+      float ss = (s4.x + s4.y) + (s4.z + s4.w);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+        ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      }
+      if (lane == 0) {
+        const int eq = mq > 0.f ? ilog2f(mq) : 0;
+        const int es = ms > 0.f ? ilog2f(ms) : 0;
+        s_scale[h] = eq;
+        s_scale[8 + h] = es;
+        // q' 2^-(eq+1) < 1 in the key operand; S q' as in the 2-bit kernels.
+        s_head[h] = make_float4(pow2i(eq + 1) * a.scale_log2, 0.f, 2.f * pow2i(es) * a.cq * a.scale_log2,
+                                -ss * a.cq * a.scale_log2);
+      }
+    }
+    {
+      float vmax = 0.f;
+      const float* vr = a.vnorm + row0;
+      for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
+        if (j + 4 <= tok1) {
+          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
+        } else {
+          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      if (lane == 0) s_vmax[warp] = vmax;
+    }
+    __syncthreads();
+    // ---- query operands: warp w builds key k-steps 2w, 2w+1 and QJL k-steps 2w, 2w+1 ----
+    {
+      const bool odd_col = (g & 1) != 0;
+      auto split = [&](float lo, float hi, bool tail) -> uint32_t {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        if (!tail) return *reinterpret_cast<const uint32_t*>(&h);
+        const float2 f = __half22float2(h);
+        return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
+      };
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int s = 2 * warp + k;
+        // Key k-step s.  MMA 0: heads 0..3, MMA 1: heads 4..7 (column g: head
+        // g/2 of the group, fp16 head if g is even, tail if odd); MMA 2: the
+        // heads of the query times the centroid tails, column g = head g/2 +
+        // 4 (g & 1), fp16 head.
+        uint32_t fr[6];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          const int h = m < 2 ? 4 * m + (g >> 1) : (g >> 1) + 4 * (g & 1);
+          const bool tail = m < 2 && odd_col;
+          const float kq = pow2i(-(s_scale[h] + 1));
+          const float* row = a.qr + (qbase + h) * 128 + 32 * t;
+          fr[2 * m] = split(row[2 * s] * kq, row[2 * s + 1] * kq, tail);
+          fr[2 * m + 1] = split(row[16 + 2 * s] * kq, row[16 + 2 * s + 1] * kq, tail);
+        }
+        uint32_t* dk = qopk + (s * 32 + lane) * QOPK;
+        *reinterpret_cast<uint4*>(dk) = make_uint4(fr[0], fr[1], fr[2], fr[3]);
+        *reinterpret_cast<uint2*>(dk + 4) = make_uint2(fr[4], fr[5]);
+        // QJL k-step s: fp16 bit operands as in the 2-bit kernels (registers
+        // u = 2s, 2s+1 of the sign word), MMA 0 heads 0..3, MMA 1 heads 4..7.
+        uint32_t fq[4];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int h = 4 * m + (g >> 1);
+          const float ks = pow2i(-s_scale[8 + h]);
+          const float* row = a.qs + (qbase + h) * 128 + 32 * t;
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            const int u = 2 * s + sl;
+            const int elo = 10 + u, ehi = (26 + u) & 31;
+            const float inv = bit_inv(bit_pos(u)) * ks;
+            fq[2 * m + sl] = split(row[elo] * inv, row[ehi] * inv, odd_col);
+          }
+        }
+        *reinterpret_cast<uint4*>(qopq + (s * 32 + lane) * QOPQ) = make_uint4(fq[0], fq[1], fq[2], fq[3]);
+      }
+    }
+    __syncthreads();
+    const float4 H0 = s_head[t], H1 = s_head[4 + t];
+    const float vmax = fmaxf(fmaxf(s_vmax[0], s_vmax[1]), fmaxf(s_vmax[2], s_vmax[3]));
+    // p <= 2^8 and |v| 2^-kv < 2^7 keep p |v| 2^-kv below 2^15.
+    const int kv = vmax >= FLT_MIN ? max(ilog2f(vmax) - 6, -120) : -120;
+    const float vmul = pow2i(-kv);
+
+    // ---- this warp's tiles: i = warp, warp + 4, ... of the piece ------------------
+    const int ntw = nt > warp ? (nt - warp + MW - 1) / MW : 0;
+    const char* kbase = reinterpret_cast<const char*>(a.kcodes + row0 * (K2W + K1W));
+    auto issue = [&](int k, int stage) {
+      const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
+      const uint32_t sb = my_s + stage * (uint32_t)sizeof(StageK4);
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int c = lane + 32 * i;
+        if (c < 48) {                          // key codes: 16 tokens x 3 chunks
+          const int tok = c / 3, part = c % 3;
+          const uint32_t dst = part < 2 ? (uint32_t)(offsetof(StageK4, k2) + tok * 32 + part * 16)
+                                        : (uint32_t)(offsetof(StageK4, k1) + tok * 16);
+          cp16(sb + dst, kbase + (t0 + tok) * 48 + part * 16, t0 + tok < tok1);
+        } else if (c < 64) {                   // QJL words: 16 tokens x 1 chunk
+          const int tok = c - 48;
+          cp16(sb + offsetof(StageK4, q) + tok * 16, a.kqjl + (row0 + t0 + tok) * QW, t0 + tok < tok1);
+        } else if (c < 76) {                   // norms: 3 arrays x 4 chunks of 4 tokens
+          const int which = (c - 64) >> 2, part = (c - 64) & 3;
+          const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
+          const uint32_t off = which == 0 ? offsetof(StageK4, kn)
+                                          : (which == 1 ? offsetof(StageK4, kr) : offsetof(StageK4, vn));
+          cp16(sb + off + part * 16, base + row0 + t0 + 4 * part, t0 + 4 * part < tok1);
+        } else if (c < 140) {                  // value codes: 16 tokens x 4 chunks
+          const int cc = c - 76, tok = cc >> 2, part = cc & 3;
+          cp16(sb + offsetof(StageK4, v) + tok * (VROW * 4) + part * 16,
+               a.vcodes + (row0 + t0 + tok) * VW + part * 4, t0 + tok < tok1);
+        }
+      }
+    };
+#pragma unroll
+    for (int k = 0; k < NSTK - 1; ++k) {
+      if (k < ntw) issue(k, k);
+      cp_commit();
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_part[2] = {0.f, 0.f};
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    for (int k = 0; k < ntw; ++k) {
+      if (k + NSTK - 1 < ntw) issue(k + NSTK - 1, (k + NSTK - 1) % NSTK);
+      cp_commit();
+      cp_wait<NSTK - 1>();
+      __syncwarp();
+      const StageK4& st = my[k % NSTK];
+      const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
+
+      // ---- logits: heads t (accH0) and 4 + t (accH1), tails (accL), QJL (acs) ----
+      float accH0[4] = {0.f, 0.f, 0.f, 0.f}, accH1[4] = {0.f, 0.f, 0.f, 0.f}, accL[4] = {0.f, 0.f, 0.f, 0.f};
+      float acs[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const uint2 wg2 = *reinterpret_cast<const uint2*>(&st.k2[g][2 * t]);
+        const uint2 wh2 = *reinterpret_cast<const uint2*>(&st.k2[g + 8][2 * t]);
+        const uint32_t wg1 = st.k1[g][t], wh1 = st.k1[g + 8][t];
+#define TQ_K4STEP(S)                                                                              \
+  {                                                                                               \
+    const uint2 A0 = lds64(klut_lane + klut_off<S, 0>(wg2.x, wg1));                               \
+    const uint2 A1 = lds64(klut_lane + klut_off<S, 0>(wh2.x, wh1));                               \
+    const uint2 A2 = lds64(klut_lane + klut_off<S, 16>(wg2.y, wg1));                              \
+    const uint2 A3 = lds64(klut_lane + klut_off<S, 16>(wh2.y, wh1));                              \
+    const uint4 ba = lds128(qopk_lane + (S) * 32 * QOPK * 4);                                     \
+    const uint2 bb = lds64(qopk_lane + (S) * 32 * QOPK * 4 + 16);                                 \
+    mma16816(accH0, A0.x, A1.x, A2.x, A3.x, ba.x, ba.y);                                          \
+    mma16816(accH1, A0.x, A1.x, A2.x, A3.x, ba.z, ba.w);                                          \
+    mma16816(accL, A0.y, A1.y, A2.y, A3.y, bb.x, bb.y);                                           \
+  }
+        TQ_K4STEP(0) TQ_K4STEP(1) TQ_K4STEP(2) TQ_K4STEP(3) TQ_K4STEP(4) TQ_K4STEP(5)
+        TQ_K4STEP(6) TQ_K4STEP(7)
+#undef TQ_K4STEP
+        const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
+#define TQ_QSTEP8(S)                                                                              \
+  {                                                                                               \
+    const uint4 bq = lds128(qopq_lane + (S) * 32 * QOPQ * 4);                                     \
+    const uint32_t x0 = bit_half2<2 * (S)>(Q0), x1 = bit_half2<2 * (S)>(Q8);                       \
+    const uint32_t x2 = bit_half2<2 * (S) + 1>(Q0), x3 = bit_half2<2 * (S) + 1>(Q8);              \
+    mma16816(acs[0], x0, x1, x2, x3, bq.x, bq.y);                                                 \
+    mma16816(acs[1], x0, x1, x2, x3, bq.z, bq.w);                                                 \
+  }
+        TQ_QSTEP8(0) TQ_QSTEP8(1) TQ_QSTEP8(2) TQ_QSTEP8(3) TQ_QSTEP8(4) TQ_QSTEP8(5)
+        TQ_QSTEP8(6) TQ_QSTEP8(7)
+#undef TQ_QSTEP8
+      }
+      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
+      const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
+      float sc[2][2];
+      {
+        // <q', c> of head t (rows g, g+8) and head 4 + t: head products plus
+        // (head x tail + tail x head) / 2^12.
+        const float lm00 = accH0[0] + (accH0[1] + accL[0]) * (1.f / 4096.f);
+        const float lm08 = accH0[2] + (accH0[3] + accL[2]) * (1.f / 4096.f);
+        const float lm10 = accH1[0] + (accH1[1] + accL[1]) * (1.f / 4096.f);
+        const float lm18 = accH1[2] + (accH1[3] + accL[3]) * (1.f / 4096.f);
+        const float qj00 = fmaf(acs[0][1], 1.f / 4096.f, acs[0][0]);
+        const float qj08 = fmaf(acs[0][3], 1.f / 4096.f, acs[0][2]);
+        const float qj10 = fmaf(acs[1][1], 1.f / 4096.f, acs[1][0]);
+        const float qj18 = fmaf(acs[1][3], 1.f / 4096.f, acs[1][2]);
+        sc[0][0] = v0 ? fmaf(kn0 * lm00, H0.x, kr0 * fmaf(qj00, H0.z, H0.w)) : -INFINITY;
+        sc[0][1] = v8 ? fmaf(kn8 * lm08, H0.x, kr8 * fmaf(qj08, H0.z, H0.w)) : -INFINITY;
+        sc[1][0] = v0 ? fmaf(kn0 * lm10, H1.x, kr0 * fmaf(qj10, H1.z, H1.w)) : -INFINITY;
+        sc[1][1] = v8 ? fmaf(kn8 * lm18, H1.x, kr8 * fmaf(qj18, H1.z, H1.w)) : -INFINITY;
+      }
+
+      // ---- online softmax, heads t and 4 + t ----------------------------------------
+      const float loc0 = fmaxf(sc[0][0], sc[0][1]), loc1 = fmaxf(sc[1][0], sc[1][1]);
+      if (__any_sync(0xffffffffu, loc0 > m_run[0] + LAZY_TAU || loc1 > m_run[1] + LAZY_TAU)) {
+        float tm0 = loc0, tm1 = loc1;
+#pragma unroll
+        for (int o_ = 4; o_ <= 16; o_ <<= 1) {
+          tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o_));
+          tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o_));
+        }
+        const float mn0 = fmaxf(m_run[0], tm0), mn1 = fmaxf(m_run[1], tm1);
+        const float al0 = ex2f(m_run[0] - mn0), al1 = ex2f(m_run[1] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        l_part[0] *= al0;
+        l_part[1] *= al1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= al0; o[mt][2] *= al0;
+          o[mt][1] *= al1; o[mt][3] *= al1;
+        }
+      }
+      const float p00 = ex2f(sc[0][0] - m_run[0]), p01 = ex2f(sc[0][1] - m_run[0]);
+      const float p10 = ex2f(sc[1][0] - m_run[1]), p11 = ex2f(sc[1][1] - m_run[1]);
+      l_part[0] += p00 + p01;
+      l_part[1] += p10 + p11;
+      const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
+      const uint32_t pb0 = movtrans(pack_half2(p00 * w0s, p10 * w0s));
+      const uint32_t pb1 = movtrans(pack_half2(p01 * w8s, p11 * w8s));
+      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
+      __syncwarp();
+    }
+    cp_wait<0>();
+    __syncwarp();
+
+    // ---- this warp's partial of the piece (heads t and 4 + t) --------------------------
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 4);
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 8);
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], 16);
+    }
+    const float vback = pow2i(kv);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float* pp = a.part + (slot * G + 4 * j + t) * (128 + 2);
+      if (g == 0) {
+        pp[0] = m_run[j];
+        pp[1] = l_part[j];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        pp[2 + 16 * g + mt] = o[mt][j] * vback;
+        pp[2 + 16 * g + 8 + mt] = o[mt][2 + j] * vback;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+bool attn_k4_supported(const tq_ctx* c, const AttnArgs& a) {
+  if (c->d != D || c->bk_lm != 3 || c->bits_v != 4 || c->qjl_m != 128 || a.G != 8) return false;
+  if (a.max_T % 4 != 0) return false;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.kqjl) |
+                       reinterpret_cast<uintptr_t>(a.knorm) | reinterpret_cast<uintptr_t>(a.krnorm) |
+                       reinterpret_cast<uintptr_t>(a.vcodes) | reinterpret_cast<uintptr_t>(a.vnorm);
+  return (al & 15) == 0;
+}
+
+cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
+  AttnArgs a = a_in;
+  if (!a.tiles || a.G != 8) return cudaErrorInvalidValue;
+  // CTA-owned ranges of at least four tiles per warp; two CTAs per SM.
+  const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
+  int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
+  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 2 ? (int64_t)c->sms * 2 : blocks);
+  a.nw = (int)blocks;
+  a.wpu = MW;
+  k_attn_k4<<<(unsigned)blocks, MW * 32, SMEMK4_BYTES, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attn_merge(c, a, out, s);
+}
+
+cudaError_t configure_attn_k4() {
+  return cudaFuncSetAttribute(k_attn_k4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMK4_BYTES);
+}
+
+}  // namespace tqk

@@ -32,20 +32,14 @@
 #include <cfloat>
 #include <cmath>
 
+#include "tq_attn_common.cuh"
 #include "tq_internal.h"
 
 namespace tqk {
 namespace {
 
-constexpr int MW = 4;           // warps per CTA
-constexpr int MT = 16;          // tokens per tile
 constexpr int NST = 4;          // pipeline stages per warp
-constexpr int D = 128;
 constexpr int KW = 8;           // key code words per token (2-bit fields)
-constexpr int QW = 4;           // QJL words per token (m = 128)
-constexpr int VW = 16;          // value code words per token (4-bit fields)
-constexpr int VROW = 20;        // padded value row (words): conflict-free LDS.64
-
 struct Stage {
   uint32_t k[MT][KW];           // 512 B
   uint32_t q[MT][QW];           // 256 B
@@ -57,87 +51,8 @@ struct Stage {
 };
 static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
 
-constexpr int LUT_WORDS = 256 * 32;
 constexpr size_t SMEM_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST * sizeof(Stage);
 
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
-  uint32_t y;
-  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
-  return v;
-}
-
-// ---------------------------------------------------------------------------
-// Key operands.  A query head takes two B columns of the key MMA: the fp16
-// head of its operand and the fp16 tail (x 2^12), so one MMA yields both
-// products of every k-step and the fp32 sum restores ~22 bits.
-//
-// Keys use exact binary A operands.  A symmetric 2-bit codebook is affine in
-// the index bits, c[i0 + 2 i1] = c0 + (c1 - c0) i0 + (c2 - c0) i1, so
-//   <q', c[idx]> = c0 sum_j q'_j + (c1 - c0) <q', i0> + (c2 - c0) <q', i1>,
-// and the QJL term is <s, sigma> = 2 <s, bit> - sum_i s_i.  A bit becomes an
-// fp16 operand by masking it into the exponent field: a lone bit at position
-// p in 10..14 of a half reads as 2^E(p), E = -14, -13, -11, -7, 1, and the
-// B operand carries the inverse power of two.  Four rotations of a 32-bit
-// code word and sixteen masks give sixteen half2 registers: register u holds
-// bit 10+u in its low half and bit (26+u) mod 32 in its high half.
-// ---------------------------------------------------------------------------
-__host__ __device__ constexpr int bit_pos(int u) {
-  return u < 5 ? 10 + u : (u < 10 ? 5 + u : (u < 15 ? u : 10));
-}
-__host__ __device__ constexpr int bit_rot(int u) { return u < 5 ? 0 : (u < 10 ? 5 : (u < 15 ? 10 : 15)); }
-__device__ __forceinline__ float bit_inv(int p) {
-  return p == 10 ? 16384.f : (p == 11 ? 8192.f : (p == 12 ? 2048.f : (p == 13 ? 128.f : 0.5f)));
-}
-
-struct Rot4 {
-  uint32_t r[4];
-};
-__device__ __forceinline__ Rot4 rotations(uint32_t w) {
-  return Rot4{{w, __funnelshift_r(w, w, 5), __funnelshift_r(w, w, 10), __funnelshift_r(w, w, 15)}};
-}
-template <int U>
-__device__ __forceinline__ uint32_t bit_half2(const Rot4& R) {
-  constexpr int p = bit_pos(U);
-  return R.r[bit_rot(U) / 5] & ((1u << p) | (1u << (p + 16)));
-}
-
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-// 2^e for an integer e in the normal fp32 range.
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
-// floor(log2(x)) for a positive normal float.
-__device__ __forceinline__ int ilog2f(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
 
 // ---------------------------------------------------------------------------
 // Group size <= 4, balanced segments.  The 16-token tiles of all (sequence,
@@ -157,8 +72,6 @@ __device__ __forceinline__ int ilog2f(float x) { return ((__float_as_int(x) >> 2
 // the value norms of a piece are scaled once, from the piece's largest norm,
 // so that p |v| stays below 2^15 in fp16.
 // ---------------------------------------------------------------------------
-constexpr float LAZY_TAU = 8.f;
-
 template <int G>
 __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   static_assert(G <= 4, "packed path");
@@ -169,10 +82,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
-  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
-    const int byte = e >> 5;
-    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
-  }
+  build_value_lut(lut, a.cv, tid, MW * 32);
   __syncthreads();   // the only block-wide barrier: warps run independently below
 
   const int64_t* P = a.tiles;
@@ -183,15 +93,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   int64_t x = wid * W / NW;
   const int64_t x1 = (wid + 1) * W / NW;
 
-  // Sequence holding tile x: P[b] <= x < P[b + 1].
-  int b = 0;
-  {
-    int hi = a.B;
-    while (hi - b > 1) {
-      const int mid = (b + hi) >> 1;
-      if (P[mid] <= x) b = mid; else hi = mid;
-    }
-  }
+  int b = locate_sequence(P, a.B, x);
 
   const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
   const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
@@ -441,28 +343,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
       const uint32_t pb0 = movtrans(pack_half2(p0 * (st.vn[g] * vmul), 0.f));
       const uint32_t pb1 = movtrans(pack_half2(p1 * (st.vn[g + 8] * vmul), 0.f));
 
-      // ---- values ---------------------------------------------------------------
-      const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
-      const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
-      const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
-      const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
-      const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
-                              (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
-                              (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
-                              (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
-      const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
-                              ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
-                              ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
-                              ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int k = mt >> 1;
-        const uint32_t* y = (mt & 1) ? yo : ye;
-        uint32_t av[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
-        mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
-      }
+      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
       __syncwarp();
     }
     cp_wait<0>();
@@ -507,14 +388,6 @@ constexpr int QOP_STEPS = 24;                 // 16 key k-steps + 8 QJL k-steps
 constexpr size_t SMEM8_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST8 * sizeof(Stage) +
                                (size_t)QOP_STEPS * 32 * 16 + 8 * 16 + MW * 4 + 16 * 4;
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-
 __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
   constexpr int G = 8;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -529,10 +402,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
-  for (int e = tid; e < LUT_WORDS; e += MW * 32) {
-    const int byte = e >> 5;
-    lut[e] = pack_half2(a.cv[byte & 15], a.cv[byte >> 4]);
-  }
+  build_value_lut(lut, a.cv, tid, MW * 32);
   __syncthreads();
 
   const int64_t* P = a.tiles;
@@ -542,14 +412,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
   if (cta >= NC) return;   // uniform over the CTA
   int64_t x = cta * W / NC;
   const int64_t x1 = (cta + 1) * W / NC;
-  int b = 0;
-  {
-    int hi = a.B;
-    while (hi - b > 1) {
-      const int mid = (b + hi) >> 1;
-      if (P[mid] <= x) b = mid; else hi = mid;
-    }
-  }
+  int b = locate_sequence(P, a.B, x);
 
   const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
   const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
@@ -792,28 +655,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
       const uint32_t pb0 = movtrans(pack_half2(p00 * w0s, p10 * w0s));
       const uint32_t pb1 = movtrans(pack_half2(p01 * w8s, p11 * w8s));
 
-      // ---- values ---------------------------------------------------------------
-      const uint2 xa = *reinterpret_cast<const uint2*>(&st.v[2 * t][2 * g]);
-      const uint2 xb = *reinterpret_cast<const uint2*>(&st.v[2 * t + 1][2 * g]);
-      const uint2 xc = *reinterpret_cast<const uint2*>(&st.v[2 * t + 8][2 * g]);
-      const uint2 xd = *reinterpret_cast<const uint2*>(&st.v[2 * t + 9][2 * g]);
-      const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
-                              (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
-                              (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
-                              (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
-      const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
-                              ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
-                              ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
-                              ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int kk = mt >> 1;
-        const uint32_t* y = (mt & 1) ? yo : ye;
-        uint32_t av[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + kk) * 128u + lut_lane);
-        mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
-      }
+      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
       __syncwarp();
     }
     cp_wait<0>();

@@ -149,6 +149,11 @@ bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
 // Upper bound on the warps of a segment-path launch (sizes the partials).
 int64_t attn_seg_max_warps(const tq_ctx* c);
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+// Tensor-core decode path for 3-bit Lloyd-Max keys (k4v4: d = 128, keys 3 + 1
+// QJL bit with m = 128, values 4 bits, group 8); needs AttnArgs::tiles.
+bool attn_k4_supported(const tq_ctx* c, const AttnArgs& a);
+cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+cudaError_t configure_attn_k4();
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
                           const float* krnorm, int64_t nk, float* out, cudaStream_t s);

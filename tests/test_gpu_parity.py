@@ -164,7 +164,8 @@ def test_attention_single_head(cuda):
     (128, 4, 2, 3, 4, 128, 1100),   # tensor-core path, group 2
     (128, 16, 2, 3, 4, 128, 1100),  # tensor-core path, group 8
     (128, 8, 2, 3, 4, 128, 1002),   # max_T % 4 != 0: generic path
-    (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: generic path
+    (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: tensor-core path, group 8
+    (128, 8, 2, 4, 4, 128, 1000),   # 3-bit keys, group 4: generic path
     (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000)])
 def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
     """Ragged lengths (0, 1, odd, chunk edges, full), GQA groups 1-8, d=64/128/200."""
@@ -182,14 +183,14 @@ def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
                       out.cpu().numpy())
 
 
-@pytest.mark.parametrize("Hq,Hkv,lens_kind", [
-    (8, 2, "mixed"), (16, 2, "mixed"), (4, 4, "mixed"), (2, 1, "mixed"),
-    (8, 2, "tiny"), (16, 2, "tiny")])
-def test_attention_many_short_rows(cuda, Hq, Hkv, lens_kind):
-    """Tensor-core path with many short sequences: the balanced tile ranges
+@pytest.mark.parametrize("Hq,Hkv,lens_kind,bk", [
+    (8, 2, "mixed", 3), (16, 2, "mixed", 3), (4, 4, "mixed", 3), (2, 1, "mixed", 3),
+    (8, 2, "tiny", 3), (16, 2, "tiny", 3), (16, 2, "mixed", 4), (16, 2, "tiny", 4)])
+def test_attention_many_short_rows(cuda, Hq, Hkv, lens_kind, bk):
+    """Tensor-core paths with many short sequences: the balanced tile ranges
     cross many (sequence, kv head) rows, and with tiny lengths there are
     fewer tiles than warps."""
-    c = _ctx(128, 3, 4, 128, seed=5)
+    c = _ctx(128, bk, 4, 128, seed=5)
     tab = P.oracle_tables(c)
     B, T = 37, 256
     g = torch.Generator().manual_seed(11)
