@@ -6,10 +6,11 @@
 // both products are GEMMs over a tile of 128 vectors:
 //   D_rot[v][j] = sum_k x[v][k] Pi'[j][k]      (M = 128 vectors, N = K = 128)
 //   D_qjl[v][i] = sum_k r[v][k] S[i][k]
-// issued by one thread per warpgroup with operands in shared memory (128-byte
-// swizzled, K-major) and fp32 accumulators in tensor memory.  Thread v of the
-// warpgroup owns TMEM lane v, i.e. one whole vector, so index computation and
-// bit packing need no cross-thread exchange.
+// issued by one thread per tile group with operands in shared memory (128-byte
+// swizzled, K-major) and fp32 accumulators in tensor memory.  TMEM lane v
+// holds vector v; two threads own it, one per half of the coordinates, so
+// index computation and bit packing need no cross-thread exchange (a packed
+// word never spans the halves) and only the two norms are combined.
 //
 // Exactness.  x (bf16 or fp16) is exact in fp16 after a per-vector power of
 // two scale.  Pi' = 2^8 Pi is split into an fp16 head and tail; both products
@@ -20,9 +21,10 @@
 // operand and accumulation rounding of the tensor-core product (a few bits
 // per thousand vectors).
 //
-// Two warpgroups per CTA work on different tiles, so one group's MMAs overlap
-// the other's epilogue.  Waits on MMA completion are bounded; on timeout the
-// kernel records a fault code, releases its tensor memory and returns.
+// Two groups of eight warps per CTA work on different tiles, so one group's
+// MMAs overlap the other's epilogue, and sixteen warps per SM hide latency.
+// Waits on MMA completion are bounded; on timeout the kernel records a fault
+// code, releases its tensor memory and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -80,24 +82,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return false;
 }
 
-// True on every thread of the warpgroup if any of its threads passes true.
-__device__ __forceinline__ bool wg_any(int wg, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(1 + wg)
-      : "memory");
-  return r != 0u;
-}
-
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void wg_sync(int wg) {
-  asm volatile("bar.sync %0, 128;\n" ::"r"(1 + wg) : "memory");
-}
 
 // 32 fp32 columns [col, col+32) of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -202,8 +189,37 @@ __device__ __noinline__ Q4 qjl_fixup(uint32_t taddr, float inv, float pmid, cons
   return qw;
 }
 
+// Thread (group gi, half h, row r): two groups of eight warps per CTA work on
+// different tiles; within a group, warps w and w + 4 share TMEM lanes 32 (w &
+// 3) .. + 31 (one vector per lane) and take coordinate halves h = 0, 1
+// (columns 64h .. 64h + 63 of every accumulator).  The two threads of a
+// vector exchange partial sums through two TMEM columns of their lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n" ::"r"(taddr), "r"(__float_as_uint(v))
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ float tmem_sum2(uint32_t taddr) {
+  uint32_t r0, r1;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+  return __uint_as_float(r0) + __uint_as_float(r1);
+}
+__device__ __forceinline__ void grp_sync(int gi) { asm volatile("bar.sync %0, 256;\n" ::"r"(1 + gi) : "memory"); }
+// True on every thread of the group if any of its threads passes true.
+__device__ __forceinline__ bool grp_any(int gi, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(1 + gi)
+      : "memory");
+  return r != 0u;
+}
+
 template <int BITS, bool QJL>
-__global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
+__global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -212,9 +228,11 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
   float* s_cen = s_snorm + 128;                                        // [16]
   float* s_pb = s_cen + 16;                                            // [8]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + OFF_MISC + 32);
-  const uint32_t bar0 = base_s + OFF_MISC;   // 4 barriers: rot wg0, rot wg1, qjl wg0, qjl wg1
+  const uint32_t bar0 = base_s + OFF_MISC;   // 4 barriers: rot g0, rot g1, qjl g0, qjl g1
 
-  const int tid = threadIdx.x, wg = tid >> 7, row = tid & 127, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gi = tid >> 8, wq = (tid >> 5) & 7, h = wq >> 2;
+  const int row = 32 * (wq & 3) + lane;
   constexpr int L = 1 << BITS;
   constexpr int PER = (BITS == 3) ? 16 : 32 / BITS;   // fields per word of the main stream
   constexpr int W_MAIN = 128 / PER;                     // words of the main stream
@@ -226,7 +244,7 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
     const int4* src_pil = reinterpret_cast<const int4*>(a.pi_lo);
     const int4* src_s = reinterpret_cast<const int4*>(a.s_img);
     int4* dst = reinterpret_cast<int4*>(base);
-    for (int e = tid; e < (int)(SMEM_TILE / 16); e += 256) {
+    for (int e = tid; e < (int)(SMEM_TILE / 16); e += 512) {
       dst[OFF_PIH / 16 + e] = src_pih[e];
       dst[OFF_PIL / 16 + e] = src_pil[e];
       if (QJL) dst[OFF_S / 16 + e] = src_s[e];
@@ -252,13 +270,16 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
   tc_after_sync();
   const uint32_t tmem = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-  const uint32_t d_rot = tmem + (uint32_t)(wg * 256);
+  const uint32_t d_rot = tmem + (uint32_t)(gi * 256);
   const uint32_t d_qjl = d_rot + 128;
-  const uint32_t sA = base_s + OFF_A + wg * 2 * SMEM_TILE;
-  unsigned char* A = base + OFF_A + wg * 2 * SMEM_TILE;
+  // Two columns of the QJL accumulator (free outside the QJL product) carry
+  // the halves' partial sums.
+  const uint32_t x_col = d_qjl + lane_base;
+  const uint32_t sA = base_s + OFF_A + gi * 2 * SMEM_TILE;
+  unsigned char* A = base + OFF_A + gi * 2 * SMEM_TILE;
   unsigned char* A2 = A + SMEM_TILE;
-  const uint32_t bar_rot = bar0 + 8 * wg, bar_q = bar0 + 16 + 8 * wg;
-  const bool leader = row == 0;
+  const uint32_t bar_rot = bar0 + 8 * gi, bar_q = bar0 + 16 + 8 * gi;
+  const bool leader = (tid & 255) == 0;
   const float* pb = s_pb;
   float snorm_max = 0.f;
   if (QJL)
@@ -274,23 +295,26 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
   auto hi_f = [&](uint32_t w) {
     return is_bf ? __uint_as_float(w & 0xFFFF0000u) : __half2float(__ushort_as_half((unsigned short)(w >> 16)));
   };
-  uint4 xr[16];
-  auto load_x = [&](int64_t t) {
+  // This half's 64 coordinates of vector `row` of tile t (zeros past the end).
+  auto load_x = [&](int64_t t, uint4 (&xr)[8]) {
     const int64_t vv = t * TILE + row;
     if (vv < a.n) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.x) + vv * a.ld);
+      const uint4* src =
+          reinterpret_cast<const uint4*>(static_cast<const unsigned short*>(a.x) + vv * a.ld + 64 * h);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) xr[c] = src[c];
+      for (int c = 0; c < 8; ++c) xr[c] = src[c];
     } else {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) xr[c] = make_uint4(0, 0, 0, 0);
+      for (int c = 0; c < 8; ++c) xr[c] = make_uint4(0, 0, 0, 0);
     }
   };
   uint32_t iter = 0;
   bool fault = false;
-  for (int64_t tile = (int64_t)blockIdx.x * 2 + wg; tile < ntiles; tile += tstride, ++iter) {
+  for (int64_t tile = (int64_t)blockIdx.x * 2 + gi; tile < ntiles; tile += tstride, ++iter) {
     const int64_t v = tile * TILE + row;
     const bool live = v < a.n;
+    uint4 xr[8];
+    load_x(tile, xr);
     {
       const int64_t nxt = tile + tstride;
       if (leader && a.ld == 128 && nxt < ntiles) {
@@ -300,11 +324,10 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
       }
     }
-    load_x(tile);
-    // ---- norm and the scaled fp16 operand ------------------------------------------
+    // ---- this half's 64 coordinates, the norm, the scaled fp16 operand ---------------
     float ssp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < 8; ++c) {
       const uint32_t w4[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -313,22 +336,26 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
         ssp[q] = fmaf(f1, f1, ssp[q]);
       }
     }
-    const float nrm = sqrtf((ssp[0] + ssp[1]) + (ssp[2] + ssp[3]));
+    tmem_st1(x_col + h, (ssp[0] + ssp[1]) + (ssp[2] + ssp[3]));
+    tc_before_sync();
+    grp_sync(gi);
+    tc_after_sync();
+    const float nrm = sqrtf(tmem_sum2(x_col));
     const int e = nrm > 0.f ? 14 - flog2(nrm) : 0;
     const float sc = pow2f(e);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 0; c < 8; ++c) {
       const uint32_t w4[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
       uint4 o;
       o.x = h2bits(lo_f(w4[0]) * sc, hi_f(w4[0]) * sc);
       o.y = h2bits(lo_f(w4[1]) * sc, hi_f(w4[1]) * sc);
       o.z = h2bits(lo_f(w4[2]) * sc, hi_f(w4[2]) * sc);
       o.w = h2bits(lo_f(w4[3]) * sc, hi_f(w4[3]) * sc);
-      *reinterpret_cast<uint4*>(A + chunk_off(row, c)) = o;
+      *reinterpret_cast<uint4*>(A + chunk_off(row, 8 * h + c)) = o;
     }
     fence_async_smem();
     tc_before_sync();
-    wg_sync(wg);
+    grp_sync(gi);
     // ---- rotation: D_rot = A (Pi'_hi + Pi'_lo)^T -----------------------------------
     if (leader) {
       tc_after_sync();
@@ -340,17 +367,17 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
       }
       mma_commit(bar_rot);
     }
-    if (wg_any(wg, !mbar_wait(bar_rot, iter & 1))) { fault = true; break; }
+    if (grp_any(gi, !mbar_wait(bar_rot, iter & 1))) { fault = true; break; }
     tc_after_sync();
 
-    // ---- epilogue 1: indices, packing, residual (32 coordinates per pass) -------------
+    // ---- epilogue 1: indices, packing, residual (this half's two 32-column chunks) ----
     // y = D_rot / (sc * nrm * 2^8); the residual goes out scaled by 2^14.
     const float inv = nrm > 0.f ? 1.f / (sc * nrm * 256.f) : 0.f;
     const int64_t rec = live ? out_rec(a, v) : 0;
     uint32_t* crow = a.codes + rec * WORDS;
     float rho2v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 2 * h; ch < 2 * h + 2; ++ch) {
       float d[32];
       tmem_ld32(d_rot + lane_base + ch * 32, d);
       // words of this chunk: b words of b-bit fields (b = 3: two 2-bit words + one bit word)
@@ -387,9 +414,9 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float r0 = d[8 * q + 2 * u], r1 = d[8 * q + 2 * u + 1];
-            const __half2 h = __floats2half2_rn(r0, r1);
-            const float2 f = __half22float2(h);
-            hv[u] = *reinterpret_cast<const uint32_t*>(&h);
+            const __half2 hh = __floats2half2_rn(r0, r1);
+            const float2 f = __half22float2(hh);
+            hv[u] = *reinterpret_cast<const uint32_t*>(&hh);
             lv[u] = h2bits(r0 - f.x, r1 - f.y);
           }
           *reinterpret_cast<uint4*>(A + chunk_off(row, ch * 4 + q)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
@@ -397,15 +424,20 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
         }
       }
     }
-    if (live) a.norm[rec] = nrm;
+    if (live && h == 0) a.norm[rec] = nrm;
     if (!QJL) {
       tc_before_sync();
-      wg_sync(wg);   // A and D_rot are free for the next tile
+      grp_sync(gi);   // A and D_rot are free for the next tile
       continue;
     }
+    tmem_st1(x_col + h, (rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3]));
     fence_async_smem();
     tc_before_sync();
-    wg_sync(wg);
+    grp_sync(gi);
+    tc_after_sync();
+    const float rho = sqrtf(tmem_sum2(x_col)) * (1.f / 16384.f);
+    tc_before_sync();
+    grp_sync(gi);   // the partial sums are read before the QJL product overwrites them
     // ---- QJL product: D_qjl = (2^14 r) S^T ----------------------------------------------
     if (leader) {
       tc_after_sync();
@@ -417,22 +449,28 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
       }
       mma_commit(bar_q);
     }
-    if (wg_any(wg, !mbar_wait(bar_q, iter & 1))) { fault = true; break; }
+    if (grp_any(gi, !mbar_wait(bar_q, iter & 1))) { fault = true; break; }
     tc_after_sync();
-    const float rho = sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) * (1.f / 16384.f);
     // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho.
     const float thr = 0.125f * rho * snorm_max;
     uint32_t qw[4] = {0u, 0u, 0u, 0u};
     uint32_t flag[4] = {0u, 0u, 0u, 0u};
+    // Bit i = sign bit of D_i (then inverted: 1 <=> D_i >= 0) and of thr - |D_i|
+    // (inverted: 1 <=> |D_i| <= thr), shifted in from the top, row 31 first.  A
+    // D_i of -0 reads as negative here, but |D_i| <= thr flags it for the exact
+    // recomputation below.
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int c2 = 0; c2 < 2; ++c2) {
       float d[32];
-      tmem_ld32(d_qjl + lane_base + ch * 32, d);
+      tmem_ld32(d_qjl + lane_base + (2 * h + c2) * 32, d);
+      uint32_t sg = 0u, fl = 0u;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        qw[ch] |= (d[i] >= 0.f ? 1u : 0u) << i;
-        flag[ch] |= (fabsf(d[i]) <= thr ? 1u : 0u) << i;
+      for (int i = 31; i >= 0; --i) {
+        sg = __funnelshift_l(__float_as_uint(d[i]), sg, 1);   // (sg << 1) | sign bit
+        fl = __funnelshift_l(__float_as_uint(thr - fabsf(d[i])), fl, 1);
       }
+      qw[2 * h + c2] = ~sg;
+      flag[2 * h + c2] = ~fl;
     }
     if (!live) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
     if (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
@@ -443,11 +481,11 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
       for (int w = 0; w < 4; ++w) qw[w] = fixed.w[w];
     }
     if (live) {
-      *reinterpret_cast<uint4*>(a.qjl + rec * 4) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
-      a.rnorm[rec] = nrm * rho;
+      *reinterpret_cast<uint2*>(a.qjl + rec * 4 + 2 * h) = make_uint2(qw[2 * h], qw[2 * h + 1]);
+      if (h == 0) a.rnorm[rec] = nrm * rho;
     }
     tc_before_sync();
-    wg_sync(wg);
+    grp_sync(gi);
   }
   if (fault) atomicExch(&g_tq_fault, 1);
   tc_before_sync();
@@ -461,9 +499,9 @@ __global__ void __launch_bounds__(256, 1) k_quant_tc(QuantTcArgs a) {
 template <int BITS>
 cudaError_t launch_bits(const QuantTcArgs& a, bool qjl, int grid, cudaStream_t s) {
   if (qjl) {
-    k_quant_tc<BITS, true><<<grid, 256, TC_SMEM, s>>>(a);
+    k_quant_tc<BITS, true><<<grid, 512, TC_SMEM, s>>>(a);
   } else {
-    k_quant_tc<BITS, false><<<grid, 256, TC_SMEM, s>>>(a);
+    k_quant_tc<BITS, false><<<grid, 512, TC_SMEM, s>>>(a);
   }
   return cudaGetLastError();
 }
