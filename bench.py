@@ -1,10 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of compressed decode attention over a packed KV cache on B200.
 
-One step = one decode step of the whole hot path for a batch of sequences:
-quantize the newest token's K and V into the packed cache (rotation, Lloyd-Max
-codes, QJL sketch), pre-rotate the queries, split-K attention straight from
-the packed codes, log-sum-exp merge and the final inverse rotation.
+One step = one decode step of the whole hot path for a batch of sequences, in
+one tq_decode_step call (three launches): quantize the newest token's K and V
+into the packed cache (rotation, Lloyd-Max codes, QJL sketch) and pre-rotate
+the queries, split-K attention straight from the packed codes, log-sum-exp
+merge and the final inverse rotation.
 
 Headline `value`: KV tokens attended per second (B * T per step) with the
 packed cache and the step inputs resident in HBM.  `e2e`: the same metric with
@@ -399,41 +400,33 @@ def run_gpu(args, w):
     lens = torch.full((B,), T, dtype=torch.int32, device=dev)
     out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
     ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
-    launches_per_step = 2 + 3  # append K, append V, prerotate + split attention + merge
+    launches_per_step = 3  # append + pre-rotate, attention, merge (tq_decode_step)
 
-    # Each step replays two CUDA graphs (quantize-append of the new K/V token,
-    # then the attention call), so host launch latency is not timed; events
-    # between the replays time the attention call alone for the roofline.
-    def append(j):
-        ctx.quantize_append(kn[j], tq.TQ_KEY, kc, pos)
-        ctx.quantize_append(vn[j], tq.TQ_VALUE, vc, pos)
+    # Each step replays one CUDA graph of tq_decode_step (append the new K/V
+    # token at slot T-1, then attend over all T tokens), so host launch latency
+    # is not timed.  The attention call alone (pre-rotate + attention + merge,
+    # tq_attn_decode) is timed in a second loop over the same inputs, with
+    # events around every replay, for the roofline.
+    def step_body(j):
+        ctx.decode_step(qs[j], kn[j], vn[j], kc, vc, pos, out=out, workspace=ws)
 
     def attend(j):
         ctx.attn_decode(qs[j], kc, vc, lens, out=out, workspace=ws)
 
     for j in range(POOL):           # eager warm-up before capture
-        append(j)
+        step_body(j)
         attend(j)
     torch.cuda.synchronize()
-    g_app, g_att = [], []
+    g_step, g_att = [], []
     for j in range(POOL):
         ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(ga):
-            append(j)
+            step_body(j)
         with torch.cuda.graph(gb):
             attend(j)
-        g_app.append(ga)
+        g_step.append(ga)
         g_att.append(gb)
     torch.cuda.synchronize()
-
-    def step(i, ev=None):
-        j = i % POOL
-        g_app[j].replay()
-        if ev is not None:
-            ev[0].record()
-        g_att[j].replay()
-        if ev is not None:
-            ev[1].record()
 
     def barrier():
         if world > 1:
@@ -443,20 +436,33 @@ def run_gpu(args, w):
     sampler = ClockSampler(local)
     sampler.start()
     for i in range(args.warmup):
-        step(i)
+        g_step[i % POOL].replay()
     barrier()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.time()
     torch.cuda.nvtx.range_push("tq:decode_steps")
     e0.record()
     for i in range(args.steps):
-        step(i, evs[i])
+        g_step[i % POOL].replay()
     e1.record()
     torch.cuda.nvtx.range_pop()
     barrier()
     sampler.mark(w0, time.time())
     t_ms = e0.elapsed_time(e1) / args.steps
+
+    for i in range(args.warmup):
+        g_att[i % POOL].replay()
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    w0 = time.time()
+    torch.cuda.nvtx.range_push("tq:attention_calls")
+    for i in range(args.steps):
+        evs[i][0].record()
+        g_att[i % POOL].replay()
+        evs[i][1].record()
+    torch.cuda.nvtx.range_pop()
+    barrier()
+    sampler.mark(w0, time.time())
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
 
     # End to end through the public API with host buffers: pinned host inputs
@@ -472,9 +478,7 @@ def run_gpu(args, w):
         dq.copy_(hq[j], non_blocking=True)
         dk.copy_(hk[j], non_blocking=True)
         dv.copy_(hv[j], non_blocking=True)
-        ctx.quantize_append(dk, tq.TQ_KEY, kc, pos)
-        ctx.quantize_append(dv, tq.TQ_VALUE, vc, pos)
-        ctx.attn_decode(dq, kc, vc, lens, out=out, workspace=ws)
+        ctx.decode_step(dq, dk, dv, kc, vc, pos, out=out, workspace=ws)
         hout.copy_(out, non_blocking=True)
 
     e2e_body(0)
@@ -498,7 +502,7 @@ def run_gpu(args, w):
     e2e_ms = e0.elapsed_time(e1) / args.steps
     h2d = hq[0].numel() * hq[0].element_size() + 2 * hk[0].numel() * hk[0].element_size()
     d2h = hout.numel() * hout.element_size()
-    del g_app, g_att, g_e2e
+    del g_step, g_att, g_e2e
 
     torch.cuda.nvtx.range_push("tq:quantize_sweep")
     quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
@@ -533,7 +537,8 @@ def run_gpu(args, w):
             "config": config_of(args, w),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic,
-                         "kernel": "tq_attn_decode (pre-rotate + split-K attention + merge)",
+                         "kernel": "tq_attn_decode (pre-rotate + split-K attention + merge), "
+                                   "timed in its own loop of K graph replays",
                          "algorithmic_bytes_per_launch": alg, "launch_ms": attn_ms,
                          "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                          "frac_of_nominal_8tbs": achieved / 8000.0},

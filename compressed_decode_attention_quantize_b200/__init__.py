@@ -61,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "tq_attn_decode": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P, SZ, P]),
         "tq_attn_decode_static": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P]),
         "tq_attn_static_scratch_bytes": (SZ, []),
+        "tq_decode_step": (I, [P, P, I, P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P, SZ, P]),
         "tq_topk_workspace_bytes": (SZ, [P, I64, I64, I]),
         "tq_topk": (I, [P, P, I, I64, P, P, P, P, I64, I, P, P, P, SZ, P]),
     }
@@ -75,7 +76,7 @@ _lib = _load()
 EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
             "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
-            "tq_attn_static_scratch_bytes", "tq_topk_workspace_bytes", "tq_topk")
+            "tq_attn_static_scratch_bytes", "tq_decode_step", "tq_topk_workspace_bytes", "tq_topk")
 
 
 def library_path() -> str:
@@ -263,6 +264,31 @@ class Context:
                                    _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(kcache["norm"]),
                                    _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
                                    max_T, _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+        return out
+
+    def decode_step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, kcache: dict,
+                    vcache: dict, pos: torch.Tensor, scale: float | None = None,
+                    out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+        """Append k_new / v_new [B, Hkv, d] at slot pos[b] of the caches, then
+        attend q [B, Hq, d] over tokens [0, pos[b]] (tq_decode_step)."""
+        q, k_new, v_new = q.contiguous(), k_new.contiguous(), v_new.contiguous()
+        B, Hq, d = q.shape
+        Hkv, max_T = kcache["norm"].shape[1], kcache["norm"].shape[2]
+        if k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) or k_new.dtype != v_new.dtype:
+            raise TQError(TQ_ERR_ARG, "decode_step: k_new / v_new must both be [B, Hkv, d] of one dtype")
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        need = self.attn_workspace_bytes(B, Hq, max_T)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _check(_lib.tq_decode_step(self.ptr, _ptr(q), _DTYPES[q.dtype], _ptr(k_new), _ptr(v_new),
+                                   _DTYPES[k_new.dtype], B, Hq, Hkv, _ptr(kcache["codes"]),
+                                   _ptr(kcache["qjl"]), _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
+                                   _ptr(vcache["codes"]), _ptr(vcache["norm"]), max_T, _ptr(pos),
+                                   float(scale), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
         return out
 

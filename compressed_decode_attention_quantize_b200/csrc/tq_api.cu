@@ -418,14 +418,14 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
   return TQ_OK;
 }
 
-// Workspace: [q' and S q' rows][tile prefix][partials].  The partials are
+// Workspace: [q' and S q' rows][tile prefix][step lengths][partials].  The partials are
 // sized for the larger of the split layout ([B Hq][splits][dpad + 2]) and
 // the segment layouts: [warps + B Hkv][G][dpad + 2] for groups up to 4, and
 // [4 (CTAs + B Hkv)][8][dpad + 2] for group 8; both are at most
 // [8 warps + 4 B Hq][dpad + 2].
 namespace {
 struct AttnWs {
-  size_t q_bytes, tiles_off, part_off, total;
+  size_t q_bytes, tiles_off, lens_off, part_off, total;
 };
 AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   int chunk = 0;
@@ -438,7 +438,8 @@ AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   AttnWs w;
   w.q_bytes = 2 * rows * c->dpad * sizeof(float);
   w.tiles_off = (w.q_bytes + 255) & ~(size_t)255;
-  w.part_off = (w.tiles_off + ((size_t)B + 1) * sizeof(int64_t) + 255) & ~(size_t)255;
+  w.lens_off = (w.tiles_off + ((size_t)B + 1) * sizeof(int64_t) + 255) & ~(size_t)255;
+  w.part_off = (w.lens_off + (size_t)B * sizeof(int32_t) + 255) & ~(size_t)255;
   w.total = w.part_off + (split_part > seg_part ? split_part : seg_part) + 256;
   return w;
 }
@@ -516,6 +517,118 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   e = mma ? tqk::launch_attn_mma(c, a, out, s)
           : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
   if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
+  return TQ_OK;
+}
+
+int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
+                   int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
+                   float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm, int64_t max_T,
+                   const int32_t* pos, float scale, float* out, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  if (int r = check_ctx(c)) return r;
+  for (int dt : {q_dtype, kv_dtype})
+    if (dt != TQ_F32 && dt != TQ_BF16 && dt != TQ_F16) return fail(TQ_ERR_ARG, "tq_decode_step: bad dtype=%d", dt);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "tq_decode_step: bad sizes");
+  if (Hq % Hkv != 0 || Hq / Hkv > 16)
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", Hq, Hkv);
+  if (B == 0) return TQ_OK;
+  if (!q || !k_new || !v_new || !kcodes || !knorm || !vcodes || !vnorm || !pos || !out)
+    return fail(TQ_ERR_ARG, "tq_decode_step: null pointer");
+  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_decode_step: keys with QJL need kqjl and krnorm");
+  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: B or Hkv too large");
+  if (!aligned(kcodes, 4) || !aligned(knorm, 4) || !aligned(vcodes, 4) || !aligned(vnorm, 4))
+    return fail(TQ_ERR_ARG, "tq_decode_step: misaligned cache");
+  const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
+  if (!workspace || ws_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "tq_decode_step: workspace %zu bytes < %zu", ws_bytes, need);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_decode_step: workspace not 256-byte aligned");
+  cudaStream_t s = as_stream(stream);
+  const size_t rows = (size_t)B * Hq;
+  const AttnWs lay = attn_ws_layout(c, B, Hq, max_T);
+  char* p = static_cast<char*>(workspace);
+  float* qr = reinterpret_cast<float*>(p);
+  float* qs = qr + rows * c->dpad;
+  int32_t* lens = reinterpret_cast<int32_t*>(p + lay.lens_off);
+
+  auto qargs = [&](bool key) {
+    tqk::QuantArgs a{};
+    a.x = key ? k_new : v_new;
+    a.dtype = kv_dtype;
+    a.n = (int64_t)B * Hkv;
+    a.ld = c->d;
+    a.d = c->d;
+    a.bits = key ? c->bk_lm : c->bits_v;
+    a.nbnd = (1 << a.bits) - 1;
+    a.m = key ? c->qjl_m : 0;
+    a.words = key ? c->wk : c->wv;
+    a.PiT = c->PiT;
+    a.ST = c->ST;
+    a.cen = key ? c->ck_f : c->cv_f;
+    a.bnd = key ? c->bk_f : c->bv_f;
+    a.codes = key ? kcodes : vcodes;
+    a.qjl = key ? kqjl : nullptr;
+    a.norm = key ? knorm : vnorm;
+    a.rnorm = key ? krnorm : nullptr;
+    a.pos = pos;
+    a.H = Hkv;
+    a.max_T = max_T;
+    return a;
+  };
+  tqk::AttnArgs a{};
+  a.qr = qr;
+  a.qs = qs;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.d = c->d;
+  a.bk = c->bk_lm;
+  a.bv = c->bits_v;
+  a.m = c->qjl_m;
+  a.wk = c->wk;
+  a.wv = c->wv;
+  a.kcodes = kcodes;
+  a.kqjl = kqjl;
+  a.knorm = knorm;
+  a.krnorm = krnorm;
+  a.vcodes = vcodes;
+  a.vnorm = vnorm;
+  a.max_T = max_T;
+  a.seq_lens = lens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
+  a.ck = c->ck_f;
+  a.cv = c->cv_f;
+  a.splits = tqk::attn_splits(c, B, Hkv, max_T, &a.chunk);
+  a.part = reinterpret_cast<float*>(p + lay.part_off);
+  a.tiles = nullptr;
+  const bool mma = tqk::attn_mma_supported(c, a);
+  const bool k4 = !mma && tqk::attn_k4_supported(c, a);
+  if (mma || k4) {
+    a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
+  } else if (a.splits > 4096) {
+    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: too many splits");
+  }
+  tqk::StepPrep sp{};
+  sp.k = qargs(true);
+  sp.v = qargs(false);
+  sp.q = q;
+  sp.qdtype = q_dtype;
+  sp.qrows = (int64_t)rows;
+  sp.qr = qr;
+  sp.qs = qs;
+  sp.pos = pos;
+  sp.lens = lens;
+  sp.B = B;
+  sp.Hkv = Hkv;
+  sp.max_T = max_T;
+  sp.tiles = a.tiles;
+  sp.nkv = (int64_t)B * Hkv;
+  cudaError_t e = tqk::launch_step_prep(c, sp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step: prepare");
+  e = mma ? tqk::launch_attn_mma(c, a, out, s)
+          : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step");
   return TQ_OK;
 }
 

@@ -137,6 +137,24 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
 cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s);
 cudaError_t configure_quant_tc();
 cudaError_t read_and_clear_fault(int* value);
+// One launch before a fused decode step: append the new K and V vectors (one
+// per (sequence, kv head)), pre-rotate the queries, write the attention
+// lengths (and the tile prefix when tiles != null).
+struct StepPrep {
+  QuantArgs k, v;
+  const void* q;
+  int qdtype;
+  int64_t qrows;
+  float* qr;
+  float* qs;
+  const int32_t* pos;
+  int32_t* lens;
+  int B, Hkv;
+  int64_t max_T;
+  int64_t* tiles;
+  int64_t nkv;
+};
+cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s);
 // With plan != null the kernel also writes plan->tiles (the segment path's
 // tile prefix) from plan->seq_lens, B, Hkv and max_T.
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,

@@ -47,10 +47,13 @@ __device__ __forceinline__ int lm_index(float y, const float* sb, int nb) {
 }
 
 // Output record of input row v (cache placement when a.pos is set).
+// Output record of vector v: v itself, or for cache appends slot pos[b] of
+// row v = b H + g; -1 (nothing written) when pos[b] is outside [0, max_T).
 __device__ __forceinline__ int64_t out_record(const QuantArgs& a, int64_t v) {
   if (a.pos == nullptr) return v;
   const int64_t b = v / a.H;
-  return v * a.max_T + a.pos[b];
+  const int64_t p = a.pos[b];
+  return (p >= 0 && p < a.max_T) ? v * a.max_T + p : -1;
 }
 
 // Lloyd-Max index of coordinate j of a packed vector (b-bit fields; for b = 3
@@ -212,8 +215,9 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
     // fills one word (b = 3: 2-bit stream of low bits, then 1-bit stream).
 #pragma unroll
     for (int v = 0; v < QV; ++v) {
-      const bool live = v0 + v < a.n;
-      const int64_t base = live ? out_record(a, v0 + v) * a.words : 0;
+      const int64_t rec = v0 + v < a.n ? out_record(a, v0 + v) : -1;
+      const bool live = rec >= 0;
+      const int64_t base = live ? rec * a.words : 0;
 #pragma unroll
       for (int i = 0; i < J; ++i) {
         const uint32_t iv = (lane + 32 * i < a.d) ? idx[i][v] : 0u;
@@ -236,7 +240,10 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 #pragma unroll
     for (int v = 0; v < QV; ++v)
       if (lane == v) my_norm = nrm[v];
-    if (lane < QV && v0 + lane < a.n) a.norm[out_record(a, v0 + lane)] = my_norm;
+    if (lane < QV && v0 + lane < a.n) {
+      const int64_t rec = out_record(a, v0 + lane);
+      if (rec >= 0) a.norm[rec] = my_norm;
+    }
     if (a.m == 0) { __syncwarp(); continue; }
 
     // Stage 2: residual r = y - c[idx], rho = |r|, QJL bits sign(S r).
@@ -279,13 +286,19 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
         const uint32_t w = __ballot_sync(0xffffffffu, bit);
         if (lane == i) mine = w;
       }
-      if (v0 + v < a.n && lane < mwords) a.qjl[out_record(a, v0 + v) * mwords + lane] = mine;
+      if (v0 + v < a.n && lane < mwords) {
+        const int64_t rec = out_record(a, v0 + v);
+        if (rec >= 0) a.qjl[rec * mwords + lane] = mine;
+      }
     }
     float my_rn = 0.f;
 #pragma unroll
     for (int v = 0; v < QV; ++v)
       if (lane == v) my_rn = nrm[v] * sqrtf(rr[v]);
-    if (lane < QV && v0 + lane < a.n) a.rnorm[out_record(a, v0 + lane)] = my_rn;
+    if (lane < QV && v0 + lane < a.n) {
+      const int64_t rec = out_record(a, v0 + lane);
+      if (rec >= 0) a.rnorm[rec] = my_rn;
+    }
     __syncwarp();
   }
 }
@@ -296,14 +309,15 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 // and S once for all QS vectors, and a few hundred vectors spread over many
 // SMs instead of filling one tile.  Same fp32 arithmetic as above.
 // ----------------------------------------------------------------------------
+// Block blk of the small-batch quantizer; sh = [QS][dpad] (x, later r) then
+// [2][MV_KC][dpad] matrix chunks.  blockDim = dpad.
 template <int QS>
-__global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
-  extern __shared__ float sh[];   // [QS][dpad]: x, later r; then [2][MV_KC][dpad] matrix chunks
+__device__ __forceinline__ void quantize_small_body(const QuantArgs& a, int dpad, int64_t blk, float* sh) {
   float* Ms = sh + QS * dpad;
   __shared__ float red[QS][8];
   __shared__ float s_cen[16], s_bnd[16];
   const int j = threadIdx.x, lane = j & 31, warp = j >> 5, nwarp = blockDim.x >> 5;
-  const int64_t v0 = (int64_t)blockIdx.x * QS;
+  const int64_t v0 = blk * QS;
   const int nv = (int)min((int64_t)QS, a.n - v0);
   if (j < 16) {
     s_cen[j] = (j < (1 << a.bits)) ? a.cen[j] : 0.f;
@@ -338,6 +352,7 @@ __global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
     r[u] = (j < a.d) ? y - s_cen[idx] : 0.f;
     if (u >= nv) continue;   // uniform over the block
     const int64_t rec = out_record(a, v0 + u);
+    if (rec < 0) continue;   // uniform too (one sequence per vector)
     // b-bit field packing within each warp (b = 3: 2-bit stream, then 1-bit stream)
     const uint32_t iv = (j < a.d) ? (uint32_t)idx : 0u;
     if (a.bits == 3) {
@@ -379,9 +394,16 @@ __global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
     const uint32_t bits = __ballot_sync(0xffffffffu, acc[u] >= 0.f && j < a.m);
     if (u >= nv) continue;
     const int64_t rec = out_record(a, v0 + u);
+    if (rec < 0) continue;
     if (lane == 0 && j < a.m) a.qjl[rec * ((a.m + 31) >> 5) + i32] = bits;
     if (j == 0) a.rnorm[rec] = nrm[u] * rho[u];
   }
+}
+
+template <int QS>
+__global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
+  extern __shared__ float sh[];
+  quantize_small_body<QS>(a, dpad, blockIdx.x, sh);
 }
 
 // ----------------------------------------------------------------------------
@@ -424,15 +446,13 @@ __device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T
 // PR query rows per block: thread j owns coordinate j of each row, so Pi and
 // S are read once per block.
 template <int PR>
-__global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int64_t rows, int d,
-                                                   int dpad, int m, const float* PiT, const float* ST,
-                                                   float* qr, float* qs, const int32_t* seq_lens,
-                                                   int B, int Hkv, int64_t max_T, int64_t* tiles) {
-  extern __shared__ float sh[];
+__device__ __forceinline__ void prerotate_body(const void* q, int dtype, int64_t rows, int d, int dpad,
+                                               int m, const float* PiT, const float* ST, float* qr,
+                                               float* qs, int64_t blk, float* sh) {
   float* sq = sh;                  // [PR][dpad]: q, later q'
   float* Ms = sh + PR * dpad;      // [2][MV_KC][dpad]
   const int j = threadIdx.x;       // blockDim = dpad
-  const int64_t row0 = (int64_t)blockIdx.x * PR;
+  const int64_t row0 = blk * PR;
   const int nr = (int)min((int64_t)PR, rows - row0);
 #pragma unroll
   for (int r = 0; r < PR; ++r) sq[r * dpad + j] = (r < nr && j < d) ? load_elem(q, dtype, (row0 + r) * d + j) : 0.f;
@@ -449,7 +469,48 @@ __global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int
 #pragma unroll
   for (int r = 0; r < PR; ++r)
     if (r < nr) qs[(row0 + r) * dpad + j] = (j < m) ? acc[r] : 0.f;
+}
+
+template <int PR>
+__global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int64_t rows, int d,
+                                                   int dpad, int m, const float* PiT, const float* ST,
+                                                   float* qr, float* qs, const int32_t* seq_lens,
+                                                   int B, int Hkv, int64_t max_T, int64_t* tiles) {
+  extern __shared__ float sh[];
+  prerotate_body<PR>(q, dtype, rows, d, dpad, m, PiT, ST, qr, qs, blockIdx.x, sh);
   if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
+}
+
+// ----------------------------------------------------------------------------
+// Decode-step preparation in one launch: blocks [0, n) append the new key
+// vectors, [n, 2n) the new value vectors (n = B Hkv, one vector per block),
+// the rest pre-rotate the queries (two rows per block); block 2n also writes
+// the attention lengths min(pos + 1, max_T) (0 for pos < 0) and, for the
+// tensor-core decode, their tile prefix.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_step_prep(StepPrep s, int d, int dpad, int m, const float* PiT,
+                                                   const float* ST) {
+  extern __shared__ float sh[];
+  int64_t blk = blockIdx.x;
+  if (blk < s.nkv) {
+    quantize_small_body<1>(s.k, dpad, blk, sh);
+    return;
+  }
+  blk -= s.nkv;
+  if (blk < s.nkv) {
+    quantize_small_body<1>(s.v, dpad, blk, sh);
+    return;
+  }
+  blk -= s.nkv;
+  prerotate_body<2>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, sh);
+  if (blk == 0) {
+    for (int b = threadIdx.x; b < s.B; b += blockDim.x) {
+      const int64_t p = s.pos[b];
+      s.lens[b] = (int32_t)max((int64_t)0, min(p + 1, s.max_T));
+    }
+    __syncthreads();
+    if (s.tiles) tile_plan(s.lens, s.B, s.Hkv, s.max_T, s.tiles);
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -1055,6 +1116,14 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
   return cudaGetLastError();
 }
 
+cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s) {
+  const int64_t blocks = 2 * sp.nkv + (sp.qrows + 1) / 2;
+  if (blocks == 0) return cudaSuccess;
+  k_step_prep<<<(unsigned)blocks, c->dpad, (2 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
+      sp, c->d, c->dpad, c->qjl_m, c->PiT, c->ST);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
                              float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
@@ -1200,6 +1269,7 @@ cudaError_t configure_kernels() {
   if ((e = cudaFuncSetAttribute(k_quantize_small<8>, ms, small_smem))) return e;
   if ((e = cudaFuncSetAttribute(k_prerotate<2>, ms, small_smem))) return e;
   if ((e = cudaFuncSetAttribute(k_prerotate<8>, ms, small_smem))) return e;
+  if ((e = cudaFuncSetAttribute(k_step_prep, ms, small_smem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   if ((e = configure_attn_k4()) != cudaSuccess) return e;
   return configure_attn_mma();

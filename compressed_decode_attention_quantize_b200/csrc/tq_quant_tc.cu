@@ -117,9 +117,12 @@ __device__ __forceinline__ uint32_t h2bits(float lo, float hi) {
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 __device__ __forceinline__ int flog2(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
 
+// Output record of vector v (slot pos[b] of row v = b H + g for cache
+// appends); -1 (nothing written) when pos[b] is outside [0, max_T).
 __device__ __forceinline__ int64_t out_rec(const QuantTcArgs& a, int64_t v) {
   if (a.pos == nullptr) return v;
-  return v * a.max_T + a.pos[v / a.H];
+  const int64_t p = a.pos[v / a.H];
+  return (p >= 0 && p < a.max_T) ? v * a.max_T + p : -1;
 }
 
 // Lloyd-Max index of y for 2^BITS symmetric levels: binary search over the
@@ -373,7 +376,9 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
     // ---- epilogue 1: indices, packing, residual (this half's two 32-column chunks) ----
     // y = D_rot / (sc * nrm * 2^8); the residual goes out scaled by 2^14.
     const float inv = nrm > 0.f ? 1.f / (sc * nrm * 256.f) : 0.f;
-    const int64_t rec = live ? out_rec(a, v) : 0;
+    const int64_t rec0 = live ? out_rec(a, v) : -1;
+    const bool writes = rec0 >= 0;   // this vector's record exists
+    const int64_t rec = writes ? rec0 : 0;
     uint32_t* crow = a.codes + rec * WORDS;
     float rho2v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
@@ -398,7 +403,7 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
           d[i] = r;
         }
       }
-      if (live) {
+      if (writes) {
         if (BITS == 4) *reinterpret_cast<uint4*>(crow + 4 * ch) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         if (BITS == 2) *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
         if (BITS == 1) crow[ch] = cw[0];
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
         }
       }
     }
-    if (live && h == 0) a.norm[rec] = nrm;
+    if (writes && h == 0) a.norm[rec] = nrm;
     if (!QJL) {
       tc_before_sync();
       grp_sync(gi);   // A and D_rot are free for the next tile
@@ -472,7 +477,7 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
       qw[2 * h + c2] = ~sg;
       flag[2 * h + c2] = ~fl;
     }
-    if (!live) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
+    if (!writes) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
     if (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
       const Q4 fixed = qjl_fixup<BITS>(d_rot + lane_base, inv, pmid, pb, s_cen, a.s_f32,
                                        Q4{{flag[0], flag[1], flag[2], flag[3]}},
@@ -480,7 +485,7 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
 #pragma unroll
       for (int w = 0; w < 4; ++w) qw[w] = fixed.w[w];
     }
-    if (live) {
+    if (writes) {
       *reinterpret_cast<uint2*>(a.qjl + rec * 4 + 2 * h) = make_uint2(qw[2 * h], qw[2 * h + 1]);
       if (h == 0) a.rnorm[rec] = nrm * rho;
     }

@@ -167,8 +167,8 @@ int tq_quantize(tq_ctx* ctx, int which, const void* x, int dtype, int64_t n,
  *   x       device, [B][H][d] rows of `dtype` (row b*H+g is head g of sequence
  *           b; row stride ld >= d elements).
  *   max_T   cache capacity per (sequence, head).
- *   pos     device, int32 [B]: the slot to write for sequence b, each in
- *           [0, max_T) (not checked on the device).
+ *   pos     device, int32 [B]: the slot to write for sequence b.  A sequence
+ *           whose pos is outside [0, max_T) is skipped (nothing written).
  *   codes/qjl/norm/rnorm  device cache arrays [B][H][max_T][...] as in
  *           tq_quantize; only the B*H addressed records are written.
  */
@@ -255,6 +255,31 @@ int tq_attn_decode_static(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
 
 /* Size in bytes of the static scratch used by tq_attn_decode_static. */
 size_t tq_attn_static_scratch_bytes(void);
+
+/*
+ * tq_decode_step - one whole decode step: append the newest key and value of
+ * every (sequence, kv head) to the packed cache, then attend over the cache
+ * including them ([WHAT] "How to implement" part 1: the cache quantizes on
+ * every update and the fused kernel attends straight from the codes).  Same
+ * results as tq_quantize_append (keys, then values) followed by
+ * tq_attn_decode with seq_lens[b] = min(pos[b] + 1, max_T), in three launches
+ * instead of five: append + query pre-rotation in one, attention, merge.
+ *   q        device, [B][Hq][d] of q_dtype.
+ *   k_new, v_new  device, [B][Hkv][d] contiguous rows of kv_dtype.
+ *   kcodes .. vnorm  the cache arrays of tq_attn_decode (written at pos).
+ *   pos      device, int32 [B]: the slot of the new token; sequence b then
+ *            attends over tokens [0, pos[b]].  pos outside [0, max_T) writes
+ *            nothing (pos < 0 attends over nothing, out = 0; pos >= max_T
+ *            attends over the full cache).
+ *   scale, out, workspace/ws_bytes  as in tq_attn_decode
+ *            (tq_attn_workspace_bytes() bytes).
+ */
+int tq_decode_step(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
+                   const void* v_new, int kv_dtype, int B, int Hq, int Hkv,
+                   uint32_t* kcodes, uint32_t* kqjl, float* knorm, float* krnorm,
+                   uint32_t* vcodes, float* vnorm, int64_t max_T, const int32_t* pos,
+                   float scale, float* out, void* workspace, size_t ws_bytes,
+                   void* stream);
 
 /* Bytes of workspace tq_topk needs. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);

@@ -344,10 +344,12 @@ def test_errors_are_reported(cuda):
 
 
 def test_quantize_append_writes_addressed_slots(cuda):
+    """Only slot pos[b] of each sequence is written; a pos outside [0, T)
+    writes nothing."""
     c = _ctx(128, 3, 4, 128, seed=0)
-    B, H, T = 3, 2, 50
+    B, H, T = 5, 2, 50
     x = tq_inputs.outlier_kv(B, H, 1, 128, seed=9)[:, :, 0].contiguous().to(cuda)
-    pos = torch.tensor([0, 49, 17], dtype=torch.int32, device=cuda)
+    pos = torch.tensor([0, 49, 17, -1, 50], dtype=torch.int32, device=cuda)
     for which in (tq.TQ_KEY, tq.TQ_VALUE):
         cache = c.empty_packed(which, (B, H, T), device=cuda)
         for v in cache.values():
@@ -363,9 +365,10 @@ def test_quantize_append_writes_addressed_slots(cuda):
             want = ref[k].cpu().reshape((B, H) + tuple(v.shape[3:]))
             for b in range(B):
                 p = int(pos[b])
-                assert torch.equal(got[b, :, p], want[b]), (k, b)
                 mask = torch.ones(T, dtype=torch.bool)
-                mask[p] = False
+                if 0 <= p < T:
+                    assert torch.equal(got[b, :, p], want[b]), (k, b)
+                    mask[p] = False
                 assert torch.all(got[b][:, mask] == -7), (k, b)
 
 
@@ -394,9 +397,15 @@ def test_quantize_append_large_batch(cuda):
     c = _ctx(128, 3, 4, 128, seed=0)
     B, H, T = 64, 128, 6
     x = tq_inputs.outlier_kv(B, H, 1, 128, seed=19)[:, :, 0].contiguous().to(cuda)
-    pos = torch.randint(0, T, (B,), generator=torch.Generator().manual_seed(3), dtype=torch.int32).to(cuda)
+    pos = torch.randint(0, T, (B,), generator=torch.Generator().manual_seed(3), dtype=torch.int32)
+    pos[5], pos[40] = -1, T          # skipped: nothing written for these sequences
+    pos = pos.to(cuda)
+    ok = (pos >= 0) & (pos < T)
     for which in (tq.TQ_KEY, tq.TQ_VALUE):
         cache = c.empty_packed(which, (B, H, T), device=cuda)
+        for v in cache.values():
+            if v is not None:
+                v.fill_(-7)
         c.quantize_append(x, which, cache, pos)
         ref = c.quantize(x.reshape(B * H, 128), which)
         torch.cuda.synchronize()
@@ -404,5 +413,46 @@ def test_quantize_append_large_batch(cuda):
             if v is None:
                 continue
             want = ref[k].reshape((B, H) + tuple(v.shape[3:]))
-            got = v[torch.arange(B, device=cuda), :, pos.long()]
-            assert torch.equal(got, want), k
+            bs = torch.arange(B, device=cuda)[ok]
+            got = v[bs, :, pos[ok].long()]
+            assert torch.equal(got, want[ok]), k
+            assert torch.all(v[~ok] == -7), k
+
+
+@pytest.mark.parametrize("Hq,Hkv,bk,max_T", [
+    (8, 2, 3, 300),     # tensor-core decode, group 4
+    (16, 2, 3, 300),    # group 8
+    (16, 2, 4, 300),    # 3-bit keys, group 8
+    (8, 2, 3, 302),     # max_T % 4 != 0: generic decode
+])
+def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
+    """tq_decode_step = quantize_append (K, V) + attn_decode over pos + 1
+    tokens: identical caches and outputs, and the outputs match the oracle.
+    Positions cover the first slot, the middle, the last slot, a skipped
+    negative position (empty context) and one past the end (no write, full
+    context)."""
+    c = _ctx(128, bk, 4, 128, seed=4)
+    tab = P.oracle_tables(c)
+    B, d = 6, 128
+    K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=31).to(cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=32).to(cuda)
+    kA, vA = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    kB = {k: (None if v is None else v.clone()) for k, v in kA.items()}
+    vB = {k: (None if v is None else v.clone()) for k, v in vA.items()}
+    q = tq_inputs.iid((B, Hq, d), seed=33, dtype=torch.bfloat16).to(cuda)
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=34)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=35)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([0, 17, 160, max_T - 1, -1, max_T], dtype=torch.int32, device=cuda)
+    outA = c.decode_step(q, kn, vn, kA, vA, pos)
+    c.quantize_append(kn, tq.TQ_KEY, kB, pos)
+    c.quantize_append(vn, tq.TQ_VALUE, vB, pos)
+    lens = torch.clamp(pos.long() + 1, 0, max_T).to(torch.int32)
+    outB = c.attn_decode(q, kB, vB, lens)
+    torch.cuda.synchronize()
+    for name, a_, b_ in (("k", kA, kB), ("v", vA, vB)):
+        for k in a_:
+            if a_[k] is not None:
+                assert torch.equal(a_[k], b_[k]), (name, k)
+    assert torch.equal(outA, outB)
+    P.check_attention(tab, q.double().cpu().numpy(), P.packed_np(kA), P.packed_np(vA),
+                      lens.cpu().numpy(), Hkv, outA.cpu().numpy())
