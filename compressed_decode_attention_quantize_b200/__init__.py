@@ -62,6 +62,10 @@ def _load() -> ctypes.CDLL:
         "tq_attn_decode_static": (I, [P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P]),
         "tq_attn_static_scratch_bytes": (SZ, []),
         "tq_decode_step": (I, [P, P, I, P, P, I, I, I, I, P, P, P, P, P, P, I64, P, F, P, P, SZ, P]),
+        "tq_quantize_append_paged": (I, [P, I, P, I, I, I, I64, P, I, I, I64, P, P, P, P, P, P]),
+        "tq_attn_decode_paged": (I, [P, P, I, I, I, I, P, P, P, P, P, P, P, I, I, I64, P, F, P, P, SZ, P]),
+        "tq_decode_step_paged": (I, [P, P, I, P, P, I, I, I, I, P, P, P, P, P, P, P, I, I, I64, P, F, P, P,
+                                     SZ, P]),
         "tq_topk_workspace_bytes": (SZ, [P, I64, I64, I]),
         "tq_topk": (I, [P, P, I, I64, P, P, P, P, I64, I, P, P, P, SZ, P]),
     }
@@ -76,7 +80,8 @@ _lib = _load()
 EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
             "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
-            "tq_attn_static_scratch_bytes", "tq_decode_step", "tq_topk_workspace_bytes", "tq_topk")
+            "tq_attn_static_scratch_bytes", "tq_decode_step", "tq_quantize_append_paged",
+            "tq_attn_decode_paged", "tq_decode_step_paged", "tq_topk_workspace_bytes", "tq_topk")
 
 
 def library_path() -> str:
@@ -290,6 +295,68 @@ class Context:
                                    _ptr(vcache["codes"]), _ptr(vcache["norm"]), max_T, _ptr(pos),
                                    float(scale), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+        return out
+
+    # ---- paged caches: arrays [num_blocks, Hkv, block_size, ...] (empty_packed
+    # with that shape), block_table int32 [B, max_blocks] of block ids --------
+    def quantize_append_paged(self, x: torch.Tensor, which: int, cache: dict, block_table: torch.Tensor,
+                              pos: torch.Tensor, stream=None) -> dict:
+        """x [B, H, d] (newest token per sequence and head) -> the slot of
+        position pos[b] in block block_table[b, pos[b] // block_size]."""
+        B, H, d = x.shape
+        if x.stride(2) != 1 or x.stride(0) != H * x.stride(1):
+            raise TQError(TQ_ERR_ARG, "x must be [B, H, d] with rows at a uniform stride")
+        nb, _, bs = cache["norm"].shape
+        _check(_lib.tq_quantize_append_paged(self.ptr, which, _ptr(x), _DTYPES[x.dtype], B, H, x.stride(1),
+                                             _ptr(block_table), block_table.shape[1], bs, nb, _ptr(pos),
+                                             _ptr(cache["codes"]), _ptr(cache.get("qjl")),
+                                             _ptr(cache["norm"]), _ptr(cache.get("rnorm")), _stream(stream)))
+        return cache
+
+    def attn_decode_paged(self, q: torch.Tensor, kcache: dict, vcache: dict, block_table: torch.Tensor,
+                          seq_lens: torch.Tensor, scale: float | None = None,
+                          out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+        q = q.contiguous()
+        B, Hq, d = q.shape
+        nb, Hkv, bs = kcache["norm"].shape
+        mb = block_table.shape[1]
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(self.attn_workspace_bytes(B, Hq, mb * bs), dtype=torch.uint8,
+                                    device=q.device)
+        _check(_lib.tq_attn_decode_paged(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
+                                         _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(kcache["norm"]),
+                                         _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
+                                         _ptr(block_table), mb, bs, nb, _ptr(seq_lens), float(scale),
+                                         _ptr(out), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+        return out
+
+    def decode_step_paged(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                          kcache: dict, vcache: dict, block_table: torch.Tensor, pos: torch.Tensor,
+                          scale: float | None = None, out: torch.Tensor | None = None,
+                          workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        q, k_new, v_new = q.contiguous(), k_new.contiguous(), v_new.contiguous()
+        B, Hq, d = q.shape
+        nb, Hkv, bs = kcache["norm"].shape
+        mb = block_table.shape[1]
+        if k_new.shape != (B, Hkv, d) or v_new.shape != (B, Hkv, d) or k_new.dtype != v_new.dtype:
+            raise TQError(TQ_ERR_ARG, "decode_step_paged: k_new / v_new must both be [B, Hkv, d] of one dtype")
+        scale = 1.0 / math.sqrt(d) if scale is None else scale
+        if out is None:
+            out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(self.attn_workspace_bytes(B, Hq, mb * bs), dtype=torch.uint8,
+                                    device=q.device)
+        _check(_lib.tq_decode_step_paged(self.ptr, _ptr(q), _DTYPES[q.dtype], _ptr(k_new), _ptr(v_new),
+                                         _DTYPES[k_new.dtype], B, Hq, Hkv, _ptr(kcache["codes"]),
+                                         _ptr(kcache["qjl"]), _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
+                                         _ptr(vcache["codes"]), _ptr(vcache["norm"]), _ptr(block_table), mb,
+                                         bs, nb, _ptr(pos), float(scale), _ptr(out), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
         return out
 
     def attn_decode_static(self, q: torch.Tensor, kcache: dict, vcache: dict,

@@ -293,10 +293,18 @@ int tq_export_tables(const tq_ctx* c, double* pi, double* S, double* ck, double*
   return TQ_OK;
 }
 
+// Block table of a paged cache: arrays [num_blocks][H][block_size][...],
+// table [B][max_blocks]; null table = contiguous [B][H][max_T][...].
+struct Paging {
+  const int32_t* table = nullptr;
+  int max_blocks = 0, block_size = 0;
+  int64_t num_blocks = 0;
+};
+
 static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64_t n, int64_t ld,
                            uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm,
                            const int32_t* pos, int H, int64_t max_T, void* stream,
-                           const char* name) {
+                           const char* name, const Paging& pg = Paging()) {
   if (int r = check_ctx(c)) return r;
   if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "%s: bad which=%d", name, which);
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
@@ -330,12 +338,16 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.pos = pos;
   a.H = H;
   a.max_T = max_T;
+  a.block_table = pg.table;
+  a.max_blocks = pg.max_blocks;
+  a.block_size = pg.block_size;
+  a.num_blocks = pg.num_blocks;
   if (n <= tqk::kSmallQuantize) {
     cudaError_t e = tqk::launch_quantize_small(c, a, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;
   }
-  const bool tc = c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+  const bool tc = !pg.table && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
     tqk::QuantTcArgs t{};
@@ -385,6 +397,22 @@ int tq_quantize_append(tq_ctx* c, int which, const void* x, int dtype, int B, in
   if (B > 0 && !pos) return fail(TQ_ERR_ARG, "tq_quantize_append: null pos");
   return quantize_common(c, which, x, dtype, (int64_t)B * H, ld, codes, qjl, norm, rnorm, pos, H,
                          max_T, stream, "tq_quantize_append");
+}
+
+int tq_quantize_append_paged(tq_ctx* c, int which, const void* x, int dtype, int B, int H,
+                             int64_t ld, const int32_t* block_table, int max_blocks, int block_size,
+                             int64_t num_blocks, const int32_t* pos, uint32_t* codes, uint32_t* qjl,
+                             float* norm, float* rnorm, void* stream) {
+  if (B < 0 || H <= 0 || max_blocks <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(TQ_ERR_ARG, "tq_quantize_append_paged: bad sizes");
+  if (B > 0 && (!pos || !block_table)) return fail(TQ_ERR_ARG, "tq_quantize_append_paged: null pos or block_table");
+  Paging pg;
+  pg.table = block_table;
+  pg.max_blocks = max_blocks;
+  pg.block_size = block_size;
+  pg.num_blocks = num_blocks;
+  return quantize_common(c, which, x, dtype, (int64_t)B * H, ld, codes, qjl, norm, rnorm, pos, H,
+                         (int64_t)max_blocks * block_size, stream, "tq_quantize_append_paged", pg);
 }
 
 int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* qjl,
@@ -450,26 +478,27 @@ size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   return attn_ws_layout(c, B, Hq, max_T).total;
 }
 
-int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
-                   const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
-                   const float* krnorm, const uint32_t* vcodes, const float* vnorm, int64_t max_T,
-                   const int32_t* seq_lens, float scale, float* out, void* workspace,
-                   size_t ws_bytes, void* stream) {
+static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
+                            const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                            const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                            int64_t max_T, const int32_t* seq_lens, float scale, float* out,
+                            void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
+                            const char* name) {
   if (int r = check_ctx(c)) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
-    return fail(TQ_ERR_ARG, "tq_attn_decode: bad dtype=%d", dtype);
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T < 0) return fail(TQ_ERR_ARG, "tq_attn_decode: bad sizes");
+    return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dtype);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T < 0) return fail(TQ_ERR_ARG, "%s: bad sizes", name);
   if (Hq % Hkv != 0 || Hq / Hkv > 16)
-    return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", Hq, Hkv);
+    return fail(TQ_ERR_UNSUPPORTED, "%s: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", name, Hq, Hkv);
   if (B == 0) return TQ_OK;
   if (!q || !kcodes || !knorm || !vcodes || !vnorm || !seq_lens || !out)
-    return fail(TQ_ERR_ARG, "tq_attn_decode: null pointer");
-  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_attn_decode: keys with QJL need kqjl and krnorm");
-  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: B or Hkv too large");
+    return fail(TQ_ERR_ARG, "%s: null pointer", name);
+  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "%s: keys with QJL need kqjl and krnorm", name);
+  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "%s: B or Hkv too large", name);
   const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
   if (!workspace || ws_bytes < need)
-    return fail(TQ_ERR_WORKSPACE, "tq_attn_decode: workspace %zu bytes < %zu", ws_bytes, need);
-  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_attn_decode: workspace not 256-byte aligned");
+    return fail(TQ_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu", name, ws_bytes, need);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "%s: workspace not 256-byte aligned", name);
   cudaStream_t s = as_stream(stream);
   const size_t rows = (size_t)B * Hq;
   const AttnWs lay = attn_ws_layout(c, B, Hq, max_T);
@@ -505,43 +534,84 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
   a.splits = tqk::attn_splits(c, B, Hkv, max_T > 0 ? max_T : 1, &a.chunk);
   a.part = part;
   a.tiles = nullptr;
+  a.block_table = pg.table;
+  a.max_blocks = pg.max_blocks;
+  a.block_size = pg.block_size;
+  a.num_blocks = pg.num_blocks;
   const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
   const bool k4 = !mma && tqk::attn_k4_supported(c, a) && max_T > 0;
+  if (pg.table && !(mma || k4))
+    return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode (d = 128, QJL m = 128, "
+                "4-bit values, 2-bit keys with group 1/2/4/8 or 3-bit keys with group 8)", name);
   if (mma || k4) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
-    return fail(TQ_ERR_UNSUPPORTED, "tq_attn_decode: too many splits");
+    return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
   }
   cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode: prerotate");
+  if (e != cudaSuccess) return cuda_fail(e, name);
   e = mma ? tqk::launch_attn_mma(c, a, out, s)
           : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
-  if (e != cudaSuccess) return cuda_fail(e, "tq_attn_decode");
+  if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
 }
 
-int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
-                   int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
-                   float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm, int64_t max_T,
-                   const int32_t* pos, float scale, float* out, void* workspace, size_t ws_bytes,
-                   void* stream) {
+static bool paging_ok(const Paging& pg) {
+  return pg.table && pg.max_blocks > 0 && pg.block_size > 0 && pg.block_size % 16 == 0 && pg.num_blocks > 0 &&
+         (int64_t)pg.max_blocks * pg.block_size <= (int64_t)1 << 30;
+}
+
+int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
+                   const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                   const float* krnorm, const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                   const int32_t* seq_lens, float scale, float* out, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  return attn_decode_impl(c, q, dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm, vcodes, vnorm, max_T,
+                          seq_lens, scale, out, workspace, ws_bytes, stream, Paging(), "tq_attn_decode");
+}
+
+int tq_attn_decode_paged(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
+                         const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                         const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                         const int32_t* block_table, int max_blocks, int block_size,
+                         int64_t num_blocks, const int32_t* seq_lens, float scale, float* out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  Paging pg;
+  pg.table = block_table;
+  pg.max_blocks = max_blocks;
+  pg.block_size = block_size;
+  pg.num_blocks = num_blocks;
+  if (B > 0 && !paging_ok(pg))
+    return fail(TQ_ERR_ARG, "tq_attn_decode_paged: bad block table (need block_size %% 16 == 0, "
+                "max_blocks, num_blocks > 0)");
+  return attn_decode_impl(c, q, dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm, vcodes, vnorm,
+                          (int64_t)max_blocks * block_size, seq_lens, scale, out, workspace, ws_bytes,
+                          stream, pg, "tq_attn_decode_paged");
+}
+
+static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k_new,
+                            const void* v_new, int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes,
+                            uint32_t* kqjl, float* knorm, float* krnorm, uint32_t* vcodes,
+                            float* vnorm, int64_t max_T, const int32_t* pos, float scale, float* out,
+                            void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
+                            const char* name) {
   if (int r = check_ctx(c)) return r;
   for (int dt : {q_dtype, kv_dtype})
-    if (dt != TQ_F32 && dt != TQ_BF16 && dt != TQ_F16) return fail(TQ_ERR_ARG, "tq_decode_step: bad dtype=%d", dt);
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "tq_decode_step: bad sizes");
+    if (dt != TQ_F32 && dt != TQ_BF16 && dt != TQ_F16) return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dt);
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "%s: bad sizes", name);
   if (Hq % Hkv != 0 || Hq / Hkv > 16)
-    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", Hq, Hkv);
+    return fail(TQ_ERR_UNSUPPORTED, "%s: Hq=%d Hkv=%d (need Hq %% Hkv == 0, group <= 16)", name, Hq, Hkv);
   if (B == 0) return TQ_OK;
   if (!q || !k_new || !v_new || !kcodes || !knorm || !vcodes || !vnorm || !pos || !out)
-    return fail(TQ_ERR_ARG, "tq_decode_step: null pointer");
-  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_decode_step: keys with QJL need kqjl and krnorm");
-  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: B or Hkv too large");
+    return fail(TQ_ERR_ARG, "%s: null pointer", name);
+  if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "%s: keys with QJL need kqjl and krnorm", name);
+  if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "%s: B or Hkv too large", name);
   if (!aligned(kcodes, 4) || !aligned(knorm, 4) || !aligned(vcodes, 4) || !aligned(vnorm, 4))
-    return fail(TQ_ERR_ARG, "tq_decode_step: misaligned cache");
+    return fail(TQ_ERR_ARG, "%s: misaligned cache", name);
   const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
   if (!workspace || ws_bytes < need)
-    return fail(TQ_ERR_WORKSPACE, "tq_decode_step: workspace %zu bytes < %zu", ws_bytes, need);
-  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_decode_step: workspace not 256-byte aligned");
+    return fail(TQ_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu", name, ws_bytes, need);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "%s: workspace not 256-byte aligned", name);
   cudaStream_t s = as_stream(stream);
   const size_t rows = (size_t)B * Hq;
   const AttnWs lay = attn_ws_layout(c, B, Hq, max_T);
@@ -572,6 +642,10 @@ int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, con
     a.pos = pos;
     a.H = Hkv;
     a.max_T = max_T;
+    a.block_table = pg.table;
+    a.max_blocks = pg.max_blocks;
+    a.block_size = pg.block_size;
+    a.num_blocks = pg.num_blocks;
     return a;
   };
   tqk::AttnArgs a{};
@@ -602,12 +676,18 @@ int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, con
   a.splits = tqk::attn_splits(c, B, Hkv, max_T, &a.chunk);
   a.part = reinterpret_cast<float*>(p + lay.part_off);
   a.tiles = nullptr;
+  a.block_table = pg.table;
+  a.max_blocks = pg.max_blocks;
+  a.block_size = pg.block_size;
+  a.num_blocks = pg.num_blocks;
   const bool mma = tqk::attn_mma_supported(c, a);
   const bool k4 = !mma && tqk::attn_k4_supported(c, a);
+  if (pg.table && !(mma || k4))
+    return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode", name);
   if (mma || k4) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
-    return fail(TQ_ERR_UNSUPPORTED, "tq_decode_step: too many splits");
+    return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
   }
   tqk::StepPrep sp{};
   sp.k = qargs(true);
@@ -625,11 +705,40 @@ int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, con
   sp.tiles = a.tiles;
   sp.nkv = (int64_t)B * Hkv;
   cudaError_t e = tqk::launch_step_prep(c, sp, s);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step: prepare");
+  if (e != cudaSuccess) return cuda_fail(e, name);
   e = mma ? tqk::launch_attn_mma(c, a, out, s)
           : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
-  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_step");
+  if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
+}
+
+int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
+                   int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
+                   float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm, int64_t max_T,
+                   const int32_t* pos, float scale, float* out, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  return decode_step_impl(c, q, q_dtype, k_new, v_new, kv_dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm,
+                          vcodes, vnorm, max_T, pos, scale, out, workspace, ws_bytes, stream, Paging(),
+                          "tq_decode_step");
+}
+
+int tq_decode_step_paged(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
+                         int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
+                         float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm,
+                         const int32_t* block_table, int max_blocks, int block_size,
+                         int64_t num_blocks, const int32_t* pos, float scale, float* out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  Paging pg;
+  pg.table = block_table;
+  pg.max_blocks = max_blocks;
+  pg.block_size = block_size;
+  pg.num_blocks = num_blocks;
+  if (B > 0 && !paging_ok(pg))
+    return fail(TQ_ERR_ARG, "tq_decode_step_paged: bad block table (need block_size %% 16 == 0, "
+                "max_blocks, num_blocks > 0)");
+  return decode_step_impl(c, q, q_dtype, k_new, v_new, kv_dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm,
+                          vcodes, vnorm, (int64_t)max_blocks * block_size, pos, scale, out, workspace,
+                          ws_bytes, stream, pg, "tq_decode_step_paged");
 }
 
 size_t tq_topk_workspace_bytes(const tq_ctx* c, int64_t nq, int64_t n, int k) {

@@ -8,6 +8,8 @@
 
 #include <cstdint>
 
+#include "tq_internal.h"
+
 namespace tqk {
 namespace {
 
@@ -143,6 +145,35 @@ __device__ __forceinline__ void value_tile(float (&o)[8][4], const uint32_t (*v)
     for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
     mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
   }
+}
+
+// Record index of token t of row (b, kv head): [B][Hkv][max_T] contiguous, or
+// paged [blocks][Hkv][block_size] through the block table (an id outside
+// [0, num_blocks) reads block 0: wrong values, no fault).  For t a multiple
+// of 4 (16 when paged with block_size % 16 == 0) the next 3 (15) tokens are
+// the next records.
+template <bool PAGED>
+__device__ __forceinline__ int64_t kv_rec(const AttnArgs& a, int b, int kvh, int64_t t);
+
+// Record base of row (b, kv head) folded into the array pointers (contiguous
+// caches), and the per-tile record offset relative to it: t itself, or for
+// paged caches the full record index (base 0).
+template <bool PAGED>
+__device__ __forceinline__ int64_t kv_base(const AttnArgs& a, int b, int kvh) {
+  return PAGED ? 0 : ((int64_t)b * a.Hkv + kvh) * a.max_T;
+}
+template <bool PAGED>
+__device__ __forceinline__ int64_t kv_off(const AttnArgs& a, int b, int kvh, int64_t t) {
+  return PAGED ? kv_rec<true>(a, b, kvh, t) : t;
+}
+
+template <bool PAGED>
+__device__ __forceinline__ int64_t kv_rec(const AttnArgs& a, int b, int kvh, int64_t t) {
+  if (!PAGED) return ((int64_t)b * a.Hkv + kvh) * a.max_T + t;
+  const int ti = (int)t;
+  int64_t blk = a.block_table[(int64_t)b * a.max_blocks + ti / a.block_size];
+  blk = (blk >= 0 && blk < a.num_blocks) ? blk : 0;
+  return (blk * a.Hkv + kvh) * a.block_size + ti % a.block_size;
 }
 
 // Sequence holding tile x of the tile prefix P[0..B]: P[b] <= x < P[b + 1].

@@ -76,6 +76,7 @@ __device__ __forceinline__ uint32_t klut_off(uint32_t w2, uint32_t w1) {
   return (nib | (top << 4)) << 8;
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
   constexpr int G = 8;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -133,7 +134,6 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
     x += nt;
 
     const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
-    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
     const int64_t tok0 = tt * MT;
     const int64_t tok1 = min(te * MT, len);
     const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * G;
@@ -166,13 +166,13 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
     }
     {
       float vmax = 0.f;
-      const float* vr = a.vnorm + row0;
       for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
+        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
         if (j + 4 <= tok1) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          const float4 v4 = *reinterpret_cast<const float4*>(vr);
           vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
         } else {
-          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+          for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
         }
       }
 #pragma unroll
@@ -237,9 +237,11 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
 
     // ---- this warp's tiles: i = warp, warp + 4, ... of the piece ------------------
     const int ntw = nt > warp ? (nt - warp + MW - 1) / MW : 0;
-    const char* kbase = reinterpret_cast<const char*>(a.kcodes + row0 * (K2W + K1W));
+    const int64_t rb = kv_base<PAGED>(a, b, kvh);   // row base (0 when paged)
+    const char* kbase = reinterpret_cast<const char*>(a.kcodes + rb * (K2W + K1W));
     auto issue = [&](int k, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
+      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(StageK4);
 #pragma unroll
       for (int i = 0; i < 5; ++i) {
@@ -248,20 +250,20 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_k4(AttnArgs a) {
           const int tok = c / 3, part = c % 3;
           const uint32_t dst = part < 2 ? (uint32_t)(offsetof(StageK4, k2) + tok * 32 + part * 16)
                                         : (uint32_t)(offsetof(StageK4, k1) + tok * 16);
-          cp16(sb + dst, kbase + (t0 + tok) * 48 + part * 16, t0 + tok < tok1);
+          cp16(sb + dst, kbase + (r + tok) * 48 + part * 16, t0 + tok < tok1);
         } else if (c < 64) {                   // QJL words: 16 tokens x 1 chunk
           const int tok = c - 48;
-          cp16(sb + offsetof(StageK4, q) + tok * 16, a.kqjl + (row0 + t0 + tok) * QW, t0 + tok < tok1);
+          cp16(sb + offsetof(StageK4, q) + tok * 16, a.kqjl + (rb + r + tok) * QW, t0 + tok < tok1);
         } else if (c < 76) {                   // norms: 3 arrays x 4 chunks of 4 tokens
           const int which = (c - 64) >> 2, part = (c - 64) & 3;
           const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
           const uint32_t off = which == 0 ? offsetof(StageK4, kn)
                                           : (which == 1 ? offsetof(StageK4, kr) : offsetof(StageK4, vn));
-          cp16(sb + off + part * 16, base + row0 + t0 + 4 * part, t0 + 4 * part < tok1);
+          cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tok1);
         } else if (c < 140) {                  // value codes: 16 tokens x 4 chunks
           const int cc = c - 76, tok = cc >> 2, part = cc & 3;
           cp16(sb + offsetof(StageK4, v) + tok * (VROW * 4) + part * 16,
-               a.vcodes + (row0 + t0 + tok) * VW + part * 4, t0 + tok < tok1);
+               a.vcodes + (rb + r + tok) * VW + part * 4, t0 + tok < tok1);
         }
       }
     };
@@ -418,14 +420,20 @@ cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a_in, float* out, cu
   blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 2 ? (int64_t)c->sms * 2 : blocks);
   a.nw = (int)blocks;
   a.wpu = MW;
-  k_attn_k4<<<(unsigned)blocks, MW * 32, SMEMK4_BYTES, s>>>(a);
+  if (a.block_table)
+    k_attn_k4<true><<<(unsigned)blocks, MW * 32, SMEMK4_BYTES, s>>>(a);
+  else
+    k_attn_k4<false><<<(unsigned)blocks, MW * 32, SMEMK4_BYTES, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_merge(c, a, out, s);
 }
 
 cudaError_t configure_attn_k4() {
-  return cudaFuncSetAttribute(k_attn_k4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMK4_BYTES);
+  const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_k4<false>, ms, (int)SMEMK4_BYTES);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_attn_k4<true>, ms, (int)SMEMK4_BYTES);
 }
 
 }  // namespace tqk

@@ -72,7 +72,7 @@ constexpr size_t SMEM_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST * sizeof(
 // the value norms of a piece are scaled once, from the piece's largest norm,
 // so that p |v| stays below 2^15 in fp16.
 // ---------------------------------------------------------------------------
-template <int G>
+template <int G, bool PAGED>
 __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
   static_assert(G <= 4, "packed path");
   extern __shared__ __align__(16) unsigned char smem[];
@@ -119,25 +119,25 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
     x += nt;
 
     const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
-    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
     const int64_t tok0 = tt * MT;
     const int64_t tok1 = min(te * MT, len);
 
     // ---- cp.async ring: lane assignment fixed for the piece -------------------
     // slot 0 = key codes, slots 1-2 = value codes, slot 3 = QJL words or norms.
-    const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;
-    const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;
+    const int64_t rb = kv_base<PAGED>(a, b, kvh);   // row base (0 when paged)
+    const char* p0 = reinterpret_cast<const char*>(a.kcodes + rb * KW) + lane * 16;
+    const char* p1 = reinterpret_cast<const char*>(a.vcodes + rb * VW) + lane * 16;
     const char* p2 = p1 + 8 * 64;
     const char* p3;
     int stride3, tok3;
     uint32_t d3;
     if (lane < 16) {
-      p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
+      p3 = reinterpret_cast<const char*>(a.kqjl + rb * QW) + lane * 16;
       stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
     } else if (lane < 28) {
       const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
       const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
-      p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
+      p3 = reinterpret_cast<const char*>(base + rb) + part * 16;
       stride3 = 4; tok3 = 4 * part;
       d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
     } else {
@@ -149,10 +149,11 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
     auto issue = [&](int i, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * i;
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
-      cp16(sb + d0, p0 + t0 * 32, t0 + (lane >> 1) < tok1);
-      cp16(sb + d1, p1 + t0 * 64, t0 + (lane >> 2) < tok1);
-      cp16(sb + d2, p2 + t0 * 64, t0 + 8 + (lane >> 2) < tok1);
-      if (lane < 28) cp16(sb + d3, p3 + t0 * stride3, t0 + tok3 < tok1);
+      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
+      cp16(sb + d0, p0 + r * 32, t0 + (lane >> 1) < tok1);
+      cp16(sb + d1, p1 + r * 64, t0 + (lane >> 2) < tok1);
+      cp16(sb + d2, p2 + r * 64, t0 + 8 + (lane >> 2) < tok1);
+      if (lane < 28) cp16(sb + d3, p3 + r * stride3, t0 + tok3 < tok1);
     };
 #pragma unroll
     for (int i = 0; i < NST - 1; ++i) {
@@ -248,13 +249,13 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
     // ---- value-norm scale of the piece ---------------------------------------
     float vmax = 0.f;
     {
-      const float* vr = a.vnorm + row0;
       for (int64_t j = tok0 + 4 * lane; j < tok1; j += 128) {
+        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
         if (j + 4 <= tok1) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          const float4 v4 = *reinterpret_cast<const float4*>(vr);
           vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
         } else {
-          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+          for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
         }
       }
 #pragma unroll
@@ -388,6 +389,7 @@ constexpr int QOP_STEPS = 24;                 // 16 key k-steps + 8 QJL k-steps
 constexpr size_t SMEM8_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST8 * sizeof(Stage) +
                                (size_t)QOP_STEPS * 32 * 16 + 8 * 16 + MW * 4 + 16 * 4;
 
+template <bool PAGED>
 __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
   constexpr int G = 8;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -433,7 +435,6 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
     x += nt;
 
     const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
-    const int64_t row0 = ((int64_t)b * a.Hkv + kvh) * a.max_T;
     const int64_t tok0 = tt * MT;
     const int64_t tok1 = min(te * MT, len);
     const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * G;
@@ -466,13 +467,13 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
     }
     {
       float vmax = 0.f;
-      const float* vr = a.vnorm + row0;
       for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
+        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
         if (j + 4 <= tok1) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vr + j);
+          const float4 v4 = *reinterpret_cast<const float4*>(vr);
           vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
         } else {
-          for (int64_t k = j; k < tok1; ++k) vmax = fmaxf(vmax, vr[k]);
+          for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
         }
       }
 #pragma unroll
@@ -528,19 +529,20 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
 
     // ---- this warp's tiles: i = warp, warp + 4, ... of the piece ------------------
     const int ntw = nt > warp ? (nt - warp + MW - 1) / MW : 0;
-    const char* p0 = reinterpret_cast<const char*>(a.kcodes + row0 * KW) + lane * 16;
-    const char* p1 = reinterpret_cast<const char*>(a.vcodes + row0 * VW) + lane * 16;
+    const int64_t rb = kv_base<PAGED>(a, b, kvh);   // row base (0 when paged)
+    const char* p0 = reinterpret_cast<const char*>(a.kcodes + rb * KW) + lane * 16;
+    const char* p1 = reinterpret_cast<const char*>(a.vcodes + rb * VW) + lane * 16;
     const char* p2 = p1 + 8 * 64;
     const char* p3;
     int stride3, tok3;
     uint32_t d3;
     if (lane < 16) {
-      p3 = reinterpret_cast<const char*>(a.kqjl + row0 * QW) + lane * 16;
+      p3 = reinterpret_cast<const char*>(a.kqjl + rb * QW) + lane * 16;
       stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
     } else if (lane < 28) {
       const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
       const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
-      p3 = reinterpret_cast<const char*>(base + row0) + part * 16;
+      p3 = reinterpret_cast<const char*>(base + rb) + part * 16;
       stride3 = 4; tok3 = 4 * part;
       d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
     } else {
@@ -552,10 +554,11 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
     auto issue = [&](int k, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
-      cp16(sb + d0, p0 + t0 * 32, t0 + (lane >> 1) < tok1);
-      cp16(sb + d1, p1 + t0 * 64, t0 + (lane >> 2) < tok1);
-      cp16(sb + d2, p2 + t0 * 64, t0 + 8 + (lane >> 2) < tok1);
-      if (lane < 28) cp16(sb + d3, p3 + t0 * stride3, t0 + tok3 < tok1);
+      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
+      cp16(sb + d0, p0 + r * 32, t0 + (lane >> 1) < tok1);
+      cp16(sb + d1, p1 + r * 64, t0 + (lane >> 2) < tok1);
+      cp16(sb + d2, p2 + r * 64, t0 + 8 + (lane >> 2) < tok1);
+      if (lane < 28) cp16(sb + d3, p3 + r * stride3, t0 + tok3 < tok1);
     };
 #pragma unroll
     for (int k = 0; k < NST8 - 1; ++k) {
@@ -711,10 +714,14 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, c
     blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
     a.nw = (int)(blocks * MW);
     a.wpu = 1;
-    switch (a.G) {
-      case 1: k_attn_seg<1><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      case 2: k_attn_seg<2><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      default: k_attn_seg<4><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+    const bool paged = a.block_table != nullptr;
+    switch (a.G * 2 + (paged ? 1 : 0)) {
+      case 2: k_attn_seg<1, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      case 3: k_attn_seg<1, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      case 4: k_attn_seg<2, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      case 5: k_attn_seg<2, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      case 8: k_attn_seg<4, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
+      default: k_attn_seg<4, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
     }
   } else if (a.G == 8) {
     if (!a.tiles) return cudaErrorInvalidValue;
@@ -724,7 +731,10 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, c
     blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
     a.nw = (int)blocks;
     a.wpu = MW;
-    k_attn_seg8<<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
+    if (a.block_table)
+      k_attn_seg8<true><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
+    else
+      k_attn_seg8<false><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
   } else {
     return cudaErrorInvalidValue;
   }
@@ -734,12 +744,17 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, c
 }
 
 cudaError_t configure_attn_mma() {
-  const int b = (int)SMEM_BYTES;
+  const int b = (int)SMEM_BYTES, b8 = (int)SMEM8_BYTES;
+  const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b))) return e;
-  return cudaFuncSetAttribute(k_attn_seg8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8_BYTES);
+  if ((e = cudaFuncSetAttribute(k_attn_seg<1, false>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<1, true>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<2, false>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<2, true>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<4, false>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg<4, true>, ms, b))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_seg8<false>, ms, b8))) return e;
+  return cudaFuncSetAttribute(k_attn_seg8<true>, ms, b8);
 }
 
 }  // namespace tqk

@@ -75,9 +75,15 @@ struct QuantArgs {
   float* rnorm;
   // Optional cache placement: when pos != nullptr, input row v = b*H + g is
   // written to cache record (b*H + g)*max_T + pos[b]; otherwise to record v.
+  // With block_table != nullptr the cache is paged: record
+  // (block_table[b][pos / block_size] * H + g) * block_size + pos % block_size,
+  // max_T = max_blocks * block_size; an invalid pos or block id writes nothing.
   const int32_t* pos;
   int H;
   int64_t max_T;
+  const int32_t* block_table;
+  int max_blocks, block_size;
+  int64_t num_blocks;
 };
 
 struct AttnArgs {
@@ -106,6 +112,12 @@ struct AttnArgs {
   int64_t* tiles;
   int nw;
   int wpu;
+  // Paged caches (tensor-core paths): block_table [B][max_blocks] of block ids
+  // in [0, num_blocks); arrays are [num_blocks][Hkv][block_size][...] and
+  // block_size is a multiple of 16.  Null for the contiguous [B][Hkv][max_T].
+  const int32_t* block_table;
+  int max_blocks, block_size;
+  int64_t num_blocks;
 };
 
 struct QuantTcArgs {

@@ -48,12 +48,18 @@ __device__ __forceinline__ int lm_index(float y, const float* sb, int nb) {
 
 // Output record of input row v (cache placement when a.pos is set).
 // Output record of vector v: v itself, or for cache appends slot pos[b] of
-// row v = b H + g; -1 (nothing written) when pos[b] is outside [0, max_T).
+// row v = b H + g (contiguous or paged cache); -1 (nothing written) when
+// pos[b] is outside [0, max_T) or its block id is invalid.
 __device__ __forceinline__ int64_t out_record(const QuantArgs& a, int64_t v) {
   if (a.pos == nullptr) return v;
   const int64_t b = v / a.H;
   const int64_t p = a.pos[b];
-  return (p >= 0 && p < a.max_T) ? v * a.max_T + p : -1;
+  if (p < 0 || p >= a.max_T) return -1;
+  if (a.block_table == nullptr) return v * a.max_T + p;
+  // Paged: slot p % block_size of block block_table[b][p / block_size].
+  const int64_t blk = a.block_table[b * a.max_blocks + p / a.block_size];
+  if (blk < 0 || blk >= a.num_blocks) return -1;
+  return (blk * a.H + (v - b * a.H)) * a.block_size + p % a.block_size;
 }
 
 // Lloyd-Max index of coordinate j of a packed vector (b-bit fields; for b = 3

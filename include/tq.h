@@ -178,6 +178,22 @@ int tq_quantize_append(tq_ctx* ctx, int which, const void* x, int dtype, int B,
                        void* stream);
 
 /*
+ * tq_quantize_append_paged - tq_quantize_append into a paged cache (blocks of
+ * block_size tokens allocated from a pool; SURVEY's "next" paged layout).
+ *   codes/qjl/norm/rnorm  device cache arrays [num_blocks][H][block_size][...].
+ *   block_table  device, int32 [B][max_blocks]: block ids in [0, num_blocks).
+ *   pos          device, int32 [B]: token position of sequence b; it goes to
+ *                slot pos % block_size of block block_table[b][pos / block_size].
+ * A sequence whose pos is outside [0, max_blocks * block_size), or whose
+ * block id is outside [0, num_blocks), is skipped (nothing written).
+ */
+int tq_quantize_append_paged(tq_ctx* ctx, int which, const void* x, int dtype, int B,
+                             int H, int64_t ld, const int32_t* block_table,
+                             int max_blocks, int block_size, int64_t num_blocks,
+                             const int32_t* pos, uint32_t* codes, uint32_t* qjl,
+                             float* norm, float* rnorm, void* stream);
+
+/*
  * tq_dequantize - x_hat = |x| Pi^T c[idx], plus for keys with QJL the
  * back-projection sqrt(pi/2)/m * gamma * Pi^T S^T sigma (sigma = +-1 from the
  * QJL bits), so that <q, x_hat> equals tq_logits.
@@ -257,6 +273,25 @@ int tq_attn_decode_static(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
 size_t tq_attn_static_scratch_bytes(void);
 
 /*
+ * tq_attn_decode_paged - tq_attn_decode over a paged cache: token t of
+ * sequence b is record (block_table[b][t / block_size] * Hkv + g) *
+ * block_size + t % block_size of the arrays [num_blocks][Hkv][block_size][...]
+ * (g = kv head).  block_size must be a multiple of 16; seq_lens[b] is clamped
+ * to max_blocks * block_size.  Block ids outside [0, num_blocks) read block 0
+ * (wrong results, no fault).  Only the tensor-core decode takes paged caches
+ * (d = 128, keys with m = 128 QJL rows, 4-bit values; 2-bit keys with GQA
+ * group 1, 2, 4 or 8, or 3-bit keys with group 8); other formats return
+ * TQ_ERR_UNSUPPORTED.  Workspace: tq_attn_workspace_bytes(ctx, B, Hq,
+ * max_blocks * block_size).
+ */
+int tq_attn_decode_paged(tq_ctx* ctx, const void* q, int dtype, int B, int Hq, int Hkv,
+                         const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+                         const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                         const int32_t* block_table, int max_blocks, int block_size,
+                         int64_t num_blocks, const int32_t* seq_lens, float scale, float* out,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * tq_decode_step - one whole decode step: append the newest key and value of
  * every (sequence, kv head) to the packed cache, then attend over the cache
  * including them ([WHAT] "How to implement" part 1: the cache quantizes on
@@ -280,6 +315,19 @@ int tq_decode_step(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
                    uint32_t* vcodes, float* vnorm, int64_t max_T, const int32_t* pos,
                    float scale, float* out, void* workspace, size_t ws_bytes,
                    void* stream);
+
+/*
+ * tq_decode_step_paged - tq_decode_step over a paged cache (block table and
+ * layout as in tq_attn_decode_paged; the new token of sequence b goes to
+ * position pos[b] as in tq_quantize_append_paged).
+ */
+int tq_decode_step_paged(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
+                         const void* v_new, int kv_dtype, int B, int Hq, int Hkv,
+                         uint32_t* kcodes, uint32_t* kqjl, float* knorm, float* krnorm,
+                         uint32_t* vcodes, float* vnorm, const int32_t* block_table,
+                         int max_blocks, int block_size, int64_t num_blocks,
+                         const int32_t* pos, float scale, float* out, void* workspace,
+                         size_t ws_bytes, void* stream);
 
 /* Bytes of workspace tq_topk needs. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);

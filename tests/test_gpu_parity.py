@@ -456,3 +456,102 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
     assert torch.equal(outA, outB)
     P.check_attention(tab, q.double().cpu().numpy(), P.packed_np(kA), P.packed_np(vA),
                       lens.cpu().numpy(), Hkv, outA.cpu().numpy())
+
+
+# --- paged caches ---------------------------------------------------------------
+def _to_paged(cache, B, Hkv, max_T, bs, perm):
+    """Scatter a contiguous [B, Hkv, max_T, ...] cache into blocks
+    [num_blocks, Hkv, bs, ...]; block i of sequence b is perm[b * mb + i]."""
+    mb = max_T // bs
+    nb = int(perm.max()) + 1
+    out = {}
+    for k, v in cache.items():
+        if v is None:
+            out[k] = None
+            continue
+        tail = tuple(v.shape[3:])
+        pv = torch.full((nb, Hkv, bs) + tail, -3, dtype=v.dtype, device=v.device)
+        blocks = v.reshape((B, Hkv, mb, bs) + tail).transpose(1, 2).reshape((B * mb, Hkv, bs) + tail)
+        pv[perm.long().to(v.device)] = blocks
+        out[k] = pv
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv,bk,bs", [(8, 2, 3, 32), (16, 2, 3, 16), (16, 2, 4, 48), (4, 4, 3, 16)])
+def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs):
+    """The paged decode reads the same records through the block table, so it
+    must reproduce the contiguous decode bit for bit (ragged lengths,
+    partial last blocks, an empty sequence, blocks in shuffled order)."""
+    c = _ctx(128, bk, 4, 128, seed=6)
+    B, d, max_T = 5, 128, 288
+    K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=41).to(cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=42).to(cuda)
+    kc, vc = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    mb = max_T // bs
+    perm = torch.randperm(B * mb + 7, generator=torch.Generator().manual_seed(5))[:B * mb].to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, max_T, bs, perm), _to_paged(vc, B, Hkv, max_T, bs, perm)
+    table = perm.reshape(B, mb).to(cuda)
+    q = tq_inputs.iid((B, Hq, d), seed=43, dtype=torch.bfloat16).to(cuda)
+    lens = torch.tensor([0, 1, bs + 3, 200, max_T], dtype=torch.int32, device=cuda)
+    ref = c.attn_decode(q, kc, vc, lens)
+    got = c.attn_decode_paged(q, kp, vp, table, lens)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv,bk", [(8, 2, 3), (16, 2, 4)])
+def test_paged_decode_step_equals_contiguous(cuda, Hq, Hkv, bk):
+    """decode_step_paged writes the new token into its block slot and attends
+    like decode_step on the equivalent contiguous cache; a sequence whose
+    block id is invalid gets nothing written."""
+    c = _ctx(128, bk, 4, 128, seed=8)
+    B, d, max_T, bs = 4, 128, 128, 32
+    K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=51).to(cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=52).to(cuda)
+    kc, vc = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    mb = max_T // bs
+    perm = torch.randperm(B * mb, generator=torch.Generator().manual_seed(9)).to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, max_T, bs, perm), _to_paged(vc, B, Hkv, max_T, bs, perm)
+    table = perm.reshape(B, mb).to(cuda)
+    q = tq_inputs.iid((B, Hq, d), seed=53, dtype=torch.bfloat16).to(cuda)
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=54)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=55)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([0, 40, 95, 127], dtype=torch.int32, device=cuda)
+    ref = c.decode_step(q, kn, vn, kc, vc, pos)
+    got = c.decode_step_paged(q, kn, vn, kp, vp, table, pos)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
+    kp2, vp2 = _to_paged(kc, B, Hkv, max_T, bs, perm), _to_paged(vc, B, Hkv, max_T, bs, perm)
+    for a_, b_ in ((kp, kp2), (vp, vp2)):
+        for k in a_:
+            if a_[k] is not None:
+                assert torch.equal(a_[k], b_[k]), k
+    # an invalid block id: the append is skipped
+    bad = table.clone()
+    bad[1, 40 // bs] = -1
+    before = {k: (None if v is None else v.clone()) for k, v in kp.items()}
+    c.quantize_append_paged(kn, tq.TQ_KEY, kp, bad, pos)
+    torch.cuda.synchronize()
+    blk = int(table[1, 40 // bs])
+    for k, v in kp.items():
+        if v is not None:
+            assert torch.equal(v[blk], before[k][blk]), k
+
+
+def test_paged_rejections(cuda):
+    c = _ctx(64, 2, 2, 0)
+    q = torch.zeros(1, 2, 64, dtype=torch.bfloat16, device=cuda)
+    kp = c.empty_packed(tq.TQ_KEY, (2, 1, 16), device=cuda)
+    vp = c.empty_packed(tq.TQ_VALUE, (2, 1, 16), device=cuda)
+    table = torch.zeros(1, 2, dtype=torch.int32, device=cuda)
+    lens = torch.ones(1, dtype=torch.int32, device=cuda)
+    with pytest.raises(tq.TQError) as e:
+        c.attn_decode_paged(q, kp, vp, table, lens)
+    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+    c2 = _ctx(128, 3, 4, 128)
+    q2 = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device=cuda)
+    kp2 = c2.empty_packed(tq.TQ_KEY, (2, 1, 24), device=cuda)
+    vp2 = c2.empty_packed(tq.TQ_VALUE, (2, 1, 24), device=cuda)
+    with pytest.raises(tq.TQError) as e:
+        c2.attn_decode_paged(q2, kp2, vp2, table, lens)
+    assert e.value.status == tq.TQ_ERR_ARG
