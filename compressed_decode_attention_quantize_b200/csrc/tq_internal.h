@@ -184,6 +184,19 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cuda
 bool attn_k4_supported(const tq_ctx* c, const AttnArgs& a);
 cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t configure_attn_k4();
+// Top-k on the tensor cores: query blocks of 64 x database chunks.
+struct TopkPlan {
+  int KL, KQ;            // padded centroid and sign widths
+  int64_t chunks, chunk; // database chunks (grid.y), vectors per chunk
+  int nlists;            // candidate lists per query (chunks x 4 warps)
+  size_t qh_bytes, qsc_bytes, cand_bytes, smem;
+};
+TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k);
+cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const float* qr, const float* qs,
+                            int64_t nq, const uint32_t* codes, const uint32_t* qjl, const float* norm,
+                            const float* rnorm, int64_t n, int k, void* qh, float* qsc, float* cand_v,
+                            int* cand_i, cudaStream_t s);
+cudaError_t configure_topk_mma();
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
                           const float* krnorm, int64_t nk, float* out, cudaStream_t s);

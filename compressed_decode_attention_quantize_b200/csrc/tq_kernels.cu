@@ -886,153 +886,12 @@ __global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int 
 }
 
 // ----------------------------------------------------------------------------
-// Top-k.  Phase 1: CTA (chunk, query tile) scores TQ queries against a chunk
-// of the database, 256 vectors per step (one per thread), and keeps each
-// query's running top-k in shared memory by warp-wide selection.  Phase 2:
-// one warp per query selects the final top-k from all chunk lists.
+// Top-k, final phase: one warp per query selects the k best of all candidate
+// lists written by the tensor-core scoring kernel (tq_topk_mma.cu).
 // Order: score descending, then index ascending.
 // ----------------------------------------------------------------------------
-constexpr int TQ = 16;      // queries per CTA
-constexpr int TTH = 256;    // threads (= database vectors per step)
-constexpr int TSTEPS = 32;  // steps per chunk
-constexpr int TKMAX = 32;
-
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
-}
-
-template <int J>
-__global__ void __launch_bounds__(TTH) k_topk_chunk(const float* qr, const float* qs, int64_t nq,
-                                                    int d, int bk, int kw, int m, const float* ck,
-                                                    float cq,
-                                                    const uint32_t* codes, const uint32_t* qjl,
-                                                    const float* norm, const float* rnorm,
-                                                    int64_t n, int K, float* cand_v, int* cand_i,
-                                                    int nchunks) {
-  constexpr int DP = J * 32;
-  extern __shared__ float sh[];
-  float* sq = sh;                    // [DP][TQ]
-  float* ssv = sq + DP * TQ;         // [DP][TQ]
-  float* sscore = ssv + DP * TQ;     // [TQ][TTH]
-  float* stop_v = sscore + TQ * TTH; // [TQ][TKMAX]
-  int* stop_i = reinterpret_cast<int*>(stop_v + TQ * TKMAX);
-  __shared__ float s_ck[16];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t q0 = (int64_t)blockIdx.y * TQ;
-  const int chunk = blockIdx.x;
-  if (tid < 16) s_ck[tid] = (tid < (1 << bk)) ? ck[tid] : 0.f;
-  for (int e = tid; e < DP * TQ; e += TTH) {
-    const int j = e / TQ, qq = e % TQ;
-    const bool ok = q0 + qq < nq;
-    sq[e] = ok ? qr[(q0 + qq) * DP + j] : 0.f;
-    ssv[e] = ok ? qs[(q0 + qq) * DP + j] : 0.f;
-  }
-  for (int e = tid; e < TQ * TKMAX; e += TTH) {
-    stop_v[e] = kNegInf;
-    stop_i[e] = INT_MAX;
-  }
-  __syncthreads();
-  const int mw = (m + 31) >> 5;
-  const int64_t base = (int64_t)chunk * TSTEPS * TTH;
-  for (int step = 0; step < TSTEPS; ++step) {
-    const int64_t v = base + (int64_t)step * TTH + tid;
-    if (v < n) {
-      uint32_t w[4 * 8];
-      for (int e = 0; e < kw; ++e) w[e] = codes[v * kw + e];
-      float acc[TQ], acc2[TQ];
-#pragma unroll
-      for (int qq = 0; qq < TQ; ++qq) acc[qq] = acc2[qq] = 0.f;
-      for (int j = 0; j < d; ++j) {
-        const float c = s_ck[code_index(w, bk, d, j)];
-        const float4* qp = reinterpret_cast<const float4*>(sq + j * TQ);
-#pragma unroll
-        for (int q4 = 0; q4 < TQ / 4; ++q4) {
-          const float4 qv = qp[q4];
-          acc[4 * q4 + 0] = fmaf(qv.x, c, acc[4 * q4 + 0]);
-          acc[4 * q4 + 1] = fmaf(qv.y, c, acc[4 * q4 + 1]);
-          acc[4 * q4 + 2] = fmaf(qv.z, c, acc[4 * q4 + 2]);
-          acc[4 * q4 + 3] = fmaf(qv.w, c, acc[4 * q4 + 3]);
-        }
-      }
-      for (int wi = 0; wi < mw; ++wi) {
-        const uint32_t bitsw = qjl[v * mw + wi];
-        const int lim = min(32, m - 32 * wi);
-        for (int e = 0; e < lim; ++e) {
-          const float sg = ((bitsw >> e) & 1u) ? 1.f : -1.f;
-          const float4* sp = reinterpret_cast<const float4*>(ssv + (32 * wi + e) * TQ);
-#pragma unroll
-          for (int q4 = 0; q4 < TQ / 4; ++q4) {
-            const float4 sv = sp[q4];
-            acc2[4 * q4 + 0] = fmaf(sg, sv.x, acc2[4 * q4 + 0]);
-            acc2[4 * q4 + 1] = fmaf(sg, sv.y, acc2[4 * q4 + 1]);
-            acc2[4 * q4 + 2] = fmaf(sg, sv.z, acc2[4 * q4 + 2]);
-            acc2[4 * q4 + 3] = fmaf(sg, sv.w, acc2[4 * q4 + 3]);
-          }
-        }
-      }
-      const float kn = norm[v];
-      const float kg = m > 0 ? rnorm[v] * cq : 0.f;
-#pragma unroll
-      for (int qq = 0; qq < TQ; ++qq) sscore[qq * TTH + tid] = kn * acc[qq] + kg * acc2[qq];
-    } else {
-#pragma unroll
-      for (int qq = 0; qq < TQ; ++qq) sscore[qq * TTH + tid] = kNegInf;
-    }
-    __syncthreads();
-    // Merge: warp w handles queries w, w+8, ...
-    for (int qq = warp; qq < TQ; qq += TTH / 32) {
-      const float kth_v = stop_v[qq * TKMAX + K - 1];
-      const int kth_i = stop_i[qq * TKMAX + K - 1];
-      float vals[TTH / 32 + 1];
-      int ids[TTH / 32 + 1];
-      bool any = false;
-#pragma unroll
-      for (int e = 0; e < TTH / 32; ++e) {
-        const int t = lane + 32 * e;
-        vals[e] = sscore[qq * TTH + t];
-        ids[e] = (int)(base + (int64_t)step * TTH + t);
-        if (vals[e] == kNegInf) ids[e] = INT_MAX;
-        any |= better(vals[e], ids[e], kth_v, kth_i);
-      }
-      if (!__any_sync(0xffffffffu, any)) continue;
-      vals[TTH / 32] = (lane < K) ? stop_v[qq * TKMAX + lane] : kNegInf;
-      ids[TTH / 32] = (lane < K) ? stop_i[qq * TKMAX + lane] : INT_MAX;
-      float nv = kNegInf;
-      int ni = INT_MAX;
-      for (int r = 0; r < K; ++r) {
-        float bv = vals[0];
-        int bi = ids[0];
-#pragma unroll
-        for (int e = 1; e <= TTH / 32; ++e)
-          if (better(vals[e], ids[e], bv, bi)) { bv = vals[e]; bi = ids[e]; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        if (lane == r) { nv = bv; ni = bi; }
-#pragma unroll
-        for (int e = 0; e <= TTH / 32; ++e)
-          if (ids[e] == bi && vals[e] == bv) { vals[e] = kNegInf; ids[e] = INT_MAX; }
-      }
-      __syncwarp();
-      if (lane < K) {
-        stop_v[qq * TKMAX + lane] = nv;
-        stop_i[qq * TKMAX + lane] = ni;
-      }
-      __syncwarp();
-    }
-    __syncthreads();
-  }
-  for (int e = tid; e < TQ * K; e += TTH) {
-    const int qq = e / K, r = e % K;
-    if (q0 + qq < nq) {
-      const int64_t o = ((q0 + qq) * nchunks + chunk) * K + r;
-      cand_v[o] = stop_v[qq * TKMAX + r];
-      cand_i[o] = stop_i[qq * TKMAX + r];
-    }
-  }
 }
 
 __global__ void __launch_bounds__(32) k_topk_final(const float* cand_v, const int* cand_i,
@@ -1199,15 +1058,11 @@ cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
   return cudaGetLastError();
 }
 
-static int64_t topk_chunks(int64_t n) {
-  const int64_t per = (int64_t)TSTEPS * TTH;
-  return (n + per - 1) / per;
-}
-
 size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k) {
-  const int64_t nch = topk_chunks(n > 0 ? n : 1);
-  size_t b = 2 * (size_t)nq * c->dpad * sizeof(float);        // q', s
-  b += (size_t)nq * nch * k * (sizeof(float) + sizeof(int));  // candidates
+  const TopkPlan p = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
+  size_t b = 2 * (((size_t)nq * c->dpad * sizeof(float) + 255) & ~(size_t)255);   // q', s
+  b += ((p.qh_bytes + 255) & ~(size_t)255) + ((p.qsc_bytes + 255) & ~(size_t)255);
+  b += (((size_t)nq * p.nlists * k * sizeof(float) + 255) & ~(size_t)255) * 2;     // candidates
   return b + 1024;
 }
 
@@ -1216,7 +1071,7 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                         const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
                         void* ws, cudaStream_t s) {
   if (nq == 0) return cudaSuccess;
-  const int64_t nch = topk_chunks(n > 0 ? n : 1);
+  const TopkPlan pl = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
   char* p = static_cast<char*>(ws);
   auto take = [&](size_t bytes) {
     char* r = p;
@@ -1225,22 +1080,15 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   };
   float* qr = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
   float* qs = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
-  float* cv = reinterpret_cast<float*>(take((size_t)nq * nch * k * sizeof(float)));
-  int* ci = reinterpret_cast<int*>(take((size_t)nq * nch * k * sizeof(int)));
+  void* qh = take(pl.qh_bytes);
+  float* qsc = reinterpret_cast<float*>(take(pl.qsc_bytes));
+  float* cv = reinterpret_cast<float*>(take((size_t)nq * pl.nlists * k * sizeof(float)));
+  int* ci = reinterpret_cast<int*>(take((size_t)nq * pl.nlists * k * sizeof(int)));
   cudaError_t e = launch_prerotate(c, q, dtype, nq, nullptr, qr, qs, s);
   if (e != cudaSuccess) return e;
-  const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
-  const size_t shm = (size_t)(2 * c->dpad * TQ + TQ * TTH + TQ * TKMAX) * sizeof(float) +
-                     (size_t)TQ * TKMAX * sizeof(int);
-  dim3 grid((unsigned)nch, (unsigned)((nq + TQ - 1) / TQ));
-  TQ_DISPATCH_J(c->J, {
-    k_topk_chunk<JV><<<grid, TTH, shm, s>>>(qr, qs, nq, c->d, c->bk_lm, c->wk, c->qjl_m, c->ck_f, cq,
-                                             codes, qjl, norm, rnorm, n, k, cv, ci, (int)nch);
-    break;
-  });
-  e = cudaGetLastError();
+  e = launch_topk_mma(c, pl, qr, qs, nq, codes, qjl, norm, rnorm, n, k, qh, qsc, cv, ci, s);
   if (e != cudaSuccess) return e;
-  k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, (int)nch, k, idx, score);
+  k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, pl.nlists, k, idx, score);
   return cudaGetLastError();
 }
 
@@ -1253,9 +1101,7 @@ static cudaError_t configure_J() {
   if (e != cudaSuccess) return e;
   const int attn_max = (2 * GMAX * J * 32 + AT * GMAX) * (int)sizeof(float) + AT * 32 * (int)sizeof(uint32_t);
   e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_max);
-  if (e != cudaSuccess) return e;
-  const int topk = (2 * J * 32 * TQ + TQ * TTH + TQ * TKMAX) * (int)sizeof(float) + TQ * TKMAX * (int)sizeof(int);
-  return cudaFuncSetAttribute(k_topk_chunk<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, topk);
+  return e;
 }
 
 cudaError_t configure_kernels() {
@@ -1278,6 +1124,7 @@ cudaError_t configure_kernels() {
   if ((e = cudaFuncSetAttribute(k_step_prep, ms, small_smem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   if ((e = configure_attn_k4()) != cudaSuccess) return e;
+  if ((e = configure_topk_mma()) != cudaSuccess) return e;
   return configure_attn_mma();
 }
 
