@@ -184,9 +184,10 @@ cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cuda
 bool attn_k4_supported(const tq_ctx* c, const AttnArgs& a);
 cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t configure_attn_k4();
-// Top-k on the tensor cores: query blocks of 64 x database chunks.
+// Top-k on the tensor cores: query blocks of 64 or 128 x database chunks.
 struct TopkPlan {
   int KL, KQ;            // padded centroid and sign widths
+  int qb;                // queries per CTA (64 or 128)
   int64_t chunks, chunk; // database chunks (grid.y), vectors per chunk
   int nlists;            // candidate lists per query (chunks x 4 warps)
   size_t qh_bytes, qsc_bytes, cand_bytes, smem;

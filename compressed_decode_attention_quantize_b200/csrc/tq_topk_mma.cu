@@ -26,10 +26,8 @@
 namespace tqk {
 namespace {
 
-constexpr int TKQ = 64;     // queries per CTA
 constexpr int TKR = 64;     // database vectors per tile
-constexpr int TKWARPS = 8;  // warp w: rows 16 (w & 3) .. +15, queries 32 (w >> 2) .. +31
-constexpr int TKMAX = 32;   // largest k
+constexpr int TKWARPS = 8;  // warp w: rows 16 (w & 3) .. +15, queries QB/2 (w >> 2) .. + QB/2 - 1
 constexpr int TKLISTS = 4;  // lists per query and chunk (the four row groups)
 
 __device__ __forceinline__ bool better_sc(float va, int ia, float vb, int ib) {
@@ -100,36 +98,40 @@ struct TopkMmaArgs {
   int* cand_i;
 };
 
-// Shared memory: B rows [TKQ][KS] and A rows [TKR][KS] in fp16 (KS = KL + KQ
-// + 8: an odd number of 16-byte chunks per row, so ldmatrix rows hit distinct
-// banks), the tile's codes and signs, norms, query scales, the pair table
-// (two coordinates' indices -> half2 of centroids, up to 256 entries) and the
-// per-warp lists [TKWARPS][TKQ / 2][K] of (score, index).
-__host__ __device__ inline size_t topk_mma_smem(int KL, int KQ, int kw, int qw, int K) {
+// Shared memory for QB queries per CTA: B rows [QB][KS] and A rows [TKR][KS]
+// in fp16 (KS = KL + KQ + 8: an odd number of 16-byte chunks per row, so
+// ldmatrix rows hit distinct banks), two staging buffers of the tile's codes,
+// signs and norms, query scales, the pair table (two coordinates' indices ->
+// half2 of centroids, up to 256 entries) and the per-warp lists
+// [TKWARPS][QB / 2][K] of (score, index).
+__host__ __device__ inline size_t topk_mma_smem(int QB, int KL, int KQ, int kw, int qw, int K) {
   const size_t KS = (size_t)KL + KQ + 8;
-  return 2 * KS * (TKQ + TKR) + 2 * (size_t)TKR * (kw + qw + 2) * 4 + (size_t)TKQ * 2 * 4 + 256 * 4 +
-         (size_t)TKWARPS * (TKQ / 2) * K * 8 + 64;
+  return 2 * KS * (QB + TKR) + 2 * (size_t)TKR * (kw + qw + 2) * 4 + (size_t)QB * 2 * 4 + 256 * 4 +
+         (size_t)TKWARPS * (QB / 2) * K * 8 + 64;
 }
 
-template <int BK>
+template <int BK, int QB>
 __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
+  constexpr int QH = QB / 2;     // queries per warp
+  constexpr int NTW = QH / 8;    // n-tiles per warp
+  constexpr int SL = 2 * NTW;    // (query) slots per thread
   extern __shared__ __align__(16) unsigned char smem[];
   const int KS = a.KL + a.KQ + 8;
   __half* sB = reinterpret_cast<__half*>(smem);
-  __half* sA = sB + (size_t)TKQ * KS;
+  __half* sA = sB + (size_t)QB * KS;
   // Two staging buffers (tile i and i + 1): codes [TKR][kw], signs [TKR][qw],
   // norms [TKR], rnorms [TKR].
   const int stage_words = TKR * (a.kw + a.qw + 2);
   uint32_t* sStage = reinterpret_cast<uint32_t*>(sA + (size_t)TKR * KS);
-  float* sQ = reinterpret_cast<float*>(sStage + 2 * stage_words);       // [TKQ][2]: 2^e, 2^f
-  uint32_t* sP = reinterpret_cast<uint32_t*>(sQ + TKQ * 2);              // [256] pair table
-  float* lv = reinterpret_cast<float*>(sP + 256);                        // [TKWARPS][TKQ/2][K]
-  int* li = reinterpret_cast<int*>(lv + TKWARPS * (TKQ / 2) * a.K);
+  float* sQ = reinterpret_cast<float*>(sStage + 2 * stage_words);       // [QB][2]: 2^e, 2^f
+  uint32_t* sP = reinterpret_cast<uint32_t*>(sQ + QB * 2);               // [256] pair table
+  float* lv = reinterpret_cast<float*>(sP + 256);                        // [TKWARPS][QH][K]
+  int* li = reinterpret_cast<int*>(lv + TKWARPS * QH * a.K);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rg = warp & 3, qg = warp >> 2;   // row group, query half
-  const int64_t q0 = (int64_t)blockIdx.x * TKQ;
+  const int64_t q0 = (int64_t)blockIdx.x * QB;
   const int64_t n0 = (int64_t)blockIdx.y * a.chunk;
   const int64_t n1 = min(a.n, n0 + a.chunk);
   const int KP = a.KL + a.KQ;
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
     const __half2 hv = __floats2half2_rn(ok ? a.ck[i0] : 0.f, ok ? a.ck[i1] : 0.f);
     sP[e] = *reinterpret_cast<const uint32_t*>(&hv);
   }
-  for (int e = tid; e < TKQ * KP / 8; e += TKWARPS * 32) {
+  for (int e = tid; e < QB * KP / 8; e += TKWARPS * 32) {
     const int r = e / (KP / 8), c8 = e % (KP / 8);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (q0 + r < a.nq) v = reinterpret_cast<const uint4*>(a.qh + (q0 + r) * KP)[c8];
@@ -164,8 +166,8 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   // Centroid columns past the code words (d < KL with < 16 fields per word):
   // zero once, no tile writes them.
   for (int e = tid; e < TKR * KS; e += TKWARPS * 32) sA[e] = __float2half_rn(0.f);
-  for (int e = tid; e < TKQ * 2; e += TKWARPS * 32) sQ[e] = (q0 + e / 2 < a.nq) ? a.qsc[q0 * 2 + e] : 0.f;
-  for (int e = tid; e < TKWARPS * (TKQ / 2) * a.K; e += TKWARPS * 32) {
+  for (int e = tid; e < QB * 2; e += TKWARPS * 32) sQ[e] = (q0 + e / 2 < a.nq) ? a.qsc[q0 * 2 + e] : 0.f;
+  for (int e = tid; e < TKWARPS * QH * a.K; e += TKWARPS * 32) {
     lv[e] = -INFINITY;
     li[e] = INT_MAX;
   }
@@ -177,14 +179,14 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   // B tiles (n-tile nt / nt+1) x (k 0-7 / 8-15) of this warp's 32 queries.
   const int ti = lane >> 3, tr = lane & 7;
   const uint32_t a_row = sA_s + (uint32_t)((16 * rg + tr + 8 * (ti & 1)) * KS + 8 * (ti >> 1)) * 2;
-  const uint32_t b_row = sB_s + (uint32_t)((32 * qg + 8 * (ti >> 1) + tr) * KS + 8 * (ti & 1)) * 2;
-  float* mylv = lv + warp * (TKQ / 2) * a.K;
-  int* myli = li + warp * (TKQ / 2) * a.K;
-  // Current worst entry of this thread's 8 queries (4 n-tiles x 2 columns).
-  float wv[8];
-  int wi[8];
+  const uint32_t b_row = sB_s + (uint32_t)((QH * qg + 8 * (ti >> 1) + tr) * KS + 8 * (ti & 1)) * 2;
+  float* mylv = lv + warp * QH * a.K;
+  int* myli = li + warp * QH * a.K;
+  // Current worst entry of this thread's SL queries (NTW n-tiles x 2 columns).
+  float wv[SL];
+  int wi[SL];
 #pragma unroll
-  for (int s = 0; s < 8; ++s) {
+  for (int s = 0; s < SL; ++s) {
     wv[s] = -INFINITY;
     wi[s] = INT_MAX;
   }
@@ -224,15 +226,24 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
         const uint32_t w = live ? sC[r * a.kw + wd] : 0u;
         uint32_t tw = 0u;
         if (bk == 3 && live) tw = sC[r * a.kw + W2 + (wd >> 1)] >> (16 * (wd & 1));
+        if (live && per * (wd + 1) <= a.d) {   // every coordinate of the word is real
 #pragma unroll
-        for (int j = 0; j < pairs_w; ++j) {
-          const int c = per * wd + 2 * j;   // first coordinate of the pair
-          uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
-          if (bk == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
-          uint32_t h2 = sP[idx];
-          if (!live || c >= a.d) h2 = 0u;
-          else if (c + 1 >= a.d) h2 &= 0xFFFFu;
-          if (c < a.KL) dst[j] = h2;
+          for (int j = 0; j < pairs_w; ++j) {
+            uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
+            if (bk == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
+            dst[j] = sP[idx];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < pairs_w; ++j) {
+            const int c = per * wd + 2 * j;   // first coordinate of the pair
+            uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
+            if (bk == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
+            uint32_t h2 = sP[idx];
+            if (!live || c >= a.d) h2 = 0u;
+            else if (c + 1 >= a.d) h2 &= 0xFFFFu;
+            if (c < a.KL) dst[j] = h2;
+          }
         }
       }
       for (int wd = tid >> 6; wd < a.qw; wd += TKWARPS * 32 / TKR) {
@@ -252,17 +263,17 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
     }
     __syncthreads();
 
-    // ---- scores of rows 16 rg .. +15 against queries 32 qg .. +31 ----------------------
-    float acc[4][4], acs[4][4];
+    // ---- scores of rows 16 rg .. +15 against queries QH qg .. + QH - 1 -------------------
+    float acc[NTW][4], acs[NTW][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NTW; ++nt)
 #pragma unroll
       for (int r = 0; r < 4; ++r) acc[nt][r] = acs[nt][r] = 0.f;
     for (int ks = 0; ks < a.KL / 16; ++ks) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4(a_row + ks * 32, a0, a1, a2, a3);
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
+      for (int np = 0; np < NTW / 2; ++np) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(b_row + (uint32_t)(16 * np * KS) * 2 + ks * 32, b0, b1, b2, b3);
         mma_f16(acc[2 * np], a0, a1, a2, a3, b0, b1);
@@ -273,7 +284,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4(a_row + ks * 32, a0, a1, a2, a3);
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
+      for (int np = 0; np < NTW / 2; ++np) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(b_row + (uint32_t)(16 * np * KS) * 2 + ks * 32, b0, b1, b2, b3);
         mma_f16(acs[2 * np], a0, a1, a2, a3, b0, b1);
@@ -281,18 +292,18 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       }
     }
 
-    // ---- candidates: slot s = 2 nt + col (query 32 qg + 8 nt + 2 t + col) ----------
+    // ---- candidates: slot s = 2 nt + col (query QH qg + 8 nt + 2 t + col) ----------
     const int ra = 16 * rg + g, rb = ra + 8;
     const bool va = ra < rows, vb = rb < rows;
     const float na = va ? sNn[ra] : 0.f, ga = (va && a.m > 0) ? sNn[TKR + ra] * a.cq : 0.f;
     const float nb = vb ? sNn[rb] : 0.f, gb = (vb && a.m > 0) ? sNn[TKR + rb] * a.cq : 0.f;
-    float sc[8][2];
+    float sc[SL][2];
     uint32_t mask = 0u;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < NTW; ++nt) {
 #pragma unroll
       for (int col = 0; col < 2; ++col) {
-        const int s = 2 * nt + col, ql = 32 * qg + 8 * nt + 2 * t + col;
+        const int s = 2 * nt + col, ql = QH * qg + 8 * nt + 2 * t + col;
         const float fe = sQ[2 * ql], ff = sQ[2 * ql + 1];
         sc[s][0] = va ? fmaf(na * fe, acc[nt][col], ga * ff * acs[nt][col]) : -INFINITY;
         sc[s][1] = vb ? fmaf(nb * fe, acc[nt][2 + col], gb * ff * acs[nt][2 + col]) : -INFINITY;
@@ -309,11 +320,11 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       const int s = bit >> 1, row = bit & 1, lt = leader & 3;
       float mine = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
+      for (int k = 0; k < 2 * SL; ++k)
         if (k == bit) mine = sc[k >> 1][k & 1];
       const float val = __shfl_sync(0xffffffffu, mine, leader);
       const int idx = (int)(v0 + 16 * rg + (leader >> 2) + 8 * row);
-      const int ql = 8 * (s >> 1) + 2 * lt + (s & 1);   // within this warp's 32 queries
+      const int ql = 8 * (s >> 1) + 2 * lt + (s & 1);   // within this warp's QH queries
       if (lane == leader) mask &= mask - 1u;
       float nwv = 0.f;
       int nwi = 0;
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       if (t == lt) {
         // Raise this query's bar and drop the candidates it no longer passes.
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < SL; ++k) {
           if (k == s) {
             wv[k] = nwv;
             wi[k] = nwi;
@@ -355,9 +366,9 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
 
   // ---- this warp's lists -> candidates of (query, chunk, row group) ------------------
   const int list = (int)blockIdx.y * TKLISTS + rg;
-  for (int e = lane; e < (TKQ / 2) * a.K; e += 32) {
+  for (int e = lane; e < QH * a.K; e += 32) {
     const int ql = e / a.K, r = e % a.K;
-    const int64_t q = q0 + 32 * qg + ql;
+    const int64_t q = q0 + QH * qg + ql;
     if (q < a.nq) {
       const int64_t o = (q * a.nlists + list) * a.K + r;
       a.cand_v[o] = mylv[ql * a.K + r];
@@ -372,7 +383,10 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   TopkPlan p{};
   p.KL = (c->d + 15) / 16 * 16;
   p.KQ = (c->qjl_m + 15) / 16 * 16;
-  const int64_t qblocks = (nq + TKQ - 1) / TKQ;
+  const int qw = (c->qjl_m + 31) / 32;
+  // 128 queries per CTA (more products per dequantized tile) when it fits.
+  p.qb = topk_mma_smem(128, p.KL, p.KQ, c->wk, qw, k) <= (size_t)227 * 1024 ? 128 : 64;
+  const int64_t qblocks = (nq + p.qb - 1) / p.qb;
   int64_t chunks = (2 * (int64_t)c->sms + qblocks - 1) / (qblocks > 0 ? qblocks : 1);
   const int64_t max_chunks = (n + 8 * TKR - 1) / (8 * TKR);   // at least eight tiles per chunk
   if (chunks > max_chunks) chunks = max_chunks;
@@ -384,7 +398,7 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   p.qh_bytes = (size_t)nq * (p.KL + p.KQ) * sizeof(__half);
   p.qsc_bytes = (size_t)nq * 2 * sizeof(float);
   p.cand_bytes = (size_t)nq * p.nlists * k * (sizeof(float) + sizeof(int));
-  p.smem = topk_mma_smem(p.KL, p.KQ, c->wk, (c->qjl_m + 31) / 32, k);
+  p.smem = topk_mma_smem(p.qb, p.KL, p.KQ, c->wk, qw, k);
   return p;
 }
 
@@ -419,27 +433,34 @@ cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const float* qr,
   a.nlists = p.nlists;
   a.cand_v = cand_v;
   a.cand_i = cand_i;
-  dim3 grid((unsigned)((nq + TKQ - 1) / TKQ), (unsigned)p.chunks);
-  switch (c->bk_lm) {
-    case 1: k_topk_mma<1><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 2: k_topk_mma<2><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 3: k_topk_mma<3><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 4: k_topk_mma<4><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+  dim3 grid((unsigned)((nq + p.qb - 1) / p.qb), (unsigned)p.chunks);
+  const bool wide = p.qb == 128;
+  switch (c->bk_lm * 2 + (wide ? 1 : 0)) {
+    case 2: k_topk_mma<1, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 3: k_topk_mma<1, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 4: k_topk_mma<2, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 5: k_topk_mma<2, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 6: k_topk_mma<3, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 7: k_topk_mma<3, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 8: k_topk_mma<4, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
+    case 9: k_topk_mma<4, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
 cudaError_t configure_topk_mma() {
-  // d, m <= 256, the widest code record (4-bit fields: 32 words) and k = 32:
-  // the largest shared-memory need.
-  const int worst = (int)topk_mma_smem(256, 256, 32, 8, TKMAX);
+  const int lim = 227 * 1024;   // the plan never asks for more
   const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<1>, ms, worst))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<2>, ms, worst))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<3>, ms, worst))) return e;
-  return cudaFuncSetAttribute(k_topk_mma<4>, ms, worst);
+  if ((e = cudaFuncSetAttribute(k_topk_mma<1, 64>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<1, 128>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<2, 64>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<2, 128>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<3, 64>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<3, 128>, ms, lim))) return e;
+  if ((e = cudaFuncSetAttribute(k_topk_mma<4, 64>, ms, lim))) return e;
+  return cudaFuncSetAttribute(k_topk_mma<4, 128>, ms, lim);
 }
 
 }  // namespace tqk

@@ -262,8 +262,9 @@ def _oracle_topk_chunked(tab, q, g, k, chunk=25_000):
     best_i = np.zeros((q.shape[0], 0), dtype=np.int64)
     for s in range(0, n, chunk):
         e = min(n, s + chunk)
-        sc = o.logits(tab, q, g["codes"][s:e], g["norm"][s:e],
-                      g["qjl"][s:e].reshape(e - s, -1), g["rnorm"][s:e])
+        qj = None if g["qjl"] is None else g["qjl"][s:e].reshape(e - s, -1)
+        rn = None if g["rnorm"] is None else g["rnorm"][s:e]
+        sc = o.logits(tab, q, g["codes"][s:e], g["norm"][s:e], qj, rn)
         best_v = np.concatenate([best_v, sc], axis=1)
         best_i = np.concatenate([best_i, np.broadcast_to(np.arange(s, e), sc.shape)], axis=1)
         order = np.lexsort((best_i, -best_v), axis=1)[:, :k]
@@ -283,8 +284,9 @@ def _check_topk(tab, q, g, idx, score, k):
             diff = set(idx[r]) ^ set(ref_i[r])
             kth = ref_v[r, -1]
             for j in diff:
-                sc = o.logits(tab, q[r:r + 1], g["codes"][j:j + 1],
-                              g["norm"][j:j + 1], g["qjl"][j:j + 1].reshape(1, -1), g["rnorm"][j:j + 1])[0, 0]
+                qj = None if g["qjl"] is None else g["qjl"][j:j + 1].reshape(1, -1)
+                rn = None if g["rnorm"] is None else g["rnorm"][j:j + 1]
+                sc = o.logits(tab, q[r:r + 1], g["codes"][j:j + 1], g["norm"][j:j + 1], qj, rn)[0, 0]
                 assert abs(sc - kth) <= 2 * tol, (r, j, sc, kth)
 
 
@@ -305,6 +307,22 @@ def test_topk_small_with_ties_and_short_db(cuda):
     torch.cuda.synchronize()
     assert np.all(idx2.cpu().numpy()[:, 5:] == -1) and np.all(np.isneginf(score2.cpu().numpy()[:, 5:]))
     assert sorted(idx2.cpu().numpy()[0, :5].tolist()) == [0, 1, 2, 3, 4]
+
+
+@pytest.mark.parametrize("d,bk,m,k", [(128, 3, 128, 32), (64, 2, 0, 1), (200, 5, 200, 16), (96, 2, 64, 12)])
+def test_topk_code_widths_and_k(cuda, d, bk, m, k):
+    """Every packed width (1 to 4 Lloyd-Max bits, with and without QJL),
+    k from 1 to 32 (both query-block sizes of the tensor-core scorer), and
+    more queries than one block with a ragged last block."""
+    c = _ctx(d, bk, 3, m, seed=13)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(3000, d, seed=31)
+    Q = tq_inputs.mixture(150, d, seed=32, means_seed=31)
+    db = c.quantize(X.to(cuda), tq.TQ_KEY)
+    idx, score = c.topk(Q.to(cuda), db, k)
+    torch.cuda.synchronize()
+    g = _flat(db, 3000)
+    _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), k)
 
 
 def test_topk_vector_search_full(cuda):
