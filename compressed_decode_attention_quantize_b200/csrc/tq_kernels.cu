@@ -1058,11 +1058,21 @@ cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
   return cudaGetLastError();
 }
 
+// Two passes when the database is large: the k-th best of the first
+// kTopkSample vectors sets every list's starting bar, so the full pass
+// inserts almost nothing.
+constexpr int64_t kTopkSample = 32768;
+
+static size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
+
 size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   const TopkPlan p = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
-  size_t b = 2 * (((size_t)nq * c->dpad * sizeof(float) + 255) & ~(size_t)255);   // q', s
-  b += ((p.qh_bytes + 255) & ~(size_t)255) + ((p.qsc_bytes + 255) & ~(size_t)255);
-  b += (((size_t)nq * p.nlists * k * sizeof(float) + 255) & ~(size_t)255) * 2;     // candidates
+  const TopkPlan ps = topk_mma_sample_plan(p, kTopkSample, c->sms);
+  size_t b = 2 * up256((size_t)nq * c->dpad * sizeof(float));                 // q', s
+  b += up256(p.qh_bytes) + up256(p.qsc_bytes);
+  b += 2 * up256((size_t)nq * p.nlists * k * sizeof(float));                  // candidates
+  b += 2 * up256((size_t)nq * ps.nlists * k * sizeof(float));                 // sample candidates
+  b += 2 * up256((size_t)nq * k * sizeof(float));                             // bars
   return b + 1024;
 }
 
@@ -1072,10 +1082,11 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                         void* ws, cudaStream_t s) {
   if (nq == 0) return cudaSuccess;
   const TopkPlan pl = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
+  const TopkPlan ps = topk_mma_sample_plan(pl, kTopkSample, c->sms);
   char* p = static_cast<char*>(ws);
   auto take = [&](size_t bytes) {
     char* r = p;
-    p += (bytes + 255) & ~(size_t)255;
+    p += up256(bytes);
     return r;
   };
   float* qr = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
@@ -1084,9 +1095,23 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   float* qsc = reinterpret_cast<float*>(take(pl.qsc_bytes));
   float* cv = reinterpret_cast<float*>(take((size_t)nq * pl.nlists * k * sizeof(float)));
   int* ci = reinterpret_cast<int*>(take((size_t)nq * pl.nlists * k * sizeof(int)));
+  float* scv = reinterpret_cast<float*>(take((size_t)nq * ps.nlists * k * sizeof(float)));
+  int* sci = reinterpret_cast<int*>(take((size_t)nq * ps.nlists * k * sizeof(int)));
+  float* barv = reinterpret_cast<float*>(take((size_t)nq * k * sizeof(float)));
+  int32_t* bari = reinterpret_cast<int32_t*>(take((size_t)nq * k * sizeof(int32_t)));
   cudaError_t e = launch_prerotate(c, q, dtype, nq, nullptr, qr, qs, s);
   if (e != cudaSuccess) return e;
-  e = launch_topk_mma(c, pl, qr, qs, nq, codes, qjl, norm, rnorm, n, k, qh, qsc, cv, ci, s);
+  if ((e = launch_topk_qprep(c, pl, qr, qs, nq, qh, qsc, s)) != cudaSuccess) return e;
+  const bool two_pass = n >= 4 * kTopkSample;
+  if (two_pass) {
+    e = launch_topk_mma(c, ps, qh, qsc, nq, codes, qjl, norm, rnorm, kTopkSample, k, nullptr, nullptr, scv,
+                        sci, s);
+    if (e != cudaSuccess) return e;
+    k_topk_final<<<(unsigned)nq, 32, 0, s>>>(scv, sci, ps.nlists, k, bari, barv);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  e = launch_topk_mma(c, pl, qh, qsc, nq, codes, qjl, norm, rnorm, n, k, two_pass ? barv : nullptr,
+                      two_pass ? bari : nullptr, cv, ci, s);
   if (e != cudaSuccess) return e;
   k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, pl.nlists, k, idx, score);
   return cudaGetLastError();

@@ -93,9 +93,14 @@ struct TopkMmaArgs {
   const float* norm;
   const float* rnorm;
   int64_t n, chunk;   // database size, vectors per chunk (multiple of TKR)
+  int64_t chunks, qblocks;   // work items = qblocks x chunks, taken round-robin
   int K, nlists;
   float* cand_v;
   int* cand_i;
+  // Optional starting bar per query: entry (q, K - 1) of bar_v / bar_i
+  // ([nq][K], index -1 = none), the k-th best of a sample of the database.
+  const float* bar_v;
+  const int* bar_i;
 };
 
 // Shared memory for QB queries per CTA: B rows [QB][KS] and A rows [TKR][KS]
@@ -131,9 +136,6 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rg = warp & 3, qg = warp >> 2;   // row group, query half
-  const int64_t q0 = (int64_t)blockIdx.x * QB;
-  const int64_t n0 = (int64_t)blockIdx.y * a.chunk;
-  const int64_t n1 = min(a.n, n0 + a.chunk);
   const int KP = a.KL + a.KQ;
   constexpr int bk = BK;
   // Code words: main (b = 3: low-bit) stream of W2 words with `per` fields each.
@@ -157,21 +159,9 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
     const __half2 hv = __floats2half2_rn(ok ? a.ck[i0] : 0.f, ok ? a.ck[i1] : 0.f);
     sP[e] = *reinterpret_cast<const uint32_t*>(&hv);
   }
-  for (int e = tid; e < QB * KP / 8; e += TKWARPS * 32) {
-    const int r = e / (KP / 8), c8 = e % (KP / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (q0 + r < a.nq) v = reinterpret_cast<const uint4*>(a.qh + (q0 + r) * KP)[c8];
-    *reinterpret_cast<uint4*>(sB + (size_t)r * KS + 8 * c8) = v;
-  }
   // Centroid columns past the code words (d < KL with < 16 fields per word):
   // zero once, no tile writes them.
   for (int e = tid; e < TKR * KS; e += TKWARPS * 32) sA[e] = __float2half_rn(0.f);
-  for (int e = tid; e < QB * 2; e += TKWARPS * 32) sQ[e] = (q0 + e / 2 < a.nq) ? a.qsc[q0 * 2 + e] : 0.f;
-  for (int e = tid; e < TKWARPS * QH * a.K; e += TKWARPS * 32) {
-    lv[e] = -INFINITY;
-    li[e] = INT_MAX;
-  }
-  __syncthreads();
 
   const uint32_t sA_s = (uint32_t)__cvta_generic_to_shared(sA);
   const uint32_t sB_s = (uint32_t)__cvta_generic_to_shared(sB);
@@ -182,13 +172,50 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   const uint32_t b_row = sB_s + (uint32_t)((QH * qg + 8 * (ti >> 1) + tr) * KS + 8 * (ti & 1)) * 2;
   float* mylv = lv + warp * QH * a.K;
   int* myli = li + warp * QH * a.K;
-  // Current worst entry of this thread's SL queries (NTW n-tiles x 2 columns).
-  float wv[SL];
+
+  // Persistent CTAs: item = (query block, database chunk).
+  const int64_t nitems = a.qblocks * a.chunks;
+  for (int64_t item = blockIdx.x; item < nitems; item += gridDim.x) {
+  const int64_t q0 = (item / a.chunks) * QB;
+  const int64_t chunk_id = item % a.chunks;
+  const int64_t n0 = chunk_id * a.chunk;
+  const int64_t n1 = min(a.n, n0 + a.chunk);
+  __syncthreads();   // the previous item's readers of sB, sQ and the lists are done
+  for (int e = tid; e < QB * KP / 8; e += TKWARPS * 32) {
+    const int r = e / (KP / 8), c8 = e % (KP / 8);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (q0 + r < a.nq) v = reinterpret_cast<const uint4*>(a.qh + (q0 + r) * KP)[c8];
+    *reinterpret_cast<uint4*>(sB + (size_t)r * KS + 8 * c8) = v;
+  }
+  for (int e = tid; e < QB * 2; e += TKWARPS * 32) sQ[e] = (q0 + e / 2 < a.nq) ? a.qsc[q0 * 2 + e] : 0.f;
+  // Lists start at the query's bar: every final top-k entry is at least as
+  // good as the k-th best of any subset, so nothing below it can enter.
+  auto bar = [&](int64_t q, float& v, int& i) {
+    v = -INFINITY;
+    i = INT_MAX;
+    if (a.bar_v && q < a.nq) {
+      const int bi = a.bar_i[q * a.K + a.K - 1];
+      if (bi >= 0) {
+        v = a.bar_v[q * a.K + a.K - 1];
+        i = bi;
+      }
+    }
+  };
+  for (int e = tid; e < TKWARPS * QH * a.K; e += TKWARPS * 32) {
+    const int ql = (e / a.K) % QH, w = e / (QH * a.K);
+    bar(q0 + QH * (w >> 2) + ql, lv[e], li[e]);
+  }
+  __syncthreads();
+  // This thread's SL queries (NTW n-tiles x 2 columns): scales and the current
+  // worst entry of their lists.
+  float fe[SL], ff[SL], wv[SL];
   int wi[SL];
 #pragma unroll
   for (int s = 0; s < SL; ++s) {
-    wv[s] = -INFINITY;
-    wi[s] = INT_MAX;
+    const int ql = QH * qg + 8 * (s >> 1) + 2 * t + (s & 1);
+    fe[s] = sQ[2 * ql];
+    ff[s] = sQ[2 * ql + 1];
+    bar(q0 + ql, wv[s], wi[s]);
   }
 
   // Copy tile v0's codes, signs and norms (contiguous in memory) into staging
@@ -303,10 +330,9 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
     for (int nt = 0; nt < NTW; ++nt) {
 #pragma unroll
       for (int col = 0; col < 2; ++col) {
-        const int s = 2 * nt + col, ql = QH * qg + 8 * nt + 2 * t + col;
-        const float fe = sQ[2 * ql], ff = sQ[2 * ql + 1];
-        sc[s][0] = va ? fmaf(na * fe, acc[nt][col], ga * ff * acs[nt][col]) : -INFINITY;
-        sc[s][1] = vb ? fmaf(nb * fe, acc[nt][2 + col], gb * ff * acs[nt][2 + col]) : -INFINITY;
+        const int s = 2 * nt + col;
+        sc[s][0] = va ? fmaf(na * fe[s], acc[nt][col], ga * ff[s] * acs[nt][col]) : -INFINITY;
+        sc[s][1] = vb ? fmaf(nb * fe[s], acc[nt][2 + col], gb * ff[s] * acs[nt][2 + col]) : -INFINITY;
         if (va && better_sc(sc[s][0], (int)(v0 + ra), wv[s], wi[s])) mask |= 1u << (2 * s);
         if (vb && better_sc(sc[s][1], (int)(v0 + rb), wv[s], wi[s])) mask |= 1u << (2 * s + 1);
       }
@@ -365,7 +391,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 
   // ---- this warp's lists -> candidates of (query, chunk, row group) ------------------
-  const int list = (int)blockIdx.y * TKLISTS + rg;
+  const int list = (int)chunk_id * TKLISTS + rg;
   for (int e = lane; e < QH * a.K; e += 32) {
     const int ql = e / a.K, r = e % a.K;
     const int64_t q = q0 + QH * qg + ql;
@@ -374,6 +400,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       a.cand_v[o] = mylv[ql * a.K + r];
       a.cand_i[o] = myli[ql * a.K + r];
     }
+  }
   }
 }
 
@@ -387,14 +414,17 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   // 128 queries per CTA (more products per dequantized tile) when it fits.
   p.qb = topk_mma_smem(128, p.KL, p.KQ, c->wk, qw, k) <= (size_t)227 * 1024 ? 128 : 64;
   const int64_t qblocks = (nq + p.qb - 1) / p.qb;
-  int64_t chunks = (2 * (int64_t)c->sms + qblocks - 1) / (qblocks > 0 ? qblocks : 1);
+  // About sixteen (query block, chunk) items per SM for the persistent grid.
+  int64_t chunks = (16 * (int64_t)c->sms + qblocks - 1) / (qblocks > 0 ? qblocks : 1);
   const int64_t max_chunks = (n + 8 * TKR - 1) / (8 * TKR);   // at least eight tiles per chunk
   if (chunks > max_chunks) chunks = max_chunks;
   if (chunks < 1) chunks = 1;
   if (chunks > 65535) chunks = 65535;
   p.chunks = chunks;
   p.chunk = ((n + chunks - 1) / chunks + TKR - 1) / TKR * TKR;
-  p.nlists = (int)(chunks * TKLISTS);
+  p.chunks = (n + p.chunk - 1) / p.chunk;   // no empty chunk after rounding
+  p.qblocks = qblocks;
+  p.nlists = (int)(p.chunks * TKLISTS);
   p.qh_bytes = (size_t)nq * (p.KL + p.KQ) * sizeof(__half);
   p.qsc_bytes = (size_t)nq * 2 * sizeof(float);
   p.cand_bytes = (size_t)nq * p.nlists * k * (sizeof(float) + sizeof(int));
@@ -402,14 +432,29 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   return p;
 }
 
-cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const float* qr, const float* qs,
-                            int64_t nq, const uint32_t* codes, const uint32_t* qjl, const float* norm,
-                            const float* rnorm, int64_t n, int k, void* qh, float* qsc, float* cand_v,
-                            int* cand_i, cudaStream_t s) {
+TopkPlan topk_mma_sample_plan(const TopkPlan& full, int64_t n_sample, int sms) {
+  TopkPlan p = full;
+  int64_t chunks = (sms + p.qblocks - 1) / p.qblocks;   // about one item per SM
+  const int64_t max_chunks = (n_sample + 8 * TKR - 1) / (8 * TKR);
+  if (chunks > max_chunks) chunks = max_chunks;
+  if (chunks < 1) chunks = 1;
+  p.chunk = ((n_sample + chunks - 1) / chunks + TKR - 1) / TKR * TKR;
+  p.chunks = (n_sample + p.chunk - 1) / p.chunk;
+  p.nlists = (int)(p.chunks * TKLISTS);
+  return p;
+}
+
+cudaError_t launch_topk_qprep(const tq_ctx* c, const TopkPlan& p, const float* qr, const float* qs,
+                              int64_t nq, void* qh, float* qsc, cudaStream_t s) {
   k_topk_qprep<<<(unsigned)((nq + 3) / 4), 128, 0, s>>>(qr, qs, nq, c->d, c->dpad, c->qjl_m, p.KL, p.KQ,
                                                           static_cast<__half*>(qh), qsc);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, const float* qsc, int64_t nq,
+                            const uint32_t* codes, const uint32_t* qjl, const float* norm,
+                            const float* rnorm, int64_t n, int k, const float* bar_v, const int* bar_i,
+                            float* cand_v, int* cand_i, cudaStream_t s) {
   TopkMmaArgs a{};
   a.qh = static_cast<const __half*>(qh);
   a.qsc = qsc;
@@ -433,7 +478,12 @@ cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const float* qr,
   a.nlists = p.nlists;
   a.cand_v = cand_v;
   a.cand_i = cand_i;
-  dim3 grid((unsigned)((nq + p.qb - 1) / p.qb), (unsigned)p.chunks);
+  a.chunks = p.chunks;
+  a.qblocks = p.qblocks;
+  a.bar_v = bar_v;
+  a.bar_i = bar_i;
+  const int64_t items = p.qblocks * p.chunks;
+  const unsigned grid = (unsigned)(items < c->sms ? items : c->sms);   // one CTA per SM
   const bool wide = p.qb == 128;
   switch (c->bk_lm * 2 + (wide ? 1 : 0)) {
     case 2: k_topk_mma<1, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;

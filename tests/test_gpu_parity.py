@@ -325,6 +325,36 @@ def test_topk_code_widths_and_k(cuda, d, bk, m, k):
     _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), k)
 
 
+def test_topk_sample_bar_pass(cuda):
+    """A database large enough for the two-pass scorer (the k-th best of a
+    leading sample bars every list): exact duplicates inside the sample (equal
+    scores, broken by index), a query whose best match sits past the sample,
+    and k larger than the number of duplicates."""
+    n, d = 150_000, 64
+    c = _ctx(d, 2, 3, 64, seed=17)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(n, d, seed=41)
+    Q = tq_inputs.mixture(64, d, seed=42, means_seed=41)
+    # queries 0 and 1 point away from every mixture component, so their own
+    # copies are their best matches by a wide margin
+    Q[0:2] = tq_inputs.iid((2, d), seed=43)
+    Q[0:2] /= torch.linalg.vector_norm(Q[0:2], dim=1, keepdim=True)
+    X[0:5] = Q[0]
+    X[n - 7] = Q[1]
+    X[n - 3] = Q[1]
+    db = c.quantize(X.to(cuda), tq.TQ_KEY)
+    idx, score = c.topk(Q.to(cuda), db, 16)
+    torch.cuda.synchronize()
+    g = _flat(db, n)
+    idx, score = idx.cpu().numpy(), score.cpu().numpy()
+    _check_topk(tab, Q.double().numpy(), g, idx, score, 16)
+    assert idx[0, :5].tolist() == [0, 1, 2, 3, 4]
+    assert idx[1, :2].tolist() == [n - 7, n - 3]
+    assert np.all(np.diff(score, axis=1) <= 0)
+    for r in range(idx.shape[0]):
+        assert len(set(idx[r].tolist())) == 16
+
+
 def test_topk_vector_search_full(cuda):
     """1e6 unit-norm d=200 mixture vectors, 1e4 queries, 3-bit + QJL, top-10;
     the oracle checks the first 32 queries on the same codes."""
