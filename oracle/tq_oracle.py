@@ -46,6 +46,11 @@ Where the pages leave a step open, the reading taken is named R<k> below:
       them by `scale` (1/sqrt(d) by default).
   R12 Values are MSE-stage only; key dequantization includes the QJL
       back-projection, so logits(q, codes) = <q, dequantize(codes)>.
+  R13 "Norm correction" (the _nc variants named in [VLLM] A3) is not
+      defined on the pages.  Reading: the stored norm becomes n / |c[idx]|,
+      so the dequantized vector n Pi^T c[idx] / |c[idx]| keeps the input's
+      norm exactly.  It applies to MSE-only vectors: values, and keys without
+      the QJL stage (the variants name no QJL bit).
   R14 A zero vector has n = 0, u = 0, every index L/2, gamma = 0.
 """
 from __future__ import annotations
@@ -212,15 +217,21 @@ class Tables:
     S: np.ndarray | None
     cb_k: Codebook
     cb_v: Codebook
+    nc_k: bool = False     # R13 norm correction of keys
+    nc_v: bool = False     # R13 norm correction of values
 
 
-def make_tables(d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int) -> Tables:
-    """bits_k counts the QJL bit when qjl_m > 0 (R3)."""
+def make_tables(d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int,
+                nc_k: bool = False, nc_v: bool = False) -> Tables:
+    """bits_k counts the QJL bit when qjl_m > 0 (R3).  nc_k / nc_v turn on
+    the R13 norm correction (keys only without QJL)."""
+    if nc_k and qjl_m > 0:
+        raise ValueError("key norm correction applies to MSE-only keys (qjl_m = 0)")
     bits_k_lm = bits_k - 1 if qjl_m > 0 else bits_k
     Pi = rotation(d, seed)
     S = qjl_matrix(qjl_m, d, seed) if qjl_m > 0 else None
     return Tables(d, bits_k_lm, bits_v, qjl_m, seed, Pi, S,
-                  lloyd_max(d, bits_k_lm), lloyd_max(d, bits_v))
+                  lloyd_max(d, bits_k_lm), lloyd_max(d, bits_v), nc_k, nc_v)
 
 
 # ----------------------------------------------------------------------------
@@ -327,11 +338,20 @@ def quantize(x: np.ndarray, tab: Tables, which: str) -> Quantized:
     u = np.where((n > 0.0)[:, None], x / safe[:, None], 0.0)
     y = u @ tab.Pi.T
     idx = lloyd_max_index(y, cb)
+    nc = tab.nc_k if which == "k" else tab.nc_v
+    stored = corrected_norm(n, idx, cb) if nc else n
     q = Quantized(idx=idx, codes=pack_codes(idx, cb.bits),
-                  norm=n.astype(np.float32), y=y)
+                  norm=stored.astype(np.float32), y=y)
     if which == "k" and tab.qjl_m > 0:
         sketch_from_indices(q, tab)
     return q
+
+
+def corrected_norm(n: np.ndarray, idx: np.ndarray, cb: Codebook) -> np.ndarray:
+    """R13: n / |c[idx]| (fp64), the norm stored under norm correction.  The
+    codebook has no zero centroid, so |c[idx]| > 0."""
+    chat = cb.centroids[idx]
+    return np.asarray(n, dtype=np.float64) / np.sqrt(np.sum(chat * chat, axis=-1))
 
 
 def sketch_from_indices(q: Quantized, tab: Tables, idx: np.ndarray | None = None) -> None:

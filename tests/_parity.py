@@ -46,7 +46,8 @@ def packed_np(p):
 
 
 def oracle_tables(ctx):
-    return o.make_tables(ctx.d, ctx.bits_k, ctx.bits_v, ctx.qjl_m, ctx.seed)
+    return o.make_tables(ctx.d, ctx.bits_k, ctx.bits_v, ctx.qjl_m, ctx.seed,
+                         nc_k=getattr(ctx, "nc_k", False), nc_v=getattr(ctx, "nc_v", False))
 
 
 def check_quantized(tab, which, x, gpu, report=None):
@@ -67,7 +68,10 @@ def check_quantized(tab, which, x, gpu, report=None):
     assert n_exc <= MAX_EXCUSED_FRAC * mism.size, f"{n_exc} excused indices"
     gnorm = gpu["norm"].reshape(n).astype(np.float64)
     onorm = np.sqrt(np.sum(x * x, axis=1))
-    assert np.all(np.abs(gnorm - onorm) <= NORM_RTOL * onorm + 1e-30), "norm"
+    # R13: under norm correction the stored scalar is n / |c[idx]|, taken on
+    # the CUDA path's own indices (an excused index changes |c[idx]|)
+    want = o.corrected_norm(onorm, gidx, cb) if (tab.nc_k if which == "k" else tab.nc_v) else onorm
+    assert np.all(np.abs(gnorm - want) <= NORM_RTOL * want + 1e-30), "norm"
     stats = {"indices": int(mism.size), "excused": n_exc, "band": int(band.sum())}
     if which == "k" and tab.qjl_m > 0:
         o.sketch_from_indices(q, tab, idx=gidx)

@@ -133,6 +133,59 @@ def test_empirical_mse_within_two_percent(bits):
     assert abs(emp / ref - 1) < 0.02
 
 
+# --- R13: norm correction ------------------------------------------------------
+@pytest.mark.parametrize("d", [64, 128])
+def test_norm_correction_one_bit_closed_form(d):
+    """At 1 bit every rotated coordinate maps to +-c1 with c1 = E|T| (closed
+    form), so |c[idx]| = sqrt(d) c1 for every vector and the stored norm is
+    n / (sqrt(d) c1)."""
+    c1 = math.exp(gammaln(d / 2) - gammaln((d + 1) / 2)) / math.sqrt(math.pi)
+    tab = o.make_tables(d, 1, 1, 0, 5, nc_k=True, nc_v=True)
+    x = np.random.default_rng(3).standard_normal((500, d)) * 2.5
+    n = np.linalg.norm(x, axis=1)
+    for which in ("k", "v"):
+        q = o.quantize(x, tab, which)
+        want = n / (math.sqrt(d) * c1)
+        assert np.all(np.abs(q.norm - want) <= 1e-7 * want)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_norm_correction_keeps_the_norm(bits):
+    """Under norm correction the dequantized vector has the input's norm
+    (up to the fp32 rounding of the stored scalar); the codes are unchanged."""
+    d = 128
+    x = np.random.default_rng(bits).standard_normal((2000, d)) * 0.3
+    x[7] = 0.0
+    n = np.linalg.norm(x, axis=1)
+    tab = o.make_tables(d, bits, bits, 0, 9, nc_k=True, nc_v=True)
+    plain = o.make_tables(d, bits, bits, 0, 9)
+    for which in ("k", "v"):
+        q = o.quantize(x, tab, which)
+        xh = o.dequantize(tab, which, q.codes, q.norm)
+        assert np.all(np.abs(np.linalg.norm(xh, axis=1) - n) <= 2e-7 * n)
+        assert q.norm[7] == 0.0 and np.all(xh[7] == 0.0)
+        qp = o.quantize(x, plain, which)
+        assert np.array_equal(qp.codes, q.codes)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_norm_correction_mean_square_is_one_minus_distortion(bits):
+    """Lloyd-Max centroids are cell means, so E|c[idx]|^2 = E|y|^2 - E|y - c|^2
+    = 1 - D_b: the mean of (n / stored)^2 over uniform directions must match
+    the codebook's distortion."""
+    d = 128
+    tab = o.make_tables(d, bits, bits, 0, 13, nc_v=True)
+    x = np.random.default_rng(40 + bits).standard_normal((40_000, d))
+    q = o.quantize(x, tab, "v")
+    ratio2 = (np.linalg.norm(x, axis=1) / q.norm.astype(np.float64)) ** 2
+    assert abs(ratio2.mean() - (1.0 - o.distortion(d, tab.cb_v))) < 3e-3
+
+
+def test_norm_correction_needs_mse_only_keys():
+    with pytest.raises(ValueError):
+        o.make_tables(64, 3, 4, 64, 1, nc_k=True)
+
+
 def test_printed_three_bit_cosine():
     want = float(_golden_lines("page_claims.txt")[0][1])
     d = 128
