@@ -50,6 +50,8 @@ WORKLOADS = {
     "70b-decode-k4v4": dict(B=4, Hq=64, Hkv=8, d=128, T=131072, bits_k=4, bits_v=4, m=128),
 }
 QUANT_SWEEP = dict(tokens=131072, heads=8, d=128, bits=(2, 3, 4))
+# The norm-corrected MSE-only cache formats, timed on the Llama-3-8B decode shape.
+NC_VARIANTS = ("k3v4_nc", "4bit_nc", "3bit_nc")
 
 
 def peaks():
@@ -328,6 +330,52 @@ def vector_search(tq, tq_inputs, torch, dev, sm_mhz_max, steps=3, warmup=1):
                          "frac": flop / t / 1e12 / peak, "peak_source": peak_src}}
 
 
+def variant_decode(tq, tq_inputs, torch, dev, hbm_peak, shape, steps=20, warmup=3):
+    """tq_attn_decode for each norm-corrected format on one decode shape."""
+    B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
+    out = {}
+    for name in NC_VARIANTS:
+        ctx = tq.Context.variant(name, d, 0)
+        kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
+        vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+        for b in range(B):
+            K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
+            V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+            ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
+            ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+            del K, V
+        q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
+        lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+        o = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+        ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
+        for _ in range(warmup):
+            ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        kb, vb = ctx.key_layout["bytes_per_vector"], ctx.value_layout["bytes_per_vector"]
+        alg = B * Hkv * T * (kb + vb) + B * Hq * d * 2 + B * Hq * d * 4
+        bits_k, bits_v, _, _ = tq.VARIANTS[name]
+        out[name] = {"kv_format": f"keys {bits_k} Lloyd-Max bits, values {bits_v} bits, MSE only, "
+                                  f"norm-corrected; {kb + vb} B per token-head",
+                     "attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
+                     "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak}
+        del g, kc, vc, ws
+        ctx.close()
+    torch.cuda.empty_cache()
+    return out
+
+
 def small_case(tq, tq_inputs, torch, dev, reps=50):
     """Latency of the smallest workload: quantize 1024 K and 1024 V (fp32,
     d = 128, k3v4), then attention of 8 query heads over them (one kv head)."""
@@ -519,12 +567,13 @@ def run_gpu(args, w):
     quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
     torch.cuda.nvtx.range_pop()
     clocks = sampler.stop()
-    vsearch = small = None
+    vsearch = small = variants = None
     if not args.skip_extra:
         torch.cuda.nvtx.range_push("tq:vector_search")
         vsearch = vector_search(tq, tq_inputs, torch, dev, clocks.get("sm_max_mhz") or 1965.0)
         torch.cuda.nvtx.range_pop()
         small = small_case(tq, tq_inputs, torch, dev)
+        variants = variant_decode(tq, tq_inputs, torch, dev, hbm_peak, WORKLOADS["llama3-8b-decode"])
 
     tm = torch.tensor([t_ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -562,6 +611,7 @@ def run_gpu(args, w):
         if vsearch is not None:
             line["vector_search"] = vsearch
             line["small_case"] = small
+            line["norm_corrected_decode"] = variants
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

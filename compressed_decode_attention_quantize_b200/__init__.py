@@ -20,6 +20,7 @@ _LIB_PATH = _PKG / "libtq.so"
 
 TQ_OK, TQ_ERR_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(5)
 TQ_KEY, TQ_VALUE = 0, 1
+TQ_NC_KEYS, TQ_NC_VALUES = 1, 2
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 _DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
@@ -49,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "tq_version": (ctypes.c_char_p, []),
         "tq_device_fault": (I, [ctypes.POINTER(ctypes.c_int)]),
         "tq_init": (P, [I, I, I, I, U64]),
+        "tq_init_ex": (P, [I, I, I, I, U64, I]),
         "tq_destroy": (None, [P]),
         "tq_layout": (I, [P, I, ctypes.POINTER(tq_layout_t)]),
         "tq_host_tables": (I, [I, I, I, I, U64, P, P, P, P, P, P]),
@@ -77,7 +79,7 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_destroy", "tq_layout", "tq_host_tables",
+EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_init_ex", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
             "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
             "tq_attn_static_scratch_bytes", "tq_decode_step", "tq_quantize_append_paged",
@@ -108,6 +110,13 @@ def _stream(stream=None):
 # ---------------------------------------------------------------------------
 def tq_init(d, bits_k, bits_v, qjl_m, seed):
     p = _lib.tq_init(d, bits_k, bits_v, qjl_m, seed)
+    if not p:
+        raise TQError(-1, _lib.tq_last_error().decode())
+    return p
+
+
+def tq_init_ex(d, bits_k, bits_v, qjl_m, seed, flags):
+    p = _lib.tq_init_ex(d, bits_k, bits_v, qjl_m, seed, flags)
     if not p:
         raise TQError(-1, _lib.tq_last_error().decode())
     return p
@@ -149,15 +158,38 @@ def tq_host_tables(d, bits_k, bits_v, qjl_m, seed):
     return {"Pi": pi, "S": S[:qjl_m], "ck": ck, "bk": bk, "cv": cv, "bv": bv}
 
 
+# Named cache formats: name -> (bits_k, bits_v, key QJL stage with m = d,
+# norm correction of keys and values).  k3v4 / k4v4 spend one key bit on QJL;
+# the _nc formats of the vLLM study are MSE-only with norm correction.
+VARIANTS = {
+    "k3v4": (3, 4, True, False),
+    "k4v4": (4, 4, True, False),
+    "k3v4_nc": (3, 4, False, True),
+    "4bit_nc": (4, 4, False, True),
+    "3bit_nc": (3, 3, False, True),
+}
+
+
 class Context:
     """A libtq context: tables for one (d, bits_k, bits_v, qjl_m, seed) on the
     current CUDA device."""
 
-    def __init__(self, d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int = 0):
+    def __init__(self, d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int = 0,
+                 nc_k: bool = False, nc_v: bool = False):
         self.d, self.bits_k, self.bits_v, self.qjl_m, self.seed = d, bits_k, bits_v, qjl_m, seed
-        self.ptr = tq_init(d, bits_k, bits_v, qjl_m, seed)
+        self.nc_k, self.nc_v = bool(nc_k), bool(nc_v)
+        flags = (TQ_NC_KEYS if nc_k else 0) | (TQ_NC_VALUES if nc_v else 0)
+        self.ptr = tq_init_ex(d, bits_k, bits_v, qjl_m, seed, flags)
         self.key_layout = tq_layout(self.ptr, TQ_KEY)
         self.value_layout = tq_layout(self.ptr, TQ_VALUE)
+
+    @classmethod
+    def variant(cls, name: str, d: int, seed: int = 0) -> "Context":
+        """A context for one of the named cache formats in VARIANTS."""
+        if name not in VARIANTS:
+            raise ValueError(f"unknown variant {name!r}; known: {', '.join(VARIANTS)}")
+        bits_k, bits_v, qjl, nc = VARIANTS[name]
+        return cls(d, bits_k, bits_v, d if qjl else 0, seed, nc_k=nc, nc_v=nc)
 
     def close(self):
         if getattr(self, "ptr", None):

@@ -112,13 +112,27 @@ int tq_host_tables(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, doub
 }
 
 tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
+  return tq_init_ex(d, bits_k, bits_v, qjl_m, seed, 0);
+}
+
+tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int flags) {
   int code = TQ_OK;
   if (!valid_dims(d, bits_k, bits_v, qjl_m, &code)) return nullptr;
+  if (flags & ~(TQ_NC_KEYS | TQ_NC_VALUES)) {
+    fail(TQ_ERR_ARG, "tq_init_ex: unknown flag bits 0x%x", flags);
+    return nullptr;
+  }
+  if ((flags & TQ_NC_KEYS) && qjl_m > 0) {
+    fail(TQ_ERR_UNSUPPORTED, "tq_init_ex: key norm correction needs MSE-only keys (qjl_m = 0)");
+    return nullptr;
+  }
   tq_ctx* c = new (std::nothrow) tq_ctx();
   if (!c) {
     fail(TQ_ERR_ARG, "host allocation failed");
     return nullptr;
   }
+  c->nc_k = (flags & TQ_NC_KEYS) != 0;
+  c->nc_v = (flags & TQ_NC_VALUES) != 0;
   c->d = d;
   c->J = (d + 31) / 32;
   c->dpad = 32 * c->J;
@@ -342,12 +356,13 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.max_blocks = pg.max_blocks;
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
+  a.nc = (key ? c->nc_k : c->nc_v) ? 1 : 0;
   if (n <= tqk::kSmallQuantize) {
     cudaError_t e = tqk::launch_quantize_small(c, a, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;
   }
-  const bool tc = !pg.table && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+  const bool tc = !pg.table && !a.nc && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
     tqk::QuantTcArgs t{};
@@ -630,6 +645,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
     a.bits = key ? c->bk_lm : c->bits_v;
     a.nbnd = (1 << a.bits) - 1;
     a.m = key ? c->qjl_m : 0;
+    a.nc = (key ? c->nc_k : c->nc_v) ? 1 : 0;
     a.words = key ? c->wk : c->wv;
     a.PiT = c->PiT;
     a.ST = c->ST;

@@ -38,6 +38,8 @@ struct tq_ctx {
   bool tc_ok = false;
   void* tc_block = nullptr;
   int sms = 148;
+  bool nc_k = false;   // norm correction of keys (MSE-only keys)
+  bool nc_v = false;   // norm correction of values
   const void* tc_pih = nullptr;   // 2^8 Pi, fp16 head
   const void* tc_pil = nullptr;   // 2^8 Pi - head, fp16
   const void* tc_s = nullptr;     // S, fp16 (exact)
@@ -84,6 +86,8 @@ struct QuantArgs {
   const int32_t* block_table;
   int max_blocks, block_size;
   int64_t num_blocks;
+  // Norm correction (MSE-only vectors): store n / |c[idx]| instead of n.
+  int nc;
 };
 
 struct AttnArgs {

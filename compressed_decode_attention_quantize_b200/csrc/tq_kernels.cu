@@ -217,6 +217,20 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
         idx[i][v] = (unsigned char)lm_index(y, s_bnd, a.nbnd);
       }
     }
+    // Norm correction: the stored scalar is n / |c[idx]| (no QJL stage then,
+    // so nrm is not needed afterwards).
+    if (a.nc) {
+#pragma unroll
+      for (int v = 0; v < QV; ++v) {
+        float cc = 0.f;
+#pragma unroll
+        for (int i = 0; i < J; ++i) {
+          const float cj = (lane + 32 * i < a.d) ? s_cen[idx[i][v]] : 0.f;
+          cc = fmaf(cj, cj, cc);
+        }
+        nrm[v] = nrm[v] / sqrtf(warp_sum(cc));
+      }
+    }
     // Field packing: lane owns coordinates lane + 32 i; a group of 32/b lanes
     // fills one word (b = 3: 2-bit stream of low bits, then 1-bit stream).
 #pragma unroll
@@ -350,12 +364,33 @@ __device__ __forceinline__ void quantize_small_body(const QuantArgs& a, int dpad
   float acc[QS];
   mv_rows<QS>(a.PiT, a.d, dpad, sh, Ms, acc);
   float r[QS];
+  int ids[QS];
   const int i32 = j >> 5;
 #pragma unroll
   for (int u = 0; u < QS; ++u) {
     const float y = (nrm[u] > 0.f && j < a.d) ? acc[u] / nrm[u] : 0.f;
-    const int idx = lm_index(y, s_bnd, a.nbnd);
-    r[u] = (j < a.d) ? y - s_cen[idx] : 0.f;
+    ids[u] = lm_index(y, s_bnd, a.nbnd);
+    r[u] = (j < a.d) ? y - s_cen[ids[u]] : 0.f;
+  }
+  if (a.nc) {   // uniform; norm correction: store n / |c[idx]| (MSE-only, no QJL stage follows)
+    __syncthreads();   // every thread has read the norm sums out of red
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      const float cj = (j < a.d) ? s_cen[ids[u]] : 0.f;
+      const float cc = warp_sum(cj * cj);
+      if (lane == 0) red[u][warp] = cc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      float t = 0.f;
+      for (int w = 0; w < nwarp; ++w) t += red[u][w];
+      nrm[u] = nrm[u] / sqrtf(t);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    const int idx = ids[u];
     if (u >= nv) continue;   // uniform over the block
     const int64_t rec = out_record(a, v0 + u);
     if (rec < 0) continue;   // uniform too (one sequence per vector)

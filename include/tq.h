@@ -27,7 +27,7 @@
  *   synchronise, nor fall back to the CPU.  Scratch memory comes from the
  *   caller's `workspace` (device, at least the size the *_workspace_bytes
  *   query returns, 256-byte aligned).
- * - Every call but tq_init/tq_destroy/tq_last_error returns a status:
+ * - Every call but tq_init/tq_init_ex/tq_destroy/tq_last_error returns a status:
  *   TQ_OK, TQ_ERR_ARG (bad pointer, size, alignment or enum),
  *   TQ_ERR_UNSUPPORTED (valid but not implemented: dimension, bit width),
  *   TQ_ERR_CUDA (a CUDA launch or runtime error), TQ_ERR_WORKSPACE (workspace
@@ -47,7 +47,8 @@
  *                      bits are 0.
  *   qjl    uint32[ceil(m/32)]  keys only: bit i%32 of word i/32 is 1 when
  *                      (S r)_i >= 0.
- *   norm   float       |x| (fp32).
+ *   norm   float       |x| (fp32); |x| / |c[idx]| under norm correction
+ *                      (see tq_init_ex).
  *   rnorm  float       keys with QJL only: gamma = |x| * |r|, r the residual
  *                      of the rotated unit vector.
  * Arrays of vectors are these records laid out as separate dense arrays
@@ -118,6 +119,27 @@ int tq_device_fault(int* code);
  * tq_last_error).
  */
 tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed);
+
+/* Flags of tq_init_ex. */
+enum tq_flags { TQ_NC_KEYS = 1, TQ_NC_VALUES = 2 };
+
+/*
+ * tq_init_ex - tq_init with options.  The norm-corrected variants named in
+ * "A First Comprehensive Study of TurboQuant: Accuracy and Performance",
+ * section A3 (k3v4_nc, 3bit_nc, 4bit_nc) leave "norm correction" undefined;
+ * this library reads it as storing n / |c[idx]| in place of n, where c[idx]
+ * is the vector of the Lloyd-Max centroids a vector's indices select in the
+ * rotated domain, so the dequantized vector n Pi^T c[idx] / |c[idx]| keeps
+ * the input's norm exactly.  The packed layout is unchanged; only the value
+ * stored in `norm` differs, so dequantize, logits, attention and top-k read
+ * it as before.
+ *   flags  TQ_NC_KEYS: norm correction of keys, which must then be MSE-only
+ *          (qjl_m = 0, else NULL with TQ_ERR_UNSUPPORTED);
+ *          TQ_NC_VALUES: norm correction of values.
+ *          Other bits: NULL with TQ_ERR_ARG.
+ * Otherwise as tq_init.
+ */
+tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int flags);
 
 /* Frees the context's device tables.  NULL is ignored. */
 void tq_destroy(tq_ctx* ctx);

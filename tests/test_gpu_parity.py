@@ -506,6 +506,57 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
                       lens.cpu().numpy(), Hkv, outA.cpu().numpy())
 
 
+# --- norm-corrected cache formats -------------------------------------------------
+@pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("4bit_nc", 16), ("3bit_nc", 8)])
+def test_norm_corrected_variants(cuda, name, Hq):
+    """The MSE-only _nc formats: quantize through the bulk and the small-batch
+    kernels (stored norm n / |c[idx]|), logits, ragged decode attention, and
+    the fused decode step (equal to append + decode), all against the oracle
+    with the same reading of norm correction."""
+    c = tq.Context.variant(name, 128, seed=8)
+    assert c.nc_k and c.nc_v and c.qjl_m == 0
+    tab = P.oracle_tables(c)
+    B, Hkv, T, d = 4, 2, 1100, 128
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=61)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=62)
+    kc, vc = _cache(c, K, V, cuda)
+    n = B * Hkv * T
+    P.check_quantized(tab, "k", P.to_np(K.reshape(n, d)), _flat(kc, n))
+    P.check_quantized(tab, "v", P.to_np(V.reshape(n, d)), _flat(vc, n))
+    small = K[0, 0, :300].contiguous()
+    ks = c.quantize(small.to(cuda), tq.TQ_KEY)
+    P.check_quantized(tab, "k", P.to_np(small), _flat(ks, 300))
+    Q = tq_inputs.iid((B, Hq, d), seed=63, dtype=torch.bfloat16)
+    lg = c.logits(Q[0].to(cuda), ks)
+    torch.cuda.synchronize()
+    P.check_logits(tab, Q[0].double().numpy(), _flat(ks, 300), lg.cpu().double().numpy())
+    lens = torch.tensor([0, 1, 517, T], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+    # fused step vs append + decode on copies of the same cache
+    kB = {k: (None if v is None else v.clone()) for k, v in kc.items()}
+    vB = {k: (None if v is None else v.clone()) for k, v in vc.items()}
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=64)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=65)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([0, 600, T - 1, -1], dtype=torch.int32, device=cuda)
+    q = Q.to(cuda)
+    outA = c.decode_step(q, kn, vn, kc, vc, pos)
+    c.quantize_append(kn, tq.TQ_KEY, kB, pos)
+    c.quantize_append(vn, tq.TQ_VALUE, vB, pos)
+    lens2 = torch.clamp(pos.long() + 1, 0, T).to(torch.int32)
+    outB = c.attn_decode(q, kB, vB, lens2)
+    torch.cuda.synchronize()
+    for a_, b_ in ((kc, kB), (vc, vB)):
+        for k in a_:
+            if a_[k] is not None:
+                assert torch.equal(a_[k], b_[k]), k
+    assert torch.equal(outA, outB)
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens2.cpu().numpy(), Hkv,
+                      outA.cpu().numpy())
+
+
 # --- paged caches ---------------------------------------------------------------
 def _to_paged(cache, B, Hkv, max_T, bs, perm):
     """Scatter a contiguous [B, Hkv, max_T, ...] cache into blocks

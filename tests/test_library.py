@@ -63,3 +63,15 @@ def test_init_without_device_reports_cuda_error():
     with pytest.raises(tq.TQError) as e:
         tq.tq_init(128, 3, 4, 128, 0)
     assert "cuda" in str(e.value).lower()
+
+
+def test_norm_correction_flags_validated_before_any_device_call():
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_init_ex(128, 3, 4, 128, 0, tq.TQ_NC_KEYS)   # keys with QJL
+    assert "norm correction" in str(e.value)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_init_ex(128, 3, 4, 0, 0, 4)
+    assert "flag" in str(e.value)
+    with pytest.raises(ValueError):
+        tq.Context.variant("k8v4", 128)
+    assert set(tq.VARIANTS) == {"k3v4", "k4v4", "k3v4_nc", "4bit_nc", "3bit_nc"}
