@@ -78,7 +78,7 @@ def kernel_source_hash() -> str:
     when these change)."""
     h = hashlib.sha256()
     csrc = ROOT / "compressed_decode_attention_quantize_b200" / "csrc"
-    for name in ("tq_attn_mma.cu", "tq_attn_k4.cu", "tq_attn_common.cuh", "tq_internal.h"):
+    for name in ("tq_attn_mma.cu", "tq_attn_lut.cu", "tq_attn_common.cuh", "tq_internal.h"):
         h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 

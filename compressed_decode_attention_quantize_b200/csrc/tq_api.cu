@@ -554,11 +554,11 @@ static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, 
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
   const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
-  const bool k4 = !mma && tqk::attn_k4_supported(c, a) && max_T > 0;
-  if (pg.table && !(mma || k4))
+  const bool lut = !mma && tqk::attn_lut_supported(c, a) && max_T > 0;
+  if (pg.table && !(mma || lut))
     return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode (d = 128, QJL m = 128, "
-                "4-bit values, 2-bit keys with group 1/2/4/8 or 3-bit keys with group 8)", name);
-  if (mma || k4) {
+                "4-bit values; 2-bit keys + QJL with group 1/2/4/8, 3-bit keys + QJL or MSE-only 3/4-bit keys with group 4/8)", name);
+  if (mma || lut) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
@@ -566,7 +566,7 @@ static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, 
   cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s);
   if (e != cudaSuccess) return cuda_fail(e, name);
   e = mma ? tqk::launch_attn_mma(c, a, out, s)
-          : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
+          : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s));
   if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
 }
@@ -697,10 +697,10 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
   const bool mma = tqk::attn_mma_supported(c, a);
-  const bool k4 = !mma && tqk::attn_k4_supported(c, a);
-  if (pg.table && !(mma || k4))
+  const bool lut = !mma && tqk::attn_lut_supported(c, a);
+  if (pg.table && !(mma || lut))
     return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode", name);
-  if (mma || k4) {
+  if (mma || lut) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
@@ -723,7 +723,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
   cudaError_t e = tqk::launch_step_prep(c, sp, s);
   if (e != cudaSuccess) return cuda_fail(e, name);
   e = mma ? tqk::launch_attn_mma(c, a, out, s)
-          : (k4 ? tqk::launch_attn_k4(c, a, out, s) : tqk::launch_attn(c, a, out, s));
+          : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s));
   if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
 }

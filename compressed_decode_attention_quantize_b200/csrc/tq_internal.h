@@ -183,11 +183,12 @@ bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
 // Upper bound on the warps of a segment-path launch (sizes the partials).
 int64_t attn_seg_max_warps(const tq_ctx* c);
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
-// Tensor-core decode path for 3-bit Lloyd-Max keys (k4v4: d = 128, keys 3 + 1
-// QJL bit with m = 128, values 4 bits, group 8); needs AttnArgs::tiles.
-bool attn_k4_supported(const tq_ctx* c, const AttnArgs& a);
-cudaError_t launch_attn_k4(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
-cudaError_t configure_attn_k4();
+// Tensor-core decode path with table-dequantized keys (d = 128, values 4
+// bits, group 4 or 8): 3-bit Lloyd-Max keys + QJL with m = 128 (k4v4), or
+// MSE-only 3- or 4-bit keys (the norm-corrected formats); needs AttnArgs::tiles.
+bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a);
+cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+cudaError_t configure_attn_lut();
 // Top-k on the tensor cores: query blocks of 64 or 128 x database chunks.
 struct TopkPlan {
   int KL, KQ;            // padded centroid and sign widths

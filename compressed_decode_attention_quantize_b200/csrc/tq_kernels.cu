@@ -1183,7 +1183,7 @@ cudaError_t configure_kernels() {
   if ((e = cudaFuncSetAttribute(k_prerotate<8>, ms, small_smem))) return e;
   if ((e = cudaFuncSetAttribute(k_step_prep, ms, small_smem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
-  if ((e = configure_attn_k4()) != cudaSuccess) return e;
+  if ((e = configure_attn_lut()) != cudaSuccess) return e;
   if ((e = configure_topk_mma()) != cudaSuccess) return e;
   return configure_attn_mma();
 }

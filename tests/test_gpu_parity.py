@@ -165,7 +165,8 @@ def test_attention_single_head(cuda):
     (128, 16, 2, 3, 4, 128, 1100),  # tensor-core path, group 8
     (128, 8, 2, 3, 4, 128, 1002),   # max_T % 4 != 0: generic path
     (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: tensor-core path, group 8
-    (128, 8, 2, 4, 4, 128, 1000),   # 3-bit keys, group 4: generic path
+    (128, 8, 2, 4, 4, 128, 1000),   # 3-bit keys: tensor-core path, group 4
+    (128, 8, 2, 4, 4, 128, 998),    # 3-bit keys, max_T % 4 != 0: generic path
     (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000)])
 def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
     """Ragged lengths (0, 1, odd, chunk edges, full), GQA groups 1-8, d=64/128/200."""
@@ -471,6 +472,7 @@ def test_quantize_append_large_batch(cuda):
     (8, 2, 3, 300),     # tensor-core decode, group 4
     (16, 2, 3, 300),    # group 8
     (16, 2, 4, 300),    # 3-bit keys, group 8
+    (8, 2, 4, 300),     # 3-bit keys, group 4
     (8, 2, 3, 302),     # max_T % 4 != 0: generic decode
 ])
 def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
@@ -507,7 +509,8 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
 
 
 # --- norm-corrected cache formats -------------------------------------------------
-@pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("4bit_nc", 16), ("3bit_nc", 8)])
+@pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("k3v4_nc", 16), ("4bit_nc", 8), ("4bit_nc", 16),
+                                     ("3bit_nc", 8)])
 def test_norm_corrected_variants(cuda, name, Hq):
     """The MSE-only _nc formats: quantize through the bulk and the small-batch
     kernels (stored norm n / |c[idx]|), logits, ragged decode attention, and
@@ -576,12 +579,14 @@ def _to_paged(cache, B, Hkv, max_T, bs, perm):
     return out
 
 
-@pytest.mark.parametrize("Hq,Hkv,bk,bs", [(8, 2, 3, 32), (16, 2, 3, 16), (16, 2, 4, 48), (4, 4, 3, 16)])
-def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs):
+@pytest.mark.parametrize("Hq,Hkv,bk,bs,variant", [
+    (8, 2, 3, 32, None), (16, 2, 3, 16, None), (16, 2, 4, 48, None), (4, 4, 3, 16, None),
+    (8, 2, 4, 16, None), (8, 2, None, 32, "4bit_nc"), (16, 2, None, 16, "k3v4_nc")])
+def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs, variant):
     """The paged decode reads the same records through the block table, so it
     must reproduce the contiguous decode bit for bit (ragged lengths,
     partial last blocks, an empty sequence, blocks in shuffled order)."""
-    c = _ctx(128, bk, 4, 128, seed=6)
+    c = tq.Context.variant(variant, 128, seed=6) if variant else _ctx(128, bk, 4, 128, seed=6)
     B, d, max_T = 5, 128, 288
     K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=41).to(cuda)
     V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=42).to(cuda)
