@@ -1,7 +1,8 @@
 // Decode attention from packed codes whose keys are dequantized through a
 // table: 3-bit Lloyd-Max keys with the QJL bit (k4v4: m = 128), and the
-// MSE-only norm-corrected formats with 3- or 4-bit keys (k3v4_nc, 4bit_nc);
-// values 4 bits, d = 128, GQA group 4 or 8, on the tensor cores (sm_100a).
+// MSE-only norm-corrected formats with 3- or 4-bit keys (k3v4_nc, 4bit_nc,
+// 3bit_nc); values 4 bits (3 bits for 3bit_nc), d = 128, GQA group 4 or 8,
+// on the tensor cores (sm_100a).
 //
 // Same quantities as the 2-bit-key kernels ("What is TurboQuant?", "How
 // TurboQuant works", closing paragraph; "How to implement" part 1):
@@ -59,7 +60,17 @@ struct KeyFmt {
   static constexpr size_t LUT_BYTES = (size_t)ENT * COP * 8;
 };
 
-template <int KB, bool QJL>
+// Values: 4-bit fields (16 words per token, rows padded to VROW) or 3-bit
+// (2-bit stream of 8 words, then 4 top-bit words: 12-word rows, on which the
+// loads of value_tile3 meet distinct banks).
+template <int VB>
+struct ValFmt {
+  static constexpr int REC = VB == 4 ? 16 : 12;       // words per value record
+  static constexpr int ROW = VB == 4 ? VROW : 12;     // staged row (words)
+  static constexpr int LUTW = VB == 4 ? LUT_WORDS : 64 * 32;
+};
+
+template <int KB, bool QJL, int VB>
 struct StageL {
   uint32_t k2[MT][KeyFmt<KB>::K2W];   // 2-bit stream (3-bit keys) or the 4-bit fields
   uint32_t k1[MT][4];                 // top-bit stream (3-bit keys)
@@ -67,13 +78,63 @@ struct StageL {
   float kn[MT];
   float kr[MT];
   float vn[MT];
-  alignas(16) uint32_t v[MT][VROW];
+  alignas(16) uint32_t v[MT][ValFmt<VB>::ROW];
 };
 
-template <int KB, bool QJL>
+template <int KB, bool QJL, int VB>
 constexpr size_t smem_lut() {
-  return KeyFmt<KB>::LUT_BYTES + (size_t)LUT_WORDS * 4 + (size_t)MW * NSTK * sizeof(StageL<KB, QJL>) +
+  return KeyFmt<KB>::LUT_BYTES + (size_t)ValFmt<VB>::LUTW * 4 + (size_t)MW * NSTK * sizeof(StageL<KB, QJL, VB>) +
          (size_t)8 * 32 * QOPK * 4 + (QJL ? (size_t)8 * 32 * QOPQ * 4 : 0) + 8 * 16 + MW * 4 + 16 * 4;
+}
+
+// 3-bit value table: entry (idx, lane) = half2(cv[ia], cv[ib]) for the codes
+// ia, ib of two tokens at one coordinate, idx = lo2(a) | lo2(b) << 2 |
+// top(a) << 4 | top(b) << 5.
+__device__ __forceinline__ void build_value_lut3(uint32_t* lut, const float* cv, int tid, int nthreads) {
+  for (int e = tid; e < 64 * 32; e += nthreads) {
+    const int idx = e >> 5;
+    const int ia = (idx & 3) | (((idx >> 4) & 1) << 2), ib = ((idx >> 2) & 3) | (((idx >> 5) & 1) << 2);
+    lut[e] = pack_half2(cv[ia], cv[ib]);
+  }
+}
+
+// Bits 0..15 of x spread to the even bit positions.
+__device__ __forceinline__ uint32_t spread16(uint32_t x) {
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return (x | (x << 1)) & 0x55555555u;
+}
+
+// value_tile for 3-bit value codes: o[mt] += V^T P over one 16-token tile.
+// Thread (g, t) covers coordinates 16g .. 16g+15 (2-bit word g, top bits
+// 16 (g & 1) .. of word 8 + g/2) of tokens 2t, 2t+1 (k 2t, 2t+1) and 2t+8,
+// 2t+9; row g of MMA mt is coordinate 16g + mt, row g+8 is 16g + 8 + mt.
+__device__ __forceinline__ void value_tile3(float (&o)[8][4], const uint32_t (*v)[12], uint32_t pb0,
+                                            uint32_t pb1, uint32_t lut_lane, int g, int t) {
+  const int sh = 16 * (g & 1);
+  uint32_t ne[2], no[2], tt[2];
+#pragma unroll
+  for (int pr = 0; pr < 2; ++pr) {
+    const int ra = 2 * t + 8 * pr;
+    const uint32_t A = v[ra][g], B = v[ra + 1][g];
+    const uint32_t TA = (v[ra][8 + (g >> 1)] >> sh) & 0xFFFFu, TB = (v[ra + 1][8 + (g >> 1)] >> sh) & 0xFFFFu;
+    ne[pr] = (A & 0x33333333u) | ((B & 0x33333333u) << 2);   // nibble k: coordinate 2k
+    no[pr] = ((A >> 2) & 0x33333333u) | (B & 0xCCCCCCCCu);   // nibble k: coordinate 2k + 1
+    tt[pr] = spread16(TA) | (spread16(TB) << 1);             // bits 2j, 2j+1: top bits of a, b
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    uint32_t av[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int pr = r >> 1, j = mt + 8 * (r & 1);
+      const uint32_t nib = ((j & 1 ? no[pr] : ne[pr]) >> (4 * (j >> 1))) & 0xFu;
+      const uint32_t top = (tt[pr] >> (2 * j)) & 3u;
+      av[r] = lds32(((nib | (top << 4)) << 7) + lut_lane);
+    }
+    mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+  }
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
@@ -96,16 +157,17 @@ __device__ __forceinline__ uint32_t klut4_off(uint32_t w) {
   return __byte_perm(w, 0, 0x4440 + B) << 7;
 }
 
-template <bool PAGED, int KB, bool QJL, int G>
+template <bool PAGED, int KB, bool QJL, int G, int VB>
 __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
   static_assert(G == 4 || G == 8, "group 4 or 8");
   using KF = KeyFmt<KB>;
-  using Stage = StageL<KB, QJL>;
+  using VF = ValFmt<VB>;
+  using Stage = StageL<KB, QJL, VB>;
   constexpr int NJ = G / 4;   // head sets per thread: t (and 4 + t)
   extern __shared__ __align__(16) unsigned char smem[];
   uint2* klut = reinterpret_cast<uint2*>(smem);                                          // [ENT][COP]
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + KF::LUT_BYTES);                     // values
-  Stage* stages = reinterpret_cast<Stage*>(smem + KF::LUT_BYTES + (size_t)LUT_WORDS * 4);
+  Stage* stages = reinterpret_cast<Stage*>(smem + KF::LUT_BYTES + (size_t)VF::LUTW * 4);
   uint32_t* qopk = reinterpret_cast<uint32_t*>(stages + MW * NSTK);                      // [8][32][8]
   uint32_t* qopq = qopk + 8 * 32 * QOPK;                                                  // [8][32][4] (QJL)
   float4* s_head = reinterpret_cast<float4*>(qopq + (QJL ? 8 * 32 * QOPQ : 0));          // [8]
@@ -115,7 +177,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
-  build_value_lut(lut, a.cv, tid, MW * 32);
+  if (VB == 4)
+    build_value_lut(lut, a.cv, tid, MW * 32);
+  else
+    build_value_lut3(lut, a.cv, tid, MW * 32);
   // Key table: entry (idx, copy) = (fp16 heads, fp16 tails x 2^12) of the
   // centroids of two coordinates; idx = f0 | f1 << 2 | top0 << 4 | top1 << 5
   // (3-bit: f = 2-bit field, top = third index bit) or the byte f0 | f1 << 4
@@ -291,7 +356,8 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
     constexpr int NKC = MT * KF::REC / 4;
     constexpr int NQC = QJL ? MT : 0;
     constexpr int NNC = (QJL ? 3 : 2) * 4;
-    constexpr int NCH = NKC + NQC + NNC + 4 * MT;
+    constexpr int NVC = MT * VF::REC / 4;
+    constexpr int NCH = NKC + NQC + NNC + NVC;
     auto issue = [&](int k, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
       const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
@@ -323,10 +389,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
           const uint32_t off = arr == 0 ? offsetof(Stage, kn)
                                         : (arr == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn));
           cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tok1);
-        } else if (c < NCH) {                  // value codes: 16 tokens x 4 chunks
-          const int cc = c - NKC - NQC - NNC, tok = cc >> 2, part = cc & 3;
-          cp16(sb + offsetof(Stage, v) + tok * (VROW * 4) + part * 16,
-               a.vcodes + (rb + r + tok) * VW + part * 4, t0 + tok < tok1);
+        } else if (c < NCH) {                  // value codes: 16 tokens x 4 (3) chunks
+          const int cc = c - NKC - NQC - NNC, tok = cc / (VF::REC / 4), part = cc % (VF::REC / 4);
+          cp16(sb + offsetof(Stage, v) + tok * (VF::ROW * 4) + part * 16,
+               a.vcodes + (rb + r + tok) * VF::REC + part * 4, t0 + tok < tok1);
         }
       }
     };
@@ -476,7 +542,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
       const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
       const uint32_t pb0 = movtrans(pack_half2(p[0][0] * w0s, p[1][0] * w0s));
       const uint32_t pb1 = movtrans(pack_half2(p[0][1] * w8s, p[1][1] * w8s));
-      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
+      if constexpr (VB == 4)
+        value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
+      else
+        value_tile3(o, st.v, pb0, pb1, lut_lane, g, t);
       __syncwarp();
     }
     cp_wait<0>();
@@ -509,9 +578,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
 }  // namespace
 
 bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
-  if (c->d != D || c->bits_v != 4 || (a.G != 4 && a.G != 8)) return false;
-  const bool k3q = c->bk_lm == 3 && c->qjl_m == 128;
-  const bool mse = (c->bk_lm == 3 || c->bk_lm == 4) && c->qjl_m == 0;
+  if (c->d != D || (a.G != 4 && a.G != 8)) return false;
+  const bool k3q = c->bk_lm == 3 && c->qjl_m == 128 && c->bits_v == 4;
+  const bool mse = c->qjl_m == 0 && ((c->bk_lm == 3 && (c->bits_v == 4 || c->bits_v == 3)) ||
+                                     (c->bk_lm == 4 && c->bits_v == 4));
   if (!k3q && !mse) return false;
   if (a.max_T % 4 != 0) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.knorm) |
@@ -520,13 +590,20 @@ bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
   return (al & 15) == 0;
 }
 
-template <int KB, bool QJL, int G>
+template <int KB, bool QJL, int VB>
 static void lut_launch(const AttnArgs& a, unsigned blocks, cudaStream_t s) {
-  constexpr size_t sm = smem_lut<KB, QJL>();
-  if (a.block_table)
-    k_attn_lut<true, KB, QJL, G><<<blocks, MW * 32, sm, s>>>(a);
-  else
-    k_attn_lut<false, KB, QJL, G><<<blocks, MW * 32, sm, s>>>(a);
+  constexpr size_t sm = smem_lut<KB, QJL, VB>();
+  if (a.block_table) {
+    if (a.G == 8)
+      k_attn_lut<true, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
+    else
+      k_attn_lut<true, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
+  } else {
+    if (a.G == 8)
+      k_attn_lut<false, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
+    else
+      k_attn_lut<false, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
+  }
 }
 
 cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
@@ -540,37 +617,38 @@ cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a_in, float* out, c
   a.wpu = MW;
   const unsigned nb = (unsigned)blocks;
   const bool q = c->qjl_m > 0;
-  if (q && c->bk_lm == 3) {
-    if (a.G == 8) lut_launch<3, true, 8>(a, nb, s); else lut_launch<3, true, 4>(a, nb, s);
-  } else if (!q && c->bk_lm == 3) {
-    if (a.G == 8) lut_launch<3, false, 8>(a, nb, s); else lut_launch<3, false, 4>(a, nb, s);
-  } else if (!q && c->bk_lm == 4) {
-    if (a.G == 8) lut_launch<4, false, 8>(a, nb, s); else lut_launch<4, false, 4>(a, nb, s);
-  } else {
+  if (q && c->bk_lm == 3 && c->bits_v == 4)
+    lut_launch<3, true, 4>(a, nb, s);
+  else if (!q && c->bk_lm == 3 && c->bits_v == 4)
+    lut_launch<3, false, 4>(a, nb, s);
+  else if (!q && c->bk_lm == 4 && c->bits_v == 4)
+    lut_launch<4, false, 4>(a, nb, s);
+  else if (!q && c->bk_lm == 3 && c->bits_v == 3)
+    lut_launch<3, false, 3>(a, nb, s);
+  else
     return cudaErrorInvalidValue;
-  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_merge(c, a, out, s);
 }
 
-template <int KB, bool QJL, int G>
+template <int KB, bool QJL, int VB>
 static cudaError_t lut_configure() {
   const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  constexpr int sm = (int)smem_lut<KB, QJL>();
-  cudaError_t e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, G>, ms, sm);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, G>, ms, sm);
+  constexpr int sm = (int)smem_lut<KB, QJL, VB>();
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, 8, VB>, ms, sm)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 8, VB>, ms, sm)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, 4, VB>, ms, sm)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 4, VB>, ms, sm);
 }
 
 cudaError_t configure_attn_lut() {
   cudaError_t e;
-  if ((e = lut_configure<3, true, 8>()) != cudaSuccess) return e;
   if ((e = lut_configure<3, true, 4>()) != cudaSuccess) return e;
-  if ((e = lut_configure<3, false, 8>()) != cudaSuccess) return e;
   if ((e = lut_configure<3, false, 4>()) != cudaSuccess) return e;
-  if ((e = lut_configure<4, false, 8>()) != cudaSuccess) return e;
-  return lut_configure<4, false, 4>();
+  if ((e = lut_configure<4, false, 4>()) != cudaSuccess) return e;
+  return lut_configure<3, false, 3>();
 }
 
 }  // namespace tqk

@@ -510,7 +510,7 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
 
 # --- norm-corrected cache formats -------------------------------------------------
 @pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("k3v4_nc", 16), ("4bit_nc", 8), ("4bit_nc", 16),
-                                     ("3bit_nc", 8)])
+                                     ("3bit_nc", 8), ("3bit_nc", 16)])
 def test_norm_corrected_variants(cuda, name, Hq):
     """The MSE-only _nc formats: quantize through the bulk and the small-batch
     kernels (stored norm n / |c[idx]|), logits, ragged decode attention, and
@@ -581,7 +581,8 @@ def _to_paged(cache, B, Hkv, max_T, bs, perm):
 
 @pytest.mark.parametrize("Hq,Hkv,bk,bs,variant", [
     (8, 2, 3, 32, None), (16, 2, 3, 16, None), (16, 2, 4, 48, None), (4, 4, 3, 16, None),
-    (8, 2, 4, 16, None), (8, 2, None, 32, "4bit_nc"), (16, 2, None, 16, "k3v4_nc")])
+    (8, 2, 4, 16, None), (8, 2, None, 32, "4bit_nc"), (16, 2, None, 16, "k3v4_nc"),
+    (8, 2, None, 16, "3bit_nc"), (16, 2, None, 48, "3bit_nc")])
 def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs, variant):
     """The paged decode reads the same records through the block table, so it
     must reproduce the contiguous decode bit for bit (ragged lengths,
