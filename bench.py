@@ -50,8 +50,9 @@ WORKLOADS = {
     "70b-decode-k4v4": dict(B=4, Hq=64, Hkv=8, d=128, T=131072, bits_k=4, bits_v=4, m=128),
 }
 QUANT_SWEEP = dict(tokens=131072, heads=8, d=128, bits=(2, 3, 4))
-# The norm-corrected MSE-only cache formats, timed on the Llama-3-8B decode shape.
-NC_VARIANTS = ("k3v4_nc", "4bit_nc", "3bit_nc")
+# The other cache formats of the vLLM study (norm-corrected MSE-only, and
+# 8-bit keys), timed on the Llama-3-8B decode shape.
+FORMAT_VARIANTS = ("k3v4_nc", "4bit_nc", "3bit_nc", "k8v4")
 
 
 def peaks():
@@ -331,10 +332,10 @@ def vector_search(tq, tq_inputs, torch, dev, sm_mhz_max, steps=3, warmup=1):
 
 
 def variant_decode(tq, tq_inputs, torch, dev, hbm_peak, shape, steps=20, warmup=3):
-    """tq_attn_decode for each norm-corrected format on one decode shape."""
+    """tq_attn_decode for each format of FORMAT_VARIANTS on one decode shape."""
     B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
     out = {}
-    for name in NC_VARIANTS:
+    for name in FORMAT_VARIANTS:
         ctx = tq.Context.variant(name, d, 0)
         kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
         vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
@@ -365,9 +366,9 @@ def variant_decode(tq, tq_inputs, torch, dev, hbm_peak, shape, steps=20, warmup=
         ms = e0.elapsed_time(e1) / steps
         kb, vb = ctx.key_layout["bytes_per_vector"], ctx.value_layout["bytes_per_vector"]
         alg = B * Hkv * T * (kb + vb) + B * Hq * d * 2 + B * Hq * d * 4
-        bits_k, bits_v, _, _ = tq.VARIANTS[name]
-        out[name] = {"kv_format": f"keys {bits_k} Lloyd-Max bits, values {bits_v} bits, MSE only, "
-                                  f"norm-corrected; {kb + vb} B per token-head",
+        bits_k, bits_v, _, nc = tq.VARIANTS[name]
+        out[name] = {"kv_format": f"keys {bits_k} Lloyd-Max bits, values {bits_v} bits, MSE only"
+                                  f"{', norm-corrected' if nc else ''}; {kb + vb} B per token-head",
                      "attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
                      "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak}
         del g, kc, vc, ws
@@ -611,7 +612,7 @@ def run_gpu(args, w):
         if vsearch is not None:
             line["vector_search"] = vsearch
             line["small_case"] = small
-            line["norm_corrected_decode"] = variants
+            line["format_variants_decode"] = variants
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)

@@ -160,13 +160,15 @@ def tq_host_tables(d, bits_k, bits_v, qjl_m, seed):
 
 # Named cache formats: name -> (bits_k, bits_v, key QJL stage with m = d,
 # norm correction of keys and values).  k3v4 / k4v4 spend one key bit on QJL;
-# the _nc formats of the vLLM study are MSE-only with norm correction.
+# the _nc formats of the vLLM study are MSE-only with norm correction, and
+# k8v4 has MSE-only 8-bit keys.
 VARIANTS = {
     "k3v4": (3, 4, True, False),
     "k4v4": (4, 4, True, False),
     "k3v4_nc": (3, 4, False, True),
     "4bit_nc": (4, 4, False, True),
     "3bit_nc": (3, 3, False, True),
+    "k8v4": (8, 4, False, False),
 }
 
 

@@ -42,13 +42,13 @@ bool valid_dims(int d, int bits_k, int bits_v, int qjl_m, int* code) {
     return false;
   }
   const int bk_lm = qjl_m > 0 ? bits_k - 1 : bits_k;
-  if (bk_lm < 1 || bk_lm > 4) {
-    *code = fail(TQ_ERR_UNSUPPORTED, "bits_k=%d with qjl_m=%d gives %d Lloyd-Max bits (need 1..4)",
+  if (!((bk_lm >= 1 && bk_lm <= 4) || bk_lm == 8)) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "bits_k=%d with qjl_m=%d gives %d Lloyd-Max bits (need 1..4 or 8)",
                  bits_k, qjl_m, bk_lm);
     return false;
   }
-  if (bits_v < 1 || bits_v > 4) {
-    *code = fail(TQ_ERR_UNSUPPORTED, "bits_v=%d unsupported (need 1..4)", bits_v);
+  if (!((bits_v >= 1 && bits_v <= 4) || bits_v == 8)) {
+    *code = fail(TQ_ERR_UNSUPPORTED, "bits_v=%d unsupported (need 1..4 or 8)", bits_v);
     return false;
   }
   return true;
@@ -156,16 +156,16 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
   }
   const int dp = c->dpad;
   const size_t nPiT = (size_t)d * dp, nPi = (size_t)d * d, nST = (size_t)d * dp, nS = (size_t)dp * d;
-  const size_t total = (nPiT + nPi + nST + nS + 4 * 16) * sizeof(float);
+  const size_t total = (nPiT + nPi + nST + nS + 4 * tqk::kMaxLevels) * sizeof(float);
   std::vector<float> h(total / sizeof(float), 0.f);
   float* hPiT = h.data();
   float* hPi = hPiT + nPiT;
   float* hST = hPi + nPi;
   float* hS = hST + nST;
   float* hck = hS + nS;
-  float* hbk = hck + 16;
-  float* hcv = hbk + 16;
-  float* hbv = hcv + 16;
+  float* hbk = hck + tqk::kMaxLevels;
+  float* hcv = hbk + tqk::kMaxLevels;
+  float* hbv = hcv + tqk::kMaxLevels;
   for (int j = 0; j < d; ++j)
     for (int k = 0; k < d; ++k) {
       hPiT[(size_t)k * dp + j] = (float)c->Pi[(size_t)j * d + k];
@@ -176,7 +176,7 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
       hST[(size_t)k * dp + i] = (float)c->S[(size_t)i * d + k];
       hS[(size_t)i * d + k] = (float)c->S[(size_t)i * d + k];
     }
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < tqk::kMaxLevels; ++i) {
     hbk[i] = INFINITY;
     hbv[i] = INFINITY;
   }
@@ -362,7 +362,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;
   }
-  const bool tc = !pg.table && !a.nc && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+  const bool tc = !pg.table && !a.nc && a.bits <= 4 && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
     tqk::QuantTcArgs t{};
@@ -769,6 +769,7 @@ int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* cod
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
     return fail(TQ_ERR_ARG, "tq_topk: bad dtype=%d", dtype);
   if (nq < 0 || n < 0 || k < 1 || k > 32) return fail(TQ_ERR_ARG, "tq_topk: bad sizes (k must be 1..32)");
+  if (c->bk_lm > 4) return fail(TQ_ERR_UNSUPPORTED, "tq_topk: keys of %d Lloyd-Max bits (need 1..4)", c->bk_lm);
   if (nq == 0) return TQ_OK;
   if (n > 0x7ffffff0LL) return fail(TQ_ERR_UNSUPPORTED, "tq_topk: n too large");
   if (nq > 65535LL * 16) return fail(TQ_ERR_UNSUPPORTED, "tq_topk: nq too large");

@@ -30,10 +30,10 @@ struct tq_ctx {
   const float* Pi_f = nullptr;  // [d][d]     row-major Pi
   const float* ST = nullptr;    // [d][dpad]  ST[k*dpad+i] = S[i][k]; zero for i >= m
   const float* S_f = nullptr;   // [dpad][d]  row-major S; zero rows for i >= m
-  const float* ck_f = nullptr;  // [16] key centroids (padded)
-  const float* bk_f = nullptr;  // [16] key boundaries (padded with +inf)
-  const float* cv_f = nullptr;  // [16]
-  const float* bv_f = nullptr;  // [16]
+  const float* ck_f = nullptr;  // [256] key centroids (padded)
+  const float* bk_f = nullptr;  // [256] key boundaries (padded with +inf)
+  const float* cv_f = nullptr;  // [256]
+  const float* bv_f = nullptr;  // [256]
   // Tensor-core quantize (d = 128): swizzled fp16 operand images and QJL row norms.
   bool tc_ok = false;
   void* tc_block = nullptr;
@@ -61,6 +61,9 @@ inline int tq_code_words(int d, int b) {
 }
 
 namespace tqk {
+
+// Codebook sizes up to 2^8 levels (Lloyd-Max bits 1..4 and 8).
+constexpr int kMaxLevels = 256;
 
 struct QuantArgs {
   const void* x;

@@ -40,7 +40,17 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Index of a coordinate: number of boundaries at or below y (ties go up).
+// The boundaries ascend, so for the 255 of an 8-bit codebook a bisection for
+// the first boundary above y gives the same count.
 __device__ __forceinline__ int lm_index(float y, const float* sb, int nb) {
+  if (nb > 15) {
+    int lo = 0, hi = nb;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (y >= sb[mid]) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  }
   int idx = 0;
   for (int t = 0; t < nb; ++t) idx += (y >= sb[t]) ? 1 : 0;
   return idx;
@@ -160,12 +170,12 @@ template <int J>
 __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
   constexpr int DP = J * 32;
   extern __shared__ float smem[];
-  __shared__ float s_cen[16], s_bnd[16];
+  __shared__ float s_cen[kMaxLevels], s_bnd[kMaxLevels];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* sx = smem + warp * (DP * QV);  // [DP][QV]
-  if (threadIdx.x < 16) {
-    s_cen[threadIdx.x] = (threadIdx.x < (1 << a.bits)) ? a.cen[threadIdx.x] : 0.f;
-    s_bnd[threadIdx.x] = (threadIdx.x < a.nbnd) ? a.bnd[threadIdx.x] : INFINITY;
+  for (int e = threadIdx.x; e < kMaxLevels; e += blockDim.x) {
+    s_cen[e] = (e < (1 << a.bits)) ? a.cen[e] : 0.f;
+    s_bnd[e] = (e < a.nbnd) ? a.bnd[e] : INFINITY;
   }
   __syncthreads();
   const int64_t ngroups = (a.n + QV - 1) / QV;
@@ -335,13 +345,13 @@ template <int QS>
 __device__ __forceinline__ void quantize_small_body(const QuantArgs& a, int dpad, int64_t blk, float* sh) {
   float* Ms = sh + QS * dpad;
   __shared__ float red[QS][8];
-  __shared__ float s_cen[16], s_bnd[16];
+  __shared__ float s_cen[kMaxLevels], s_bnd[kMaxLevels];
   const int j = threadIdx.x, lane = j & 31, warp = j >> 5, nwarp = blockDim.x >> 5;
   const int64_t v0 = blk * QS;
   const int nv = (int)min((int64_t)QS, a.n - v0);
-  if (j < 16) {
-    s_cen[j] = (j < (1 << a.bits)) ? a.cen[j] : 0.f;
-    s_bnd[j] = (j < a.nbnd) ? a.bnd[j] : INFINITY;
+  for (int e = j; e < kMaxLevels; e += blockDim.x) {
+    s_cen[e] = (e < (1 << a.bits)) ? a.cen[e] : 0.f;
+    s_bnd[e] = (e < a.nbnd) ? a.bnd[e] : INFINITY;
   }
   float nrm[QS];
 #pragma unroll
@@ -574,15 +584,15 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
   float* ssv = sq + a.G * DP;           // [G][DP]
   float* sp = ssv + a.G * DP;           // [AT][G]   p * |v|
   uint32_t* svc = reinterpret_cast<uint32_t*>(sp + AT * a.G);  // [AT][wv]
-  __shared__ float s_ck[16], s_cv[16];
+  __shared__ float s_ck[kMaxLevels], s_cv[kMaxLevels];
   __shared__ float s_wred[AT / 32][GMAX];
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.G;
-  if (tid < 16) {
-    s_ck[tid] = (tid < (1 << a.bk)) ? a.ck[tid] : 0.f;
-    s_cv[tid] = (tid < (1 << a.bv)) ? a.cv[tid] : 0.f;
+  for (int e = tid; e < kMaxLevels; e += AT) {
+    s_ck[e] = (e < (1 << a.bk)) ? a.ck[e] : 0.f;
+    s_cv[e] = (e < (1 << a.bv)) ? a.cv[e] : 0.f;
   }
   for (int e = tid; e < G * DP; e += AT) {
     const int h = e / DP, j = e % DP;
@@ -614,7 +624,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
     for (int h = 0; h < GMAX; ++h) sc[h] = kNegInf;
     if (valid) {
       const int64_t r = kv_row0 + t;
-      uint32_t w[4 * 8];
+      uint32_t w[64];   // up to d = 256 at 8 bits
       for (int e = 0; e < kw; ++e) w[e] = a.kcodes[r * kw + e];
       float acc[GMAX], acc2[GMAX];
 #pragma unroll
@@ -830,10 +840,10 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
                                                 int64_t nk, float* out) {
   constexpr int DP = J * 32;
   __shared__ float sx[LQB][DP], sq[LQB][DP], ss[LQB][DP];
-  __shared__ float s_ck[16];
+  __shared__ float s_ck[kMaxLevels];
   const int tid = threadIdx.x;
   const int64_t q0 = (int64_t)blockIdx.y * LQB;
-  if (tid < 16) s_ck[tid] = (tid < (1 << bk)) ? ck[tid] : 0.f;
+  for (int e = tid; e < kMaxLevels; e += blockDim.x) s_ck[e] = (e < (1 << bk)) ? ck[e] : 0.f;
   for (int e = tid; e < LQB * DP; e += blockDim.x) {
     const int qq = e / DP, k = e % DP;
     sx[qq][k] = (k < d && q0 + qq < nq) ? load_elem(q, dtype, (q0 + qq) * d + k) : 0.f;
@@ -857,7 +867,7 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
   const int64_t key = (int64_t)blockIdx.x * blockDim.x + tid;
   if (key >= nk) return;
   const int mw = (m + 31) >> 5;
-  uint32_t w[4 * 8];
+  uint32_t w[64];   // up to d = 256 at 8 bits
   for (int e = 0; e < kw; ++e) w[e] = kcodes[key * kw + e];
   float acc[LQB], acc2[LQB];
 #pragma unroll
@@ -1159,7 +1169,7 @@ static cudaError_t configure_J() {
   cudaError_t e = cudaFuncSetAttribute(k_quantize<J>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)(QWARPS * J * 32 * QV * sizeof(float)));
   if (e != cudaSuccess) return e;
-  const int attn_max = (2 * GMAX * J * 32 + AT * GMAX) * (int)sizeof(float) + AT * 32 * (int)sizeof(uint32_t);
+  const int attn_max = (2 * GMAX * J * 32 + AT * GMAX) * (int)sizeof(float) + AT * 64 * (int)sizeof(uint32_t);
   e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_max);
   return e;
 }

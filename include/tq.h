@@ -33,13 +33,14 @@
  *   TQ_ERR_CUDA (a CUDA launch or runtime error), TQ_ERR_WORKSPACE (workspace
  *   missing or too small).  tq_last_error() then returns a message (per
  *   thread; valid until the next call on that thread).
- * - Sizes: 8 <= d <= 256 with d % 8 == 0; Lloyd-Max bits 1..4;
+ * - Sizes: 8 <= d <= 256 with d % 8 == 0; Lloyd-Max bits 1..4 or 8 (8-bit
+ *   codes serve the k8v4 format; tq_topk takes 1..4);
  *   0 <= qjl_m <= 32*ceil(d/32), qjl_m % 8 == 0.
  *
  * Packed layout of one vector
  * ---------------------------
  *   codes  uint32[W]   Lloyd-Max indices as b-bit fields, LSB first, 32/b
- *                      fields per word, for b in {1, 2, 4}: coordinate j sits
+ *                      fields per word, for b in {1, 2, 4, 8}: coordinate j sits
  *                      in word j/(32/b) at bit b*(j%(32/b)); W = ceil(d*b/32).
  *                      For b = 3 the low two bits of every index form a 2-bit
  *                      field stream (ceil(d/16) words) followed by a 1-bit
@@ -362,7 +363,8 @@ size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
  *   codes/qjl/norm/rnorm  device key arrays for the n database vectors.
  *   k        1..32.
  *   idx      device, int32 [nq][k];  score  device, float [nq][k].
- * If n < k the missing slots get index -1 and score -inf.
+ * If n < k the missing slots get index -1 and score -inf.  Keys of 8
+ * Lloyd-Max bits: TQ_ERR_UNSUPPORTED.
  */
 int tq_topk(tq_ctx* ctx, const void* q, int dtype, int64_t nq,
             const uint32_t* codes, const uint32_t* qjl, const float* norm,

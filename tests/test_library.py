@@ -49,7 +49,8 @@ def test_host_tables_match_oracle(d, bits_k, bits_v, m, seed):
 
 
 @pytest.mark.parametrize("args", [(7, 3, 4, 0), (300, 3, 4, 0), (128, 1, 4, 128), (128, 6, 4, 0),
-                                  (128, 3, 5, 0), (128, 3, 4, 12), (128, 3, 4, 160)])
+                                  (128, 3, 5, 0), (128, 3, 4, 12), (128, 3, 4, 160), (128, 8, 4, 128),
+                                  (128, 3, 7, 0), (128, 9, 4, 0)])
 def test_unsupported_sizes_rejected(args):
     with pytest.raises(tq.TQError) as e:
         tq.tq_host_tables(*args, 0)
@@ -73,5 +74,5 @@ def test_norm_correction_flags_validated_before_any_device_call():
         tq.tq_init_ex(128, 3, 4, 0, 0, 4)
     assert "flag" in str(e.value)
     with pytest.raises(ValueError):
-        tq.Context.variant("k8v4", 128)
-    assert set(tq.VARIANTS) == {"k3v4", "k4v4", "k3v4_nc", "4bit_nc", "3bit_nc"}
+        tq.Context.variant("k2v2", 128)
+    assert set(tq.VARIANTS) == {"k3v4", "k4v4", "k3v4_nc", "4bit_nc", "3bit_nc", "k8v4"}

@@ -82,7 +82,7 @@ def test_rotated_coordinates_follow_beta_law(d):
 
 
 # --- R2 / Lloyd-Max codebook ------------------------------------------------
-@pytest.mark.parametrize("d,bits", [(128, 1), (128, 2), (128, 3), (128, 4), (200, 3), (37, 2)])
+@pytest.mark.parametrize("d,bits", [(128, 1), (128, 2), (128, 3), (128, 4), (200, 3), (37, 2), (128, 8)])
 def test_lloyd_max_fixed_point(d, bits):
     cb = o.lloyd_max(d, bits)
     L = 1 << bits
@@ -121,7 +121,7 @@ def test_large_d_limit_is_max_gaussian_table():
         assert abs(o.distortion(d, cb) - mse) < 2e-3 * mse + 5e-5
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
 def test_empirical_mse_within_two_percent(bits):
     d = 128
     tab = o.make_tables(d, bits, bits, 0, 21)
@@ -184,6 +184,20 @@ def test_norm_correction_mean_square_is_one_minus_distortion(bits):
 def test_norm_correction_needs_mse_only_keys():
     with pytest.raises(ValueError):
         o.make_tables(64, 3, 4, 64, 1, nc_k=True)
+
+
+@pytest.mark.parametrize("d", [128, 200])
+def test_eight_bit_distortion_near_panter_dite(d):
+    """High-resolution theory (Panter & Dite 1951): with L levels the least
+    mean-square distortion tends to (int f^(1/3))^3 / (12 L^2).  At 256 levels
+    the 8-bit codebook must sit just below it (within 1.5 %), and the 4-bit
+    one visibly further below (the bound is asymptotic)."""
+    f3 = integrate.quad(lambda t: o.beta_density(np.array([t]), d)[0] ** (1 / 3), -1, 1, points=[0],
+                        limit=400, epsabs=1e-14)[0]
+    for bits, lo, hi in ((8, -0.015, 0.0), (4, -0.15, -0.05)):
+        pd = d * f3 ** 3 / (12 * (1 << bits) ** 2)
+        ratio = o.distortion(d, o.lloyd_max(d, bits)) / pd - 1
+        assert lo < ratio < hi, (bits, ratio)
 
 
 def test_printed_three_bit_cosine():
