@@ -187,28 +187,87 @@ static void cell_integrals(int d, double a, double b, const std::vector<double>&
   *moment = m1;
 }
 
+// One Lloyd-Max step on the upper-half centroids c (boundary 0 in the
+// middle): edges at the midpoints, each centroid the mean of its cell.  Also
+// returns the cells' (unnormalised) masses and edges.  Panels of at most 0.02
+// rad in theta = asin t keep the 24-point rule exact to rounding for every
+// supported d.
+static void lloyd_step(int d, const std::vector<double>& c, const std::vector<double>& gx,
+                       const std::vector<double>& gw, std::vector<double>& u, std::vector<double>& mass,
+                       std::vector<double>& edge) {
+  const int half = (int)c.size();
+  edge.resize(half + 1);
+  edge[0] = 0.0;
+  for (int i = 1; i < half; ++i) edge[i] = 0.5 * (c[i - 1] + c[i]);
+  edge[half] = 1.0;
+  u.resize(half);
+  mass.resize(half);
+  for (int i = 0; i < half; ++i) {
+    const double a = std::asin(edge[i]), b = std::asin(edge[i + 1]);
+    const int panels = std::max(1, (int)std::ceil((b - a) / 0.02));
+    double m0, m1;
+    cell_integrals(d, a, b, gx, gw, panels, &m0, &m1);
+    u[i] = m1 / m0;
+    mass[i] = m0;
+  }
+}
+
 // Lloyd-Max centroids (2^bits, increasing) and interior boundaries for f_d.
+// The plain alternation of the two optimality conditions converges slowly
+// with many levels (8 bits), so once its steps fall below 1e-7 (or after 4000
+// of them) Newton steps on c - U(c) finish the same fixed point: U_i depends
+// on c_{i-1}, c_i, c_{i+1} through the two midpoints, with
+// dU_i/dhi = f(hi) (hi - U_i) / P_i and dU_i/dlo = f(lo) (U_i - lo) / P_i, so
+// each step is a tridiagonal solve.  Newton stops at 1e-15 or, after eight
+// steps, below 1e-12 (the rounding floor of the cell masses).
 static void lloyd_max_solve(int d, int bits, std::vector<double>& cen, std::vector<double>& bnd) {
   const int L = 1 << bits, half = L / 2;
   std::vector<double> gx, gw;
   gauss_legendre(24, gx, gw);
-  const int panels = 48;
-  std::vector<double> c(half);
+  std::vector<double> c(half), u, mass, edge;
   for (int i = 0; i < half; ++i) c[i] = (i + 0.5) / half * 3.0 / std::sqrt((double)d);
-  std::vector<double> edge(half + 1);
-  for (int it = 0; it < 200000; ++it) {
-    edge[0] = 0.0;
-    for (int i = 1; i < half; ++i) edge[i] = 0.5 * (c[i - 1] + c[i]);
-    edge[half] = 1.0;
-    double delta = 0.0;
+  double delta = 1.0;
+  for (int it = 0; it < 4000; ++it) {
+    lloyd_step(d, c, gx, gw, u, mass, edge);
+    delta = 0.0;
+    for (int i = 0; i < half; ++i) delta = std::max(delta, std::fabs(u[i] - c[i]));
+    c = u;
+    if (delta < 1e-15 || (delta < 1e-7 && half > 1)) break;
+  }
+  const double ex = 0.5 * (d - 3);
+  auto dens = [&](double t) { return t >= 1.0 ? 0.0 : std::pow(1.0 - t * t, ex); };
+  std::vector<double> lo(half), di(half), up(half), r(half), step(half), cand(half);
+  for (int newton = 1; delta >= 1e-15 && half > 1 && newton <= 200; ++newton) {
+    lloyd_step(d, c, gx, gw, u, mass, edge);
     for (int i = 0; i < half; ++i) {
-      double m0, m1;
-      cell_integrals(d, std::asin(edge[i]), std::asin(edge[i + 1]), gx, gw, panels, &m0, &m1);
-      const double cn = m1 / m0;
-      delta = std::max(delta, std::fabs(cn - c[i]));
-      c[i] = cn;
+      const double dh = i + 1 < half ? dens(edge[i + 1]) * (edge[i + 1] - u[i]) / mass[i] : 0.0;
+      const double dl = i > 0 ? dens(edge[i]) * (u[i] - edge[i]) / mass[i] : 0.0;
+      lo[i] = -0.5 * dl;              // (I - J)_{i,i-1}
+      up[i] = -0.5 * dh;              // (I - J)_{i,i+1}
+      di[i] = 1.0 - 0.5 * (dl + dh);
+      r[i] = u[i] - c[i];
     }
-    if (delta < 1e-15) break;
+    // Thomas algorithm for (I - J) step = r.
+    for (int i = 1; i < half; ++i) {
+      const double w = lo[i] / di[i - 1];
+      di[i] -= w * up[i - 1];
+      r[i] -= w * r[i - 1];
+    }
+    step[half - 1] = r[half - 1] / di[half - 1];
+    for (int i = half - 2; i >= 0; --i) step[i] = (r[i] - up[i] * step[i + 1]) / di[i];
+    double scale = 1.0;
+    for (int tries = 0; tries < 60; ++tries, scale *= 0.5) {   // keep the centroids increasing in (0, 1)
+      bool ok = true;
+      for (int i = 0; i < half; ++i) {
+        cand[i] = c[i] + scale * step[i];
+        if (cand[i] <= (i ? cand[i - 1] : 0.0) || cand[i] >= 1.0) ok = false;
+      }
+      if (ok) break;
+    }
+    delta = 0.0;
+    for (int i = 0; i < half; ++i) delta = std::max(delta, std::fabs(cand[i] - c[i]));
+    c = cand;
+    if (newton >= 8 && delta < 1e-12) break;
   }
   cen.resize(L);
   for (int i = 0; i < half; ++i) {
