@@ -1,8 +1,8 @@
 // Decode attention from packed codes whose keys are dequantized through a
 // table: 3-bit Lloyd-Max keys with the QJL bit (k4v4: m = 128), and the
-// MSE-only norm-corrected formats with 3- or 4-bit keys (k3v4_nc, 4bit_nc,
-// 3bit_nc); values 4 bits (3 bits for 3bit_nc), d = 128, GQA group 4 or 8,
-// on the tensor cores (sm_100a).
+// MSE-only formats: norm-corrected 3- or 4-bit keys (k3v4_nc, 4bit_nc,
+// 3bit_nc) and 8-bit keys (k8v4); values 4 bits (3 bits for 3bit_nc),
+// d = 128, GQA group 4 or 8, on the tensor cores (sm_100a).
 //
 // Same quantities as the 2-bit-key kernels ("What is TurboQuant?", "How
 // TurboQuant works", closing paragraph; "How to implement" part 1):
@@ -51,13 +51,19 @@ constexpr int NSTK = 3;      // pipeline stages per warp
 constexpr int QOPK = 8;      // words per lane and key k-step (G = 8: 6 used, G = 4: 4 used)
 constexpr int QOPQ = 4;      // words per lane and QJL k-step (2 MMAs x 2)
 
+// Key formats.  3 and 4 bits: a table entry covers two coordinates (8 bytes:
+// heads, tails).  8 bits: an entry covers one coordinate (4 bytes: head,
+// tail), 32 copies, and staged rows of 36 words keep the 16-byte loads of
+// each quarter-warp on distinct banks.
 template <int KB>
 struct KeyFmt {
-  static constexpr int K2W = KB == 3 ? 8 : 16;     // words of the 2-bit stream / of the 4-bit fields
-  static constexpr int REC = KB == 3 ? 12 : 16;    // words per key record
-  static constexpr int ENT = KB == 3 ? 64 : 256;   // table entries (two coordinates)
-  static constexpr int COP = KB == 3 ? 32 : 16;    // copies of the table
-  static constexpr size_t LUT_BYTES = (size_t)ENT * COP * 8;
+  static constexpr int K2W = KB == 3 ? 8 : (KB == 4 ? 16 : 36);   // staged row (words)
+  static constexpr int REC = KB == 3 ? 12 : (KB == 4 ? 16 : 32);  // words per key record
+  static constexpr int ENT = KB == 3 ? 64 : 256;                  // table entries
+  static constexpr int COP = KB == 4 ? 16 : 32;                   // copies of the table
+  static constexpr int ESZ = KB == 8 ? 4 : 8;                     // bytes per entry
+  static constexpr size_t LUT_BYTES = (size_t)ENT * COP * ESZ;
+  static constexpr int NS = KB == 8 ? 2 : NSTK;                   // pipeline stages (shared memory)
 };
 
 // Values: 4-bit fields (16 words per token, rows padded to VROW) or 3-bit
@@ -72,8 +78,8 @@ struct ValFmt {
 
 template <int KB, bool QJL, int VB>
 struct StageL {
-  uint32_t k2[MT][KeyFmt<KB>::K2W];   // 2-bit stream (3-bit keys) or the 4-bit fields
-  uint32_t k1[MT][4];                 // top-bit stream (3-bit keys)
+  uint32_t k2[MT][KeyFmt<KB>::K2W];   // 2-bit stream (3-bit keys) or the 4- / 8-bit fields
+  uint32_t k1[MT][KB == 3 ? 4 : 1];   // top-bit stream (3-bit keys)
   uint32_t q[MT][QJL ? QW : 1];       // QJL words
   float kn[MT];
   float kr[MT];
@@ -83,7 +89,8 @@ struct StageL {
 
 template <int KB, bool QJL, int VB>
 constexpr size_t smem_lut() {
-  return KeyFmt<KB>::LUT_BYTES + (size_t)ValFmt<VB>::LUTW * 4 + (size_t)MW * NSTK * sizeof(StageL<KB, QJL, VB>) +
+  return KeyFmt<KB>::LUT_BYTES + (size_t)ValFmt<VB>::LUTW * 4 +
+         (size_t)MW * KeyFmt<KB>::NS * sizeof(StageL<KB, QJL, VB>) +
          (size_t)8 * 32 * QOPK * 4 + (QJL ? (size_t)8 * 32 * QOPQ * 4 : 0) + 8 * 16 + MW * 4 + 16 * 4;
 }
 
@@ -151,10 +158,17 @@ __device__ __forceinline__ uint32_t klut_off(uint32_t w2, uint32_t w1) {
   const uint32_t top = (w1 >> (SH + 2 * S)) & 3u;
   return (nib | (top << 4)) << 8;
 }
-// 4-bit keys: byte B of word w indexes the table (16 copies * 8 bytes).
+// 4-bit keys: byte B of word w indexes the table (16 copies * 8 bytes); 8-bit
+// keys likewise (32 copies * 4 bytes).
 template <int B>
 __device__ __forceinline__ uint32_t klut4_off(uint32_t w) {
   return __byte_perm(w, 0, 0x4440 + B) << 7;
+}
+// 8-bit keys: the (head, tail) operand pair of coordinates in bytes B, B+1 of w.
+template <int B>
+__device__ __forceinline__ uint2 k8_pair(uint32_t lane_base, uint32_t w) {
+  const uint32_t x0 = lds32(lane_base + klut4_off<B>(w)), x1 = lds32(lane_base + klut4_off<B + 1>(w));
+  return make_uint2(__byte_perm(x0, x1, 0x5410), __byte_perm(x0, x1, 0x7632));
 }
 
 template <bool PAGED, int KB, bool QJL, int G, int VB>
@@ -168,7 +182,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
   uint2* klut = reinterpret_cast<uint2*>(smem);                                          // [ENT][COP]
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + KF::LUT_BYTES);                     // values
   Stage* stages = reinterpret_cast<Stage*>(smem + KF::LUT_BYTES + (size_t)VF::LUTW * 4);
-  uint32_t* qopk = reinterpret_cast<uint32_t*>(stages + MW * NSTK);                      // [8][32][8]
+  uint32_t* qopk = reinterpret_cast<uint32_t*>(stages + MW * KF::NS);                    // [8][32][8]
   uint32_t* qopq = qopk + 8 * 32 * QOPK;                                                  // [8][32][4] (QJL)
   float4* s_head = reinterpret_cast<float4*>(qopq + (QJL ? 8 * 32 * QOPQ : 0));          // [8]
   float* s_vmax = reinterpret_cast<float*>(s_head + 8);                                  // [MW]
@@ -187,6 +201,12 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
   // (4-bit fields).
   for (int e = tid; e < KF::ENT * KF::COP; e += MW * 32) {
     const int idx = e / KF::COP;
+    if (KB == 8) {   // one coordinate: (head, tail x 2^12)
+      const float c0 = a.ck[idx];
+      const float h0 = __half2float(__float2half_rn(c0));
+      reinterpret_cast<uint32_t*>(klut)[e] = pack_half2(h0, (c0 - h0) * 4096.f);
+      continue;
+    }
     int i0, i1;
     if (KB == 3) {
       i0 = (idx & 3) | (((idx >> 4) & 1) << 2);
@@ -210,11 +230,12 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
   const int64_t x1 = (cta + 1) * W / NC;
   int b = locate_sequence(P, a.B, x);
 
-  const uint32_t klut_lane = (uint32_t)__cvta_generic_to_shared(klut) + (lane % KF::COP) * 8;
+  const uint32_t klut_lane = (uint32_t)__cvta_generic_to_shared(klut) + (lane % KF::COP) * KF::ESZ;
+  constexpr int NS = KF::NS;
   const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
   const uint32_t qopk_lane = (uint32_t)__cvta_generic_to_shared(qopk) + lane * QOPK * 4;
   const uint32_t qopq_lane = (uint32_t)__cvta_generic_to_shared(qopq) + lane * QOPQ * 4;
-  Stage* my = stages + warp * NSTK;
+  Stage* my = stages + warp * NS;
   const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
 
   while (x < x1) {
@@ -373,10 +394,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
             part = c % 3;
             dst = part < 2 ? (uint32_t)(offsetof(Stage, k2) + tok * 32 + part * 16)
                            : (uint32_t)(offsetof(Stage, k1) + tok * 16);
-          } else {                             // 16 tokens x 4 chunks
-            tok = c >> 2;
-            part = c & 3;
-            dst = (uint32_t)(offsetof(Stage, k2) + tok * 64 + part * 16);
+          } else {                             // 16 tokens x 4 (8) chunks
+            tok = c / (KF::REC / 4);
+            part = c % (KF::REC / 4);
+            dst = (uint32_t)(offsetof(Stage, k2) + tok * (KF::K2W * 4) + part * 16);
           }
           cp16(sb + dst, kbase + (r + tok) * (KF::REC * 4) + part * 16, t0 + tok < tok1);
         } else if (c < NKC + NQC) {            // QJL words: 16 tokens x 1 chunk
@@ -397,7 +418,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
       }
     };
 #pragma unroll
-    for (int k = 0; k < NSTK - 1; ++k) {
+    for (int k = 0; k < NS - 1; ++k) {
       if (k < ntw) issue(k, k);
       cp_commit();
     }
@@ -413,11 +434,11 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
     for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
     for (int k = 0; k < ntw; ++k) {
-      if (k + NSTK - 1 < ntw) issue(k + NSTK - 1, (k + NSTK - 1) % NSTK);
+      if (k + NS - 1 < ntw) issue(k + NS - 1, (k + NS - 1) % NS);
       cp_commit();
-      cp_wait<NSTK - 1>();
+      cp_wait<NS - 1>();
       __syncwarp();
-      const Stage& st = my[k % NSTK];
+      const Stage& st = my[k % NS];
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
 
       // ---- logits: heads t (accH0) and 4 + t (accH1), tails (accL), QJL (acs) ----
@@ -447,6 +468,19 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
           TQ_K3STEP(0) TQ_K3STEP(1) TQ_K3STEP(2) TQ_K3STEP(3) TQ_K3STEP(4) TQ_K3STEP(5)
           TQ_K3STEP(6) TQ_K3STEP(7)
 #undef TQ_K3STEP
+        } else if (KB == 8) {
+          // k-step s: bytes 2 (s & 1), +1 of word s >> 1 of the first and of
+          // the second 16 coordinates (words 8t + (s >> 1), 8t + 4 + (s >> 1)).
+          const uint4 ga = *reinterpret_cast<const uint4*>(&st.k2[g][8 * t]);
+          const uint4 gb = *reinterpret_cast<const uint4*>(&st.k2[g][8 * t + 4]);
+          const uint4 ha = *reinterpret_cast<const uint4*>(&st.k2[g + 8][8 * t]);
+          const uint4 hb = *reinterpret_cast<const uint4*>(&st.k2[g + 8][8 * t + 4]);
+#define TQ_K8STEP(S, W)                                                                           \
+  kstep(S, k8_pair<2 * ((S) & 1)>(klut_lane, ga.W), k8_pair<2 * ((S) & 1)>(klut_lane, ha.W),     \
+        k8_pair<2 * ((S) & 1)>(klut_lane, gb.W), k8_pair<2 * ((S) & 1)>(klut_lane, hb.W));
+          TQ_K8STEP(0, x) TQ_K8STEP(1, x) TQ_K8STEP(2, y) TQ_K8STEP(3, y)
+          TQ_K8STEP(4, z) TQ_K8STEP(5, z) TQ_K8STEP(6, w) TQ_K8STEP(7, w)
+#undef TQ_K8STEP
         } else {
           const uint4 wg = *reinterpret_cast<const uint4*>(&st.k2[g][4 * t]);
           const uint4 wh = *reinterpret_cast<const uint4*>(&st.k2[g + 8][4 * t]);
@@ -581,7 +615,7 @@ bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
   if (c->d != D || (a.G != 4 && a.G != 8)) return false;
   const bool k3q = c->bk_lm == 3 && c->qjl_m == 128 && c->bits_v == 4;
   const bool mse = c->qjl_m == 0 && ((c->bk_lm == 3 && (c->bits_v == 4 || c->bits_v == 3)) ||
-                                     (c->bk_lm == 4 && c->bits_v == 4));
+                                     ((c->bk_lm == 4 || c->bk_lm == 8) && c->bits_v == 4));
   if (!k3q && !mse) return false;
   if (a.max_T % 4 != 0) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.knorm) |
@@ -625,6 +659,8 @@ cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a_in, float* out, c
     lut_launch<4, false, 4>(a, nb, s);
   else if (!q && c->bk_lm == 3 && c->bits_v == 3)
     lut_launch<3, false, 3>(a, nb, s);
+  else if (!q && c->bk_lm == 8 && c->bits_v == 4)
+    lut_launch<8, false, 4>(a, nb, s);
   else
     return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
@@ -648,7 +684,8 @@ cudaError_t configure_attn_lut() {
   if ((e = lut_configure<3, true, 4>()) != cudaSuccess) return e;
   if ((e = lut_configure<3, false, 4>()) != cudaSuccess) return e;
   if ((e = lut_configure<4, false, 4>()) != cudaSuccess) return e;
-  return lut_configure<3, false, 3>();
+  if ((e = lut_configure<3, false, 3>()) != cudaSuccess) return e;
+  return lut_configure<8, false, 4>();
 }
 
 }  // namespace tqk

@@ -167,7 +167,10 @@ def test_attention_single_head(cuda):
     (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: tensor-core path, group 8
     (128, 8, 2, 4, 4, 128, 1000),   # 3-bit keys: tensor-core path, group 4
     (128, 8, 2, 4, 4, 128, 998),    # 3-bit keys, max_T % 4 != 0: generic path
-    (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000)])
+    (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000),
+    (128, 8, 2, 8, 4, 0, 1000),     # 8-bit keys (k8v4): tensor-core path, group 4
+    (128, 16, 2, 8, 4, 0, 998),     # 8-bit keys, max_T % 4 != 0: generic path
+    (256, 4, 2, 8, 8, 0, 300)])     # 8-bit keys and values at d = 256 (64 code words)
 def test_attention_ragged_outlier(cuda, d, Hq, Hkv, bk, bv, m, T):
     """Ragged lengths (0, 1, odd, chunk edges, full), GQA groups 1-8, d=64/128/200."""
     c = _ctx(d, bk, bv, m, seed=7)
@@ -560,6 +563,53 @@ def test_norm_corrected_variants(cuda, name, Hq):
                       outA.cpu().numpy())
 
 
+@pytest.mark.parametrize("Hq", [8, 16])
+def test_eight_bit_keys(cuda, Hq):
+    """k8v4: 8-bit Lloyd-Max keys (MSE only), 4-bit values.  Quantize through
+    the bulk and the small-batch kernels, logits, ragged decode and the fused
+    step against the oracle; top-k declines 8-bit keys."""
+    c = tq.Context.variant("k8v4", 128, seed=9)
+    assert c.key_layout["bits"] == 8 and c.key_layout["bytes_per_vector"] == 132
+    tab = P.oracle_tables(c)
+    B, Hkv, T, d = 3, 2, 700, 128
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=71)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=72)
+    kc, vc = _cache(c, K, V, cuda)
+    n = B * Hkv * T
+    P.check_quantized(tab, "k", P.to_np(K.reshape(n, d)), _flat(kc, n))
+    small = K[1, 1, :200].contiguous()
+    ks = c.quantize(small.to(cuda), tq.TQ_KEY)
+    P.check_quantized(tab, "k", P.to_np(small), _flat(ks, 200))
+    Q = tq_inputs.iid((B, Hq, d), seed=73, dtype=torch.bfloat16)
+    lg = c.logits(Q[0].to(cuda), ks)
+    torch.cuda.synchronize()
+    P.check_logits(tab, Q[0].double().numpy(), _flat(ks, 200), lg.cpu().double().numpy())
+    lens = torch.tensor([1, 333, T], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+    kB = {k: (None if v is None else v.clone()) for k, v in kc.items()}
+    vB = {k: (None if v is None else v.clone()) for k, v in vc.items()}
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=74)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=75)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([5, T - 1, 400], dtype=torch.int32, device=cuda)
+    q = Q.to(cuda)
+    outA = c.decode_step(q, kn, vn, kc, vc, pos)
+    c.quantize_append(kn, tq.TQ_KEY, kB, pos)
+    c.quantize_append(vn, tq.TQ_VALUE, vB, pos)
+    outB = c.attn_decode(q, kB, vB, (pos + 1).to(torch.int32))
+    torch.cuda.synchronize()
+    for a_, b_ in ((kc, kB), (vc, vB)):
+        for k in a_:
+            if a_[k] is not None:
+                assert torch.equal(a_[k], b_[k]), k
+    assert torch.equal(outA, outB)
+    with pytest.raises(tq.TQError) as e:
+        c.topk(Q[0].to(cuda), ks, 4)
+    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+
+
 # --- paged caches ---------------------------------------------------------------
 def _to_paged(cache, B, Hkv, max_T, bs, perm):
     """Scatter a contiguous [B, Hkv, max_T, ...] cache into blocks
@@ -582,7 +632,8 @@ def _to_paged(cache, B, Hkv, max_T, bs, perm):
 @pytest.mark.parametrize("Hq,Hkv,bk,bs,variant", [
     (8, 2, 3, 32, None), (16, 2, 3, 16, None), (16, 2, 4, 48, None), (4, 4, 3, 16, None),
     (8, 2, 4, 16, None), (8, 2, None, 32, "4bit_nc"), (16, 2, None, 16, "k3v4_nc"),
-    (8, 2, None, 16, "3bit_nc"), (16, 2, None, 48, "3bit_nc")])
+    (8, 2, None, 16, "3bit_nc"), (16, 2, None, 48, "3bit_nc"), (8, 2, None, 32, "k8v4"),
+    (16, 2, None, 16, "k8v4")])
 def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs, variant):
     """The paged decode reads the same records through the block table, so it
     must reproduce the contiguous decode bit for bit (ragged lengths,
