@@ -198,18 +198,20 @@ struct TopkPlan {
   int qb;                // queries per CTA (64 or 128)
   int64_t chunks, chunk; // database chunks, vectors per chunk
   int64_t qblocks;       // query blocks; work items = qblocks x chunks
-  int nlists;            // candidate lists per query (chunks x 4 warps)
-  size_t qh_bytes, qsc_bytes, cand_bytes, smem;
+  int nlists;            // candidate lists per query (chunks x 2 row groups)
+  size_t qh_bytes, qsc_bytes, cand_bytes, rows_bytes, smem;
 };
 TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k);
 // The same queries over the first n_sample database vectors (the bar pass).
 TopkPlan topk_mma_sample_plan(const TopkPlan& full, int64_t n_sample, int sms);
 cudaError_t launch_topk_qprep(const tq_ctx* c, const TopkPlan& p, const float* qr, const float* qs,
                               int64_t nq, void* qh, float* qsc, cudaStream_t s);
+// Dequantized database rows [n][KL + KQ] in fp16 (centroids | signs).
+cudaError_t launch_topk_dequant(const tq_ctx* c, const TopkPlan& p, const uint32_t* codes, const uint32_t* qjl,
+                                int64_t n, void* rows, cudaStream_t s);
 cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, const float* qsc, int64_t nq,
-                            const uint32_t* codes, const uint32_t* qjl, const float* norm,
-                            const float* rnorm, int64_t n, int k, const float* bar_v, const int* bar_i,
-                            float* cand_v, int* cand_i, cudaStream_t s);
+                            const void* rows, const float* norm, const float* rnorm, int64_t n, int k,
+                            const float* bar_v, const int* bar_i, float* cand_v, int* cand_i, cudaStream_t s);
 cudaError_t configure_topk_mma();
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,

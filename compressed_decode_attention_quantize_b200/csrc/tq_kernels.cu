@@ -1114,7 +1114,7 @@ size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   const TopkPlan p = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
   const TopkPlan ps = topk_mma_sample_plan(p, kTopkSample, c->sms);
   size_t b = 2 * up256((size_t)nq * c->dpad * sizeof(float));                 // q', s
-  b += up256(p.qh_bytes) + up256(p.qsc_bytes);
+  b += up256(p.qh_bytes) + up256(p.qsc_bytes) + up256(p.rows_bytes);
   b += 2 * up256((size_t)nq * p.nlists * k * sizeof(float));                  // candidates
   b += 2 * up256((size_t)nq * ps.nlists * k * sizeof(float));                 // sample candidates
   b += 2 * up256((size_t)nq * k * sizeof(float));                             // bars
@@ -1138,6 +1138,7 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   float* qs = reinterpret_cast<float*>(take((size_t)nq * c->dpad * sizeof(float)));
   void* qh = take(pl.qh_bytes);
   float* qsc = reinterpret_cast<float*>(take(pl.qsc_bytes));
+  void* rows = take(pl.rows_bytes);
   float* cv = reinterpret_cast<float*>(take((size_t)nq * pl.nlists * k * sizeof(float)));
   int* ci = reinterpret_cast<int*>(take((size_t)nq * pl.nlists * k * sizeof(int)));
   float* scv = reinterpret_cast<float*>(take((size_t)nq * ps.nlists * k * sizeof(float)));
@@ -1147,15 +1148,15 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   cudaError_t e = launch_prerotate(c, q, dtype, nq, nullptr, qr, qs, s);
   if (e != cudaSuccess) return e;
   if ((e = launch_topk_qprep(c, pl, qr, qs, nq, qh, qsc, s)) != cudaSuccess) return e;
+  if ((e = launch_topk_dequant(c, pl, codes, qjl, n, rows, s)) != cudaSuccess) return e;
   const bool two_pass = n >= 4 * kTopkSample;
   if (two_pass) {
-    e = launch_topk_mma(c, ps, qh, qsc, nq, codes, qjl, norm, rnorm, kTopkSample, k, nullptr, nullptr, scv,
-                        sci, s);
+    e = launch_topk_mma(c, ps, qh, qsc, nq, rows, norm, rnorm, kTopkSample, k, nullptr, nullptr, scv, sci, s);
     if (e != cudaSuccess) return e;
     k_topk_final<<<(unsigned)nq, 32, 0, s>>>(scv, sci, ps.nlists, k, bari, barv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  e = launch_topk_mma(c, pl, qh, qsc, nq, codes, qjl, norm, rnorm, n, k, two_pass ? barv : nullptr,
+  e = launch_topk_mma(c, pl, qh, qsc, nq, rows, norm, rnorm, n, k, two_pass ? barv : nullptr,
                       two_pass ? bari : nullptr, cv, ci, s);
   if (e != cudaSuccess) return e;
   k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, pl.nlists, k, idx, score);

@@ -5,16 +5,21 @@
 // and keeps the k best (score descending, then index ascending).
 //
 // The scores form a dense contraction of the queries with the dequantized
-// database: per 64-vector database tile the CTA expands the codes into fp16
-// rows [c[idx] (d, padded to 16) | sigma (m, padded to 16)] in shared memory,
-// and four warps multiply them with 64 queries ([q' 2^-e_q | S q' 2^-f_q] in
-// fp16, loaded once) with mma.sync m16n8k16, two fp32 accumulators (centroid
-// part, sign part).  fp16 rounding of q', S q' and the centroids moves a score
-// by ~1e-5 |q| |k|, far below the logit tolerance that separates
-// interchangeable near-ties.  Each warp keeps a top-k list per query in shared
-// memory; a score enters only if it beats the list's current worst, so after
-// the first tiles almost every score costs one comparison.  The lists of all
-// warps and database chunks are merged by k_topk_final.
+// database.  k_topk_dequant expands every vector's codes once into an fp16
+// row [c[idx] (d, padded to 16) | sigma (m, padded to 16)] in global memory
+// (a pair table maps two coordinates' indices to a half2 of centroids).
+// k_topk_gemm streams 32-row tiles of those rows through a three-stage
+// cp.async ring into shared memory and multiplies them with up to 128 queries
+// ([q' 2^-e_q | S q' 2^-f_q] in fp16, loaded once per work item) with
+// mma.sync m16n8k16 into two fp32 accumulators (centroid part, sign part);
+// n and sqrt(pi/2)/m gamma are applied per row in fp32.  Work items (query
+// block, database chunk) run chunk-major on a persistent grid, so the CTAs
+// in flight read the same few chunks and the rows come from L2.  fp16
+// rounding of q', S q' and the centroids moves a score by ~1e-5 |q| |k|, far
+// below the logit tolerance that separates interchangeable near-ties.  Each
+// warp keeps a top-k list per query in shared memory; a score enters only if
+// it beats the list's current worst.  The lists of all warps and chunks are
+// merged by k_topk_final.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -26,17 +31,23 @@
 namespace tqk {
 namespace {
 
-constexpr int TKR = 64;     // database vectors per tile
-constexpr int TKWARPS = 8;  // warp w: rows 16 (w & 3) .. +15, queries QB/2 (w >> 2) .. + QB/2 - 1
-constexpr int TKLISTS = 4;  // lists per query and chunk (the four row groups)
+constexpr int TKR = 32;     // database vectors per tile
+constexpr int TKWARPS = 8;  // warp w: rows 16 (w & 1) .. +15, queries QB/4 (w >> 1) .. + QB/4 - 1
+constexpr int TKLISTS = 2;  // lists per query and chunk (the two row groups)
+constexpr int TKST = 3;     // tile stages in flight
 
 __device__ __forceinline__ bool better_sc(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-__device__ __forceinline__ void cp4(void* dst, const void* src) {
+__device__ __forceinline__ void cp4(void* dst, const void* src, bool valid) {
   const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp16z(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -85,15 +96,13 @@ struct TopkMmaArgs {
   const __half* qh;
   const float* qsc;
   int64_t nq;
-  int d, bk, kw, m, qw, KL, KQ;
-  const float* ck;
+  int KL, KQ, m;
   float cq;   // sqrt(pi/2) / m
-  const uint32_t* codes;
-  const uint32_t* qjl;
+  const __half* rows;   // dequantized database [n][KL + KQ]
   const float* norm;
   const float* rnorm;
   int64_t n, chunk;   // database size, vectors per chunk (multiple of TKR)
-  int64_t chunks, qblocks;   // work items = qblocks x chunks, taken round-robin
+  int64_t chunks, qblocks;   // work items = chunks x qblocks, chunk-major
   int K, nlists;
   float* cand_v;
   int* cand_i;
@@ -103,84 +112,147 @@ struct TopkMmaArgs {
   const int* bar_i;
 };
 
-// Shared memory for QB queries per CTA: B rows [QB][KS] and A rows [TKR][KS]
-// in fp16 (KS = KL + KQ + 8: an odd number of 16-byte chunks per row, so
-// ldmatrix rows hit distinct banks), two staging buffers of the tile's codes,
-// signs and norms, query scales, the pair table (two coordinates' indices ->
-// half2 of centroids, up to 256 entries) and the per-warp lists
-// [TKWARPS][QB / 2][K] of (score, index).
-__host__ __device__ inline size_t topk_mma_smem(int QB, int KL, int KQ, int kw, int qw, int K) {
-  const size_t KS = (size_t)KL + KQ + 8;
-  return 2 * KS * (QB + TKR) + 2 * (size_t)TKR * (kw + qw + 2) * 4 + (size_t)QB * 2 * 4 + 256 * 4 +
-         (size_t)TKWARPS * (QB / 2) * K * 8 + 64;
+// Database rows: thread task (v, w) writes the half2 pairs of code word w of
+// vector v (w < W2), the +-1 halves of sign word w - W2 (w < W2 + qw), or
+// zeros for centroid columns past the code words (last task).
+template <int BK>
+__global__ void __launch_bounds__(256) k_topk_dequant(const uint32_t* codes, const uint32_t* qjl, int64_t n,
+                                                      int d, int kw, int qw, int m, int KL, int KQ,
+                                                      const float* ck, __half* rows) {
+  __shared__ uint32_t sP[256];
+  constexpr int per = BK == 3 ? 16 : 32 / BK;   // fields per word of the main stream
+  constexpr int fb = BK == 3 ? 2 : BK;          // bits per field of the main stream
+  constexpr int pairs_w = per / 2;
+  // Pair table: entry i -> half2(c[i0], c[i1]); for b = 3, i = f0 | f1 << 2 |
+  // t0 << 4 | t1 << 5 (fields, then top bits), else i = i0 | i1 << b.
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    int i0, i1;
+    if (BK == 3) {
+      i0 = (e & 3) | (((e >> 4) & 1) << 2);
+      i1 = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+    } else {
+      i0 = e & ((1 << BK) - 1);
+      i1 = (e >> BK) & ((1 << BK) - 1);
+    }
+    const bool ok = BK == 3 ? e < 64 : e < (1 << (2 * BK));
+    const __half2 hv = __floats2half2_rn(ok ? ck[i0] : 0.f, ok ? ck[i1] : 0.f);
+    sP[e] = *reinterpret_cast<const uint32_t*>(&hv);
+  }
+  __syncthreads();
+  const int W2 = (d + per - 1) / per;
+  const int tasks = W2 + qw + 1;
+  const int KP = KL + KQ;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * tasks;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t v = e / tasks;
+    const int wd = (int)(e - v * tasks);
+    uint32_t* row = reinterpret_cast<uint32_t*>(rows + v * KP);
+    if (wd < W2) {
+      const uint32_t w = codes[v * kw + wd];
+      uint32_t tw = 0u;
+      if (BK == 3) tw = codes[v * kw + W2 + (wd >> 1)] >> (16 * (wd & 1));
+#pragma unroll
+      for (int j = 0; j < pairs_w; ++j) {
+        const int c = per * wd + 2 * j;   // first coordinate of the pair
+        uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
+        if (BK == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
+        uint32_t h2 = sP[idx];
+        if (c >= d) h2 = 0u;
+        else if (c + 1 >= d) h2 &= 0xFFFFu;
+        if (c < KL) row[c / 2] = h2;
+      }
+    } else if (wd < W2 + qw) {
+      const int j0 = wd - W2;
+      const uint32_t bits = qjl[v * qw + j0];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = 32 * j0 + 2 * j;   // first sketch row of the pair
+        const uint32_t b2 = bits >> (2 * j);
+        // -1 (0xBC00) per half, +1 where the bit is set: flip the sign bit.
+        uint32_t h2 = 0xBC00BC00u ^ ((b2 & 1u) << 15) ^ ((b2 & 2u) << 30);
+        if (c >= m) h2 = 0u;
+        else if (c + 1 >= m) h2 &= 0xFFFFu;
+        if (c < KQ) row[(KL + c) / 2] = h2;
+      }
+    } else {
+      for (int c = per * W2; c < KL; c += 2) row[c / 2] = 0u;
+    }
+  }
 }
 
-template <int BK, int QB>
-__global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
-  constexpr int QH = QB / 2;     // queries per warp
+// Shared memory for QB queries per CTA: B rows [QB][KS] and TKST stages of A
+// rows [TKR][KS] in fp16 (KS = KL + KQ + 8: an odd number of 16-byte chunks
+// per row, so ldmatrix rows hit distinct banks), the stages' norms and
+// rnorms, query scales and the per-warp lists [TKWARPS][QB / 4][K] of
+// (score, index).
+__host__ __device__ inline size_t topk_mma_smem(int QB, int KL, int KQ, int K) {
+  const size_t KS = (size_t)KL + KQ + 8;
+  return 2 * KS * (QB + TKST * TKR) + (size_t)TKST * 2 * TKR * 4 + (size_t)QB * 2 * 4 +
+         (size_t)TKWARPS * (QB / 4) * K * 8 + 64;
+}
+
+template <int QB>
+__global__ void __launch_bounds__(TKWARPS * 32) k_topk_gemm(TopkMmaArgs a) {
+  constexpr int QH = QB / 4;     // queries per warp
   constexpr int NTW = QH / 8;    // n-tiles per warp
   constexpr int SL = 2 * NTW;    // (query) slots per thread
   extern __shared__ __align__(16) unsigned char smem[];
   const int KS = a.KL + a.KQ + 8;
+  const int KP = a.KL + a.KQ;
   __half* sB = reinterpret_cast<__half*>(smem);
-  __half* sA = sB + (size_t)QB * KS;
-  // Two staging buffers (tile i and i + 1): codes [TKR][kw], signs [TKR][qw],
-  // norms [TKR], rnorms [TKR].
-  const int stage_words = TKR * (a.kw + a.qw + 2);
-  uint32_t* sStage = reinterpret_cast<uint32_t*>(sA + (size_t)TKR * KS);
-  float* sQ = reinterpret_cast<float*>(sStage + 2 * stage_words);       // [QB][2]: 2^e, 2^f
-  uint32_t* sP = reinterpret_cast<uint32_t*>(sQ + QB * 2);               // [256] pair table
-  float* lv = reinterpret_cast<float*>(sP + 256);                        // [TKWARPS][QH][K]
+  __half* sA = sB + (size_t)QB * KS;                                          // [TKST][TKR][KS]
+  float* sN = reinterpret_cast<float*>(sA + (size_t)TKST * TKR * KS);         // [TKST][2][TKR]
+  float* sQ = sN + TKST * 2 * TKR;                                            // [QB][2]: 2^e, 2^f
+  float* lv = sQ + QB * 2;                                                    // [TKWARPS][QH][K]
   int* li = reinterpret_cast<int*>(lv + TKWARPS * QH * a.K);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int rg = warp & 3, qg = warp >> 2;   // row group, query half
-  const int KP = a.KL + a.KQ;
-  constexpr int bk = BK;
-  // Code words: main (b = 3: low-bit) stream of W2 words with `per` fields each.
-  constexpr int per = bk == 3 ? 16 : 32 / bk;
-  constexpr int fb = bk == 3 ? 2 : bk;       // bits per field in the main stream
-  constexpr int pairs_w = per / 2;           // coordinate pairs per word
-  const int W2 = (a.d + per - 1) / per;
-
-  // Pair table: entry i -> half2(c[i0], c[i1]); for b = 3, i = f0 | f1 << 2 |
-  // t0 << 4 | t1 << 5 (fields, then top bits), else i = i0 | i1 << b.
-  for (int e = tid; e < 256; e += TKWARPS * 32) {
-    int i0, i1;
-    if (bk == 3) {
-      i0 = (e & 3) | (((e >> 4) & 1) << 2);
-      i1 = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
-    } else {
-      i0 = e & ((1 << bk) - 1);
-      i1 = (e >> bk) & ((1 << bk) - 1);
-    }
-    const bool ok = bk == 3 ? e < 64 : e < (1 << (2 * bk));
-    const __half2 hv = __floats2half2_rn(ok ? a.ck[i0] : 0.f, ok ? a.ck[i1] : 0.f);
-    sP[e] = *reinterpret_cast<const uint32_t*>(&hv);
-  }
-  // Centroid columns past the code words (d < KL with < 16 fields per word):
-  // zero once, no tile writes them.
-  for (int e = tid; e < TKR * KS; e += TKWARPS * 32) sA[e] = __float2half_rn(0.f);
+  const int rg = warp & 1, qg = warp >> 1;   // row group, query quarter
 
   const uint32_t sA_s = (uint32_t)__cvta_generic_to_shared(sA);
   const uint32_t sB_s = (uint32_t)__cvta_generic_to_shared(sB);
+  const uint32_t stage_bytes = (uint32_t)(TKR * KS * 2);
   // ldmatrix row addresses: A tiles (rows 0-7 / 8-15) x (k 0-7 / 8-15);
-  // B tiles (n-tile nt / nt+1) x (k 0-7 / 8-15) of this warp's 32 queries.
+  // B tiles (n-tile nt / nt+1) x (k 0-7 / 8-15) of this warp's queries.
   const int ti = lane >> 3, tr = lane & 7;
-  const uint32_t a_row = sA_s + (uint32_t)((16 * rg + tr + 8 * (ti & 1)) * KS + 8 * (ti >> 1)) * 2;
+  const uint32_t a_row0 = sA_s + (uint32_t)((16 * rg + tr + 8 * (ti & 1)) * KS + 8 * (ti >> 1)) * 2;
   const uint32_t b_row = sB_s + (uint32_t)((QH * qg + 8 * (ti >> 1) + tr) * KS + 8 * (ti & 1)) * 2;
   float* mylv = lv + warp * QH * a.K;
   int* myli = li + warp * QH * a.K;
+  const int c16 = KP / 8;   // 16-byte chunks per row
 
-  // Persistent CTAs: item = (query block, database chunk).
+  // Persistent CTAs: item = (database chunk, query block), chunk-major.
   const int64_t nitems = a.qblocks * a.chunks;
   for (int64_t item = blockIdx.x; item < nitems; item += gridDim.x) {
-  const int64_t q0 = (item / a.chunks) * QB;
-  const int64_t chunk_id = item % a.chunks;
+  const int64_t q0 = (item % a.qblocks) * QB;
+  const int64_t chunk_id = item / a.qblocks;
   const int64_t n0 = chunk_id * a.chunk;
   const int64_t n1 = min(a.n, n0 + a.chunk);
-  __syncthreads();   // the previous item's readers of sB, sQ and the lists are done
+  const int ntile = (int)((n1 - n0 + TKR - 1) / TKR);
+  __syncthreads();   // the previous item's readers of sB, sA, sQ and the lists are done
+
+  // Tile i of the chunk into stage st: its rows (zero past n1), norms, rnorms.
+  auto stage = [&](int i, int st) {
+    const int64_t v0 = n0 + (int64_t)i * TKR;
+    const uint32_t dst = sA_s + st * stage_bytes;
+    for (int e = tid; e < TKR * c16; e += TKWARPS * 32) {
+      const int r = e / c16, c = e - r * c16;
+      const bool ok = v0 + r < n1;
+      cp16z(dst + (uint32_t)(r * KS + 8 * c) * 2, a.rows + (ok ? (v0 + r) * KP + 8 * c : 0), ok);
+    }
+    if (tid < 2 * TKR) {
+      const int r = tid & (TKR - 1);
+      const bool ok = v0 + r < n1 && (tid < TKR || a.m > 0);
+      const float* src = tid < TKR ? a.norm : a.rnorm;
+      cp4(sN + st * 2 * TKR + tid, ok ? src + v0 + r : a.norm, ok);
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < TKST - 1; ++i) {
+    if (i < ntile) stage(i, i);
+    asm volatile("cp.async.commit_group;\n" ::);
+  }
   for (int e = tid; e < QB * KP / 8; e += TKWARPS * 32) {
     const int r = e / (KP / 8), c8 = e % (KP / 8);
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -203,7 +275,7 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
   };
   for (int e = tid; e < TKWARPS * QH * a.K; e += TKWARPS * 32) {
     const int ql = (e / a.K) % QH, w = e / (QH * a.K);
-    bar(q0 + QH * (w >> 2) + ql, lv[e], li[e]);
+    bar(q0 + QH * (w >> 1) + ql, lv[e], li[e]);
   }
   __syncthreads();
   // This thread's SL queries (NTW n-tiles x 2 columns): scales and the current
@@ -218,77 +290,16 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
     bar(q0 + ql, wv[s], wi[s]);
   }
 
-  // Copy tile v0's codes, signs and norms (contiguous in memory) into staging
-  // buffer buf with 4-byte cp.async: in flight while the previous tile is
-  // scored.
-  auto stage = [&](int64_t v0, int buf) {
+  for (int i = 0; i < ntile; ++i) {
+    const int64_t v0 = n0 + (int64_t)i * TKR;
     const int rows = (int)min((int64_t)TKR, n1 - v0);
-    uint32_t* dC = sStage + buf * stage_words;
-    uint32_t* dS = dC + TKR * a.kw;
-    uint32_t* dN = dS + TKR * a.qw;
-    for (int e = tid; e < rows * a.kw; e += TKWARPS * 32) cp4(dC + e, a.codes + v0 * a.kw + e);
-    for (int e = tid; e < rows * a.qw; e += TKWARPS * 32) cp4(dS + e, a.qjl + v0 * a.qw + e);
-    for (int e = tid; e < rows; e += TKWARPS * 32) {
-      cp4(dN + e, a.norm + v0 + e);
-      if (a.m > 0) cp4(dN + TKR + e, a.rnorm + v0 + e);
-    }
+    const int st = i % TKST;
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(TKST - 2) : "memory");
+    __syncthreads();   // tile i landed; every warp is done with tile i - 1's stage
+    if (i + TKST - 1 < ntile) stage(i + TKST - 1, (i + TKST - 1) % TKST);
     asm volatile("cp.async.commit_group;\n" ::);
-  };
-  if (n0 < n1) stage(n0, 0);
-  int buf = 0;
-  for (int64_t v0 = n0; v0 < n1; v0 += TKR, buf ^= 1) {
-    const int rows = (int)min((int64_t)TKR, n1 - v0);
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-    __syncthreads();   // tile v0 staged; the other buffer is free
-    if (v0 + TKR < n1) stage(v0 + TKR, buf ^ 1);
-    const uint32_t* sC = sStage + buf * stage_words;
-    const uint32_t* sS = sC + TKR * a.kw;
-    const float* sNn = reinterpret_cast<const float*>(sS + TKR * a.qw);   // norms, then rnorms
-    // ---- dequantize: thread -> row tid % 64, code words tid / 64, +4, ... -----------
-    {
-      const int r = tid & (TKR - 1);
-      const bool live = r < rows;
-      for (int wd = tid >> 6; wd < W2; wd += TKWARPS * 32 / TKR) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(sA + (size_t)r * KS) + wd * pairs_w;
-        const uint32_t w = live ? sC[r * a.kw + wd] : 0u;
-        uint32_t tw = 0u;
-        if (bk == 3 && live) tw = sC[r * a.kw + W2 + (wd >> 1)] >> (16 * (wd & 1));
-        if (live && per * (wd + 1) <= a.d) {   // every coordinate of the word is real
-#pragma unroll
-          for (int j = 0; j < pairs_w; ++j) {
-            uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
-            if (bk == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
-            dst[j] = sP[idx];
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < pairs_w; ++j) {
-            const int c = per * wd + 2 * j;   // first coordinate of the pair
-            uint32_t idx = (w >> (2 * fb * j)) & ((1u << (2 * fb)) - 1u);
-            if (bk == 3) idx |= ((tw >> (2 * j)) & 3u) << 4;
-            uint32_t h2 = sP[idx];
-            if (!live || c >= a.d) h2 = 0u;
-            else if (c + 1 >= a.d) h2 &= 0xFFFFu;
-            if (c < a.KL) dst[j] = h2;
-          }
-        }
-      }
-      for (int wd = tid >> 6; wd < a.qw; wd += TKWARPS * 32 / TKR) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(sA + (size_t)r * KS + a.KL) + wd * 16;
-        const uint32_t bits = live ? sS[r * a.qw + wd] : 0u;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int c = 32 * wd + 2 * j;   // first sketch row of the pair
-          const uint32_t b2 = bits >> (2 * j);
-          // -1 (0xBC00) per half, +1 where the bit is set: flip the sign bit.
-          uint32_t h2 = 0xBC00BC00u ^ ((b2 & 1u) << 15) ^ ((b2 & 2u) << 30);
-          if (!live || c >= a.m) h2 = 0u;
-          else if (c + 1 >= a.m) h2 &= 0xFFFFu;
-          if (c < a.KQ) dst[j] = h2;
-        }
-      }
-    }
-    __syncthreads();
+    const float* sNn = sN + st * 2 * TKR;   // norms, then rnorms
+    const uint32_t a_row = a_row0 + st * stage_bytes;
 
     // ---- scores of rows 16 rg .. +15 against queries QH qg .. + QH - 1 -------------------
     float acc[NTW][4], acs[NTW][4];
@@ -386,7 +397,6 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_mma(TopkMmaArgs a) {
       }
       __syncwarp();
     }
-    __syncthreads();   // the next tile overwrites sA
   }
   asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 
@@ -410,17 +420,15 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   TopkPlan p{};
   p.KL = (c->d + 15) / 16 * 16;
   p.KQ = (c->qjl_m + 15) / 16 * 16;
-  const int qw = (c->qjl_m + 31) / 32;
-  // 128 queries per CTA (more products per dequantized tile) when it fits.
-  p.qb = topk_mma_smem(128, p.KL, p.KQ, c->wk, qw, k) <= (size_t)227 * 1024 ? 128 : 64;
+  // 128 queries per CTA (more products per staged tile) when it fits.
+  p.qb = topk_mma_smem(128, p.KL, p.KQ, k) <= (size_t)227 * 1024 ? 128 : 64;
   const int64_t qblocks = (nq + p.qb - 1) / p.qb;
-  // About sixteen (query block, chunk) items per SM for the persistent grid.
+  // About sixteen (chunk, query block) items per SM for the persistent grid.
   int64_t chunks = (16 * (int64_t)c->sms + qblocks - 1) / (qblocks > 0 ? qblocks : 1);
   const int64_t max_chunks = (n + 8 * TKR - 1) / (8 * TKR);   // at least eight tiles per chunk
   if (chunks > max_chunks) chunks = max_chunks;
   if (chunks < 1) chunks = 1;
   if (chunks > 65535) chunks = 65535;
-  p.chunks = chunks;
   p.chunk = ((n + chunks - 1) / chunks + TKR - 1) / TKR * TKR;
   p.chunks = (n + p.chunk - 1) / p.chunk;   // no empty chunk after rounding
   p.qblocks = qblocks;
@@ -428,7 +436,8 @@ TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k) {
   p.qh_bytes = (size_t)nq * (p.KL + p.KQ) * sizeof(__half);
   p.qsc_bytes = (size_t)nq * 2 * sizeof(float);
   p.cand_bytes = (size_t)nq * p.nlists * k * (sizeof(float) + sizeof(int));
-  p.smem = topk_mma_smem(p.qb, p.KL, p.KQ, c->wk, qw, k);
+  p.rows_bytes = (size_t)n * (p.KL + p.KQ) * sizeof(__half);
+  p.smem = topk_mma_smem(p.qb, p.KL, p.KQ, k);
   return p;
 }
 
@@ -451,25 +460,38 @@ cudaError_t launch_topk_qprep(const tq_ctx* c, const TopkPlan& p, const float* q
   return cudaGetLastError();
 }
 
+cudaError_t launch_topk_dequant(const tq_ctx* c, const TopkPlan& p, const uint32_t* codes, const uint32_t* qjl,
+                                int64_t n, void* rows, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int qw = (c->qjl_m + 31) / 32;
+  const int per = c->bk_lm == 3 ? 16 : 32 / c->bk_lm;
+  const int64_t tasks = n * ((c->d + per - 1) / per + qw + 1);
+  int64_t blocks = (tasks + 255) / 256;
+  blocks = blocks > (int64_t)c->sms * 16 ? (int64_t)c->sms * 16 : blocks;
+  __half* r = static_cast<__half*>(rows);
+  const int qwv = qw;
+  switch (c->bk_lm) {
+    case 1: k_topk_dequant<1><<<(unsigned)blocks, 256, 0, s>>>(codes, qjl, n, c->d, c->wk, qwv, c->qjl_m, p.KL, p.KQ, c->ck_f, r); break;
+    case 2: k_topk_dequant<2><<<(unsigned)blocks, 256, 0, s>>>(codes, qjl, n, c->d, c->wk, qwv, c->qjl_m, p.KL, p.KQ, c->ck_f, r); break;
+    case 3: k_topk_dequant<3><<<(unsigned)blocks, 256, 0, s>>>(codes, qjl, n, c->d, c->wk, qwv, c->qjl_m, p.KL, p.KQ, c->ck_f, r); break;
+    case 4: k_topk_dequant<4><<<(unsigned)blocks, 256, 0, s>>>(codes, qjl, n, c->d, c->wk, qwv, c->qjl_m, p.KL, p.KQ, c->ck_f, r); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, const float* qsc, int64_t nq,
-                            const uint32_t* codes, const uint32_t* qjl, const float* norm,
-                            const float* rnorm, int64_t n, int k, const float* bar_v, const int* bar_i,
-                            float* cand_v, int* cand_i, cudaStream_t s) {
+                            const void* rows, const float* norm, const float* rnorm, int64_t n, int k,
+                            const float* bar_v, const int* bar_i, float* cand_v, int* cand_i, cudaStream_t s) {
   TopkMmaArgs a{};
   a.qh = static_cast<const __half*>(qh);
   a.qsc = qsc;
   a.nq = nq;
-  a.d = c->d;
-  a.bk = c->bk_lm;
-  a.kw = c->wk;
-  a.m = c->qjl_m;
-  a.qw = (c->qjl_m + 31) / 32;
   a.KL = p.KL;
   a.KQ = p.KQ;
-  a.ck = c->ck_f;
+  a.m = c->qjl_m;
   a.cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
-  a.codes = codes;
-  a.qjl = qjl;
+  a.rows = static_cast<const __half*>(rows);
   a.norm = norm;
   a.rnorm = rnorm;
   a.n = n;
@@ -484,18 +506,10 @@ cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, 
   a.bar_i = bar_i;
   const int64_t items = p.qblocks * p.chunks;
   const unsigned grid = (unsigned)(items < c->sms ? items : c->sms);   // one CTA per SM
-  const bool wide = p.qb == 128;
-  switch (c->bk_lm * 2 + (wide ? 1 : 0)) {
-    case 2: k_topk_mma<1, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 3: k_topk_mma<1, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 4: k_topk_mma<2, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 5: k_topk_mma<2, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 6: k_topk_mma<3, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 7: k_topk_mma<3, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 8: k_topk_mma<4, 64><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    case 9: k_topk_mma<4, 128><<<grid, TKWARPS * 32, p.smem, s>>>(a); break;
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.qb == 128)
+    k_topk_gemm<128><<<grid, TKWARPS * 32, p.smem, s>>>(a);
+  else
+    k_topk_gemm<64><<<grid, TKWARPS * 32, p.smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -503,14 +517,8 @@ cudaError_t configure_topk_mma() {
   const int lim = 227 * 1024;   // the plan never asks for more
   const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<1, 64>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<1, 128>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<2, 64>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<2, 128>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<3, 64>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<3, 128>, ms, lim))) return e;
-  if ((e = cudaFuncSetAttribute(k_topk_mma<4, 64>, ms, lim))) return e;
-  return cudaFuncSetAttribute(k_topk_mma<4, 128>, ms, lim);
+  if ((e = cudaFuncSetAttribute(k_topk_gemm<64>, ms, lim))) return e;
+  return cudaFuncSetAttribute(k_topk_gemm<128>, ms, lim);
 }
 
 }  // namespace tqk
