@@ -73,8 +73,11 @@ const char* tq_version(void) { return "libtq 0.1 (sm_100a)"; }
 
 int tq_device_fault(int* code) {
   if (!code) return fail(TQ_ERR_ARG, "tq_device_fault: null output");
-  cudaError_t e = tqk::read_and_clear_fault(code);
+  int q = 0, t = 0;
+  cudaError_t e = tqk::read_and_clear_fault(&q);
+  if (e == cudaSuccess) e = tqk::read_and_clear_topk_fault(&t);
   if (e != cudaSuccess) return cuda_fail(e, "tq_device_fault");
+  *code = q | (t << 1);
   return TQ_OK;
 }
 

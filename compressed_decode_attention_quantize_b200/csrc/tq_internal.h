@@ -200,6 +200,8 @@ struct TopkPlan {
   int64_t qblocks;       // query blocks; work items = qblocks x chunks
   int nlists;            // candidate lists per query (chunks x 2 row groups)
   size_t qh_bytes, qsc_bytes, cand_bytes, rows_bytes, smem;
+  int nkb = 0, stages = 0;   // tensor-core scorer: K blocks of 64, shared-memory stages
+  bool use_tc = false;       // the tcgen05 scorer fits (else the mma.sync one)
 };
 TopkPlan topk_mma_plan(const tq_ctx* c, int64_t nq, int64_t n, int k);
 // The same queries over the first n_sample database vectors (the bar pass).
@@ -213,6 +215,14 @@ cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, 
                             const void* rows, const float* norm, const float* rnorm, int64_t n, int k,
                             const float* bar_v, const int* bar_i, float* cand_v, int* cand_i, cudaStream_t s);
 cudaError_t configure_topk_mma();
+// The tcgen05 scorer (128 queries per item, TMA-fed, TMEM accumulators).
+// n_sample > 0 plans the bar pass over the first n_sample vectors.
+TopkPlan topk_tc_plan(const tq_ctx* c, int64_t nq, int64_t n, int k, int64_t n_sample);
+cudaError_t launch_topk_tc(const tq_ctx* c, const TopkPlan& p, const void* qh, const float* qsc, int64_t nq,
+                           const void* rows, const float* norm, const float* rnorm, int64_t n, int k,
+                           const float* bar_v, const int* bar_i, float* cand_v, int* cand_i, cudaStream_t s);
+cudaError_t configure_topk_tc();
+cudaError_t read_and_clear_topk_fault(int* value);
 cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                           const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
                           const float* krnorm, int64_t nk, float* out, cudaStream_t s);

@@ -1110,9 +1110,20 @@ constexpr int64_t kTopkSample = 32768;
 
 static size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// The plans of both passes: the tcgen05 scorer when it fits, else mma.sync.
+static void topk_plans(const tq_ctx* c, int64_t nq, int64_t n, int k, TopkPlan& p, TopkPlan& ps) {
+  p = topk_tc_plan(c, nq, n > 0 ? n : 1, k, 0);
+  if (p.use_tc) {
+    ps = topk_tc_plan(c, nq, n > 0 ? n : 1, k, kTopkSample);
+  } else {
+    p = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
+    ps = topk_mma_sample_plan(p, kTopkSample, c->sms);
+  }
+}
+
 size_t topk_workspace(const tq_ctx* c, int64_t nq, int64_t n, int k) {
-  const TopkPlan p = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
-  const TopkPlan ps = topk_mma_sample_plan(p, kTopkSample, c->sms);
+  TopkPlan p, ps;
+  topk_plans(c, nq, n, k, p, ps);
   size_t b = 2 * up256((size_t)nq * c->dpad * sizeof(float));                 // q', s
   b += up256(p.qh_bytes) + up256(p.qsc_bytes) + up256(p.rows_bytes);
   b += 2 * up256((size_t)nq * p.nlists * k * sizeof(float));                  // candidates
@@ -1126,8 +1137,9 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
                         const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
                         void* ws, cudaStream_t s) {
   if (nq == 0) return cudaSuccess;
-  const TopkPlan pl = topk_mma_plan(c, nq, n > 0 ? n : 1, k);
-  const TopkPlan ps = topk_mma_sample_plan(pl, kTopkSample, c->sms);
+  TopkPlan pl, ps;
+  topk_plans(c, nq, n, k, pl, ps);
+  auto score_pass = pl.use_tc ? launch_topk_tc : launch_topk_mma;
   char* p = static_cast<char*>(ws);
   auto take = [&](size_t bytes) {
     char* r = p;
@@ -1151,12 +1163,12 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   if ((e = launch_topk_dequant(c, pl, codes, qjl, n, rows, s)) != cudaSuccess) return e;
   const bool two_pass = n >= 4 * kTopkSample;
   if (two_pass) {
-    e = launch_topk_mma(c, ps, qh, qsc, nq, rows, norm, rnorm, kTopkSample, k, nullptr, nullptr, scv, sci, s);
+    e = score_pass(c, ps, qh, qsc, nq, rows, norm, rnorm, kTopkSample, k, nullptr, nullptr, scv, sci, s);
     if (e != cudaSuccess) return e;
     k_topk_final<<<(unsigned)nq, 32, 0, s>>>(scv, sci, ps.nlists, k, bari, barv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  e = launch_topk_mma(c, pl, qh, qsc, nq, rows, norm, rnorm, n, k, two_pass ? barv : nullptr,
+  e = score_pass(c, pl, qh, qsc, nq, rows, norm, rnorm, n, k, two_pass ? barv : nullptr,
                       two_pass ? bari : nullptr, cv, ci, s);
   if (e != cudaSuccess) return e;
   k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, pl.nlists, k, idx, score);
@@ -1196,6 +1208,7 @@ cudaError_t configure_kernels() {
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   if ((e = configure_attn_lut()) != cudaSuccess) return e;
   if ((e = configure_topk_mma()) != cudaSuccess) return e;
+  if ((e = configure_topk_tc()) != cudaSuccess) return e;
   return configure_attn_mma();
 }
 

@@ -98,8 +98,9 @@ const char* tq_version(void);
 /*
  * tq_device_fault - synchronising diagnostic: reads and clears the device
  * fault code that kernels set when a bounded wait on the tensor cores gives
- * up (0 = none).  The kernel that set it has released its resources and
- * returned; its outputs for the affected tiles are undefined.
+ * up: 0 = none, bit 0 = quantize, bit 1 = top-k scorer.  The kernel that set
+ * it has released its resources and returned; its outputs for the affected
+ * tiles are undefined.
  */
 int tq_device_fault(int* code);
 
