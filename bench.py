@@ -97,6 +97,22 @@ def recorded_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(vals, world: int, device):
+    """Element-wise max of vals over all ranks: the slowest rank sets the
+    job's time.  One all-reduce on the process group when world > 1."""
+    import torch
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units all ranks processed per second, over the max-over-ranks time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def kv_bytes(w, ctx) -> int:
     kb = ctx.key_layout["bytes_per_vector"]
     vb = ctx.value_layout["bytes_per_vector"]
@@ -587,23 +603,19 @@ def run_gpu(args, w):
         small = small_case(tq, tq_inputs, torch, dev)
         variants = variant_decode(tq, tq_inputs, torch, dev, hbm_peak, WORKLOADS["llama3-8b-decode"])
 
-    tm = torch.tensor([t_ms, attn_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-    t_ms, attn_ms, e2e_ms = tm.tolist()
+    t_ms, attn_ms, e2e_ms = max_over_ranks([t_ms, attn_ms, e2e_ms], world, dev)
 
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline_from_device(w, ctx, kc, vc, qs[0])
 
     if rank == 0:
-        tokens = world * B * T
         kvb = kv_bytes(w, ctx)
         alg = kvb + B * Hq * d * 2 + B * Hq * d * 4  # packed cache + bf16 queries + fp32 output
         achieved = alg / (attn_ms / 1e3) / 1e9
         traffic = recorded_traffic(args.workload)
         line = {
-            "metric": METRIC, "value": tokens / (t_ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": whole_job_rate(B * T, world, t_ms), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_of(args, w),
@@ -614,7 +626,7 @@ def run_gpu(args, w):
                          "algorithmic_bytes_per_launch": alg, "launch_ms": attn_ms,
                          "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                          "frac_of_nominal_8tbs": achieved / 8000.0},
-            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_rate(B * T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
