@@ -17,8 +17,9 @@
 //  - the accumulators are double-buffered, so sixteen epilogue warps read the
 //    scores of tile i (tcgen05.ld; warp w: rows 32 (w & 3).., queries
 //    32 (w >> 2)..) while the tensor cores compute tile i + 1;
-//  - each (row quarter, query) keeps a top-k list in shared memory; a score
-//    enters only if it beats the list's worst entry (the bar).
+//  - each (row quarter, query) keeps a top-k list (k <= 12) in the registers
+//    of one lane; a score enters only if it beats the list's worst entry
+//    (the bar, kept in a shared-memory column record).
 // Work items (database chunk, query block) run chunk-major on a persistent
 // grid, so the CTAs in flight read the same chunks from L2.  Every mbarrier
 // wait is bounded; on expiry the kernel records a fault, drains its copies
@@ -45,6 +46,7 @@ constexpr uint32_t BLK = 128 * 128;         // one 64-wide K block of 128 rows (
 constexpr int EPI_WARPS = 16;               // warp w: rows 32 (w & 3).., queries 32 (w >> 2)..
 constexpr int TC_THREADS = (EPI_WARPS + 2) * 32;   // + producer warp + MMA warp
 constexpr int TC_LISTS = 4;                 // lists per query and chunk (row quarters)
+constexpr int TC_KMAX = 12;                 // largest k kept in registers
 constexpr uint32_t IDESC_TK = tc_idesc_f16(TC_Q);
 
 struct TopkTcArgs {
@@ -75,6 +77,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 16 fp32 columns [col, col+16) of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Shared memory above the 1024-byte aligned base: query K blocks, A stages,
 // then barriers, the TMEM address, query scales, bars and lists.
 struct TcLayout {
@@ -87,12 +102,13 @@ __host__ __device__ inline TcLayout tc_layout(int nkb, int stages, int K) {
   L.bar_off = L.a_off + (uint32_t)stages * BLK;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2], bfull, done; then tmem slot
   L.misc_off = L.bar_off + (uint32_t)(2 * stages + 6) * 8 + 16;
-  const uint32_t misc = EPI_WARPS * 32 * 16 + (uint32_t)TC_LISTS * TC_Q * K * 8;
+  const uint32_t misc = EPI_WARPS * 32 * 16;
+  (void)K;
   L.total = L.misc_off + misc + 1024;   // + alignment slack
   return L;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __maxnreg__(96)
     k_topk_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TopkTcArgs a) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
@@ -107,7 +123,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + LY.bar_off + (2 * S + 6) * 8);
   // Per epilogue warp and column: (2^e, 2^f, bar score, bar index bits).
   float4* sCol = reinterpret_cast<float4*>(base + LY.misc_off);        // [EPI_WARPS][32]
-  float* lv = reinterpret_cast<float*>(sCol + EPI_WARPS * 32);         // [TC_LISTS][TC_Q][K]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == EPI_WARPS * 32) {
@@ -242,8 +257,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __syncwarp();
   } else {
     // ---- epilogue warps -------------------------------------------------------------
-    // Warp w owns the lists of (row quarter w & 3, queries 32 (w >> 2) .. + 31)
-    // and the column records of those queries: no barrier between warps.
+    // Warp w owns the lists of (row quarter w & 3, queries 32 (w >> 2) .. + 31):
+    // lane l keeps the list of query 32 (w >> 2) + l in registers, and the
+    // column records of those queries sit in shared memory (read by all
+    // lanes, written by the owner).  No barrier between warps.
     const int rq = warp & 3, qc = warp >> 2;
     float4* col = sCol + warp * 32;
     uint32_t tcount = 0;
@@ -253,27 +270,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int64_t n0 = chunk_id * a.chunk;
       const int64_t n1 = min(a.n, n0 + a.chunk);
       const int ntile = (int)((n1 - n0 + TC_ROWS - 1) / TC_ROWS);
-      __syncwarp();   // the previous item's lists are written out
+      // This lane's list starts at its query's bar (the k-th best of a
+      // sample bounds the final k-th best from below).
+      const int64_t myq = q0 + 32 * qc + lane;
+      float lv[TC_KMAX];
+      int li[TC_KMAX];
       {
-        // Lists start at the query's bar (the k-th best of a sample bounds
-        // the final k-th best from below).
-        const int64_t q = q0 + 32 * qc + lane;
         float v = -INFINITY;
         int ix = INT_MAX;
-        if (a.bar_v && q < a.nq && a.bar_i[q * a.K + a.K - 1] >= 0) {
-          v = a.bar_v[q * a.K + a.K - 1];
-          ix = a.bar_i[q * a.K + a.K - 1];
+        if (a.bar_v && myq < a.nq && a.bar_i[myq * a.K + a.K - 1] >= 0) {
+          v = a.bar_v[myq * a.K + a.K - 1];
+          ix = a.bar_i[myq * a.K + a.K - 1];
         }
-        const bool in = q < a.nq;
-        col[lane] = make_float4(in ? a.qsc[2 * q] : 0.f, in ? a.qsc[2 * q + 1] : 0.f, v, __int_as_float(ix));
-        float* L = lv + (rq * TC_Q + 32 * qc + lane) * a.K;
-        int* I = reinterpret_cast<int*>(lv + TC_LISTS * TC_Q * a.K) + (rq * TC_Q + 32 * qc + lane) * a.K;
-        for (int r = 0; r < a.K; ++r) {
-          L[r] = v;
-          I[r] = ix;
+#pragma unroll
+        for (int r = 0; r < TC_KMAX; ++r) {
+          lv[r] = v;
+          li[r] = ix;
         }
+        const bool in = myq < a.nq;
+        __syncwarp();   // every lane is done with the previous item's records
+        col[lane] = make_float4(in ? a.qsc[2 * myq] : 0.f, in ? a.qsc[2 * myq + 1] : 0.f, v, __int_as_float(ix));
+        __syncwarp();
       }
-      __syncwarp();
       // Row norms one tile ahead.
       auto norms = [&](int t, float& nv, float& gv) {
         const int64_t v = n0 + (int64_t)t * TC_ROWS + 32 * rq + lane;
@@ -295,35 +313,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         tc_after_sync();
         const uint32_t t_lm = tmem + ((uint32_t)(32 * rq) << 16) + ab * 256 + 32 * qc;
-        float dl[32], dq[32];
-        tmem_ld32(t_lm, dl);
-        if (a.m > 0) {
-          tmem_ld32(t_lm + 128, dq);
-        } else {
+        // Scores of the 32 columns in two halves of 16 (fewer live registers)
+        // and this lane's candidate bits: one 16-byte column record and one
+        // comparison per score.
+        float sc[32];
+        uint32_t cm = 0u;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) dq[i] = 0.f;
+        for (int hf = 0; hf < 2; ++hf) {
+          float dq[16];
+          float* dl = sc + 16 * hf;
+          tmem_ld16(t_lm + 16 * hf, dl);
+          if (a.m > 0) {
+            tmem_ld16(t_lm + 128 + 16 * hf, dq);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dq[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float4 ci = col[16 * hf + i];
+            dl[i] = valid ? fmaf(nv * ci.x, dl[i], gv * ci.y * dq[i]) : -INFINITY;
+            if (valid && better_tc(dl[i], (int)v, ci.z, __float_as_int(ci.w))) cm |= 1u << (16 * hf + i);
+          }
         }
         tc_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_acce + 8 * ab);   // the scores are in registers
         ++tcount;
-        // Scores of the 32 columns and this lane's candidate bits (straight-
-        // line code: one 16-byte column record and one comparison per score).
-        float sc[32];
-        uint32_t cm = 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float4 ci = col[i];
-          sc[i] = valid ? fmaf(nv * ci.x, dl[i], gv * ci.y * dq[i]) : -INFINITY;
-          if (valid && better_tc(sc[i], (int)v, ci.z, __float_as_int(ci.w))) cm |= 1u << i;
-        }
-        // Rare once the bars are up: insert column by column, lane 0
-        // updating the list, every lane re-checking against the new bar.
+        // Rare once the bars are up: insert column by column; the lane that
+        // owns the column's list updates it and its record, every lane
+        // re-checks against the new bar.
         uint32_t cols = __reduce_or_sync(0xffffffffu, cm);
         while (cols) {
           const int i = __ffs(cols) - 1;
           cols &= cols - 1u;
-          const int lq = rq * TC_Q + 32 * qc + i;
           float mine = 0.f;
 #pragma unroll
           for (int k = 0; k < 32; ++k)
@@ -334,21 +357,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int leader = __ffs(mask) - 1;
             const float val = __shfl_sync(0xffffffffu, mine, leader);
             const int idx = __shfl_sync(0xffffffffu, (int)v, leader);
-            if (lane == 0) {
-              float* L = lv + lq * a.K;
-              int* I = reinterpret_cast<int*>(lv + TC_LISTS * TC_Q * a.K) + lq * a.K;
+            if (lane == i) {
+              // Replace the worst entry, then find the new worst (the bar).
               int wpos = 0;
-              for (int e = 1; e < a.K; ++e)
-                if (better_tc(L[wpos], I[wpos], L[e], I[e])) wpos = e;
-              if (better_tc(val, idx, L[wpos], I[wpos])) {
-                L[wpos] = val;
-                I[wpos] = idx;
-                wpos = 0;
-                for (int e = 1; e < a.K; ++e)
-                  if (better_tc(L[wpos], I[wpos], L[e], I[e])) wpos = e;
+              float wv = lv[0];
+              int wi = li[0];
+#pragma unroll
+              for (int r = 1; r < TC_KMAX; ++r)
+                if (r < a.K && better_tc(wv, wi, lv[r], li[r])) {
+                  wpos = r;
+                  wv = lv[r];
+                  wi = li[r];
+                }
+              if (better_tc(val, idx, wv, wi)) {
+#pragma unroll
+                for (int r = 0; r < TC_KMAX; ++r)
+                  if (r == wpos) {
+                    lv[r] = val;
+                    li[r] = idx;
+                  }
+                wv = lv[0];
+                wi = li[0];
+#pragma unroll
+                for (int r = 1; r < TC_KMAX; ++r)
+                  if (r < a.K && better_tc(wv, wi, lv[r], li[r])) {
+                    wv = lv[r];
+                    wi = li[r];
+                  }
               }
-              col[i].z = L[wpos];
-              col[i].w = __int_as_float(I[wpos]);
+              col[i].z = wv;
+              col[i].w = __int_as_float(wi);
             }
             __syncwarp();
             if (lane == leader) cand = false;
@@ -359,17 +397,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       if (fault) break;
-      // This warp's lists -> candidates of (query, chunk, row quarter).
-      __syncwarp();
-      const int* li = reinterpret_cast<const int*>(lv + TC_LISTS * TC_Q * a.K);
-      for (int e = lane; e < 32 * a.K; e += 32) {
-        const int ql = 32 * qc + e / a.K, r = e % a.K;
-        const int64_t q = q0 + ql;
-        if (q < a.nq) {
-          const int64_t o = (q * a.nlists + chunk_id * TC_LISTS + rq) * a.K + r;
-          a.cand_v[o] = lv[(rq * TC_Q + ql) * a.K + r];
-          a.cand_i[o] = li[(rq * TC_Q + ql) * a.K + r];
-        }
+      // This lane's list -> candidates of (query, chunk, row quarter).
+      if (myq < a.nq) {
+        const int64_t o = (myq * a.nlists + chunk_id * TC_LISTS + rq) * a.K;
+#pragma unroll
+        for (int r = 0; r < TC_KMAX; ++r)
+          if (r < a.K) {
+            a.cand_v[o + r] = lv[r];
+            a.cand_i[o + r] = li[r];
+          }
       }
     }
   }
@@ -425,7 +461,7 @@ TopkPlan topk_tc_plan(const tq_ctx* c, int64_t nq, int64_t n, int k, int64_t n_s
   const size_t room = (size_t)227 * 1024 > fixed ? (size_t)227 * 1024 - fixed : 0;
   p.stages = (int)(room / BLK);
   if (p.stages > 8) p.stages = 8;
-  p.use_tc = p.stages >= 3 && encode_fn() != nullptr;
+  p.use_tc = p.stages >= 3 && k <= TC_KMAX && encode_fn() != nullptr;
   const int64_t qblocks = (nq + TC_Q - 1) / TC_Q;
   const int64_t nn = n_sample > 0 ? n_sample : n;
   // Full pass: about sixteen items per SM; sample pass: about one.
