@@ -76,6 +76,25 @@ def test_quantize_bit_sweep_outlier_bf16(cuda, bits, qjl):
     P.check_quantized(tab, "v", x, _flat(pv, n))
 
 
+@pytest.mark.parametrize("bits,qjl", [(3, True), (4, False)])
+def test_quantize_prefill_full_size_sampled(cuda, bits, qjl):
+    """The bench's quantize launch at full size: 131072 tokens x 8 kv heads of
+    bf16 K (1,048,576 vectors, the tensor-core path), the oracle on 6144
+    sampled vectors (first, middle and last 2048)."""
+    m = 128 if qjl else 0
+    c = _ctx(128, bits, bits, m, seed=12)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.outlier_kv(1, 8, 131072, 128, seed=90 + bits, device=cuda)[0].reshape(-1, 128)
+    n = X.shape[0]
+    pk = c.quantize(X, tq.TQ_KEY)
+    torch.cuda.synchronize()
+    for s0 in (0, n // 2 - 1024, n - 2048):
+        sl = slice(s0, s0 + 2048)
+        P.check_quantized(tab, "k", P.to_np(X[sl]), _flat({k: (None if v is None else v[sl]) for k, v in pk.items()}, 2048))
+    del X, pk
+    torch.cuda.empty_cache()
+
+
 def test_quantize_d200_mixture(cuda):
     """d=200 (7 words per plane), 3-bit Lloyd-Max + QJL with m=200, unit-norm mixture."""
     c = _ctx(200, 4, 3, 200, seed=5)
