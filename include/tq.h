@@ -353,13 +353,20 @@ int tq_decode_step_paged(tq_ctx* ctx, const void* q, int q_dtype, const void* k_
                          const int32_t* pos, float scale, float* out, void* workspace,
                          size_t ws_bytes, void* stream);
 
-/* Bytes of workspace tq_topk needs. */
+/*
+ * Bytes of workspace tq_topk needs: the database dequantized once into fp16
+ * rows (n * (d + m, each rounded up to 16) * 2 bytes; 832 MB for 1e6
+ * vectors at d = m = 200), the queries' operands, and the candidate lists.
+ */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 
 /*
  * tq_topk - exact top-k of the compressed inner-product scores of nq queries
  * against n packed database keys ([WHAT] "Benchmarks": vector search by
- * inner product), ordered by (score desc, index asc).  Scores are tq_logits.
+ * inner product), ordered by (score desc, index asc).  Scores are tq_logits
+ * up to the fp16 rounding of the scorer's operands (~1e-5 |q| |k|): the
+ * database rows and the queries are rounded to fp16 for the tensor cores,
+ * the norms and the accumulation stay fp32.
  *   q        device, [nq][d] of `dtype`.
  *   codes/qjl/norm/rnorm  device key arrays for the n database vectors.
  *   k        1..32.
