@@ -2,7 +2,7 @@
 // table: 3-bit Lloyd-Max keys with the QJL bit (k4v4: m = 128), and the
 // MSE-only formats: norm-corrected 3- or 4-bit keys (k3v4_nc, 4bit_nc,
 // 3bit_nc) and 8-bit keys (k8v4); values 4 bits (3 bits for 3bit_nc),
-// d = 128, GQA group 4 or 8, on the tensor cores (sm_100a).
+// d = 128, any GQA group of 1, 2, 4 or 8, on the tensor cores (sm_100a).
 //
 // Same quantities as the 2-bit-key kernels ("What is TurboQuant?", "How
 // TurboQuant works", closing paragraph; "How to implement" part 1):
@@ -173,11 +173,12 @@ __device__ __forceinline__ uint2 k8_pair(uint32_t lane_base, uint32_t w) {
 
 template <bool PAGED, int KB, bool QJL, int G, int VB>
 __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
-  static_assert(G == 4 || G == 8, "group 4 or 8");
+  static_assert(G == 2 || G == 4 || G == 8, "group template 2 (groups 1, 2), 4 or 8");
   using KF = KeyFmt<KB>;
   using VF = ValFmt<VB>;
   using Stage = StageL<KB, QJL, VB>;
-  constexpr int NJ = G / 4;   // head sets per thread: t (and 4 + t)
+  constexpr int NJ = G == 8 ? 2 : 1;   // head sets per thread: t (and 4 + t)
+  const int Gr = G == 2 ? a.G : G;      // heads in the group (1 or 2 under the template 2)
   extern __shared__ __align__(16) unsigned char smem[];
   uint2* klut = reinterpret_cast<uint2*>(smem);                                          // [ENT][COP]
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + KF::LUT_BYTES);                     // values
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
+  const bool hv0 = t < Gr;              // this thread's head t exists
 
   if (VB == 4)
     build_value_lut(lut, a.cv, tid, MW * 32);
@@ -252,14 +254,14 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
     const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
     const int64_t tok0 = tt * MT;
     const int64_t tok1 = min(te * MT, len);
-    const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * G;
+    const int64_t qbase = (int64_t)b * a.Hq + (int64_t)kvh * Gr;
 
     __syncthreads();   // the previous piece's readers of the operands are done
     // ---- per-head scales (warp w: heads 2w, 2w+1) and the value-norm maximum ----
 #pragma unroll
     for (int hsel = 0; hsel < 2; ++hsel) {
       const int h = 2 * warp + hsel;
-      if (h >= G) continue;   // uniform over the warp
+      if (h >= Gr) continue;   // uniform over the warp
       const float4 q4 = reinterpret_cast<const float4*>(a.qr + (qbase + h) * 128)[lane];
       float mq = fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w)));
       float ms = 0.f, ss = 0.f;
@@ -323,10 +325,10 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
         uint32_t fr[6];
 #pragma unroll
         for (int mi = 0; mi < NM; ++mi) {
-          const int m = (G == 4 && mi == 1) ? 2 : mi;
+          const int m = (G != 8 && mi == 1) ? 2 : mi;
           const int h = m < 2 ? 4 * m + (g >> 1) : (g >> 1) + 4 * (g & 1);
           const bool tail = m < 2 && odd_col;
-          if (h < G) {
+          if (h < Gr) {
             const float kq = pow2i(-(s_scale[h] + 1));
             const float* row = a.qr + (qbase + h) * 128 + 32 * t;
             fr[2 * mi] = split(row[2 * s] * kq, row[2 * s + 1] * kq, tail);
@@ -345,6 +347,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
 #pragma unroll
           for (int m = 0; m < NJ; ++m) {
             const int h = 4 * m + (g >> 1);
+            if (h >= Gr) continue;   // empty columns of a missing head
             const float ks = pow2i(-s_scale[8 + h]);
             const float* row = a.qs + (qbase + h) * 128 + 32 * t;
 #pragma unroll
@@ -523,15 +526,16 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
         }
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
+          const bool hv = j > 0 || hv0;
           if (QJL) {
             const float kr0 = st.kr[g], kr8 = st.kr[g + 8];
             const float qj0 = fmaf(acs[j][1], 1.f / 4096.f, acs[j][0]);
             const float qj8 = fmaf(acs[j][3], 1.f / 4096.f, acs[j][2]);
-            sc[j][0] = v0 ? fmaf(kn0 * lm[j][0], H[j].x, kr0 * fmaf(qj0, H[j].z, H[j].w)) : -INFINITY;
-            sc[j][1] = v8 ? fmaf(kn8 * lm[j][1], H[j].x, kr8 * fmaf(qj8, H[j].z, H[j].w)) : -INFINITY;
+            sc[j][0] = (hv && v0) ? fmaf(kn0 * lm[j][0], H[j].x, kr0 * fmaf(qj0, H[j].z, H[j].w)) : -INFINITY;
+            sc[j][1] = (hv && v8) ? fmaf(kn8 * lm[j][1], H[j].x, kr8 * fmaf(qj8, H[j].z, H[j].w)) : -INFINITY;
           } else {
-            sc[j][0] = v0 ? kn0 * lm[j][0] * H[j].x : -INFINITY;
-            sc[j][1] = v8 ? kn8 * lm[j][1] * H[j].x : -INFINITY;
+            sc[j][0] = (hv && v0) ? kn0 * lm[j][0] * H[j].x : -INFINITY;
+            sc[j][1] = (hv && v8) ? kn8 * lm[j][1] * H[j].x : -INFINITY;
           }
         }
       }
@@ -552,7 +556,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
 #pragma unroll
           for (int o_ = 4; o_ <= 16; o_ <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o_));
           const float mn = fmaxf(m_run[j], tm);
-          al[j] = ex2f(m_run[j] - mn);
+          al[j] = mn == -INFINITY ? 1.f : ex2f(m_run[j] - mn);   // -inf only for a missing head
           m_run[j] = mn;
           l_part[j] *= al[j];
         }
@@ -569,8 +573,9 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
       float p[2][2] = {{0.f, 0.f}, {0.f, 0.f}};   // [head set][row g, g + 8]
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        p[j][0] = ex2f(sc[j][0] - m_run[j]);
-        p[j][1] = ex2f(sc[j][1] - m_run[j]);
+        const bool hv = j > 0 || hv0;
+        p[j][0] = hv ? ex2f(sc[j][0] - m_run[j]) : 0.f;
+        p[j][1] = hv ? ex2f(sc[j][1] - m_run[j]) : 0.f;
         l_part[j] += p[j][0] + p[j][1];
       }
       const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
@@ -595,7 +600,8 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
     const float vback = pow2i(kv);
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      float* pp = a.part + (slot * G + 4 * j + t) * (128 + 2);
+      if (4 * j + t >= Gr) continue;   // a missing head
+      float* pp = a.part + (slot * Gr + 4 * j + t) * (128 + 2);
       if (g == 0) {
         pp[0] = m_run[j];
         pp[1] = l_part[j];
@@ -612,7 +618,7 @@ __global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
 }  // namespace
 
 bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
-  if (c->d != D || (a.G != 4 && a.G != 8)) return false;
+  if (c->d != D || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8)) return false;
   const bool k3q = c->bk_lm == 3 && c->qjl_m == 128 && c->bits_v == 4;
   const bool mse = c->qjl_m == 0 && ((c->bk_lm == 3 && (c->bits_v == 4 || c->bits_v == 3)) ||
                                      ((c->bk_lm == 4 || c->bk_lm == 8) && c->bits_v == 4));
@@ -627,22 +633,22 @@ bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
 template <int KB, bool QJL, int VB>
 static void lut_launch(const AttnArgs& a, unsigned blocks, cudaStream_t s) {
   constexpr size_t sm = smem_lut<KB, QJL, VB>();
-  if (a.block_table) {
-    if (a.G == 8)
-      k_attn_lut<true, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
-    else
-      k_attn_lut<true, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
-  } else {
-    if (a.G == 8)
-      k_attn_lut<false, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
-    else
-      k_attn_lut<false, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
+  const bool pg = a.block_table != nullptr;
+  if (a.G == 8) {
+    if (pg) k_attn_lut<true, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
+    else k_attn_lut<false, KB, QJL, 8, VB><<<blocks, MW * 32, sm, s>>>(a);
+  } else if (a.G == 4) {
+    if (pg) k_attn_lut<true, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
+    else k_attn_lut<false, KB, QJL, 4, VB><<<blocks, MW * 32, sm, s>>>(a);
+  } else {   // groups 1 and 2
+    if (pg) k_attn_lut<true, KB, QJL, 2, VB><<<blocks, MW * 32, sm, s>>>(a);
+    else k_attn_lut<false, KB, QJL, 2, VB><<<blocks, MW * 32, sm, s>>>(a);
   }
 }
 
 cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
   AttnArgs a = a_in;
-  if (!a.tiles || (a.G != 4 && a.G != 8)) return cudaErrorInvalidValue;
+  if (!a.tiles || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8)) return cudaErrorInvalidValue;
   // CTA-owned ranges of at least four tiles per warp; two CTAs per SM.
   const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
   int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
@@ -676,7 +682,9 @@ static cudaError_t lut_configure() {
   if ((e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, 8, VB>, ms, sm)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 8, VB>, ms, sm)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, 4, VB>, ms, sm)) != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 4, VB>, ms, sm);
+  if ((e = cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 4, VB>, ms, sm)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_lut<false, KB, QJL, 2, VB>, ms, sm)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_attn_lut<true, KB, QJL, 2, VB>, ms, sm);
 }
 
 cudaError_t configure_attn_lut() {

@@ -186,6 +186,8 @@ def test_attention_single_head(cuda):
     (128, 16, 2, 4, 4, 128, 1000),  # 3-bit keys: tensor-core path, group 8
     (128, 8, 2, 4, 4, 128, 1000),   # 3-bit keys: tensor-core path, group 4
     (128, 8, 2, 4, 4, 128, 998),    # 3-bit keys, max_T % 4 != 0: generic path
+    (128, 4, 4, 4, 4, 128, 1000),   # 3-bit keys, group 1: tensor-core path
+    (128, 4, 2, 4, 4, 128, 1000),   # 3-bit keys, group 2: tensor-core path
     (200, 6, 3, 4, 3, 200, 1000), (64, 4, 4, 2, 2, 0, 1000),
     (128, 8, 2, 8, 4, 0, 1000),     # 8-bit keys (k8v4): tensor-core path, group 4
     (128, 16, 2, 8, 4, 0, 998),     # 8-bit keys, max_T % 4 != 0: generic path
@@ -348,6 +350,27 @@ def test_topk_code_widths_and_k(cuda, d, bk, m, k):
     _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), k)
 
 
+@pytest.mark.parametrize("d,bk,m,nq,n,k", [
+    (64, 2, 64, 1, 127, 12),      # one query, a database shorter than one 128-row tile
+    (96, 3, 64, 129, 129, 5),     # ragged query block and tile, K padded to 16s
+    (256, 4, 256, 40, 1000, 3),   # eight 64-wide K blocks (the largest query operand)
+    (256, 2, 0, 200, 700, 12),    # MSE-only keys (no sign accumulator), k at the register-list limit
+])
+def test_topk_tensor_core_edges(cuda, d, bk, m, nq, n, k):
+    """Edge shapes of the tcgen05 scorer: partial tiles and query blocks,
+    the widest query operand, MSE-only keys; no device fault is raised."""
+    c = _ctx(d, bk, 3, m, seed=23)
+    tab = P.oracle_tables(c)
+    X = tq_inputs.mixture(n, d, seed=51)
+    Q = tq_inputs.mixture(nq, d, seed=52, means_seed=51)
+    db = c.quantize(X.to(cuda), tq.TQ_KEY)
+    idx, score = c.topk(Q.to(cuda), db, k)
+    torch.cuda.synchronize()
+    assert tq.tq_device_fault() == 0
+    g = _flat(db, n)
+    _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), k)
+
+
 def test_topk_sample_bar_pass(cuda):
     """A database large enough for the two-pass scorer (the k-th best of a
     leading sample bars every list): exact duplicates inside the sample (equal
@@ -393,6 +416,7 @@ def test_topk_vector_search_full(cuda):
     g = _flat(db, 1_000_000)
     _check_topk(tab, P.to_np(Q[:32]), g, idx[:32].cpu().numpy(), score[:32].cpu().numpy(), 10)
     assert np.all(np.diff(score.cpu().numpy(), axis=1) <= 0)
+    assert tq.tq_device_fault() == 0
 
 
 # --- error reporting through the C ABI ----------------------------------------------
@@ -532,7 +556,7 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
 
 # --- norm-corrected cache formats -------------------------------------------------
 @pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("k3v4_nc", 16), ("4bit_nc", 8), ("4bit_nc", 16),
-                                     ("3bit_nc", 8), ("3bit_nc", 16)])
+                                     ("3bit_nc", 8), ("3bit_nc", 16), ("4bit_nc", 2), ("3bit_nc", 4)])
 def test_norm_corrected_variants(cuda, name, Hq):
     """The MSE-only _nc formats: quantize through the bulk and the small-batch
     kernels (stored norm n / |c[idx]|), logits, ragged decode attention, and
@@ -582,7 +606,7 @@ def test_norm_corrected_variants(cuda, name, Hq):
                       outA.cpu().numpy())
 
 
-@pytest.mark.parametrize("Hq", [8, 16])
+@pytest.mark.parametrize("Hq", [8, 16, 2])
 def test_eight_bit_keys(cuda, Hq):
     """k8v4: 8-bit Lloyd-Max keys (MSE only), 4-bit values.  Quantize through
     the bulk and the small-batch kernels, logits, ragged decode and the fused
@@ -652,7 +676,7 @@ def _to_paged(cache, B, Hkv, max_T, bs, perm):
     (8, 2, 3, 32, None), (16, 2, 3, 16, None), (16, 2, 4, 48, None), (4, 4, 3, 16, None),
     (8, 2, 4, 16, None), (8, 2, None, 32, "4bit_nc"), (16, 2, None, 16, "k3v4_nc"),
     (8, 2, None, 16, "3bit_nc"), (16, 2, None, 48, "3bit_nc"), (8, 2, None, 32, "k8v4"),
-    (16, 2, None, 16, "k8v4")])
+    (16, 2, None, 16, "k8v4"), (4, 2, None, 16, "k3v4_nc"), (2, 2, 4, 32, None)])
 def test_paged_decode_equals_contiguous(cuda, Hq, Hkv, bk, bs, variant):
     """The paged decode reads the same records through the block table, so it
     must reproduce the contiguous decode bit for bit (ragged lengths,
