@@ -554,6 +554,50 @@ def test_decode_step_equals_append_then_decode(cuda, Hq, Hkv, bk, max_T):
                       lens.cpu().numpy(), Hkv, outA.cpu().numpy())
 
 
+@pytest.mark.parametrize("fmt,Hq", [("k3v4", 8), ("k3v4", 16), ("k3v4", 2), ("k4v4", 8), ("k4v4", 4),
+                                    ("k3v4_nc", 8), ("4bit_nc", 2), ("3bit_nc", 16), ("k8v4", 8)])
+def test_decode_logit_precision(cuda, fmt, Hq):
+    """Two keys whose logits are large but differ by 1/100 of their size,
+    the query scaled so the difference is one unit: the softmax weights then
+    expose logit errors 100x magnified.  The tensor-core decode carries ~22
+    bits (fp16 head + tail of both operands), so the output stays within
+    the attention bound; a dropped tail term (~11 bits, ~6e-3 here) would
+    not."""
+    c = tq.Context.variant(fmt, 128, seed=31)
+    tab = P.oracle_tables(c)
+    B, Hkv, d = 4, 2, 128
+    G = Hq // Hkv
+    pool = tq_inputs.iid((2048, d), seed=71)
+    pk = c.quantize(pool.to(cuda), tq.TQ_KEY)
+    torch.cuda.synchronize()
+    g = _flat(pk, 2048)
+    q0 = tq_inputs.iid((B, Hkv, d), seed=72).double().numpy()
+    Q = np.zeros((B, Hq, d))
+    pick = np.zeros((B, Hkv, 2), dtype=np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            lg = o.logits(tab, q0[b, h][None], g["codes"], g["norm"], g.get("qjl"), g.get("rnorm"))[0]
+            order = np.argsort(lg)
+            gaps = np.diff(lg[order])
+            size = np.maximum(np.abs(lg[order][:-1]), np.abs(lg[order][1:]))
+            r = np.argmin(np.abs(np.log(np.maximum(gaps, 1e-30) * 100.0 / np.maximum(size, 1e-30))))
+            i, j = order[r], order[r + 1]
+            pick[b, h] = (i, j)
+            f = 1.0 / (lg[j] - lg[i]) * math.sqrt(d)   # scaled logit difference of one
+            Q[b, h * G:(h + 1) * G] = q0[b, h] * f
+    kc = {k: (None if v is None else v[torch.as_tensor(pick).reshape(-1).to(cuda)].reshape(
+        (B, Hkv, 2) + tuple(v.shape[1:]))) for k, v in pk.items()}
+    kc = {k: (None if v is None else torch.cat([v, v], dim=2).contiguous()) for k, v in kc.items()}   # max_T 4
+    V = tq_inputs.outlier_kv(B, Hkv, 4, d, seed=73)
+    vc = c.quantize(V.to(cuda), tq.TQ_VALUE)
+    lens = torch.full((B,), 2, dtype=torch.int32)
+    Qt = torch.from_numpy(Q).float()
+    out = c.attn_decode(Qt.to(cuda), kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Qt.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+
+
 # --- norm-corrected cache formats -------------------------------------------------
 @pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("k3v4_nc", 16), ("4bit_nc", 8), ("4bit_nc", 16),
                                      ("3bit_nc", 8), ("3bit_nc", 16), ("4bit_nc", 2), ("3bit_nc", 4)])
