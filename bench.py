@@ -74,25 +74,26 @@ def tensor_peak():
     return 1590.0, "fallback 1.59 PFLOP/s bf16"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources of the decode-attention kernel (its counters go stale
-    when these change)."""
+def kernel_source_hash(files) -> str:
+    """Hash of the sources a decode-attention kernel is built from (its
+    counters go stale when these change)."""
     h = hashlib.sha256()
     csrc = ROOT / "compressed_decode_attention_quantize_b200" / "csrc"
-    for name in ("tq_attn_mma.cu", "tq_attn_lut.cu", "tq_attn_common.cuh", "tq_internal.h"):
+    for name in files:
         h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
     """DRAM bytes per attention launch from a committed ncu summary, or None if
-    the kernel sources changed since the counters were taken."""
+    the sources of that workload's kernel changed since the counters were
+    taken."""
     p = ROOT / "profiles" / "attn_traffic.json"
     if not p.exists():
         return None
     j = json.loads(p.read_text())
     e = j.get(workload)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("source_files", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
