@@ -17,8 +17,10 @@
 // product dequantizes: two neighbouring coordinates of a token (a 6-bit index
 // from their two 2-bit fields and two top bits, or the byte of their two
 // 4-bit fields) select a half2 of centroids from a table in shared memory,
-// one copy per lane (3-bit) or per half-warp lane (4-bit: 16 copies keep the
-// 64-bit reads of each half-warp on distinct banks).  Each entry holds the
+// 16 copies (each half-warp lane reads its own, so the 64-bit reads of a
+// half-warp hit distinct banks); 8-bit keys take one coordinate per entry,
+// 32 copies.  3-bit keys run three CTAs per SM with two pipeline stages per
+// warp (their tables are small enough), the others two CTAs.  Each entry holds the
 // fp16 head of the centroid pair and its tail x 2^12; the query operand
 // likewise carries an fp16 head and tail, and three MMAs per k-step form
 // head*head + head*tail + tail*head (~22 bits).  The QJL product, the
@@ -60,10 +62,11 @@ struct KeyFmt {
   static constexpr int K2W = KB == 3 ? 8 : (KB == 4 ? 16 : 36);   // staged row (words)
   static constexpr int REC = KB == 3 ? 12 : (KB == 4 ? 16 : 32);  // words per key record
   static constexpr int ENT = KB == 3 ? 64 : 256;                  // table entries
-  static constexpr int COP = KB == 4 ? 16 : 32;                   // copies of the table
+  static constexpr int COP = KB == 8 ? 32 : 16;                   // copies of the table
   static constexpr int ESZ = KB == 8 ? 4 : 8;                     // bytes per entry
   static constexpr size_t LUT_BYTES = (size_t)ENT * COP * ESZ;
-  static constexpr int NS = KB == 8 ? 2 : NSTK;                   // pipeline stages (shared memory)
+  static constexpr int NS = KB == 4 ? NSTK : 2;                   // pipeline stages (shared memory)
+  static constexpr int CTAS = KB == 3 ? 3 : 2;                    // CTAs per SM
 };
 
 // Values: 4-bit fields (16 words per token, rows padded to VROW) or 3-bit
@@ -151,12 +154,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
 }
 
 // Byte offset of the 3-bit key-table entry of coordinates 2s, 2s+1 of word
-// pair (w2, w1 >> sh), without the lane offset: idx * 32 copies * 8 bytes.
+// pair (w2, w1 >> sh), without the lane offset: idx * 16 copies * 8 bytes.
 template <int S, int SH>
 __device__ __forceinline__ uint32_t klut_off(uint32_t w2, uint32_t w1) {
   const uint32_t nib = (w2 >> (4 * S)) & 0xFu;
   const uint32_t top = (w1 >> (SH + 2 * S)) & 3u;
-  return (nib | (top << 4)) << 8;
+  return (nib | (top << 4)) << 7;
 }
 // 4-bit keys: byte B of word w indexes the table (16 copies * 8 bytes); 8-bit
 // keys likewise (32 copies * 4 bytes).
@@ -172,7 +175,7 @@ __device__ __forceinline__ uint2 k8_pair(uint32_t lane_base, uint32_t w) {
 }
 
 template <bool PAGED, int KB, bool QJL, int G, int VB>
-__global__ void __launch_bounds__(MW * 32, 2) k_attn_lut(AttnArgs a) {
+__global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs a) {
   static_assert(G == 2 || G == 4 || G == 8, "group template 2 (groups 1, 2), 4 or 8");
   using KF = KeyFmt<KB>;
   using VF = ValFmt<VB>;
@@ -649,10 +652,12 @@ static void lut_launch(const AttnArgs& a, unsigned blocks, cudaStream_t s) {
 cudaError_t launch_attn_lut(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
   AttnArgs a = a_in;
   if (!a.tiles || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8)) return cudaErrorInvalidValue;
-  // CTA-owned ranges of at least four tiles per warp; two CTAs per SM.
+  // CTA-owned ranges of at least four tiles per warp; two CTAs per SM (three
+  // for 3-bit keys, whose tables and two-stage rings fit three times).
   const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
+  const int64_t per_sm = c->bk_lm == 3 ? 3 : 2;
   int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
-  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 2 ? (int64_t)c->sms * 2 : blocks);
+  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * per_sm ? (int64_t)c->sms * per_sm : blocks);
   a.nw = (int)blocks;
   a.wpu = MW;
   const unsigned nb = (unsigned)blocks;
