@@ -1157,6 +1157,10 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   int* sci = reinterpret_cast<int*>(take((size_t)nq * ps.nlists * k * sizeof(int)));
   float* barv = reinterpret_cast<float*>(take((size_t)nq * k * sizeof(float)));
   int32_t* bari = reinterpret_cast<int32_t*>(take((size_t)nq * k * sizeof(int32_t)));
+  if (n == 0) {   // nothing to score: every slot is (-1, -inf)
+    k_topk_final<<<(unsigned)nq, 32, 0, s>>>(cv, ci, 0, k, idx, score);
+    return cudaGetLastError();
+  }
   cudaError_t e = launch_prerotate(c, q, dtype, nq, nullptr, qr, qs, s);
   if (e != cudaSuccess) return e;
   if ((e = launch_topk_qprep(c, pl, qr, qs, nq, qh, qsc, s)) != cudaSuccess) return e;

@@ -332,6 +332,11 @@ def test_topk_small_with_ties_and_short_db(cuda):
     torch.cuda.synchronize()
     assert np.all(idx2.cpu().numpy()[:, 5:] == -1) and np.all(np.isneginf(score2.cpu().numpy()[:, 5:]))
     assert sorted(idx2.cpu().numpy()[0, :5].tolist()) == [0, 1, 2, 3, 4]
+    # an empty database: every slot is (-1, -inf)
+    empty = {k: (None if v is None else v[:0]) for k, v in db.items()}
+    idx3, score3 = c.topk(Q[:3].to(cuda), empty, 4)
+    torch.cuda.synchronize()
+    assert np.all(idx3.cpu().numpy() == -1) and np.all(np.isneginf(score3.cpu().numpy()))
 
 
 @pytest.mark.parametrize("d,bk,m,k", [(128, 3, 128, 32), (64, 2, 0, 1), (200, 5, 200, 16), (96, 2, 64, 12)])
