@@ -203,7 +203,8 @@ int tq_quantize_append(tq_ctx* ctx, int which, const void* x, int dtype, int B,
 
 /*
  * tq_quantize_append_paged - tq_quantize_append into a paged cache (blocks of
- * block_size tokens allocated from a pool; SURVEY's "next" paged layout).
+ * block_size tokens allocated from a pool, as serving engines lay out their
+ * KV caches; "A First Comprehensive Study of TurboQuant", section A3).
  *   codes/qjl/norm/rnorm  device cache arrays [num_blocks][H][block_size][...].
  *   block_table  device, int32 [B][max_blocks]: block ids in [0, num_blocks).
  *   pos          device, int32 [B]: token position of sequence b; it goes to
