@@ -20,7 +20,7 @@ _LIB_PATH = _PKG / "libtq.so"
 
 TQ_OK, TQ_ERR_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(5)
 TQ_KEY, TQ_VALUE = 0, 1
-TQ_NC_KEYS, TQ_NC_VALUES = 1, 2
+TQ_NC_KEYS, TQ_NC_VALUES, TQ_NORM_F16 = 1, 2, 4
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 _DTYPES = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
@@ -35,7 +35,8 @@ class TQError(RuntimeError):
 class tq_layout_t(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("bits", ctypes.c_int32), ("words", ctypes.c_int32),
                 ("qjl_m", ctypes.c_int32), ("qjl_words", ctypes.c_int32),
-                ("has_rnorm", ctypes.c_int32), ("bytes_per_vector", ctypes.c_int64)]
+                ("has_rnorm", ctypes.c_int32), ("bytes_per_vector", ctypes.c_int64),
+                ("norm_bytes", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -177,21 +178,23 @@ class Context:
     current CUDA device."""
 
     def __init__(self, d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int = 0,
-                 nc_k: bool = False, nc_v: bool = False):
+                 nc_k: bool = False, nc_v: bool = False, norm_f16: bool = False):
         self.d, self.bits_k, self.bits_v, self.qjl_m, self.seed = d, bits_k, bits_v, qjl_m, seed
-        self.nc_k, self.nc_v = bool(nc_k), bool(nc_v)
-        flags = (TQ_NC_KEYS if nc_k else 0) | (TQ_NC_VALUES if nc_v else 0)
+        self.nc_k, self.nc_v, self.norm_f16 = bool(nc_k), bool(nc_v), bool(norm_f16)
+        flags = ((TQ_NC_KEYS if nc_k else 0) | (TQ_NC_VALUES if nc_v else 0) |
+                 (TQ_NORM_F16 if norm_f16 else 0))
         self.ptr = tq_init_ex(d, bits_k, bits_v, qjl_m, seed, flags)
         self.key_layout = tq_layout(self.ptr, TQ_KEY)
         self.value_layout = tq_layout(self.ptr, TQ_VALUE)
 
     @classmethod
-    def variant(cls, name: str, d: int, seed: int = 0) -> "Context":
-        """A context for one of the named cache formats in VARIANTS."""
+    def variant(cls, name: str, d: int, seed: int = 0, norm_f16: bool = False) -> "Context":
+        """A context for one of the named cache formats in VARIANTS; norm_f16
+        stores the norms as binary16 (formats without QJL)."""
         if name not in VARIANTS:
             raise ValueError(f"unknown variant {name!r}; known: {', '.join(VARIANTS)}")
         bits_k, bits_v, qjl, nc = VARIANTS[name]
-        return cls(d, bits_k, bits_v, d if qjl else 0, seed, nc_k=nc, nc_v=nc)
+        return cls(d, bits_k, bits_v, d if qjl else 0, seed, nc_k=nc, nc_v=nc, norm_f16=norm_f16)
 
     def close(self):
         if getattr(self, "ptr", None):
@@ -227,7 +230,8 @@ class Context:
         lead = tuple(lead_shape)
         out = {
             "codes": torch.empty(lead + (L["words"],), dtype=torch.int32, device=device),
-            "norm": torch.empty(lead, dtype=torch.float32, device=device),
+            "norm": torch.empty(lead, dtype=torch.float16 if L["norm_bytes"] == 2 else torch.float32,
+                                device=device),
             "qjl": None, "rnorm": None,
         }
         if L["has_rnorm"]:

@@ -121,12 +121,16 @@ tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed) {
 tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int flags) {
   int code = TQ_OK;
   if (!valid_dims(d, bits_k, bits_v, qjl_m, &code)) return nullptr;
-  if (flags & ~(TQ_NC_KEYS | TQ_NC_VALUES)) {
+  if (flags & ~(TQ_NC_KEYS | TQ_NC_VALUES | TQ_NORM_F16)) {
     fail(TQ_ERR_ARG, "tq_init_ex: unknown flag bits 0x%x", flags);
     return nullptr;
   }
   if ((flags & TQ_NC_KEYS) && qjl_m > 0) {
     fail(TQ_ERR_UNSUPPORTED, "tq_init_ex: key norm correction needs MSE-only keys (qjl_m = 0)");
+    return nullptr;
+  }
+  if ((flags & TQ_NORM_F16) && qjl_m > 0) {
+    fail(TQ_ERR_UNSUPPORTED, "tq_init_ex: fp16 norms need MSE-only keys (qjl_m = 0)");
     return nullptr;
   }
   tq_ctx* c = new (std::nothrow) tq_ctx();
@@ -136,6 +140,7 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
   }
   c->nc_k = (flags & TQ_NC_KEYS) != 0;
   c->nc_v = (flags & TQ_NC_VALUES) != 0;
+  c->norm_f16 = (flags & TQ_NORM_F16) != 0;
   c->d = d;
   c->J = (d + 31) / 32;
   c->dpad = 32 * c->J;
@@ -293,7 +298,8 @@ int tq_layout(const tq_ctx* c, int which, tq_layout_t* out) {
   out->qjl_m = key ? c->qjl_m : 0;
   out->qjl_words = (out->qjl_m + 31) / 32;
   out->has_rnorm = (key && c->qjl_m > 0) ? 1 : 0;
-  out->bytes_per_vector = (int64_t)out->words * 4 + (int64_t)out->qjl_words * 4 + 4 +
+  out->norm_bytes = c->norm_f16 ? 2 : 4;
+  out->bytes_per_vector = (int64_t)out->words * 4 + (int64_t)out->qjl_words * 4 + out->norm_bytes +
                           (out->has_rnorm ? 4 : 0);
   return TQ_OK;
 }
@@ -319,7 +325,7 @@ struct Paging {
 };
 
 static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64_t n, int64_t ld,
-                           uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm,
+                           uint32_t* codes, uint32_t* qjl, void* norm, float* rnorm,
                            const int32_t* pos, int H, int64_t max_T, void* stream,
                            const char* name, const Paging& pg = Paging()) {
   if (int r = check_ctx(c)) return r;
@@ -350,7 +356,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.bnd = key ? c->bk_f : c->bv_f;
   a.codes = codes;
   a.qjl = qjl;
-  a.norm = norm;
+  a.norm = static_cast<float*>(norm);
   a.rnorm = rnorm;
   a.pos = pos;
   a.H = H;
@@ -360,12 +366,13 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
   a.nc = (key ? c->nc_k : c->nc_v) ? 1 : 0;
+  a.nf16 = c->norm_f16 ? 1 : 0;
   if (n <= tqk::kSmallQuantize) {
     cudaError_t e = tqk::launch_quantize_small(c, a, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;
   }
-  const bool tc = !pg.table && !a.nc && a.bits <= 4 && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+  const bool tc = !pg.table && !a.nc && !a.nf16 && a.bits <= 4 && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
     tqk::QuantTcArgs t{};
@@ -382,7 +389,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
     t.s_f32 = c->S_f;
     t.codes = codes;
     t.qjl = qjl;
-    t.norm = norm;
+    t.norm = static_cast<float*>(norm);
     t.rnorm = rnorm;
     t.pos = pos;
     t.H = H;
@@ -403,14 +410,14 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
 }
 
 int tq_quantize(tq_ctx* c, int which, const void* x, int dtype, int64_t n, int64_t ld,
-                uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm, void* stream) {
+                uint32_t* codes, uint32_t* qjl, void* norm, float* rnorm, void* stream) {
   return quantize_common(c, which, x, dtype, n, ld, codes, qjl, norm, rnorm, nullptr, 0, 0, stream,
                          "tq_quantize");
 }
 
 int tq_quantize_append(tq_ctx* c, int which, const void* x, int dtype, int B, int H, int64_t ld,
                        int64_t max_T, const int32_t* pos, uint32_t* codes, uint32_t* qjl,
-                       float* norm, float* rnorm, void* stream) {
+                       void* norm, float* rnorm, void* stream) {
   if (B < 0 || H <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "tq_quantize_append: bad sizes");
   if (B > 0 && !pos) return fail(TQ_ERR_ARG, "tq_quantize_append: null pos");
   return quantize_common(c, which, x, dtype, (int64_t)B * H, ld, codes, qjl, norm, rnorm, pos, H,
@@ -420,7 +427,7 @@ int tq_quantize_append(tq_ctx* c, int which, const void* x, int dtype, int B, in
 int tq_quantize_append_paged(tq_ctx* c, int which, const void* x, int dtype, int B, int H,
                              int64_t ld, const int32_t* block_table, int max_blocks, int block_size,
                              int64_t num_blocks, const int32_t* pos, uint32_t* codes, uint32_t* qjl,
-                             float* norm, float* rnorm, void* stream) {
+                             void* norm, float* rnorm, void* stream) {
   if (B < 0 || H <= 0 || max_blocks <= 0 || block_size <= 0 || num_blocks <= 0)
     return fail(TQ_ERR_ARG, "tq_quantize_append_paged: bad sizes");
   if (B > 0 && (!pos || !block_table)) return fail(TQ_ERR_ARG, "tq_quantize_append_paged: null pos or block_table");
@@ -434,7 +441,7 @@ int tq_quantize_append_paged(tq_ctx* c, int which, const void* x, int dtype, int
 }
 
 int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* qjl,
-                  const float* norm, const float* rnorm, int64_t n, float* out, void* stream) {
+                  const void* norm, const float* rnorm, int64_t n, float* out, void* stream) {
   if (int r = check_ctx(c)) return r;
   if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "tq_dequantize: bad which=%d", which);
   if (n < 0) return fail(TQ_ERR_ARG, "tq_dequantize: n < 0");
@@ -442,13 +449,13 @@ int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* q
   if (!codes || !norm || !out) return fail(TQ_ERR_ARG, "tq_dequantize: null pointer");
   if (which == TQ_KEY && c->qjl_m > 0 && (!qjl || !rnorm))
     return fail(TQ_ERR_ARG, "tq_dequantize: keys with QJL need qjl and rnorm");
-  cudaError_t e = tqk::launch_dequant(c, which, codes, qjl, norm, rnorm, n, out, as_stream(stream));
+  cudaError_t e = tqk::launch_dequant(c, which, codes, qjl, static_cast<const float*>(norm), rnorm, n, out, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_dequantize");
   return TQ_OK;
 }
 
 int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* kcodes,
-              const uint32_t* kqjl, const float* knorm, const float* krnorm, int64_t nk, float* out,
+              const uint32_t* kqjl, const void* knorm, const float* krnorm, int64_t nk, float* out,
               void* stream) {
   if (int r = check_ctx(c)) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
@@ -458,7 +465,7 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
   if (!q || !kcodes || !knorm || !out) return fail(TQ_ERR_ARG, "tq_logits: null pointer");
   if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "tq_logits: keys with QJL need kqjl and krnorm");
   if (nq > 65535LL * 8) return fail(TQ_ERR_UNSUPPORTED, "tq_logits: nq too large");
-  cudaError_t e = tqk::launch_logits(c, q, dtype, nq, kcodes, kqjl, knorm, krnorm, nk, out,
+  cudaError_t e = tqk::launch_logits(c, q, dtype, nq, kcodes, kqjl, static_cast<const float*>(knorm), krnorm, nk, out,
                                      as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_logits");
   return TQ_OK;
@@ -497,8 +504,8 @@ size_t tq_attn_workspace_bytes(const tq_ctx* c, int B, int Hq, int64_t max_T) {
 }
 
 static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
-                            const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
-                            const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                            const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,
+                            const float* krnorm, const uint32_t* vcodes, const void* vnorm,
                             int64_t max_T, const int32_t* seq_lens, float scale, float* out,
                             void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
                             const char* name) {
@@ -539,10 +546,11 @@ static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, 
   a.wv = c->wv;
   a.kcodes = kcodes;
   a.kqjl = kqjl;
-  a.knorm = knorm;
+  a.knorm = static_cast<const float*>(knorm);
   a.krnorm = krnorm;
   a.vcodes = vcodes;
-  a.vnorm = vnorm;
+  a.vnorm = static_cast<const float*>(vnorm);
+  a.nf16 = c->norm_f16 ? 1 : 0;
   a.max_T = max_T;
   a.seq_lens = seq_lens;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -580,8 +588,8 @@ static bool paging_ok(const Paging& pg) {
 }
 
 int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
-                   const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
-                   const float* krnorm, const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                   const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,
+                   const float* krnorm, const uint32_t* vcodes, const void* vnorm, int64_t max_T,
                    const int32_t* seq_lens, float scale, float* out, void* workspace,
                    size_t ws_bytes, void* stream) {
   return attn_decode_impl(c, q, dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm, vcodes, vnorm, max_T,
@@ -589,8 +597,8 @@ int tq_attn_decode(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
 }
 
 int tq_attn_decode_paged(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
-                         const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
-                         const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                         const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,
+                         const float* krnorm, const uint32_t* vcodes, const void* vnorm,
                          const int32_t* block_table, int max_blocks, int block_size,
                          int64_t num_blocks, const int32_t* seq_lens, float scale, float* out,
                          void* workspace, size_t ws_bytes, void* stream) {
@@ -609,8 +617,8 @@ int tq_attn_decode_paged(tq_ctx* c, const void* q, int dtype, int B, int Hq, int
 
 static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k_new,
                             const void* v_new, int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes,
-                            uint32_t* kqjl, float* knorm, float* krnorm, uint32_t* vcodes,
-                            float* vnorm, int64_t max_T, const int32_t* pos, float scale, float* out,
+                            uint32_t* kqjl, void* knorm, float* krnorm, uint32_t* vcodes,
+                            void* vnorm, int64_t max_T, const int32_t* pos, float scale, float* out,
                             void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
                             const char* name) {
   if (int r = check_ctx(c)) return r;
@@ -649,6 +657,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
     a.nbnd = (1 << a.bits) - 1;
     a.m = key ? c->qjl_m : 0;
     a.nc = (key ? c->nc_k : c->nc_v) ? 1 : 0;
+    a.nf16 = c->norm_f16 ? 1 : 0;
     a.words = key ? c->wk : c->wv;
     a.PiT = c->PiT;
     a.ST = c->ST;
@@ -656,7 +665,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
     a.bnd = key ? c->bk_f : c->bv_f;
     a.codes = key ? kcodes : vcodes;
     a.qjl = key ? kqjl : nullptr;
-    a.norm = key ? knorm : vnorm;
+    a.norm = static_cast<float*>(key ? knorm : vnorm);
     a.rnorm = key ? krnorm : nullptr;
     a.pos = pos;
     a.H = Hkv;
@@ -682,10 +691,11 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
   a.wv = c->wv;
   a.kcodes = kcodes;
   a.kqjl = kqjl;
-  a.knorm = knorm;
+  a.knorm = static_cast<const float*>(knorm);
   a.krnorm = krnorm;
   a.vcodes = vcodes;
-  a.vnorm = vnorm;
+  a.vnorm = static_cast<const float*>(vnorm);
+  a.nf16 = c->norm_f16 ? 1 : 0;
   a.max_T = max_T;
   a.seq_lens = lens;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -733,7 +743,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
 
 int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
                    int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
-                   float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm, int64_t max_T,
+                   void* knorm, float* krnorm, uint32_t* vcodes, void* vnorm, int64_t max_T,
                    const int32_t* pos, float scale, float* out, void* workspace, size_t ws_bytes,
                    void* stream) {
   return decode_step_impl(c, q, q_dtype, k_new, v_new, kv_dtype, B, Hq, Hkv, kcodes, kqjl, knorm, krnorm,
@@ -743,7 +753,7 @@ int tq_decode_step(tq_ctx* c, const void* q, int q_dtype, const void* k_new, con
 
 int tq_decode_step_paged(tq_ctx* c, const void* q, int q_dtype, const void* k_new, const void* v_new,
                          int kv_dtype, int B, int Hq, int Hkv, uint32_t* kcodes, uint32_t* kqjl,
-                         float* knorm, float* krnorm, uint32_t* vcodes, float* vnorm,
+                         void* knorm, float* krnorm, uint32_t* vcodes, void* vnorm,
                          const int32_t* block_table, int max_blocks, int block_size,
                          int64_t num_blocks, const int32_t* pos, float scale, float* out,
                          void* workspace, size_t ws_bytes, void* stream) {
@@ -766,7 +776,7 @@ size_t tq_topk_workspace_bytes(const tq_ctx* c, int64_t nq, int64_t n, int k) {
 }
 
 int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* codes,
-            const uint32_t* qjl, const float* norm, const float* rnorm, int64_t n, int k,
+            const uint32_t* qjl, const void* norm, const float* rnorm, int64_t n, int k,
             int32_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
   if (int r = check_ctx(c)) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
@@ -783,7 +793,7 @@ int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* cod
   if (!workspace || ws_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "tq_topk: workspace %zu bytes < %zu", ws_bytes, need);
   if (!aligned(workspace, 256)) return fail(TQ_ERR_ARG, "tq_topk: workspace not 256-byte aligned");
-  cudaError_t e = tqk::launch_topk(c, q, dtype, nq, codes, qjl, norm, rnorm, n, k, idx, score,
+  cudaError_t e = tqk::launch_topk(c, q, dtype, nq, codes, qjl, static_cast<const float*>(norm), rnorm, n, k, idx, score,
                                    workspace, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_topk");
   return TQ_OK;
@@ -835,8 +845,8 @@ extern "C" size_t tq_attn_static_scratch_bytes(void) { return kStaticScratchByte
 
 extern "C" int tq_attn_decode_static(tq_ctx* c, const void* q, int dtype, int B, int Hq, int Hkv,
                                      const uint32_t* kcodes, const uint32_t* kqjl,
-                                     const float* knorm, const float* krnorm,
-                                     const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                                     const void* knorm, const float* krnorm,
+                                     const uint32_t* vcodes, const void* vnorm, int64_t max_T,
                                      const int32_t* seq_lens, float scale, float* out,
                                      void* stream) {
   if (int r = check_ctx(c)) return r;

@@ -294,12 +294,25 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
     {
       float vmax = 0.f;
       for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
-        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
-        if (j + 4 <= tok1) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vr);
-          vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
+        const int64_t rec = kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
+        if (a.nf16) {
+          const __half* vr = reinterpret_cast<const __half*>(a.vnorm) + rec;
+          if (j + 4 <= tok1) {
+            const uint2 w = *reinterpret_cast<const uint2*>(vr);
+            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+            vmax = fmaxf(vmax, fmaxf(fmaxf(f0.x, f0.y), fmaxf(f1.x, f1.y)));
+          } else {
+            for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, __half2float(vr[k]));
+          }
         } else {
-          for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
+          const float* vr = a.vnorm + rec;
+          if (j + 4 <= tok1) {
+            const float4 v4 = *reinterpret_cast<const float4*>(vr);
+            vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
+          } else {
+            for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
+          }
         }
       }
 #pragma unroll
@@ -415,7 +428,12 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
           const float* base = arr == 0 ? a.knorm : (arr == 1 ? a.krnorm : a.vnorm);
           const uint32_t off = arr == 0 ? offsetof(Stage, kn)
                                         : (arr == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn));
-          cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tok1);
+          if (!a.nf16) {
+            cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tok1);
+          } else if (part < 2) {   // binary16 norms: 8 tokens per chunk
+            cp16(sb + off + part * 16, reinterpret_cast<const __half*>(base) + rb + r + 8 * part,
+                 t0 + 8 * part < tok1);
+          }
         } else if (c < NCH) {                  // value codes: 16 tokens x 4 (3) chunks
           const int cc = c - NKC - NQC - NNC, tok = cc / (VF::REC / 4), part = cc % (VF::REC / 4);
           cp16(sb + offsetof(Stage, v) + tok * (VF::ROW * 4) + part * 16,
@@ -515,7 +533,10 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
         }
       }
       const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
-      const float kn0 = st.kn[g], kn8 = st.kn[g + 8];
+      auto snorm = [&](const float* arr, int i) {
+        return a.nf16 ? __half2float(reinterpret_cast<const __half*>(arr)[i]) : arr[i];
+      };
+      const float kn0 = snorm(st.kn, g), kn8 = snorm(st.kn, g + 8);
       float sc[NJ][2];
       {
         // <q', c> of head t (rows g, g+8) and head 4 + t: head products plus
@@ -581,7 +602,7 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
         p[j][1] = hv ? ex2f(sc[j][1] - m_run[j]) : 0.f;
         l_part[j] += p[j][0] + p[j][1];
       }
-      const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
+      const float w0s = snorm(st.vn, g) * vmul, w8s = snorm(st.vn, g + 8) * vmul;
       const uint32_t pb0 = movtrans(pack_half2(p[0][0] * w0s, p[1][0] * w0s));
       const uint32_t pb1 = movtrans(pack_half2(p[0][1] * w8s, p[1][1] * w8s));
       if constexpr (VB == 4)
@@ -627,6 +648,7 @@ bool attn_lut_supported(const tq_ctx* c, const AttnArgs& a) {
                                      ((c->bk_lm == 4 || c->bk_lm == 8) && c->bits_v == 4));
   if (!k3q && !mse) return false;
   if (a.max_T % 4 != 0) return false;
+  if (c->norm_f16 && (k3q || a.max_T % 8 != 0)) return false;   // binary16 norms: 8-token chunks
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.knorm) |
                        reinterpret_cast<uintptr_t>(a.vcodes) | reinterpret_cast<uintptr_t>(a.vnorm) |
                        (k3q ? reinterpret_cast<uintptr_t>(a.kqjl) | reinterpret_cast<uintptr_t>(a.krnorm) : 0);

@@ -691,6 +691,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
 }  // namespace
 
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
+  if (c->norm_f16) return false;   // QJL formats keep fp32 norms
   if (c->d != D || c->bk_lm != 2 || c->bits_v != 4 || c->qjl_m != 128) return false;
   if (!(a.G == 1 || a.G == 2 || a.G == 4 || a.G == 8)) return false;
   if (a.max_T % 4 != 0) return false;

@@ -6,6 +6,7 @@
 #include <string>
 #include <vector>
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "tq.h"
@@ -40,6 +41,7 @@ struct tq_ctx {
   int sms = 148;
   bool nc_k = false;   // norm correction of keys (MSE-only keys)
   bool nc_v = false;   // norm correction of values
+  bool norm_f16 = false;   // norms stored as binary16 (MSE-only keys)
   const void* tc_pih = nullptr;   // 2^8 Pi, fp16 head
   const void* tc_pil = nullptr;   // 2^8 Pi - head, fp16
   const void* tc_s = nullptr;     // S, fp16 (exact)
@@ -64,6 +66,17 @@ namespace tqk {
 
 // Codebook sizes up to 2^8 levels (Lloyd-Max bits 1..4 and 8).
 constexpr int kMaxLevels = 256;
+
+// Per-vector norms are fp32, or binary16 when the context stores them so.
+__device__ __forceinline__ float load_norm(const float* p, int64_t i, int f16) {
+  return f16 ? __half2float(reinterpret_cast<const __half*>(p)[i]) : p[i];
+}
+__device__ __forceinline__ void store_norm(float* p, int64_t i, float v, int f16) {
+  if (f16)
+    reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  else
+    p[i] = v;
+}
 
 struct QuantArgs {
   const void* x;
@@ -91,6 +104,8 @@ struct QuantArgs {
   int64_t num_blocks;
   // Norm correction (MSE-only vectors): store n / |c[idx]| instead of n.
   int nc;
+  // Norms stored as binary16 (the norm pointer then addresses __half values).
+  int nf16;
 };
 
 struct AttnArgs {
@@ -125,6 +140,8 @@ struct AttnArgs {
   const int32_t* block_table;
   int max_blocks, block_size;
   int64_t num_blocks;
+  // Norms stored as binary16 (knorm / vnorm then address __half values).
+  int nf16;
 };
 
 struct QuantTcArgs {

@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
       if (lane == v) my_norm = nrm[v];
     if (lane < QV && v0 + lane < a.n) {
       const int64_t rec = out_record(a, v0 + lane);
-      if (rec >= 0) a.norm[rec] = my_norm;
+      if (rec >= 0) store_norm(a.norm, rec, my_norm, a.nf16);
     }
     if (a.m == 0) { __syncwarp(); continue; }
 
@@ -419,7 +419,7 @@ __device__ __forceinline__ void quantize_small_body(const QuantArgs& a, int dpad
       const int wi = a.bits * i32 + lane / per;
       if (lane % per == 0 && wi < a.words) a.codes[rec * a.words + wi] = wv;
     }
-    if (j == 0) a.norm[rec] = nrm[u];
+    if (j == 0) store_norm(a.norm, rec, nrm[u], a.nf16);
   }
   if (a.m == 0) return;
   float rho[QS];
@@ -646,7 +646,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
             if (h < G) acc2[h] += pos ? ssv[h * DP + i] : -ssv[h * DP + i];
         }
       }
-      const float kn = a.knorm[r];
+      const float kn = load_norm(a.knorm, r, a.nf16);
       const float kg = a.m > 0 ? a.krnorm[r] * a.cq : 0.f;
 #pragma unroll
       for (int h = 0; h < GMAX; ++h)
@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(AT) k_attn_split(AttnArgs a) {
         alpha[h] = (mnew[h] == kNegInf) ? 1.f : exp2f(m_run[h] - mnew[h]);
       }
     }
-    const float vn = valid ? a.vnorm[kv_row0 + t] : 0.f;
+    const float vn = valid ? load_norm(a.vnorm, kv_row0 + t, a.nf16) : 0.f;
     float psum[GMAX];
 #pragma unroll
     for (int h = 0; h < GMAX; ++h) {
@@ -837,7 +837,7 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
                                                 const float* ST, const float* ck, float cq,
                                                 const uint32_t* kcodes, const uint32_t* kqjl,
                                                 const float* knorm, const float* krnorm,
-                                                int64_t nk, float* out) {
+                                                int64_t nk, int nf16, float* out) {
   constexpr int DP = J * 32;
   __shared__ float sx[LQB][DP], sq[LQB][DP], ss[LQB][DP];
   __shared__ float s_ck[kMaxLevels];
@@ -886,7 +886,7 @@ __global__ void __launch_bounds__(128) k_logits(const void* q, int dtype, int64_
       for (int qq = 0; qq < LQB; ++qq) acc2[qq] += pos ? ss[qq][32 * wi + e] : -ss[qq][32 * wi + e];
     }
   }
-  const float kn = knorm[key];
+  const float kn = load_norm(knorm, key, nf16);
   const float kg = m > 0 ? krnorm[key] * cq : 0.f;
 #pragma unroll
   for (int qq = 0; qq < LQB; ++qq)
@@ -902,13 +902,13 @@ __global__ void __launch_bounds__(128) k_dequant(int d, int dpad, int bits, int 
                                                  const float* cen, float cq,
                                                  const uint32_t* codes, const uint32_t* qjl,
                                                  const float* norm, const float* rnorm,
-                                                 float* out) {
+                                                 int nf16, float* out) {
   extern __shared__ float sh[];
   float* srot = sh;  // [dpad]
   const int64_t v = blockIdx.x;
   const int mw = (m + 31) >> 5;
   const uint32_t* w = codes + v * words;
-  const float n = norm[v];
+  const float n = load_norm(norm, v, nf16);
   const float kg = m > 0 ? rnorm[v] * cq : 0.f;
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     float r = n * cen[code_index(w, bits, d, j)];
@@ -1085,7 +1085,7 @@ cudaError_t launch_logits(const tq_ctx* c, const void* q, int dtype, int64_t nq,
   const float cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
   TQ_DISPATCH_J(c->J, k_logits<JV><<<grid, 128, 0, s>>>(q, dtype, nq, c->d, c->bk_lm, c->wk, c->qjl_m,
                                                         c->PiT, c->ST, c->ck_f, cq, kcodes, kqjl,
-                                                        knorm, krnorm, nk, out);
+                                                        knorm, krnorm, nk, c->norm_f16 ? 1 : 0, out);
                 return cudaGetLastError());
 }
 
@@ -1099,7 +1099,7 @@ cudaError_t launch_dequant(const tq_ctx* c, int which, const uint32_t* codes,
   k_dequant<<<(unsigned)n, 128, c->dpad * sizeof(float), s>>>(
       c->d, c->dpad, key ? c->bk_lm : c->bits_v, key ? c->wk : c->wv, m, c->Pi_f, c->S_f,
       key ? c->ck_f : c->cv_f, cq,
-      codes, qjl, norm, rnorm, out);
+      codes, qjl, norm, rnorm, c->norm_f16 ? 1 : 0, out);
   return cudaGetLastError();
 }
 

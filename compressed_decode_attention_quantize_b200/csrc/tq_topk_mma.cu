@@ -99,8 +99,9 @@ struct TopkMmaArgs {
   int KL, KQ, m;
   float cq;   // sqrt(pi/2) / m
   const __half* rows;   // dequantized database [n][KL + KQ]
-  const float* norm;
+  const float* norm;     // binary16 values when nf16
   const float* rnorm;
+  int nf16;
   int64_t n, chunk;   // database size, vectors per chunk (multiple of TKR)
   int64_t chunks, qblocks;   // work items = chunks x qblocks, chunk-major
   int K, nlists;
@@ -244,8 +245,12 @@ __global__ void __launch_bounds__(TKWARPS * 32) k_topk_gemm(TopkMmaArgs a) {
     if (tid < 2 * TKR) {
       const int r = tid & (TKR - 1);
       const bool ok = v0 + r < n1 && (tid < TKR || a.m > 0);
-      const float* src = tid < TKR ? a.norm : a.rnorm;
-      cp4(sN + st * 2 * TKR + tid, ok ? src + v0 + r : a.norm, ok);
+      if (a.nf16 && tid < TKR) {   // binary16 norms: a plain load (no 2-byte cp.async)
+        sN[st * 2 * TKR + tid] = ok ? load_norm(a.norm, v0 + r, 1) : 0.f;
+      } else {
+        const float* src = tid < TKR ? a.norm : a.rnorm;
+        cp4(sN + st * 2 * TKR + tid, ok ? src + v0 + r : a.norm, ok);
+      }
     }
   };
 #pragma unroll
@@ -494,6 +499,7 @@ cudaError_t launch_topk_mma(const tq_ctx* c, const TopkPlan& p, const void* qh, 
   a.rows = static_cast<const __half*>(rows);
   a.norm = norm;
   a.rnorm = rnorm;
+  a.nf16 = c->norm_f16 ? 1 : 0;
   a.n = n;
   a.chunk = p.chunk;
   a.K = k;

@@ -55,8 +55,9 @@ struct TopkTcArgs {
   int KL, KQ, nkb;    // K blocks of 64 covering KL + KQ
   int m;
   float cq;           // sqrt(pi/2) / m
-  const float* norm;
+  const float* norm;   // binary16 values when nf16
   const float* rnorm;
+  int nf16;
   int64_t n, chunk, chunks, qblocks;
   int K, nlists, stages;
   float* cand_v;
@@ -296,7 +297,7 @@ __global__ void __maxnreg__(96)
       auto norms = [&](int t, float& nv, float& gv) {
         const int64_t v = n0 + (int64_t)t * TC_ROWS + 32 * rq + lane;
         const bool ok = t < ntile && v < n1;
-        nv = ok ? a.norm[v] : 0.f;
+        nv = ok ? load_norm(a.norm, v, a.nf16) : 0.f;
         gv = (ok && a.m > 0) ? a.rnorm[v] * a.cq : 0.f;
       };
       float nv_next, gv_next;
@@ -497,6 +498,7 @@ cudaError_t launch_topk_tc(const tq_ctx* c, const TopkPlan& p, const void* qh, c
   a.cq = c->qjl_m > 0 ? (float)(std::sqrt(M_PI / 2.0) / c->qjl_m) : 0.f;
   a.norm = norm;
   a.rnorm = rnorm;
+  a.nf16 = c->norm_f16 ? 1 : 0;
   a.n = n;
   a.chunk = p.chunk;
   a.chunks = p.chunks;

@@ -49,7 +49,8 @@
  *   qjl    uint32[ceil(m/32)]  keys only: bit i%32 of word i/32 is 1 when
  *                      (S r)_i >= 0.
  *   norm   float       |x| (fp32); |x| / |c[idx]| under norm correction
- *                      (see tq_init_ex).
+ *                      (see tq_init_ex); binary16 under TQ_NORM_F16 (the
+ *                      norm pointers of the calls are void* for this).
  *   rnorm  float       keys with QJL only: gamma = |x| * |r|, r the residual
  *                      of the rotated unit vector.
  * Arrays of vectors are these records laid out as separate dense arrays
@@ -87,6 +88,7 @@ typedef struct tq_layout_t {
   int32_t qjl_words;      /* ceil(qjl_m/32)                                  */
   int32_t has_rnorm;      /* 1 when an rnorm (gamma) array is produced       */
   int64_t bytes_per_vector; /* codes + qjl + norm (+ rnorm) bytes            */
+  int32_t norm_bytes;     /* 4 (fp32 norms) or 2 (fp16, TQ_NORM_F16)         */
 } tq_layout_t;
 
 /* Message for the last failed call on this thread ("" if none). */
@@ -123,7 +125,7 @@ int tq_device_fault(int* code);
 tq_ctx* tq_init(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed);
 
 /* Flags of tq_init_ex. */
-enum tq_flags { TQ_NC_KEYS = 1, TQ_NC_VALUES = 2 };
+enum tq_flags { TQ_NC_KEYS = 1, TQ_NC_VALUES = 2, TQ_NORM_F16 = 4 };
 
 /*
  * tq_init_ex - tq_init with options.  The norm-corrected variants named in
@@ -137,7 +139,12 @@ enum tq_flags { TQ_NC_KEYS = 1, TQ_NC_VALUES = 2 };
  * it as before.
  *   flags  TQ_NC_KEYS: norm correction of keys, which must then be MSE-only
  *          (qjl_m = 0, else NULL with TQ_ERR_UNSUPPORTED);
- *          TQ_NC_VALUES: norm correction of values.
+ *          TQ_NC_VALUES: norm correction of values;
+ *          TQ_NORM_F16: the per-vector norms of keys and values are stored as
+ *          IEEE binary16 (2 bytes, rounded to nearest even from the fp32
+ *          value) instead of fp32, as the serving formats of that study do;
+ *          keys must then be MSE-only (qjl_m = 0: gamma stays fp32-only).
+ *          The `norm` arrays of every call are then uint16 arrays.
  *          Other bits: NULL with TQ_ERR_ARG.
  * Otherwise as tq_init.
  */
@@ -180,7 +187,7 @@ int tq_export_tables(const tq_ctx* ctx, double* pi, double* S, double* ck,
  * Inputs must be finite with |x|^2 representable in fp32.
  */
 int tq_quantize(tq_ctx* ctx, int which, const void* x, int dtype, int64_t n,
-                int64_t ld, uint32_t* codes, uint32_t* qjl, float* norm,
+                int64_t ld, uint32_t* codes, uint32_t* qjl, void* norm,
                 float* rnorm, void* stream);
 
 /*
@@ -198,7 +205,7 @@ int tq_quantize(tq_ctx* ctx, int which, const void* x, int dtype, int64_t n,
  */
 int tq_quantize_append(tq_ctx* ctx, int which, const void* x, int dtype, int B,
                        int H, int64_t ld, int64_t max_T, const int32_t* pos,
-                       uint32_t* codes, uint32_t* qjl, float* norm, float* rnorm,
+                       uint32_t* codes, uint32_t* qjl, void* norm, float* rnorm,
                        void* stream);
 
 /*
@@ -216,7 +223,7 @@ int tq_quantize_append_paged(tq_ctx* ctx, int which, const void* x, int dtype, i
                              int H, int64_t ld, const int32_t* block_table,
                              int max_blocks, int block_size, int64_t num_blocks,
                              const int32_t* pos, uint32_t* codes, uint32_t* qjl,
-                             float* norm, float* rnorm, void* stream);
+                             void* norm, float* rnorm, void* stream);
 
 /*
  * tq_dequantize - x_hat = |x| Pi^T c[idx], plus for keys with QJL the
@@ -226,7 +233,7 @@ int tq_quantize_append_paged(tq_ctx* ctx, int which, const void* x, int dtype, i
  *   out     device, float [n][d].
  */
 int tq_dequantize(tq_ctx* ctx, int which, const uint32_t* codes,
-                  const uint32_t* qjl, const float* norm, const float* rnorm,
+                  const uint32_t* qjl, const void* norm, const float* rnorm,
                   int64_t n, float* out, void* stream);
 
 /*
@@ -239,7 +246,7 @@ int tq_dequantize(tq_ctx* ctx, int which, const uint32_t* codes,
  *   out     device, float [nq][nk].
  */
 int tq_logits(tq_ctx* ctx, const void* q, int dtype, int64_t nq,
-              const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
+              const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,
               const float* krnorm, int64_t nk, float* out, void* stream);
 
 /* Bytes of workspace tq_attn_decode needs for these sizes. */
@@ -265,8 +272,8 @@ size_t tq_attn_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int64_t max_T);
  */
 int tq_attn_decode(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
                    int Hkv, const uint32_t* kcodes, const uint32_t* kqjl,
-                   const float* knorm, const float* krnorm,
-                   const uint32_t* vcodes, const float* vnorm, int64_t max_T,
+                   const void* knorm, const float* krnorm,
+                   const uint32_t* vcodes, const void* vnorm, int64_t max_T,
                    const int32_t* seq_lens, float scale, float* out,
                    void* workspace, size_t ws_bytes, void* stream);
 
@@ -289,8 +296,8 @@ int tq_attn_decode(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
  */
 int tq_attn_decode_static(tq_ctx* ctx, const void* q, int dtype, int B, int Hq,
                           int Hkv, const uint32_t* kcodes, const uint32_t* kqjl,
-                          const float* knorm, const float* krnorm,
-                          const uint32_t* vcodes, const float* vnorm,
+                          const void* knorm, const float* krnorm,
+                          const uint32_t* vcodes, const void* vnorm,
                           int64_t max_T, const int32_t* seq_lens, float scale,
                           float* out, void* stream);
 
@@ -310,8 +317,8 @@ size_t tq_attn_static_scratch_bytes(void);
  * max_blocks * block_size).
  */
 int tq_attn_decode_paged(tq_ctx* ctx, const void* q, int dtype, int B, int Hq, int Hkv,
-                         const uint32_t* kcodes, const uint32_t* kqjl, const float* knorm,
-                         const float* krnorm, const uint32_t* vcodes, const float* vnorm,
+                         const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,
+                         const float* krnorm, const uint32_t* vcodes, const void* vnorm,
                          const int32_t* block_table, int max_blocks, int block_size,
                          int64_t num_blocks, const int32_t* seq_lens, float scale, float* out,
                          void* workspace, size_t ws_bytes, void* stream);
@@ -336,8 +343,8 @@ int tq_attn_decode_paged(tq_ctx* ctx, const void* q, int dtype, int B, int Hq, i
  */
 int tq_decode_step(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
                    const void* v_new, int kv_dtype, int B, int Hq, int Hkv,
-                   uint32_t* kcodes, uint32_t* kqjl, float* knorm, float* krnorm,
-                   uint32_t* vcodes, float* vnorm, int64_t max_T, const int32_t* pos,
+                   uint32_t* kcodes, uint32_t* kqjl, void* knorm, float* krnorm,
+                   uint32_t* vcodes, void* vnorm, int64_t max_T, const int32_t* pos,
                    float scale, float* out, void* workspace, size_t ws_bytes,
                    void* stream);
 
@@ -348,8 +355,8 @@ int tq_decode_step(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
  */
 int tq_decode_step_paged(tq_ctx* ctx, const void* q, int q_dtype, const void* k_new,
                          const void* v_new, int kv_dtype, int B, int Hq, int Hkv,
-                         uint32_t* kcodes, uint32_t* kqjl, float* knorm, float* krnorm,
-                         uint32_t* vcodes, float* vnorm, const int32_t* block_table,
+                         uint32_t* kcodes, uint32_t* kqjl, void* knorm, float* krnorm,
+                         uint32_t* vcodes, void* vnorm, const int32_t* block_table,
                          int max_blocks, int block_size, int64_t num_blocks,
                          const int32_t* pos, float scale, float* out, void* workspace,
                          size_t ws_bytes, void* stream);
@@ -376,7 +383,7 @@ size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
  * Lloyd-Max bits: TQ_ERR_UNSUPPORTED.
  */
 int tq_topk(tq_ctx* ctx, const void* q, int dtype, int64_t nq,
-            const uint32_t* codes, const uint32_t* qjl, const float* norm,
+            const uint32_t* codes, const uint32_t* qjl, const void* norm,
             const float* rnorm, int64_t n, int k, int32_t* idx, float* score,
             void* workspace, size_t ws_bytes, void* stream);
 

@@ -263,19 +263,23 @@ class Tables:
     cb_v: Codebook
     nc_k: bool = False     # R13 norm correction of keys
     nc_v: bool = False     # R13 norm correction of values
+    norm_f16: bool = False # norms stored as binary16 (MSE-only keys)
 
 
 def make_tables(d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int,
-                nc_k: bool = False, nc_v: bool = False) -> Tables:
+                nc_k: bool = False, nc_v: bool = False, norm_f16: bool = False) -> Tables:
     """bits_k counts the QJL bit when qjl_m > 0 (R3).  nc_k / nc_v turn on
-    the R13 norm correction (keys only without QJL)."""
+    the R13 norm correction (keys only without QJL); norm_f16 stores the
+    per-vector norms as binary16 (MSE-only keys)."""
     if nc_k and qjl_m > 0:
         raise ValueError("key norm correction applies to MSE-only keys (qjl_m = 0)")
+    if norm_f16 and qjl_m > 0:
+        raise ValueError("binary16 norms apply to MSE-only keys (qjl_m = 0)")
     bits_k_lm = bits_k - 1 if qjl_m > 0 else bits_k
     Pi = rotation(d, seed)
     S = qjl_matrix(qjl_m, d, seed) if qjl_m > 0 else None
     return Tables(d, bits_k_lm, bits_v, qjl_m, seed, Pi, S,
-                  lloyd_max(d, bits_k_lm), lloyd_max(d, bits_v), nc_k, nc_v)
+                  lloyd_max(d, bits_k_lm), lloyd_max(d, bits_v), nc_k, nc_v, norm_f16)
 
 
 # ----------------------------------------------------------------------------
@@ -384,8 +388,9 @@ def quantize(x: np.ndarray, tab: Tables, which: str) -> Quantized:
     idx = lloyd_max_index(y, cb)
     nc = tab.nc_k if which == "k" else tab.nc_v
     stored = corrected_norm(n, idx, cb) if nc else n
+    # The stored scalar: fp32 (R4), or binary16 rounded to nearest even.
     q = Quantized(idx=idx, codes=pack_codes(idx, cb.bits),
-                  norm=stored.astype(np.float32), y=y)
+                  norm=stored.astype(np.float16 if tab.norm_f16 else np.float32), y=y)
     if which == "k" and tab.qjl_m > 0:
         sketch_from_indices(q, tab)
     return q

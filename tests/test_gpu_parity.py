@@ -702,6 +702,81 @@ def test_eight_bit_keys(cuda, Hq):
     assert e.value.status == tq.TQ_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("name,Hq", [("k3v4_nc", 8), ("4bit_nc", 4), ("3bit_nc", 16), ("k8v4", 8)])
+def test_binary16_norm_variants(cuda, name, Hq):
+    """The MSE-only formats with binary16 norms: layout, quantize (bulk and
+    small batch), logits, dequantize, decode on the tensor-core path
+    (max_T % 8 == 0) and the generic path, the fused step, paged caches and
+    (for keys of at most 4 bits) top-k, all against the oracle."""
+    c = tq.Context.variant(name, 128, seed=14, norm_f16=True)
+    assert c.key_layout["norm_bytes"] == 2 and c.value_layout["norm_bytes"] == 2
+    tab = P.oracle_tables(c)
+    B, Hkv, T, d = 4, 2, 1104, 128
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=81)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=82)
+    kc, vc = _cache(c, K, V, cuda)
+    assert kc["norm"].dtype == torch.float16
+    n = B * Hkv * T
+    P.check_quantized(tab, "k", P.to_np(K.reshape(n, d)), _flat(kc, n))
+    P.check_quantized(tab, "v", P.to_np(V.reshape(n, d)), _flat(vc, n))
+    small = V[1, 0, :300].contiguous()
+    vs = c.quantize(small.to(cuda), tq.TQ_VALUE)
+    P.check_quantized(tab, "v", P.to_np(small), _flat(vs, 300))
+    Q = tq_inputs.iid((B, Hq, d), seed=83, dtype=torch.bfloat16)
+    ks = {k: (None if v is None else v[0, 0, :256].contiguous()) for k, v in kc.items()}
+    lg = c.logits(Q[0].to(cuda), ks)
+    xh = c.dequantize(tq.TQ_VALUE, vs)
+    torch.cuda.synchronize()
+    P.check_logits(tab, Q[0].double().numpy(), _flat(ks, 256), lg.cpu().double().numpy())
+    g = _flat(vs, 300)
+    ref = o.dequantize(tab, "v", g["codes"], g["norm"])
+    assert np.abs(xh.cpu().double().numpy() - ref).max() <= 1e-5 * np.abs(ref).max()
+    lens = torch.tensor([0, 1, 517, T], dtype=torch.int32)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    kg = {k: (None if v is None else v[:, :, :T - 2].contiguous()) for k, v in kc.items()}   # generic path
+    vg = {k: (None if v is None else v[:, :, :T - 2].contiguous()) for k, v in vc.items()}
+    lens_g = torch.tensor([0, 1, 517, T - 2], dtype=torch.int32)
+    outg = c.attn_decode(Q.to(cuda), kg, vg, lens_g.to(cuda))
+    torch.cuda.synchronize()
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kg), P.packed_np(vg), lens_g.numpy(), Hkv,
+                      outg.cpu().numpy())
+    # fused step vs append + decode
+    kB = {k: (None if v is None else v.clone()) for k, v in kc.items()}
+    vB = {k: (None if v is None else v.clone()) for k, v in vc.items()}
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=84)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=85)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([3, 700, T - 1, 64], dtype=torch.int32, device=cuda)
+    q = Q.to(cuda)
+    outA = c.decode_step(q, kn, vn, kc, vc, pos)
+    c.quantize_append(kn, tq.TQ_KEY, kB, pos)
+    c.quantize_append(vn, tq.TQ_VALUE, vB, pos)
+    outB = c.attn_decode(q, kB, vB, (pos + 1).to(torch.int32))
+    torch.cuda.synchronize()
+    for a_, b_ in ((kc, kB), (vc, vB)):
+        for k in a_:
+            if a_[k] is not None:
+                assert torch.equal(a_[k], b_[k]), k
+    assert torch.equal(outA, outB)
+    # paged: the same records through a shuffled block table
+    bs, mb = 16, T // 16
+    perm = torch.randperm(B * mb, generator=torch.Generator().manual_seed(3)).to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, T, bs, perm), _to_paged(vc, B, Hkv, T, bs, perm)
+    got = c.attn_decode_paged(q, kp, vp, perm.reshape(B, mb).to(cuda), lens.to(cuda))
+    ref_c = c.attn_decode(q, kc, vc, lens.to(cuda))
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref_c)
+    if c.key_layout["bits"] <= 4:
+        X = tq_inputs.mixture(3000, d, seed=86)
+        Qs = tq_inputs.mixture(60, d, seed=87, means_seed=86)
+        db = c.quantize(X.to(cuda), tq.TQ_KEY)
+        idx, score = c.topk(Qs.to(cuda), db, 8)
+        torch.cuda.synchronize()
+        assert tq.tq_device_fault() == 0
+        _check_topk(tab, Qs.double().numpy(), _flat(db, 3000), idx.cpu().numpy(), score.cpu().numpy(), 8)
+
+
 # --- paged caches ---------------------------------------------------------------
 def _to_paged(cache, B, Hkv, max_T, bs, perm):
     """Scatter a contiguous [B, Hkv, max_T, ...] cache into blocks

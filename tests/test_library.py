@@ -76,8 +76,11 @@ def test_norm_correction_flags_validated_before_any_device_call():
         tq.tq_init_ex(128, 3, 4, 128, 0, tq.TQ_NC_KEYS)   # keys with QJL
     assert "norm correction" in str(e.value)
     with pytest.raises(tq.TQError) as e:
-        tq.tq_init_ex(128, 3, 4, 0, 0, 4)
+        tq.tq_init_ex(128, 3, 4, 0, 0, 8)
     assert "flag" in str(e.value)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_init_ex(128, 3, 4, 128, 0, tq.TQ_NORM_F16)   # binary16 norms with QJL keys
+    assert "fp16 norms" in str(e.value)
     with pytest.raises(ValueError):
         tq.Context.variant("k2v2", 128)
     assert set(tq.VARIANTS) == {"k3v4", "k4v4", "k3v4_nc", "4bit_nc", "3bit_nc", "k8v4"}

@@ -181,6 +181,24 @@ def test_norm_correction_mean_square_is_one_minus_distortion(bits):
     assert abs(ratio2.mean() - (1.0 - o.distortion(d, tab.cb_v))) < 3e-3
 
 
+@pytest.mark.parametrize("bits", [3, 4])
+def test_binary16_norms(bits):
+    """Binary16 norms: the stored scalar is the fp64 value rounded to the
+    nearest binary16, so the dequantized vector keeps the corrected norm to
+    half a binary16 step (2^-11 relative), and QJL keys are refused."""
+    d = 128
+    x = np.random.default_rng(bits + 60).standard_normal((3000, d)) * 7.0
+    n = np.linalg.norm(x, axis=1)
+    tab = o.make_tables(d, bits, bits, 0, 4, nc_k=True, nc_v=True, norm_f16=True)
+    for which in ("k", "v"):
+        q = o.quantize(x, tab, which)
+        assert q.norm.dtype == np.float16
+        xh = o.dequantize(tab, which, q.codes, q.norm)
+        assert np.all(np.abs(np.linalg.norm(xh, axis=1) - n) <= 2.0 ** -11 * n * (1 + 1e-9))
+    with pytest.raises(ValueError):
+        o.make_tables(d, bits, bits, 64, 4, norm_f16=True)
+
+
 def test_norm_correction_needs_mse_only_keys():
     with pytest.raises(ValueError):
         o.make_tables(64, 3, 4, 64, 1, nc_k=True)
