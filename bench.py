@@ -363,46 +363,59 @@ def variant_decode(tq, tq_inputs, torch, dev, hbm_peak, shape, steps=20, warmup=
     """tq_attn_decode for each format of FORMAT_VARIANTS on one decode shape."""
     B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
     out = {}
-    for name in FORMAT_VARIANTS:
-        ctx = tq.Context.variant(name, d, 0)
-        kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
-        vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
-        for b in range(B):
-            K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
-            V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
-            ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
-            ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
-            del K, V
-        q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
-        lens = torch.full((B,), T, dtype=torch.int32, device=dev)
-        o = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
-        ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
-        for _ in range(warmup):
-            ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(steps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / steps
-        kb, vb = ctx.key_layout["bytes_per_vector"], ctx.value_layout["bytes_per_vector"]
-        alg = B * Hkv * T * (kb + vb) + B * Hq * d * 2 + B * Hq * d * 4
-        bits_k, bits_v, _, nc = tq.VARIANTS[name]
-        out[name] = {"kv_format": f"keys {bits_k} Lloyd-Max bits, values {bits_v} bits, MSE only"
-                                  f"{', norm-corrected' if nc else ''}; {kb + vb} B per token-head",
-                     "attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
-                     "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak}
-        del g, kc, vc, ws
-        ctx.close()
+    runs = [(name, False) for name in FORMAT_VARIANTS] + [(name, True) for name in FORMAT_VARIANTS]
+    for name, f16 in runs:
+        label = name + ("+fp16norms" if f16 else "")
+        try:
+            out[label] = _variant_once(tq, tq_inputs, torch, dev, hbm_peak, shape, name, f16, steps, warmup)
+        except Exception as e:   # a failed extra must not cost the headline line
+            out[label] = {"error": f"{type(e).__name__}: {e}"}
     torch.cuda.empty_cache()
     return out
+
+
+def _variant_once(tq, tq_inputs, torch, dev, hbm_peak, shape, name, f16, steps, warmup):
+    """One format: cache build (untimed), then graph replays of tq_attn_decode."""
+    B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
+    ctx = tq.Context.variant(name, d, 0, norm_f16=f16)
+    kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
+    vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+    for b in range(B):
+        K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
+        V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+        ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
+        ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+        del K, V
+    q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    o = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    kb, vb = ctx.key_layout["bytes_per_vector"], ctx.value_layout["bytes_per_vector"]
+    alg = B * Hkv * T * (kb + vb) + B * Hq * d * 2 + B * Hq * d * 4
+    bits_k, bits_v, _, nc = tq.VARIANTS[name]
+    res = {"kv_format": f"keys {bits_k} Lloyd-Max bits, values {bits_v} bits, MSE only"
+                        f"{', norm-corrected' if nc else ''}{', binary16 norms' if f16 else ''}; "
+                        f"{kb + vb} B per token-head",
+           "attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
+           "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak}
+    del g, kc, vc, ws
+    ctx.close()
+    return res
 
 
 def small_case(tq, tq_inputs, torch, dev, reps=50):
