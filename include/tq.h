@@ -181,7 +181,7 @@ int tq_export_tables(const tq_ctx* ctx, double* pi, double* S, double* ck,
  *           ld >= d; rows 16-byte aligned when dtype is 16-bit and ld%8==0.
  *   codes   device, uint32 [n][W].
  *   qjl     device, uint32 [n][ceil(m/32)] (keys with QJL; else ignored, may be NULL).
- *   norm    device, float [n].
+ *   norm    device, float [n] (binary16 under TQ_NORM_F16).
  *   rnorm   device, float [n] (keys with QJL; else ignored, may be NULL).
  * n = 0 is a no-op.  A zero vector gets norm 0, every index 2^bits/2, rnorm 0.
  * Inputs must be finite with |x|^2 representable in fp32.
@@ -262,8 +262,10 @@ size_t tq_attn_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int64_t max_T);
  * log-sum-exp and the Pi^T is applied once per head after the merge.
  *   q        device, [B][Hq][d] of `dtype`.
  *   kcodes   device, uint32 [B][Hkv][max_T][Wk]; kqjl [B][Hkv][max_T][ceil(m/32)];
- *   knorm, krnorm  device, float [B][Hkv][max_T].
- *   vcodes   device, uint32 [B][Hkv][max_T][Wv]; vnorm float [B][Hkv][max_T].
+ *   knorm, krnorm  device, float [B][Hkv][max_T] (knorm binary16 under
+ *            TQ_NORM_F16).
+ *   vcodes   device, uint32 [B][Hkv][max_T][Wv]; vnorm float [B][Hkv][max_T]
+ *            (binary16 under TQ_NORM_F16).
  *   seq_lens device, int32 [B], each in [0, max_T]; a length of 0 gives out = 0.
  *   scale    softmax scale (callers usually pass 1/sqrt(d)).
  *   out      device, float [B][Hq][d].
