@@ -35,7 +35,8 @@ def test_library_exports_every_declared_symbol():
 
 @pytest.mark.parametrize("d,bits_k,bits_v,m,seed", [
     (128, 3, 4, 128, 0), (128, 4, 4, 128, 1), (200, 4, 3, 200, 0), (64, 2, 1, 0, 9),
-    (8, 5, 2, 32, 3), (256, 5, 4, 256, 2), (96, 3, 3, 64, 12345678901234), (128, 8, 4, 0, 4)])
+    (8, 5, 2, 32, 3), (256, 5, 4, 256, 2), (96, 3, 3, 64, 12345678901234), (128, 8, 4, 0, 4),
+    (64, 2, 8, 32, 6)])
 def test_host_tables_match_oracle(d, bits_k, bits_v, m, seed):
     h = tq.tq_host_tables(d, bits_k, bits_v, m, seed)
     ot = o.make_tables(d, bits_k, bits_v, m, seed)
