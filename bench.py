@@ -183,9 +183,11 @@ def oracle_decode_sample(w, kc_host, vc_host, q_host, tab):
                        kc_host.get("rnorm"), vc_host["codes"], vc_host["norm"], [T], 1)
 
 
-def cpu_baseline_from_device(w, ctx, kc, vc, q, budget_s: float = 10.0):
+def cpu_baseline_from_device(w, ctx, kc, vc, q, gpu_out, budget_s: float = 10.0):
     """The fp64 oracle on whole (sequence, kv head) slices of the bench's own
-    cache, one after another until about budget_s seconds of CPU work."""
+    cache, one after another until about budget_s seconds of CPU work.  The
+    same oracle outputs are compared with the GPU's attention output for
+    these slices (gpu_out: host [B, Hq, d] from the same query and cache)."""
     import numpy as np
     import torch
     from oracle import tq_oracle as o
@@ -199,26 +201,74 @@ def cpu_baseline_from_device(w, ctx, kc, vc, q, budget_s: float = 10.0):
         return a.numpy().view(np.uint32) if a.dtype == torch.int32 else a.numpy()
 
     tab = o.make_tables(w["d"], w["bits_k"], w["bits_v"], w["m"], 0)
-    slices, dt = 0, 0.0
+    slices, dt, worst = 0, 0.0, 0.0
     for b in range(w["B"]):
         for h in range(w["Hkv"]):
             kh = {k: host(v, b, h) for k, v in kc.items()}
             vh = {k: host(v, b, h) for k, v in vc.items()}
             qh = q[b:b + 1, h * G:(h + 1) * G].float().cpu().numpy().astype(np.float64)
             t0 = time.perf_counter()
-            oracle_decode_sample(w, kh, vh, qh, tab)
+            ref = oracle_decode_sample(w, kh, vh, qh, tab)
             dt += time.perf_counter() - t0
+            got = gpu_out[b, h * G:(h + 1) * G].astype(np.float64)
+            rel = np.linalg.norm(got - ref[0], axis=-1) / np.linalg.norm(ref[0], axis=-1)
+            worst = max(worst, float(rel.max()))
             slices += 1
             if dt >= budget_s:
                 break
         if dt >= budget_s:
             break
     tokens_equiv = slices * T / w["Hkv"]   # Hkv slices of T tokens make T full-width KV tokens
-    return {"value": tokens_equiv / dt, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+    base = {"value": tokens_equiv / dt, "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
             "kind": "oracle",
             "sample": f"fp64 oracle attention of the {G} query heads of {slices} (sequence, kv head) slices "
                       f"of {T} packed tokens ({dt:.1f} s); tokens/s counts {w['Hkv']} slices as {T} "
                       f"full-width KV tokens"}
+    attn = {"pairs": slices * G, "max_rel_l2": worst, "tol": 2e-3, "ok": worst <= 2e-3,
+            "sample": f"the GPU attention output of the same {slices} (sequence, kv head) slices "
+                      f"against the oracle's (same query, same packed cache)"}
+    return base, attn
+
+
+def code_parity(w, kc, vc, xs):
+    """Excused-index counts: the oracle quantizes the sampled input slices
+    (bf16 K/V kept on the host when the cache was built) and compares its
+    indices and QJL bits with the cache's codes for the same tokens.  An index
+    may differ only within 1e-5 of a decision boundary on the rotated
+    unit-vector scale; the counts also give the in-band fraction on the
+    standardized sqrt(d) scale."""
+    import numpy as np
+    import torch
+    from oracle import tq_oracle as o
+    tab = o.make_tables(w["d"], w["bits_k"], w["bits_v"], w["m"], 0)
+
+    def host(t, b, h, n):
+        if t is None:
+            return None
+        a = t[b, h, :n].cpu()
+        return a.numpy().view(np.uint32) if a.dtype == torch.int32 else a.numpy()
+
+    out = {}
+    for which, cache in (("k", kc), ("v", vc)):
+        tot = {}
+        for (b, h), (xk, xv) in xs.items():
+            x = (xk if which == "k" else xv).astype(np.float64)
+            n = x.shape[0]
+            c = o.code_agreement(tab, which, x, host(cache["codes"], b, h, n),
+                                 host(cache.get("qjl"), b, h, n))
+            for k, v in c.items():
+                tot[k] = tot.get(k, 0) + v
+        tot["excused_frac"] = tot["mismatches"] / tot["indices"]
+        tot["in_band_unit_frac"] = tot["in_band_unit"] / tot["indices"]
+        tot["in_band_std_frac"] = tot["in_band_std"] / tot["indices"]
+        tot["ok"] = tot["outside_band"] == 0 and tot["excused_frac"] <= 1e-4 and \
+            tot.get("qjl_outside_band", 0) == 0
+        out["keys" if which == "k" else "values"] = tot
+    n = sum(x[0].shape[0] for x in xs.values())
+    out["sample"] = (f"{n} K and {n} V vectors: tokens [0, {n // len(xs)}) of (sequence, kv head) "
+                     f"{', '.join(str(k) for k in xs)}; band 1e-5 on the unit scale "
+                     f"(standardized scale: 1e-5 / sqrt(d))")
+    return out
 
 
 def run_reference(args, w):
@@ -484,11 +534,18 @@ def run_gpu(args, w):
     # Build the packed cache (setup, not timed): bf16 K/V with outlier channels.
     kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
     vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+    # Inputs of two sampled (sequence, kv head) slices stay on the host for the
+    # oracle's code check (tokens below T - 1, which the timed steps rewrite).
+    nsample = min(16384, T - 1)
+    keep = {(0, 0): None, (B - 1, Hkv - 1): None}
     for b in range(B):
         K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
         V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
         ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
         ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+        for (kb, kh) in keep:
+            if kb == b:
+                keep[(kb, kh)] = (K[kh, :nsample].float().cpu().numpy(), V[kh, :nsample].float().cpu().numpy())
         del K, V
     torch.cuda.synchronize()
     POOL = 8  # distinct step inputs, reused round-robin
@@ -619,9 +676,13 @@ def run_gpu(args, w):
 
     t_ms, attn_ms, e2e_ms = max_over_ranks([t_ms, attn_ms, e2e_ms], world, dev)
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline_from_device(w, ctx, kc, vc, qs[0])
+        ctx.attn_decode(qs[0], kc, vc, lens, out=out, workspace=ws)
+        gpu_out = out.cpu().numpy()
+        cpu, attn_parity = cpu_baseline_from_device(w, ctx, kc, vc, qs[0], gpu_out)
+        parity = code_parity(w, kc, vc, keep)
+        parity["attention"] = attn_parity
 
     if rank == 0:
         kvb = kv_bytes(w, ctx)
@@ -652,6 +713,7 @@ def run_gpu(args, w):
             line["format_variants_decode"] = variants
         if cpu is not None:
             line["cpu_baseline"] = cpu
+            line["parity"] = parity
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

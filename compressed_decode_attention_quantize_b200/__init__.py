@@ -210,6 +210,16 @@ class Context:
     def layout(self, which: int) -> dict:
         return self.key_layout if which == TQ_KEY else self.value_layout
 
+    def _norm(self, which: int, packed: dict):
+        """The packed dict's norm array, refused unless it holds this
+        context's norm type (fp32, or binary16 under TQ_NORM_F16): the C ABI
+        takes norms as untyped pointers and cannot tell them apart."""
+        t = packed["norm"]
+        want = torch.float16 if self.layout(which)["norm_bytes"] == 2 else torch.float32
+        if t.dtype != want:
+            raise TQError(TQ_ERR_ARG, f"norm array of dtype {t.dtype}; this context stores {want} norms")
+        return t
+
     def tables(self):
         import numpy as np
         d, kl = self.d, self.key_layout
@@ -246,7 +256,7 @@ class Context:
             raise TQError(TQ_ERR_ARG, "x must have a unit inner stride")
         n = x2.shape[0]
         _check(_lib.tq_quantize(self.ptr, which, _ptr(x2), _DTYPES[x.dtype], n, x2.stride(0),
-                                _ptr(packed["codes"]), _ptr(packed["qjl"]), _ptr(packed["norm"]),
+                                _ptr(packed["codes"]), _ptr(packed["qjl"]), _ptr(self._norm(which, packed)),
                                 _ptr(packed["rnorm"]), _stream(stream)))
         return packed
 
@@ -263,7 +273,7 @@ class Context:
         max_T = cache["norm"].shape[2]
         _check(_lib.tq_quantize_append(self.ptr, which, _ptr(x), _DTYPES[x.dtype], B, H,
                                        x.stride(1), max_T, _ptr(pos), _ptr(cache["codes"]),
-                                       _ptr(cache["qjl"]), _ptr(cache["norm"]), _ptr(cache["rnorm"]),
+                                       _ptr(cache["qjl"]), _ptr(self._norm(which, cache)), _ptr(cache["rnorm"]),
                                        _stream(stream)))
         return cache
 
@@ -273,7 +283,7 @@ class Context:
             out = torch.empty(packed["norm"].shape + (self.d,), dtype=torch.float32,
                               device=packed["norm"].device)
         _check(_lib.tq_dequantize(self.ptr, which, _ptr(packed["codes"]), _ptr(packed["qjl"]),
-                                  _ptr(packed["norm"]), _ptr(packed["rnorm"]), n, _ptr(out),
+                                  _ptr(self._norm(which, packed)), _ptr(packed["rnorm"]), n, _ptr(out),
                                   _stream(stream)))
         return out
 
@@ -283,7 +293,7 @@ class Context:
         if out is None:
             out = torch.empty(q2.shape[0], nk, dtype=torch.float32, device=q.device)
         _check(_lib.tq_logits(self.ptr, _ptr(q2), _DTYPES[q.dtype], q2.shape[0],
-                              _ptr(keys["codes"]), _ptr(keys["qjl"]), _ptr(keys["norm"]),
+                              _ptr(keys["codes"]), _ptr(keys["qjl"]), _ptr(self._norm(TQ_KEY, keys)),
                               _ptr(keys["rnorm"]), nk, _ptr(out), _stream(stream)))
         return out
 
@@ -304,8 +314,8 @@ class Context:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _check(_lib.tq_attn_decode(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
-                                   _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(kcache["norm"]),
-                                   _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
+                                   _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(self._norm(TQ_KEY, kcache)),
+                                   _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(self._norm(TQ_VALUE, vcache)),
                                    max_T, _ptr(seq_lens), float(scale), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
         return out
@@ -329,8 +339,8 @@ class Context:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _check(_lib.tq_decode_step(self.ptr, _ptr(q), _DTYPES[q.dtype], _ptr(k_new), _ptr(v_new),
                                    _DTYPES[k_new.dtype], B, Hq, Hkv, _ptr(kcache["codes"]),
-                                   _ptr(kcache["qjl"]), _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
-                                   _ptr(vcache["codes"]), _ptr(vcache["norm"]), max_T, _ptr(pos),
+                                   _ptr(kcache["qjl"]), _ptr(self._norm(TQ_KEY, kcache)), _ptr(kcache["rnorm"]),
+                                   _ptr(vcache["codes"]), _ptr(self._norm(TQ_VALUE, vcache)), max_T, _ptr(pos),
                                    float(scale), _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
         return out
@@ -348,7 +358,7 @@ class Context:
         _check(_lib.tq_quantize_append_paged(self.ptr, which, _ptr(x), _DTYPES[x.dtype], B, H, x.stride(1),
                                              _ptr(block_table), block_table.shape[1], bs, nb, _ptr(pos),
                                              _ptr(cache["codes"]), _ptr(cache.get("qjl")),
-                                             _ptr(cache["norm"]), _ptr(cache.get("rnorm")), _stream(stream)))
+                                             _ptr(self._norm(which, cache)), _ptr(cache.get("rnorm")), _stream(stream)))
         return cache
 
     def attn_decode_paged(self, q: torch.Tensor, kcache: dict, vcache: dict, block_table: torch.Tensor,
@@ -366,8 +376,8 @@ class Context:
             workspace = torch.empty(self.attn_workspace_bytes(B, Hq, mb * bs), dtype=torch.uint8,
                                     device=q.device)
         _check(_lib.tq_attn_decode_paged(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
-                                         _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(kcache["norm"]),
-                                         _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(vcache["norm"]),
+                                         _ptr(kcache["codes"]), _ptr(kcache["qjl"]), _ptr(self._norm(TQ_KEY, kcache)),
+                                         _ptr(kcache["rnorm"]), _ptr(vcache["codes"]), _ptr(self._norm(TQ_VALUE, vcache)),
                                          _ptr(block_table), mb, bs, nb, _ptr(seq_lens), float(scale),
                                          _ptr(out), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -391,8 +401,8 @@ class Context:
                                     device=q.device)
         _check(_lib.tq_decode_step_paged(self.ptr, _ptr(q), _DTYPES[q.dtype], _ptr(k_new), _ptr(v_new),
                                          _DTYPES[k_new.dtype], B, Hq, Hkv, _ptr(kcache["codes"]),
-                                         _ptr(kcache["qjl"]), _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
-                                         _ptr(vcache["codes"]), _ptr(vcache["norm"]), _ptr(block_table), mb,
+                                         _ptr(kcache["qjl"]), _ptr(self._norm(TQ_KEY, kcache)), _ptr(kcache["rnorm"]),
+                                         _ptr(vcache["codes"]), _ptr(self._norm(TQ_VALUE, vcache)), _ptr(block_table), mb,
                                          bs, nb, _ptr(pos), float(scale), _ptr(out), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(stream)))
         return out
@@ -410,8 +420,8 @@ class Context:
             out = torch.empty(B, Hq, d, dtype=torch.float32, device=q.device)
         _check(_lib.tq_attn_decode_static(self.ptr, _ptr(q), _DTYPES[q.dtype], B, Hq, Hkv,
                                           _ptr(kcache["codes"]), _ptr(kcache["qjl"]),
-                                          _ptr(kcache["norm"]), _ptr(kcache["rnorm"]),
-                                          _ptr(vcache["codes"]), _ptr(vcache["norm"]), max_T,
+                                          _ptr(self._norm(TQ_KEY, kcache)), _ptr(kcache["rnorm"]),
+                                          _ptr(vcache["codes"]), _ptr(self._norm(TQ_VALUE, vcache)), max_T,
                                           _ptr(seq_lens), float(scale), _ptr(out), _stream(stream)))
         return out
 
@@ -428,6 +438,6 @@ class Context:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _check(_lib.tq_topk(self.ptr, _ptr(q2), _DTYPES[q.dtype], nq, _ptr(db["codes"]),
-                            _ptr(db["qjl"]), _ptr(db["norm"]), _ptr(db["rnorm"]), n, k, _ptr(idx),
+                            _ptr(db["qjl"]), _ptr(self._norm(TQ_KEY, db)), _ptr(db["rnorm"]), n, k, _ptr(idx),
                             _ptr(score), _ptr(workspace), workspace.numel(), _stream(stream)))
         return idx, score

@@ -61,6 +61,19 @@ int check_ctx(const tq_ctx* c) {
   return TQ_OK;
 }
 
+// Compute calls launch on the current device, and the context's tables live
+// on the device it was created on: a mismatch is refused before any launch.
+int check_ctx_dev(const tq_ctx* c, const char* name) {
+  if (!c) return fail(TQ_ERR_ARG, "%s: null context", name);
+  int cur = -1;
+  const cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  if (cur != c->device)
+    return fail(TQ_ERR_ARG, "%s: the context belongs to device %d but device %d is current", name,
+                c->device, cur);
+  return TQ_OK;
+}
+
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
@@ -328,7 +341,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
                            uint32_t* codes, uint32_t* qjl, void* norm, float* rnorm,
                            const int32_t* pos, int H, int64_t max_T, void* stream,
                            const char* name, const Paging& pg = Paging()) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, name)) return r;
   if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "%s: bad which=%d", name, which);
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
     return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dtype);
@@ -339,7 +352,8 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
   const int m = key ? c->qjl_m : 0;
   if (!x || !codes || !norm) return fail(TQ_ERR_ARG, "%s: null pointer", name);
   if (m > 0 && (!qjl || !rnorm)) return fail(TQ_ERR_ARG, "%s: keys with QJL need qjl and rnorm", name);
-  if (!aligned(codes, 4) || !aligned(norm, 4)) return fail(TQ_ERR_ARG, "%s: misaligned output", name);
+  if (!aligned(codes, 4) || !aligned(norm, c->norm_f16 ? 2 : 4))
+    return fail(TQ_ERR_ARG, "%s: misaligned output", name);
   tqk::QuantArgs a{};
   a.x = x;
   a.dtype = dtype;
@@ -442,7 +456,7 @@ int tq_quantize_append_paged(tq_ctx* c, int which, const void* x, int dtype, int
 
 int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* qjl,
                   const void* norm, const float* rnorm, int64_t n, float* out, void* stream) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, "tq_dequantize")) return r;
   if (which != TQ_KEY && which != TQ_VALUE) return fail(TQ_ERR_ARG, "tq_dequantize: bad which=%d", which);
   if (n < 0) return fail(TQ_ERR_ARG, "tq_dequantize: n < 0");
   if (n == 0) return TQ_OK;
@@ -457,7 +471,7 @@ int tq_dequantize(tq_ctx* c, int which, const uint32_t* codes, const uint32_t* q
 int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* kcodes,
               const uint32_t* kqjl, const void* knorm, const float* krnorm, int64_t nk, float* out,
               void* stream) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, "tq_logits")) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
     return fail(TQ_ERR_ARG, "tq_logits: bad dtype=%d", dtype);
   if (nq < 0 || nk < 0) return fail(TQ_ERR_ARG, "tq_logits: negative size");
@@ -509,7 +523,7 @@ static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, 
                             int64_t max_T, const int32_t* seq_lens, float scale, float* out,
                             void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
                             const char* name) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, name)) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
     return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dtype);
   if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T < 0) return fail(TQ_ERR_ARG, "%s: bad sizes", name);
@@ -621,7 +635,7 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
                             void* vnorm, int64_t max_T, const int32_t* pos, float scale, float* out,
                             void* workspace, size_t ws_bytes, void* stream, const Paging& pg,
                             const char* name) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, name)) return r;
   for (int dt : {q_dtype, kv_dtype})
     if (dt != TQ_F32 && dt != TQ_BF16 && dt != TQ_F16) return fail(TQ_ERR_ARG, "%s: bad dtype=%d", name, dt);
   if (B < 0 || Hq <= 0 || Hkv <= 0 || max_T <= 0) return fail(TQ_ERR_ARG, "%s: bad sizes", name);
@@ -632,7 +646,8 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
     return fail(TQ_ERR_ARG, "%s: null pointer", name);
   if (c->qjl_m > 0 && (!kqjl || !krnorm)) return fail(TQ_ERR_ARG, "%s: keys with QJL need kqjl and krnorm", name);
   if (B > 65535 || Hkv > 65535) return fail(TQ_ERR_UNSUPPORTED, "%s: B or Hkv too large", name);
-  if (!aligned(kcodes, 4) || !aligned(knorm, 4) || !aligned(vcodes, 4) || !aligned(vnorm, 4))
+  if (!aligned(kcodes, 4) || !aligned(knorm, c->norm_f16 ? 2 : 4) || !aligned(vcodes, 4) ||
+      !aligned(vnorm, c->norm_f16 ? 2 : 4))
     return fail(TQ_ERR_ARG, "%s: misaligned cache", name);
   const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
   if (!workspace || ws_bytes < need)
@@ -778,7 +793,7 @@ size_t tq_topk_workspace_bytes(const tq_ctx* c, int64_t nq, int64_t n, int k) {
 int tq_topk(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* codes,
             const uint32_t* qjl, const void* norm, const float* rnorm, int64_t n, int k,
             int32_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
-  if (int r = check_ctx(c)) return r;
+  if (int r = check_ctx_dev(c, "tq_topk")) return r;
   if (dtype != TQ_F32 && dtype != TQ_BF16 && dtype != TQ_F16)
     return fail(TQ_ERR_ARG, "tq_topk: bad dtype=%d", dtype);
   if (nq < 0 || n < 0 || k < 1 || k > 32) return fail(TQ_ERR_ARG, "tq_topk: bad sizes (k must be 1..32)");
@@ -849,7 +864,9 @@ extern "C" int tq_attn_decode_static(tq_ctx* c, const void* q, int dtype, int B,
                                      const uint32_t* vcodes, const void* vnorm, int64_t max_T,
                                      const int32_t* seq_lens, float scale, float* out,
                                      void* stream) {
-  if (int r = check_ctx(c)) return r;
+  // The scratch address below is the current device's: refuse a context of
+  // another device first.
+  if (int r = check_ctx_dev(c, "tq_attn_decode_static")) return r;
   const size_t need = tq_attn_workspace_bytes(c, B, Hq, max_T);
   if (need > kStaticScratchBytes)
     return fail(TQ_ERR_WORKSPACE,

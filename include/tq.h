@@ -23,6 +23,12 @@
  * - Pointers marked "device" are CUDA device pointers on the context's device,
  *   allocated and owned by the caller; the library never frees or keeps them.
  *   `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * - Compute calls (quantize, dequantize, logits, attention, decode step,
+ *   top-k) launch on the current device, which must be the context's device
+ *   (the one current at tq_init); otherwise they return TQ_ERR_ARG before any
+ *   launch.
+ * - Norm arrays are 4-byte aligned fp32, or 2-byte aligned binary16 under
+ *   TQ_NORM_F16; code and QJL arrays are 4-byte aligned.
  * - Compute calls only enqueue kernels on `stream`: they neither allocate,
  *   synchronise, nor fall back to the CPU.  Scratch memory comes from the
  *   caller's `workspace` (device, at least the size the *_workspace_bytes

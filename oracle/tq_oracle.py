@@ -285,7 +285,7 @@ def make_tables(d: int, bits_k: int, bits_v: int, qjl_m: int, seed: int,
 # ----------------------------------------------------------------------------
 # Bit packing (the library's own layout; the pages only say the fused kernel
 # reads the indices directly).  A vector's Lloyd-Max indices are packed as
-# b-bit fields, LSB first, 32/b fields per uint32 word, for b in {1, 2, 4}:
+# b-bit fields, LSB first, 32/b fields per uint32 word, for b in {1, 2, 4, 8}:
 # coordinate j sits in word j // (32/b) at bit b * (j % (32/b)).  For b = 3
 # the low two bits of every index form a 2-bit field stream and the top bit a
 # 1-bit stream that follows it.  Padding bits are zero.  QJL bits form a 1-bit
@@ -355,11 +355,6 @@ def lloyd_max_index(y: np.ndarray, cb: Codebook) -> np.ndarray:
     return (y[..., None] >= cb.boundaries).sum(axis=-1).astype(np.int64)
 
 
-def qjl_signs(S: np.ndarray, r: np.ndarray) -> np.ndarray:
-    """sigma = sign(S r) with sign(0) = +1 (R6), returned as 0/1 bits."""
-    return (r @ S.T >= 0.0).astype(np.int64)
-
-
 @dataclass
 class Quantized:
     idx: np.ndarray        # [N, d] int64 Lloyd-Max indices
@@ -404,8 +399,8 @@ def corrected_norm(n: np.ndarray, idx: np.ndarray, cb: Codebook) -> np.ndarray:
 
 
 def sketch_from_indices(q: Quantized, tab: Tables, idx: np.ndarray | None = None) -> None:
-    """[WHAT] stage 2: residual r = y - c[idx], rho = |r|, sigma = sign(S r),
-    gamma = n rho.  `idx` overrides the indices (used to rebuild the sketch
+    """[WHAT] stage 2: residual r = y - c[idx], rho = |r|, sigma = sign(S r)
+    with sign(0) = +1 (R6, stored as bit 1), gamma = n rho.  `idx` overrides the indices (used to rebuild the sketch
     for codes produced elsewhere)."""
     idx = q.idx if idx is None else idx
     r = q.y - tab.cb_k.centroids[idx]
@@ -420,6 +415,47 @@ def sketch_from_indices(q: Quantized, tab: Tables, idx: np.ndarray | None = None
 def boundary_distance(y: np.ndarray, cb: Codebook) -> np.ndarray:
     """|y - nearest decision boundary| on the rotated unit-vector scale."""
     return np.min(np.abs(y[..., None] - cb.boundaries), axis=-1)
+
+
+# ----------------------------------------------------------------------------
+# Agreement counts: another implementation's codes against this oracle.
+# "Within 1e-5 of a decision boundary" is read on the rotated unit-vector
+# scale (the scale on which the Beta law and the boundaries live): an index
+# may differ from the oracle's only when |y_j - beta_i| < band.  The counts
+# also give the in-band fraction on the standardized scale sqrt(d) * y, where
+# the same band is sqrt(d) times narrower.
+# ----------------------------------------------------------------------------
+def code_agreement(tab: Tables, which: str, x: np.ndarray, codes: np.ndarray,
+                   qjl: np.ndarray | None = None, band: float = 1e-5) -> dict:
+    """Counts for codes (and QJL words) produced elsewhere from the rows of x.
+
+    Returns indices, mismatches, mismatches outside the unit-scale band (a
+    real disagreement), in-band counts on the unit and standardized scales,
+    mismatches outside the standardized band, and for keys with QJL the same
+    for the sign bits (band |(S r)_i| < band * |r|, with the sketch rebuilt
+    from the other side's indices).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    cb = tab.cb_k if which == "k" else tab.cb_v
+    n = x.shape[0]
+    q = quantize(x, tab, which)
+    gidx = unpack_codes(np.asarray(codes).reshape(n, -1), cb.bits, tab.d)
+    dist = boundary_distance(q.y, cb)
+    mism = gidx != q.idx
+    in_unit = dist < band
+    in_std = dist < band / math.sqrt(tab.d)
+    out = {"indices": int(mism.size), "mismatches": int(mism.sum()),
+           "outside_band": int(np.sum(mism & ~in_unit)),
+           "in_band_unit": int(in_unit.sum()), "in_band_std": int(in_std.sum()),
+           "mismatches_outside_std_band": int(np.sum(mism & ~in_std))}
+    if which == "k" and tab.qjl_m > 0 and qjl is not None:
+        sketch_from_indices(q, tab, idx=gidx)
+        gbits = unpack_bits(np.asarray(qjl).reshape(n, -1), tab.qjl_m)
+        qm = gbits != q.qjl_bits
+        qband = np.abs(q.proj) < band * q.rho[:, None]
+        out.update(qjl_bits=int(qm.size), qjl_mismatches=int(qm.sum()),
+                   qjl_outside_band=int(np.sum(qm & ~qband)), qjl_in_band=int(qband.sum()))
+    return out
 
 
 # ----------------------------------------------------------------------------

@@ -79,7 +79,10 @@ def check_quantized(tab, which, x, gpu, report=None):
         assert np.all(np.abs(gnorm - want) <= 2.0 ** -10 * want + 1e-30), "norm"
     else:
         assert np.all(np.abs(gnorm - want) <= NORM_RTOL * want + 1e-30), "norm"
-    stats = {"indices": int(mism.size), "excused": n_exc, "band": int(band.sum())}
+    dist = o.boundary_distance(q.y, cb)
+    band_std = dist < BAND / np.sqrt(d)
+    stats = {"indices": int(mism.size), "excused": n_exc, "band": int(band.sum()),
+             "band_std": int(band_std.sum()), "excused_outside_std_band": int(np.sum(mism & ~band_std))}
     if which == "k" and tab.qjl_m > 0:
         o.sketch_from_indices(q, tab, idx=gidx)
         gbits = o.unpack_bits(gpu["qjl"].reshape(n, -1), tab.qjl_m)

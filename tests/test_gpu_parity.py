@@ -443,6 +443,42 @@ def test_errors_are_reported(cuda):
     assert e.value.status == tq.TQ_ERR_ARG
 
 
+def test_norm_dtype_mismatch_is_refused(cuda):
+    """Norms reach the C ABI as untyped pointers, so the binding refuses a norm
+    array of the wrong type (binary16 for an fp32-norm context, and the
+    reverse) before any launch."""
+    c = _ctx(128, 3, 4, 128)
+    K = torch.randn(2, 1, 16, 128, device=cuda)
+    kc, vc = _cache(c, K, K, cuda)
+    q = torch.randn(2, 4, 128, device=cuda)
+    lens = torch.full((2,), 16, dtype=torch.int32, device=cuda)
+    bad = dict(kc, norm=kc["norm"].half())
+    for call in (lambda: c.attn_decode(q, bad, vc, lens), lambda: c.logits(q[0], bad),
+                 lambda: c.dequantize(tq.TQ_KEY, bad), lambda: c.quantize_into(K, tq.TQ_KEY, bad)):
+        with pytest.raises(tq.TQError) as e:
+            call()
+        assert e.value.status == tq.TQ_ERR_ARG
+    c16 = tq.Context.variant("4bit_nc", 128, norm_f16=True)
+    vc16 = c16.quantize(K, tq.TQ_VALUE)
+    with pytest.raises(tq.TQError) as e:
+        c16.dequantize(tq.TQ_VALUE, dict(vc16, norm=vc16["norm"].float()))
+    assert e.value.status == tq.TQ_ERR_ARG
+
+
+def test_context_of_another_device_is_refused(cuda):
+    """A context's tables live on the device current at tq_init; a compute
+    call with another device current is refused before any launch."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    c = _ctx(128, 3, 4, 128)
+    x = torch.randn(4, 128, device="cuda:1")
+    pk = {k: (None if v is None else v.to("cuda:1")) for k, v in c.empty_packed(tq.TQ_KEY, (4,)).items()}
+    with torch.cuda.device(1):
+        with pytest.raises(tq.TQError) as e:
+            c.quantize_into(x, tq.TQ_KEY, pk)
+    assert e.value.status == tq.TQ_ERR_ARG and "device" in str(e.value)
+
+
 def test_quantize_append_writes_addressed_slots(cuda):
     """Only slot pos[b] of each sequence is written; a pos outside [0, T)
     writes nothing."""

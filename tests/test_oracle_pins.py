@@ -240,18 +240,51 @@ def test_packing_worked_example():
         assert codes.dtype == np.uint32 and codes.shape == (1, o.code_words(40, bits))
         assert list(codes[0]) == rows[f"b{bits}"], bits
         assert np.array_equal(o.unpack_codes(codes, bits, 40), idx)
+    # 8-bit codes (the k8v4 format): one byte per coordinate, LSB first
+    idx = (np.arange(40) ^ 0xA0)[None, :]
+    codes = o.pack_codes(idx, 8)
+    assert codes.dtype == np.uint32 and codes.shape == (1, o.code_words(40, 8)) == (1, 10)
+    assert list(codes[0]) == rows["b8"]
+    assert np.array_equal(o.unpack_codes(codes, 8, 40), idx)
 
 
 def test_pack_roundtrip_random():
     rng = np.random.default_rng(1)
-    for bits in (1, 2, 3, 4):
-        for d in (200, 128, 8):
+    for bits in (1, 2, 3, 4, 8):
+        for d in (200, 128, 8, 36):
             idx = rng.integers(0, 1 << bits, size=(50, d))
             assert np.array_equal(o.unpack_codes(o.pack_codes(idx, bits), bits, d), idx)
     bits = rng.integers(0, 2, size=(50, 72))
     w = o.pack_bits(bits)
     assert w.shape == (50, 3) and np.all(w[:, 2] >> np.uint32(8) == 0)
     assert np.array_equal(o.unpack_bits(w, 72), bits)
+
+
+# --- agreement counts used to report excused indices -----------------------------
+def test_code_agreement_counts():
+    """The counting helper: identical codes give no mismatch, a planted
+    mismatch far from every boundary is a real disagreement, and the in-band
+    counts over uniform directions match the integrated density at the
+    boundaries, sum_i 2 band f_d(beta_i) per coordinate, on the unit scale and
+    sqrt(d) times fewer on the standardized scale."""
+    d = 128
+    tab = o.make_tables(d, 3, 2, d, 5)   # keys: 2 Lloyd-Max bits + QJL (m = d); values: 2 bits
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((20000, d))
+    q = o.quantize(x, tab, "k")
+    c = o.code_agreement(tab, "k", x, q.codes, q.qjl)
+    assert c["indices"] == x.size and c["mismatches"] == 0 and c["outside_band"] == 0
+    assert c["qjl_bits"] == x.size and c["qjl_mismatches"] == 0
+    idx = q.idx.copy()
+    far = int(np.argmax(o.boundary_distance(q.y, tab.cb_k).ravel()))
+    r, j = divmod(far, d)
+    idx[r, j] ^= 1
+    c2 = o.code_agreement(tab, "k", x, o.pack_codes(idx, 2))
+    assert (c2["mismatches"], c2["outside_band"], c2["mismatches_outside_std_band"]) == (1, 1, 1)
+    band = 1e-5
+    expect = x.size * float(np.sum(2 * band * o.beta_density(tab.cb_k.boundaries, d)))
+    for got, mean in ((c["in_band_unit"], expect), (c["in_band_std"], expect / math.sqrt(d))):
+        assert abs(got - mean) <= 5 * math.sqrt(mean), (got, mean)
 
 
 # --- R14: zero vector ---------------------------------------------------------
