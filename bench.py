@@ -424,6 +424,66 @@ def variant_decode(tq, tq_inputs, torch, dev, hbm_peak, shape, steps=20, warmup=
     return out
 
 
+def decode_70b(tq, tq_inputs, torch, dev, hbm_peak, steps=20, warmup=3):
+    """The 70B-shaped long-context decode (B=4, Hq=64, Hkv=8, T=131072,
+    GQA 8) in both of its formats: the attention call (pre-rotate, split-K
+    attention, merge) timed like the headline's."""
+    out = {}
+    for name in ("70b-decode-k3v4", "70b-decode-k4v4"):
+        w = WORKLOADS[name]
+        try:
+            ctx = tq.Context(w["d"], w["bits_k"], w["bits_v"], w["m"], 0)
+            res = _decode_call(tq, tq_inputs, torch, dev, hbm_peak, w, ctx, steps, warmup)
+            res["kv_format"] = (f"k{w['bits_k']}v{w['bits_v']}: keys {w['bits_k'] - 1} Lloyd-Max bits + 1 QJL "
+                                f"bit (m={w['m']}), values {w['bits_v']} bits")
+            out[name] = res
+        except Exception as e:   # a failed extra must not cost the headline line
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+    torch.cuda.empty_cache()
+    return out
+
+
+def _decode_call(tq, tq_inputs, torch, dev, hbm_peak, shape, ctx, steps, warmup):
+    """Cache build (untimed), then CUDA-event timing of tq_attn_decode graph
+    replays; returns ms per call, KV tokens/s and the fraction of measured HBM
+    bandwidth on the algorithmic bytes (packed cache + queries + output)."""
+    B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
+    kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
+    vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+    for b in range(B):
+        K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
+        V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+        ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
+        ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+        del K, V
+    q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    o = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ctx.attn_decode(q, kc, vc, lens, out=o, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    kb, vb = ctx.key_layout["bytes_per_vector"], ctx.value_layout["bytes_per_vector"]
+    alg = B * Hkv * T * (kb + vb) + B * Hq * d * 2 + B * Hq * d * 4
+    del g, kc, vc, ws
+    ctx.close()
+    return {"attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
+            "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes": alg,
+            "shape": f"B={B} Hq={Hq} Hkv={Hkv} d={d} T={T}", "timing": f"{steps} CUDA-graph replays"}
+
+
 def _variant_once(tq, tq_inputs, torch, dev, hbm_peak, shape, name, f16, steps, warmup):
     """One format: cache build (untimed), then graph replays of tq_attn_decode."""
     B, Hq, Hkv, d, T = shape["B"], shape["Hq"], shape["Hkv"], shape["d"], shape["T"]
@@ -623,23 +683,37 @@ def run_gpu(args, w):
     sampler.mark(w0, time.time())
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
 
-    # End to end through the public API with host buffers: pinned host inputs
-    # copied in and the output copied out inside the timed region (captured
-    # with the kernels in one graph per input slot).
+    # End to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory and reads its output back, inside the
+    # timed region.  The copies run on a side stream beside the kernels (two
+    # buffer sets): the graph of step j copies step j+1's inputs in and step
+    # j-1's output out while step j attends; graphs replay in order, so each
+    # buffer is free when it is reused.
     hq = [x.cpu().pin_memory() for x in qs]
     hk = [x.cpu().pin_memory() for x in kn]
     hv = [x.cpu().pin_memory() for x in vn]
-    hout = torch.empty(B, Hq, d, dtype=torch.float32).pin_memory()
-    dq, dk, dv = torch.empty_like(qs[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    hout = [torch.empty(B, Hq, d, dtype=torch.float32).pin_memory() for _ in range(POOL)]
+    dq = [torch.empty_like(qs[0]) for _ in range(2)]
+    dk = [torch.empty_like(kn[0]) for _ in range(2)]
+    dv = [torch.empty_like(vn[0]) for _ in range(2)]
+    dout = [torch.empty(B, Hq, d, dtype=torch.float32, device=dev) for _ in range(2)]
+    side = torch.cuda.Stream(device=dev)
 
     def e2e_body(j):
-        dq.copy_(hq[j], non_blocking=True)
-        dk.copy_(hk[j], non_blocking=True)
-        dv.copy_(hv[j], non_blocking=True)
-        ctx.decode_step(dq, dk, dv, kc, vc, pos, out=out, workspace=ws)
-        hout.copy_(out, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        side.wait_stream(cur)
+        with torch.cuda.stream(side):
+            n, nb, pb = (j + 1) % POOL, (j + 1) % 2, (j - 1) % 2
+            dq[nb].copy_(hq[n], non_blocking=True)
+            dk[nb].copy_(hk[n], non_blocking=True)
+            dv[nb].copy_(hv[n], non_blocking=True)
+            hout[(j - 1) % POOL].copy_(dout[pb], non_blocking=True)
+        ctx.decode_step(dq[j % 2], dk[j % 2], dv[j % 2], kc, vc, pos, out=dout[j % 2], workspace=ws)
+        cur.wait_stream(side)
 
-    e2e_body(0)
+    dq[0].copy_(hq[0])
+    dk[0].copy_(hk[0])
+    dv[0].copy_(hv[0])
     torch.cuda.synchronize()
     g_e2e = []
     for j in range(POOL):
@@ -652,27 +726,30 @@ def run_gpu(args, w):
     barrier()
     w0 = time.time()
     e0.record()
-    for i in range(args.steps):
+    for i in range(args.warmup, args.warmup + args.steps):
         g_e2e[i % POOL].replay()
+    last = args.warmup + args.steps - 1
+    hout[last % POOL].copy_(dout[last % 2], non_blocking=True)   # the last step's output
     e1.record()
     barrier()
     sampler.mark(w0, time.time())
     e2e_ms = e0.elapsed_time(e1) / args.steps
     h2d = hq[0].numel() * hq[0].element_size() + 2 * hk[0].numel() * hk[0].element_size()
-    d2h = hout.numel() * hout.element_size()
+    d2h = hout[0].numel() * hout[0].element_size()
     del g_step, g_att, g_e2e
 
     torch.cuda.nvtx.range_push("tq:quantize_sweep")
     quant = quantize_sweep(tq, tq_inputs, torch, dev, hbm_peak)
     torch.cuda.nvtx.range_pop()
     clocks = sampler.stop()
-    vsearch = small = variants = None
+    vsearch = small = variants = d70 = None
     if not args.skip_extra:
         torch.cuda.nvtx.range_push("tq:vector_search")
         vsearch = vector_search(tq, tq_inputs, torch, dev, clocks.get("sm_max_mhz") or 1965.0)
         torch.cuda.nvtx.range_pop()
         small = small_case(tq, tq_inputs, torch, dev)
         variants = variant_decode(tq, tq_inputs, torch, dev, hbm_peak, WORKLOADS["llama3-8b-decode"])
+        d70 = decode_70b(tq, tq_inputs, torch, dev, hbm_peak)
 
     t_ms, attn_ms, e2e_ms = max_over_ranks([t_ms, attn_ms, e2e_ms], world, dev)
 
@@ -692,7 +769,9 @@ def run_gpu(args, w):
         line = {
             "metric": METRIC, "value": whole_job_rate(B * T, world, t_ms), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 key-bit x 4-limb query MMA + fp16 value MMA, fp32 accumulate and softmax",
+            "data": "synthetic",
             "config": config_of(args, w),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic,
@@ -702,7 +781,9 @@ def run_gpu(args, w):
                          "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                          "frac_of_nominal_8tbs": achieved / 8000.0},
             "e2e": {"value": whole_job_rate(B * T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "copies": "pinned host <-> device on a side stream, overlapped with the previous / next "
+                              "step's kernels (two buffer sets), all inside the timed region"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "quantize": quant,
@@ -711,6 +792,7 @@ def run_gpu(args, w):
             line["vector_search"] = vsearch
             line["small_case"] = small
             line["format_variants_decode"] = variants
+            line["decode_70b"] = d70
         if cpu is not None:
             line["cpu_baseline"] = cpu
             line["parity"] = parity
@@ -718,6 +800,78 @@ def run_gpu(args, w):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_case(args):
+    """One library call on a synthetic case, repeated (for profilers: a small
+    case of one kernel).  Prints the mean CUDA-event time per call and the
+    algorithmic bytes per call."""
+    import torch
+    import compressed_decode_attention_quantize_b200 as tq
+    import tq_inputs
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.case == "decode":
+        w = dict(WORKLOADS[args.workload])
+        for k in ("B", "T"):
+            if getattr(args, k) is not None:
+                w[k] = getattr(args, k)
+        B, Hq, Hkv, d, T = w["B"], w["Hq"], w["Hkv"], w["d"], w["T"]
+        ctx = tq.Context(d, w["bits_k"], w["bits_v"], w["m"], 0)
+        kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
+        vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+        for b in range(B):
+            K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
+            V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+            ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
+            ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+            del K, V
+        q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
+        lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+        out = torch.empty(B, Hq, d, device=dev)
+        ws = torch.empty(ctx.attn_workspace_bytes(B, Hq, T), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: ctx.attn_decode(q, kc, vc, lens, out=out, workspace=ws))
+        byts = kv_bytes(w, ctx)
+        desc = f"{args.workload} B={B} T={T}"
+    elif args.case == "quantize":
+        n = args.n or (1 << 20)
+        m = args.d if args.qjl else 0
+        ctx = tq.Context(args.d, args.bits, args.bits, m, 0)
+        if args.d == 128:
+            X = tq_inputs.outlier_kv(1, 8, n // 8, args.d, seed=31, device=dev)[0].reshape(-1, args.d)
+        else:
+            X = tq_inputs.mixture(n, args.d, seed=21, device=dev)
+        pk = ctx.empty_packed(tq.TQ_KEY, (X.shape[0],), device=dev)
+        ms = timed(lambda: ctx.quantize_into(X, tq.TQ_KEY, pk))
+        byts = X.shape[0] * (args.d * X.element_size() + ctx.key_layout["bytes_per_vector"])
+        desc = f"n={X.shape[0]} d={args.d} bits={args.bits} qjl={args.qjl}"
+    else:
+        s = VSEARCH
+        n = args.n or s["n"]
+        ctx = tq.Context(s["d"], s["bits_k"], 3, s["m"], 0)
+        X = tq_inputs.mixture(n, s["d"], seed=21, device=dev)
+        Q = tq_inputs.mixture(args.nq, s["d"], seed=22, means_seed=21, device=dev)
+        db = ctx.quantize(X, tq.TQ_KEY)
+        ws = torch.empty(ctx.topk_workspace_bytes(args.nq, n, s["k"]), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: ctx.topk(Q, db, s["k"], workspace=ws))
+        byts = n * ctx.key_layout["bytes_per_vector"]
+        desc = f"n={n} nq={args.nq} d={s['d']} k={s['k']}"
+    print(json.dumps({"case": args.case, "config": desc, "ms_per_call": ms, "bytes_per_call": byts,
+                      "gbs": byts / (ms / 1e3) / 1e9}), flush=True)
     return 0
 
 
@@ -730,9 +884,21 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--skip-extra", dest="skip_extra", action="store_true",
                     help="omit the vector-search and small-case measurements")
+    ap.add_argument("--case", choices=["decode", "quantize", "topk"],
+                    help="profiling case: one library call repeated (--steps times after --warmup), "
+                         "no JSON bench line")
+    ap.add_argument("--B", type=int, help="--case decode: batch (default: the workload's)")
+    ap.add_argument("--T", type=int, help="--case decode: context (default: the workload's)")
+    ap.add_argument("--n", type=int, help="--case quantize / topk: vectors")
+    ap.add_argument("--nq", type=int, default=1000, help="--case topk: queries")
+    ap.add_argument("--d", type=int, default=128, help="--case quantize: dimension")
+    ap.add_argument("--bits", type=int, default=3, help="--case quantize: bits (keys count the QJL bit)")
+    ap.add_argument("--qjl", type=int, default=1, help="--case quantize: QJL stage (m = d) on/off")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

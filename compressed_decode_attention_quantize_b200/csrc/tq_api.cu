@@ -485,14 +485,15 @@ int tq_logits(tq_ctx* c, const void* q, int dtype, int64_t nq, const uint32_t* k
   return TQ_OK;
 }
 
-// Workspace: [q' and S q' rows][tile prefix][step lengths][partials].  The partials are
+// Workspace: [q' and S q' rows][tile prefix][step lengths][int8 query-operand
+// images, one per (sequence, kv head), sized for B Hq][partials].  The partials are
 // sized for the larger of the split layout ([B Hq][splits][dpad + 2]) and
 // the segment layouts: [warps + B Hkv][G][dpad + 2] for groups up to 4, and
 // [4 (CTAs + B Hkv)][8][dpad + 2] for group 8; both are at most
 // [8 warps + 4 B Hq][dpad + 2].
 namespace {
 struct AttnWs {
-  size_t q_bytes, tiles_off, lens_off, part_off, total;
+  size_t q_bytes, tiles_off, lens_off, qimg_off, part_off, total;
 };
 AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   int chunk = 0;
@@ -506,7 +507,8 @@ AttnWs attn_ws_layout(const tq_ctx* c, int B, int Hq, int64_t max_T) {
   w.q_bytes = 2 * rows * c->dpad * sizeof(float);
   w.tiles_off = (w.q_bytes + 255) & ~(size_t)255;
   w.lens_off = (w.tiles_off + ((size_t)B + 1) * sizeof(int64_t) + 255) & ~(size_t)255;
-  w.part_off = (w.lens_off + (size_t)B * sizeof(int32_t) + 255) & ~(size_t)255;
+  w.qimg_off = (w.lens_off + (size_t)B * sizeof(int32_t) + 255) & ~(size_t)255;
+  w.part_off = (w.qimg_off + rows * (size_t)tqk::kQopBytes + 255) & ~(size_t)255;
   w.total = w.part_off + (split_part > seg_part ? split_part : seg_part) + 256;
   return w;
 }
@@ -578,20 +580,29 @@ static int attn_decode_impl(tq_ctx* c, const void* q, int dtype, int B, int Hq, 
   a.max_blocks = pg.max_blocks;
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
-  const bool mma = tqk::attn_mma_supported(c, a) && max_T > 0;
-  const bool lut = !mma && tqk::attn_lut_supported(c, a) && max_T > 0;
-  if (pg.table && !(mma || lut))
-    return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode (d = 128, QJL m = 128, "
-                "4-bit values; 2-bit keys + QJL with group 1/2/4/8, 3-bit keys + QJL or MSE-only 3/4-bit keys with group 4/8)", name);
-  if (mma || lut) {
+  const bool i8 = tqk::attn_i8_supported(c, a) && max_T > 0;
+  const bool mma = !i8 && tqk::attn_mma_supported(c, a) && max_T > 0;
+  const bool lut = !i8 && !mma && tqk::attn_lut_supported(c, a) && max_T > 0;
+  if (pg.table && !(i8 || mma || lut))
+    return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode (d = 128, 4-bit values; "
+                "2- or 3-bit keys + QJL with m = 128, or MSE-only 3/4/8-bit keys)", name);
+  tqk::QopPlan qop{};
+  if (i8 || mma || lut) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
   }
-  cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s);
+  if (i8) {
+    unsigned char* img = reinterpret_cast<unsigned char*>(p + lay.qimg_off);
+    a.qimg = img;
+    qop = tqk::attn_i8_qop(c, a, img);
+  }
+  cudaError_t e = tqk::launch_prerotate(c, q, dtype, (int64_t)rows, a.tiles ? &a : nullptr, qr, qs, s,
+                                        i8 ? &qop : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, name);
-  e = mma ? tqk::launch_attn_mma(c, a, out, s)
-          : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s));
+  e = i8 ? tqk::launch_attn_i8(c, a, out, s)
+         : (mma ? tqk::launch_attn_mma(c, a, out, s)
+                : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s)));
   if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
 }
@@ -724,15 +735,17 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
   a.max_blocks = pg.max_blocks;
   a.block_size = pg.block_size;
   a.num_blocks = pg.num_blocks;
-  const bool mma = tqk::attn_mma_supported(c, a);
-  const bool lut = !mma && tqk::attn_lut_supported(c, a);
-  if (pg.table && !(mma || lut))
+  const bool i8 = tqk::attn_i8_supported(c, a);
+  const bool mma = !i8 && tqk::attn_mma_supported(c, a);
+  const bool lut = !i8 && !mma && tqk::attn_lut_supported(c, a);
+  if (pg.table && !(i8 || mma || lut))
     return fail(TQ_ERR_UNSUPPORTED, "%s: paged caches need the tensor-core decode", name);
-  if (mma || lut) {
+  if (i8 || mma || lut) {
     a.tiles = reinterpret_cast<int64_t*>(p + lay.tiles_off);
   } else if (a.splits > 4096) {
     return fail(TQ_ERR_UNSUPPORTED, "%s: too many splits", name);
   }
+  if (i8) a.qimg = reinterpret_cast<unsigned char*>(p + lay.qimg_off);
   tqk::StepPrep sp{};
   sp.k = qargs(true);
   sp.v = qargs(false);
@@ -748,10 +761,12 @@ static int decode_step_impl(tq_ctx* c, const void* q, int q_dtype, const void* k
   sp.max_T = max_T;
   sp.tiles = a.tiles;
   sp.nkv = (int64_t)B * Hkv;
+  sp.qop = i8 ? tqk::attn_i8_qop(c, a, const_cast<unsigned char*>(a.qimg)) : tqk::QopPlan{};
   cudaError_t e = tqk::launch_step_prep(c, sp, s);
   if (e != cudaSuccess) return cuda_fail(e, name);
-  e = mma ? tqk::launch_attn_mma(c, a, out, s)
-          : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s));
+  e = i8 ? tqk::launch_attn_i8(c, a, out, s)
+         : (mma ? tqk::launch_attn_mma(c, a, out, s)
+                : (lut ? tqk::launch_attn_lut(c, a, out, s) : tqk::launch_attn(c, a, out, s)));
   if (e != cudaSuccess) return cuda_fail(e, name);
   return TQ_OK;
 }

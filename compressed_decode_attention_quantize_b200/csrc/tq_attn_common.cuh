@@ -22,6 +22,12 @@ constexpr int VROW = 20;        // padded value row (words): conflict-free LDS.6
 constexpr int LUT_WORDS = 256 * 32;   // value table: 256 code pairs x 32 lane copies
 // The running maximum moves only when a tile exceeds it by 2^8 (exp2 units).
 constexpr float LAZY_TAU = 8.f;
+// Running maximum before the first valid token: finite, so that a tile whose
+// tokens are all masked (logits -inf, e.g. an invalid block of a paged cache)
+// gives exp2(-inf - M_EMPTY) = 0 instead of NaN.  A partial that saw no token
+// keeps it (with l = 0, o = 0) and gets weight 0 in the merge next to any
+// partial that saw one.
+constexpr float M_EMPTY = -1e30f;
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -148,10 +154,10 @@ __device__ __forceinline__ void value_tile(float (&o)[8][4], const uint32_t (*v)
 }
 
 // Record index of token t of row (b, kv head): [B][Hkv][max_T] contiguous, or
-// paged [blocks][Hkv][block_size] through the block table (an id outside
-// [0, num_blocks) reads block 0: wrong values, no fault).  For t a multiple
-// of 4 (16 when paged with block_size % 16 == 0) the next 3 (15) tokens are
-// the next records.
+// paged [blocks][Hkv][block_size] through the block table; -1 when the
+// block id is outside [0, num_blocks) (the caller masks those tokens).  For
+// t a multiple of 4 (16 when paged with block_size % 16 == 0) the next 3 (15)
+// tokens are the next records.
 template <bool PAGED>
 __device__ __forceinline__ int64_t kv_rec(const AttnArgs& a, int b, int kvh, int64_t t);
 
@@ -171,8 +177,8 @@ template <bool PAGED>
 __device__ __forceinline__ int64_t kv_rec(const AttnArgs& a, int b, int kvh, int64_t t) {
   if (!PAGED) return ((int64_t)b * a.Hkv + kvh) * a.max_T + t;
   const int ti = (int)t;
-  int64_t blk = a.block_table[(int64_t)b * a.max_blocks + ti / a.block_size];
-  blk = (blk >= 0 && blk < a.num_blocks) ? blk : 0;
+  const int64_t blk = a.block_table[(int64_t)b * a.max_blocks + ti / a.block_size];
+  if (blk < 0 || blk >= a.num_blocks) return -1;
   return (blk * a.Hkv + kvh) * a.block_size + ti % a.block_size;
 }
 

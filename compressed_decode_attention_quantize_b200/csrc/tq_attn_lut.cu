@@ -295,6 +295,7 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
       float vmax = 0.f;
       for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
         const int64_t rec = kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
+        if (PAGED && rec < 0) continue;                    // invalid block: masked
         if (a.nf16) {
           const __half* vr = reinterpret_cast<const __half*>(a.vnorm) + rec;
           if (j + 4 <= tok1) {
@@ -398,9 +399,16 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
     constexpr int NNC = (QJL ? 3 : 2) * 4;
     constexpr int NVC = MT * VF::REC / 4;
     constexpr int NCH = NKC + NQC + NNC + NVC;
+    uint32_t bad = 0;   // paged: bit (k % 32) set when the warp's k-th tile has an invalid block id
     auto issue = [&](int k, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
-      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
+      int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
+      // an invalid block copies nothing: every chunk is zero-filled
+      const int64_t tend = (PAGED && r < 0) ? t0 : tok1;
+      if (PAGED && r < 0) {
+        r = 0;
+        bad |= 1u << (k & 31);
+      }
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
 #pragma unroll
       for (int i = 0; i < (NCH + 31) / 32; ++i) {
@@ -418,10 +426,10 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
             part = c % (KF::REC / 4);
             dst = (uint32_t)(offsetof(Stage, k2) + tok * (KF::K2W * 4) + part * 16);
           }
-          cp16(sb + dst, kbase + (r + tok) * (KF::REC * 4) + part * 16, t0 + tok < tok1);
+          cp16(sb + dst, kbase + (r + tok) * (KF::REC * 4) + part * 16, t0 + tok < tend);
         } else if (c < NKC + NQC) {            // QJL words: 16 tokens x 1 chunk
           const int tok = c - NKC;
-          cp16(sb + offsetof(Stage, q) + tok * 16, a.kqjl + (rb + r + tok) * QW, t0 + tok < tok1);
+          cp16(sb + offsetof(Stage, q) + tok * 16, a.kqjl + (rb + r + tok) * QW, t0 + tok < tend);
         } else if (c < NKC + NQC + NNC) {      // norms: arrays x 4 chunks of 4 tokens
           const int which = (c - NKC - NQC) >> 2, part = (c - NKC - NQC) & 3;
           const int arr = QJL ? which : (which == 0 ? 0 : 2);   // 0 |k|, 1 gamma, 2 |v|
@@ -429,15 +437,15 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
           const uint32_t off = arr == 0 ? offsetof(Stage, kn)
                                         : (arr == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn));
           if (!a.nf16) {
-            cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tok1);
+            cp16(sb + off + part * 16, base + rb + r + 4 * part, t0 + 4 * part < tend);
           } else if (part < 2) {   // binary16 norms: 8 tokens per chunk
             cp16(sb + off + part * 16, reinterpret_cast<const __half*>(base) + rb + r + 8 * part,
-                 t0 + 8 * part < tok1);
+                 t0 + 8 * part < tend);
           }
         } else if (c < NCH) {                  // value codes: 16 tokens x 4 (3) chunks
           const int cc = c - NKC - NQC - NNC, tok = cc / (VF::REC / 4), part = cc % (VF::REC / 4);
           cp16(sb + offsetof(Stage, v) + tok * (VF::ROW * 4) + part * 16,
-               a.vcodes + (rb + r + tok) * VF::REC + part * 4, t0 + tok < tok1);
+               a.vcodes + (rb + r + tok) * VF::REC + part * 4, t0 + tok < tend);
         }
       }
     };
@@ -450,7 +458,7 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
     float m_run[NJ], l_part[NJ];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      m_run[j] = -INFINITY;
+      m_run[j] = M_EMPTY;
       l_part[j] = 0.f;
     }
     float o[8][4];
@@ -532,7 +540,8 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
 #undef TQ_QSTEP8
         }
       }
-      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
+      const bool tile_ok = !PAGED || !((bad >> (k & 31)) & 1u);
+      const bool v0 = tile_ok && t0 + g < tok1, v8 = tile_ok && t0 + g + 8 < tok1;
       auto snorm = [&](const float* arr, int i) {
         return a.nf16 ? __half2float(reinterpret_cast<const __half*>(arr)[i]) : arr[i];
       };

@@ -10,10 +10,10 @@
 //   o    = sum exp(s_i - m) |v_i| c_v[vidx_i]          (rotated domain)
 // The merge kernel combines the pieces by log-sum-exp and applies Pi^T once.
 //
-// Fast path: d = 128, keys 2 Lloyd-Max bits + 128 QJL rows, values 4 bits,
-// GQA group size 1, 2, 4 or 8.  Work is split into balanced contiguous ranges
-// of 16-token tiles over all (sequence, kv head) rows; a warp walks its tiles
-// with its own cp.async ring and online softmax.  Per tile:
+// Format: d = 128, keys 2 Lloyd-Max bits + 128 QJL rows, values 4 bits, GQA
+// group size 8 (groups of at most four heads take the int8 key product of
+// tq_attn_i8.cu).  Work is split into balanced contiguous ranges of 16-token
+// tiles over all (sequence, kv head) rows.  Per tile:
 //  * logits: mma.sync m16n8k16, A = key code bits as exact fp16 powers of two
 //    (16 tokens x 16 bit-planes), B = pre-rotated query (fp16 head and tail
 //    per head), fp32 accumulate; the centroid values enter through an affine
@@ -38,7 +38,6 @@
 namespace tqk {
 namespace {
 
-constexpr int NST = 4;          // pipeline stages per warp
 constexpr int KW = 8;           // key code words per token (2-bit fields)
 struct Stage {
   uint32_t k[MT][KW];           // 512 B
@@ -51,324 +50,7 @@ struct Stage {
 };
 static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
 
-constexpr size_t SMEM_BYTES = (size_t)LUT_WORDS * 4 + (size_t)MW * NST * sizeof(Stage);
 
-
-// ---------------------------------------------------------------------------
-// Group size <= 4, balanced segments.  The 16-token tiles of all (sequence,
-// kv head) rows form one sequence of W tiles (row-major over b, kv head,
-// tile; the prefix a.tiles[b] counts the tiles of rows before sequence b).
-// Warp w of the launch takes tiles [w W / N, (w + 1) W / N), N = min(warps,
-// W), so every warp gets a non-empty, equal share whatever the length mix.
-// A warp's range crosses row boundaries at most a few times; for each row
-// piece it builds the query operands once, streams the tiles through its own
-// cp.async ring and writes one partial (m, l, o) per head to slot
-// w + b Hkv + kv head, which is unique because consecutive rows' pieces come
-// from non-decreasing warps.  The merge finds a row's slots from the same
-// arithmetic.
-//
-// Softmax: the running maximum only moves when a tile's maximum exceeds it
-// by more than 2^8 (in exp2 units); probabilities then stay below 2^8, and
-// the value norms of a piece are scaled once, from the piece's largest norm,
-// so that p |v| stays below 2^15 in fp16.
-// ---------------------------------------------------------------------------
-template <int G, bool PAGED>
-__global__ void __launch_bounds__(MW * 32, 3) k_attn_seg(AttnArgs a) {
-  static_assert(G <= 4, "packed path");
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  Stage* stages = reinterpret_cast<Stage*>(smem + (size_t)LUT_WORDS * 4);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-
-  build_value_lut(lut, a.cv, tid, MW * 32);
-  __syncthreads();   // the only block-wide barrier: warps run independently below
-
-  const int64_t* P = a.tiles;
-  const int64_t W = P[a.B];
-  const int64_t NW = min((int64_t)gridDim.x * MW, W);
-  const int64_t wid = (int64_t)blockIdx.x * MW + warp;
-  if (wid >= NW) return;
-  int64_t x = wid * W / NW;
-  const int64_t x1 = (wid + 1) * W / NW;
-
-  int b = locate_sequence(P, a.B, x);
-
-  const float c0 = a.ck[0], w0 = a.ck[1] - a.ck[0], w1 = a.ck[2] - a.ck[0];
-  const int ew = ilog2f(fmaxf(fabsf(w0), fabsf(w1)));
-  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
-  Stage* my = stages + warp * NST;
-  const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
-  // Column g of the query-side B operands carries head g/2: even columns the
-  // fp16 head of the operand, odd columns its tail (x 2^12).
-  const int hh = g >> 1;
-  const bool tail_col = (g & 1) != 0;
-  const bool head_ok = hh < G;
-  const bool own_head = t < G;   // accumulator columns 2t, 2t+1 belong to head t
-
-  while (x < x1) {
-    while (P[b + 1] <= x) ++b;
-    const int64_t tb = (P[b + 1] - P[b]) / a.Hkv;
-    const int64_t rel = x - P[b];
-    const int kvh = (int)(rel / tb);
-    const int64_t tt = rel - (int64_t)kvh * tb;
-    const int64_t te = min(tb, tt + (x1 - x));
-    const int nt = (int)(te - tt);
-    const int64_t slot = wid + (int64_t)b * a.Hkv + kvh;
-    x += nt;
-
-    const int64_t len = min((int64_t)max(a.seq_lens[b], 0), a.max_T);
-    const int64_t tok0 = tt * MT;
-    const int64_t tok1 = min(te * MT, len);
-
-    // ---- cp.async ring: lane assignment fixed for the piece -------------------
-    // slot 0 = key codes, slots 1-2 = value codes, slot 3 = QJL words or norms.
-    const int64_t rb = kv_base<PAGED>(a, b, kvh);   // row base (0 when paged)
-    const char* p0 = reinterpret_cast<const char*>(a.kcodes + rb * KW) + lane * 16;
-    const char* p1 = reinterpret_cast<const char*>(a.vcodes + rb * VW) + lane * 16;
-    const char* p2 = p1 + 8 * 64;
-    const char* p3;
-    int stride3, tok3;
-    uint32_t d3;
-    if (lane < 16) {
-      p3 = reinterpret_cast<const char*>(a.kqjl + rb * QW) + lane * 16;
-      stride3 = 16; tok3 = lane; d3 = offsetof(Stage, q) + lane * 16;
-    } else if (lane < 28) {
-      const int which = (lane - 16) >> 2, part = (lane - 16) & 3;
-      const float* base = which == 0 ? a.knorm : (which == 1 ? a.krnorm : a.vnorm);
-      p3 = reinterpret_cast<const char*>(base + rb) + part * 16;
-      stride3 = 4; tok3 = 4 * part;
-      d3 = (which == 0 ? offsetof(Stage, kn) : (which == 1 ? offsetof(Stage, kr) : offsetof(Stage, vn))) + part * 16;
-    } else {
-      p3 = nullptr; stride3 = 0; tok3 = 1 << 30; d3 = 0;
-    }
-    const uint32_t d0 = offsetof(Stage, k) + lane * 16;
-    const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
-    const uint32_t d2 = d1 + 8 * (VROW * 4);
-    auto issue = [&](int i, int stage) {
-      const int64_t t0 = tok0 + (int64_t)MT * i;
-      const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
-      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
-      cp16(sb + d0, p0 + r * 32, t0 + (lane >> 1) < tok1);
-      cp16(sb + d1, p1 + r * 64, t0 + (lane >> 2) < tok1);
-      cp16(sb + d2, p2 + r * 64, t0 + 8 + (lane >> 2) < tok1);
-      if (lane < 28) cp16(sb + d3, p3 + r * stride3, t0 + tok3 < tok1);
-    };
-#pragma unroll
-    for (int i = 0; i < NST - 1; ++i) {
-      if (i < nt) issue(i, i);
-      cp_commit();
-    }
-
-    // ---- query-side operands (while the first tiles are in flight) ------------
-    const int64_t qrow_i = (int64_t)b * a.Hq + (int64_t)kvh * G + (head_ok ? hh : 0);
-    const float* qrow = a.qr + qrow_i * 128 + 32 * t;
-    const float* srow = a.qs + qrow_i * 128 + 32 * t;
-    float qv[32], sv[32];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 xq = reinterpret_cast<const float4*>(qrow)[i];
-      const float4 yq = reinterpret_cast<const float4*>(srow)[i];
-      qv[4 * i] = xq.x; qv[4 * i + 1] = xq.y; qv[4 * i + 2] = xq.z; qv[4 * i + 3] = xq.w;
-      sv[4 * i] = yq.x; sv[4 * i + 1] = yq.y; sv[4 * i + 2] = yq.z; sv[4 * i + 3] = yq.w;
-    }
-    float mq = 0.f, ms = 0.f, sumq = 0.f, sums = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      mq = fmaxf(mq, fabsf(qv[i]));
-      ms = fmaxf(ms, fabsf(sv[i]));
-      sumq += qv[i];
-      sums += sv[i];
-    }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
-      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
-      sumq += __shfl_xor_sync(0xffffffffu, sumq, o);
-      sums += __shfl_xor_sync(0xffffffffu, sums, o);
-    }
-    const int eq = mq > 0.f ? ilog2f(mq) : 0;
-    const int es = ms > 0.f ? ilog2f(ms) : 0;
-    // q' * w * 2^-(eq+ew+1) < 2, times at most 2^14: fits fp16.
-    const float kq = head_ok ? pow2i(-(eq + ew + 1)) : 0.f;
-    const float ks = head_ok ? pow2i(-es) : 0.f;
-    const float wq0 = w0 * kq, wq1 = w1 * kq;
-    auto operand = [&](float lo, float hi) -> uint32_t {
-      const __half2 h = __floats2half2_rn(lo, hi);
-      if (!tail_col) return *reinterpret_cast<const uint32_t*>(&h);
-      const float2 f = __half22float2(h);
-      return pack_half2((lo - f.x) * 4096.f, (hi - f.y) * 4096.f);
-    };
-    // Keys: k-step s (0..15) reads word s>>3 of the thread's two code words;
-    // slots 0/1 use registers u = 2(s&7) and 2(s&7)+1.
-    uint2 bk[16];
-#pragma unroll
-    for (int s = 0; s < 16; ++s) {
-      uint32_t pr[2];
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const int u = 2 * (s & 7) + sl;
-        const int elo = 10 + u, ehi = (26 + u) & 31;
-        const float inv = bit_inv(bit_pos(u));
-        const int dlo = 16 * (s >> 3) + (elo >> 1), dhi = 16 * (s >> 3) + (ehi >> 1);
-        const float vlo = qv[dlo] * ((elo & 1) ? wq1 : wq0) * inv;
-        const float vhi = qv[dhi] * ((ehi & 1) ? wq1 : wq0) * inv;
-        pr[sl] = operand(vlo, vhi);
-      }
-      bk[s] = make_uint2(pr[0], pr[1]);
-    }
-    // QJL: k-step s (0..7), slots 0/1 use registers 2s, 2s+1 of the thread's word.
-    uint2 bj[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      uint32_t pr[2];
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const int u = 2 * s + sl;
-        const int elo = 10 + u, ehi = (26 + u) & 31;
-        const float inv = bit_inv(bit_pos(u)) * ks;
-        pr[sl] = operand(sv[elo] * inv, sv[ehi] * inv);
-      }
-      bj[s] = make_uint2(pr[0], pr[1]);
-    }
-    // Logit constants of head t:  s2 = kn (acc KA + KB) + kr (acs QA + QB).
-    float KA, KB, QA, QB;
-    {
-      const int src = 8 * t;   // lanes with g = 2t hold head t's operand scales
-      const int eqj = __shfl_sync(0xffffffffu, eq, src);
-      const int esj = __shfl_sync(0xffffffffu, es, src);
-      const float sqj = __shfl_sync(0xffffffffu, sumq, src);
-      const float ssj = __shfl_sync(0xffffffffu, sums, src);
-      KA = pow2i(eqj + ew + 1) * a.scale_log2;
-      KB = c0 * sqj * a.scale_log2;
-      QA = 2.f * pow2i(esj) * a.cq * a.scale_log2;
-      QB = -ssj * a.cq * a.scale_log2;
-    }
-
-    // ---- value-norm scale of the piece ---------------------------------------
-    float vmax = 0.f;
-    {
-      for (int64_t j = tok0 + 4 * lane; j < tok1; j += 128) {
-        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
-        if (j + 4 <= tok1) {
-          const float4 v4 = *reinterpret_cast<const float4*>(vr);
-          vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
-        } else {
-          for (int64_t k = 0; k < tok1 - j; ++k) vmax = fmaxf(vmax, vr[k]);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    }
-    // p <= 2^8 and |v| 2^-kv < 2^7 keep p |v| 2^-kv below 2^15.
-    const int kv = vmax >= FLT_MIN ? max(ilog2f(vmax) - 6, -120) : -120;
-    const float vmul = pow2i(-kv);
-
-    float m_run = own_head ? -INFINITY : 0.f;
-    float l_part = 0.f;
-    float o[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-    for (int i = 0; i < nt; ++i) {
-      if (i + NST - 1 < nt) issue(i + NST - 1, (i + NST - 1) % NST);
-      cp_commit();
-      cp_wait<NST - 1>();
-      __syncwarp();
-      const Stage& st = my[i % NST];
-      const int64_t t0 = tok0 + (int64_t)MT * i;
-
-      // ---- logits -----------------------------------------------------------
-      // Two accumulators per product halve the dependent MMA chains.
-      float acc[4] = {0.f, 0.f, 0.f, 0.f}, acs[4] = {0.f, 0.f, 0.f, 0.f};
-      float acc2[4] = {0.f, 0.f, 0.f, 0.f}, acs2[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const uint2 kg0 = *reinterpret_cast<const uint2*>(&st.k[g][2 * t]);
-        const uint2 kg8 = *reinterpret_cast<const uint2*>(&st.k[g + 8][2 * t]);
-        const Rot4 R00 = rotations(kg0.x), R01 = rotations(kg0.y);
-        const Rot4 R80 = rotations(kg8.x), R81 = rotations(kg8.y);
-#define TQ_KSTEP(S)                                                                               \
-  mma16816(((S) & 1) ? acc2 : acc, bit_half2<2 * ((S) & 7)>((S) < 8 ? R00 : R01),                 \
-           bit_half2<2 * ((S) & 7)>((S) < 8 ? R80 : R81),                                         \
-           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R00 : R01),                                     \
-           bit_half2<2 * ((S) & 7) + 1>((S) < 8 ? R80 : R81), bk[S].x, bk[S].y);
-        TQ_KSTEP(0) TQ_KSTEP(1) TQ_KSTEP(2) TQ_KSTEP(3) TQ_KSTEP(4) TQ_KSTEP(5) TQ_KSTEP(6)
-        TQ_KSTEP(7) TQ_KSTEP(8) TQ_KSTEP(9) TQ_KSTEP(10) TQ_KSTEP(11) TQ_KSTEP(12) TQ_KSTEP(13)
-        TQ_KSTEP(14) TQ_KSTEP(15)
-#undef TQ_KSTEP
-        const Rot4 Q0 = rotations(st.q[g][t]), Q8 = rotations(st.q[g + 8][t]);
-#define TQ_QSTEP(S)                                                                               \
-  mma16816(((S) & 1) ? acs2 : acs, bit_half2<2 * (S)>(Q0), bit_half2<2 * (S)>(Q8),                \
-           bit_half2<2 * (S) + 1>(Q0),                                                             \
-           bit_half2<2 * (S) + 1>(Q8), bj[S].x, bj[S].y);
-        TQ_QSTEP(0) TQ_QSTEP(1) TQ_QSTEP(2) TQ_QSTEP(3) TQ_QSTEP(4) TQ_QSTEP(5) TQ_QSTEP(6)
-        TQ_QSTEP(7)
-#undef TQ_QSTEP
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          acc[r] += acc2[r];
-          acs[r] += acs2[r];
-        }
-      }
-      // Columns 2t (head) and 2t+1 (tail) of head t; rows g and g+8 are tokens.
-      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
-      const float lm0 = fmaf(acc[1], 1.f / 4096.f, acc[0]), lm8 = fmaf(acc[3], 1.f / 4096.f, acc[2]);
-      const float qj0 = fmaf(acs[1], 1.f / 4096.f, acs[0]), qj8 = fmaf(acs[3], 1.f / 4096.f, acs[2]);
-      const float sc0 = (own_head && v0) ? fmaf(st.kn[g], fmaf(lm0, KA, KB), st.kr[g] * fmaf(qj0, QA, QB))
-                                         : -INFINITY;
-      const float sc1 = (own_head && v8)
-                            ? fmaf(st.kn[g + 8], fmaf(lm8, KA, KB), st.kr[g + 8] * fmaf(qj8, QA, QB))
-                            : -INFINITY;
-
-      // ---- online softmax, head t ---------------------------------------------
-      const float loc = fmaxf(sc0, sc1);
-      if (__any_sync(0xffffffffu, loc > m_run + LAZY_TAU)) {
-        float tmax = loc;
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-        const float mnew = fmaxf(m_run, tmax);
-        const float alpha = ex2f(m_run - mnew);   // 0 on the first update, 1 if unchanged
-        m_run = mnew;
-        l_part *= alpha;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          o[mt][0] *= alpha;
-          o[mt][2] *= alpha;
-        }
-      }
-      const float p0 = ex2f(sc0 - m_run), p1 = ex2f(sc1 - m_run);
-      l_part += p0 + p1;
-      // P tile (16 tokens x 8 columns): column 2t = head t, odd columns zero.
-      const uint32_t pb0 = movtrans(pack_half2(p0 * (st.vn[g] * vmul), 0.f));
-      const uint32_t pb1 = movtrans(pack_half2(p1 * (st.vn[g + 8] * vmul), 0.f));
-
-      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
-      __syncwarp();
-    }
-    cp_wait<0>();
-    __syncwarp();   // the next piece's ring refills stages this one read
-
-    // ---- partial of the piece ------------------------------------------------
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 8);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 16);
-    if (own_head) {
-      float* pp = a.part + (slot * G + t) * (128 + 2);
-      const float vback = pow2i(kv);
-      if (g == 0) {
-        pp[0] = m_run;
-        pp[1] = l_part;
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        pp[2 + 16 * g + mt] = o[mt][0] * vback;
-        pp[2 + 16 * g + 8 + mt] = o[mt][2] * vback;
-      }
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Group size 8.  Eight heads with fp16 head and tail columns need sixteen B
@@ -468,7 +150,9 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
     {
       float vmax = 0.f;
       for (int64_t j = tok0 + 4 * tid; j < tok1; j += 4 * MW * 32) {
-        const float* vr = a.vnorm + kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
+        const int64_t rec = kv_rec<PAGED>(a, b, kvh, j);   // 4 tokens in a row
+        if (PAGED && rec < 0) continue;                    // invalid block: masked
+        const float* vr = a.vnorm + rec;
         if (j + 4 <= tok1) {
           const float4 v4 = *reinterpret_cast<const float4*>(vr);
           vmax = fmaxf(vmax, fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w)));
@@ -551,14 +235,21 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
     const uint32_t d0 = offsetof(Stage, k) + lane * 16;
     const uint32_t d1 = offsetof(Stage, v) + (lane >> 2) * (VROW * 4) + (lane & 3) * 16;
     const uint32_t d2 = d1 + 8 * (VROW * 4);
+    uint32_t bad = 0;   // paged: bit (k % 32) set when the warp's k-th tile has an invalid block id
     auto issue = [&](int k, int stage) {
       const int64_t t0 = tok0 + (int64_t)MT * (warp + MW * k);
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
-      const int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
-      cp16(sb + d0, p0 + r * 32, t0 + (lane >> 1) < tok1);
-      cp16(sb + d1, p1 + r * 64, t0 + (lane >> 2) < tok1);
-      cp16(sb + d2, p2 + r * 64, t0 + 8 + (lane >> 2) < tok1);
-      if (lane < 28) cp16(sb + d3, p3 + r * stride3, t0 + tok3 < tok1);
+      int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
+      bool ok = true;
+      if (PAGED && r < 0) {
+        ok = false;
+        r = 0;
+        bad |= 1u << (k & 31);
+      }
+      cp16(sb + d0, p0 + r * 32, ok && t0 + (lane >> 1) < tok1);
+      cp16(sb + d1, p1 + r * 64, ok && t0 + (lane >> 2) < tok1);
+      cp16(sb + d2, p2 + r * 64, ok && t0 + 8 + (lane >> 2) < tok1);
+      if (lane < 28) cp16(sb + d3, p3 + r * stride3, ok && t0 + tok3 < tok1);
     };
 #pragma unroll
     for (int k = 0; k < NST8 - 1; ++k) {
@@ -566,7 +257,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
       cp_commit();
     }
 
-    float m_run[2] = {-INFINITY, -INFINITY};
+    float m_run[2] = {M_EMPTY, M_EMPTY};
     float l_part[2] = {0.f, 0.f};
     float o[8][4];
 #pragma unroll
@@ -615,7 +306,8 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
         TQ_QSTEP8(6) TQ_QSTEP8(7)
 #undef TQ_QSTEP8
       }
-      const bool v0 = t0 + g < tok1, v8 = t0 + g + 8 < tok1;
+      const bool tile_ok = !PAGED || !((bad >> (k & 31)) & 1u);
+      const bool v0 = tile_ok && t0 + g < tok1, v8 = tile_ok && t0 + g + 8 < tok1;
       const float kn0 = st.kn[g], kn8 = st.kn[g + 8], kr0 = st.kr[g], kr8 = st.kr[g + 8];
       float sc[2][2];
 #pragma unroll
@@ -693,7 +385,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a) {
   if (c->norm_f16) return false;   // QJL formats keep fp32 norms
   if (c->d != D || c->bk_lm != 2 || c->bits_v != 4 || c->qjl_m != 128) return false;
-  if (!(a.G == 1 || a.G == 2 || a.G == 4 || a.G == 8)) return false;
+  if (a.G != 8) return false;
   if (a.max_T % 4 != 0) return false;
   const uintptr_t al = reinterpret_cast<uintptr_t>(a.kcodes) | reinterpret_cast<uintptr_t>(a.kqjl) |
                        reinterpret_cast<uintptr_t>(a.knorm) | reinterpret_cast<uintptr_t>(a.krnorm) |
@@ -706,54 +398,26 @@ int64_t attn_seg_max_warps(const tq_ctx* c) { return (int64_t)c->sms * 3 * MW; }
 
 cudaError_t launch_attn_mma(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
   AttnArgs a = a_in;
-  if (a.G == 1 || a.G == 2 || a.G == 4) {
-    if (!a.tiles) return cudaErrorInvalidValue;
-    // At least four tiles per warp, at most attn_seg_max_warps warps; the
-    // kernel trims the warp count to the real tile count.
-    const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
-    int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
-    blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
-    a.nw = (int)(blocks * MW);
-    a.wpu = 1;
-    const bool paged = a.block_table != nullptr;
-    switch (a.G * 2 + (paged ? 1 : 0)) {
-      case 2: k_attn_seg<1, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      case 3: k_attn_seg<1, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      case 4: k_attn_seg<2, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      case 5: k_attn_seg<2, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      case 8: k_attn_seg<4, false><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-      default: k_attn_seg<4, true><<<(unsigned)blocks, MW * 32, SMEM_BYTES, s>>>(a); break;
-    }
-  } else if (a.G == 8) {
-    if (!a.tiles) return cudaErrorInvalidValue;
-    // CTA-owned ranges of at least four tiles per warp.
-    const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
-    int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
-    blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
-    a.nw = (int)blocks;
-    a.wpu = MW;
-    if (a.block_table)
-      k_attn_seg8<true><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
-    else
-      k_attn_seg8<false><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
-  } else {
-    return cudaErrorInvalidValue;
-  }
+  if (a.G != 8 || !a.tiles) return cudaErrorInvalidValue;
+  // CTA-owned ranges of at least four tiles per warp.
+  const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
+  int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
+  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
+  a.nw = (int)blocks;
+  a.wpu = MW;
+  if (a.block_table)
+    k_attn_seg8<true><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
+  else
+    k_attn_seg8<false><<<(unsigned)blocks, MW * 32, SMEM8_BYTES, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_merge(c, a, out, s);
 }
 
 cudaError_t configure_attn_mma() {
-  const int b = (int)SMEM_BYTES, b8 = (int)SMEM8_BYTES;
+  const int b8 = (int)SMEM8_BYTES;
   const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<1, false>, ms, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<1, true>, ms, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<2, false>, ms, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<2, true>, ms, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<4, false>, ms, b))) return e;
-  if ((e = cudaFuncSetAttribute(k_attn_seg<4, true>, ms, b))) return e;
   if ((e = cudaFuncSetAttribute(k_attn_seg8<false>, ms, b8))) return e;
   return cudaFuncSetAttribute(k_attn_seg8<true>, ms, b8);
 }

@@ -108,6 +108,24 @@ struct QuantArgs {
   int nf16;
 };
 
+// Query operands of the int8 key product (decode with 2-bit keys + QJL,
+// d = m = 128, groups of at most four query heads).  Per (sequence, kv head)
+// one image of kQopBytes: 48 registers per lane in lane order
+// ([12][32 lanes][4] uint32), each four signed bytes, then four float4 of
+// per-head logit constants.  Register r = (k-step s, N tile j, half hb):
+// keys r = 4 s + 2 j + hb (s < 8), QJL r = 32 + 4 s + 2 j + hb (s < 4).
+// Column n of an N tile is head n / 2, limb 2 j + n % 2 of that head's
+// balanced base-256 digits.
+constexpr int kQopRegs = 48;
+constexpr int kQopBytes = kQopRegs * 32 * 4 + 4 * 16;
+struct QopPlan {
+  unsigned char* img;  // [B * Hkv][kQopBytes]; null = no image
+  int Hq, G;           // query heads, heads per kv group (<= 4)
+  float scale_log2;    // softmax scale * log2(e)
+  float cq;            // sqrt(pi/2) / m
+  float c0, c1, c2;    // 2-bit key centroids 0..2
+};
+
 struct AttnArgs {
   const float* qr;   // [B*Hq][dpad] pre-rotated queries
   const float* qs;   // [B*Hq][dpad] S q'
@@ -142,6 +160,8 @@ struct AttnArgs {
   int64_t num_blocks;
   // Norms stored as binary16 (knorm / vnorm then address __half values).
   int nf16;
+  // Query-operand images of the int8 key product (see QopPlan).
+  const unsigned char* qimg;
 };
 
 struct QuantTcArgs {
@@ -189,16 +209,26 @@ struct StepPrep {
   int64_t max_T;
   int64_t* tiles;
   int64_t nkv;
+  QopPlan qop;
 };
 cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s);
 // With plan != null the kernel also writes plan->tiles (the segment path's
-// tile prefix) from plan->seq_lens, B, Hkv and max_T.
+// tile prefix) from plan->seq_lens, B, Hkv and max_T; with qop != null and
+// qop->img != null it writes the int8 query-operand images.
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
-                             float* qr, float* qs, cudaStream_t s);
+                             float* qr, float* qs, cudaStream_t s, const QopPlan* qop = nullptr);
+// The int8 key-product decode (2-bit keys + QJL, m = 128, 4-bit values,
+// d = 128, group 1, 2 or 4): whether it applies, and the plan of its
+// query-operand images.
+bool attn_i8_supported(const tq_ctx* c, const AttnArgs& a);
+QopPlan attn_i8_qop(const tq_ctx* c, const AttnArgs& a, unsigned char* img);
+// Needs AttnArgs::tiles (the tile prefix) and AttnArgs::qimg (the images).
+cudaError_t launch_attn_i8(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
+cudaError_t configure_attn_i8();
 cudaError_t launch_attn(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s);
-// Tensor-core decode path (d = 128, k3 with m = 128, v4, group 1, 2, 4 or 8);
-// it needs AttnArgs::tiles (the tile prefix) set.
+// Tensor-core decode path with fp16 bit operands (d = 128, k3 with m = 128,
+// v4, group 8); it needs AttnArgs::tiles (the tile prefix) set.
 bool attn_mma_supported(const tq_ctx* c, const AttnArgs& a);
 // Upper bound on the warps of a segment-path launch (sizes the partials).
 int64_t attn_seg_max_warps(const tq_ctx* c);

@@ -494,12 +494,108 @@ __device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T
   }
 }
 
+// Query operands of the int8 key product, for the PR rows of a block (thread
+// j = coordinate j and QJL row j; d = m = blockDim = 128).
+//
+// The logit of a 2-bit key is l = n <q', c[idx]> + cq gamma <s, sigma>.  A
+// symmetric 2-bit codebook is affine in the index bits, c[i0 + 2 i1] =
+// c0 + w0 i0 + w1 i1 (w0 = c1 - c0, w1 = c2 - c0), and <s, sigma> =
+// 2 <s, bit> - sum s, so both products are sums of query terms over set code
+// bits.  The decode kernel's A operand holds code bit b of a word in byte
+// b / 8, at bit position p = b % 8 (value 2^p); this side supplies for that
+// position the integer Q = round(2^(S - p) w q'_j) (or 2^(S' - p) s_i),
+// with S chosen so |Q| < 2^30, as four balanced base-256 digits (signed
+// bytes), one per N-tile column.  The int32 products then sum to
+// 2^S <w q', bits> exactly, digit by digit, and
+//   scale * log2(e) * l = n (KA acc_key + KB) + gamma (QA acc_qjl + QB)
+// with KA = 2^-S sl, KB = c0 sum(q') sl, QA = 2^(1-S') cq sl,
+// QB = -sum(s) cq sl (sl = scale * log2(e)).
+template <int PR>
+__device__ void write_qop(const QopPlan& P, const float (&qv)[PR], const float (&sv)[PR], int64_t row0,
+                          int nr) {
+  __shared__ float s_red[PR][8][4];
+  const int j = threadIdx.x, lane = j & 31, warp = j >> 5, nwarp = blockDim.x >> 5;
+#pragma unroll
+  for (int r = 0; r < PR; ++r) {
+    float mq = fabsf(qv[r]), sq = qv[r], ms = fabsf(sv[r]), ss = sv[r];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    if (lane == 0) {
+      s_red[r][warp][0] = mq;
+      s_red[r][warp][1] = sq;
+      s_red[r][warp][2] = ms;
+      s_red[r][warp][3] = ss;
+    }
+  }
+  __syncthreads();
+  const double c0 = P.c0, w0 = (double)P.c1 - c0, w1 = (double)P.c2 - c0;
+  const double wmax = fmax(fabs(w0), fabs(w1));
+#pragma unroll
+  for (int r = 0; r < PR; ++r) {
+    if (r >= nr) break;   // uniform over the block
+    float mq = 0.f, ms = 0.f;
+    double sq = 0.0, ss = 0.0;
+    for (int w = 0; w < nwarp; ++w) {
+      mq = fmaxf(mq, s_red[r][w][0]);
+      sq += s_red[r][w][1];
+      ms = fmaxf(ms, s_red[r][w][2]);
+      ss += s_red[r][w][3];
+    }
+    // 2^e <= max |w q'| < 2^(e+1), S = 29 - e: |Q| < 2^30 at p = 0.
+    const double mk = wmax * mq;
+    const int S = mk > 0.0 ? 29 - ilogb(mk) : 0;
+    const int S2 = ms > 0.f ? 29 - ilogb((double)ms) : 0;
+    const int64_t row = row0 + r;
+    const int64_t b = row / P.Hq;
+    const int h = (int)(row % P.Hq), kvh = h / P.G, hg = h % P.G;
+    unsigned char* img = P.img + (b * (P.Hq / P.G) + kvh) * (int64_t)kQopBytes;
+    auto put = [&](int reg, int tt, int e, int64_t Q) {
+      // four balanced digits, digit l to column 2 hg + l % 2 of N tile l / 2
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        const int dg = (int)(signed char)(Q & 0xFF);
+        Q = (Q - dg) >> 8;
+        const int rr = reg + 2 * (l >> 1);
+        const int ln = 4 * (2 * hg + (l & 1)) + tt;
+        img[(((rr >> 2) * 32 + ln) * 4 + (rr & 3)) * 4 + e] = (unsigned char)(dg & 0xFF);
+      }
+    };
+    {
+      const double q = qv[r];
+#pragma unroll
+      for (int pl = 0; pl < 2; ++pl) {
+        const int bit = 2 * (j & 15) + pl, w = j >> 4, p = bit & 7;
+        const int64_t Q = llrint(ldexp((pl ? w1 : w0) * q, S - p));
+        put(4 * p + (w >> 2), w & 3, bit >> 3, Q);
+      }
+      const int bit = j & 31, p = bit & 7;
+      const int64_t Q = llrint(ldexp((double)sv[r], S2 - p));
+      put(32 + 4 * (p >> 1) + (p & 1), j >> 5, bit >> 3, Q);
+    }
+    if (j == 0) {
+      const double sl = P.scale_log2;
+      float4 cst;
+      cst.x = (float)ldexp(sl, -S);
+      cst.y = (float)(c0 * sq * sl);
+      cst.z = (float)ldexp(2.0 * (double)P.cq * sl, -S2);
+      cst.w = (float)(-ss * (double)P.cq * sl);
+      reinterpret_cast<float4*>(img + kQopRegs * 32 * 4)[hg] = cst;
+    }
+  }
+}
+
 // PR query rows per block: thread j owns coordinate j of each row, so Pi and
 // S are read once per block.
 template <int PR>
 __device__ __forceinline__ void prerotate_body(const void* q, int dtype, int64_t rows, int d, int dpad,
                                                int m, const float* PiT, const float* ST, float* qr,
-                                               float* qs, int64_t blk, float* sh) {
+                                               float* qs, int64_t blk, float* sh,
+                                               const QopPlan* qop = nullptr) {
   float* sq = sh;                  // [PR][dpad]: q, later q'
   float* Ms = sh + PR * dpad;      // [2][MV_KC][dpad]
   const int j = threadIdx.x;       // blockDim = dpad
@@ -508,27 +604,32 @@ __device__ __forceinline__ void prerotate_body(const void* q, int dtype, int64_t
 #pragma unroll
   for (int r = 0; r < PR; ++r) sq[r * dpad + j] = (r < nr && j < d) ? load_elem(q, dtype, (row0 + r) * d + j) : 0.f;
   __syncthreads();
-  float acc[PR];
+  float acc[PR], qv[PR];
   mv_rows<PR>(PiT, d, dpad, sq, Ms, acc);
 #pragma unroll
   for (int r = 0; r < PR; ++r) {
+    qv[r] = acc[r];
     sq[r * dpad + j] = acc[r];
     if (r < nr) qr[(row0 + r) * dpad + j] = acc[r];
   }
   __syncthreads();
   mv_rows<PR>(ST, d, dpad, sq, Ms, acc);
 #pragma unroll
-  for (int r = 0; r < PR; ++r)
-    if (r < nr) qs[(row0 + r) * dpad + j] = (j < m) ? acc[r] : 0.f;
+  for (int r = 0; r < PR; ++r) {
+    acc[r] = (j < m) ? acc[r] : 0.f;
+    if (r < nr) qs[(row0 + r) * dpad + j] = acc[r];
+  }
+  if (qop && qop->img) write_qop<PR>(*qop, qv, acc, row0, nr);
 }
 
 template <int PR>
 __global__ void __launch_bounds__(256) k_prerotate(const void* q, int dtype, int64_t rows, int d,
                                                    int dpad, int m, const float* PiT, const float* ST,
                                                    float* qr, float* qs, const int32_t* seq_lens,
-                                                   int B, int Hkv, int64_t max_T, int64_t* tiles) {
+                                                   int B, int Hkv, int64_t max_T, int64_t* tiles,
+                                                   QopPlan qop) {
   extern __shared__ float sh[];
-  prerotate_body<PR>(q, dtype, rows, d, dpad, m, PiT, ST, qr, qs, blockIdx.x, sh);
+  prerotate_body<PR>(q, dtype, rows, d, dpad, m, PiT, ST, qr, qs, blockIdx.x, sh, &qop);
   if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
 }
 
@@ -553,7 +654,7 @@ __global__ void __launch_bounds__(256) k_step_prep(StepPrep s, int d, int dpad, 
     return;
   }
   blk -= s.nkv;
-  prerotate_body<2>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, sh);
+  prerotate_body<2>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, sh, &s.qop);
   if (blk == 0) {
     for (int b = threadIdx.x; b < s.B; b += blockDim.x) {
       const int64_t p = s.pos[b];
@@ -1035,18 +1136,20 @@ cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s
 }
 
 cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t rows, const AttnArgs* plan,
-                             float* qr, float* qs, cudaStream_t s) {
+                             float* qr, float* qs, cudaStream_t s, const QopPlan* qop) {
   if (rows == 0) return cudaSuccess;
   const int32_t* sl = plan ? plan->seq_lens : nullptr;
   const int pB = plan ? plan->B : 0, pH = plan ? plan->Hkv : 1;
   const int64_t pT = plan ? plan->max_T : 0;
   int64_t* tl = plan ? plan->tiles : nullptr;
+  QopPlan qp{};
+  if (qop) qp = *qop;
   if (rows <= 1024) {
     k_prerotate<2><<<(unsigned)((rows + 1) / 2), c->dpad, (2 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
-        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl);
+        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl, qp);
   } else {
     k_prerotate<8><<<(unsigned)((rows + 7) / 8), c->dpad, (8 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
-        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl);
+        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl, qp);
   }
   return cudaGetLastError();
 }
@@ -1211,6 +1314,7 @@ cudaError_t configure_kernels() {
   if ((e = cudaFuncSetAttribute(k_step_prep, ms, small_smem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   if ((e = configure_attn_lut()) != cudaSuccess) return e;
+  if ((e = configure_attn_i8()) != cudaSuccess) return e;
   if ((e = configure_topk_mma()) != cudaSuccess) return e;
   if ((e = configure_topk_tc()) != cudaSuccess) return e;
   return configure_attn_mma();

@@ -317,12 +317,14 @@ size_t tq_attn_static_scratch_bytes(void);
  * sequence b is record (block_table[b][t / block_size] * Hkv + g) *
  * block_size + t % block_size of the arrays [num_blocks][Hkv][block_size][...]
  * (g = kv head).  block_size must be a multiple of 16; seq_lens[b] is clamped
- * to max_blocks * block_size.  Block ids outside [0, num_blocks) read block 0
- * (wrong results, no fault).  Only the tensor-core decode takes paged caches
- * (d = 128, keys with m = 128 QJL rows, 4-bit values; 2-bit keys with GQA
- * group 1, 2, 4 or 8, or 3-bit keys with group 8); other formats return
- * TQ_ERR_UNSUPPORTED.  Workspace: tq_attn_workspace_bytes(ctx, B, Hq,
- * max_blocks * block_size).
+ * to max_blocks * block_size.  The tokens of a block whose id is outside
+ * [0, num_blocks) are masked: like tokens past seq_lens[b] they get no
+ * weight (a sequence with every token masked gets out = 0).  Only the
+ * tensor-core decode takes paged caches: d = 128, GQA group 1, 2, 4 or 8, and
+ * keys of 2 or 3 Lloyd-Max bits + 128 QJL rows with 4-bit values, or MSE-only
+ * keys of 3, 4 or 8 bits with 4-bit values (3-bit keys also with 3-bit
+ * values); other formats return TQ_ERR_UNSUPPORTED.  Workspace:
+ * tq_attn_workspace_bytes(ctx, B, Hq, max_blocks * block_size).
  */
 int tq_attn_decode_paged(tq_ctx* ctx, const void* q, int dtype, int B, int Hq, int Hkv,
                          const uint32_t* kcodes, const uint32_t* kqjl, const void* knorm,

@@ -897,6 +897,101 @@ def test_paged_decode_step_equals_contiguous(cuda, Hq, Hkv, bk):
             assert torch.equal(v[blk], before[k][blk]), k
 
 
+def _from_paged(cache_np, table, B, bs):
+    """Host copy of a paged cache [blocks, Hkv, bs, ...] as a contiguous
+    [B, Hkv, max_blocks * bs, ...] cache through the block table (invalid ids
+    give zero records, which the callers never read)."""
+    mb = table.shape[1]
+    out = {}
+    for k, v in cache_np.items():
+        if v is None:
+            out[k] = None
+            continue
+        rows = []
+        for b in range(B):
+            blocks = [v[int(i)] if 0 <= int(i) < v.shape[0] else np.zeros_like(v[0]) for i in table[b]]
+            rows.append(np.concatenate(blocks, axis=1))
+        out[k] = np.stack(rows)
+    return out
+
+
+def _drop_tokens(cache_np, b, lo, hi):
+    """Sequence b's records with tokens [lo, hi) removed (softmax . V is
+    invariant to the order of the (key, value) pairs, so a masked block is the
+    same as a shorter context without it)."""
+    return {k: (None if v is None else np.delete(v[b:b + 1], np.s_[lo:hi], axis=2)) for k, v in cache_np.items()}
+
+
+@pytest.mark.parametrize("fmt,Hq,bs", [("k3v4", 8, 32), ("k3v4", 16, 16), ("k3v4", 2, 16), ("k4v4", 8, 16),
+                                       ("k4v4", 16, 48), ("4bit_nc", 8, 32), ("3bit_nc", 16, 16)])
+def test_paged_decode_matches_oracle(cuda, fmt, Hq, bs):
+    """The paged decode against the fp64 oracle on the same codes: shuffled
+    blocks, ragged lengths (empty, one token, a partial last block, full), an
+    invalid block id inside a sequence (its tokens are masked: the reference
+    is the context without them) and one past a sequence's length (no
+    effect)."""
+    c = tq.Context.variant(fmt, 128, seed=6)
+    tab = P.oracle_tables(c)
+    B, Hkv, d, max_T = 5, 2, 128, 288
+    K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=41)
+    V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=42)
+    kc, vc = c.quantize(K.to(cuda), tq.TQ_KEY), c.quantize(V.to(cuda), tq.TQ_VALUE)
+    mb = max_T // bs
+    perm = torch.randperm(B * mb + 7, generator=torch.Generator().manual_seed(5))[:B * mb].to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, max_T, bs, perm), _to_paged(vc, B, Hkv, max_T, bs, perm)
+    table = perm.reshape(B, mb).clone()
+    lens = torch.tensor([0, 1, bs + 3, 200, max_T], dtype=torch.int32)
+    table[4, 1] = -1          # inside sequence 4: tokens [bs, 2 bs) masked
+    table[2, mb - 1] = 10**6  # past sequence 2's length: never read
+    q = tq_inputs.iid((B, Hq, d), seed=43, dtype=torch.bfloat16)
+    got = c.attn_decode_paged(q.to(cuda), kp, vp, table.to(cuda), lens.to(cuda))
+    torch.cuda.synchronize()
+    kh, vh = P.packed_np(kc), P.packed_np(vc)
+    qn, gn = q.double().numpy(), got.cpu().numpy()
+    for b in range(B):
+        L = int(lens[b])
+        if b == 4:
+            kb, vb, L = _drop_tokens(kh, b, bs, 2 * bs), _drop_tokens(vh, b, bs, 2 * bs), L - bs
+        else:
+            kb = {k: (None if v is None else v[b:b + 1]) for k, v in kh.items()}
+            vb = {k: (None if v is None else v[b:b + 1]) for k, v in vh.items()}
+        P.check_attention(tab, qn[b:b + 1], kb, vb, np.array([L]), Hkv, gn[b:b + 1])
+
+
+@pytest.mark.parametrize("fmt,Hq", [("k3v4", 8), ("k4v4", 16), ("k3v4_nc", 8)])
+def test_paged_decode_step_matches_oracle(cuda, fmt, Hq):
+    """decode_step_paged against the oracle: the appended tokens are read back
+    from the paged cache, which is gathered into contiguous order on the host,
+    and the attention over [0, pos] is checked on the same codes."""
+    c = tq.Context.variant(fmt, 128, seed=8)
+    tab = P.oracle_tables(c)
+    B, Hkv, d, max_T, bs = 4, 2, 128, 128, 32
+    K = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=51).to(cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, max_T, d, seed=52).to(cuda)
+    kc, vc = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    mb = max_T // bs
+    perm = torch.randperm(B * mb, generator=torch.Generator().manual_seed(9)).to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, max_T, bs, perm), _to_paged(vc, B, Hkv, max_T, bs, perm)
+    table = perm.reshape(B, mb)
+    q = tq_inputs.iid((B, Hq, d), seed=53, dtype=torch.bfloat16).to(cuda)
+    kn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=54)[:, :, 0].contiguous().to(cuda)
+    vn = tq_inputs.outlier_kv(B, Hkv, 1, d, seed=55)[:, :, 0].contiguous().to(cuda)
+    pos = torch.tensor([0, 40, 95, 127], dtype=torch.int32, device=cuda)
+    got = c.decode_step_paged(q, kn, vn, kp, vp, table.to(cuda), pos)
+    torch.cuda.synchronize()
+    tn = table.numpy()
+    kh = _from_paged(P.packed_np(kp), tn, B, bs)
+    vh = _from_paged(P.packed_np(vp), tn, B, bs)
+    # the appended records are the oracle's quantization of the new tokens
+    for which, x, h in (("k", kn, kh), ("v", vn, vh)):
+        recs = {k: (None if v is None else np.stack([v[b, :, int(pos[b])] for b in range(B)]).reshape(B * Hkv, -1)
+                    if v.ndim > 3 else np.stack([v[b, :, int(pos[b])] for b in range(B)]).reshape(B * Hkv))
+                for k, v in h.items()}
+        P.check_quantized(tab, which, P.to_np(x.reshape(B * Hkv, d)), recs)
+    lens = (pos + 1).cpu().numpy()
+    P.check_attention(tab, q.double().cpu().numpy(), kh, vh, lens, Hkv, got.cpu().numpy())
+
+
 def test_paged_rejections(cuda):
     c = _ctx(64, 2, 2, 0)
     q = torch.zeros(1, 2, 64, dtype=torch.bfloat16, device=cuda)
