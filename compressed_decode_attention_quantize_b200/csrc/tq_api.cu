@@ -176,7 +176,10 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
     return nullptr;
   }
   const int dp = c->dpad;
-  const size_t nPiT = (size_t)d * dp, nPi = (size_t)d * d, nST = (size_t)d * dp, nS = (size_t)dp * d;
+  // Every table starts on a 16-byte boundary (kernels copy them with 16-byte
+  // asynchronous copies): Pi's d * d entries are padded to a multiple of 4.
+  const size_t nPiT = (size_t)d * dp, nPi = ((size_t)d * d + 3) & ~(size_t)3, nST = (size_t)d * dp,
+               nS = (size_t)dp * d;
   const size_t total = (nPiT + nPi + nST + nS + 4 * tqk::kMaxLevels) * sizeof(float);
   std::vector<float> h(total / sizeof(float), 0.f);
   float* hPiT = h.data();

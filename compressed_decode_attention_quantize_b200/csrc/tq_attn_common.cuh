@@ -124,6 +124,17 @@ __device__ __forceinline__ void build_value_lut(uint32_t* lut, const float* cv, 
   }
 }
 
+// Wide value table for kernels with one CTA per SM: entry (byte, lane) at
+// byte offset 256 byte + 4 lane, so one byte permute forms the address from
+// the code-pair byte and the lane's offset (64 KB; half of each entry unused).
+constexpr int WLUT_BYTES = 256 * 256;
+__device__ __forceinline__ void build_value_wlut(uint32_t* lut, const float* cv, int tid, int nthreads) {
+  for (int e = tid; e < 256 * 32; e += nthreads) {
+    const int byte = e >> 5, ln = e & 31;
+    lut[byte * 64 + ln] = pack_half2(cv[byte & 15], cv[byte >> 4]);
+  }
+}
+
 // o[mt] += V^T P for one 16-token tile: A = dequantized values (16 dims x 16
 // tokens per mt), B = [pb0; pb1] (16 tokens x 8 columns).  v holds the tile's
 // 16 value-code rows (VROW words each); a code pair (two tokens, one dim)
@@ -149,6 +160,33 @@ __device__ __forceinline__ void value_tile(float (&o)[8][4], const uint32_t (*v)
     uint32_t av[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) av[r] = lds32(__byte_perm(y[r], 0, 0x4440 + k) * 128u + lut_lane);
+    mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
+  }
+}
+
+// value_tile with the wide table at shared address lut_s; lane4 = 4 * lane.
+__device__ __forceinline__ void value_tile_w(float (&o)[8][4], const uint32_t (*v)[VROW], uint32_t pb0,
+                                             uint32_t pb1, uint32_t lut_s, uint32_t lane4, int g, int t) {
+  const uint2 xa = *reinterpret_cast<const uint2*>(&v[2 * t][2 * g]);
+  const uint2 xb = *reinterpret_cast<const uint2*>(&v[2 * t + 1][2 * g]);
+  const uint2 xc = *reinterpret_cast<const uint2*>(&v[2 * t + 8][2 * g]);
+  const uint2 xd = *reinterpret_cast<const uint2*>(&v[2 * t + 9][2 * g]);
+  const uint32_t ye[4] = {(xa.x & 0x0F0F0F0Fu) | ((xb.x << 4) & 0xF0F0F0F0u),
+                          (xa.y & 0x0F0F0F0Fu) | ((xb.y << 4) & 0xF0F0F0F0u),
+                          (xc.x & 0x0F0F0F0Fu) | ((xd.x << 4) & 0xF0F0F0F0u),
+                          (xc.y & 0x0F0F0F0Fu) | ((xd.y << 4) & 0xF0F0F0F0u)};
+  const uint32_t yo[4] = {((xa.x >> 4) & 0x0F0F0F0Fu) | (xb.x & 0xF0F0F0F0u),
+                          ((xa.y >> 4) & 0x0F0F0F0Fu) | (xb.y & 0xF0F0F0F0u),
+                          ((xc.x >> 4) & 0x0F0F0F0Fu) | (xd.x & 0xF0F0F0F0u),
+                          ((xc.y >> 4) & 0x0F0F0F0Fu) | (xd.y & 0xF0F0F0F0u)};
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int k = mt >> 1;
+    const uint32_t* y = (mt & 1) ? yo : ye;
+    uint32_t av[4];
+    // byte 0 = 4 lane, byte 1 = code-pair byte k of y, bytes 2-3 = 0
+#pragma unroll
+    for (int r = 0; r < 4; ++r) av[r] = lds32(lut_s + __byte_perm(lane4, y[r], 0x1140 + 16 * k));
     mma16816(o[mt], av[0], av[1], av[2], av[3], pb0, pb1);
   }
 }

@@ -43,7 +43,8 @@
 namespace tqk {
 namespace {
 
-constexpr int NSI = 4;     // pipeline stages per warp
+constexpr int MWI = 12;    // warps per CTA (one CTA per SM: the value table is shared)
+constexpr int NSI = 5;     // pipeline stages per warp
 constexpr int KWI = 8;     // key code words per token (2-bit fields)
 constexpr int KROW = 12;   // padded key row in shared memory: the 32-bit loads of words t and t + 4
                            // by the lanes (g, t) of a warp hit 32 distinct banks
@@ -59,7 +60,7 @@ struct StageI {
 static_assert(sizeof(StageI) % 16 == 0, "stage alignment");
 static_assert(offsetof(StageI, v) % 16 == 0, "value rows alignment");
 
-constexpr size_t SMEM_I8 = (size_t)LUT_WORDS * 4 + (size_t)MW * NSI * sizeof(StageI);
+constexpr size_t SMEM_I8 = (size_t)WLUT_BYTES + (size_t)MWI * NSI * sizeof(StageI);
 
 __device__ __forceinline__ void imma16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -95,28 +96,28 @@ __device__ __forceinline__ float limbs(int d0, int d1, int d2, int d3) {
 // position.
 // ---------------------------------------------------------------------------
 template <int G, bool PAGED>
-__global__ void __launch_bounds__(MW * 32, 3) k_attn_i8(AttnArgs a) {
+__global__ void __launch_bounds__(MWI * 32, 1) k_attn_i8(AttnArgs a) {
   static_assert(G <= 4, "four heads per N tile pair");
   extern __shared__ __align__(16) unsigned char smem[];
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem);
-  StageI* stages = reinterpret_cast<StageI*>(smem + (size_t)LUT_WORDS * 4);
+  StageI* stages = reinterpret_cast<StageI*>(smem + (size_t)WLUT_BYTES);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
-  build_value_lut(lut, a.cv, tid, MW * 32);
+  build_value_wlut(lut, a.cv, tid, MWI * 32);
   __syncthreads();   // the only block-wide barrier: warps run independently below
 
   const int64_t* P = a.tiles;
   const int64_t W = P[a.B];
-  const int64_t NW = min((int64_t)gridDim.x * MW, W);
-  const int64_t wid = (int64_t)blockIdx.x * MW + warp;
+  const int64_t NW = min((int64_t)gridDim.x * MWI, W);
+  const int64_t wid = (int64_t)blockIdx.x * MWI + warp;
   if (wid >= NW) return;
   int64_t x = wid * W / NW;
   const int64_t x1 = (wid + 1) * W / NW;
   int b = locate_sequence(P, a.B, x);
 
-  const uint32_t lut_lane = (uint32_t)__cvta_generic_to_shared(lut) + lane * 4;
+  const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut), lane4 = 4u * lane;
   StageI* my = stages + warp * NSI;
   const uint32_t my_s = (uint32_t)__cvta_generic_to_shared(my);
   const bool own_head = t < G;   // accumulator columns 2t, 2t+1 belong to head t
@@ -168,12 +169,19 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_i8(AttnArgs a) {
       const int64_t t0 = tok0 + (int64_t)MT * i;
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(StageI);
       int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
-      bool ok = true;
-      if (PAGED && r < 0) {
-        ok = false;
-        r = 0;
-        bad |= 1u << (i & 31);
+      if (PAGED) {   // the bit of tile i is rewritten by every issue (tile i + 32 reuses it)
+        bad = (bad & ~(1u << (i & 31))) | ((r < 0 ? 1u : 0u) << (i & 31));
       }
+      if (PAGED && r < 0) {   // invalid block: nothing copied, the tile is masked
+        r = 0;
+      } else if (t0 + MT <= tok1) {   // a full tile: no predicates
+        cp16(sb + d0, p0 + r * 32, true);
+        cp16(sb + d1, p1 + r * 64, true);
+        cp16(sb + d2, p2 + r * 64, true);
+        if (lane < 28) cp16(sb + d3, p3 + r * stride3, true);
+        return;
+      }
+      const bool ok = !(PAGED && ((bad >> (i & 31)) & 1u));
       cp16(sb + d0, p0 + r * 32, ok && t0 + (lane >> 1) < tok1);
       cp16(sb + d1, p1 + r * 64, ok && t0 + (lane >> 2) < tok1);
       cp16(sb + d2, p2 + r * 64, ok && t0 + 8 + (lane >> 2) < tok1);
@@ -286,7 +294,7 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_i8(AttnArgs a) {
       const uint32_t pb0 = movtrans(pack_half2(p0 * (st.vn[g] * vmul), 0.f));
       const uint32_t pb1 = movtrans(pack_half2(p1 * (st.vn[g + 8] * vmul), 0.f));
 
-      value_tile(o, st.v, pb0, pb1, lut_lane, g, t);
+      value_tile_w(o, st.v, pb0, pb1, lut_s, lane4, g, t);
       __syncwarp();
     }
     cp_wait<0>();
@@ -342,21 +350,21 @@ QopPlan attn_i8_qop(const tq_ctx* c, const AttnArgs& a, unsigned char* img) {
 cudaError_t launch_attn_i8(const tq_ctx* c, const AttnArgs& a_in, float* out, cudaStream_t s) {
   AttnArgs a = a_in;
   if (!a.tiles || !a.qimg) return cudaErrorInvalidValue;
-  // At least four tiles per warp, at most attn_seg_max_warps warps; the
+  // One CTA of twelve warps per SM (at least four tiles per warp); the
   // kernel trims the warp count to the real tile count.
   const int64_t wmax = (int64_t)a.B * a.Hkv * ((a.max_T + MT - 1) / MT);
-  int64_t blocks = (wmax + 4 * MW - 1) / (4 * MW);
-  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms * 3 ? (int64_t)c->sms * 3 : blocks);
-  a.nw = (int)(blocks * MW);
+  int64_t blocks = (wmax + 4 * MWI - 1) / (4 * MWI);
+  blocks = blocks < 1 ? 1 : (blocks > (int64_t)c->sms ? (int64_t)c->sms : blocks);
+  a.nw = (int)(blocks * MWI);
   a.wpu = 1;
   const bool paged = a.block_table != nullptr;
   switch (a.G * 2 + (paged ? 1 : 0)) {
-    case 2: k_attn_i8<1, false><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
-    case 3: k_attn_i8<1, true><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
-    case 4: k_attn_i8<2, false><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
-    case 5: k_attn_i8<2, true><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
-    case 8: k_attn_i8<4, false><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
-    case 9: k_attn_i8<4, true><<<(unsigned)blocks, MW * 32, SMEM_I8, s>>>(a); break;
+    case 2: k_attn_i8<1, false><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
+    case 3: k_attn_i8<1, true><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
+    case 4: k_attn_i8<2, false><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
+    case 5: k_attn_i8<2, true><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
+    case 8: k_attn_i8<4, false><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
+    case 9: k_attn_i8<4, true><<<(unsigned)blocks, MWI * 32, SMEM_I8, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();

@@ -405,9 +405,9 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
       int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
       // an invalid block copies nothing: every chunk is zero-filled
       const int64_t tend = (PAGED && r < 0) ? t0 : tok1;
-      if (PAGED && r < 0) {
-        r = 0;
-        bad |= 1u << (k & 31);
+      if (PAGED) {   // the bit of ring tile k is rewritten by every issue (tile k + 32 reuses it)
+        bad = (bad & ~(1u << (k & 31))) | ((r < 0 ? 1u : 0u) << (k & 31));
+        r = r < 0 ? 0 : r;
       }
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
 #pragma unroll

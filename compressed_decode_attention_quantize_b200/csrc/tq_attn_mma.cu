@@ -241,10 +241,10 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
       const uint32_t sb = my_s + stage * (uint32_t)sizeof(Stage);
       int64_t r = kv_off<PAGED>(a, b, kvh, t0);   // records of tokens t0.. (16 in a row)
       bool ok = true;
-      if (PAGED && r < 0) {
-        ok = false;
-        r = 0;
-        bad |= 1u << (k & 31);
+      if (PAGED) {   // the bit of ring tile k is rewritten by every issue (tile k + 32 reuses it)
+        ok = r >= 0;
+        bad = (bad & ~(1u << (k & 31))) | ((ok ? 0u : 1u) << (k & 31));
+        r = ok ? r : 0;
       }
       cp16(sb + d0, p0 + r * 32, ok && t0 + (lane >> 1) < tok1);
       cp16(sb + d1, p1 + r * 64, ok && t0 + (lane >> 2) < tok1);

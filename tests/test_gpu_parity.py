@@ -958,6 +958,38 @@ def test_paged_decode_matches_oracle(cuda, fmt, Hq, bs):
         P.check_attention(tab, qn[b:b + 1], kb, vb, np.array([L]), Hkv, gn[b:b + 1])
 
 
+@pytest.mark.parametrize("fmt,Hq", [("k3v4", 32), ("k3v4", 64), ("k4v4", 32)])
+def test_paged_decode_long_pieces_mask_only_invalid_tiles(cuda, fmt, Hq):
+    """Pieces of more than 32 tiles per warp (1 x 8 heads x 131072 tokens):
+    an invalid first block masks its own tiles only.  The kernels keep one
+    mask bit per tile modulo 32, so tile k + 32 of the same warp reuses tile
+    k's bit; value vectors 1000x larger at the tokens of those later tiles
+    (tiles 32-35 and 128-131 of the first piece) make a stale bit visible."""
+    c = tq.Context.variant(fmt, 128, seed=12)
+    tab = P.oracle_tables(c)
+    B, Hkv, d, T, bs = 1, 8, 128, 131072, 64
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=61).to(cuda)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=62).to(cuda)
+    V[0, 0, 512:576] *= 1000
+    V[0, 0, 2048:2112] *= 1000
+    kc, vc = c.quantize(K, tq.TQ_KEY), c.quantize(V, tq.TQ_VALUE)
+    del K, V
+    mb = T // bs
+    perm = torch.randperm(B * mb, generator=torch.Generator().manual_seed(13)).to(torch.int32)
+    kp, vp = _to_paged(kc, B, Hkv, T, bs, perm), _to_paged(vc, B, Hkv, T, bs, perm)
+    table = perm.reshape(B, mb).clone()
+    table[0, 0] = -1   # tokens [0, 64) masked
+    lens = torch.tensor([T], dtype=torch.int32)
+    q = tq_inputs.iid((B, Hq, d), seed=63, dtype=torch.bfloat16)
+    got = c.attn_decode_paged(q.to(cuda), kp, vp, table.to(cuda), lens.to(cuda))
+    torch.cuda.synchronize()
+    G = Hq // Hkv
+    kh = _drop_tokens(P.packed_np({k: (None if v is None else v[:, :1]) for k, v in kc.items()}), 0, 0, bs)
+    vh = _drop_tokens(P.packed_np({k: (None if v is None else v[:, :1]) for k, v in vc.items()}), 0, 0, bs)
+    P.check_attention(tab, q[:, :G].double().numpy(), kh, vh, np.array([T - bs]), 1,
+                      got[:, :G].cpu().numpy())
+
+
 @pytest.mark.parametrize("fmt,Hq", [("k3v4", 8), ("k4v4", 16), ("k3v4_nc", 8)])
 def test_paged_decode_step_matches_oracle(cuda, fmt, Hq):
     """decode_step_paged against the oracle: the appended tokens are read back
