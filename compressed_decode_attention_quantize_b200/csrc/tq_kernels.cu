@@ -14,6 +14,7 @@
 #include <cmath>
 
 #include "tq_internal.h"
+#include "tq_qop.cuh"
 
 namespace tqk {
 
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(256) k_quantize_small(QuantArgs a, int dpad) {
 // Tile prefix of the segment-partitioned decode: tiles[b] = Hkv * sum over
 // b' < b of ceil(len_b' / 16), len = min(max(seq_lens, 0), max_T); one block.
 __device__ void tile_plan(const int32_t* seq_lens, int B, int Hkv, int64_t max_T, int64_t* tiles) {
-  __shared__ int64_t s_w[8];
+  __shared__ int64_t s_w[32];
   __shared__ int64_t s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
   if (tid == 0) {
@@ -533,8 +534,6 @@ __device__ void write_qop(const QopPlan& P, const float (&qv)[PR], const float (
     }
   }
   __syncthreads();
-  const double c0 = P.c0, w0 = (double)P.c1 - c0, w1 = (double)P.c2 - c0;
-  const double wmax = fmax(fabs(w0), fabs(w1));
 #pragma unroll
   for (int r = 0; r < PR; ++r) {
     if (r >= nr) break;   // uniform over the block
@@ -546,46 +545,13 @@ __device__ void write_qop(const QopPlan& P, const float (&qv)[PR], const float (
       ms = fmaxf(ms, s_red[r][w][2]);
       ss += s_red[r][w][3];
     }
-    // 2^e <= max |w q'| < 2^(e+1), S = 29 - e: |Q| < 2^30 at p = 0.
-    const double mk = wmax * mq;
-    const int S = mk > 0.0 ? 29 - ilogb(mk) : 0;
-    const int S2 = ms > 0.f ? 29 - ilogb((double)ms) : 0;
+    const QopExp ex = qop_exponents(P, mq, ms);
     const int64_t row = row0 + r;
     const int64_t b = row / P.Hq;
     const int h = (int)(row % P.Hq), kvh = h / P.G, hg = h % P.G;
     unsigned char* img = P.img + (b * (P.Hq / P.G) + kvh) * (int64_t)kQopBytes;
-    auto put = [&](int reg, int tt, int e, int64_t Q) {
-      // four balanced digits, digit l to column 2 hg + l % 2 of N tile l / 2
-#pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        const int dg = (int)(signed char)(Q & 0xFF);
-        Q = (Q - dg) >> 8;
-        const int rr = reg + 2 * (l >> 1);
-        const int ln = 4 * (2 * hg + (l & 1)) + tt;
-        img[(((rr >> 2) * 32 + ln) * 4 + (rr & 3)) * 4 + e] = (unsigned char)(dg & 0xFF);
-      }
-    };
-    {
-      const double q = qv[r];
-#pragma unroll
-      for (int pl = 0; pl < 2; ++pl) {
-        const int bit = 2 * (j & 15) + pl, w = j >> 4, p = bit & 7;
-        const int64_t Q = llrint(ldexp((pl ? w1 : w0) * q, S - p));
-        put(4 * p + (w >> 2), w & 3, bit >> 3, Q);
-      }
-      const int bit = j & 31, p = bit & 7;
-      const int64_t Q = llrint(ldexp((double)sv[r], S2 - p));
-      put(32 + 4 * (p >> 1) + (p & 1), j >> 5, bit >> 3, Q);
-    }
-    if (j == 0) {
-      const double sl = P.scale_log2;
-      float4 cst;
-      cst.x = (float)ldexp(sl, -S);
-      cst.y = (float)(c0 * sq * sl);
-      cst.z = (float)ldexp(2.0 * (double)P.cq * sl, -S2);
-      cst.w = (float)(-ss * (double)P.cq * sl);
-      reinterpret_cast<float4*>(img + kQopRegs * 32 * 4)[hg] = cst;
-    }
+    qop_put_coord(P, img, hg, j, qv[r], sv[r], ex);
+    if (j == 0) qop_put_constants(P, img, hg, ex, sq, ss);
   }
 }
 
@@ -655,6 +621,323 @@ __global__ void __launch_bounds__(256) k_step_prep(StepPrep s, int d, int dpad, 
   }
   blk -= s.nkv;
   prerotate_body<2>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, sh, &s.qop);
+  if (blk == 0) {
+    for (int b = threadIdx.x; b < s.B; b += blockDim.x) {
+      const int64_t p = s.pos[b];
+      s.lens[b] = (int32_t)max((int64_t)0, min(p + 1, s.max_T));
+    }
+    __syncthreads();
+    if (s.tiles) tile_plan(s.lens, s.B, s.Hkv, s.max_T, s.tiles);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Latency-shaped small kernels for d <= 128 (dpad <= 128): the decode step's
+// appends, the query pre-rotation and the merge process a few vectors each,
+// so their time is a chain of dependent memory round trips, not bandwidth.
+// A CTA of FAST_T = 512 threads splits every matrix product four ways over
+// the k range: thread (j, quarter) = (tid % 128, tid / 128) reads its 32
+// matrix entries in one unrolled burst of independent L1/L2 loads (no chain
+// of streamed chunks), and the four partial sums meet in shared memory as
+// (p0 + p1) + (p2 + p3).  Every caller of these helpers uses the same order,
+// so an append inside the decode step and a separate append (or the query
+// rotation of the decode step and of a separate decode) agree bit for bit.
+// ----------------------------------------------------------------------------
+constexpr int FAST_T = 512;
+constexpr int FAST_KQ = 32;   // k entries per thread: four quarters cover d <= 128
+
+// This thread's entries M[k][j] of its k quarter (M is [d][dpad], k-major;
+// zero beyond d or dpad): issued together, one round trip.  The loads are
+// volatile asm so that they stay where the caller puts them (ahead of the
+// other round trips) instead of being sunk to their first use.
+__device__ __forceinline__ void load_quarter(const float* __restrict__ M, int d, int dpad, float (&w)[FAST_KQ]) {
+  const int j = threadIdx.x & 127, k0 = (threadIdx.x >> 7) * FAST_KQ;
+  const bool jok = j < dpad;
+#pragma unroll
+  for (int kk = 0; kk < FAST_KQ; ++kk) {
+    float v = 0.f;
+    if (jok && k0 + kk < d)
+      asm volatile("ld.global.nc.f32 %0, [%1];\n" : "=f"(v) : "l"(M + (size_t)(k0 + kk) * dpad + j));
+    w[kk] = v;
+  }
+}
+// acc[r] = sum over this thread's k quarter of w[kk] x[r][k0 + kk] (w from
+// load_quarter; x rows of 128 floats with zeros beyond d).
+template <int R>
+__device__ __forceinline__ void dot_w(const float (&w)[FAST_KQ], const float* x, float (&acc)[R]) {
+  const int k0 = (threadIdx.x >> 7) * FAST_KQ;
+#pragma unroll
+  for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < FAST_KQ; kk += 4) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 x4 = *reinterpret_cast<const float4*>(x + r * 128 + k0 + kk);
+      acc[r] = fmaf(w[kk], x4.x, acc[r]);
+      acc[r] = fmaf(w[kk + 1], x4.y, acc[r]);
+      acc[r] = fmaf(w[kk + 2], x4.z, acc[r]);
+      acc[r] = fmaf(w[kk + 3], x4.w, acc[r]);
+    }
+  }
+}
+// The four quarters' partial sums of output (r, j) (red: [4][R][128]).
+__device__ __forceinline__ float sum_quarters(const float* red, int R, int r, int j) {
+  return (red[(0 * R + r) * 128 + j] + red[(1 * R + r) * 128 + j]) +
+         (red[(2 * R + r) * 128 + j] + red[(3 * R + r) * 128 + j]);
+}
+
+// quantize_small_body for QS vectors per 512-thread CTA: the coordinate
+// threads tid < dpad (warps 0 .. dpad / 32 - 1) take the roles of the
+// small body's threads (Lloyd-Max index, packing, QJL signs); all threads
+// take part in the two matrix products.  sh: [QS][128] + [4][QS][128] floats.
+template <int QS>
+__device__ __forceinline__ void quantize_fast_body(const QuantArgs& a, int dpad, int64_t blk, float* sh) {
+  float* xs = sh;                // [QS][128]: x, later r
+  float* red = sh + QS * 128;    // [4][QS][128]
+  __shared__ float s_nx[QS][4], s_nc[QS][4], s_nr[QS][4];
+  __shared__ float s_cen[kMaxLevels], s_bnd[kMaxLevels];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, j = tid & 127;
+  const int nwarp = dpad >> 5;
+  const bool cw = tid < dpad;    // a coordinate thread (j = tid)
+  const int64_t v0 = blk * QS;
+  const int nv = (int)min((int64_t)QS, a.n - v0);
+  for (int e = tid; e < kMaxLevels; e += blockDim.x) {
+    s_cen[e] = (e < (1 << a.bits)) ? a.cen[e] : 0.f;
+    s_bnd[e] = (e < a.nbnd) ? a.bnd[e] : INFINITY;
+  }
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    float xj = 0.f;
+    if (tid < 128) {
+      xj = (u < nv && j < a.d) ? load_elem(a.x, a.dtype, (v0 + u) * a.ld + j) : 0.f;
+      xs[u * 128 + j] = xj;
+    }
+    const float t = warp_sum(xj * xj);
+    if (lane == 0 && warp < 4) s_nx[u][warp] = t;
+  }
+  __syncthreads();
+  float nrm[QS];
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    float t = 0.f;
+    for (int w = 0; w < nwarp; ++w) t += s_nx[u][w];
+    nrm[u] = sqrtf(t);
+  }
+  {
+    float acc[QS], wp[FAST_KQ];   // (loaded here: two CTAs per SM fit the registers)
+    load_quarter(a.PiT, a.d, dpad, wp);
+    dot_w<QS>(wp, xs, acc);
+#pragma unroll
+    for (int u = 0; u < QS; ++u) red[((tid >> 7) * QS + u) * 128 + j] = acc[u];
+  }
+  __syncthreads();
+  float r[QS];
+  int ids[QS];
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    ids[u] = 0;
+    r[u] = 0.f;
+    if (cw) {
+      const float pj = sum_quarters(red, QS, u, j);
+      const float y = (nrm[u] > 0.f && j < a.d) ? pj / nrm[u] : 0.f;
+      ids[u] = lm_index(y, s_bnd, a.nbnd);
+      r[u] = (j < a.d) ? y - s_cen[ids[u]] : 0.f;
+    }
+  }
+  if (a.nc) {   // uniform; norm correction: store n / |c[idx]| (MSE-only, no QJL stage follows)
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      const float cj = (cw && j < a.d) ? s_cen[ids[u]] : 0.f;
+      const float cc = warp_sum(cj * cj);
+      if (lane == 0 && warp < 4) s_nc[u][warp] = cc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      float t = 0.f;
+      for (int w = 0; w < nwarp; ++w) t += s_nc[u][w];
+      nrm[u] = nrm[u] / sqrtf(t);
+    }
+  }
+  const int i32 = j >> 5;
+  if (warp < nwarp) {   // warp-uniform: the coordinate warps pack and store
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      if (u >= nv) continue;
+      const int64_t rec = out_record(a, v0 + u);
+      if (rec < 0) continue;   // uniform (one sequence per vector)
+      const uint32_t iv = (j < a.d) ? (uint32_t)ids[u] : 0u;
+      if (a.bits == 3) {
+        const int w2 = (a.d + 15) >> 4;
+        const uint32_t lo = field_word(iv & 3u, 2, lane);
+        const uint32_t hi = field_word(iv >> 2, 1, lane);
+        const int wlo = 2 * i32 + (lane >> 4);
+        if ((lane & 15) == 0 && wlo < w2) a.codes[rec * a.words + wlo] = lo;
+        if (lane == 0) a.codes[rec * a.words + w2 + i32] = hi;
+      } else {
+        const int per = 32 / a.bits;
+        const uint32_t wv = field_word(iv, a.bits, lane);
+        const int wi = a.bits * i32 + lane / per;
+        if (lane % per == 0 && wi < a.words) a.codes[rec * a.words + wi] = wv;
+      }
+      if (j == 0) store_norm(a.norm, rec, nrm[u], a.nf16);
+    }
+  }
+  if (a.m == 0) return;
+#pragma unroll
+  for (int u = 0; u < QS; ++u) {
+    if (tid < 128) xs[u * 128 + j] = r[u];   // r = 0 beyond d
+    const float t = warp_sum(r[u] * r[u]);
+    if (lane == 0 && warp < 4) s_nr[u][warp] = t;
+  }
+  __syncthreads();   // also: every read of red above is done
+  {
+    float acc[QS], ws[FAST_KQ];
+    load_quarter(a.ST, a.d, dpad, ws);
+    dot_w<QS>(ws, xs, acc);
+#pragma unroll
+    for (int u = 0; u < QS; ++u) red[((tid >> 7) * QS + u) * 128 + j] = acc[u];
+  }
+  __syncthreads();
+  if (warp < nwarp) {
+#pragma unroll
+    for (int u = 0; u < QS; ++u) {
+      float rho = 0.f;
+      for (int w = 0; w < nwarp; ++w) rho += s_nr[u][w];
+      rho = sqrtf(rho);
+      const float sj = sum_quarters(red, QS, u, j);
+      const uint32_t bits = __ballot_sync(0xffffffffu, sj >= 0.f && j < a.m);
+      if (u >= nv) continue;
+      const int64_t rec = out_record(a, v0 + u);
+      if (rec < 0) continue;
+      if (lane == 0 && j < a.m) a.qjl[rec * ((a.m + 31) >> 5) + i32] = bits;
+      if (j == 0) a.rnorm[rec] = nrm[u] * rho;
+    }
+  }
+}
+
+template <int QS>
+__global__ void __launch_bounds__(FAST_T) k_quantize_fast(QuantArgs a, int dpad) {
+  __shared__ __align__(16) float sh[5 * QS * 128];
+  quantize_fast_body<QS>(a, dpad, blockIdx.x, sh);
+}
+
+// Query rows row0 .. row0 + R - 1 (R rows of one CTA): q' = Pi q, s = S q',
+// written to qr / qs ([rows][dpad]) and, with qop->img, as int8 operand
+// images (tq_qop.cuh).  sh: [R][128] q', [R][128] s, [4][R][128].
+template <int R, bool HOIST>
+__device__ __forceinline__ void prerotate_fast_body(const void* q, int dtype, int64_t rows, int d, int dpad,
+                                                    int m, const float* PiT, const float* ST, float* qr, float* qs,
+                                                    int64_t blk, const QopPlan* qop, float* sh) {
+  float* xs = sh;               // [R][128]: q, then q'
+  float* ys = sh + R * 128;     // [R][128]: s
+  float* red = ys + R * 128;    // [4][R][128]
+  __shared__ float s_sum[R][2];
+  __shared__ int s_ex[R][2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, j = tid & 127;
+  const int64_t row0 = blk * R;
+  const int nr = (int)min((int64_t)R, rows - row0);
+  float wm[2][FAST_KQ];   // quarters of Pi^T and S^T: up front (HOIST) or before each product
+  if (HOIST) {
+    load_quarter(PiT, d, dpad, wm[0]);
+    load_quarter(ST, d, dpad, wm[1]);
+  }
+  for (int e = tid; e < R * 128; e += blockDim.x) {
+    const int r = e >> 7, jj = e & 127;
+    xs[e] = (r < nr && jj < d) ? load_elem(q, dtype, (row0 + r) * d + jj) : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    float acc[R];
+    if (!HOIST) load_quarter(pass == 0 ? PiT : ST, d, dpad, wm[pass]);
+    dot_w<R>(wm[pass], xs, acc);
+#pragma unroll
+    for (int r = 0; r < R; ++r) red[((tid >> 7) * R + r) * 128 + j] = acc[r];
+    __syncthreads();
+    float* y = pass == 0 ? xs : ys;   // q' replaces q: every read of xs is done
+    float* g = pass == 0 ? qr : qs;
+    for (int e = tid; e < R * 128; e += blockDim.x) {
+      const int r = e >> 7, jj = e & 127;
+      float v = sum_quarters(red, R, r, jj);
+      if (pass == 1 && jj >= m) v = 0.f;
+      y[e] = v;
+      if (r < nr && jj < dpad) g[(row0 + r) * dpad + jj] = v;
+    }
+    __syncthreads();
+  }
+  if (!qop || !qop->img) return;
+  if (warp < R) {   // head statistics of row warp: max |q'|, sum q', max |s|, sum s
+    float mq = 0.f, sq = 0.f, ms = 0.f, ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float qv = xs[warp * 128 + lane + 32 * i], sv = ys[warp * 128 + lane + 32 * i];
+      mq = fmaxf(mq, fabsf(qv));
+      sq += qv;
+      ms = fmaxf(ms, fabsf(sv));
+      ss += sv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    if (lane == 0) {
+      const QopExp ex = qop_exponents(*qop, mq, ms);
+      s_ex[warp][0] = ex.S;
+      s_ex[warp][1] = ex.S2;
+      s_sum[warp][0] = sq;
+      s_sum[warp][1] = ss;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nr * 128; e += blockDim.x) {
+    const int r = e >> 7, jj = e & 127;
+    const int64_t row = row0 + r;
+    const int64_t b = row / qop->Hq;
+    const int h = (int)(row % qop->Hq), kvh = h / qop->G, hg = h % qop->G;
+    unsigned char* img = qop->img + (b * (qop->Hq / qop->G) + kvh) * (int64_t)kQopBytes;
+    QopExp ex;
+    ex.S = s_ex[r][0];
+    ex.S2 = s_ex[r][1];
+    qop_put_coord(*qop, img, hg, jj, xs[e], ys[e], ex);
+    if (jj == 0) qop_put_constants(*qop, img, hg, ex, (double)s_sum[r][0], (double)s_sum[r][1]);
+  }
+}
+
+constexpr int FAST_R = 4;   // query rows per pre-rotation CTA
+
+__global__ void __launch_bounds__(FAST_T) k_prerotate_fast(const void* q, int dtype, int64_t rows, int d, int dpad,
+                                                         int m, const float* PiT, const float* ST, float* qr,
+                                                         float* qs, const int32_t* seq_lens, int B, int Hkv,
+                                                         int64_t max_T, int64_t* tiles, QopPlan qop) {
+  __shared__ __align__(16) float sh[6 * FAST_R * 128];
+  prerotate_fast_body<FAST_R, true>(q, dtype, rows, d, dpad, m, PiT, ST, qr, qs, blockIdx.x, &qop, sh);
+  if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
+}
+
+// The decode step's preparation with the fast bodies: blocks [0, n) append
+// the new keys, [n, 2n) the new values (n = B Hkv), the rest pre-rotate
+// FAST_R query rows each; the first query block writes the lengths and the
+// tile prefix.
+__global__ void __launch_bounds__(FAST_T) k_step_prep_fast(StepPrep s, int d, int dpad, int m, const float* PiT,
+                                                         const float* ST) {
+  __shared__ __align__(16) float sh[6 * FAST_R * 128];
+  int64_t blk = blockIdx.x;
+  if (blk < s.nkv) {
+    quantize_fast_body<1>(s.k, dpad, blk, sh);
+    return;
+  }
+  blk -= s.nkv;
+  if (blk < s.nkv) {
+    quantize_fast_body<1>(s.v, dpad, blk, sh);
+    return;
+  }
+  blk -= s.nkv;
+  // matrix loads before each product: two CTAs per SM fit the registers
+  prerotate_fast_body<FAST_R, false>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, &s.qop, sh);
   if (blk == 0) {
     for (int b = threadIdx.x; b < s.B; b += blockDim.x) {
       const int64_t p = s.pos[b];
@@ -927,6 +1210,105 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* part, int split
 }
 
 // ----------------------------------------------------------------------------
+// The merge for d <= 128, one 512-thread CTA per KV group (its G <= 16 rows
+// share the segment path's slot range): per row, weights w_s / L from the
+// partials' (m, l) (one warp per row), o = sum (w_s / L) o_s, then
+// out = Pi^T o with the k range of the product split four ways as in
+// dot_w (Pi is [d][d] row-major: out_i = sum_j Pi[j][i] o_j), four
+// rows at a time.  sh: [Gp][128] o (Gp = G rounded up to 4, zero padding
+// rows), [4][4][128] partial sums, [G][slot_cap] weights.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(FAST_T) k_attn_merge_fast(const float* part, int splits, int d, int dpad,
+                                                          const float* Pi, float* out, const int64_t* tiles, int B,
+                                                          int Hq, int Hkv, int nw, int wpu, int slot_cap) {
+  extern __shared__ __align__(16) float sh[];
+  const int G = Hq / Hkv, Gp = (G + 3) & ~3;
+  float* so = sh;                       // [Gp][128]
+  float* red = so + Gp * 128;           // [4][4][128]
+  float* sw = red + 4 * 4 * 128;        // [G][slot_cap]
+  const int u = blockIdx.x, b = u / Hkv, kvh = u % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const float* pr0;
+  int64_t sstride, rstride;
+  int nsl;
+  if (tiles) {
+    const int64_t W = tiles[B];
+    const int64_t tb = (tiles[b + 1] - tiles[b]) / Hkv;
+    nsl = 0;
+    pr0 = part;
+    if (tb > 0) {
+      const int64_t N = min((int64_t)nw, W);
+      const int64_t S = tiles[b] + kvh * tb, E = S + tb;
+      const int64_t f = ((S + 1) * N + W - 1) / W - 1, l = (E * N + W - 1) / W - 1;
+      pr0 = part + wpu * (f + (int64_t)b * Hkv + kvh) * G * (int64_t)(dpad + 2);
+      nsl = (int)(wpu * (l - f + 1));
+    }
+    sstride = (int64_t)G * (dpad + 2);
+    rstride = dpad + 2;
+  } else {
+    pr0 = part + (int64_t)u * G * splits * (dpad + 2);
+    sstride = dpad + 2;
+    rstride = (int64_t)splits * (dpad + 2);
+    nsl = splits;
+  }
+  for (int r = warp; r < G; r += nwarp) {
+    const float* pr = pr0 + r * rstride;
+    // (m, l) of the first 32 slots stay in registers; more slots are re-read
+    const float2 ml0 = lane < nsl ? *reinterpret_cast<const float2*>(pr + lane * sstride)
+                                  : make_float2(-INFINITY, 0.f);
+    float mx = ml0.x;
+    for (int sl = lane + 32; sl < nsl; sl += 32) mx = fmaxf(mx, pr[sl * sstride]);
+    mx = warp_max(mx);
+    float lsum = 0.f;
+    for (int sl = lane; sl < nsl; sl += 32) {
+      const float2 ml = sl < 32 ? ml0 : *reinterpret_cast<const float2*>(pr + sl * sstride);
+      const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mx);
+      sw[r * slot_cap + sl] = w;
+      lsum = fmaf(w, ml.y, lsum);
+    }
+    lsum = warp_sum(lsum);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    __syncwarp();
+    for (int sl = lane; sl < nsl; sl += 32) sw[r * slot_cap + sl] *= inv;
+  }
+  __syncthreads();
+  for (int e = tid; e < Gp * 128; e += blockDim.x) {
+    const int r = e >> 7, j = e & 127;
+    float tot = 0.f;
+    if (r < G && j < d) {
+      const float* pr = pr0 + r * rstride + 2 + j;
+      const float* wr = sw + r * slot_cap;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int sl = 0;
+      for (; sl + 8 <= nsl; sl += 8) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[v] = fmaf(wr[sl + v], pr[(int64_t)(sl + v) * sstride], acc[v]);
+      }
+      for (; sl < nsl; ++sl) acc[0] = fmaf(wr[sl], pr[(int64_t)sl * sstride], acc[0]);
+      tot = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    }
+    so[e] = tot;
+  }
+  __syncthreads();
+  // out_i = sum_j Pi[j][i] o_j: dot_w over Pi ([d][d], k = j) with x = o
+  float wpi[FAST_KQ];   // this thread's quarter of Pi
+  load_quarter(Pi, d, d, wpi);
+  for (int r0 = 0; r0 < G; r0 += 4) {
+    float acc[4];
+    dot_w<4>(wpi, so + r0 * 128, acc);
+    const int i = tid & 127, qt = tid >> 7;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) red[(qt * 4 + r) * 128 + i] = acc[r];
+    __syncthreads();
+    for (int e = tid; e < 4 * 128; e += blockDim.x) {
+      const int r = e >> 7, i2 = e & 127;
+      if (r0 + r < G && i2 < d) out[((int64_t)u * G + r0 + r) * d + i2] = sum_quarters(red, 4, r, i2);
+    }
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Logits of nq queries against nk packed keys.  Each CTA pre-rotates its QB
 // queries into shared memory, then thread t scores key t of its slice.
 // ----------------------------------------------------------------------------
@@ -1117,7 +1499,15 @@ cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s)
 cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;
   // One vector per block while that still fills the GPU; eight per block
-  // (one read of Pi and S for all eight) beyond.
+  // (one read of Pi and S for all eight) beyond.  d <= 128: the fast bodies
+  // (the same per-vector arithmetic for both batchings).
+  if (c->dpad <= 128) {
+    if (a.n <= 1024)
+      k_quantize_fast<1><<<(unsigned)a.n, FAST_T, 0, s>>>(a, c->dpad);
+    else
+      k_quantize_fast<8><<<(unsigned)((a.n + 7) / 8), FAST_T, 0, s>>>(a, c->dpad);
+    return cudaGetLastError();
+  }
   if (a.n <= 1024) {
     k_quantize_small<1><<<(unsigned)a.n, c->dpad, (1 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(a, c->dpad);
   } else {
@@ -1128,6 +1518,12 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
 }
 
 cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s) {
+  if (c->dpad <= 128) {
+    const int64_t blocks = 2 * sp.nkv + (sp.qrows + FAST_R - 1) / FAST_R;
+    if (blocks == 0) return cudaSuccess;
+    k_step_prep_fast<<<(unsigned)blocks, FAST_T, 0, s>>>(sp, c->d, c->dpad, c->qjl_m, c->PiT, c->ST);
+    return cudaGetLastError();
+  }
   const int64_t blocks = 2 * sp.nkv + (sp.qrows + 1) / 2;
   if (blocks == 0) return cudaSuccess;
   k_step_prep<<<(unsigned)blocks, c->dpad, (2 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
@@ -1144,7 +1540,10 @@ cudaError_t launch_prerotate(const tq_ctx* c, const void* q, int dtype, int64_t 
   int64_t* tl = plan ? plan->tiles : nullptr;
   QopPlan qp{};
   if (qop) qp = *qop;
-  if (rows <= 1024) {
+  if (c->dpad <= 128) {
+    k_prerotate_fast<<<(unsigned)((rows + FAST_R - 1) / FAST_R), FAST_T, 0, s>>>(
+        q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl, qp);
+  } else if (rows <= 1024) {
     k_prerotate<2><<<(unsigned)((rows + 1) / 2), c->dpad, (2 + 2 * MV_KC) * c->dpad * sizeof(float), s>>>(
         q, dtype, rows, c->d, c->dpad, c->qjl_m, c->PiT, c->ST, qr, qs, sl, pB, pH, pT, tl, qp);
   } else {
@@ -1169,8 +1568,18 @@ int attn_splits(const tq_ctx* c, int B, int Hkv, int64_t max_T, int* chunk) {
   return (int)splits;
 }
 
+// Shared memory limit of the fast merge.
+constexpr size_t kMergeFastSmem = 200 * 1024;
+
 cudaError_t launch_attn_merge(const tq_ctx* c, const AttnArgs& a, float* out, cudaStream_t s) {
   const int slots = a.tiles ? a.nw * a.wpu : a.splits;
+  const int G = a.Hq / a.Hkv, Gp = (G + 3) & ~3;
+  const size_t fsm = ((size_t)Gp * 128 + 4 * 4 * 128 + (size_t)G * slots) * sizeof(float);
+  if (c->dpad <= 128 && fsm <= kMergeFastSmem) {
+    k_attn_merge_fast<<<(unsigned)((int64_t)a.B * a.Hkv), FAST_T, fsm, s>>>(
+        a.part, a.splits, c->d, c->dpad, c->Pi_f, out, a.tiles, a.B, a.Hq, a.Hkv, a.nw, a.wpu, slots);
+    return cudaGetLastError();
+  }
   k_attn_merge<<<(unsigned)(a.B * a.Hq), 128, (c->dpad + slots) * sizeof(float), s>>>(
       a.part, a.splits, c->d, c->dpad, c->Pi_f, out, a.tiles, a.B, a.Hq, a.Hkv, a.nw, a.wpu);
   return cudaGetLastError();
@@ -1312,6 +1721,7 @@ cudaError_t configure_kernels() {
   if ((e = cudaFuncSetAttribute(k_prerotate<2>, ms, small_smem))) return e;
   if ((e = cudaFuncSetAttribute(k_prerotate<8>, ms, small_smem))) return e;
   if ((e = cudaFuncSetAttribute(k_step_prep, ms, small_smem))) return e;
+  if ((e = cudaFuncSetAttribute(k_attn_merge_fast, ms, (int)kMergeFastSmem))) return e;
   if ((e = configure_quant_tc()) != cudaSuccess) return e;
   if ((e = configure_attn_lut()) != cudaSuccess) return e;
   if ((e = configure_attn_i8()) != cudaSuccess) return e;
