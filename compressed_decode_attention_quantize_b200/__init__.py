@@ -50,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_version": (ctypes.c_char_p, []),
         "tq_device_fault": (I, [ctypes.POINTER(ctypes.c_int)]),
+        "tq_set_wait_limit": (I, [P, I]),
         "tq_init": (P, [I, I, I, I, U64]),
         "tq_init_ex": (P, [I, I, I, I, U64, I]),
         "tq_destroy": (None, [P]),
@@ -80,7 +81,7 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_init", "tq_init_ex", "tq_destroy", "tq_layout", "tq_host_tables",
+EXPORTED = ("tq_last_error", "tq_version", "tq_device_fault", "tq_set_wait_limit", "tq_init", "tq_init_ex", "tq_destroy", "tq_layout", "tq_host_tables",
             "tq_export_tables", "tq_quantize", "tq_quantize_append", "tq_dequantize", "tq_logits",
             "tq_attn_workspace_bytes", "tq_attn_decode", "tq_attn_decode_static",
             "tq_attn_static_scratch_bytes", "tq_decode_step", "tq_quantize_append_paged",
@@ -132,6 +133,12 @@ def tq_device_fault() -> int:
     v = ctypes.c_int(0)
     _check(_lib.tq_device_fault(ctypes.byref(v)))
     return v.value
+
+
+def tq_set_wait_limit(ctx, polls: int) -> None:
+    """Test diagnostic: the context's tensor-core kernels give up their main
+    bounded waits after `polls` polls (0 = the full limit)."""
+    _check(_lib.tq_set_wait_limit(ctx, polls))
 
 
 def tq_version() -> str:
@@ -195,6 +202,12 @@ class Context:
             raise ValueError(f"unknown variant {name!r}; known: {', '.join(VARIANTS)}")
         bits_k, bits_v, qjl, nc = VARIANTS[name]
         return cls(d, bits_k, bits_v, d if qjl else 0, seed, nc_k=nc, nc_v=nc, norm_f16=norm_f16)
+
+    def set_wait_limit(self, polls: int) -> None:
+        """Test diagnostic (tq_set_wait_limit): main bounded waits of this
+        context's tensor-core kernels give up after `polls` polls; 0 restores
+        the full limit."""
+        tq_set_wait_limit(self.ptr, polls)
 
     def close(self):
         if getattr(self, "ptr", None):

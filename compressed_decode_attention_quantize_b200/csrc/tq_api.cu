@@ -84,6 +84,12 @@ const char* tq_last_error(void) { return g_err.c_str(); }
 
 const char* tq_version(void) { return "libtq 0.1 (sm_100a)"; }
 
+int tq_set_wait_limit(tq_ctx* c, int polls) {
+  if (!c || polls < 0) return fail(TQ_ERR_ARG, "tq_set_wait_limit: null context or negative polls");
+  c->wait_limit = polls;
+  return TQ_OK;
+}
+
 int tq_device_fault(int* code) {
   if (!code) return fail(TQ_ERR_ARG, "tq_device_fault: null output");
   int q = 0, t = 0;
@@ -417,6 +423,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
       t.cen[i] = i < (int)cen.size() ? (float)cen[i] : 0.f;
       t.bnd[i] = i < (int)bnd.size() ? (float)bnd[i] : INFINITY;
     }
+    t.wait_limit = c->wait_limit;
     cudaError_t e = tqk::launch_quant_tc(t, c->sms, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;

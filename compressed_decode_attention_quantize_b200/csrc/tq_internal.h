@@ -46,6 +46,10 @@ struct tq_ctx {
   const void* tc_pil = nullptr;   // 2^8 Pi - head, fp16
   const void* tc_s = nullptr;     // S, fp16 (exact)
   const float* tc_snorm = nullptr;  // |S_i|
+  // Polls before a tensor-core kernel's main bounded wait gives up (0 = the
+  // kernels' full limit); set only by tq_set_wait_limit, for testing the
+  // fault path.
+  int wait_limit = 0;
 };
 
 namespace tqh {
@@ -183,6 +187,7 @@ struct QuantTcArgs {
   int64_t max_T;
   float cen[16];
   float bnd[16];
+  int wait_limit;   // polls of the main MMA waits (the full limit when 0)
 };
 
 cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);

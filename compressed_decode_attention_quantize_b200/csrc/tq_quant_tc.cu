@@ -23,8 +23,9 @@
 //
 // Two groups of eight warps per CTA work on different tiles, so one group's
 // MMAs overlap the other's epilogue, and sixteen warps per SM hide latency.
-// Waits on MMA completion are bounded; on timeout the kernel records a fault
-// code, releases its tensor memory and returns.
+// Waits on MMA completion are bounded; on timeout the group waits (with the
+// full limit) for the MMAs it issued, the kernel records a fault code,
+// releases its tensor memory and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -322,7 +323,11 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
       }
       mma_commit(bar_rot);
     }
-    if (grp_any(gi, !mbar_wait(bar_rot, iter & 1))) { fault = true; break; }
+    if (grp_any(gi, !mbar_wait(bar_rot, iter & 1, a.wait_limit))) {
+      mbar_wait(bar_rot, iter & 1);   // drain: the group's MMAs finish before TMEM is released
+      fault = true;
+      break;
+    }
     tc_after_sync();
 
     // ---- epilogue 1: indices, packing, residual (this half's two 32-column chunks) ----
@@ -406,7 +411,11 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
       }
       mma_commit(bar_q);
     }
-    if (grp_any(gi, !mbar_wait(bar_q, iter & 1))) { fault = true; break; }
+    if (grp_any(gi, !mbar_wait(bar_q, iter & 1, a.wait_limit))) {
+      mbar_wait(bar_q, iter & 1);   // drain, as above
+      fault = true;
+      break;
+    }
     tc_after_sync();
     // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho.
     const float thr = 0.125f * rho * snorm_max;
@@ -487,7 +496,9 @@ cudaError_t configure_quant_tc() {
   return configure_bits<4>();
 }
 
-cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s) {
+cudaError_t launch_quant_tc(const QuantTcArgs& a_in, int sms, cudaStream_t s) {
+  QuantTcArgs a = a_in;
+  if (a.wait_limit <= 0) a.wait_limit = TC_WAIT_LIMIT;
   const int64_t tiles = (a.n + TILE - 1) / TILE;
   int64_t grid = (tiles + 1) / 2;
   if (grid > sms) grid = sms;

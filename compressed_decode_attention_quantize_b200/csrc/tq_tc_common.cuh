@@ -44,9 +44,24 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                : "memory");
 }
 
-// Wait for the phase with the given parity; false after TC_WAIT_LIMIT polls.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (int it = 0; it < TC_WAIT_LIMIT; ++it) {
+// Wait for the phase with the given parity; false after `limit` polls
+// (TC_WAIT_LIMIT unless a test shortens the kernels' main waits; drains keep
+// the full limit).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int limit = TC_WAIT_LIMIT) {
+  if (limit < TC_WAIT_LIMIT) {   // shortened: non-blocking polls, so that the count is the limit
+    for (int it = 0; it < limit; ++it) {
+      uint32_t ok;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+      if (ok) return true;
+    }
+    return false;
+  }
+  for (int it = 0; it < limit; ++it) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"

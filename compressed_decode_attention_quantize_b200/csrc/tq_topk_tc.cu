@@ -64,6 +64,7 @@ struct TopkTcArgs {
   int* cand_i;
   const float* bar_v;   // optional starting bar: entry (q, K - 1) of [nq][K]
   const int* bar_i;
+  int wait_limit;       // polls of the main waits (drains keep the full limit)
 };
 
 __device__ __forceinline__ bool better_tc(float va, int ia, float vb, int ib) {
@@ -166,7 +167,8 @@ __global__ void __maxnreg__(96)
         const int64_t n1 = min(a.n, n0 + a.chunk);
         const int ntile = (int)((n1 - n0 + TC_ROWS - 1) / TC_ROWS);
         // The previous item's MMAs read the query blocks: let them finish.
-        if (tiles_before > 0 && !mbar_wait(bar_accf + 8 * ((tiles_before - 1) & 1), ((tiles_before - 1) >> 1) & 1)) {
+        if (tiles_before > 0 &&
+            !mbar_wait(bar_accf + 8 * ((tiles_before - 1) & 1), ((tiles_before - 1) >> 1) & 1, a.wait_limit)) {
           fault = true;
           break;
         }
@@ -178,7 +180,7 @@ __global__ void __maxnreg__(96)
           const int y = (int)(n0 + (int64_t)t * TC_ROWS);
           for (int kb = 0; kb < a.nkb; ++kb) {
             // The stage's previous K block has been consumed by its MMAs.
-            if (loaded >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, up ^ 1)) {
+            if (loaded >= (uint32_t)S && !mbar_wait(bar_empty + 8 * s, up ^ 1, a.wait_limit)) {
               fault = true;
               break;
             }
@@ -211,20 +213,20 @@ __global__ void __maxnreg__(96)
         const int64_t n0 = (item / a.qblocks) * a.chunk;
         const int64_t n1 = min(a.n, n0 + a.chunk);
         const int ntile = (int)((n1 - n0 + TC_ROWS - 1) / TC_ROWS);
-        if (!mbar_wait(bar_b, icount & 1)) {
+        if (!mbar_wait(bar_b, icount & 1, a.wait_limit)) {
           fault = true;
           break;
         }
         for (int t = 0; t < ntile && !fault; ++t) {
           const uint32_t ab = tcount & 1;
-          if (!mbar_wait(bar_acce + 8 * ab, ((tcount >> 1) & 1) ^ 1)) {
+          if (!mbar_wait(bar_acce + 8 * ab, ((tcount >> 1) & 1) ^ 1, a.wait_limit)) {
             fault = true;
             break;
           }
           tc_after_sync();
           const uint32_t d_lm = tmem + ab * 256, d_q = d_lm + 128;
           for (int kb = 0; kb < a.nkb; ++kb) {
-            if (!mbar_wait(bar_full + 8 * s, up)) {
+            if (!mbar_wait(bar_full + 8 * s, up, a.wait_limit)) {
               fault = true;
               break;
             }
@@ -308,7 +310,7 @@ __global__ void __maxnreg__(96)
         const float nv = nv_next, gv = gv_next;
         norms(t + 1, nv_next, gv_next);
         const uint32_t ab = tcount & 1;
-        if (!mbar_wait(bar_accf + 8 * ab, (tcount >> 1) & 1)) {
+        if (!mbar_wait(bar_accf + 8 * ab, (tcount >> 1) & 1, a.wait_limit)) {
           fault = true;
           break;
         }
@@ -510,6 +512,7 @@ cudaError_t launch_topk_tc(const tq_ctx* c, const TopkPlan& p, const void* qh, c
   a.cand_i = cand_i;
   a.bar_v = bar_v;
   a.bar_i = bar_i;
+  a.wait_limit = c->wait_limit > 0 ? c->wait_limit : TC_WAIT_LIMIT;
   const int64_t items = p.qblocks * p.chunks;
   const unsigned grid = (unsigned)(items < c->sms ? items : c->sms);   // one CTA per SM
   k_topk_tc<<<grid, TC_THREADS, p.smem, s>>>(ma, mb, a);

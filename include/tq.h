@@ -113,6 +113,19 @@ const char* tq_version(void);
 int tq_device_fault(int* code);
 
 /*
+ * tq_set_wait_limit - diagnostic for testing the fault path: the tensor-core
+ * quantize and top-k kernels launched with context c after this call give up
+ * a bounded wait on an MMA or copy after `polls` polls instead of their full
+ * limit (polls = 0 restores the full limit).  A kernel that gives up first
+ * waits, with the full limit, for the MMAs and copies it has issued, then
+ * sets its tq_device_fault bit, releases its tensor memory and returns; its
+ * outputs are undefined.  Not for production use: a short limit makes
+ * ordinary launches fail.  Errors: TQ_ERR_ARG for a null context or
+ * polls < 0.  Host-only; no device work.
+ */
+int tq_set_wait_limit(tq_ctx* c, int polls);
+
+/*
  * tq_init - build the per-context tables on the host in fp64 and upload them
  * to the current CUDA device ([WHAT] stage 1 steps 1-2, stage 2).
  *   d       vector dimension.

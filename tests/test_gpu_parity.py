@@ -355,6 +355,43 @@ def test_topk_code_widths_and_k(cuda, d, bk, m, k):
     _check_topk(tab, Q.double().numpy(), g, idx.cpu().numpy(), score.cpu().numpy(), k)
 
 
+def test_bounded_wait_expiry_sets_fault_and_recovers(cuda):
+    """The tensor-core quantize and top-k kernels with their main bounded
+    waits cut to one non-blocking poll (tq_set_wait_limit): on an ordinary
+    launch the first wait gives up, the kernel waits with the full limit for
+    the MMAs and copies it issued, sets its tq_device_fault bit (1 quantize,
+    2 top-k) and returns; the next launch with the full limit is correct."""
+    c = _ctx(128, 3, 4, 128, seed=2)
+    tab = P.oracle_tables(c)
+    n = 8192   # above the small-batch bound: the tensor-core quantize
+    X = tq_inputs.outlier_kv(1, 1, n, 128, seed=12)[0, 0].to(torch.bfloat16)
+    xd = X.to(cuda)
+    assert tq.tq_device_fault() == 0
+    c.set_wait_limit(1)
+    c.quantize(xd, tq.TQ_KEY)
+    assert tq.tq_device_fault() == 1
+    c.set_wait_limit(0)
+    pk = c.quantize(xd, tq.TQ_KEY)
+    torch.cuda.synchronize()
+    assert tq.tq_device_fault() == 0
+    P.check_quantized(tab, "k", X.double().numpy(), _flat(pk, n))
+
+    ct = _ctx(96, 3, 3, 64, seed=23)
+    tabt = P.oracle_tables(ct)
+    nq, nd, k = 129, 129, 5   # a ragged query block and tile on the tcgen05 scorer
+    Xd = tq_inputs.mixture(nd, 96, seed=51)
+    Q = tq_inputs.mixture(nq, 96, seed=52, means_seed=51)
+    db = ct.quantize(Xd.to(cuda), tq.TQ_KEY)
+    ct.set_wait_limit(1)
+    ct.topk(Q.to(cuda), db, k)
+    assert tq.tq_device_fault() == 2
+    ct.set_wait_limit(0)
+    idx, score = ct.topk(Q.to(cuda), db, k)
+    torch.cuda.synchronize()
+    assert tq.tq_device_fault() == 0
+    _check_topk(tabt, Q.double().numpy(), _flat(db, nd), idx.cpu().numpy(), score.cpu().numpy(), k)
+
+
 @pytest.mark.parametrize("d,bk,m,nq,n,k", [
     (64, 2, 64, 1, 127, 12),      # one query, a database shorter than one 128-row tile
     (96, 3, 64, 129, 129, 5),     # ragged query block and tile, K padded to 16s
