@@ -238,7 +238,9 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
   // K-major, two 64-wide K blocks, 16-byte chunks swizzled with the row.
   if (cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) c->sms = 148;
   if (d == 128) {
-    std::vector<uint16_t> img(3 * 128 * 128, 0);
+    // images: 0 fp16 head, 1 fp16 tail, 2 S, then (after the row norms) the
+    // three bf16 terms of 2^8 Pi
+    std::vector<uint16_t> img(3 * 128 * 128, 0), imgb(3 * 128 * 128, 0);
     std::vector<float> snorm(128, 0.f);
     auto put = [&](int which, int r, int k, double v) {
       const int kb = k >> 6, kk = k & 63, ch = kk >> 3, w = kk & 7;
@@ -247,12 +249,33 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
       const __half h = __float2half_rn((float)v);
       img[(size_t)which * 16384 + off / 2] = *reinterpret_cast<const uint16_t*>(&h);
     };
+    auto bf16_rn = [](double v) {   // nearest bf16 (ties to even) of the fp32 rounding of v
+      const float f = (float)v;
+      uint32_t u;
+      std::memcpy(&u, &f, 4);
+      u += 0x7FFFu + ((u >> 16) & 1u);
+      const uint16_t h = (uint16_t)(u >> 16);
+      uint32_t back = (uint32_t)h << 16;
+      float g;
+      std::memcpy(&g, &back, 4);
+      return std::make_pair(h, (double)g);
+    };
     for (int j = 0; j < 128; ++j)
       for (int k = 0; k < 128; ++k) {
         const double v = 256.0 * c->Pi[(size_t)j * d + k];
         const double hi = tqh::round_to_half(v);
         put(0, j, k, hi);
         put(1, j, k, tqh::round_to_half(v - hi));
+        // bf16 terms: v = b0 + b1 + b2 to ~24 bits
+        double rem = v;
+        const int kb = k >> 6, kk = k & 63, ch = kk >> 3, w = kk & 7;
+        const size_t off = (size_t)kb * 16384 + (size_t)(j >> 3) * 1024 + (size_t)(j & 7) * 128 +
+                           (size_t)((ch ^ (j & 7)) << 4) + (size_t)w * 2;
+        for (int t = 0; t < 3; ++t) {
+          const auto b = bf16_rn(rem);
+          imgb[(size_t)t * 16384 + off / 2] = b.first;
+          rem -= b.second;
+        }
       }
     for (int i = 0; i < qjl_m; ++i) {
       double nn = 0.0;
@@ -263,12 +286,15 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
       snorm[i] = (float)std::sqrt(nn);
     }
     void* tc = nullptr;
-    e = cudaMalloc(&tc, img.size() * 2 + snorm.size() * 4);
+    const size_t boff = 98304 + 1024;   // bf16 images after the row norms, 1 KB aligned
+    e = cudaMalloc(&tc, boff + imgb.size() * 2);
     if (e == cudaSuccess) {
       e = cudaMemcpy(tc, img.data(), img.size() * 2, cudaMemcpyHostToDevice);
       if (e == cudaSuccess)
         e = cudaMemcpy(static_cast<char*>(tc) + img.size() * 2, snorm.data(), snorm.size() * 4,
                        cudaMemcpyHostToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy(static_cast<char*>(tc) + boff, imgb.data(), imgb.size() * 2, cudaMemcpyHostToDevice);
     }
     if (e != cudaSuccess) {
       cuda_fail(e, "tq_init: tensor-core tables");
@@ -282,6 +308,7 @@ tq_ctx* tq_init_ex(int d, int bits_k, int bits_v, int qjl_m, uint64_t seed, int 
     c->tc_pil = static_cast<char*>(tc) + 32768;
     c->tc_s = static_cast<char*>(tc) + 65536;
     c->tc_snorm = reinterpret_cast<const float*>(static_cast<char*>(tc) + 98304);
+    c->tc_pib = static_cast<char*>(tc) + boff;
     c->tc_ok = true;
   }
   const float* base = static_cast<const float*>(c->dev_block);
@@ -407,6 +434,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
     t.m = m;
     t.pi_hi = c->tc_pih;
     t.pi_lo = c->tc_pil;
+    t.pi_b = c->tc_pib;
     t.s_img = c->tc_s;
     t.snorm = c->tc_snorm;
     t.s_f32 = c->S_f;

@@ -46,6 +46,7 @@ struct tq_ctx {
   const void* tc_pil = nullptr;   // 2^8 Pi - head, fp16
   const void* tc_s = nullptr;     // S, fp16 (exact)
   const float* tc_snorm = nullptr;  // |S_i|
+  const void* tc_pib = nullptr;   // 2^8 Pi as three bf16 terms (head, middle, tail), 3 x 32 KB
   // Polls before a tensor-core kernel's main bounded wait gives up (0 = the
   // kernels' full limit); set only by tq_set_wait_limit, for testing the
   // fault path.
@@ -175,6 +176,7 @@ struct QuantTcArgs {
   int bits, m;
   const void* pi_hi;
   const void* pi_lo;
+  const void* pi_b;    // three bf16 terms of 2^8 Pi (bf16 inputs)
   const void* s_img;
   const float* snorm;
   const float* s_f32;

@@ -26,6 +26,7 @@
 // Waits on MMA completion are bounded; on timeout the group waits (with the
 // full limit) for the MMAs it issued, the kernel records a fault code,
 // releases its tensor memory and returns.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -462,6 +463,438 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised form (k_quant_ws): one CTA of ten warps per SM, persistent
+// over its tiles of 128 vectors.  Warp 0 lane 0 loads the raw input tiles
+// (bf16 or fp16, no register pass) with TMA into 128B-swizzled slots; warp 1
+// owns the tensor memory and its lane 0 issues every MMA; warps 2-5 and 6-9
+// are two epilogue groups taking alternate tiles, each with its own TMEM
+// accumulators (rotation 128 columns, QJL 128 columns), so that one tile's
+// rotation runs under the previous tile's epilogue.  The rotation multiplies
+// the input as it is stored: bf16 inputs against three bf16 terms of 2^8 Pi,
+// fp16 inputs against the fp16 head and tail, both to ~24 bits; the norm is
+// taken from the rotated vector (|Pi x| = |x|).  The epilogue writes the exact
+// residual 2^14 r back over its rotation columns while it computes the
+// indices, and only then (once the previous tile's QJL product has released
+// it) converts it into the one shared fp16 head/tail operand of the QJL
+// product; exact sign fix-ups read it from there.
+// Shared memory: Pi images 96 KB, S 32 KB, residual 64 KB, input slots
+// (one with QJL, four without), 1 KB of barriers and tables.
+// ---------------------------------------------------------------------------
+constexpr int WS_WARPS = 10;
+constexpr uint32_t WS_OFF_S = 3 * SMEM_TILE;
+constexpr uint32_t WS_OFF_R = 4 * SMEM_TILE;
+constexpr uint32_t WS_OFF_MISC = 7 * SMEM_TILE;
+constexpr uint32_t WS_SMEM = WS_OFF_MISC + 1024 + 1024;   // + 1 KB misc + alignment slack
+constexpr uint32_t IDESC_BF16 = tc_idesc_f16(128) | (1u << 7) | (1u << 10);   // A and B bf16
+// barrier slots (8 bytes each) at WS_OFF_MISC
+enum : uint32_t { B_XF = 0, B_XE = 4, B_RF = 8, B_TE = 10, B_QF = 12, B_RFULL = 14, B_REMPTY = 15, B_DONE = 16 };
+
+__device__ __forceinline__ void tma_load_x(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_x(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
+// A bounded wait that also gives up once another role has set *abort.
+__device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, int limit, volatile int* abort) {
+  for (int it = 0;; ++it) {
+    uint32_t ok;
+    if (limit < TC_WAIT_LIMIT)
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    else
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    if (ok) return true;
+    if (*abort != 0 || it + 1 >= limit) return false;
+  }
+}
+
+// 32 fp32 columns [col, col+32) of this thread's TMEM lane, written.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// Exact fp32 signs of the flagged QJL rows from the residual 2^14 r that the
+// epilogue left in its rotation columns (taddr), two rows per lane per pass;
+// warp-collective like qjl_fixup.
+__device__ __noinline__ Q4 qjl_fixup_r(uint32_t taddr, const float* s_f32, Q4 flag, Q4 qw) {
+  while (__any_sync(0xffffffffu, (flag.w[0] | flag.w[1] | flag.w[2] | flag.w[3]) != 0u)) {
+    int rows[2] = {-1, -1};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+      for (int fw = 0; fw < 4; ++fw) {
+        if (rows[q] < 0 && flag.w[fw] != 0u) {
+          const int bit = __ffs(flag.w[fw]) - 1;
+          flag.w[fw] &= flag.w[fw] - 1;
+          rows[q] = fw * 32 + bit;
+        }
+      }
+    }
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      float d[32];
+      tmem_ld32(taddr + ch * 32, d);
+      if (rows[0] >= 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          acc0 = fmaf(__ldg(s_f32 + (size_t)rows[0] * 128 + ch * 32 + i), d[i], acc0);
+          if (rows[1] >= 0) acc1 = fmaf(__ldg(s_f32 + (size_t)rows[1] * 128 + ch * 32 + i), d[i], acc1);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (rows[q] >= 0) {
+        const int fw = rows[q] >> 5, bit = rows[q] & 31;
+        const bool pos = (q == 0 ? acc0 : acc1) >= 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (w == fw) qw.w[w] = (qw.w[w] & ~(1u << bit)) | ((pos ? 1u : 0u) << bit);
+      }
+    }
+  }
+  return qw;
+}
+
+template <int BITS, bool QJL, bool BF>
+__global__ void __launch_bounds__(WS_WARPS * 32, 1)
+    k_quant_ws(const __grid_constant__ CUtensorMap tmx, QuantTcArgs a) {
+  constexpr int NPI = BF ? 3 : 2;
+  constexpr uint32_t XBASE = QJL ? 6 * SMEM_TILE : 3 * SMEM_TILE;
+  constexpr int NX = (int)((WS_OFF_MISC - XBASE) / SMEM_TILE);
+  constexpr int L = 1 << BITS;
+  constexpr int PER = (BITS == 3) ? 16 : 32 / BITS;
+  constexpr int W_MAIN = 128 / PER;
+  constexpr int WORDS = (BITS == 3) ? W_MAIN + 4 : W_MAIN;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  unsigned char* base = smem_raw + (base_s - raw_s);
+  const uint32_t bars = base_s + WS_OFF_MISC;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(base + WS_OFF_MISC + 256);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(base + WS_OFF_MISC + 260);
+  float* s_snorm = reinterpret_cast<float*>(base + WS_OFF_MISC + 320);   // [128]
+  float* s_cen = s_snorm + 128;                                           // [16]
+  float* s_pb = s_cen + 16;                                               // [8]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- tables: Pi images, S, QJL row norms, codebook ----------------------------------
+  {
+    const int4* src_pi = reinterpret_cast<const int4*>(BF ? a.pi_b : a.pi_hi);
+    const int4* src_pl = reinterpret_cast<const int4*>(a.pi_lo);
+    const int4* src_s = reinterpret_cast<const int4*>(a.s_img);
+    int4* dst = reinterpret_cast<int4*>(base);
+    constexpr int CH = (int)(SMEM_TILE / 16);
+    for (int e = tid; e < CH; e += WS_WARPS * 32) {
+      dst[e] = src_pi[e];
+      dst[CH + e] = BF ? src_pi[CH + e] : src_pl[e];
+      if (BF) dst[2 * CH + e] = src_pi[2 * CH + e];
+      if (QJL) dst[WS_OFF_S / 16 + e] = src_s[e];
+    }
+    if (tid < 128) s_snorm[tid] = QJL ? a.snorm[tid] : 0.f;
+    if (tid < 16) s_cen[tid] = tid < L ? a.cen[tid] * (QJL ? 16384.f : 1.f) : 0.f;
+    if (tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < NX; ++i) {
+      mbar_init(bars + 8 * (B_XF + i), 1);
+      mbar_init(bars + 8 * (B_XE + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + 8 * (B_RF + i), 1);
+      mbar_init(bars + 8 * (B_TE + i), 128);
+      mbar_init(bars + 8 * (B_QF + i), 1);
+    }
+    mbar_init(bars + 8 * B_RFULL, 128);
+    mbar_init(bars + 8 * B_REMPTY, 1);
+    mbar_init(bars + 8 * B_DONE, 1);
+    *s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(s_tmem))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  fence_async_smem();
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tmem = *s_tmem;
+  const int64_t ntiles = (a.n + TILE - 1) / TILE;
+  const int nk = blockIdx.x < ntiles ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  const int lim = a.wait_limit;
+  bool fault = false;
+
+  if (warp == 0) {
+    // ---- producer: TMA of the input tiles ------------------------------------------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int k = 0; k < nk && !*s_abort; ++k) {
+        const int slot = k % NX;
+        if (k >= NX && !ws_wait(bars + 8 * (B_XE + slot), ((k / NX) - 1) & 1, lim, s_abort)) {
+          fault = true;
+          break;
+        }
+        const int y = (int)((blockIdx.x + (int64_t)k * gridDim.x) * TILE);
+        const uint32_t xf = bars + 8 * (B_XF + slot);
+        mbar_expect_tx(xf, SMEM_TILE);
+        tma_load_x(base_s + XBASE + slot * SMEM_TILE, &tmx, 0, y, xf);
+        tma_load_x(base_s + XBASE + slot * SMEM_TILE + 16384, &tmx, 64, y, xf);
+        ++issued;
+        if (k + NX < nk) {   // the tile that reuses this slot: into L2 now
+          const int y2 = (int)((blockIdx.x + (int64_t)(k + NX) * gridDim.x) * TILE);
+          tma_prefetch_x(&tmx, 0, y2);
+          tma_prefetch_x(&tmx, 64, y2);
+        }
+      }
+      // drain: the last load of each slot (consumed or not)
+      for (int k = issued - 1; k >= 0 && k >= issued - NX; --k)
+        mbar_wait(bars + 8 * (B_XF + k % NX), (k / NX) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issue --------------------------------------------------------------------------
+    if (lane == 0) {
+      auto qjl_mma = [&](int j) -> bool {
+        if (!ws_wait(bars + 8 * B_RFULL, j & 1, lim, s_abort)) return false;
+        tc_after_sync();
+        const uint32_t d_q = tmem + (uint32_t)((j & 1) * 256 + 128);
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+          const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
+          tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + koff), smem_desc(base_s + WS_OFF_S + koff), IDESC,
+                     st > 0 ? 1u : 0u);
+          tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + SMEM_TILE + koff), smem_desc(base_s + WS_OFF_S + koff),
+                     IDESC, 1u);
+        }
+        tc_commit(bars + 8 * (B_QF + (j & 1)));
+        tc_commit(bars + 8 * B_REMPTY);
+        return true;
+      };
+      int k = 0;
+      for (; k < nk && !*s_abort; ++k) {
+        const int e = k & 1, slot = k % NX;
+        if (k >= 2 && !ws_wait(bars + 8 * (B_TE + e), ((k >> 1) - 1) & 1, lim, s_abort)) {
+          fault = true;
+          break;
+        }
+        if (!ws_wait(bars + 8 * (B_XF + slot), (k / NX) & 1, lim, s_abort)) {
+          fault = true;
+          break;
+        }
+        tc_after_sync();
+        const uint32_t d_rot = tmem + (uint32_t)(e * 256);
+        const uint32_t xs = base_s + XBASE + slot * SMEM_TILE;
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+          const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
+#pragma unroll
+          for (int t = 0; t < NPI; ++t)
+            tc_mma_f16(d_rot, smem_desc(xs + koff), smem_desc(base_s + t * SMEM_TILE + koff),
+                       BF ? IDESC_BF16 : IDESC, (st | t) ? 1u : 0u);
+        }
+        tc_commit(bars + 8 * (B_RF + e));
+        tc_commit(bars + 8 * (B_XE + slot));
+        if (QJL && k >= 1 && !qjl_mma(k - 1)) {
+          fault = true;
+          break;
+        }
+      }
+      if (QJL && !fault && !*s_abort && nk >= 1 && !qjl_mma(nk - 1)) fault = true;
+      // drain: every MMA issued
+      tc_commit(bars + 8 * B_DONE);
+      mbar_wait(bars + 8 * B_DONE, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue groups: warps 2-5 and 6-9 take alternate tiles ------------------------
+    const int g = (warp - 2) >> 2, quad = warp & 3;
+    const int row = 32 * quad + lane;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const float* pb = s_pb;
+    const float pmid = BITS >= 2 ? s_pb[(L >> 2) - 1] : 0.f;
+    float snorm_max = 0.f;
+    if (QJL)
+      for (int i = 0; i < 128; ++i) snorm_max = fmaxf(snorm_max, s_snorm[i]);
+    unsigned char* R = base + WS_OFF_R;
+    for (int k = g; k < nk; k += 2) {
+      const int e = g;
+      const int64_t v = (blockIdx.x + (int64_t)k * gridDim.x) * TILE + row;
+      const bool live = v < a.n;
+      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_RF + e), (k >> 1) & 1, lim, s_abort))) {
+        fault = true;
+        *s_abort = 1;
+        break;
+      }
+      tc_after_sync();
+      const uint32_t d_rot = tmem + (uint32_t)(e * 256) + lane_base;
+      float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float d[32];
+        tmem_ld32(d_rot + ch * 32, d);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss[i & 3] = fmaf(d[i], d[i], ss[i & 3]);
+      }
+      const float nrm_r = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));   // 2^8 |Pi x|
+      const float inv = nrm_r > 0.f ? 1.f / nrm_r : 0.f;
+      const float nrm = nrm_r * (1.f / 256.f);
+      const int64_t rec0 = live ? out_rec(a, v) : -1;
+      const bool writes = rec0 >= 0;
+      const int64_t rec = writes ? rec0 : 0;
+      uint32_t* crow = a.codes + rec * WORDS;
+      float rho2v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float d[32];
+        tmem_ld32(d_rot + ch * 32, d);
+        uint32_t cw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float y = d[i] * inv;
+          const int idx = lm_idx<BITS>(y, pmid, pb);
+          if (BITS == 3) {
+            cw[i >> 4] |= (uint32_t)(idx & 3) << (2 * (i & 15));
+            cw[2] |= (uint32_t)(idx >> 2) << i;
+          } else {
+            cw[i / PER] |= (uint32_t)idx << (BITS * (i % PER));
+          }
+          if (QJL) {
+            const float r = fmaf(y, 16384.f, -s_cen[idx]);   // s_cen holds 2^14 c
+            rho2v[i & 3] = fmaf(r, r, rho2v[i & 3]);
+            d[i] = r;
+          }
+        }
+        if (writes) {
+          if (BITS == 4) *reinterpret_cast<uint4*>(crow + 4 * ch) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          if (BITS == 2) *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
+          if (BITS == 1) crow[ch] = cw[0];
+          if (BITS == 3) {
+            *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
+            crow[W_MAIN + ch] = cw[2];
+          }
+        }
+        if (QJL) tmem_st32(d_rot + ch * 32, d);   // the exact residual replaces the chunk
+      }
+      if (writes) a.norm[rec] = nrm;
+      if (!QJL) {
+        tc_before_sync();
+        mbar_arrive(bars + 8 * (B_TE + e));
+        continue;
+      }
+      // The shared residual operand is free once the previous tile's QJL product is done.
+      if (k >= 1 && __any_sync(0xffffffffu, !ws_wait(bars + 8 * B_REMPTY, (k - 1) & 1, lim, s_abort))) {
+        fault = true;
+        *s_abort = 1;
+        break;
+      }
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float d[32];
+        tmem_ld32(d_rot + ch * 32, d);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float r0 = d[8 * q + 2 * u], r1 = d[8 * q + 2 * u + 1];
+            const __half2 hh = __floats2half2_rn(r0, r1);
+            const float2 f = __half22float2(hh);
+            hv[u] = *reinterpret_cast<const uint32_t*>(&hh);
+            lv[u] = h2bits(r0 - f.x, r1 - f.y);
+          }
+          *reinterpret_cast<uint4*>(R + chunk_off(row, ch * 4 + q)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(R + SMEM_TILE + chunk_off(row, ch * 4 + q)) =
+              make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(bars + 8 * B_RFULL);
+      const float rho = sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) * (1.f / 16384.f);
+      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_QF + e), (k >> 1) & 1, lim, s_abort))) {
+        fault = true;
+        *s_abort = 1;
+        break;
+      }
+      tc_after_sync();
+      const uint32_t d_q = tmem + (uint32_t)(e * 256 + 128) + lane_base;
+      // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho (exact recomputation below).
+      const float thr = 0.125f * rho * snorm_max;
+      uint32_t qw[4], flag[4];
+#pragma unroll 1
+      for (int c2 = 0; c2 < 4; ++c2) {
+        float d[32];
+        tmem_ld32(d_q + c2 * 32, d);
+        uint32_t sg = 0u, fl = 0u;
+#pragma unroll
+        for (int i = 31; i >= 0; --i) {
+          sg = __funnelshift_l(__float_as_uint(d[i]), sg, 1);
+          fl = __funnelshift_l(__float_as_uint(thr - fabsf(d[i])), fl, 1);
+        }
+        qw[c2] = ~sg;
+        flag[c2] = ~fl;
+      }
+      if (!writes) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
+      if (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
+        const Q4 fixed = qjl_fixup_r(d_rot, a.s_f32, Q4{{flag[0], flag[1], flag[2], flag[3]}},
+                                     Q4{{qw[0], qw[1], qw[2], qw[3]}});
+#pragma unroll
+        for (int w = 0; w < 4; ++w) qw[w] = fixed.w[w];
+      }
+      if (writes) {
+        *reinterpret_cast<uint4*>(a.qjl + rec * 4) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+        a.rnorm[rec] = nrm * rho;
+      }
+      tc_before_sync();
+      mbar_arrive(bars + 8 * (B_TE + e));
+    }
+  }
+  if (fault) {
+    *s_abort = 1;
+    atomicExch(&g_tq_fault, 1);
+  }
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem) : "memory");
+  }
+}
+
 template <int BITS>
 cudaError_t launch_bits(const QuantTcArgs& a, bool qjl, int grid, cudaStream_t s) {
   if (qjl) {
@@ -474,9 +907,56 @@ cudaError_t launch_bits(const QuantTcArgs& a, bool qjl, int grid, cudaStream_t s
 
 template <int BITS>
 cudaError_t configure_bits() {
-  cudaError_t e = cudaFuncSetAttribute(k_quant_tc<BITS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
+  const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(k_quant_tc<BITS, true>, ms, (int)TC_SMEM);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_quant_tc<BITS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM);
+  if ((e = cudaFuncSetAttribute(k_quant_tc<BITS, false>, ms, (int)TC_SMEM))) return e;
+  if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, true, true>, ms, (int)WS_SMEM))) return e;
+  if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, true, false>, ms, (int)WS_SMEM))) return e;
+  if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, false, true>, ms, (int)WS_SMEM))) return e;
+  return cudaFuncSetAttribute(k_quant_ws<BITS, false, false>, ms, (int)WS_SMEM);
+}
+
+template <int BITS>
+cudaError_t launch_ws(const CUtensorMap& map, const QuantTcArgs& a, bool qjl, bool bf, int grid, cudaStream_t s) {
+  const dim3 b(WS_WARPS * 32);
+  if (qjl && bf) k_quant_ws<BITS, true, true><<<grid, b, WS_SMEM, s>>>(map, a);
+  if (qjl && !bf) k_quant_ws<BITS, true, false><<<grid, b, WS_SMEM, s>>>(map, a);
+  if (!qjl && bf) k_quant_ws<BITS, false, true><<<grid, b, WS_SMEM, s>>>(map, a);
+  if (!qjl && !bf) k_quant_ws<BITS, false, false><<<grid, b, WS_SMEM, s>>>(map, a);
+  return cudaGetLastError();
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Input rows [n][ld] (16-bit), the first 128 of each row: boxes of 64 x 128,
+// 128-byte swizzle (the K-major operand layout of chunk_off); rows past n read
+// as zeros.
+bool make_x_map(CUtensorMap* map, const QuantTcArgs& a) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)a.n};
+  const cuuint64_t strides[1] = {(cuuint64_t)a.ld * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t es[2] = {1, 1};
+  const CUtensorMapDataType t = a.dtype == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(map, t, 2, const_cast<void*>(a.x), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -500,6 +980,19 @@ cudaError_t launch_quant_tc(const QuantTcArgs& a_in, int sms, cudaStream_t s) {
   QuantTcArgs a = a_in;
   if (a.wait_limit <= 0) a.wait_limit = TC_WAIT_LIMIT;
   const int64_t tiles = (a.n + TILE - 1) / TILE;
+  CUtensorMap map;
+  if (a.pi_b && (a.dtype == TQ_BF16 || a.dtype == TQ_F16) && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
+      (a.ld * 2) % 16 == 0 && a.n < ((int64_t)1 << 31) - TILE && make_x_map(&map, a)) {
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    const bool qjl = a.m > 0, bf = a.dtype == TQ_BF16;
+    switch (a.bits) {
+      case 1: return launch_ws<1>(map, a, qjl, bf, grid, s);
+      case 2: return launch_ws<2>(map, a, qjl, bf, grid, s);
+      case 3: return launch_ws<3>(map, a, qjl, bf, grid, s);
+      case 4: return launch_ws<4>(map, a, qjl, bf, grid, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   int64_t grid = (tiles + 1) / 2;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
