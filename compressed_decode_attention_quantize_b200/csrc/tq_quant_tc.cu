@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
 // Shared memory: Pi images 96 KB, S 32 KB, residual 64 KB, input slots
 // (one with QJL, four without), 1 KB of barriers and tables.
 // ---------------------------------------------------------------------------
-constexpr int WS_WARPS = 10;
+constexpr int WS_WARPS = 11;   // + warp 10: the QJL product's issuing thread
 constexpr uint32_t WS_OFF_S = 3 * SMEM_TILE;
 constexpr uint32_t WS_OFF_R = 4 * SMEM_TILE;
 constexpr uint32_t WS_OFF_MISC = 7 * SMEM_TILE;
@@ -489,6 +489,7 @@ constexpr uint32_t WS_SMEM = WS_OFF_MISC + 1024 + 1024;   // + 1 KB misc + align
 constexpr uint32_t IDESC_BF16 = tc_idesc_f16(128) | (1u << 7) | (1u << 10);   // A and B bf16
 // barrier slots (8 bytes each) at WS_OFF_MISC
 enum : uint32_t { B_XF = 0, B_XE = 4, B_RF = 8, B_TE = 10, B_QF = 12, B_RFULL = 14, B_REMPTY = 15, B_DONE = 16 };
+// (B_DONE + 1: the QJL thread's drain)
 
 __device__ __forceinline__ void tma_load_x(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -640,6 +641,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
     mbar_init(bars + 8 * B_RFULL, 128);
     mbar_init(bars + 8 * B_REMPTY, 1);
     mbar_init(bars + 8 * B_DONE, 1);
+    mbar_init(bars + 8 * (B_DONE + 1), 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -659,6 +661,22 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
   const int lim = a.wait_limit;
   bool fault = false;
 
+    auto qjl_mma = [&](int j) -> bool {
+      if (!ws_wait(bars + 8 * B_RFULL, j & 1, lim, s_abort)) return false;
+      tc_after_sync();
+      const uint32_t d_q = tmem + (uint32_t)((j & 1) * 256 + 128);
+#pragma unroll
+      for (int st = 0; st < 8; ++st) {
+        const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
+        tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + koff), smem_desc(base_s + WS_OFF_S + koff), IDESC,
+                   st > 0 ? 1u : 0u);
+        tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + SMEM_TILE + koff), smem_desc(base_s + WS_OFF_S + koff),
+                   IDESC, 1u);
+      }
+      tc_commit(bars + 8 * (B_QF + (j & 1)));
+      tc_commit(bars + 8 * B_REMPTY);
+      return true;
+    };
   if (warp == 0) {
     // ---- producer: TMA of the input tiles ------------------------------------------------
     if (lane == 0) {
@@ -689,22 +707,6 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
   } else if (warp == 1) {
     // ---- MMA issue --------------------------------------------------------------------------
     if (lane == 0) {
-      auto qjl_mma = [&](int j) -> bool {
-        if (!ws_wait(bars + 8 * B_RFULL, j & 1, lim, s_abort)) return false;
-        tc_after_sync();
-        const uint32_t d_q = tmem + (uint32_t)((j & 1) * 256 + 128);
-#pragma unroll
-        for (int st = 0; st < 8; ++st) {
-          const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
-          tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + koff), smem_desc(base_s + WS_OFF_S + koff), IDESC,
-                     st > 0 ? 1u : 0u);
-          tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + SMEM_TILE + koff), smem_desc(base_s + WS_OFF_S + koff),
-                     IDESC, 1u);
-        }
-        tc_commit(bars + 8 * (B_QF + (j & 1)));
-        tc_commit(bars + 8 * B_REMPTY);
-        return true;
-      };
       int k = 0;
       for (; k < nk && !*s_abort; ++k) {
         const int e = k & 1, slot = k % NX;
@@ -729,15 +731,23 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
         }
         tc_commit(bars + 8 * (B_RF + e));
         tc_commit(bars + 8 * (B_XE + slot));
-        if (QJL && k >= 1 && !qjl_mma(k - 1)) {
+      }
+      // drain: every MMA issued
+      tc_commit(bars + 8 * B_DONE);
+      mbar_wait(bars + 8 * B_DONE, 0);
+    }
+    __syncwarp();
+  } else if (warp == WS_WARPS - 1) {
+    // ---- QJL product issue (its own thread, so rotations never queue behind it) --------
+    if (QJL && lane == 0) {
+      for (int j = 0; j < nk && !*s_abort; ++j) {
+        if (!qjl_mma(j)) {
           fault = true;
           break;
         }
       }
-      if (QJL && !fault && !*s_abort && nk >= 1 && !qjl_mma(nk - 1)) fault = true;
-      // drain: every MMA issued
-      tc_commit(bars + 8 * B_DONE);
-      mbar_wait(bars + 8 * B_DONE, 0);
+      tc_commit(bars + 8 * (B_DONE + 1));
+      mbar_wait(bars + 8 * (B_DONE + 1), 0);
     }
     __syncwarp();
   } else {
