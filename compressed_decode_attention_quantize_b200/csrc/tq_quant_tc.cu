@@ -464,32 +464,38 @@ __global__ void __launch_bounds__(512, 1) k_quant_tc(QuantTcArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp-specialised form (k_quant_ws): one CTA of ten warps per SM, persistent
-// over its tiles of 128 vectors.  Warp 0 lane 0 loads the raw input tiles
-// (bf16 or fp16, no register pass) with TMA into 128B-swizzled slots; warp 1
-// owns the tensor memory and its lane 0 issues every MMA; warps 2-5 and 6-9
-// are two epilogue groups taking alternate tiles, each with its own TMEM
-// accumulators (rotation 128 columns, QJL 128 columns), so that one tile's
-// rotation runs under the previous tile's epilogue.  The rotation multiplies
-// the input as it is stored: bf16 inputs against three bf16 terms of 2^8 Pi,
-// fp16 inputs against the fp16 head and tail, both to ~24 bits; the norm is
-// taken from the rotated vector (|Pi x| = |x|).  The epilogue writes the exact
-// residual 2^14 r back over its rotation columns while it computes the
-// indices, and only then (once the previous tile's QJL product has released
-// it) converts it into the one shared fp16 head/tail operand of the QJL
-// product; exact sign fix-ups read it from there.
-// Shared memory: Pi images 96 KB, S 32 KB, residual 64 KB, input slots
-// (one with QJL, four without), 1 KB of barriers and tables.
+// Warp-specialised form (k_quant_ws): one CTA per SM, persistent over its
+// tiles of 128 vectors.  Warp 0 lane 0 loads the raw input tiles (bf16 or
+// fp16, no register pass) with TMA into 128B-swizzled slots; warp 1 owns the
+// tensor memory and its lane 0 issues the rotations; warp 2 lane 0 issues the
+// QJL products; NB epilogue groups of four warps (one thread per vector =
+// TMEM lane) take the tiles in turn, tile k in group and rotation buffer
+// k % NB (128 TMEM columns each), so NB tiles are in flight.  With QJL, NB =
+// 3 and the remaining 128 columns hold the one QJL accumulator, which the
+// groups use in tile order; without QJL, NB = 4.
+// The rotation multiplies the input as it is stored: bf16 inputs against
+// three bf16 terms of 2^8 Pi, fp16 inputs against the fp16 head and tail,
+// both to ~24 bits; the norm is taken from the rotated vector (|Pi x| = |x|).
+// The epilogue leaves the residual 2^14 r in its rotation columns as fp16
+// head and tail, the A operand (from tensor memory) of the QJL product;
+// near-zero QJL signs are recomputed in fp32 from head + tail (~22 bits: a
+// sign it could still miss lies within 2^-22 |S_i| |r| of zero, inside the
+// 1e-5 |r| band of the comparison rule).
+// Shared memory: Pi images 96 KB, S 32 KB (with QJL), input slots (three
+// with QJL, four without), 1 KB of barriers and tables.
 // ---------------------------------------------------------------------------
-constexpr int WS_WARPS = 11;   // + warp 10: the QJL product's issuing thread
 constexpr uint32_t WS_OFF_S = 3 * SMEM_TILE;
-constexpr uint32_t WS_OFF_R = 4 * SMEM_TILE;
 constexpr uint32_t WS_OFF_MISC = 7 * SMEM_TILE;
 constexpr uint32_t WS_SMEM = WS_OFF_MISC + 1024 + 1024;   // + 1 KB misc + alignment slack
 constexpr uint32_t IDESC_BF16 = tc_idesc_f16(128) | (1u << 7) | (1u << 10);   // A and B bf16
-// barrier slots (8 bytes each) at WS_OFF_MISC
-enum : uint32_t { B_XF = 0, B_XE = 4, B_RF = 8, B_TE = 10, B_QF = 12, B_RFULL = 14, B_REMPTY = 15, B_DONE = 16 };
-// (B_DONE + 1: the QJL thread's drain)
+__host__ __device__ constexpr int ws_groups(bool qjl) { return qjl ? 3 : 4; }
+__host__ __device__ constexpr int ws_warps(bool qjl) { return 3 + 4 * ws_groups(qjl); }
+// barrier slots (8 bytes each) at WS_OFF_MISC: x full / empty [4], rotation
+// full / buffer empty / residual ready / QJL done [4 buffers], QJL accumulator
+// empty, two drains.  A barrier that several groups wait on at different
+// phases would alias its phase parity, so every per-tile signal a group waits
+// for has one barrier per buffer (each group waits on its own, in order).
+enum : uint32_t { B_XF = 0, B_XE = 4, B_RF = 8, B_TE = 12, B_RR = 16, B_QF = 20, B_QE = 24, B_DONE = 25 };
 
 __device__ __forceinline__ void tma_load_x(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -545,9 +551,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
-// Exact fp32 signs of the flagged QJL rows from the residual 2^14 r that the
-// epilogue left in its rotation columns (taddr), two rows per lane per pass;
-// warp-collective like qjl_fixup.
+// tcgen05.mma kind::f16 with the A operand in tensor memory (lane = row m;
+// a K-step of 16 halves in 8 consecutive columns, two per column, the lower
+// K index in the low half).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(accumulate), "r"(idesc));
+}
+
+// fp32 signs of the flagged QJL rows from the residual 2^14 r that the
+// epilogue left in its rotation columns (taddr) as fp16 head and tail:
+// chunk c (coordinates 32 c ..) in columns 32 c .. 32 c + 15 (heads, two per
+// column) and 32 c + 16 .. (tails); r = head + tail carries ~22 bits.  Two
+// rows per lane per pass; warp-collective like qjl_fixup.
 __device__ __noinline__ Q4 qjl_fixup_r(uint32_t taddr, const float* s_f32, Q4 flag, Q4 qw) {
   while (__any_sync(0xffffffffu, (flag.w[0] | flag.w[1] | flag.w[2] | flag.w[3]) != 0u)) {
     int rows[2] = {-1, -1};
@@ -569,9 +588,18 @@ __device__ __noinline__ Q4 qjl_fixup_r(uint32_t taddr, const float* s_f32, Q4 fl
       tmem_ld32(taddr + ch * 32, d);
       if (rows[0] >= 0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc0 = fmaf(__ldg(s_f32 + (size_t)rows[0] * 128 + ch * 32 + i), d[i], acc0);
-          if (rows[1] >= 0) acc1 = fmaf(__ldg(s_f32 + (size_t)rows[1] * 128 + ch * 32 + i), d[i], acc1);
+        for (int u = 0; u < 16; ++u) {
+          const float2 hh = __half22float2(*reinterpret_cast<const __half2*>(&d[u]));
+          const float2 ll = __half22float2(*reinterpret_cast<const __half2*>(&d[16 + u]));
+          const float r0 = hh.x + ll.x, r1 = hh.y + ll.y;
+          const float* s0 = s_f32 + (size_t)rows[0] * 128 + ch * 32 + 2 * u;
+          acc0 = fmaf(__ldg(s0), r0, acc0);
+          acc0 = fmaf(__ldg(s0 + 1), r1, acc0);
+          if (rows[1] >= 0) {
+            const float* s1 = s_f32 + (size_t)rows[1] * 128 + ch * 32 + 2 * u;
+            acc1 = fmaf(__ldg(s1), r0, acc1);
+            acc1 = fmaf(__ldg(s1 + 1), r1, acc1);
+          }
         }
       }
     }
@@ -590,10 +618,11 @@ __device__ __noinline__ Q4 qjl_fixup_r(uint32_t taddr, const float* s_f32, Q4 fl
 }
 
 template <int BITS, bool QJL, bool BF>
-__global__ void __launch_bounds__(WS_WARPS * 32, 1)
+__global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
     k_quant_ws(const __grid_constant__ CUtensorMap tmx, QuantTcArgs a) {
+  constexpr int NB = ws_groups(QJL);
   constexpr int NPI = BF ? 3 : 2;
-  constexpr uint32_t XBASE = QJL ? 6 * SMEM_TILE : 3 * SMEM_TILE;
+  constexpr uint32_t XBASE = QJL ? 4 * SMEM_TILE : 3 * SMEM_TILE;
   constexpr int NX = (int)((WS_OFF_MISC - XBASE) / SMEM_TILE);
   constexpr int L = 1 << BITS;
   constexpr int PER = (BITS == 3) ? 16 : 32 / BITS;
@@ -610,6 +639,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
   float* s_cen = s_snorm + 128;                                           // [16]
   float* s_pb = s_cen + 16;                                               // [8]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NT = ws_warps(QJL) * 32;
 
   // ---- tables: Pi images, S, QJL row norms, codebook ----------------------------------
   {
@@ -618,7 +648,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
     const int4* src_s = reinterpret_cast<const int4*>(a.s_img);
     int4* dst = reinterpret_cast<int4*>(base);
     constexpr int CH = (int)(SMEM_TILE / 16);
-    for (int e = tid; e < CH; e += WS_WARPS * 32) {
+    for (int e = tid; e < CH; e += NT) {
       dst[e] = src_pi[e];
       dst[CH + e] = BF ? src_pi[CH + e] : src_pl[e];
       if (BF) dst[2 * CH + e] = src_pi[2 * CH + e];
@@ -629,17 +659,15 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
     if (tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
   }
   if (tid == 0) {
-    for (int i = 0; i < NX; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bars + 8 * (B_XF + i), 1);
       mbar_init(bars + 8 * (B_XE + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(bars + 8 * (B_RF + i), 1);
       mbar_init(bars + 8 * (B_TE + i), 128);
+      mbar_init(bars + 8 * (B_RR + i), 128);
       mbar_init(bars + 8 * (B_QF + i), 1);
     }
-    mbar_init(bars + 8 * B_RFULL, 128);
-    mbar_init(bars + 8 * B_REMPTY, 1);
+    mbar_init(bars + 8 * B_QE, 128);
     mbar_init(bars + 8 * B_DONE, 1);
     mbar_init(bars + 8 * (B_DONE + 1), 1);
     *s_abort = 0;
@@ -656,27 +684,12 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
   __syncthreads();
   tc_after_sync();
   const uint32_t tmem = *s_tmem;
+  const uint32_t d_qjl0 = tmem + 384;   // the QJL accumulator (with QJL)
   const int64_t ntiles = (a.n + TILE - 1) / TILE;
   const int nk = blockIdx.x < ntiles ? (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
   const int lim = a.wait_limit;
   bool fault = false;
 
-    auto qjl_mma = [&](int j) -> bool {
-      if (!ws_wait(bars + 8 * B_RFULL, j & 1, lim, s_abort)) return false;
-      tc_after_sync();
-      const uint32_t d_q = tmem + (uint32_t)((j & 1) * 256 + 128);
-#pragma unroll
-      for (int st = 0; st < 8; ++st) {
-        const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
-        tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + koff), smem_desc(base_s + WS_OFF_S + koff), IDESC,
-                   st > 0 ? 1u : 0u);
-        tc_mma_f16(d_q, smem_desc(base_s + WS_OFF_R + SMEM_TILE + koff), smem_desc(base_s + WS_OFF_S + koff),
-                   IDESC, 1u);
-      }
-      tc_commit(bars + 8 * (B_QF + (j & 1)));
-      tc_commit(bars + 8 * B_REMPTY);
-      return true;
-    };
   if (warp == 0) {
     // ---- producer: TMA of the input tiles ------------------------------------------------
     if (lane == 0) {
@@ -705,12 +718,11 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- MMA issue --------------------------------------------------------------------------
+    // ---- rotation MMAs into buffer k % NB ------------------------------------------------
     if (lane == 0) {
-      int k = 0;
-      for (; k < nk && !*s_abort; ++k) {
-        const int e = k & 1, slot = k % NX;
-        if (k >= 2 && !ws_wait(bars + 8 * (B_TE + e), ((k >> 1) - 1) & 1, lim, s_abort)) {
+      for (int k = 0; k < nk && !*s_abort; ++k) {
+        const int b = k % NB, slot = k % NX;
+        if (k >= NB && !ws_wait(bars + 8 * (B_TE + b), ((k / NB) - 1) & 1, lim, s_abort)) {
           fault = true;
           break;
         }
@@ -719,7 +731,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
           break;
         }
         tc_after_sync();
-        const uint32_t d_rot = tmem + (uint32_t)(e * 256);
+        const uint32_t d_rot = tmem + (uint32_t)(b * 128);
         const uint32_t xs = base_s + XBASE + slot * SMEM_TILE;
 #pragma unroll
         for (int st = 0; st < 8; ++st) {
@@ -729,30 +741,41 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
             tc_mma_f16(d_rot, smem_desc(xs + koff), smem_desc(base_s + t * SMEM_TILE + koff),
                        BF ? IDESC_BF16 : IDESC, (st | t) ? 1u : 0u);
         }
-        tc_commit(bars + 8 * (B_RF + e));
+        tc_commit(bars + 8 * (B_RF + b));
         tc_commit(bars + 8 * (B_XE + slot));
       }
-      // drain: every MMA issued
-      tc_commit(bars + 8 * B_DONE);
+      tc_commit(bars + 8 * B_DONE);   // drain: every MMA issued
       mbar_wait(bars + 8 * B_DONE, 0);
     }
     __syncwarp();
-  } else if (warp == WS_WARPS - 1) {
-    // ---- QJL product issue (its own thread, so rotations never queue behind it) --------
+  } else if (warp == 2) {
+    // ---- QJL MMAs, tile order, A = the residual in rotation buffer j % NB ----------------
     if (QJL && lane == 0) {
       for (int j = 0; j < nk && !*s_abort; ++j) {
-        if (!qjl_mma(j)) {
+        const int b = j % NB;
+        if (!ws_wait(bars + 8 * (B_RR + b), (j / NB) & 1, lim, s_abort) ||
+            (j >= 1 && !ws_wait(bars + 8 * B_QE, (j - 1) & 1, lim, s_abort))) {
           fault = true;
           break;
         }
+        tc_after_sync();
+        const uint32_t a_r = tmem + (uint32_t)(b * 128);
+#pragma unroll
+        for (int st = 0; st < 8; ++st) {
+          const uint32_t koff = (uint32_t)((st >> 2) * 16384 + (st & 3) * 32);
+          const uint32_t acol = (uint32_t)(32 * (st >> 1) + 8 * (st & 1));   // heads; tails 16 columns on
+          tc_mma_f16_ts(d_qjl0, a_r + acol, smem_desc(base_s + WS_OFF_S + koff), IDESC, st > 0 ? 1u : 0u);
+          tc_mma_f16_ts(d_qjl0, a_r + acol + 16, smem_desc(base_s + WS_OFF_S + koff), IDESC, 1u);
+        }
+        tc_commit(bars + 8 * (B_QF + b));
       }
-      tc_commit(bars + 8 * (B_DONE + 1));
+      tc_commit(bars + 8 * (B_DONE + 1));   // drain
       mbar_wait(bars + 8 * (B_DONE + 1), 0);
     }
     __syncwarp();
   } else {
-    // ---- epilogue groups: warps 2-5 and 6-9 take alternate tiles ------------------------
-    const int g = (warp - 2) >> 2, quad = warp & 3;
+    // ---- epilogue groups: warps 3 + 4g .. 3 + 4g + 3 take tiles g, g + NB, ... -----------
+    const int g = (warp - 3) >> 2, quad = warp & 3;
     const int row = 32 * quad + lane;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const float* pb = s_pb;
@@ -760,18 +783,17 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
     float snorm_max = 0.f;
     if (QJL)
       for (int i = 0; i < 128; ++i) snorm_max = fmaxf(snorm_max, s_snorm[i]);
-    unsigned char* R = base + WS_OFF_R;
-    for (int k = g; k < nk; k += 2) {
-      const int e = g;
+    for (int k = g; k < nk; k += NB) {
+      const int b = g;
       const int64_t v = (blockIdx.x + (int64_t)k * gridDim.x) * TILE + row;
       const bool live = v < a.n;
-      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_RF + e), (k >> 1) & 1, lim, s_abort))) {
+      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_RF + b), (k / NB) & 1, lim, s_abort))) {
         fault = true;
         *s_abort = 1;
         break;
       }
       tc_after_sync();
-      const uint32_t d_rot = tmem + (uint32_t)(e * 256) + lane_base;
+      const uint32_t d_rot = tmem + (uint32_t)(b * 128) + lane_base;
       float ss[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -818,51 +840,38 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
             crow[W_MAIN + ch] = cw[2];
           }
         }
-        if (QJL) tmem_st32(d_rot + ch * 32, d);   // the exact residual replaces the chunk
-      }
-      if (writes) a.norm[rec] = nrm;
-      if (!QJL) {
-        tc_before_sync();
-        mbar_arrive(bars + 8 * (B_TE + e));
-        continue;
-      }
-      // The shared residual operand is free once the previous tile's QJL product is done.
-      if (k >= 1 && __any_sync(0xffffffffu, !ws_wait(bars + 8 * B_REMPTY, (k - 1) & 1, lim, s_abort))) {
-        fault = true;
-        *s_abort = 1;
-        break;
-      }
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        float d[32];
-        tmem_ld32(d_rot + ch * 32, d);
+        if (QJL) {
+          // The residual as the QJL product's A operand, in place: the chunk's 32 fp32
+          // columns become 16 columns of fp16 heads and 16 of tails.
+          float o[32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t hv[4], lv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float r0 = d[8 * q + 2 * u], r1 = d[8 * q + 2 * u + 1];
+          for (int u = 0; u < 16; ++u) {
+            const float r0 = d[2 * u], r1 = d[2 * u + 1];
             const __half2 hh = __floats2half2_rn(r0, r1);
             const float2 f = __half22float2(hh);
-            hv[u] = *reinterpret_cast<const uint32_t*>(&hh);
-            lv[u] = h2bits(r0 - f.x, r1 - f.y);
+            o[u] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&hh));
+            o[16 + u] = __uint_as_float(h2bits(r0 - f.x, r1 - f.y));
           }
-          *reinterpret_cast<uint4*>(R + chunk_off(row, ch * 4 + q)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          *reinterpret_cast<uint4*>(R + SMEM_TILE + chunk_off(row, ch * 4 + q)) =
-              make_uint4(lv[0], lv[1], lv[2], lv[3]);
+          tmem_st32(d_rot + ch * 32, o);
         }
       }
-      fence_async_smem();
-      mbar_arrive(bars + 8 * B_RFULL);
+      if (writes) a.norm[rec] = nrm;
+      if constexpr (!QJL) {
+        tc_before_sync();
+        mbar_arrive(bars + 8 * (B_TE + b));
+        continue;
+      }
+      tc_before_sync();
+      mbar_arrive(bars + 8 * (B_RR + b));   // this lane's residual operand is in place
       const float rho = sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) * (1.f / 16384.f);
-      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_QF + e), (k >> 1) & 1, lim, s_abort))) {
+      if (__any_sync(0xffffffffu, !ws_wait(bars + 8 * (B_QF + b), (k / NB) & 1, lim, s_abort))) {
         fault = true;
         *s_abort = 1;
         break;
       }
       tc_after_sync();
-      const uint32_t d_q = tmem + (uint32_t)(e * 256 + 128) + lane_base;
-      // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho (exact recomputation below).
+      const uint32_t d_q = d_qjl0 + lane_base;
+      // D = 2^14 (S r); flag |D_i| <= 2^14 * 2^-17 max_i |S_i| rho (recomputation below).
       const float thr = 0.125f * rho * snorm_max;
       uint32_t qw[4], flag[4];
 #pragma unroll 1
@@ -878,6 +887,8 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
         qw[c2] = ~sg;
         flag[c2] = ~fl;
       }
+      tc_before_sync();
+      mbar_arrive(bars + 8 * B_QE);   // the QJL accumulator is read: the next tile's product may go
       if (!writes) flag[0] = flag[1] = flag[2] = flag[3] = 0u;
       if (__any_sync(0xffffffffu, (flag[0] | flag[1] | flag[2] | flag[3]) != 0u)) {
         const Q4 fixed = qjl_fixup_r(d_rot, a.s_f32, Q4{{flag[0], flag[1], flag[2], flag[3]}},
@@ -890,7 +901,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 1)
         a.rnorm[rec] = nrm * rho;
       }
       tc_before_sync();
-      mbar_arrive(bars + 8 * (B_TE + e));
+      mbar_arrive(bars + 8 * (B_TE + b));
     }
   }
   if (fault) {
@@ -929,11 +940,11 @@ cudaError_t configure_bits() {
 
 template <int BITS>
 cudaError_t launch_ws(const CUtensorMap& map, const QuantTcArgs& a, bool qjl, bool bf, int grid, cudaStream_t s) {
-  const dim3 b(WS_WARPS * 32);
-  if (qjl && bf) k_quant_ws<BITS, true, true><<<grid, b, WS_SMEM, s>>>(map, a);
-  if (qjl && !bf) k_quant_ws<BITS, true, false><<<grid, b, WS_SMEM, s>>>(map, a);
-  if (!qjl && bf) k_quant_ws<BITS, false, true><<<grid, b, WS_SMEM, s>>>(map, a);
-  if (!qjl && !bf) k_quant_ws<BITS, false, false><<<grid, b, WS_SMEM, s>>>(map, a);
+  const dim3 bq(ws_warps(true) * 32), bn(ws_warps(false) * 32);
+  if (qjl && bf) k_quant_ws<BITS, true, true><<<grid, bq, WS_SMEM, s>>>(map, a);
+  if (qjl && !bf) k_quant_ws<BITS, true, false><<<grid, bq, WS_SMEM, s>>>(map, a);
+  if (!qjl && bf) k_quant_ws<BITS, false, true><<<grid, bn, WS_SMEM, s>>>(map, a);
+  if (!qjl && !bf) k_quant_ws<BITS, false, false><<<grid, bn, WS_SMEM, s>>>(map, a);
   return cudaGetLastError();
 }
 
