@@ -291,8 +291,10 @@ __global__ void __launch_bounds__(MWI * 32, 1) k_attn_i8(AttnArgs a) {
       const float p0 = ex2f(sc0 - m_run), p1 = ex2f(sc1 - m_run);
       l_part += p0 + p1;
       // P tile (16 tokens x 8 columns): column 2t = head t, odd columns zero.
-      const uint32_t pb0 = movtrans(pack_half2(p0 * (st.vn[g] * vmul), 0.f));
-      const uint32_t pb1 = movtrans(pack_half2(p1 * (st.vn[g + 8] * vmul), 0.f));
+      // A 16-byte norm copy may reach past the row's end: those norms are not data.
+      const float vn0 = v0 ? st.vn[g] : 0.f, vn8 = v8 ? st.vn[g + 8] : 0.f;
+      const uint32_t pb0 = movtrans(pack_half2(p0 * (vn0 * vmul), 0.f));
+      const uint32_t pb1 = movtrans(pack_half2(p1 * (vn8 * vmul), 0.f));
 
       value_tile_w(o, st.v, pb0, pb1, lut_s, lane4, g, t);
       __syncwarp();

@@ -611,7 +611,8 @@ __global__ void __launch_bounds__(MW * 32, KeyFmt<KB>::CTAS) k_attn_lut(AttnArgs
         p[j][1] = hv ? ex2f(sc[j][1] - m_run[j]) : 0.f;
         l_part[j] += p[j][0] + p[j][1];
       }
-      const float w0s = snorm(st.vn, g) * vmul, w8s = snorm(st.vn, g + 8) * vmul;
+      // A 16-byte norm copy may reach past the row's end: those norms are not data.
+      const float w0s = v0 ? snorm(st.vn, g) * vmul : 0.f, w8s = v8 ? snorm(st.vn, g + 8) * vmul : 0.f;
       const uint32_t pb0 = movtrans(pack_half2(p[0][0] * w0s, p[1][0] * w0s));
       const uint32_t pb1 = movtrans(pack_half2(p[0][1] * w8s, p[1][1] * w8s));
       if constexpr (VB == 4)

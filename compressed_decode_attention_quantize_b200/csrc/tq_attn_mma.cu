@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(MW * 32, 3) k_attn_seg8(AttnArgs a) {
       const float p10 = ex2f(sc[1][0] - m_run[1]), p11 = ex2f(sc[1][1] - m_run[1]);
       l_part[0] += p00 + p01;
       l_part[1] += p10 + p11;
-      const float w0s = st.vn[g] * vmul, w8s = st.vn[g + 8] * vmul;
+      // A 16-byte norm copy may reach past the row's end: those norms are not data.
+      const float w0s = v0 ? st.vn[g] * vmul : 0.f, w8s = v8 ? st.vn[g + 8] * vmul : 0.f;
       const uint32_t pb0 = movtrans(pack_half2(p00 * w0s, p10 * w0s));
       const uint32_t pb1 = movtrans(pack_half2(p01 * w8s, p11 * w8s));
 

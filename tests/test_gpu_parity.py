@@ -1078,3 +1078,44 @@ def test_paged_rejections(cuda):
     with pytest.raises(tq.TQError) as e:
         c2.attn_decode_paged(q2, kp2, vp2, table, lens)
     assert e.value.status == tq.TQ_ERR_ARG
+
+
+@pytest.mark.parametrize("fmt,Hq,f16", [("k3v4", 8, False), ("k3v4", 16, False), ("k4v4", 8, False),
+                                        ("k3v4_nc", 8, False), ("4bit_nc", 4, True)])
+def test_decode_ignores_records_past_seq_len(cuda, fmt, Hq, f16):
+    """Records at or past seq_lens[b] are not data: filled with NaN norms and
+    all-ones codes they leave the output bit-identical to a clean cache.  The
+    lengths are not multiples of 4 (or 8), so 16-byte norm copies reach past
+    the end of each row.  Value norms spanning 2^-e .. 2^e inside a row
+    exercise the fp16 scale of the value product (e = 13, or 5 where the
+    norms are binary16, whose largest finite value is 65504)."""
+    c = tq.Context.variant(fmt, 128, seed=17, norm_f16=f16)
+    tab = P.oracle_tables(c)
+    B, Hkv, T, d = 4, 2, 1104, 128
+    K = tq_inputs.outlier_kv(B, Hkv, T, d, seed=91)
+    V = tq_inputs.outlier_kv(B, Hkv, T, d, seed=92)
+    e = 5 if f16 else 13
+    V[:, :, :40] *= 2.0 ** -e
+    V[:, :, 600:660] *= 2.0 ** e
+    V[:, :, 900:905] *= 2.0 ** 6
+    kc, vc = _cache(c, K, V, cuda)
+    lens = torch.tensor([1101, 0, 619, 3], dtype=torch.int32)
+    kp = {k: (None if v is None else v.clone()) for k, v in kc.items()}
+    vp = {k: (None if v is None else v.clone()) for k, v in vc.items()}
+    for cache in (kp, vp):
+        for k, v in cache.items():
+            if v is None:
+                continue
+            for b in range(B):
+                if v.is_floating_point():
+                    v[b, :, int(lens[b]):] = float("nan")
+                else:
+                    v[b, :, int(lens[b]):] = 0xFF
+    Q = tq_inputs.iid((B, Hq, d), seed=93, dtype=torch.bfloat16)
+    out = c.attn_decode(Q.to(cuda), kc, vc, lens.to(cuda))
+    outp = c.attn_decode(Q.to(cuda), kp, vp, lens.to(cuda))
+    torch.cuda.synchronize()
+    assert torch.isfinite(outp).all()
+    assert torch.equal(out, outp)
+    P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
+                      out.cpu().numpy())
