@@ -182,7 +182,7 @@ struct QuantTcArgs {
   const float* s_f32;
   uint32_t* codes;
   uint32_t* qjl;
-  float* norm;
+  float* norm;      // binary16 [n] when nf16
   float* rnorm;
   const int32_t* pos;
   int H;
@@ -190,13 +190,19 @@ struct QuantTcArgs {
   float cen[16];
   float bnd[16];
   int wait_limit;   // polls of the main MMA waits (the full limit when 0)
+  int nc;           // norm correction: store n / |c[idx]| (MSE-only formats)
+  int nf16;         // binary16 norms (MSE-only formats)
 };
 
 cudaError_t launch_quantize(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
 // One block per vector, for small batches (n <= kSmallQuantize).
 constexpr int64_t kSmallQuantize = 4096;
 cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStream_t s);
-// Tensor-core quantize for d = 128 (16-bit inputs).
+// Tensor-core quantize for d = 128 (16-bit inputs).  Norm-corrected and
+// binary16-norm formats run on the warp-specialised kernel only
+// (quant_ws_eligible); launch_quant_tc returns cudaErrorNotSupported for them
+// when the input cannot take that form.
+bool quant_ws_eligible(const QuantTcArgs& a);
 cudaError_t launch_quant_tc(const QuantTcArgs& a, int sms, cudaStream_t s);
 cudaError_t configure_quant_tc();
 cudaError_t read_and_clear_fault(int* value);

@@ -617,9 +617,10 @@ __device__ __noinline__ Q4 qjl_fixup_r(uint32_t taddr, const float* s_f32, Q4 fl
   return qw;
 }
 
-template <int BITS, bool QJL, bool BF>
+template <int BITS, bool QJL, bool BF, bool NC = false>
 __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
     k_quant_ws(const __grid_constant__ CUtensorMap tmx, QuantTcArgs a) {
+  static_assert(!(NC && QJL), "norm correction is for MSE-only formats");
   constexpr int NB = ws_groups(QJL);
   constexpr int NPI = BF ? 3 : 2;
   constexpr uint32_t XBASE = QJL ? 4 * SMEM_TILE : 3 * SMEM_TILE;
@@ -809,7 +810,7 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
       const bool writes = rec0 >= 0;
       const int64_t rec = writes ? rec0 : 0;
       uint32_t* crow = a.codes + rec * WORDS;
-      float rho2v[4] = {0.f, 0.f, 0.f, 0.f};
+      float rho2v[4] = {0.f, 0.f, 0.f, 0.f};   // |r|^2 with QJL, |c[idx]|^2 under norm correction
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         float d[32];
@@ -829,6 +830,10 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
             const float r = fmaf(y, 16384.f, -s_cen[idx]);   // s_cen holds 2^14 c
             rho2v[i & 3] = fmaf(r, r, rho2v[i & 3]);
             d[i] = r;
+          }
+          if (NC) {
+            const float cj = s_cen[idx];   // s_cen holds c
+            rho2v[i & 3] = fmaf(cj, cj, rho2v[i & 3]);
           }
         }
         if (writes) {
@@ -855,12 +860,20 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
           tmem_st32(d_rot + ch * 32, o);
         }
       }
-      if (writes) a.norm[rec] = nrm;
       if constexpr (!QJL) {
+        // Norm correction stores n / |c[idx]|; binary16 norms round the fp32 value.
+        const float st = NC ? nrm / sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) : nrm;
+        if (writes) {
+          if (a.nf16)
+            reinterpret_cast<__half*>(a.norm)[rec] = __float2half_rn(st);
+          else
+            a.norm[rec] = st;
+        }
         tc_before_sync();
         mbar_arrive(bars + 8 * (B_TE + b));
         continue;
       }
+      if (writes) a.norm[rec] = nrm;
       tc_before_sync();
       mbar_arrive(bars + 8 * (B_RR + b));   // this lane's residual operand is in place
       const float rho = sqrtf((rho2v[0] + rho2v[1]) + (rho2v[2] + rho2v[3])) * (1.f / 16384.f);
@@ -935,7 +948,9 @@ cudaError_t configure_bits() {
   if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, true, true>, ms, (int)WS_SMEM))) return e;
   if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, true, false>, ms, (int)WS_SMEM))) return e;
   if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, false, true>, ms, (int)WS_SMEM))) return e;
-  return cudaFuncSetAttribute(k_quant_ws<BITS, false, false>, ms, (int)WS_SMEM);
+  if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, false, false>, ms, (int)WS_SMEM))) return e;
+  if ((e = cudaFuncSetAttribute(k_quant_ws<BITS, false, true, true>, ms, (int)WS_SMEM))) return e;
+  return cudaFuncSetAttribute(k_quant_ws<BITS, false, false, true>, ms, (int)WS_SMEM);
 }
 
 template <int BITS>
@@ -943,8 +958,11 @@ cudaError_t launch_ws(const CUtensorMap& map, const QuantTcArgs& a, bool qjl, bo
   const dim3 bq(ws_warps(true) * 32), bn(ws_warps(false) * 32);
   if (qjl && bf) k_quant_ws<BITS, true, true><<<grid, bq, WS_SMEM, s>>>(map, a);
   if (qjl && !bf) k_quant_ws<BITS, true, false><<<grid, bq, WS_SMEM, s>>>(map, a);
-  if (!qjl && bf) k_quant_ws<BITS, false, true><<<grid, bn, WS_SMEM, s>>>(map, a);
-  if (!qjl && !bf) k_quant_ws<BITS, false, false><<<grid, bn, WS_SMEM, s>>>(map, a);
+  const bool nc = a.nc != 0;
+  if (!qjl && bf && !nc) k_quant_ws<BITS, false, true><<<grid, bn, WS_SMEM, s>>>(map, a);
+  if (!qjl && !bf && !nc) k_quant_ws<BITS, false, false><<<grid, bn, WS_SMEM, s>>>(map, a);
+  if (!qjl && bf && nc) k_quant_ws<BITS, false, true, true><<<grid, bn, WS_SMEM, s>>>(map, a);
+  if (!qjl && !bf && nc) k_quant_ws<BITS, false, false, true><<<grid, bn, WS_SMEM, s>>>(map, a);
   return cudaGetLastError();
 }
 
@@ -997,13 +1015,18 @@ cudaError_t configure_quant_tc() {
   return configure_bits<4>();
 }
 
+bool quant_ws_eligible(const QuantTcArgs& a) {
+  if ((a.nc || a.nf16) && a.m != 0) return false;   // MSE-only variants
+  return a.pi_b && (a.dtype == TQ_BF16 || a.dtype == TQ_F16) && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
+         (a.ld * 2) % 16 == 0 && a.n < ((int64_t)1 << 31) - TILE;
+}
+
 cudaError_t launch_quant_tc(const QuantTcArgs& a_in, int sms, cudaStream_t s) {
   QuantTcArgs a = a_in;
   if (a.wait_limit <= 0) a.wait_limit = TC_WAIT_LIMIT;
   const int64_t tiles = (a.n + TILE - 1) / TILE;
   CUtensorMap map;
-  if (a.pi_b && (a.dtype == TQ_BF16 || a.dtype == TQ_F16) && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
-      (a.ld * 2) % 16 == 0 && a.n < ((int64_t)1 << 31) - TILE && make_x_map(&map, a)) {
+  if (quant_ws_eligible(a) && make_x_map(&map, a)) {
     const int grid = (int)(tiles < sms ? tiles : sms);
     const bool qjl = a.m > 0, bf = a.dtype == TQ_BF16;
     switch (a.bits) {
@@ -1014,6 +1037,8 @@ cudaError_t launch_quant_tc(const QuantTcArgs& a_in, int sms, cudaStream_t s) {
       default: return cudaErrorInvalidValue;
     }
   }
+  // The register-staged form writes plain fp32 norms only.
+  if (a.nc || a.nf16) return cudaErrorNotSupported;
   int64_t grid = (tiles + 1) / 2;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;

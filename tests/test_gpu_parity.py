@@ -1119,3 +1119,50 @@ def test_decode_ignores_records_past_seq_len(cuda, fmt, Hq, f16):
     assert torch.equal(out, outp)
     P.check_attention(tab, Q.double().numpy(), P.packed_np(kc), P.packed_np(vc), lens.numpy(), Hkv,
                       out.cpu().numpy())
+
+
+@pytest.mark.parametrize("name,f16,dtype", [("k3v4_nc", False, torch.bfloat16), ("k3v4_nc", True, torch.float16),
+                                            ("4bit_nc", True, torch.float16), ("3bit_nc", False, torch.bfloat16),
+                                            ("k8v4", True, torch.bfloat16)])
+def test_quantize_tensor_core_norm_variants(cuda, name, f16, dtype):
+    """Norm-corrected formats and binary16 norms on the tensor-core quantize
+    (16-bit input, more than 4096 vectors, row pitch 136, a zero row, a
+    ragged last tile): codes and stored norms against the oracle; an append
+    of 6144 rows at per-sequence slots equals the bulk call on the same rows
+    and leaves the other slots alone.  (8-bit keys take the fp32 kernels.)"""
+    c = tq.Context.variant(name, 128, seed=23, norm_f16=f16)
+    tab = P.oracle_tables(c)
+    n = 6000
+    X = tq_inputs.outlier_kv(1, 1, n, 128, seed=24)[0, 0].to(dtype)
+    X[11] = 0
+    big = torch.zeros(n, 136, dtype=dtype)
+    big[:, :128] = X
+    src = big.to(cuda)[:, :128]
+    for which, wch in ((tq.TQ_KEY, "k"), (tq.TQ_VALUE, "v")):
+        pk = c.empty_packed(which, (n,))
+        c.quantize_into(src, which, pk)
+        torch.cuda.synchronize()
+        assert tq.tq_device_fault() == 0
+        assert pk["norm"].dtype == (torch.float16 if f16 else torch.float32)
+        P.check_quantized(tab, wch, X.double().numpy(), _flat(pk, n))
+    B, H, T = 64, 96, 5
+    x = tq_inputs.outlier_kv(B, H, 1, 128, seed=25)[:, :, 0].to(dtype).contiguous().to(cuda)
+    pos = torch.randint(0, T, (B,), generator=torch.Generator().manual_seed(4), dtype=torch.int32)
+    pos[3], pos[50] = -1, T
+    pos = pos.to(cuda)
+    ok = (pos >= 0) & (pos < T)
+    for which in (tq.TQ_KEY, tq.TQ_VALUE):
+        cache = c.empty_packed(which, (B, H, T), device=cuda)
+        for v in cache.values():
+            if v is not None:
+                v.fill_(-7)
+        c.quantize_append(x, which, cache, pos)
+        ref = c.quantize(x.reshape(B * H, 128), which)
+        torch.cuda.synchronize()
+        for k, v in cache.items():
+            if v is None:
+                continue
+            want = ref[k].reshape((B, H) + tuple(v.shape[3:]))
+            bs = torch.arange(B, device=cuda)[ok]
+            assert torch.equal(v[bs, :, pos[ok].long()], want[ok]), k
+            assert torch.all(v[~ok] == -7), k
