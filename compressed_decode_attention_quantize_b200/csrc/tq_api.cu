@@ -422,7 +422,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
     if (e != cudaSuccess) return cuda_fail(e, name);
     return TQ_OK;
   }
-  const bool tc = !pg.table && a.bits <= 4 && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
+  const bool tc = !pg.table && (a.bits <= 4 || a.bits == 8) && c->tc_ok && c->d == 128 && (dtype == TQ_BF16 || dtype == TQ_F16) && ld % 8 == 0 &&
                   aligned(x, 16) && aligned(codes, 16) && (m == 0 || (m == 128 && aligned(qjl, 16)));
   if (tc) {
     tqk::QuantTcArgs t{};
@@ -454,6 +454,7 @@ static int quantize_common(tq_ctx* c, int which, const void* x, int dtype, int64
     t.wait_limit = c->wait_limit;
     t.nc = a.nc ? 1 : 0;
     t.nf16 = a.nf16 ? 1 : 0;
+    t.bnd_dev = a.bnd;
     cudaError_t e = tqk::launch_quant_tc(t, c->sms, as_stream(stream));
     if (e != cudaErrorNotSupported) {   // unsupported: nothing was launched, the fp32 kernels take it
       if (e != cudaSuccess) return cuda_fail(e, name);

@@ -189,6 +189,7 @@ struct QuantTcArgs {
   int64_t max_T;
   float cen[16];
   float bnd[16];
+  const float* bnd_dev;   // device fp32 thresholds [2^bits - 1] (8-bit codes)
   int wait_limit;   // polls of the main MMA waits (the full limit when 0)
   int nc;           // norm correction: store n / |c[idx]| (MSE-only formats)
   int nf16;         // binary16 norms (MSE-only formats)

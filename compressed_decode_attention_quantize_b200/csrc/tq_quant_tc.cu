@@ -87,6 +87,17 @@ template <int BITS>
 __device__ __forceinline__ int lm_idx(float y, float pmid, const float* pb) {
   constexpr int H = 1 << (BITS - 1);
   const float a = fabsf(y);
+  if constexpr (BITS == 8) {
+    // pb: the 127 positive thresholds in breadth-first order of the balanced
+    // search tree (node i has children 2i + 1, 2i + 2), so the lanes of one
+    // level read a contiguous range of banks.  Leaf i - 127 = the count of
+    // thresholds <= |y|.
+    int i = 0;
+#pragma unroll
+    for (int l = 0; l < 7; ++l) i = 2 * i + 1 + (a >= pb[i] ? 1 : 0);
+    const int j = i - 127;
+    return (y >= 0.f) ? H + j : H - 1 - j;
+  }
   int j = 0;
   if (BITS >= 2) j = (a >= pmid) ? (H >> 1) : 0;
   if (BITS >= 4) j += (a >= pb[j + 1]) ? 2 : 0;
@@ -655,9 +666,15 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
       if (BF) dst[2 * CH + e] = src_pi[2 * CH + e];
       if (QJL) dst[WS_OFF_S / 16 + e] = src_s[e];
     }
-    if (tid < 128) s_snorm[tid] = QJL ? a.snorm[tid] : 0.f;
+    if (tid < 128 && BITS != 8) s_snorm[tid] = QJL ? a.snorm[tid] : 0.f;
     if (tid < 16) s_cen[tid] = tid < L ? a.cen[tid] * (QJL ? 16384.f : 1.f) : 0.f;
-    if (tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
+    if (BITS <= 4 && tid < 8) s_pb[tid] = (tid < L / 2 - 1) ? a.bnd[L / 2 + tid] : INFINITY;
+    if (BITS == 8 && tid < 127) {
+      // Breadth-first node tid (level l, position p) holds the threshold of
+      // in-order rank (2p + 1) 2^(6 - l) - 1 among the 127 positive ones.
+      const int l = 31 - __clz(tid + 1), p = tid + 1 - (1 << l);
+      s_snorm[tid] = a.bnd_dev[L / 2 + (2 * p + 1) * (1 << (6 - l)) - 1];
+    }
   }
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -779,8 +796,8 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
     const int g = (warp - 3) >> 2, quad = warp & 3;
     const int row = 32 * quad + lane;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-    const float* pb = s_pb;
-    const float pmid = BITS >= 2 ? s_pb[(L >> 2) - 1] : 0.f;
+    const float* pb = BITS == 8 ? s_snorm : s_pb;   // 8 bits: the search tree (no QJL rows then)
+    const float pmid = (BITS >= 2 && BITS <= 4) ? s_pb[(L >> 2) - 1] : 0.f;
     float snorm_max = 0.f;
     if (QJL)
       for (int i = 0; i < 128; ++i) snorm_max = fmaxf(snorm_max, s_snorm[i]);
@@ -815,7 +832,7 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
       for (int ch = 0; ch < 4; ++ch) {
         float d[32];
         tmem_ld32(d_rot + ch * 32, d);
-        uint32_t cw[4] = {0u, 0u, 0u, 0u};
+        uint32_t cw[BITS == 8 ? 8 : 4] = {};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float y = d[i] * inv;
@@ -837,6 +854,10 @@ __global__ void __launch_bounds__(ws_warps(QJL) * 32, 1)
           }
         }
         if (writes) {
+          if (BITS == 8) {
+            *reinterpret_cast<uint4*>(crow + 8 * ch) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint4*>(crow + 8 * ch + 4) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          }
           if (BITS == 4) *reinterpret_cast<uint4*>(crow + 4 * ch) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
           if (BITS == 2) *reinterpret_cast<uint2*>(crow + 2 * ch) = make_uint2(cw[0], cw[1]);
           if (BITS == 1) crow[ch] = cw[0];
@@ -966,6 +987,15 @@ cudaError_t launch_ws(const CUtensorMap& map, const QuantTcArgs& a, bool qjl, bo
   return cudaGetLastError();
 }
 
+cudaError_t launch_ws8(const CUtensorMap& map, const QuantTcArgs& a, bool bf, int grid, cudaStream_t s) {
+  const dim3 bn(ws_warps(false) * 32);
+  if (bf)
+    k_quant_ws<8, false, true><<<grid, bn, WS_SMEM, s>>>(map, a);
+  else
+    k_quant_ws<8, false, false><<<grid, bn, WS_SMEM, s>>>(map, a);
+  return cudaGetLastError();
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1012,11 +1042,15 @@ cudaError_t configure_quant_tc() {
   if ((e = configure_bits<1>()) != cudaSuccess) return e;
   if ((e = configure_bits<2>()) != cudaSuccess) return e;
   if ((e = configure_bits<3>()) != cudaSuccess) return e;
-  return configure_bits<4>();
+  if ((e = configure_bits<4>()) != cudaSuccess) return e;
+  const cudaFuncAttribute ms = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if ((e = cudaFuncSetAttribute(k_quant_ws<8, false, true>, ms, (int)WS_SMEM))) return e;
+  return cudaFuncSetAttribute(k_quant_ws<8, false, false>, ms, (int)WS_SMEM);
 }
 
 bool quant_ws_eligible(const QuantTcArgs& a) {
   if ((a.nc || a.nf16) && a.m != 0) return false;   // MSE-only variants
+  if (a.bits == 8 && (a.m != 0 || a.nc || !a.bnd_dev)) return false;   // 8 bits: plain MSE codes only
   return a.pi_b && (a.dtype == TQ_BF16 || a.dtype == TQ_F16) && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
          (a.ld * 2) % 16 == 0 && a.n < ((int64_t)1 << 31) - TILE;
 }
@@ -1026,7 +1060,13 @@ cudaError_t launch_quant_tc(const QuantTcArgs& a_in, int sms, cudaStream_t s) {
   if (a.wait_limit <= 0) a.wait_limit = TC_WAIT_LIMIT;
   const int64_t tiles = (a.n + TILE - 1) / TILE;
   CUtensorMap map;
-  if (quant_ws_eligible(a) && make_x_map(&map, a)) {
+  const bool ws = quant_ws_eligible(a) && make_x_map(&map, a);
+  if (a.bits == 8) {   // the warp-specialised kernel only
+    if (!ws) return cudaErrorNotSupported;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    return launch_ws8(map, a, a.dtype == TQ_BF16, grid, s);
+  }
+  if (ws) {
     const int grid = (int)(tiles < sms ? tiles : sms);
     const bool qjl = a.m > 0, bf = a.dtype == TQ_BF16;
     switch (a.bits) {

@@ -1123,13 +1123,14 @@ def test_decode_ignores_records_past_seq_len(cuda, fmt, Hq, f16):
 
 @pytest.mark.parametrize("name,f16,dtype", [("k3v4_nc", False, torch.bfloat16), ("k3v4_nc", True, torch.float16),
                                             ("4bit_nc", True, torch.float16), ("3bit_nc", False, torch.bfloat16),
-                                            ("k8v4", True, torch.bfloat16)])
+                                            ("k8v4", True, torch.bfloat16), ("k8v4", False, torch.float16)])
 def test_quantize_tensor_core_norm_variants(cuda, name, f16, dtype):
     """Norm-corrected formats and binary16 norms on the tensor-core quantize
     (16-bit input, more than 4096 vectors, row pitch 136, a zero row, a
     ragged last tile): codes and stored norms against the oracle; an append
     of 6144 rows at per-sequence slots equals the bulk call on the same rows
-    and leaves the other slots alone.  (8-bit keys take the fp32 kernels.)"""
+    and leaves the other slots alone.  k8v4 keys take the 8-bit codes of the
+    same kernel (thresholds in a breadth-first search tree)."""
     c = tq.Context.variant(name, 128, seed=23, norm_f16=f16)
     tab = P.oracle_tables(c)
     n = 6000
