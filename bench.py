@@ -490,11 +490,20 @@ def _variant_once(tq, tq_inputs, torch, dev, hbm_peak, shape, name, f16, steps, 
     ctx = tq.Context.variant(name, d, 0, norm_f16=f16)
     kc = ctx.empty_packed(tq.TQ_KEY, (B, Hkv, T), device=dev)
     vc = ctx.empty_packed(tq.TQ_VALUE, (B, Hkv, T), device=dev)
+    # The cache build's quantize calls of sequences 1.. are timed (sequence 0 warms up).
+    qa, qb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q_ms = 0.0
     for b in range(B):
         K = tq_inputs.outlier_kv(1, Hkv, T, d, seed=1000 + b, device=dev, scale_seed=1)[0]
         V = tq_inputs.outlier_kv(1, Hkv, T, d, seed=2000 + b, device=dev, scale_seed=2)[0]
+        if b > 0:
+            qa.record()
         ctx.quantize_into(K, tq.TQ_KEY, {k: (None if v is None else v[b]) for k, v in kc.items()})
         ctx.quantize_into(V, tq.TQ_VALUE, {k: (None if v is None else v[b]) for k, v in vc.items()})
+        if b > 0:
+            qb.record()
+            torch.cuda.synchronize()
+            q_ms += qa.elapsed_time(qb)
         del K, V
     q = tq_inputs.iid((B, Hq, d), seed=10, device=dev, dtype=torch.bfloat16)
     lens = torch.full((B,), T, dtype=torch.int32, device=dev)
@@ -523,6 +532,10 @@ def _variant_once(tq, tq_inputs, torch, dev, hbm_peak, shape, name, f16, steps, 
                         f"{kb + vb} B per token-head",
            "attn_ms": ms, "kv_tokens_per_s": B * T / (ms / 1e3),
            "hbm_frac": alg / (ms / 1e3) / 1e9 / hbm_peak}
+    if B > 1 and q_ms > 0:
+        res["quantize_mvec_per_s"] = 2 * (B - 1) * Hkv * T / (q_ms / 1e3) / 1e6
+        res["quantize_sample"] = (f"cache build of sequences 1..{B - 1}: {Hkv * T} bf16 K and {Hkv * T} "
+                                  f"bf16 V vectors per sequence, CUDA events around the quantize calls")
     del g, kc, vc, ws
     ctx.close()
     return res
