@@ -918,24 +918,29 @@ __global__ void __launch_bounds__(FAST_T) k_prerotate_fast(const void* q, int dt
   if (tiles && blockIdx.x == 0) tile_plan(seq_lens, B, Hkv, max_T, tiles);
 }
 
-// The decode step's preparation with the fast bodies: blocks [0, n) append
-// the new keys, [n, 2n) the new values (n = B Hkv), the rest pre-rotate
-// FAST_R query rows each; the first query block writes the lengths and the
-// tile prefix.
-__global__ void __launch_bounds__(FAST_T) k_step_prep_fast(StepPrep s, int d, int dpad, int m, const float* PiT,
-                                                         const float* ST) {
+// The decode step's preparation with the fast bodies: blocks [0, a) append
+// the new keys, STEP_QS per block, [a, 2a) the new values (a = ceil(B Hkv /
+// STEP_QS)), the rest pre-rotate FAST_R query rows each; the first query
+// block writes the lengths and the tile prefix.  Two vectors per append block
+// share each thread's matrix loads and keep the grid within one wave of two
+// 512-thread CTAs per SM on the Llama-3-8B decode shape.
+constexpr int STEP_QS = 2;
+__global__ void __launch_bounds__(FAST_T, 2) k_step_prep_fast(StepPrep s, int d, int dpad, int m,
+                                                            const float* PiT, const float* ST) {
   __shared__ __align__(16) float sh[6 * FAST_R * 128];
+  static_assert(5 * STEP_QS * 128 <= 6 * FAST_R * 128, "append staging fits the shared buffer");
+  const int64_t na = (s.nkv + STEP_QS - 1) / STEP_QS;
   int64_t blk = blockIdx.x;
-  if (blk < s.nkv) {
-    quantize_fast_body<1>(s.k, dpad, blk, sh);
+  if (blk < na) {
+    quantize_fast_body<STEP_QS>(s.k, dpad, blk, sh);
     return;
   }
-  blk -= s.nkv;
-  if (blk < s.nkv) {
-    quantize_fast_body<1>(s.v, dpad, blk, sh);
+  blk -= na;
+  if (blk < na) {
+    quantize_fast_body<STEP_QS>(s.v, dpad, blk, sh);
     return;
   }
-  blk -= s.nkv;
+  blk -= na;
   // matrix loads before each product: two CTAs per SM fit the registers
   prerotate_fast_body<FAST_R, false>(s.q, s.qdtype, s.qrows, d, dpad, m, PiT, ST, s.qr, s.qs, blk, &s.qop, sh);
   if (blk == 0) {
@@ -1519,7 +1524,7 @@ cudaError_t launch_quantize_small(const tq_ctx* c, const QuantArgs& a, cudaStrea
 
 cudaError_t launch_step_prep(const tq_ctx* c, const StepPrep& sp, cudaStream_t s) {
   if (c->dpad <= 128) {
-    const int64_t blocks = 2 * sp.nkv + (sp.qrows + FAST_R - 1) / FAST_R;
+    const int64_t blocks = 2 * ((sp.nkv + STEP_QS - 1) / STEP_QS) + (sp.qrows + FAST_R - 1) / FAST_R;
     if (blocks == 0) return cudaSuccess;
     k_step_prep_fast<<<(unsigned)blocks, FAST_T, 0, s>>>(sp, c->d, c->dpad, c->qjl_m, c->PiT, c->ST);
     return cudaGetLastError();
