@@ -95,7 +95,7 @@ __device__ __forceinline__ uint32_t field_word(uint32_t val, int b, int lane) {
 }
 
 // ----------------------------------------------------------------------------
-// Quantize: one warp quantizes QV vectors at a time.  Lane l owns the output
+// Quantize: one warp quantizes QV vectors at a time (quant_qv).  Lane l owns the output
 // coordinates j = l + 32 i (i < J), so the Lloyd-Max bits of plane p, word i
 // of a vector are one __ballot_sync.  The rotation y = Pi x / |x| and the
 // sketch S r are fp32 FMA dot products (PiT and ST are k-major so lanes read
@@ -164,12 +164,20 @@ __device__ __forceinline__ void mv_rows(const float* M, int d, int dpad, const f
   }
 }
 
-constexpr int QV = 8;
 constexpr int QWARPS = 8;
+// Vectors per warp: eight up to d = 128; four beyond, where eight would hold
+// 8 J accumulators and indices per lane (d = 200: 242 registers, one
+// 256-thread CTA per SM) and leave the matrix loads' latency uncovered.
+template <int J>
+__host__ __device__ constexpr int quant_qv() {
+  return J >= 5 ? 4 : 8;
+}
 
 template <int J>
 __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
   constexpr int DP = J * 32;
+  constexpr int QV = quant_qv<J>();
+  static_assert(QV % 4 == 0, "x rows are read as float4");
   extern __shared__ float smem[];
   __shared__ float s_cen[kMaxLevels], s_bnd[kMaxLevels];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -205,9 +213,16 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 #pragma unroll
       for (int v = 0; v < QV; ++v) acc[i][v] = 0.f;
     for (int k = 0; k < a.d; ++k) {
-      const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
-      const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
-      const float xv[QV] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      float xv[QV];
+      if constexpr (QV == 8) {
+        const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+        const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
+        xv[0] = x0.x, xv[1] = x0.y, xv[2] = x0.z, xv[3] = x0.w;
+        xv[4] = x1.x, xv[5] = x1.y, xv[6] = x1.z, xv[7] = x1.w;
+      } else {
+        const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+        xv[0] = x0.x, xv[1] = x0.y, xv[2] = x0.z, xv[3] = x0.w;
+      }
 #pragma unroll
       for (int i = 0; i < J; ++i) {
         const float p = __ldg(a.PiT + (size_t)k * DP + lane + 32 * i);
@@ -298,9 +313,16 @@ __global__ void __launch_bounds__(QWARPS * 32) k_quantize(QuantArgs a) {
 #pragma unroll
       for (int v = 0; v < QV; ++v) acc[i][v] = 0.f;
     for (int k = 0; k < a.d; ++k) {
-      const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
-      const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
-      const float xv[QV] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      float xv[QV];
+      if constexpr (QV == 8) {
+        const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+        const float4 x1 = *reinterpret_cast<const float4*>(sx + k * QV + 4);
+        xv[0] = x0.x, xv[1] = x0.y, xv[2] = x0.z, xv[3] = x0.w;
+        xv[4] = x1.x, xv[5] = x1.y, xv[6] = x1.z, xv[7] = x1.w;
+      } else {
+        const float4 x0 = *reinterpret_cast<const float4*>(sx + k * QV);
+        xv[0] = x0.x, xv[1] = x0.y, xv[2] = x0.z, xv[3] = x0.w;
+      }
 #pragma unroll
       for (int i = 0; i < J; ++i) {
         const float p = __ldg(a.ST + (size_t)k * DP + lane + 32 * i);
@@ -1463,6 +1485,7 @@ __global__ void __launch_bounds__(32) k_topk_final(const float* cand_v, const in
 
 template <int J>
 cudaError_t quantize_J(const QuantArgs& a, cudaStream_t s) {
+  constexpr int QV = quant_qv<J>();
   const size_t shm = (size_t)QWARPS * J * 32 * QV * sizeof(float);
   const int64_t groups = (a.n + QV - 1) / QV;
   int64_t blocks = (groups + QWARPS - 1) / QWARPS;
@@ -1701,7 +1724,7 @@ cudaError_t launch_topk(const tq_ctx* c, const void* q, int dtype, int64_t nq,
 template <int J>
 static cudaError_t configure_J() {
   cudaError_t e = cudaFuncSetAttribute(k_quantize<J>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(QWARPS * J * 32 * QV * sizeof(float)));
+                                       (int)(QWARPS * J * 32 * quant_qv<J>() * sizeof(float)));
   if (e != cudaSuccess) return e;
   const int attn_max = (2 * GMAX * J * 32 + AT * GMAX) * (int)sizeof(float) + AT * 64 * (int)sizeof(uint32_t);
   e = cudaFuncSetAttribute(k_attn_split<J>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_max);
